@@ -1,0 +1,532 @@
+/*
+ * nf4_oracle.c -- CPU oracle for the host-streamed NF4 LoRA hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY (see nf4_oracle.h): loaded by the tests, the
+ * smoke check and the benchmark's CPU-baseline leg, never by the product.
+ * Plain C11, libm and pthreads; no BLAS, no blocking, no reordering of any
+ * sum: every output element is one loop in index order, accumulated in
+ * double and rounded once.  Threads only split the set of output elements.
+ */
+#include "nf4_oracle.h"
+
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* bf16 <-> fp32                                                            */
+/* ------------------------------------------------------------------------ */
+
+float orc_bf16_to_f32(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+/* Round to nearest, ties to even.  NaN becomes a quiet NaN. */
+uint16_t orc_f32_to_bf16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x0040u);
+  uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7fffu + lsb;
+  return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------------------ */
+/* NormalFloat-4 codebook                                                   */
+/* ------------------------------------------------------------------------ */
+/* The pages name the data type (4-bit NF4, Poros API reference,
+ * PorosTrainer.from_pretrained "quantization") but print no values.  The
+ * plainest reading is the published NormalFloat construction (QLoRA,
+ * Dettmers et al. 2023, section "4-bit NormalFloat Quantization"):
+ * standard-normal quantiles at probabilities spaced evenly from
+ * delta = 1 - (1/32 + 1/30)/2 down to 1/2 -- eight on the positive side
+ * (the 1/2 end excluded), seven mirrored on the negative side (likewise),
+ * plus an exact zero -- all divided by the largest magnitude, so that the
+ * ends are exactly -1 and +1.  The probabilities are formed as exact
+ * rationals, the quantiles in double, and each ratio is rounded once to
+ * fp32. */
+
+static double normal_cdf(double x) { return 0.5 * erfc(-x / sqrt(2.0)); }
+
+double orc_normal_quantile(double p) {
+  double lo = -40.0, hi = 40.0;
+  for (int it = 0; it < 4000; ++it) {
+    double mid = 0.5 * (lo + hi);
+    if (mid <= lo || mid >= hi) break;
+    if (normal_cdf(mid) < p)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+void orc_nf4_codebook(float out[16]) {
+  /* delta = 1 - (1/32 + 1/30)/2 = 929/960. */
+  const double top = orc_normal_quantile(929.0 / 960.0);
+  /* negative side: p_j = delta + j (1/2 - delta) / 7, j = 0..6
+   *              = (929*7 - 449 j) / 6720                                  */
+  for (int j = 0; j < 7; ++j) {
+    double p = (929.0 * 7.0 - 449.0 * j) / 6720.0;
+    out[j] = (float)(-orc_normal_quantile(p) / top);
+  }
+  out[7] = 0.0f;
+  /* positive side: p_j = delta + j (1/2 - delta) / 8, j = 0..7
+   *              = (929*8 - 449 j) / 7680; largest first, stored ascending */
+  for (int j = 0; j < 8; ++j) {
+    double p = (929.0 * 8.0 - 449.0 * j) / 7680.0;
+    out[15 - j] = (float)(orc_normal_quantile(p) / top);
+  }
+  out[0] = -1.0f; /* the j = 0 ratios are x/x = 1 exactly */
+  out[15] = 1.0f;
+}
+
+/* Nearest codebook entry by a linear scan of fp32 distances |x - c_i|.
+ * Reading: the pages fix no tie rule; a strict '<' keeps the lower index. */
+static int nearest_code(const float cb[16], float x) {
+  int best = 0;
+  float bd = fabsf(x - cb[0]);
+  for (int i = 1; i < 16; ++i) {
+    float d = fabsf(x - cb[i]);
+    if (d < bd) {
+      bd = d;
+      best = i;
+    }
+  }
+  return best;
+}
+
+int orc_nf4_nearest(float x) {
+  float cb[16];
+  orc_nf4_codebook(cb);
+  return nearest_code(cb, x);
+}
+
+/* ------------------------------------------------------------------------ */
+/* NF4 storage format                                                       */
+/* ------------------------------------------------------------------------ */
+/* Format reading: row-major W[n_out, k_in], flat index e = n*k_in + k,
+ * 64-element blocks along e (so a block never crosses a row when
+ * k_in % 64 == 0), one fp32 absmax per block, 4-bit codes two per byte with
+ * the even element in the high nibble.  0.5 + 4/64 = 0.5625 byte/param,
+ * which is what reproduces the ~4/~18/~40 GB host footprints quoted for the
+ * NF4 base ("Poros on consumer GPUs", "What you need besides VRAM"). */
+
+int64_t orc_nf4_storage_bytes(int64_t n_out, int64_t k_in) {
+  int64_t p = n_out * k_in;
+  return p / 2 + 4 * (p / 64);
+}
+
+static int shape_ok(int64_t n_out, int64_t k_in) {
+  return n_out > 0 && k_in > 0 && (k_in % 64) == 0;
+}
+
+int orc_nf4_quantize(const uint16_t *w, int64_t n_out, int64_t k_in,
+                     uint8_t *codes, float *absmax) {
+  if (!shape_ok(n_out, k_in)) return -1;
+  float cb[16];
+  orc_nf4_codebook(cb);
+  const int64_t nblk = n_out * k_in / 64;
+  for (int64_t b = 0; b < nblk; ++b) {
+    const uint16_t *blk = w + b * 64;
+    float a = 0.0f;
+    for (int i = 0; i < 64; ++i) {
+      float v = fabsf(orc_bf16_to_f32(blk[i]));
+      if (v > a) a = v;
+    }
+    absmax[b] = a;
+    for (int i = 0; i < 64; ++i) {
+      int code;
+      if (a == 0.0f) {
+        code = 7; /* all-zero block: the exact-zero entry */
+      } else {
+        float x = orc_bf16_to_f32(blk[i]) / a; /* IEEE fp32 division */
+        code = nearest_code(cb, x);
+      }
+      int64_t e = b * 64 + i;
+      if ((e & 1) == 0)
+        codes[e >> 1] = (uint8_t)(code << 4);
+      else
+        codes[e >> 1] = (uint8_t)(codes[e >> 1] | code);
+    }
+  }
+  return 0;
+}
+
+static int code_at(const uint8_t *codes, int64_t e) {
+  uint8_t byte = codes[e >> 1];
+  return (e & 1) ? (byte & 0x0f) : (byte >> 4);
+}
+
+int orc_nf4_dequant(const uint8_t *codes, const float *absmax, int64_t n_out,
+                    int64_t k_in, uint16_t *out) {
+  if (!shape_ok(n_out, k_in)) return -1;
+  float cb[16];
+  orc_nf4_codebook(cb);
+  const int64_t total = n_out * k_in;
+  for (int64_t e = 0; e < total; ++e) {
+    float v = cb[code_at(codes, e)] * absmax[e / 64]; /* fp32 product */
+    out[e] = orc_f32_to_bf16(v);
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* a minimal parallel-for over an index range                               */
+/* ------------------------------------------------------------------------ */
+
+typedef void (*range_fn)(void *ctx, int64_t lo, int64_t hi);
+
+typedef struct {
+  range_fn fn;
+  void *ctx;
+  int64_t lo, hi;
+} range_job;
+
+static void *range_thread(void *p) {
+  range_job *j = (range_job *)p;
+  j->fn(j->ctx, j->lo, j->hi);
+  return NULL;
+}
+
+static void parallel_for(int64_t n, int n_threads, range_fn fn, void *ctx) {
+  if (n_threads < 1) n_threads = 1;
+  if (n_threads > 256) n_threads = 256;
+  if ((int64_t)n_threads > n) n_threads = (int)(n > 0 ? n : 1);
+  if (n_threads == 1) {
+    fn(ctx, 0, n);
+    return;
+  }
+  pthread_t th[256];
+  range_job jobs[256];
+  int started[256];
+  for (int i = 0; i < n_threads; ++i) {
+    jobs[i].fn = fn;
+    jobs[i].ctx = ctx;
+    jobs[i].lo = n * i / n_threads;
+    jobs[i].hi = n * (i + 1) / n_threads;
+    started[i] = pthread_create(&th[i], NULL, range_thread, &jobs[i]) == 0;
+    if (!started[i]) fn(ctx, jobs[i].lo, jobs[i].hi);
+  }
+  for (int i = 0; i < n_threads; ++i)
+    if (started[i]) pthread_join(th[i], NULL);
+}
+
+/* ------------------------------------------------------------------------ */
+/* LoRA linear                                                              */
+/* ------------------------------------------------------------------------ */
+/* The layer computed for every projection (q/k/v/o/gate/up/down) with the
+ * frozen base W and the trainable rank-r adapter (A [r,K], B [N,r]),
+ * Poros API reference, PorosTrainer.from_pretrained (lora_rank, lora_alpha;
+ * dropout 0 here):
+ *   forward   Y  = X W^T + (alpha/r) (X A^T) B^T
+ *   backward  dX = dY W + (alpha/r) (dY B) A
+ *             dB = (alpha/r) dY^T (X A^T)
+ *             dA = (alpha/r) (dY B)^T X
+ * W is frozen -- read, never written (HN comment on host-RAM streaming). */
+
+/* A source of rows of W, as doubles, for columns [k0, k1). */
+typedef struct {
+  const double *dense; /* [N,K] or NULL */
+  const uint8_t *codes;
+  const float *absmax;
+  float cb[16];
+  int64_t K;
+} wsrc;
+
+static void w_row(const wsrc *w, int64_t n, int64_t k0, int64_t k1,
+                  double *out) {
+  if (w->dense) {
+    for (int64_t k = k0; k < k1; ++k) out[k - k0] = w->dense[n * w->K + k];
+    return;
+  }
+  for (int64_t k = k0; k < k1; ++k) {
+    int64_t e = n * w->K + k;
+    float v = w->cb[code_at(w->codes, e)] * w->absmax[e / 64];
+    out[k - k0] = (double)orc_bf16_to_f32(orc_f32_to_bf16(v));
+  }
+}
+
+/* ---- forward: parallel over output columns n ---- */
+typedef struct {
+  const wsrc *w;
+  const double *X; /* [n_rows, K] token rows to compute */
+  const double *t; /* [n_rows, r] */
+  const double *B; /* [N, r] */
+  int64_t n_rows, N, K;
+  int r;
+  double s;
+  double *Y; /* [n_rows, N] */
+} fwd_ctx;
+
+static void fwd_cols(void *p, int64_t lo, int64_t hi) {
+  fwd_ctx *c = (fwd_ctx *)p;
+  double *row = (double *)malloc(sizeof(double) * (size_t)c->K);
+  if (!row) return;
+  for (int64_t n = lo; n < hi; ++n) {
+    w_row(c->w, n, 0, c->K, row);
+    for (int64_t i = 0; i < c->n_rows; ++i) {
+      const double *x = c->X + i * c->K;
+      double acc = 0.0;
+      for (int64_t k = 0; k < c->K; ++k) acc += x[k] * row[k];
+      double lora = 0.0;
+      for (int j = 0; j < c->r; ++j) lora += c->t[i * c->r + j] * c->B[n * c->r + j];
+      c->Y[i * c->N + n] = acc + c->s * lora;
+    }
+  }
+  free(row);
+}
+
+/* t = X A^T for the given rows (cheap; single thread) */
+static void lora_down(const double *X, const double *A, int64_t rows,
+                      int64_t K, int r, double *t) {
+  for (int64_t i = 0; i < rows; ++i)
+    for (int j = 0; j < r; ++j) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += X[i * K + k] * A[j * K + k];
+      t[i * r + j] = acc;
+    }
+}
+
+/* ---- dX: parallel over output columns k (contraction over n in order) ---- */
+typedef struct {
+  const wsrc *w;
+  const double *dY; /* [n_rows, N] */
+  const double *u;  /* [n_rows, r] */
+  const double *A;  /* [r, K] */
+  int64_t n_rows, N, K;
+  int r;
+  double s;
+  double *dX; /* [n_rows, K] */
+} dx_ctx;
+
+static void dx_cols(void *p, int64_t lo, int64_t hi) {
+  dx_ctx *c = (dx_ctx *)p;
+  int64_t width = hi - lo;
+  if (width <= 0) return;
+  double *row = (double *)malloc(sizeof(double) * (size_t)width);
+  double *acc = (double *)calloc((size_t)(c->n_rows * width), sizeof(double));
+  if (!row || !acc) {
+    free(row);
+    free(acc);
+    return;
+  }
+  for (int64_t n = 0; n < c->N; ++n) {
+    w_row(c->w, n, lo, hi, row);
+    for (int64_t i = 0; i < c->n_rows; ++i) {
+      double g = c->dY[i * c->N + n];
+      double *a = acc + i * width;
+      for (int64_t k = 0; k < width; ++k) a[k] += g * row[k];
+    }
+  }
+  for (int64_t i = 0; i < c->n_rows; ++i)
+    for (int64_t k = lo; k < hi; ++k) {
+      double lora = 0.0;
+      for (int j = 0; j < c->r; ++j) lora += c->u[i * c->r + j] * c->A[j * c->K + k];
+      c->dX[i * c->K + k] = acc[i * width + (k - lo)] + c->s * lora;
+    }
+  free(row);
+  free(acc);
+}
+
+/* dB[n, j] = s sum_i dY[i, n] t[i, j];  dA[j, k] = s sum_i u[i, j] X[i, k] */
+static void lora_grads(const double *X, const double *dY, const double *t,
+                       const double *u, int64_t T, int64_t N, int64_t K, int r,
+                       double s, double *dA, double *dB) {
+  for (int64_t n = 0; n < N; ++n)
+    for (int j = 0; j < r; ++j) {
+      double acc = 0.0;
+      for (int64_t i = 0; i < T; ++i) acc += dY[i * N + n] * t[i * r + j];
+      dB[n * r + j] = s * acc;
+    }
+  for (int j = 0; j < r; ++j)
+    for (int64_t k = 0; k < K; ++k) {
+      double acc = 0.0;
+      for (int64_t i = 0; i < T; ++i) acc += u[i * r + j] * X[i * K + k];
+      dA[j * K + k] = s * acc;
+    }
+}
+
+/* u = dY B  ([T,N] x [N,r]) */
+static void lora_up_t(const double *dY, const double *B, int64_t T, int64_t N,
+                      int r, double *u) {
+  for (int64_t i = 0; i < T; ++i)
+    for (int j = 0; j < r; ++j) {
+      double acc = 0.0;
+      for (int64_t n = 0; n < N; ++n) acc += dY[i * N + n] * B[n * r + j];
+      u[i * r + j] = acc;
+    }
+}
+
+void orc_lora_fwd_f64(const double *W, const double *X, const double *A,
+                      const double *B, int64_t T, int64_t N, int64_t K, int r,
+                      double s, double *Y, double *t) {
+  wsrc w;
+  memset(&w, 0, sizeof w);
+  w.dense = W;
+  w.K = K;
+  lora_down(X, A, T, K, r, t);
+  fwd_ctx c = {&w, X, t, B, T, N, K, r, s, Y};
+  fwd_cols(&c, 0, N);
+}
+
+void orc_lora_bwd_f64(const double *W, const double *X, const double *A,
+                      const double *B, const double *dY, int64_t T, int64_t N,
+                      int64_t K, int r, double s, double *dX, double *dA,
+                      double *dB) {
+  wsrc w;
+  memset(&w, 0, sizeof w);
+  w.dense = W;
+  w.K = K;
+  double *t = (double *)malloc(sizeof(double) * (size_t)(T * r));
+  double *u = (double *)malloc(sizeof(double) * (size_t)(T * r));
+  if (!t || !u) {
+    free(t);
+    free(u);
+    return;
+  }
+  lora_down(X, A, T, K, r, t);
+  lora_up_t(dY, B, T, N, r, u);
+  dx_ctx c = {&w, dY, u, A, T, N, K, r, s, dX};
+  dx_cols(&c, 0, K);
+  lora_grads(X, dY, t, u, T, N, K, r, s, dA, dB);
+  free(t);
+  free(u);
+}
+
+/* ---- the method's data types ---- */
+
+static double *widen_bf16(const uint16_t *src, int64_t n) {
+  double *d = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+  if (!d) return NULL;
+  for (int64_t i = 0; i < n; ++i) d[i] = (double)orc_bf16_to_f32(src[i]);
+  return d;
+}
+
+static double *gather_rows(const double *M, int64_t cols, const int64_t *rows,
+                           int64_t n_rows) {
+  double *d = (double *)malloc(sizeof(double) * (size_t)(n_rows * cols > 0 ? n_rows * cols : 1));
+  if (!d) return NULL;
+  for (int64_t i = 0; i < n_rows; ++i)
+    memcpy(d + i * cols, M + rows[i] * cols, sizeof(double) * (size_t)cols);
+  return d;
+}
+
+static int lora_args_ok(int64_t N, int64_t K, int64_t T, int r,
+                        const int64_t *rows, int64_t n_rows) {
+  if (!shape_ok(N, K) || T <= 0 || r <= 0) return 0;
+  if (rows) {
+    for (int64_t i = 0; i < n_rows; ++i)
+      if (rows[i] < 0 || rows[i] >= T) return 0;
+  }
+  return 1;
+}
+
+int orc_lora_fwd(const uint8_t *codes, const float *absmax, int64_t N,
+                 int64_t K, const uint16_t *X, int64_t T, const uint16_t *A,
+                 const uint16_t *B, int r, float alpha, const int64_t *rows,
+                 int64_t n_rows, float *Y, float *t_out, int n_threads) {
+  if (!lora_args_ok(N, K, T, r, rows, n_rows)) return -1;
+  if (!rows) n_rows = T;
+  const double s = (double)alpha / (double)r;
+  wsrc w;
+  memset(&w, 0, sizeof w);
+  w.codes = codes;
+  w.absmax = absmax;
+  w.K = K;
+  orc_nf4_codebook(w.cb);
+
+  double *Xd = widen_bf16(X, T * K);
+  double *Ad = widen_bf16(A, (int64_t)r * K);
+  double *Bd = widen_bf16(B, N * r);
+  double *t = (double *)malloc(sizeof(double) * (size_t)(T * r));
+  double *Yd = (double *)malloc(sizeof(double) * (size_t)(n_rows * N > 0 ? n_rows * N : 1));
+  double *Xs = NULL, *ts = NULL;
+  int rc = -1;
+  if (!Xd || !Ad || !Bd || !t || !Yd) goto done;
+  lora_down(Xd, Ad, T, K, r, t);
+  if (rows) {
+    Xs = gather_rows(Xd, K, rows, n_rows);
+    ts = gather_rows(t, r, rows, n_rows);
+    if (!Xs || !ts) goto done;
+  }
+  {
+    fwd_ctx c = {&w, rows ? Xs : Xd, rows ? ts : t, Bd, n_rows, N, K, r, s, Yd};
+    parallel_for(N, n_threads, fwd_cols, &c);
+  }
+  for (int64_t i = 0; i < n_rows * N; ++i) Y[i] = (float)Yd[i];
+  if (t_out)
+    for (int64_t i = 0; i < T * r; ++i) t_out[i] = (float)t[i];
+  rc = 0;
+done:
+  free(Xd);
+  free(Ad);
+  free(Bd);
+  free(t);
+  free(Yd);
+  free(Xs);
+  free(ts);
+  return rc;
+}
+
+int orc_lora_bwd(const uint8_t *codes, const float *absmax, int64_t N,
+                 int64_t K, const uint16_t *X, int64_t T, const uint16_t *A,
+                 const uint16_t *B, int r, float alpha, const uint16_t *dY,
+                 const int64_t *rows, int64_t n_rows, float *dX, float *dA,
+                 float *dB, int n_threads) {
+  if (!lora_args_ok(N, K, T, r, rows, n_rows)) return -1;
+  if (!rows) n_rows = T;
+  const double s = (double)alpha / (double)r;
+  wsrc w;
+  memset(&w, 0, sizeof w);
+  w.codes = codes;
+  w.absmax = absmax;
+  w.K = K;
+  orc_nf4_codebook(w.cb);
+
+  double *Xd = widen_bf16(X, T * K);
+  double *Ad = widen_bf16(A, (int64_t)r * K);
+  double *Bd = widen_bf16(B, N * r);
+  double *dYd = widen_bf16(dY, T * N);
+  double *t = (double *)malloc(sizeof(double) * (size_t)(T * r));
+  double *u = (double *)malloc(sizeof(double) * (size_t)(T * r));
+  double *dXd = (double *)malloc(sizeof(double) * (size_t)(n_rows * K > 0 ? n_rows * K : 1));
+  double *dAd = (double *)malloc(sizeof(double) * (size_t)(r * K));
+  double *dBd = (double *)malloc(sizeof(double) * (size_t)(N * r));
+  double *dYs = NULL, *us = NULL;
+  int rc = -1;
+  if (!Xd || !Ad || !Bd || !dYd || !t || !u || !dXd || !dAd || !dBd) goto done;
+  lora_down(Xd, Ad, T, K, r, t);
+  lora_up_t(dYd, Bd, T, N, r, u);
+  if (rows) {
+    dYs = gather_rows(dYd, N, rows, n_rows);
+    us = gather_rows(u, r, rows, n_rows);
+    if (!dYs || !us) goto done;
+  }
+  {
+    dx_ctx c = {&w, rows ? dYs : dYd, rows ? us : u, Ad, n_rows, N, K, r, s, dXd};
+    parallel_for(K, n_threads, dx_cols, &c);
+  }
+  lora_grads(Xd, dYd, t, u, T, N, K, r, s, dAd, dBd);
+  for (int64_t i = 0; i < n_rows * K; ++i) dX[i] = (float)dXd[i];
+  for (int64_t i = 0; i < (int64_t)r * K; ++i) dA[i] = (float)dAd[i];
+  for (int64_t i = 0; i < N * r; ++i) dB[i] = (float)dBd[i];
+  rc = 0;
+done:
+  free(Xd);
+  free(Ad);
+  free(Bd);
+  free(dYd);
+  free(t);
+  free(u);
+  free(dXd);
+  free(dAd);
+  free(dBd);
+  free(dYs);
+  free(us);
+  return rc;
+}

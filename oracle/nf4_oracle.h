@@ -1,0 +1,103 @@
+/*
+ * nf4_oracle.h -- CPU oracle for the host-streamed NF4 LoRA hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This is the plain, slow, obviously correct
+ * reference that the CUDA path is checked against.  Only the test suite,
+ * the smoke check and the benchmark's CPU-baseline leg may load it.  It
+ * shares no code, header, table or constant generator with the CUDA
+ * library, and it never calls it.
+ *
+ * Sources (the web pages this method is documented on):
+ *   [P1] "Poros on consumer GPUs", section "What you need besides VRAM":
+ *        the frozen base is stored NF4 and lives in host RAM; its size is
+ *        fixed by the NF4 storage format (~4 / ~18 / ~40 GB at 7B/32B/72B).
+ *   [P2] Poros API reference, PorosTrainer.from_pretrained: quantization
+ *        "nf4" = 4-bit NF4 QLoRA; lora_rank 16, lora_alpha 32.
+ *   [P3] HN comment (host-RAM base, prefetch-one-ahead ring): the base is
+ *        frozen, read and never written, and must only arrive before the
+ *        matmul that uses it.
+ * The pages give no codebook, block length or formula.  The readings used
+ * here (NormalFloat construction, 64-element blocks with an fp32 absmax,
+ * nibble order, tie-break, LoRA formulas) are stated next to each function.
+ *
+ * Parity pins: every function below is pinned by tests that do not re-type
+ * its formula (closed forms, exact round trips, brute-force nearest search,
+ * permutation/selection closed forms, finite differences).
+ */
+#ifndef NF4_ORACLE_H
+#define NF4_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* NormalFloat-4 codebook, 16 ascending fp32 values, derived in double. */
+void orc_nf4_codebook(float out[16]);
+
+/* Standard normal quantile by bisection on erfc (double).  Exposed so the
+ * tests can compare it to an independent inverse-CDF algorithm. */
+double orc_normal_quantile(double p);
+
+/* Index of the codebook entry nearest to x (fp32 distances, ties -> lower). */
+int orc_nf4_nearest(float x);
+
+/* Host bytes of one [n_out, k_in] NF4 weight: codes (2 per byte) + fp32
+ * absmax per 64-element block. */
+int64_t orc_nf4_storage_bytes(int64_t n_out, int64_t k_in);
+
+/* Quantize a row-major bf16 weight [n_out, k_in] (bit patterns).
+ * codes: n_out*k_in/2 bytes, element e in byte e/2, even e in the HIGH nibble.
+ * absmax: n_out*k_in/64 floats.  Returns 0, or -1 if sizes are invalid. */
+int orc_nf4_quantize(const uint16_t *w, int64_t n_out, int64_t k_in,
+                     uint8_t *codes, float *absmax);
+
+/* Dequantize to bf16 bit patterns: bf16_rne(fp32(c[code] * absmax)). */
+int orc_nf4_dequant(const uint8_t *codes, const float *absmax, int64_t n_out,
+                    int64_t k_in, uint16_t *out);
+
+/* float <-> bf16 (round to nearest even), exposed for tests. */
+uint16_t orc_f32_to_bf16(float f);
+float orc_bf16_to_f32(uint16_t h);
+
+/* ---- LoRA linear, double core (used directly by the finite-difference
+ * tests; inputs are dense doubles, W is the dense [N,K] base matrix). ----
+ *   t = X A^T                     [T,r]
+ *   Y = X W^T + s t B^T           [T,N]
+ *   u = dY B                      [T,r]
+ *   dX = dY W + s u A             [T,K]
+ *   dB = s dY^T t                 [N,r]
+ *   dA = s u^T X                  [r,K]
+ */
+void orc_lora_fwd_f64(const double *W, const double *X, const double *A,
+                      const double *B, int64_t T, int64_t N, int64_t K, int r,
+                      double s, double *Y, double *t);
+void orc_lora_bwd_f64(const double *W, const double *X, const double *A,
+                      const double *B, const double *dY, int64_t T, int64_t N,
+                      int64_t K, int r, double s, double *dX, double *dA,
+                      double *dB);
+
+/* ---- LoRA linear on the method's data types ----
+ * W given as NF4 codes + absmax; X, A, B, dY as bf16 bit patterns; every
+ * input is widened exactly, every sum is accumulated in double and rounded
+ * once to fp32.  s = alpha / r.
+ * rows/n_rows: the token rows of Y (fwd) or dX (bwd) to compute (NULL = all
+ * T rows, in order); outputs are packed [n_rows, N] / [n_rows, K].
+ * t_out [T,r], dA [r,K] and dB [N,r] always cover every token.
+ * n_threads: worker threads over output rows; results do not depend on it.
+ * Returns 0, or -1 on invalid sizes. */
+int orc_lora_fwd(const uint8_t *codes, const float *absmax, int64_t N,
+                 int64_t K, const uint16_t *X, int64_t T, const uint16_t *A,
+                 const uint16_t *B, int r, float alpha, const int64_t *rows,
+                 int64_t n_rows, float *Y, float *t_out, int n_threads);
+int orc_lora_bwd(const uint8_t *codes, const float *absmax, int64_t N,
+                 int64_t K, const uint16_t *X, int64_t T, const uint16_t *A,
+                 const uint16_t *B, int r, float alpha, const uint16_t *dY,
+                 const int64_t *rows, int64_t n_rows, float *dX, float *dA,
+                 float *dB, int n_threads);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,351 @@
+"""Pins of the CPU oracle against facts fixed by the pages and by mathematics.
+
+None of these tests re-types an oracle formula: each one checks a closed
+form, an exact round trip, an independent algorithm, a brute-force search
+or a finite-difference derivative, chosen so that a plausible mistake in the
+oracle (a dropped term, a wrong sign or scale, a transposed operand, a
+swapped nibble, a wrong tie-break) fails at least one of them.
+"""
+import json
+import os
+import statistics
+
+import numpy as np
+import pytest
+
+from host_streamed_nf4_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- codebook
+
+def test_codebook_structure(orc):
+    cb = orc.codebook()
+    assert cb.dtype == np.float32 and cb.shape == (16,)
+    assert np.all(np.diff(cb) > 0), "strictly ascending"
+    assert cb[0] == -1.0 and cb[7] == 0.0 and cb[15] == 1.0
+    assert (cb < 0).sum() == 7 and (cb > 0).sum() == 8
+
+
+def _independent_codebook():
+    """NormalFloat construction with Python's own inverse normal CDF
+    (statistics.NormalDist, a rational-approximation algorithm unrelated to
+    the oracle's bisection on erfc)."""
+    nd = statistics.NormalDist()
+    delta = 1.0 - 0.5 * (1.0 / 32.0 + 1.0 / 30.0)
+    top = nd.inv_cdf(delta)
+    pos = [nd.inv_cdf(delta + j * (0.5 - delta) / 8.0) / top for j in range(8)]
+    neg = [-nd.inv_cdf(delta + j * (0.5 - delta) / 7.0) / top for j in range(7)]
+    return np.array(sorted(neg + [0.0] + pos), np.float64)
+
+
+def test_codebook_matches_independent_quantiles(orc):
+    cb = orc.codebook().astype(np.float64)
+    ref = _independent_codebook()
+    # equal to within one fp32 ulp of the value (the two double quantile
+    # algorithms agree to ~1e-15; fp32 rounding can differ only at a tie)
+    ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
+    assert np.all(np.abs(cb - ref) <= ulp)
+    assert np.array_equal(cb.astype(np.float32), ref.astype(np.float32))
+
+
+def test_normal_quantile_against_stdlib(orc):
+    nd = statistics.NormalDist()
+    for p in (0.5, 0.55, 0.6, 0.75, 0.9, 0.9677083333333334, 0.99, 1e-6, 0.025):
+        assert abs(orc.normal_quantile(p) - nd.inv_cdf(p)) < 1e-12
+
+
+# ---------------------------------------------------------------- nearest code
+
+def test_nearest_exact_codebook_values(orc):
+    cb = orc.codebook()
+    for i, c in enumerate(cb):
+        assert orc.nearest(c) == i
+
+
+def test_nearest_tie_goes_to_lower_index(orc):
+    cb = orc.codebook()
+    # c8/2 is exactly halfway between 0 (code 7) and c8 (both distances are
+    # the same fp32 number by Sterbenz), likewise c6/2 between c6 and 0.
+    assert orc.nearest(np.float32(cb[8] / 2)) == 7
+    assert orc.nearest(np.float32(cb[6] / 2)) == 6
+
+
+def test_nearest_bruteforce_all_bf16_in_range(orc):
+    """Every bf16 value in [-1, 1] maps to a code at minimum distance
+    (distances in exact double arithmetic, allowing fp32-rounding ties)."""
+    cb = orc.codebook().astype(np.float64)
+    bits = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    xf = synth.bits_to_f32(bits)
+    keep = np.isfinite(xf) & (np.abs(xf) <= 1.0)
+    bits, x = bits[keep], xf[keep].astype(np.float64)
+    # sample to keep the ctypes loop short, plus the extremes
+    rng = np.random.default_rng(0)
+    idx = np.unique(np.concatenate([rng.choice(x.size, 6000, replace=False),
+                                    np.argsort(np.abs(x))[:50]]))
+    d = np.abs(x[idx, None] - cb[None, :])
+    dmin = d.min(axis=1)
+    for j, i in enumerate(idx):
+        code = orc.nearest(np.float32(x[i]))
+        # nearest in exact arithmetic, or tied after fp32 rounding
+        got = np.float32(d[j, code])
+        assert got <= np.float32(dmin[j]) or d[j, code] <= dmin[j] * (1 + 2**-23), (x[i], code)
+        # among exact-distance ties the lowest index wins
+        ties = np.flatnonzero(np.float32(d[j]) == np.float32(dmin[j]))
+        assert code == ties[0]
+
+
+# ---------------------------------------------------------------- quantize / dequant
+
+def _block_from_codes(rng, cb, a_bits, n_blocks):
+    """Blocks whose values are exactly dequant's outputs for random codes at a
+    bf16 scale `a`, with one element at +-a so that a is the block absmax."""
+    a = synth.bits_to_f32(np.array([a_bits], np.uint16))[0]
+    codes = rng.integers(0, 16, size=(n_blocks, 64))
+    codes[:, rng.integers(0, 64)] = rng.choice([0, 15])
+    vals = cb[codes].astype(np.float32) * np.float32(a)
+    return codes, synth.to_bf16_bits(vals), a
+
+
+def test_roundtrip_codebook_exact_blocks(orc):
+    cb = orc.codebook()
+    rng = np.random.default_rng(1)
+    # power-of-two scales and general bf16 scales, normal range only
+    for a in [2.0**m for m in (-12, -6, -1, 0, 3)] + [0.02, 0.3721, 5.5, 117.0]:
+        a_bits = synth.to_bf16_bits(np.array([a], np.float32))[0]
+        codes, w, a_f = _block_from_codes(rng, cb, a_bits, 8)
+        w = w.reshape(8, 64)
+        qc, qa = orc.quantize(w)
+        assert np.all(qa == np.float32(a_f))
+        hi, lo = qc >> 4, qc & 15
+        got = np.empty(8 * 64, np.int64)
+        got[0::2], got[1::2] = hi, lo
+        assert np.array_equal(got, codes.reshape(-1))
+        back = orc.dequant(qc, qa, 8, 64)
+        assert np.array_equal(back, w)
+
+
+def test_dequant_code_sweep_is_bf16_of_codebook(orc):
+    """codes 0..15 at absmax 1 dequantize to bf16 of the independently
+    derived codebook, in order (pins the lookup and the nibble order)."""
+    ref = _independent_codebook().astype(np.float32)
+    seq = np.tile(np.arange(16), 4)                  # 64 elements
+    packed = ((seq[0::2] << 4) | seq[1::2]).astype(np.uint8)
+    out = orc.dequant(packed, np.ones(1, np.float32), 1, 64)
+    assert np.array_equal(out.reshape(-1), synth.to_bf16_bits(ref[seq]))
+
+
+def test_all_zero_block(orc):
+    w = np.zeros((2, 64), np.uint16)
+    w[1] = 0x8000  # -0.0
+    codes, absmax = orc.quantize(w)
+    assert np.all(codes == 0x77) and np.all(absmax == 0.0)
+    out = orc.dequant(codes, absmax, 2, 64)
+    assert np.all(out == 0)  # +0.0 bit pattern
+
+
+def test_nibble_order_even_element_high(orc):
+    w = np.zeros((1, 64), np.float32)
+    w[0, 0], w[0, 1], w[0, 3] = 1.0, -1.0, 1.0
+    codes, absmax = orc.quantize(synth.to_bf16_bits(w))
+    assert absmax[0] == 1.0
+    assert codes[0] == 0xF0 and codes[1] == 0x7F and codes[2] == 0x77
+
+
+def test_absmax_is_block_max_abs(orc):
+    rng = np.random.default_rng(2)
+    w = synth.normal_bf16(rng, (32, 256), 0.02)
+    _, absmax = orc.quantize(w)
+    ref = np.abs(synth.bits_to_f32(w)).reshape(-1, 64).max(axis=1)
+    assert np.array_equal(absmax, ref)
+
+
+def test_quantize_error_bounded_by_half_gap(orc):
+    """|w - deq(w)| <= absmax * (largest half-gap) + bf16 rounding."""
+    cb = orc.codebook().astype(np.float64)
+    half_gap = np.max(np.diff(cb)) / 2
+    rng = np.random.default_rng(3)
+    w = synth.normal_bf16(rng, (64, 512), 0.02)
+    codes, absmax = orc.quantize(w)
+    back = synth.bits_to_f32(orc.dequant(codes, absmax, 64, 512)).astype(np.float64)
+    wf = synth.bits_to_f32(w).astype(np.float64)
+    a = np.repeat(absmax.astype(np.float64), 64).reshape(64, 512)
+    assert np.all(np.abs(wf - back) <= a * half_gap * (1 + 1e-6) + a * 2**-8)
+
+
+def test_rejects_bad_shapes(orc):
+    with pytest.raises(ValueError):
+        orc.quantize(np.zeros((2, 48), np.uint16))
+
+
+# ---------------------------------------------------------------- storage format
+
+def test_storage_footprint_matches_pages(orc):
+    """0.5 byte/param of codes + one fp32 per 64 params reproduces the host
+    footprints the consumer-GPU page prints for the NF4 base."""
+    g = json.load(open(os.path.join(GOLDEN, "nf4_host_footprint.json")))
+    for fam, quoted in g["quoted_gb"].items():
+        f = synth.FAMILIES[fam]
+        total = f.layers * sum(orc.storage_bytes(n, k) for _, n, k in f.projections())
+        gb = total / 1e9
+        assert abs(gb - quoted) / quoted <= g["relative_tolerance"], (fam, gb, quoted)
+
+
+def test_storage_bytes_equals_buffer_sizes(orc):
+    w = np.zeros((128, 192), np.uint16)
+    codes, absmax = orc.quantize(w)
+    assert codes.nbytes + absmax.nbytes == orc.storage_bytes(128, 192)
+
+
+# ---------------------------------------------------------------- LoRA forward
+
+def _nf4_from_dense_pm1(W):
+    """NF4 codes/absmax for a matrix with entries in {-1, 0, +1}: absmax 1
+    per block (0 for all-zero blocks), codes 0 / 7 / 15."""
+    N, K = W.shape
+    flat = W.reshape(-1)
+    codes_full = np.where(flat > 0, 15, np.where(flat < 0, 0, 7))
+    packed = ((codes_full[0::2] << 4) | codes_full[1::2]).astype(np.uint8)
+    absmax = (np.abs(flat).reshape(-1, 64).max(axis=1)).astype(np.float32)
+    return packed, absmax
+
+
+def test_fwd_permutation_base_no_adapter(orc):
+    """W = permutation-like selection, B = 0  =>  Y[t, n] = X[t, pi(n)]."""
+    rng = np.random.default_rng(4)
+    T, N, K, r = 5, 96, 128, 4
+    pi = rng.permutation(K)[:N]
+    W = np.zeros((N, K))
+    W[np.arange(N), pi] = 1.0
+    codes, absmax = _nf4_from_dense_pm1(W)
+    X = synth.normal_bf16(rng, (T, K), 1.0)
+    A = synth.normal_bf16(rng, (r, K), 0.1)
+    B = np.zeros((N, r), np.uint16)
+    Y, _ = orc.lora_fwd(codes, absmax, N, K, X, A, B, 32.0)
+    assert np.array_equal(Y, synth.bits_to_f32(X)[:, pi])
+
+
+@pytest.mark.parametrize("alpha,r", [(32.0, 16), (16.0, 16), (8.0, 4), (1.0, 4)])
+def test_fwd_adapter_selection_closed_form(orc, alpha, r):
+    """W = 0, A selects input columns sigma(j), B routes rank j to output
+    tau(j) with weight b_j (powers of two): Y[:, tau(j)] = (alpha/r) b_j X[:, sigma(j)]."""
+    rng = np.random.default_rng(5)
+    T, N, K = 3, 64, 128
+    sigma = rng.permutation(K)[:r]
+    tau = rng.permutation(N)[:r]
+    b = 2.0 ** rng.integers(-3, 3, size=r)
+    A = np.zeros((r, K), np.float32)
+    A[np.arange(r), sigma] = 1.0
+    B = np.zeros((N, r), np.float32)
+    B[tau, np.arange(r)] = b
+    codes, absmax = _nf4_from_dense_pm1(np.zeros((N, K)))
+    X = synth.normal_bf16(rng, (T, K), 1.0)
+    Y, t = orc.lora_fwd(codes, absmax, N, K, X, synth.to_bf16_bits(A), synth.to_bf16_bits(B), alpha)
+    Xf = synth.bits_to_f32(X).astype(np.float64)
+    ref = np.zeros((T, N))
+    ref[:, tau] = (alpha / r) * b[None, :] * Xf[:, sigma]
+    assert np.array_equal(Y, ref.astype(np.float32))
+    assert np.array_equal(t, Xf[:, sigma].astype(np.float32))
+
+
+def test_fwd_additive_in_base_and_adapter(orc):
+    rng = np.random.default_rng(6)
+    c = synth.linear_case(7, 4, 64, 128, r=4)
+    codes, absmax = orc.quantize(c.W)
+    zero_codes, zero_abs = _nf4_from_dense_pm1(np.zeros((64, 128)))
+    Yfull, _ = orc.lora_fwd(codes, absmax, 64, 128, c.X, c.A, c.B, 32.0)
+    Ybase, _ = orc.lora_fwd(codes, absmax, 64, 128, c.X, c.A, np.zeros_like(c.B), 32.0)
+    Ylora, _ = orc.lora_fwd(zero_codes, zero_abs, 64, 128, c.X, c.A, c.B, 32.0)
+    assert np.allclose(Yfull, Ybase.astype(np.float64) + Ylora, rtol=1e-6, atol=1e-6)
+    assert not np.allclose(Ylora, 0)
+
+
+def test_fwd_rows_subset_and_threads_deterministic(orc):
+    c = synth.linear_case(8, 16, 128, 192)
+    codes, absmax = orc.quantize(c.W)
+    Y1, t1 = orc.lora_fwd(codes, absmax, 128, 192, c.X, c.A, c.B, 32.0, n_threads=1)
+    Y8, t8 = orc.lora_fwd(codes, absmax, 128, 192, c.X, c.A, c.B, 32.0, n_threads=8)
+    rows = np.array([3, 0, 15])
+    Ys, _ = orc.lora_fwd(codes, absmax, 128, 192, c.X, c.A, c.B, 32.0, rows=rows, n_threads=3)
+    assert np.array_equal(Y1, Y8) and np.array_equal(t1, t8)
+    assert np.array_equal(Ys, Y1[rows])
+
+
+# ---------------------------------------------------------------- LoRA backward
+
+def _fd_case(seed, T=4, N=64, K=64, r=2):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((N, K)), rng.standard_normal((T, K)),
+            rng.standard_normal((r, K)), rng.standard_normal((N, r)),
+            rng.standard_normal((T, N)))
+
+
+def test_bwd_matches_central_finite_differences(orc):
+    """loss = <G, Y(X, A, B)> is linear in X and in B and bilinear in (A, B),
+    so central differences are exact up to rounding."""
+    W, X, A, B, G = _fd_case(9)
+    s = 2.0
+    dX, dA, dB = orc.lora_bwd_f64(W, X, A, B, G, s)
+
+    def loss(X_, A_, B_):
+        Y, _ = orc.lora_fwd_f64(W, X_, A_, B_, s)
+        return float(np.sum(G * Y))
+
+    h = 0.5
+    rng = np.random.default_rng(10)
+    for name, M, grad in (("X", X, dX), ("A", A, dA), ("B", B, dB)):
+        for _ in range(12):
+            idx = tuple(rng.integers(0, d) for d in M.shape)
+            P, Mm = M.copy(), M.copy()
+            P[idx] += h
+            Mm[idx] -= h
+            args_p = {"X": (P, A, B), "A": (X, P, B), "B": (X, A, P)}[name]
+            args_m = {"X": (Mm, A, B), "A": (X, Mm, B), "B": (X, A, Mm)}[name]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-9 * max(1.0, abs(fd)), (name, idx, fd, grad[idx])
+
+
+def test_bwd_zero_adapters(orc):
+    W, X, A, B, G = _fd_case(11)
+    _, _, dB = orc.lora_bwd_f64(W, X, np.zeros_like(A), B, G, 2.0)
+    assert np.all(dB == 0)
+    dX0, dA, _ = orc.lora_bwd_f64(W, X, A, np.zeros_like(B), G, 2.0)
+    assert np.all(dA == 0)
+    assert np.allclose(dX0, G @ W, rtol=0, atol=1e-12)  # no adapter => plain dY W
+
+
+def test_bwd_permutation_base_closed_form(orc):
+    """W[n, pi(n)] = 1, B = 0  =>  dX[t, pi(n)] = dY[t, n], other columns 0."""
+    rng = np.random.default_rng(12)
+    T, N, K, r = 3, 64, 128, 4
+    pi = rng.permutation(K)[:N]
+    W = np.zeros((N, K))
+    W[np.arange(N), pi] = 1.0
+    codes, absmax = _nf4_from_dense_pm1(W)
+    X = synth.normal_bf16(rng, (T, K), 1.0)
+    A = synth.normal_bf16(rng, (r, K), 0.1)
+    dY = synth.normal_bf16(rng, (T, N), 1.0)
+    dX, dA, dB = orc.lora_bwd(codes, absmax, N, K, X, A, np.zeros((N, r), np.uint16), dY, 32.0)
+    ref = np.zeros((T, K), np.float32)
+    ref[:, pi] = synth.bits_to_f32(dY)
+    assert np.array_equal(dX, ref)
+    assert np.all(dA == 0)
+
+
+def test_bf16_wrapper_equals_fp32_rounding_of_double_core(orc):
+    """The NF4/bf16 entry points are the FD-pinned double core on widened
+    inputs, rounded once to fp32."""
+    c = synth.linear_case(13, 8, 64, 128, r=4)
+    codes, absmax = orc.quantize(c.W)
+    Wd = synth.bits_to_f32(orc.dequant(codes, absmax, 64, 128)).astype(np.float64)
+    f = lambda a: synth.bits_to_f32(a).astype(np.float64)
+    Y, t = orc.lora_fwd(codes, absmax, 64, 128, c.X, c.A, c.B, 32.0)
+    s = 32.0 / 4
+    Yd, td = orc.lora_fwd_f64(Wd, f(c.X), f(c.A), f(c.B), s)
+    assert np.array_equal(Y, Yd.astype(np.float32)) and np.array_equal(t, td.astype(np.float32))
+    dX, dA, dB = orc.lora_bwd(codes, absmax, 64, 128, c.X, c.A, c.B, c.dY, 32.0)
+    dXd, dAd, dBd = orc.lora_bwd_f64(Wd, f(c.X), f(c.A), f(c.B), f(c.dY), s)
+    assert np.array_equal(dX, dXd.astype(np.float32))
+    assert np.array_equal(dA, dAd.astype(np.float32))
+    assert np.array_equal(dB, dBd.astype(np.float32))
