@@ -1,0 +1,333 @@
+"""ctypes binding of libhsnf4.so (the C ABI in include/hsnf4.h).
+
+Argument marshalling only: torch tensors provide device memory and streams,
+every step of the path runs in the library's CUDA kernels.  There is no
+fallback -- if the library or a CUDA device is missing, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, Structure, c_char_p, c_float, c_int, c_int64, c_size_t, c_uint32, \
+    c_uint64, c_void_p
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhsnf4.so")
+MAX_PROJ = 8
+
+OK, ERR_INVALID, ERR_OOM, ERR_CUDA, ERR_TIMEOUT, ERR_STATE, ERR_DEVICE = range(7)
+
+
+class Nf4WeightC(Structure):
+    _fields_ = [("codes", c_void_p), ("absmax", c_void_p), ("n_out", c_int64), ("k_in", c_int64)]
+
+
+class LayerDesc(Structure):
+    _fields_ = [("n_proj", c_int), ("n_out", c_int64 * MAX_PROJ), ("k_in", c_int64 * MAX_PROJ)]
+
+
+class StreamConfig(Structure):
+    _fields_ = [("block_size", c_int), ("enable_prefetch", c_int), ("reuse_resident", c_int),
+                ("poison_on_release", c_int)]
+
+
+class StreamStats(Structure):
+    _fields_ = [("h2d_bytes", c_uint64), ("copies", c_uint64), ("reuses", c_uint64),
+                ("acquires", c_uint64), ("releases", c_uint64)]
+
+
+class HsNf4Error(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"[{status}] {detail}")
+        self.status = status
+        self.detail = detail
+
+
+_lib = None
+
+_SIGS = {
+    "hsnf4_status_string": ([c_int], c_char_p),
+    "hsnf4_last_error": ([c_char_p, c_size_t], c_int),
+    "hsnf4_device_status": ([c_void_p, POINTER(c_uint32)], c_int),
+    "hsnf4_inject_fault": ([c_char_p], c_int),
+    "nf4_codebook": ([POINTER(c_float)], c_int),
+    "nf4_quantize_pack": ([c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p], c_int),
+    "nf4_dequant": ([c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p], c_int),
+    "lora_linear_fwd_workspace": ([c_int64, c_int64, c_int64, c_int], c_size_t),
+    "lora_linear_bwd_workspace": ([c_int64, c_int64, c_int64, c_int], c_size_t),
+    "lora_linear_fwd": ([POINTER(Nf4WeightC), c_void_p, c_int64, c_void_p, c_void_p, c_int, c_float,
+                         c_void_p, c_void_p, c_void_p, c_size_t, c_void_p], c_int),
+    "lora_linear_bwd": ([POINTER(Nf4WeightC), c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_int,
+                         c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                         c_void_p], c_int),
+    "stream_layer_bytes": ([POINTER(LayerDesc), POINTER(c_size_t)], c_int),
+    "stream_layer_offsets": ([POINTER(LayerDesc), c_int, POINTER(c_size_t), POINTER(c_size_t)], c_int),
+    "stream_slab_bytes": ([POINTER(LayerDesc), c_int, POINTER(c_size_t)], c_int),
+    "stream_ring_bytes": ([POINTER(LayerDesc), c_int, c_int, POINTER(c_size_t)], c_int),
+    "stream_create": ([c_void_p, c_size_t, POINTER(LayerDesc), c_int, POINTER(StreamConfig), c_void_p,
+                       c_size_t, c_void_p, POINTER(c_void_p)], c_int),
+    "stream_num_blocks": ([c_void_p], c_int),
+    "stream_block_prefetch": ([c_void_p, c_int], c_int),
+    "stream_block_acquire": ([c_void_p, c_int, c_void_p, POINTER(Nf4WeightC), c_int], c_int),
+    "stream_block_acquire_host": ([c_void_p, c_int, c_int], c_int),
+    "stream_block_release": ([c_void_p, c_int, c_void_p], c_int),
+    "stream_stats": ([c_void_p, POINTER(StreamStats)], c_int),
+    "stream_destroy": ([c_void_p], c_int),
+}
+
+EXPORTS = tuple(_SIGS)
+
+
+def lib():
+    """Load libhsnf4.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with "
+                              "`python -m host_streamed_nf4_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    buf = ctypes.create_string_buffer(512)
+    lib().hsnf4_last_error(buf, 512)
+    return buf.value.decode(errors="replace")
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise HsNf4Error(rc, last_error())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, device=True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+# ------------------------------------------------------------------ diagnostics
+
+def device_status(stream=None) -> int:
+    flags = c_uint32(0)
+    rc = lib().hsnf4_device_status(_stream(stream), ctypes.byref(flags))
+    if rc not in (OK, ERR_DEVICE):
+        _check(rc)
+    return int(flags.value)
+
+
+def inject_fault(site: str | None):
+    _check(lib().hsnf4_inject_fault(site.encode() if site else None))
+
+
+def codebook() -> list[float]:
+    out = (c_float * 16)()
+    _check(lib().nf4_codebook(out))
+    return list(out)
+
+
+# ------------------------------------------------------------------ NF4
+
+@dataclass
+class Nf4Weight:
+    """An NF4 weight in device memory (codes uint8, absmax fp32)."""
+    codes: torch.Tensor
+    absmax: torch.Tensor
+    n_out: int
+    k_in: int
+
+    def c(self) -> Nf4WeightC:
+        return Nf4WeightC(self.codes.data_ptr(), self.absmax.data_ptr(), self.n_out, self.k_in)
+
+
+def nf4_quantize_pack(w: torch.Tensor, codes=None, absmax=None, stream=None) -> Nf4Weight:
+    _need(w, "w", torch.bfloat16)
+    n, k = w.shape
+    if codes is None:
+        codes = torch.empty(n * k // 2, dtype=torch.uint8, device=w.device)
+    if absmax is None:
+        absmax = torch.empty(n * k // 64, dtype=torch.float32, device=w.device)
+    _check(lib().nf4_quantize_pack(_ptr(w), n, k, _ptr(codes), _ptr(absmax), _stream(stream)))
+    return Nf4Weight(codes, absmax, n, k)
+
+
+def nf4_dequant(W: Nf4Weight, out=None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(W.n_out, W.k_in, dtype=torch.bfloat16, device=W.codes.device)
+    _check(lib().nf4_dequant(_ptr(W.codes), _ptr(W.absmax), W.n_out, W.k_in, _ptr(out),
+                             _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------ LoRA linear
+
+def fwd_workspace_bytes(T, n_out, k_in, r) -> int:
+    return int(lib().lora_linear_fwd_workspace(T, n_out, k_in, r))
+
+
+def bwd_workspace_bytes(T, n_out, k_in, r) -> int:
+    return int(lib().lora_linear_bwd_workspace(T, n_out, k_in, r))
+
+
+def _weight_arg(W):
+    return ctypes.byref(W.c() if isinstance(W, Nf4Weight) else W)
+
+
+def lora_linear_fwd(W, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                    Y=None, t_save=None, workspace=None, stream=None):
+    """Y = X deq(W)^T + (alpha/r) (X A^T) B^T.  Returns (Y bf16 [T, n_out], t fp32 [T, r])."""
+    n_out, k_in = W.n_out, W.k_in
+    T, r = X.shape[0], A.shape[0]
+    if Y is None:
+        Y = torch.empty(T, n_out, dtype=torch.bfloat16, device=X.device)
+    if t_save is None:
+        t_save = torch.empty(T, r, dtype=torch.float32, device=X.device)
+    ws = fwd_workspace_bytes(T, n_out, k_in, r)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=X.device)
+    _check(lib().lora_linear_fwd(_weight_arg(W), _ptr(X), T, _ptr(A), _ptr(B), r, float(alpha),
+                                 _ptr(Y), _ptr(t_save), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)))
+    return Y, t_save
+
+
+def lora_linear_bwd(W, X, t_save, A, B, dY, alpha: float, dX=None, dA=None, dB=None,
+                    workspace=None, stream=None):
+    """Returns (dX bf16 [T, k_in], dA fp32 [r, k_in], dB fp32 [n_out, r])."""
+    n_out, k_in = W.n_out, W.k_in
+    T, r = X.shape[0], A.shape[0]
+    dev = X.device
+    if dX is None:
+        dX = torch.empty(T, k_in, dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty(r, k_in, dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty(n_out, r, dtype=torch.float32, device=dev)
+    ws = bwd_workspace_bytes(T, n_out, k_in, r)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+    _check(lib().lora_linear_bwd(_weight_arg(W), _ptr(X), _ptr(t_save), T, _ptr(A), _ptr(B), r,
+                                 float(alpha), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB),
+                                 _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dX, dA, dB
+
+
+# ------------------------------------------------------------------ streamer
+
+def layer_desc(shapes) -> LayerDesc:
+    """shapes: [(n_out, k_in), ...] of one layer's projections."""
+    d = LayerDesc()
+    d.n_proj = len(shapes)
+    for i, (n, k) in enumerate(shapes):
+        d.n_out[i] = n
+        d.k_in[i] = k
+    return d
+
+
+def layer_bytes(desc: LayerDesc) -> int:
+    out = c_size_t(0)
+    _check(lib().stream_layer_bytes(ctypes.byref(desc), ctypes.byref(out)))
+    return out.value
+
+
+def layer_offsets(desc: LayerDesc, proj: int):
+    co, ao = c_size_t(0), c_size_t(0)
+    _check(lib().stream_layer_offsets(ctypes.byref(desc), proj, ctypes.byref(co), ctypes.byref(ao)))
+    return co.value, ao.value
+
+
+def _desc_array(descs):
+    arr = (LayerDesc * len(descs))(*descs)
+    return arr
+
+
+def slab_bytes(descs) -> int:
+    out = c_size_t(0)
+    _check(lib().stream_slab_bytes(_desc_array(descs), len(descs), ctypes.byref(out)))
+    return out.value
+
+
+def ring_bytes(descs, block_size: int) -> int:
+    out = c_size_t(0)
+    _check(lib().stream_ring_bytes(_desc_array(descs), len(descs), block_size, ctypes.byref(out)))
+    return out.value
+
+
+class Streamer:
+    """Pinned-host NF4 stack -> 2-slot VRAM ring, prefetched one block ahead."""
+
+    def __init__(self, slab: torch.Tensor, descs, block_size: int, ring: torch.Tensor,
+                 copy_stream: torch.cuda.Stream, enable_prefetch=True, reuse_resident=True,
+                 poison_on_release=False):
+        _need(slab, "slab", torch.uint8, device=False)
+        if not slab.is_pinned():
+            raise ValueError("slab must be page-locked (pin_memory)")
+        _need(ring, "ring", torch.uint8)
+        self.descs = list(descs)
+        self._arr = _desc_array(self.descs)
+        cfg = StreamConfig(block_size, int(bool(enable_prefetch)), int(bool(reuse_resident)),
+                           int(bool(poison_on_release)))
+        h = c_void_p()
+        _check(lib().stream_create(_ptr(slab), slab.numel(), self._arr, len(self.descs),
+                                   ctypes.byref(cfg), _ptr(ring), ring.numel(),
+                                   ctypes.c_void_p(copy_stream.cuda_stream), ctypes.byref(h)))
+        self._h = h
+        self.slab, self.ring, self.copy_stream = slab, ring, copy_stream
+        self.block_size = block_size
+        self.n_blocks = lib().stream_num_blocks(h)
+
+    def prefetch(self, b: int):
+        _check(lib().stream_block_prefetch(self._h, b))
+
+    def acquire(self, b: int, stream=None):
+        first = b * self.block_size
+        n = sum(d.n_proj for d in self.descs[first:first + self.block_size])
+        out = (Nf4WeightC * n)()
+        _check(lib().stream_block_acquire(self._h, b, _stream(stream), out, n))
+        return list(out)
+
+    def acquire_host(self, b: int, timeout_ms: int):
+        _check(lib().stream_block_acquire_host(self._h, b, timeout_ms))
+
+    def release(self, b: int, stream=None):
+        _check(lib().stream_block_release(self._h, b, _stream(stream)))
+
+    def stats(self) -> dict:
+        s = StreamStats()
+        _check(lib().stream_stats(self._h, ctypes.byref(s)))
+        return {f: int(getattr(s, f)) for f, _ in StreamStats._fields_}
+
+    def close(self):
+        if self._h:
+            rc = lib().stream_destroy(self._h)
+            self._h = None
+            _check(rc)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

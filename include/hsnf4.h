@@ -1,0 +1,277 @@
+/*
+ * hsnf4.h -- C ABI of libhsnf4.so: host-streamed NF4 LoRA layers for B200
+ * (sm_100a).
+ *
+ * The method (from the Poros documentation pages and an HN comment by the
+ * author of a similar trainer):
+ *   - LoRA fine-tuning keeps the base weights frozen: they are read, never
+ *     written, so they need not live in VRAM; they only have to arrive
+ *     before the matmul that uses them (HN comment, "host-RAM base,
+ *     prefetch-one-ahead ring").
+ *   - The base is stored as 4-bit NF4 (Poros API reference,
+ *     PorosTrainer.from_pretrained, quantization="nf4") in pinned host RAM
+ *     ("Poros on consumer GPUs", "What you need besides VRAM") and streams
+ *     into a small pool of pre-allocated VRAM buffers, block_size decoder
+ *     layers at a time, one block ahead, on a dedicated copy stream
+ *     (HN comment; Poros API reference, block_size / enable_prefetch).
+ *   - Every targeted projection is a LoRA linear (rank r, alpha; Poros API
+ *     reference, lora_rank / lora_alpha):
+ *        Y  = X deq(W)^T + (alpha/r) (X A^T) B^T
+ *        dX = dY deq(W) + (alpha/r) (dY B) A
+ *        dB = (alpha/r) dY^T (X A^T),   dA = (alpha/r) (dY B)^T X
+ *
+ * Conventions for every entry point:
+ *   - All tensors are row-major and contiguous.  bf16 tensors are passed as
+ *     raw 16-bit storage (void*).  Pointers are DEVICE pointers unless a
+ *     parameter says "host".  Device pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *     default stream.  Work is enqueued asynchronously on it; results are
+ *     valid once the stream has reached that point.
+ *   - The caller owns every buffer (weights, activations, workspace, the
+ *     pinned slab, the ring).  The library allocates no device memory on
+ *     any call; it owns only CUDA events and the streamer's host state.
+ *   - Calls never throw.  They return an hsnf4_status; on failure a
+ *     human-readable detail (with the offending sizes) is kept per thread
+ *     and read with hsnf4_last_error().  Arguments are validated before
+ *     anything is enqueued, so a rejected call has no device side effect.
+ *   - Kernels never spin without bound: every pipeline wait gives up after
+ *     a time limit, records a flag on the device and returns.  Read and
+ *     clear those flags with hsnf4_device_status().
+ *   - Results are deterministic: no floating-point atomics, fixed
+ *     reduction orders, no dependence on buffer addresses.
+ *
+ * NF4 storage format (the reading fixed once for this library; the pages
+ * name the type but print no layout):
+ *   - W is [n_out, k_in] row-major; flat index e = n*k_in + k.
+ *   - 64-element blocks along e, one fp32 absmax per block:
+ *     absmax[n_out*k_in/64].  k_in must be a multiple of 64, so a block
+ *     never crosses a row.
+ *   - 4-bit codes, two per byte: codes[n_out*k_in/2]; element e is in byte
+ *     e/2, even e in the HIGH nibble.
+ *   - code i means the i-th entry of the 16-value NormalFloat codebook
+ *     (nf4_codebook()); value = bf16_rne(fp32(codebook[i] * absmax)).
+ *   - 0.5625 byte/param, which reproduces the host footprints of
+ *     "What you need besides VRAM" (~4 / ~18 / ~40 GB at 7B / 32B / 72B).
+ */
+#ifndef HSNF4_H
+#define HSNF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HSNF4_OK = 0,
+  HSNF4_ERR_INVALID = 1, /* bad argument (size, pointer, alignment, rank) */
+  HSNF4_ERR_OOM = 2,     /* a caller-provided buffer is too small */
+  HSNF4_ERR_CUDA = 3,    /* a CUDA runtime call failed (detail names it) */
+  HSNF4_ERR_TIMEOUT = 4, /* a bounded host wait ran out */
+  HSNF4_ERR_STATE = 5,   /* streamer protocol misuse */
+  HSNF4_ERR_DEVICE = 6   /* a kernel recorded a failed (timed-out) wait */
+} hsnf4_status;
+
+/* One NF4 weight as the kernels consume it (device pointers). */
+typedef struct {
+  const void *codes;    /* uint8 [n_out*k_in/2] */
+  const float *absmax;  /* fp32 [n_out*k_in/64] */
+  int64_t n_out, k_in;
+} hsnf4_nf4_weight;
+
+/* ----------------------------------------------------------------------- */
+/* errors and diagnostics                                                  */
+/* ----------------------------------------------------------------------- */
+
+/* Static string for a status code. */
+const char *hsnf4_status_string(int status);
+
+/* Copy this thread's last error detail into buf (NUL-terminated, truncated
+ * to n bytes).  Returns the status of that last failed call (0 if none). */
+int hsnf4_last_error(char *buf, size_t n);
+
+/* Synchronize `stream`, then read and clear the device-side failure flags
+ * that bounded waits in the kernels record (bit set = a wait gave up).
+ * *flags (host) receives the flags; returns HSNF4_ERR_DEVICE if any was set. */
+int hsnf4_device_status(void *stream, uint32_t *flags);
+
+/* Host-side fault injection for failure-path tests: the next call that
+ * reaches `site` fails with HSNF4_ERR_CUDA without calling CUDA.  Sites:
+ * "copy_enqueue" (the streamer's H2D copy), "event_record" (streamer event
+ * records).  NULL or "" clears.  Nothing is injected on the device. */
+int hsnf4_inject_fault(const char *site);
+
+/* ----------------------------------------------------------------------- */
+/* NF4 quantize / dequantize                                               */
+/* ----------------------------------------------------------------------- */
+
+/* The 16 fp32 codebook values the kernels use, ascending (host out[16]).
+ * NormalFloat construction: standard-normal quantiles at probabilities
+ * evenly spaced from 1 - (1/32 + 1/30)/2 down to 1/2 (8 positive, 7
+ * negative, plus 0), divided by the largest; derived once in double. */
+int nf4_codebook(float *out);
+
+/* Quantize + pack a bf16 weight (Poros API reference: quantization="nf4").
+ * w_bf16 [n_out, k_in] -> codes [n_out*k_in/2], absmax [n_out*k_in/64].
+ * Per block: absmax = max|w| (exact), x = w / absmax (IEEE fp32 division),
+ * code = nearest codebook entry by fp32 |x - c_i| (ties -> lower index);
+ * an all-zero block gets absmax 0 and code 7 (the 0.0 entry).
+ * Errors: INVALID if n_out < 1, k_in < 1, k_in % 64, null or misaligned
+ * pointers.  Non-finite inputs give unspecified codes. */
+int nf4_quantize_pack(const void *w_bf16, int64_t n_out, int64_t k_in,
+                      void *codes, float *absmax, void *stream);
+
+/* Dequantize NF4 to bf16: out[e] = bf16_rne(fp32(codebook[code[e]] *
+ * absmax[e/64])), bit-exact by construction.  Same errors as above. */
+int nf4_dequant(const void *codes, const float *absmax, int64_t n_out,
+                int64_t k_in, void *w_bf16_out, void *stream);
+
+/* ----------------------------------------------------------------------- */
+/* LoRA linear forward / backward (north of the ring: weights may live in  */
+/* a ring slot or in a resident buffer -- the result is bitwise the same)  */
+/* ----------------------------------------------------------------------- */
+
+/* Limits: 8 <= r <= 64 and r % 8 == 0; T >= 1; n_out, k_in multiples of
+ * 64.  alpha is any finite float; the scale is s = alpha / r (fp32). */
+
+/* Workspace bytes lora_linear_fwd needs for these sizes. */
+size_t lora_linear_fwd_workspace(int64_t T, int64_t n_out, int64_t k_in, int r);
+
+/* Forward of one LoRA linear (fused NF4 dequant + tcgen05 GEMM, the rank-r
+ * term added as an extra K-slice of the same tensor-core accumulation):
+ *   t = X A^T (fp32, written to t_save if not NULL)
+ *   Y = X deq(W)^T + s t B^T   (fp32 accumulate, bf16 out)
+ * W: NF4 weight [n_out, k_in];  X bf16 [T, k_in];  A bf16 [r, k_in];
+ * B bf16 [n_out, r];  Y bf16 [T, n_out];  t_save fp32 [T, r] or NULL.
+ * workspace: device scratch of >= lora_linear_fwd_workspace() bytes,
+ * 256-byte aligned, not read before being written, free after the stream
+ * passes the call.  Errors: INVALID (sizes, rank, pointers), OOM
+ * (workspace too small; detail gives needed vs given). */
+int lora_linear_fwd(const hsnf4_nf4_weight *W, const void *X, int64_t T,
+                    const void *A, const void *B, int r, float alpha, void *Y,
+                    float *t_save, void *workspace, size_t ws_bytes,
+                    void *stream);
+
+/* Workspace bytes lora_linear_bwd needs for these sizes. */
+size_t lora_linear_bwd_workspace(int64_t T, int64_t n_out, int64_t k_in, int r);
+
+/* Backward of one LoRA linear; W is only read:
+ *   u  = dY B                         (fp32)
+ *   dX = dY deq(W) + s u A            (bf16 out, fp32 accumulate)
+ *   dB = s dY^T t,   dA = s u^T X     (fp32 out, overwritten)
+ * t_save: fp32 [T, r] from lora_linear_fwd (t = X A^T).  dY bf16 [T, n_out],
+ * dX bf16 [T, k_in], dA fp32 [r, k_in], dB fp32 [n_out, r].
+ * Errors as for lora_linear_fwd. */
+int lora_linear_bwd(const hsnf4_nf4_weight *W, const void *X,
+                    const float *t_save, int64_t T, const void *A,
+                    const void *B, int r, float alpha, const void *dY,
+                    void *dX, float *dA, float *dB, void *workspace,
+                    size_t ws_bytes, void *stream);
+
+/* ----------------------------------------------------------------------- */
+/* Host-pinned NF4 base -> VRAM ring streamer                              */
+/* ----------------------------------------------------------------------- */
+/* HN comment: the base sits in host RAM and streams into a small pool of
+ * pre-allocated VRAM buffers, prefetched one ahead on a dedicated CUDA
+ * stream.  Poros API reference: block_size (layers per block, default 4;
+ * larger = fewer transfers, more VRAM; never affects parity),
+ * enable_prefetch, and the block manager's cross-stream lifetime safety.
+ *
+ * Layout: a stack is n_layers layers; layer l has n_proj projections.  The
+ * pinned slab holds the layers back to back; inside a layer, projection p's
+ * codes then its absmax, each starting on a 1 KiB boundary
+ * (stream_layer_offsets).  A block is block_size consecutive layers (the
+ * last block may be shorter) and is one contiguous byte range of the slab.
+ * The ring holds 2 block slots in caller-provided device memory.
+ *
+ * Protocol for block b (prefetch one ahead):
+ *   acquire(b) -> prefetch(next) -> compute on b -> release(b)
+ * prefetch(b) enqueues the H2D copy of block b on the copy stream after
+ * the target slot's previous block was released (the copy stream waits on
+ * that release event -- the lifetime fence); acquire(b) makes the compute
+ * stream wait for the copy.  A block still resident in a slot is reused
+ * without a copy (the turn-around between forward and backward passes)
+ * unless reuse is disabled. */
+
+#define HSNF4_MAX_PROJ 8
+
+typedef struct {
+  int n_proj;
+  int64_t n_out[HSNF4_MAX_PROJ];
+  int64_t k_in[HSNF4_MAX_PROJ];
+} hsnf4_layer_desc;
+
+typedef struct {
+  int block_size;      /* layers per block, >= 1 */
+  int enable_prefetch; /* 0: acquire() issues the copy itself (no overlap) */
+  int reuse_resident;  /* 1: a block already in a slot is not copied again */
+  int poison_on_release; /* debug: fill a released slot with 0xFF bytes */
+} hsnf4_stream_config;
+
+typedef struct {
+  uint64_t h2d_bytes;  /* bytes copied host -> device */
+  uint64_t copies;     /* H2D copies issued */
+  uint64_t reuses;     /* prefetches satisfied by a resident block */
+  uint64_t acquires, releases;
+} hsnf4_stream_stats;
+
+typedef struct hsnf4_streamer hsnf4_streamer;
+
+/* Bytes of one layer in the slab (multiple of 1 KiB). */
+int stream_layer_bytes(const hsnf4_layer_desc *layer, size_t *out_bytes);
+
+/* Byte offsets of projection p's codes and absmax inside its layer. */
+int stream_layer_offsets(const hsnf4_layer_desc *layer, int proj,
+                         size_t *codes_off, size_t *absmax_off);
+
+/* Total slab bytes for n_layers layers (host out). */
+int stream_slab_bytes(const hsnf4_layer_desc *layers, int n_layers,
+                      size_t *out_bytes);
+
+/* Device bytes the 2-slot ring needs for this stack and block_size. */
+int stream_ring_bytes(const hsnf4_layer_desc *layers, int n_layers,
+                      int block_size, size_t *out_bytes);
+
+/* Create a streamer.  pinned_slab: HOST pointer to page-locked memory of
+ * slab_bytes holding the stack; ring_dev: device memory of ring_bytes
+ * (>= stream_ring_bytes(), 1 KiB aligned); copy_stream: the dedicated H2D
+ * stream.  The caller keeps all three alive until stream_destroy.  Errors:
+ * INVALID, OOM (ring or slab too small: needed vs given), CUDA. */
+int stream_create(const void *pinned_slab, size_t slab_bytes,
+                  const hsnf4_layer_desc *layers, int n_layers,
+                  const hsnf4_stream_config *cfg, void *ring_dev,
+                  size_t ring_bytes, void *copy_stream,
+                  hsnf4_streamer **out);
+
+/* Number of blocks (ceil(n_layers / block_size)). */
+int stream_num_blocks(const hsnf4_streamer *s);
+
+/* Enqueue block b's H2D copy into a free slot (asynchronous).  STATE if the
+ * only candidate slot holds a block that was acquired and not released. */
+int stream_block_prefetch(hsnf4_streamer *s, int block);
+
+/* Make `compute_stream` wait for block b and return its weights:
+ * out[i*n_proj + p] for layer (first layer of b) + i, projection p;
+ * max_out must be >= layers_in_block * n_proj.  With enable_prefetch = 0
+ * the copy is issued here.  STATE if b is not prefetched. */
+int stream_block_acquire(hsnf4_streamer *s, int block, void *compute_stream,
+                         hsnf4_nf4_weight *out, int max_out);
+
+/* Host-side bounded wait until block b's copy has landed (polls the ready
+ * event); TIMEOUT after timeout_ms.  STATE if b is not prefetched. */
+int stream_block_acquire_host(hsnf4_streamer *s, int block, int timeout_ms);
+
+/* Record that compute on block b (enqueued so far on compute_stream) is
+ * done with its slot; the slot can be overwritten after that point. */
+int stream_block_release(hsnf4_streamer *s, int block, void *compute_stream);
+
+int stream_stats(const hsnf4_streamer *s, hsnf4_stream_stats *out);
+
+/* Destroy (synchronizes the copy stream; events are released). */
+int stream_destroy(hsnf4_streamer *s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -18,3 +18,10 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _fresh_library():
+    """Rebuild libhsnf4.so if any source is newer than it (no-op otherwise)."""
+    from host_streamed_nf4_b200 import build
+    build.build()

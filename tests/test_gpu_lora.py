@@ -1,0 +1,86 @@
+"""LoRA linear forward/backward on the GPU (fused NF4 dequant + tcgen05 GEMM)
+vs the fp32/double oracle, within the stated tolerance."""
+import numpy as np
+import pytest
+import torch
+
+from host_streamed_nf4_b200 import hsnf4, synth
+from gpu_util import assert_lora_close, bf16_to_f64, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(case, rows=None):
+    T, N, K, r = case.shape
+    W = hsnf4.nf4_quantize_pack(to_dev_bf16(case.W))
+    X, A, B, dY = (to_dev_bf16(a) for a in (case.X, case.A, case.B, case.dY))
+    Y, t = hsnf4.lora_linear_fwd(W, X, A, B, case.alpha)
+    dX, dA, dB = hsnf4.lora_linear_bwd(W, X, t, A, B, dY, case.alpha)
+    torch.cuda.synchronize()
+    assert hsnf4.device_status() == 0
+    return W, Y, t, dX, dA, dB
+
+
+def _check(orc, case, got, rows=None, what=""):
+    T, N, K, r = case.shape
+    W, Y, t, dX, dA, dB = got
+    codes, absmax = W.codes.cpu().numpy(), W.absmax.cpu().numpy()
+    Yr, tr = orc.lora_fwd(codes, absmax, N, K, case.X, case.A, case.B, case.alpha, rows=rows)
+    dXr, dAr, dBr = orc.lora_bwd(codes, absmax, N, K, case.X, case.A, case.B, case.dY,
+                                 case.alpha, rows=rows)
+    Yg, dXg = bf16_to_f64(Y), bf16_to_f64(dX)
+    if rows is not None:
+        Yg, dXg = Yg[rows], dXg[rows]
+    assert_lora_close(Yg, Yr, what + " Y")
+    assert_lora_close(t.cpu().numpy(), tr, what + " t")
+    assert_lora_close(dXg, dXr, what + " dX")
+    assert_lora_close(dA.cpu().numpy(), dAr, what + " dA")
+    assert_lora_close(dB.cpu().numpy(), dBr, what + " dB")
+
+
+CASES = [
+    # T, N, K, r, alpha
+    (64, 512, 512, 16, 32.0),     # the single-linear case
+    (1, 128, 128, 16, 32.0),      # one token
+    (37, 64, 64, 16, 32.0),       # smallest weight, ragged T
+    (100, 192, 320, 8, 16.0),     # N, K not multiples of 128; r = 8
+    (300, 256, 384, 32, 64.0),    # two token tiles, the second ragged
+    (256, 128, 2048, 24, 48.0),   # r = 24 (padded rank slice), long K
+    (512, 640, 1152, 64, 128.0),  # r = 64
+    (129, 384, 192, 16, 7.0),     # alpha/r not a power of two
+]
+
+
+@pytest.mark.parametrize("T,N,K,r,alpha", CASES)
+def test_lora_fwd_bwd_vs_oracle(orc, T, N, K, r, alpha):
+    case = synth.linear_case(1000 + T + N + K + r, T, N, K, r=r, alpha=alpha)
+    _check(orc, case, _run(case), what=f"T{T} N{N} K{K} r{r}")
+
+
+def test_deterministic_bitwise():
+    case = synth.linear_case(5, 300, 384, 640, r=16)
+    a = _run(case)
+    b = _run(case)
+    for x, y in zip(a[1:], b[1:]):
+        assert torch.equal(x, y)
+
+
+def test_zero_adapter_B_gives_base_only(orc):
+    """B = 0: Y is the plain NF4 matmul; dA = 0 exactly."""
+    case = synth.linear_case(6, 128, 256, 512)
+    case.B[:] = 0
+    got = _run(case)
+    _check(orc, case, got, what="B=0")
+    assert torch.count_nonzero(got[4]) == 0
+
+
+@pytest.mark.parametrize("name", ["q", "k", "o", "gate", "down"])
+def test_full_size_qwen7b_projection_sampled(orc, name):
+    """Full Qwen2.5-7B shapes at T = 512 (the benchmarked launch
+    configuration); Y and dX on 8 sampled token rows, t, dA, dB in full."""
+    fam = synth.FAMILIES["qwen2.5-7b"]
+    idx = synth.PROJ_NAMES.index(name)
+    _, N, K = fam.projections()[idx]
+    case = synth.linear_case(synth.sub_seed(42, 0, idx) % (2**31), 512, N, K)
+    rows = np.array([0, 1, 127, 128, 255, 256, 400, 511])
+    _check(orc, case, _run(case), rows=rows, what=name)
