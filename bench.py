@@ -1,0 +1,504 @@
+#!/usr/bin/env python3
+"""Benchmark of the host-streamed NF4 LoRA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload qwen2.5-7b-layer|llama-3.1-8b-stack|qwen2.5-32b-stack|
+                                qwen2.5-72b-stack]
+                    [--mode streamed|resident] [--block-size B] [--seq T]
+
+One step = forward + backward of every LoRA-targeted projection (q, k, v,
+o, gate, up, down) of the workload's layers at T tokens, with the frozen NF4
+base streamed from pinned host RAM into the 2-slot VRAM ring one block
+ahead (mode "streamed") or read from VRAM (mode "resident").  The default
+workload is one Qwen2.5-7B-shaped layer at 512 tokens, streamed: its NF4
+bytes (131 MB) cross PCIe once per step, the next step's copy running
+during this step's compute.
+
+Prints one JSON line (rank 0).  `value` is device-timed whole-job tokens/s
+with inputs resident in HBM; `e2e` is the same metric through the public
+API with the step's inputs copied from pinned host memory and its adapter
+gradients read back, every step.  `--impl reference` times the CPU oracle
+(the slow, obviously-correct implementation the tests check against) on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "tokens/s fwd+bwd NF4-streamed LoRA layers; % of PCIe/tensor roofline"
+PCIE_GEN5_X16_GBPS = 63.0  # per direction, theoretical (32 GT/s x 16 lanes, 128b/130b)
+
+WORKLOADS = {
+    # name: (family, layers, default block size, default mode)
+    "qwen2.5-7b-layer": ("qwen2.5-7b", 1, 1, "streamed"),
+    "llama-3.1-8b-stack": ("llama-3.1-8b", 32, 4, "streamed"),
+    "qwen2.5-32b-stack": ("qwen2.5-32b", 64, 4, "streamed"),
+    "qwen2.5-72b-stack": ("qwen2.5-72b", 80, 4, "streamed"),
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen2.5-7b-layer")
+    ap.add_argument("--mode", choices=["streamed", "resident"], default=None)
+    ap.add_argument("--block-size", type=int, default=None)
+    ap.add_argument("--seq", type=int, default=512)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=4.0,
+                    help="target seconds per step of the oracle sample")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    fam, L, bs, mode = WORKLOADS[a.workload]
+    a.family, a.layers = fam, L
+    a.block_size = a.block_size or bs
+    a.mode = a.mode or mode
+    return a
+
+
+# ---------------------------------------------------------------------- dist
+
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        if args.impl == "ours":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(ws, x: float) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "200"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------- peaks
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs"), d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def gemm_source_digest():
+    h = hashlib.sha256()
+    for f in ("lora_gemm.cu", "ptx.cuh", "nf4_device.cuh"):
+        h.update(open(os.path.join(ROOT, "host_streamed_nf4_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from a committed ncu summary under
+    profiles/ (a line `traffic_record: {json}`), if it was taken on the
+    current kernel source; else None."""
+    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for line in open(p, errors="replace"):
+            if not line.startswith("traffic_record:"):
+                continue
+            try:
+                d = json.loads(line.split(":", 1)[1])
+            except ValueError:
+                continue
+            if d.get("kernel") == kernel and d.get("workload") == workload and \
+                    d.get("source_digest") == gemm_source_digest():
+                return d.get("dram_bytes_per_launch")
+    return None
+
+
+# ---------------------------------------------------------------------- our arm
+
+def run_ours(args, ws, rank, local):
+    import numpy as np
+    import torch
+
+    from host_streamed_nf4_b200 import hsnf4, synth
+    from host_streamed_nf4_b200.stack import LayerStack
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fam = synth.FAMILIES[args.family]
+    streamed = args.mode == "streamed"
+    single = args.layers == 1
+    # A one-layer workload re-streams its layer every step (the layer's bytes
+    # cross PCIe once per step, the next copy overlapping this step's
+    # compute); a stack reuses the blocks still resident at each turn-around.
+    stack = LayerStack(fam, args.layers, args.seq, block_size=args.block_size, streamed=streamed,
+                       reuse_resident=not single, seed=42 + rank, device=dev)
+    compute = stack.compute
+
+    def one_step():
+        if streamed and single:
+            stack.step_single_block()
+        else:
+            stack.step()
+
+    def drain_copies():
+        # make the compute stream wait for the copy stream, so that an
+        # interval closed on the compute stream includes every copy issued
+        if streamed:
+            ev = torch.cuda.Event()
+            ev.record(stack.copy_stream)
+            compute.wait_event(ev)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize(dev)
+    assert hsnf4.device_status() == 0, "a kernel wait gave up during warm-up"
+    st0 = stack.streamer.stats() if streamed else None
+
+    # ------------------------------------------------ device-timed region
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        barrier(ws)
+        torch.cuda.synchronize(dev)
+        e0.record(compute)
+        for _ in range(K):
+            one_step()
+        drain_copies()
+        e1.record(compute)
+        torch.cuda.synchronize(dev)
+        barrier(ws)
+    ms_total = max_over_ranks(ws, e0.elapsed_time(e1))
+    ms_step = ms_total / K
+    tokens_per_step = stack.tokens_per_step()
+    value = ws * tokens_per_step * K / (ms_total / 1e3)
+    h2d_step = 0
+    if streamed:
+        st1 = stack.streamer.stats()
+        h2d_step = (st1["h2d_bytes"] - st0["h2d_bytes"]) / K
+    assert hsnf4.device_status() == 0, "a kernel wait gave up in the timed region"
+
+    # ------------------------------------------------ per-kernel timing (roofline)
+    hsnf4.profile(True)
+    for _ in range(max(2, min(K, 5))):
+        one_step()
+    torch.cuda.synchronize(dev)
+    kt = hsnf4.profile_read()
+    hsnf4.profile(False)
+    _, bf16_burst, bf16_sus, peak_src = measured_peaks()
+    gemms = {k: v for k, v in kt.items() if k.startswith("lora_gemm")}
+    dom = max(gemms, key=lambda k: gemms[k]["total_ms"])
+    d = gemms[dom]
+    achieved_tflops = d["work"] / (d["total_ms"] / 1e3) / 1e12
+    flops_per_launch = d["work"] / d["launches"]
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved_tflops, 1),
+                "peak": bf16_sus, "unit": "TFLOP/s",
+                "frac": round(achieved_tflops / bf16_sus, 4),
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a step)",
+                "traffic": recorded_traffic(dom, args.workload),
+                "flops_per_launch": flops_per_launch,
+                "avg_launch_us": round(d["total_ms"] / d["launches"] * 1e3, 2),
+                "all_kernels": {k: {"launches": v["launches"],
+                                    "avg_us": round(v["total_ms"] / v["launches"] * 1e3, 2),
+                                    "achieved": round(v["work"] / (v["total_ms"] / 1e3) / 1e12, 1)}
+                                for k, v in gemms.items()}}
+
+    # step-level binding roofline: max(PCIe bytes / link rate, FLOPs / tensor peak)
+    flops_step = sum(2.0 * args.seq * n * k * 2 for _, n, k in fam.projections()) * args.layers
+    flops_step += sum(2.0 * args.seq * stack.r * (2 * k + 2 * n) + 2.0 * args.seq * stack.r * (k + n)
+                      for _, n, k in fam.projections()) * args.layers
+    t_pcie = h2d_step / (PCIE_GEN5_X16_GBPS * 1e9)
+    t_tensor = flops_step / (bf16_sus * 1e12)
+    t_bound = max(t_pcie, t_tensor)
+    step_roofline = {"binding": "pcie" if t_pcie >= t_tensor else "tensor",
+                     "bound_ms": round(t_bound * 1e3, 4), "ms_per_step": round(ms_step, 4),
+                     "frac": round(t_bound / (ms_step / 1e3), 4),
+                     "h2d_bytes_per_step": int(h2d_step),
+                     "h2d_GBps": round(h2d_step / (ms_step / 1e3) / 1e9, 2) if streamed else None,
+                     "pcie_peak_GBps": PCIE_GEN5_X16_GBPS, "flops_per_step": flops_step}
+
+    # ------------------------------------------------ end to end through the API
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, stack, one_step, drain_copies, ws, dev)
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded normal weights/activations; no dataset)",
+        "config": {"workload": args.workload, "family": args.family, "layers": args.layers,
+                   "tokens": args.seq, "batch": 1, "mode": args.mode,
+                   "block_size": args.block_size, "rank": stack.r, "alpha": stack.alpha,
+                   "projections": [p[0] for p in fam.projections()],
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single",
+                   "l2": "no flush: every step reads > 126 MB L2 (NF4 weights + activations)"},
+        "roofline": roofline, "step_roofline": step_roofline, "e2e": e2e,
+        "gpu_launches": K * stack.kernels_per_step(),
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args, fam)
+    stack.close()
+    return out
+
+
+def run_e2e(args, stack, one_step, drain_copies, ws, dev):
+    """Same step through the public API with host buffers: each step copies
+    its activations and upstream gradients from pinned host memory and reads
+    the layer stack's adapter gradients back (device-timed)."""
+    import torch
+    host_in = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in stack.X.items()}
+    host_dy = [torch.empty_like(v, device="cpu").pin_memory() for v in stack.dY]
+    for k, v in stack.X.items():
+        host_in[k].copy_(v)
+    for h, v in zip(host_dy, stack.dY):
+        h.copy_(v)
+    grads = [g for l in range(stack.L) for g in (stack.dA[l] + stack.dB[l])]
+    host_grads = [torch.empty_like(g, device="cpu").pin_memory() for g in grads]
+    h2d = sum(t.numel() * t.element_size() for t in list(host_in.values()) + host_dy)
+    d2h = sum(t.numel() * t.element_size() for t in host_grads)
+    compute = stack.compute
+
+    def step_e2e():
+        for k, v in stack.X.items():
+            v.copy_(host_in[k], non_blocking=True)
+        for d, h in zip(stack.dY, host_dy):
+            d.copy_(h, non_blocking=True)
+        one_step()
+        for h, g in zip(host_grads, grads):
+            h.copy_(g, non_blocking=True)
+
+    for _ in range(2):
+        step_e2e()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    e0.record(compute)
+    for _ in range(K):
+        step_e2e()
+    drain_copies()
+    e1.record(compute)
+    torch.cuda.synchronize(dev)
+    barrier(ws)
+    ms = max_over_ranks(ws, e0.elapsed_time(e1))
+    return {"value": round(ws * stack.tokens_per_step() * K / (ms / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms / K, 4), "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------------- oracle
+
+_ORACLE_W = {}
+
+
+def oracle_sample(family, tokens: int, seed: int = 7):
+    """Inputs for `tokens` tokens through one layer of `family` (host arrays);
+    the layer's NF4 weights are drawn and quantized once per family."""
+    import numpy as np
+
+    import oracle
+    from host_streamed_nf4_b200 import synth
+    if family.name not in _ORACLE_W:
+        rng = np.random.default_rng(seed)
+        ws = []
+        for name, n, k in family.projections():
+            codes, absmax = oracle.quantize(synth.normal_bf16(rng, (n, k), synth.W_STD))
+            ws.append((n, k, codes, absmax,
+                       synth.normal_bf16(rng, (synth.RANK, k), synth.A_STD),
+                       synth.normal_bf16(rng, (n, synth.RANK), synth.B_STD)))
+        _ORACLE_W[family.name] = ws
+    rng = np.random.default_rng(seed + tokens)
+    cases = []
+    for n, k, codes, absmax, A, B in _ORACLE_W[family.name]:
+        cases.append((n, k, codes, absmax, synth.normal_bf16(rng, (tokens, k), 1.0), A, B,
+                      synth.normal_bf16(rng, (tokens, n), 1.0)))
+    return cases
+
+
+def oracle_step(cases, threads):
+    import oracle
+    for n, k, codes, absmax, X, A, B, dY in cases:
+        oracle.lora_fwd(codes, absmax, n, k, X, A, B, 32.0, n_threads=threads)
+    for n, k, codes, absmax, X, A, B, dY in reversed(cases):
+        oracle.lora_bwd(codes, absmax, n, k, X, A, B, dY, 32.0, n_threads=threads)
+
+
+def calibrate_tokens(family, target_s, threads):
+    """Largest sample (in tokens) whose oracle step stays near target_s."""
+    cases = oracle_sample(family, 1)
+    t = time.perf_counter()
+    oracle_step(cases, threads)
+    one = time.perf_counter() - t
+    cases = oracle_sample(family, 2)
+    t = time.perf_counter()
+    oracle_step(cases, threads)
+    two = time.perf_counter() - t
+    per_token = max(two - one, 1e-3)
+    fixed = max(one - per_token, 0.0)
+    return max(1, min(512, int((target_s - fixed) / per_token)))
+
+
+def cpu_baseline(args, family):
+    """The oracle, as it stands, on the host cores over a bounded sample of
+    the workload: `tokens` tokens through one layer, fwd + bwd, scaled to
+    tokens/s for the workload's layer count."""
+    import oracle
+    oracle.build()
+    threads = os.cpu_count() or 1
+    tokens = calibrate_tokens(family, 2.0, threads)
+    cases = oracle_sample(family, tokens)
+    times = []
+    t_end = time.perf_counter() + 15.0
+    while time.perf_counter() < t_end or len(times) < 2:
+        t = time.perf_counter()
+        oracle_step(cases, threads)
+        times.append(time.perf_counter() - t)
+        if len(times) >= 8:
+            break
+    per_layer = statistics.median(times)
+    value = tokens / (per_layer * args.layers)
+    return {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{tokens} tokens x 1 layer of {family.name} (7 projections, fwd+bwd, "
+                      f"median of {len(times)} runs), scaled to {args.layers} layer(s)"}
+
+
+def run_reference(args, ws, rank):
+    import oracle
+    from host_streamed_nf4_b200 import synth
+    if rank != 0:
+        return None
+    oracle.build()
+    family = synth.FAMILIES[args.family]
+    threads = os.cpu_count() or 1
+    tokens = calibrate_tokens(family, args.ref_seconds, threads)
+    cases = oracle_sample(family, tokens)
+    for _ in range(args.warmup):
+        oracle_step(cases, threads)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(cases, threads)
+    dt = (time.perf_counter() - t) / args.steps
+    value = tokens / (dt * args.layers)
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * args.layers * 1e3 * (args.seq / tokens), 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "family": args.family, "layers": args.layers,
+                       "tokens": args.seq, "batch": 1, "mode": "cpu-oracle"},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle",
+                             "sample": f"{tokens} tokens x 1 layer per step, scaled to "
+                                       f"{args.layers} layer(s)"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    ws, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        out = run_reference(args, ws, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    out = run_ours(args, ws, rank, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

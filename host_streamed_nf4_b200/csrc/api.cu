@@ -129,6 +129,11 @@ int hsnf4_device_status(void* stream, uint32_t* flags) {
   return HSNF4_OK;
 }
 
+int hsnf4_selftest_stall(void* stream) {
+  return cuda_status(launch_selftest_stall(static_cast<cudaStream_t>(stream)),
+                     "hsnf4_selftest_stall launch");
+}
+
 int hsnf4_inject_fault(const char* site) {
   if (!site || !*site) {
     g_fault.store(kFaultNone);

@@ -56,6 +56,14 @@ int launch_lora_gemm(GemmMode mode, const hsnf4_nf4_weight* W, const void* act, 
                      const void* lo_a, int r, int r_pad, const void* lo_b, void* out,
                      cudaStream_t st);
 
+cudaError_t launch_selftest_stall(cudaStream_t st);
+
+// Kernel timing (hsnf4_profile): bracket a launch with prof_begin/prof_end.
+enum ProfKind { kProfGemmFwd = 0, kProfGemmDx = 1, kProfDequant = 2, kProfKinds = 3 };
+bool profiling();
+void* prof_begin(cudaStream_t st);
+void prof_end(void* token, int kind, double work, cudaStream_t st);
+
 // Read and clear the device failure flags the GEMM kernels record.
 cudaError_t read_gemm_flags(uint32_t* flags);
 

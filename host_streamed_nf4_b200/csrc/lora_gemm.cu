@@ -44,6 +44,7 @@ enum : unsigned int {
   kFlagLora = 8u,
   kFlagEpilogue = 16u,
   kFlagDrain = 32u,
+  kFlagSelftest = 64u,
 };
 
 constexpr int kTileM = 128;     // rows of the MMA (W rows or k_in columns)
@@ -299,6 +300,24 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
   }
 }
 
+// One thread waits on a barrier nothing arrives at: the bounded wait must
+// give up, flag it and let the kernel finish.
+__global__ void selftest_stall_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_word = 0;
+    fence_mbar_init();
+    mbar_wait(&bar, 0, &abort_word, &g_gemm_flags, kFlagSelftest);
+  }
+}
+
+cudaError_t launch_selftest_stall(cudaStream_t st) {
+  selftest_stall_kernel<<<1, 32, 0, st>>>();
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- host side
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -388,14 +407,20 @@ int launch_lora_gemm(GemmMode mode, const hsnf4_nf4_weight* W, const void* act, 
   dim3 grid(static_cast<unsigned>((mdim + kTileM - 1) / kTileM),
             static_cast<unsigned>((T + p.BN - 1) / p.BN));
   cudaError_t e;
-  if (mode == kGemmFwd) {
-    if (configure_once<kGemmFwd>() != 0) return fail(HSNF4_ERR_CUDA, "lora gemm: smem attribute");
+  if (configure_once<kGemmFwd>() != 0 || configure_once<kGemmDx>() != 0)
+    return fail(HSNF4_ERR_CUDA, "lora gemm: smem attribute");
+  void* prof = prof_begin(st);
+  if (mode == kGemmFwd)
     lora_gemm_kernel<kGemmFwd><<<grid, kThreads, smem, st>>>(p);
-  } else {
-    if (configure_once<kGemmDx>() != 0) return fail(HSNF4_ERR_CUDA, "lora gemm: smem attribute");
+  else
     lora_gemm_kernel<kGemmDx><<<grid, kThreads, smem, st>>>(p);
-  }
   e = cudaGetLastError();
+  if (prof) {
+    // algorithmic FLOPs: the base product plus the rank-r slice
+    const double flops = (mode == kGemmFwd) ? 2.0 * T * n_out * (k_in + r)
+                                            : 2.0 * T * k_in * (n_out + r);
+    prof_end(prof, mode == kGemmFwd ? kProfGemmFwd : kProfGemmDx, flops, st);
+  }
   return cuda_status(e, "lora gemm launch");
 }
 

@@ -119,10 +119,14 @@ cudaError_t launch_nf4_dequant(const void* codes, const float* absmax, int64_t n
   const int64_t cap = static_cast<int64_t>(sms) * 8;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
+  void* prof = prof_begin(st);
   nf4_dequant_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(
       static_cast<const uint32_t*>(codes), absmax, static_cast<uint4*>(out), n_groups,
       codebook());
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  // algorithmic bytes: 0.5 B codes + 4/64 B absmax read, 2 B written per element
+  if (prof) prof_end(prof, kProfDequant, 2.5625 * static_cast<double>(n_out) * k_in, st);
+  return e;
 }
 
 }  // namespace hsnf4

@@ -103,9 +103,10 @@ struct hsnf4_streamer {
     const int l = end_layer(b) - 1;
     return layer_off[l] + layer_size[l] - layer_off[first_layer(b)];
   }
-  int find(int b) const {
+  // Slot holding block b in `state`, or -1.
+  int find(int b, SlotState state) const {
     for (int i = 0; i < 2; ++i)
-      if (slots[i].block == b && slots[i].state != kEmpty) return i;
+      if (slots[i].block == b && slots[i].state == state) return i;
     return -1;
   }
 };
@@ -290,11 +291,20 @@ int stream_block_prefetch(hsnf4_streamer* s, int block) {
   int rc = check_block("stream_block_prefetch", s, block);
   if (rc) return rc;
   std::lock_guard<std::mutex> lk(s->mu);
-  const int have = s->find(block);
-  if (have >= 0) {
-    Slot& sl = s->slots[have];
-    if (s->cfg.reuse_resident || sl.state == kLoaded || sl.state == kAcquired) {
-      if (sl.state == kReleased) sl.state = kLoaded;
+  // Already copied and not yet consumed: nothing to do.
+  if (s->find(block, kLoaded) >= 0) {
+    s->stats.reuses += 1;
+    return HSNF4_OK;
+  }
+  // Still resident from an earlier acquire (the forward/backward turn-around).
+  if (s->cfg.reuse_resident) {
+    const int rel = s->find(block, kReleased);
+    if (rel >= 0) {
+      s->slots[rel].state = kLoaded;
+      s->stats.reuses += 1;
+      return HSNF4_OK;
+    }
+    if (s->find(block, kAcquired) >= 0) {
       s->stats.reuses += 1;
       return HSNF4_OK;
     }
@@ -317,10 +327,12 @@ int stream_block_acquire(hsnf4_streamer* s, int block, void* compute_stream,
   if (max_out < need)
     return fail(HSNF4_ERR_INVALID, "stream_block_acquire: out holds %d weights, block needs %d",
                 max_out, need);
-  int i = s->find(block);
-  if (i >= 0 && s->slots[i].state == kReleased && !s->cfg.reuse_resident) i = -1;
-  if (i >= 0 && s->slots[i].state == kAcquired)
-    return fail(HSNF4_ERR_STATE, "stream_block_acquire: block %d is already acquired", block);
+  int i = s->find(block, kLoaded);
+  if (i < 0 && s->cfg.reuse_resident) {
+    if (s->find(block, kAcquired) >= 0)
+      return fail(HSNF4_ERR_STATE, "stream_block_acquire: block %d is already acquired", block);
+    i = s->find(block, kReleased);
+  }
   if (i < 0) {
     if (s->cfg.enable_prefetch)
       return fail(HSNF4_ERR_STATE, "stream_block_acquire: block %d was not prefetched", block);
@@ -359,7 +371,8 @@ int stream_block_acquire_host(hsnf4_streamer* s, int block, int timeout_ms) {
   cudaEvent_t ev;
   {
     std::lock_guard<std::mutex> lk(s->mu);
-    const int i = s->find(block);
+    int i = s->find(block, kLoaded);
+    if (i < 0) i = s->find(block, kAcquired);
     if (i < 0)
       return fail(HSNF4_ERR_STATE, "stream_block_acquire_host: block %d was not prefetched",
                   block);
@@ -382,8 +395,8 @@ int stream_block_release(hsnf4_streamer* s, int block, void* compute_stream) {
   int rc = check_block("stream_block_release", s, block);
   if (rc) return rc;
   std::lock_guard<std::mutex> lk(s->mu);
-  const int i = s->find(block);
-  if (i < 0 || s->slots[i].state != kAcquired)
+  const int i = s->find(block, kAcquired);
+  if (i < 0)
     return fail(HSNF4_ERR_STATE, "stream_block_release: block %d is not acquired", block);
   Slot& sl = s->slots[i];
   rc = record(sl.free, static_cast<cudaStream_t>(compute_stream), "release: record free");

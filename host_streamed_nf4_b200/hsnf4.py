@@ -39,6 +39,11 @@ class StreamStats(Structure):
                 ("acquires", c_uint64), ("releases", c_uint64)]
 
 
+class KernelTime(Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", c_uint64), ("total_ms", ctypes.c_double),
+                ("work", ctypes.c_double)]
+
+
 class HsNf4Error(RuntimeError):
     def __init__(self, status: int, detail: str):
         super().__init__(f"[{status}] {detail}")
@@ -53,6 +58,9 @@ _SIGS = {
     "hsnf4_last_error": ([c_char_p, c_size_t], c_int),
     "hsnf4_device_status": ([c_void_p, POINTER(c_uint32)], c_int),
     "hsnf4_inject_fault": ([c_char_p], c_int),
+    "hsnf4_selftest_stall": ([c_void_p], c_int),
+    "hsnf4_profile": ([c_int], c_int),
+    "hsnf4_profile_read": ([POINTER(KernelTime), c_int], c_int),
     "nf4_codebook": ([POINTER(c_float)], c_int),
     "nf4_quantize_pack": ([c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p], c_int),
     "nf4_dequant": ([c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p], c_int),
@@ -137,6 +145,24 @@ def device_status(stream=None) -> int:
     if rc not in (OK, ERR_DEVICE):
         _check(rc)
     return int(flags.value)
+
+
+def profile(enable: bool):
+    _check(lib().hsnf4_profile(int(bool(enable))))
+
+
+def profile_read() -> dict:
+    """{kernel name: {"launches", "total_ms", "work"}} since profile(True)."""
+    out = (KernelTime * 8)()
+    n = lib().hsnf4_profile_read(out, 8)
+    if n < 0:
+        _check(-n)
+    return {out[i].name.decode(): {"launches": int(out[i].launches), "total_ms": out[i].total_ms,
+                                   "work": out[i].work} for i in range(n)}
+
+
+def selftest_stall(stream=None):
+    _check(lib().hsnf4_selftest_stall(_stream(stream)))
 
 
 def inject_fault(site: str | None):

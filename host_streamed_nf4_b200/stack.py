@@ -1,0 +1,237 @@
+"""A stack of NF4 LoRA layers driven through the C ABI, streamed or resident.
+
+Each layer has the 7 LoRA-targeted projections of its model family.  The
+frozen NF4 base of the whole stack lives in one pinned host slab (quantized
+on the GPU, layer by layer, and copied down -- the bounded-residency load
+the consumer-GPU page describes for its streamed loader); adapters,
+activations, gradients and workspaces live in VRAM.
+
+One step = forward through the layers in order, then backward in reverse
+order (the backward needs every block's weights again).
+  * streamed: blocks of `block_size` layers are fetched into the 2-slot
+    ring, one block ahead on the copy stream; a block still resident at the
+    forward/backward turn-around is reused unless `reuse_resident=False`.
+  * resident: the whole slab is copied to VRAM once; the same kernels read
+    the same bytes from there.
+
+Inputs (synthetic, seeded): every layer sees the same activations -- X [T,
+hidden] for q/k/v/gate/up, a [T, heads*head_dim] input for o, a [T, inter]
+input for down -- and per-projection upstream gradients dY [T, n_out].  The
+layers are not chained (no attention or MLP between them): what the path is
+about is that weights arrive before their matmul and that streaming does
+not change a single bit.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import hsnf4, synth
+
+INPUT_OF = {"q": "h", "k": "h", "v": "h", "o": "o", "gate": "h", "up": "h", "down": "i"}
+
+
+def _randn_bf16(shape, std, gen, device):
+    return (torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * std).to(
+        torch.bfloat16)
+
+
+def _gen(device, seed, *keys):
+    return torch.Generator(device=device).manual_seed(synth.sub_seed(seed, *keys) % (2**63))
+
+
+class LayerStack:
+    def __init__(self, family: synth.Family, n_layers: int, T: int, *, block_size: int = 4,
+                 streamed: bool = True, reuse_resident: bool = True, enable_prefetch: bool = True,
+                 poison_on_release: bool = False, r: int = synth.RANK, alpha: float = synth.ALPHA,
+                 seed: int = 42, device=None):
+        self.device = torch.device(device) if device is not None else torch.device(
+            "cuda", torch.cuda.current_device())
+        dev = self.device
+        self.family, self.L, self.T, self.r, self.alpha = family, n_layers, T, r, alpha
+        self.block_size, self.streamed = block_size, streamed
+        self.projs = family.projections()
+        self.P = len(self.projs)
+        self.desc = hsnf4.layer_desc([(n, k) for _, n, k in self.projs])
+        self.descs = [self.desc] * n_layers
+        self.layer_bytes = hsnf4.layer_bytes(self.desc)
+        self.offs = [hsnf4.layer_offsets(self.desc, p) for p in range(self.P)]
+        self.n_blocks = (n_layers + block_size - 1) // block_size
+        self.slab = torch.empty(hsnf4.slab_bytes(self.descs), dtype=torch.uint8, pin_memory=True)
+        self._fill_slab(seed)
+
+        self.compute = torch.cuda.current_stream(dev)
+        if streamed:
+            self.ring = torch.empty(hsnf4.ring_bytes(self.descs, block_size), dtype=torch.uint8,
+                                    device=dev)
+            self.copy_stream = torch.cuda.Stream(dev)
+            self.streamer = hsnf4.Streamer(self.slab, self.descs, block_size, self.ring,
+                                           self.copy_stream, enable_prefetch=enable_prefetch,
+                                           reuse_resident=reuse_resident,
+                                           poison_on_release=poison_on_release)
+        else:
+            self.dev_slab = self.slab.to(dev)
+            self.streamer = None
+
+        # activations and upstream gradients (shared by all layers)
+        h, d = family.hidden, family.head_dim
+        g = _gen(dev, seed, 1_000_001)
+        self.X = {"h": _randn_bf16((T, h), 1.0, g, dev),
+                  "o": _randn_bf16((T, family.heads * d), 1.0, g, dev),
+                  "i": _randn_bf16((T, family.inter), 1.0, g, dev)}
+        self.dY = [_randn_bf16((T, n), 1.0, g, dev) for _, n, _ in self.projs]
+        # adapters (always resident) and per-(layer, projection) outputs kept for the backward
+        self.A, self.B, self.t, self.dA, self.dB = [], [], [], [], []
+        for l in range(n_layers):
+            ga = _gen(dev, seed, 2_000_000 + l)
+            self.A.append([_randn_bf16((r, k), synth.A_STD, ga, dev) for _, _, k in self.projs])
+            self.B.append([_randn_bf16((n, r), synth.B_STD, ga, dev) for _, n, _ in self.projs])
+            self.t.append([torch.empty(T, r, dtype=torch.float32, device=dev) for _ in self.projs])
+            self.dA.append([torch.empty(r, k, dtype=torch.float32, device=dev)
+                            for _, _, k in self.projs])
+            self.dB.append([torch.empty(n, r, dtype=torch.float32, device=dev)
+                            for _, n, _ in self.projs])
+        self.Y = [torch.empty(T, n, dtype=torch.bfloat16, device=dev) for _, n, _ in self.projs]
+        self.dX = [torch.empty(T, k, dtype=torch.bfloat16, device=dev) for _, _, k in self.projs]
+        ws_f = max(hsnf4.fwd_workspace_bytes(T, n, k, r) for _, n, k in self.projs)
+        ws_b = max(hsnf4.bwd_workspace_bytes(T, n, k, r) for _, n, k in self.projs)
+        self.ws_f = torch.empty(ws_f, dtype=torch.uint8, device=dev)
+        self.ws_b = torch.empty(ws_b, dtype=torch.uint8, device=dev)
+        self._prefetched = False
+        torch.cuda.synchronize(dev)
+
+    # ------------------------------------------------------------------ setup
+
+    def _fill_slab(self, seed: int):
+        dev = self.device
+        for l in range(self.L):
+            base = l * self.layer_bytes
+            for p, (_, n, k) in enumerate(self.projs):
+                w = _randn_bf16((n, k), synth.W_STD, _gen(dev, seed, l, p), dev)
+                W = hsnf4.nf4_quantize_pack(w)
+                co, ao = self.offs[p]
+                self.slab[base + co: base + co + n * k // 2].copy_(W.codes)
+                self.slab[base + ao: base + ao + n * k // 16].view(torch.float32).copy_(W.absmax)
+                del w, W
+        torch.cuda.synchronize(dev)
+
+    def layer_weights(self, l: int):
+        """Resident-mode weights of layer l (views into the device copy)."""
+        base = l * self.layer_bytes
+        out = []
+        for p, (_, n, k) in enumerate(self.projs):
+            co, ao = self.offs[p]
+            out.append(hsnf4.Nf4WeightC(self.dev_slab.data_ptr() + base + co,
+                                        self.dev_slab.data_ptr() + base + ao, n, k))
+        return out
+
+    def block_layers(self, b: int):
+        return range(b * self.block_size, min((b + 1) * self.block_size, self.L))
+
+    # ------------------------------------------------------------------ passes
+
+    def _weights(self, b: int):
+        if self.streamed:
+            return self.streamer.acquire(b, self.compute)
+        ws = []
+        for l in self.block_layers(b):
+            ws += self.layer_weights(l)
+        return ws
+
+    def _release(self, b: int):
+        if self.streamed:
+            self.streamer.release(b, self.compute)
+
+    def _fwd_block(self, ws, b, record):
+        for i, l in enumerate(self.block_layers(b)):
+            for p, (name, _, _) in enumerate(self.projs):
+                hsnf4.lora_linear_fwd(ws[i * self.P + p], self.X[INPUT_OF[name]], self.A[l][p],
+                                      self.B[l][p], self.alpha, Y=self.Y[p], t_save=self.t[l][p],
+                                      workspace=self.ws_f, stream=self.compute)
+                if record is not None:
+                    record(l, p, "Y", self.Y[p])
+
+    def _bwd_block(self, ws, b, record):
+        layers = list(self.block_layers(b))
+        for i in reversed(range(len(layers))):
+            l = layers[i]
+            for p in reversed(range(self.P)):
+                name = self.projs[p][0]
+                hsnf4.lora_linear_bwd(ws[i * self.P + p], self.X[INPUT_OF[name]], self.t[l][p],
+                                      self.A[l][p], self.B[l][p], self.dY[p], self.alpha,
+                                      dX=self.dX[p], dA=self.dA[l][p], dB=self.dB[l][p],
+                                      workspace=self.ws_b, stream=self.compute)
+                if record is not None:
+                    record(l, p, "dX", self.dX[p])
+
+    def forward(self, record=None):
+        nb = self.n_blocks
+        if self.streamed:
+            self.streamer.prefetch(0)
+        for b in range(nb):
+            ws = self._weights(b)
+            if self.streamed and b + 1 < nb:
+                self.streamer.prefetch(b + 1)
+            self._fwd_block(ws, b, record)
+            self._release(b)
+
+    def backward(self, record=None):
+        nb = self.n_blocks
+        if self.streamed:
+            self.streamer.prefetch(nb - 1)
+        for b in reversed(range(nb)):
+            ws = self._weights(b)
+            if self.streamed and b > 0:
+                self.streamer.prefetch(b - 1)
+            self._bwd_block(ws, b, record)
+            self._release(b)
+
+    def step(self, record=None):
+        self.forward(record)
+        self.backward(record)
+
+    def step_single_block(self, record=None):
+        """A one-block stack whose block is re-streamed every step: acquire the
+        copy made during the previous step, start the next step's copy into the
+        other slot, run forward and backward on the block, release it.  (Needs
+        reuse_resident=False, so that the prefetch makes a fresh copy.)"""
+        if not (self.streamed and self.n_blocks == 1):
+            raise ValueError("step_single_block needs a streamed one-block stack")
+        if not self._prefetched:
+            self.streamer.prefetch(0)
+            self._prefetched = True
+        ws = self.streamer.acquire(0, self.compute)
+        self.streamer.prefetch(0)
+        self._fwd_block(ws, 0, record)
+        self._bwd_block(ws, 0, record)
+        self.streamer.release(0, self.compute)
+
+    # ------------------------------------------------------------------ accounting
+
+    def block_bytes(self, b: int) -> int:
+        return len(self.block_layers(b)) * self.layer_bytes
+
+    def steady_h2d_bytes_per_step(self, reuse_resident: bool = True) -> int:
+        """Bytes one steady-state step copies host -> device.  Without reuse
+        every block crosses once per pass; with reuse the two blocks resident
+        at each turn-around (forward -> backward and backward -> the next
+        forward) are not copied again."""
+        nb = self.n_blocks
+        total = 2 * sum(self.block_bytes(b) for b in range(nb))
+        if not reuse_resident:
+            return total
+        if nb <= 2:
+            return 0
+        return total - self.block_bytes(nb - 1) - self.block_bytes(nb - 2) \
+            - self.block_bytes(0) - self.block_bytes(1)
+
+    def kernels_per_step(self) -> int:
+        # forward: rank-r projection + fused GEMM; backward: projection, GEMM, dB, dA
+        return self.L * self.P * (2 + 4)
+
+    def tokens_per_step(self) -> int:
+        return self.T
+
+    def close(self):
+        if self.streamer is not None:
+            self.streamer.close()
+            self.streamer = None

@@ -96,6 +96,31 @@ int hsnf4_last_error(char *buf, size_t n);
  * *flags (host) receives the flags; returns HSNF4_ERR_DEVICE if any was set. */
 int hsnf4_device_status(void *stream, uint32_t *flags);
 
+/* Self-test of the kernels' bounded waits: launches one CTA whose thread
+ * waits on a shared-memory barrier that nothing arrives at, through the same
+ * bounded wait the pipeline kernels use.  The wait gives up after its time
+ * limit (about 2 s), records flag 0x40 and the kernel returns; the context
+ * stays usable.  Read the flag with hsnf4_device_status(). */
+int hsnf4_selftest_stall(void *stream);
+
+/* Kernel timing for roofline reports.  While enabled, the library brackets
+ * every launch of its fused GEMM (forward and dX modes) and of the NF4
+ * dequant kernel with CUDA events on the launch stream, and accumulates
+ * per kernel: launches, device time and algorithmic work (FLOPs for the
+ * GEMMs, bytes read + written for dequant).  hsnf4_profile(1) starts (and
+ * clears), hsnf4_profile(0) stops.  hsnf4_profile_read synchronizes on the
+ * recorded events and fills out[0..n) (host), returning the number of
+ * entries (<= max_out) or a negative status. */
+typedef struct {
+  char name[32];        /* "lora_gemm_fwd", "lora_gemm_dx", "nf4_dequant" */
+  uint64_t launches;
+  double total_ms;      /* sum of per-launch event durations */
+  double work;          /* total algorithmic FLOPs or bytes */
+} hsnf4_kernel_time;
+
+int hsnf4_profile(int enable);
+int hsnf4_profile_read(hsnf4_kernel_time *out, int max_out);
+
 /* Host-side fault injection for failure-path tests: the next call that
  * reaches `site` fails with HSNF4_ERR_CUDA without calling CUDA.  Sites:
  * "copy_enqueue" (the streamer's H2D copy), "event_record" (streamer event
@@ -205,7 +230,10 @@ typedef struct {
 typedef struct {
   int block_size;      /* layers per block, >= 1 */
   int enable_prefetch; /* 0: acquire() issues the copy itself (no overlap) */
-  int reuse_resident;  /* 1: a block already in a slot is not copied again */
+  int reuse_resident;  /* 1: a prefetch of a block still resident in a slot
+                          (in use or released) is satisfied without a copy;
+                          0: only a copy not yet acquired satisfies it, so
+                          every pass re-streams its blocks */
   int poison_on_release; /* debug: fill a released slot with 0xFF bytes */
 } hsnf4_stream_config;
 

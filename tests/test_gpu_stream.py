@@ -1,0 +1,177 @@
+"""The pinned-host -> VRAM ring on the GPU.
+
+The pages' correctness bar for streaming is bitwise identity with a
+resident run, at any block_size ("Poros on consumer GPUs": NF4 is the
+precision with 0.00e+00 parity to a fully resident run; block_size never
+affects parity.  Poros API reference: elementwise-exact resident parity,
+torch.equal).  These tests hold the ring to exactly that, plus its byte
+accounting, lifetime fences and protocol errors.
+"""
+import pytest
+import torch
+
+from host_streamed_nf4_b200 import hsnf4, synth
+from host_streamed_nf4_b200.stack import LayerStack
+
+pytestmark = pytest.mark.gpu
+
+TINY = synth.Family("tiny", hidden=256, inter=640, heads=2, kv_heads=1, head_dim=128, layers=6)
+
+
+def _run(stack, steps=2):
+    rec = {}
+
+    def record(l, p, name, t):
+        rec[(l, p, name)] = t.clone()
+
+    for _ in range(steps):
+        rec.clear()
+        stack.step(record)
+    torch.cuda.synchronize()
+    assert hsnf4.device_status() == 0
+    for l in range(stack.L):
+        for p in range(stack.P):
+            rec[(l, p, "t")] = stack.t[l][p].clone()
+            rec[(l, p, "dA")] = stack.dA[l][p].clone()
+            rec[(l, p, "dB")] = stack.dB[l][p].clone()
+    return rec
+
+
+def _assert_bitwise(a, b):
+    assert a.keys() == b.keys()
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
+@pytest.fixture(scope="module")
+def resident6():
+    s = LayerStack(TINY, 6, 96, streamed=False)
+    rec = _run(s)
+    s.close()
+    return rec
+
+
+@pytest.mark.parametrize("bs", [1, 2, 4])
+def test_streamed_equals_resident_bitwise(resident6, bs):
+    s = LayerStack(TINY, 6, 96, block_size=bs, streamed=True)
+    rec = _run(s)
+    s.close()
+    _assert_bitwise(rec, resident6)
+
+
+def test_partial_last_block_bitwise():
+    res = LayerStack(TINY, 5, 64, streamed=False)
+    a = _run(res)
+    res.close()
+    for bs in (2, 4):
+        s = LayerStack(TINY, 5, 64, block_size=bs, streamed=True)
+        _assert_bitwise(_run(s), a)
+        s.close()
+
+
+@pytest.mark.parametrize("bs,reuse", [(1, True), (2, True), (4, True), (1, False), (2, False)])
+def test_h2d_bytes_match_the_schedule(bs, reuse):
+    s = LayerStack(TINY, 6, 32, block_size=bs, streamed=True, reuse_resident=reuse)
+    s.step()
+    before = s.streamer.stats()
+    s.step()
+    torch.cuda.synchronize()
+    after = s.streamer.stats()
+    moved = after["h2d_bytes"] - before["h2d_bytes"]
+    assert moved == s.steady_h2d_bytes_per_step(reuse_resident=reuse)
+    assert after["acquires"] - before["acquires"] == 2 * s.n_blocks
+    assert after["releases"] - before["releases"] == 2 * s.n_blocks
+    s.close()
+
+
+def test_poisoned_release_still_bitwise(resident6):
+    """A released slot is overwritten with 0xFF: any read after release would
+    break the bitwise comparison."""
+    s = LayerStack(TINY, 6, 96, block_size=2, streamed=True, poison_on_release=True)
+    _assert_bitwise(_run(s), resident6)
+    s.close()
+
+
+def test_no_prefetch_mode_bitwise(resident6):
+    s = LayerStack(TINY, 6, 96, block_size=2, streamed=True, enable_prefetch=False)
+    _assert_bitwise(_run(s), resident6)
+    s.close()
+
+
+# ---------------------------------------------------------------- protocol
+
+def _small_streamer(reuse=True, n_layers=4, bs=1):
+    descs = [hsnf4.layer_desc([(128, 256), (64, 128)])] * n_layers
+    slab = torch.zeros(hsnf4.slab_bytes(descs), dtype=torch.uint8, pin_memory=True)
+    ring = torch.empty(hsnf4.ring_bytes(descs, bs), dtype=torch.uint8, device="cuda")
+    cs = torch.cuda.Stream()
+    return hsnf4.Streamer(slab, descs, bs, ring, cs, reuse_resident=reuse), cs
+
+
+def _status(fn):
+    with pytest.raises(hsnf4.HsNf4Error) as e:
+        fn()
+    return e.value.status
+
+
+def test_protocol_misuse_is_reported():
+    st, _ = _small_streamer()
+    assert _status(lambda: st.release(0)) == hsnf4.ERR_STATE          # never acquired
+    assert _status(lambda: st.acquire(1)) == hsnf4.ERR_STATE          # never prefetched
+    assert _status(lambda: st.prefetch(4)) == hsnf4.ERR_INVALID       # out of range
+    st.prefetch(0)
+    st.prefetch(1)
+    assert _status(lambda: st.prefetch(2)) == hsnf4.ERR_STATE         # two ahead: no free slot
+    st.acquire(0)
+    assert _status(lambda: st.acquire(0)) == hsnf4.ERR_STATE          # double acquire
+    st.release(0)
+    st.prefetch(2)                                                   # slot of block 0 is free now
+    torch.cuda.synchronize()
+    st.close()
+
+
+def test_ring_too_small_is_oom_with_sizes():
+    descs = [hsnf4.layer_desc([(128, 256)])] * 4
+    slab = torch.zeros(hsnf4.slab_bytes(descs), dtype=torch.uint8, pin_memory=True)
+    need = hsnf4.ring_bytes(descs, 2)
+    ring = torch.empty(need - 1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(hsnf4.HsNf4Error) as e:
+        hsnf4.Streamer(slab, descs, 2, ring, torch.cuda.Stream())
+    assert e.value.status == hsnf4.ERR_OOM
+    assert str(need) in e.value.detail and "block_size" in e.value.detail
+
+
+def test_host_wait_times_out_then_succeeds():
+    st, cs = _small_streamer()
+    with torch.cuda.stream(cs):
+        torch.cuda._sleep(400_000_000)  # keep the copy stream busy (~0.2 s)
+    st.prefetch(0)
+    assert _status(lambda: st.acquire_host(0, 1)) == hsnf4.ERR_TIMEOUT
+    st.acquire_host(0, 20_000)
+    torch.cuda.synchronize()
+    st.close()
+
+
+@pytest.mark.parametrize("site", ["copy_enqueue", "event_record"])
+def test_injected_host_fault_leaves_streamer_usable(site):
+    st, _ = _small_streamer()
+    hsnf4.inject_fault(site)
+    assert _status(lambda: st.prefetch(0)) == hsnf4.ERR_CUDA
+    hsnf4.inject_fault(None)
+    st.prefetch(0)  # retry works
+    st.acquire(0)
+    st.release(0)
+    torch.cuda.synchronize()
+    st.close()
+
+
+def test_device_bounded_wait_gives_up_and_context_survives():
+    """A kernel waits on a barrier nothing arrives at: the bounded wait gives
+    up, records its flag, the kernel returns and the context stays usable."""
+    assert hsnf4.device_status() == 0
+    hsnf4.selftest_stall()
+    flags = hsnf4.device_status()
+    assert flags & 0x40
+    assert hsnf4.device_status() == 0  # reading clears
+    x = torch.arange(10, device="cuda").sum().item()
+    assert x == 45
