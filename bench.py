@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--mode", choices=["streamed", "resident"], default=None)
     ap.add_argument("--block-size", type=int, default=None)
     ap.add_argument("--seq", type=int, default=512)
+    ap.add_argument("--grouping", choices=["decoder", "layer", "none"], default="decoder",
+                    help="how a layer's projections are batched into grouped launches")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=4.0,
@@ -219,7 +221,8 @@ def run_ours(args, ws, rank, local):
     # cross PCIe once per step, the next copy overlapping this step's
     # compute); a stack reuses the blocks still resident at each turn-around.
     stack = LayerStack(fam, args.layers, args.seq, block_size=args.block_size, streamed=streamed,
-                       reuse_resident=not single, seed=42 + rank, device=dev)
+                       reuse_resident=not single, seed=42 + rank, device=dev,
+                       grouping=args.grouping)
     compute = stack.compute
 
     def one_step():
@@ -317,6 +320,7 @@ def run_ours(args, ws, rank, local):
         "config": {"workload": args.workload, "family": args.family, "layers": args.layers,
                    "tokens": args.seq, "batch": 1, "mode": args.mode,
                    "block_size": args.block_size, "rank": stack.r, "alpha": stack.alpha,
+                   "grouping": args.grouping,
                    "projections": [p[0] for p in fam.projections()],
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single",
                    "l2": "no flush: every step reads > 126 MB L2 (NF4 weights + activations)"},

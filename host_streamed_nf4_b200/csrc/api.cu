@@ -202,98 +202,243 @@ int nf4_dequant(const void* codes, const float* absmax, int64_t n_out, int64_t k
 
 static int r_padded(int r) { return (r + 15) / 16 * 16; }
 
-static int check_lora(const char* fn, const hsnf4_nf4_weight* W, int64_t T, int r) {
-  if (!W) return fail(HSNF4_ERR_INVALID, "%s: W is NULL", fn);
-  if (W->n_out < 64 || W->n_out % 64 || W->k_in < 64 || W->k_in % 64)
+static int check_weight(const char* fn, int i, const hsnf4_nf4_weight& W) {
+  if (W.n_out < 64 || W.n_out % 64 || W.k_in < 64 || W.k_in % 64)
     return fail(HSNF4_ERR_INVALID,
-                "%s: n_out and k_in must be positive multiples of 64 (got %lld x %lld)", fn,
-                (long long)W->n_out, (long long)W->k_in);
-  if (W->n_out > (1 << 30) || W->k_in > (1 << 30))
-    return fail(HSNF4_ERR_INVALID, "%s: weight dimension too large", fn);
-  if (T < 1 || T > (int64_t(1) << 30))
-    return fail(HSNF4_ERR_INVALID, "%s: T must be in [1, 2^30] (got %lld)", fn, (long long)T);
+                "%s: problem %d: n_out and k_in must be positive multiples of 64 (got %lld x %lld)",
+                fn, i, (long long)W.n_out, (long long)W.k_in);
+  if (W.n_out > (1 << 30) || W.k_in > (1 << 30))
+    return fail(HSNF4_ERR_INVALID, "%s: problem %d: weight dimension too large", fn, i);
+  return HSNF4_OK;
+}
+
+static int check_group(const char* fn, int n, int64_t T, int r, float alpha) {
+  if (n < 1 || n > 8)
+    return fail(HSNF4_ERR_INVALID, "%s: 1..8 problems per call (got %d)", fn, n);
+  if (T < 1 || T > 32768)
+    return fail(HSNF4_ERR_INVALID, "%s: T must be in [1, 32768] (got %lld)", fn, (long long)T);
   if (r < 8 || r > 64 || r % 8)
     return fail(HSNF4_ERR_INVALID, "%s: rank must be a multiple of 8 in [8, 64] (got %d)", fn, r);
-  return check_ptrs(fn, {{W->codes, "W->codes"}, {W->absmax, "W->absmax"}});
+  if (!isfinite(alpha)) return fail(HSNF4_ERR_INVALID, "%s: alpha is not finite", fn);
+  return HSNF4_OK;
+}
+
+// Workspace layout of a forward group:
+//   [s*t bf16 [T, r_pad] per problem][t fp32 [T, r] per problem without t_save]
+//   [projection partials][GEMM split-K partials + counters]
+struct FwdLayout {
+  size_t zs[8], tscratch[8], prj, gemm, total;
+};
+
+static void fwd_layout(const hsnf4_lora_fwd_args* p, int n, int64_t T, int r, FwdLayout* L) {
+  const int rp = r_padded(r);
+  size_t off = 0;
+  for (int i = 0; i < n; ++i) {
+    L->zs[i] = off;
+    off += round_up(static_cast<size_t>(T) * rp * 2, 256);
+  }
+  for (int i = 0; i < n; ++i) {
+    L->tscratch[i] = off;
+    if (!p[i].t_save) off += round_up(static_cast<size_t>(T) * r * 4, 256);
+  }
+  ProjectDesc pd[8];
+  GemmProblemDesc gd[8];
+  for (int i = 0; i < n; ++i) {
+    pd[i] = {p[i].X, p[i].W.k_in, p[i].A, true, nullptr, nullptr};
+    gd[i] = {p[i].W.codes, p[i].W.absmax, p[i].W.n_out, p[i].W.k_in, p[i].X, p[i].B, nullptr,
+             p[i].Y};
+  }
+  L->prj = off;
+  off += project_workspace_bytes(pd, n, T, r);
+  L->gemm = off;
+  off += gemm_workspace_bytes(kGemmFwd, gd, n, T, r);
+  L->total = off;
+}
+
+// Workspace layout of a backward group:
+//   [s*u bf16 [T, r_pad] per problem][u fp32 [T, r] per problem]
+//   [projection partials][GEMM split-K partials + counters]
+struct BwdLayout {
+  size_t su[8], u[8], prj, gemm, total;
+};
+
+static void bwd_layout(const hsnf4_lora_bwd_args* p, int n, int64_t T, int r, BwdLayout* L) {
+  const int rp = r_padded(r);
+  size_t off = 0;
+  for (int i = 0; i < n; ++i) {
+    L->su[i] = off;
+    off += round_up(static_cast<size_t>(T) * rp * 2, 256);
+  }
+  for (int i = 0; i < n; ++i) {
+    L->u[i] = off;
+    off += round_up(static_cast<size_t>(T) * r * 4, 256);
+  }
+  ProjectDesc pd[8];
+  GemmProblemDesc gd[8];
+  for (int i = 0; i < n; ++i) {
+    pd[i] = {p[i].dY, p[i].W.n_out, p[i].B, false, nullptr, nullptr};
+    gd[i] = {p[i].W.codes, p[i].W.absmax, p[i].W.n_out, p[i].W.k_in, p[i].dY, p[i].A, nullptr,
+             p[i].dX};
+  }
+  L->prj = off;
+  off += project_workspace_bytes(pd, n, T, r);
+  L->gemm = off;
+  off += gemm_workspace_bytes(kGemmDx, gd, n, T, r);
+  L->total = off;
+}
+
+size_t lora_group_fwd_workspace(const hsnf4_lora_fwd_args* probs, int n, int64_t T, int r) {
+  if (!probs || n < 1 || n > 8 || T < 1 || r < 1) return 0;
+  FwdLayout L;
+  fwd_layout(probs, n, T, r, &L);
+  return L.total;
+}
+
+size_t lora_group_bwd_workspace(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r) {
+  if (!probs || n < 1 || n > 8 || T < 1 || r < 1) return 0;
+  BwdLayout L;
+  bwd_layout(probs, n, T, r, &L);
+  return L.total;
+}
+
+static int check_workspace(const char* fn, void* ws, size_t have, size_t need) {
+  if (have < need)
+    return fail(HSNF4_ERR_OOM, "%s: workspace too small: need %zu bytes, given %zu", fn, need,
+                have);
+  if (need && !ws) return fail(HSNF4_ERR_INVALID, "%s: workspace is NULL", fn);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(HSNF4_ERR_INVALID, "%s: workspace must be 256-byte aligned", fn);
+  return HSNF4_OK;
+}
+
+int lora_group_fwd(const hsnf4_lora_fwd_args* probs, int n, int64_t T, int r, float alpha,
+                   void* workspace, size_t ws_bytes, void* stream) {
+  static const char* fn = "lora_group_fwd";
+  if (!probs) return fail(HSNF4_ERR_INVALID, "%s: probs is NULL", fn);
+  int rc = check_group(fn, n, T, r, alpha);
+  if (rc) return rc;
+  for (int i = 0; i < n; ++i) {
+    const hsnf4_lora_fwd_args& p = probs[i];
+    rc = check_weight(fn, i, p.W);
+    if (!rc)
+      rc = check_ptrs(fn, {{p.W.codes, "W.codes"}, {p.W.absmax, "W.absmax"}, {p.X, "X"},
+                           {p.A, "A"}, {p.B, "B"}, {p.Y, "Y"}});
+    if (!rc && p.t_save && !aligned16(p.t_save))
+      rc = fail(HSNF4_ERR_INVALID, "%s: problem %d: t_save misaligned", fn, i);
+    if (rc) return rc;
+  }
+  FwdLayout L;
+  fwd_layout(probs, n, T, r, &L);
+  rc = check_workspace(fn, workspace, ws_bytes, L.total);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const float s = alpha / static_cast<float>(r);
+  ProjectDesc pd[8];
+  GemmProblemDesc gd[8];
+  for (int i = 0; i < n; ++i) {
+    const hsnf4_lora_fwd_args& p = probs[i];
+    float* t_out = p.t_save ? p.t_save : reinterpret_cast<float*>(ws + L.tscratch[i]);
+    pd[i] = {p.X, p.W.k_in, p.A, true, t_out, ws + L.zs[i]};
+    gd[i] = {p.W.codes, p.W.absmax, p.W.n_out, p.W.k_in, p.X, p.B, ws + L.zs[i], p.Y};
+  }
+  rc = cuda_status(launch_lora_project_group(pd, n, T, r, s, ws + L.prj, st),
+                   "lora_group_fwd: projection launch");
+  if (rc) return rc;
+  return launch_lora_gemm_group(kGemmFwd, gd, n, T, r, ws + L.gemm, L.total - L.gemm, st);
+}
+
+int lora_group_bwd(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r, float alpha,
+                   void* workspace, size_t ws_bytes, void* stream) {
+  static const char* fn = "lora_group_bwd";
+  if (!probs) return fail(HSNF4_ERR_INVALID, "%s: probs is NULL", fn);
+  int rc = check_group(fn, n, T, r, alpha);
+  if (rc) return rc;
+  for (int i = 0; i < n; ++i) {
+    const hsnf4_lora_bwd_args& p = probs[i];
+    rc = check_weight(fn, i, p.W);
+    if (!rc)
+      rc = check_ptrs(fn, {{p.W.codes, "W.codes"}, {p.W.absmax, "W.absmax"}, {p.X, "X"},
+                           {p.t_save, "t_save"}, {p.A, "A"}, {p.B, "B"}, {p.dY, "dY"},
+                           {p.dX, "dX"}, {p.dA, "dA"}, {p.dB, "dB"}});
+    if (rc) return rc;
+  }
+  BwdLayout L;
+  bwd_layout(probs, n, T, r, &L);
+  rc = check_workspace(fn, workspace, ws_bytes, L.total);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const float s = alpha / static_cast<float>(r);
+  ProjectDesc pd[8];
+  GemmProblemDesc gd[8];
+  GradDesc grd[16];
+  for (int i = 0; i < n; ++i) {
+    const hsnf4_lora_bwd_args& p = probs[i];
+    float* u = reinterpret_cast<float*>(ws + L.u[i]);
+    pd[i] = {p.dY, p.W.n_out, p.B, false, u, ws + L.su[i]};
+    gd[i] = {p.W.codes, p.W.absmax, p.W.n_out, p.W.k_in, p.dY, p.A, ws + L.su[i], p.dX};
+    grd[2 * i] = {p.dY, p.W.n_out, p.t_save, p.dB, true};  // dB = s dY^T t  [n_out, r]
+    grd[2 * i + 1] = {p.X, p.W.k_in, u, p.dA, false};      // dA = s u^T X   [r, k_in]
+  }
+  rc = cuda_status(launch_lora_project_group(pd, n, T, r, s, ws + L.prj, st),
+                   "lora_group_bwd: projection launch");
+  if (rc) return rc;
+  rc = launch_lora_gemm_group(kGemmDx, gd, n, T, r, ws + L.gemm, L.total - L.gemm, st);
+  if (rc) return rc;
+  return cuda_status(launch_lora_grad_group(grd, 2 * n, T, r, s, st),
+                     "lora_group_bwd: gradient launch");
+}
+
+static hsnf4_lora_fwd_args one_fwd(const hsnf4_nf4_weight* W, const void* X, const void* A,
+                                   const void* B, void* Y, float* t_save) {
+  hsnf4_lora_fwd_args a;
+  a.W = *W;
+  a.X = X;
+  a.A = A;
+  a.B = B;
+  a.Y = Y;
+  a.t_save = t_save;
+  return a;
 }
 
 size_t lora_linear_fwd_workspace(int64_t T, int64_t n_out, int64_t k_in, int r) {
-  (void)n_out;
-  (void)k_in;
-  if (T < 1 || r < 1) return 0;
-  return round_up(static_cast<size_t>(T) * r_padded(r) * 2, 256) +  // s*t, bf16
-         round_up(static_cast<size_t>(T) * r * 4, 256);             // t, fp32 (if no t_save)
+  hsnf4_nf4_weight W = {nullptr, nullptr, n_out, k_in};
+  hsnf4_lora_fwd_args a = one_fwd(&W, nullptr, nullptr, nullptr, nullptr, nullptr);
+  return lora_group_fwd_workspace(&a, 1, T, r);
 }
 
 size_t lora_linear_bwd_workspace(int64_t T, int64_t n_out, int64_t k_in, int r) {
-  (void)n_out;
-  (void)k_in;
-  if (T < 1 || r < 1) return 0;
-  return round_up(static_cast<size_t>(T) * r_padded(r) * 2, 256) +  // s*u, bf16
-         round_up(static_cast<size_t>(T) * r * 4, 256);             // u, fp32
+  hsnf4_lora_bwd_args a;
+  memset(&a, 0, sizeof a);
+  a.W.n_out = n_out;
+  a.W.k_in = k_in;
+  return lora_group_bwd_workspace(&a, 1, T, r);
 }
 
 int lora_linear_fwd(const hsnf4_nf4_weight* W, const void* X, int64_t T, const void* A,
                     const void* B, int r, float alpha, void* Y, float* t_save, void* workspace,
                     size_t ws_bytes, void* stream) {
-  static const char* fn = "lora_linear_fwd";
-  int rc = check_lora(fn, W, T, r);
-  if (rc) return rc;
-  rc = check_ptrs(fn, {{X, "X"}, {A, "A"}, {B, "B"}, {Y, "Y"}, {workspace, "workspace"}});
-  if (rc) return rc;
-  if (t_save && !aligned16(t_save)) return fail(HSNF4_ERR_INVALID, "%s: t_save misaligned", fn);
-  if (!isfinite(alpha)) return fail(HSNF4_ERR_INVALID, "%s: alpha is not finite", fn);
-  const size_t need = lora_linear_fwd_workspace(T, W->n_out, W->k_in, r);
-  if (ws_bytes < need)
-    return fail(HSNF4_ERR_OOM, "%s: workspace too small: need %zu bytes, given %zu", fn, need,
-                ws_bytes);
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(HSNF4_ERR_INVALID, "%s: workspace must be 256-byte aligned", fn);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int rp = r_padded(r);
-  const float s = alpha / static_cast<float>(r);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  void* ts = ws;
-  float* t_out = t_save ? t_save
-                        : reinterpret_cast<float*>(ws + round_up(static_cast<size_t>(T) * rp * 2, 256));
-  rc = cuda_status(launch_lora_project(X, T, W->k_in, A, true, r, rp, s, t_out, ts, st),
-                   "lora_linear_fwd: project launch");
-  if (rc) return rc;
-  return launch_lora_gemm(kGemmFwd, W, X, T, B, r, rp, ts, Y, st);
+  if (!W) return fail(HSNF4_ERR_INVALID, "lora_linear_fwd: W is NULL");
+  hsnf4_lora_fwd_args a = one_fwd(W, X, A, B, Y, t_save);
+  return lora_group_fwd(&a, 1, T, r, alpha, workspace, ws_bytes, stream);
 }
 
 int lora_linear_bwd(const hsnf4_nf4_weight* W, const void* X, const float* t_save, int64_t T,
                     const void* A, const void* B, int r, float alpha, const void* dY, void* dX,
                     float* dA, float* dB, void* workspace, size_t ws_bytes, void* stream) {
-  static const char* fn = "lora_linear_bwd";
-  int rc = check_lora(fn, W, T, r);
-  if (rc) return rc;
-  rc = check_ptrs(fn, {{X, "X"}, {t_save, "t_save"}, {A, "A"}, {B, "B"}, {dY, "dY"}, {dX, "dX"},
-                       {dA, "dA"}, {dB, "dB"}, {workspace, "workspace"}});
-  if (rc) return rc;
-  if (!isfinite(alpha)) return fail(HSNF4_ERR_INVALID, "%s: alpha is not finite", fn);
-  const size_t need = lora_linear_bwd_workspace(T, W->n_out, W->k_in, r);
-  if (ws_bytes < need)
-    return fail(HSNF4_ERR_OOM, "%s: workspace too small: need %zu bytes, given %zu", fn, need,
-                ws_bytes);
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(HSNF4_ERR_INVALID, "%s: workspace must be 256-byte aligned", fn);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int rp = r_padded(r);
-  const float s = alpha / static_cast<float>(r);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  void* su = ws;
-  float* u = reinterpret_cast<float*>(ws + round_up(static_cast<size_t>(T) * rp * 2, 256));
-  rc = cuda_status(launch_lora_project(dY, T, W->n_out, B, false, r, rp, s, u, su, st),
-                   "lora_linear_bwd: project launch");
-  if (rc) return rc;
-  rc = launch_lora_gemm(kGemmDx, W, dY, T, A, r, rp, su, dX, st);
-  if (rc) return rc;
-  rc = cuda_status(launch_lora_grad(dY, T, W->n_out, t_save, r, s, dB, true, st),
-                   "lora_linear_bwd: dB launch");
-  if (rc) return rc;
-  return cuda_status(launch_lora_grad(X, T, W->k_in, u, r, s, dA, false, st),
-                     "lora_linear_bwd: dA launch");
+  if (!W) return fail(HSNF4_ERR_INVALID, "lora_linear_bwd: W is NULL");
+  hsnf4_lora_bwd_args a;
+  a.W = *W;
+  a.X = X;
+  a.t_save = t_save;
+  a.A = A;
+  a.B = B;
+  a.dY = dY;
+  a.dX = dX;
+  a.dA = dA;
+  a.dB = dB;
+  return lora_group_bwd(&a, 1, T, r, alpha, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"

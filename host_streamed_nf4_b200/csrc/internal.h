@@ -35,26 +35,51 @@ cudaError_t launch_nf4_quantize(const void* w, int64_t n_out, int64_t k_in, void
 cudaError_t launch_nf4_dequant(const void* codes, const float* absmax, int64_t n_out,
                                int64_t k_in, void* out, cudaStream_t st);
 
-// t = Z Adp^T (fp32 [T, r]) and zs = bf16(s * t) [T, r_pad] (pad columns 0).
-// adp_rows_major: adapter stored [r, C] (A) if true, [C, r] (B) if false.
-cudaError_t launch_lora_project(const void* Z, int64_t T, int64_t C, const void* adp,
-                                bool adp_r_major, int r, int r_pad, float s, float* t_out,
-                                void* zs, cudaStream_t st);
+// ---- rank-r projections, grouped: t_q = Z_q Adp_q^T (fp32 [T, r]) and
+// zs_q = bf16(s * t_q) ([T, r_pad], pad columns 0).  Adp is A [r, C]
+// (r_major) or B [C, r].  Workspace: project_workspace_bytes().
+struct ProjectDesc {
+  const void* Z;
+  int64_t C;
+  const void* adp;
+  bool r_major;
+  float* t_out;
+  void* zs;
+};
+size_t project_workspace_bytes(const ProjectDesc* d, int n, int64_t T, int r);
+cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, int r, float s,
+                                      void* ws, cudaStream_t st);
 
-// out = s * Z^T V: Z bf16 [T, C], V fp32 [T, r].  out_c_major: out is [C, r]
-// (dB) if true, [r, C] (dA) if false.
-cudaError_t launch_lora_grad(const void* Z, int64_t T, int64_t C, const float* V, int r,
-                             float s, float* out, bool out_c_major, cudaStream_t st);
+// ---- adapter gradients, grouped: out_q = s Z_q^T V_q, Z bf16 [T, C],
+// V fp32 [T, r]; out is [C, r] (c_major, dB) or [r, C] (dA).
+struct GradDesc {
+  const void* Z;
+  int64_t C;
+  const float* V;
+  float* out;
+  bool c_major;
+};
+cudaError_t launch_lora_grad_group(const GradDesc* d, int n, int64_t T, int r, float s,
+                                   cudaStream_t st);
 
 enum GemmMode { kGemmFwd = 0, kGemmDx = 1 };
 
-// Fused NF4 dequant + tcgen05 GEMM with the rank-r slice.
+// ---- fused NF4 dequant + tcgen05 GEMM with the rank-r slice, grouped:
 //  fwd: out[T, n_out] = act[T, k_in] deq(W)^T + lo_b[T, r_pad] lo_a[n_out, r]^T
 //  dx : out[T, k_in]  = act[T, n_out] deq(W) + lo_b[T, r_pad] lo_a[r, k_in]
 // lo_b is the pre-scaled bf16 rank-r factor (s*t or s*u).
-int launch_lora_gemm(GemmMode mode, const hsnf4_nf4_weight* W, const void* act, int64_t T,
-                     const void* lo_a, int r, int r_pad, const void* lo_b, void* out,
-                     cudaStream_t st);
+struct GemmProblemDesc {
+  const void* codes;
+  const float* absmax;
+  int64_t n_out, k_in;
+  const void* act;
+  const void* lo_a;
+  const void* lo_b;
+  void* out;
+};
+size_t gemm_workspace_bytes(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r);
+int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r,
+                           void* workspace, size_t ws_bytes, cudaStream_t st);
 
 cudaError_t launch_selftest_stall(cudaStream_t st);
 

@@ -1,5 +1,6 @@
 // lora_gemm.cu -- fused NF4 dequant + tcgen05 GEMM with the rank-r LoRA term
-// folded into the same tensor-core accumulation (sm_100a).
+// folded into the same tensor-core accumulation (sm_100a), for a group of
+// independent LoRA linears in one persistent launch.
 //
 // Forward of a LoRA linear (Poros API reference, lora_rank/lora_alpha; the
 // frozen base is only read -- HN comment on host-RAM streaming):
@@ -8,27 +9,40 @@
 //     dX[T, k_in] = dY[T, n_out] deq(W) + (s u)[T, r] A[r, k_in]
 //
 // Both are computed transposed, with the weight on the MMA's M side so that
-// a CTA dequantizes one 128-row slab of W once for all of its tokens:
-//     fwd: D[n, t] = sum_k deq(W)[n, k] X[t, k]      (A op K-major)
-//     dx : D[k, t] = sum_n deq(W)[n, k] dY[t, n]     (A op MN-major)
+// a CTA dequantizes each 128-row slab of W once for up to 512 tokens:
+//     fwd: D[n, t] = sum_k deq(W)[n, k] X[t, k]      (A operand K-major)
+//     dx : D[k, t] = sum_n deq(W)[n, k] dY[t, n]     (A operand MN-major)
 // The rank-r term is one more K-slice of the same accumulator:
 //     fwd: D[n, t] += sum_j B[n, j] (s t)[t, j]
 //     dx : D[k, t] += sum_j A[j, k] (s u)[t, j]
 //
-// CTA roles (192 threads, one output tile of 128 x BN per CTA):
-//   warp 4      TMA producer: activation tile (bf16, 128B swizzle) and the
-//               raw code tile per 64-wide K step, plus the rank-r operands;
-//   warp 5      TMEM owner and UMMA issuer (one elected thread);
-//   warps 0..3  dequantize the code tile into the UMMA A-operand layout in
-//               shared memory (one 64-element block = one 128-byte line per
-//               thread), then run the epilogue (TMEM -> bf16 -> global).
+// Work units are (problem, 128-row tile, token tile, K split).  The host
+// assigns them to persistent CTAs longest-first (static, deterministic).
+// A problem whose units are long and few is split along K: each split
+// writes its fp32 tile to workspace and the last split to arrive adds them
+// in split order, so the sum does not depend on timing.
+//
+// CTA roles (15 warps):
+//   warps 0-3, 4-7   two dequant warpgroups taking alternate K steps: raw
+//                    codes (smem) -> bf16 A tile in the UMMA 128B-swizzled
+//                    layout, one 64-element block (one 128-byte line) per
+//                    thread;
+//   warps 8-11       epilogue: TMEM -> registers -> smem transpose ->
+//                    coalesced bf16 rows of the output (or fp32 partials);
+//   warp 12          TMA producer of the activation tiles and rank-r operands;
+//   warp 13          TMA producer of the raw code tiles;
+//   warp 14          TMEM owner and UMMA issuer (one elected thread).
 // Every wait is bounded (ptx.cuh); a timed-out wait records a flag in
 // g_gemm_flags, the CTA drains what it started and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <cstddef>
 #include <mutex>
+#include <queue>
+#include <vector>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -47,82 +61,139 @@ enum : unsigned int {
   kFlagSelftest = 64u,
 };
 
-constexpr int kTileM = 128;     // rows of the MMA (W rows or k_in columns)
-constexpr int kStepK = 64;      // contraction per pipeline stage
-constexpr int kCodeBytes = 4096;          // raw codes of one stage (128 x 64 / 2)
-constexpr int kATileBytes = kTileM * 128;  // dequantized bf16 A tile
-constexpr int kMaxSmem = 232448;           // 227 KiB opt-in per block
-constexpr int kThreads = 192;
+constexpr int kTileM = 128;                    // rows of the MMA (W rows or k_in columns)
+constexpr int kStepK = 64;                     // contraction per pipeline step
+constexpr int kCodeBytes = 4096;               // raw codes of one step (128 x 64 / 2)
+constexpr int kATileBytes = kTileM * 128;      // dequantized bf16 A tile
+constexpr int kStageElems = 16 * kTileM;       // epilogue transpose buffer: 16 tokens x 128 rows
+constexpr int kMaxSmem = 232448;               // 227 KiB opt-in per block
+constexpr int kThreads = 15 * 32;
+constexpr int kWarpEpi = 8, kWarpProdX = 12, kWarpProdC = 13, kWarpMma = 14;
+
+struct GemmProblem {
+  CUtensorMap map_act;    // X / dY: bf16 [T, contraction], box {64, min(BN,256)}, 128B swizzle
+  CUtensorMap map_codes;  // uint8 [n_out, k_in/2]; box {32, 128} fwd, {64, 64} dx
+  CUtensorMap map_lo_a;   // fwd: B [n_out, r] box {16, 128} 32B; dx: A [r, k_in] box {64, r_pad} 128B
+  CUtensorMap map_lo_b;   // s*t or s*u: bf16 [T, r_pad], box {16, min(BN,256)}, 32B swizzle
+  const float* absmax;
+  uint16_t* out;          // bf16 [T, m_total]
+  float* partial;         // split-K partial tiles (fp32 [128][BN] each), or null
+  unsigned int* counter;  // split-K arrival counters, one per (row tile, token tile)
+  int n_out, k_in, m_total, nk, kblocks, m_tiles, splits;
+};
+
+constexpr int kMaxProblems = 8;
+constexpr int kMaxCtas = 160;
+constexpr int kMaxUnits = 3072;
 
 struct GemmParams {
-  CUtensorMap map_act;    // X / dY: bf16 [T, contraction], box {64, BN}, 128B swizzle
-  CUtensorMap map_codes;  // uint8 [n_out, k_in/2]; box {32, 128} fwd, {64, 64} dx
-  CUtensorMap map_lo_a;   // fwd: B [n_out, r] box {16, 128} 32B swz; dx: A [r, k_in] box {64, r_pad} 128B swz
-  CUtensorMap map_lo_b;   // s*t or s*u: bf16 [T, r_pad], box {16, BN}, 32B swizzle
-  const float* absmax;
-  uint16_t* out;
+  GemmProblem prob[kMaxProblems];
   Nf4Codebook cb;
-  int T, n_out, k_in, r_pad;
-  int BN, stages, tmem_cols;
+  int T, BN, r_pad, n_acc, sx, sc, sa, tmem_cols;
+  uint16_t cta_off[kMaxCtas + 1];
+  uint32_t units[kMaxUnits];  // problem(3) | split(5) | token tile(6) | row tile(18)
 };
+
+__host__ __device__ inline uint32_t pack_unit(int p, int s, int tt, int mt) {
+  return (static_cast<uint32_t>(p) << 29) | (static_cast<uint32_t>(s) << 24) |
+         (static_cast<uint32_t>(tt) << 18) | static_cast<uint32_t>(mt);
+}
+
+struct Unit {
+  int p, split, tt, mt, kb0, kb1;
+};
+
+__device__ __forceinline__ Unit unpack_unit(const GemmParams& P, uint32_t u) {
+  Unit r;
+  r.p = u >> 29;
+  r.split = (u >> 24) & 31;
+  r.tt = (u >> 18) & 63;
+  r.mt = u & 0x3FFFF;
+  const int nk = P.prob[r.p].nk, S = P.prob[r.p].splits;
+  r.kb0 = r.split * nk / S;
+  r.kb1 = (r.split + 1) * nk / S;
+  return r;
+}
 
 struct SmemPlan {
-  int stage_bytes, lora_a_bytes, lora_b_bytes, bar_off, total;
+  int x_bytes, a_off, c_off, la_off, lb_off, st_off, bar_off, total;
 };
 
-__host__ __device__ inline SmemPlan smem_plan(int mode, int BN, int stages, int r_pad) {
+__host__ __device__ inline SmemPlan smem_plan(int mode, int BN, int sx, int sc, int sa, int r_pad) {
   SmemPlan p;
-  p.stage_bytes = BN * 128 + kATileBytes + kCodeBytes;
   const int slices = r_pad / 16;
-  p.lora_a_bytes = (mode == kGemmFwd) ? slices * 4096 : 2 * r_pad * 128;
-  p.lora_b_bytes = slices * BN * 32;
-  p.bar_off = stages * p.stage_bytes + p.lora_a_bytes + p.lora_b_bytes;
-  p.total = p.bar_off + (3 * stages + 3) * 8 + 16;
+  p.x_bytes = BN * 128;
+  p.a_off = sx * p.x_bytes;
+  p.c_off = p.a_off + sa * kATileBytes;
+  p.la_off = p.c_off + sc * kCodeBytes;
+  const int la = (mode == kGemmFwd) ? slices * 4096 : 2 * r_pad * 128;
+  p.lb_off = p.la_off + la;
+  p.st_off = p.lb_off + slices * BN * 32;
+  p.bar_off = p.st_off + 2 * kStageElems * 2;
+  p.total = p.bar_off + (2 * sx + 2 * sc + 2 * sa + 8) * 8 + 32;
   return p;
 }
 
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_constant__ GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int S = p.stages, BN = p.BN;
-  const SmemPlan plan = smem_plan(MODE, BN, S, p.r_pad);
+  const int BN = P.BN, SX = P.sx, SC = P.sc, SA = P.sa;
+  const SmemPlan plan = smem_plan(MODE, BN, SX, SC, SA, P.r_pad);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kTileM;  // W row (fwd) / k_in column (dx)
-  const int t0 = blockIdx.y * BN;
-  const int nk = (MODE == kGemmFwd) ? p.k_in / kStepK : p.n_out / kStepK;
-  const int slices = p.r_pad / 16;
-  const int kblocks = p.k_in / 64;  // absmax blocks per W row
+  const int slices = P.r_pad / 16;
+  const int u_begin = P.cta_off[blockIdx.x], u_end = P.cta_off[blockIdx.x + 1];
+  const int box_rows = BN < 256 ? BN : 256;  // TMA boxes of activations / rank-r factor
 
-  uint8_t* lora_a = smem + S * plan.stage_bytes;
-  uint8_t* lora_b = lora_a + plan.lora_a_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + plan.bar_off);
-  uint64_t* deq = full + S;
-  uint64_t* empty = deq + S;
-  uint64_t* lora_bar = empty + S;
-  uint64_t* acc_bar = lora_bar + 1;
-  uint64_t* drain_bar = acc_bar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint8_t* lora_a = smem + plan.la_off;
+  uint8_t* lora_b = smem + plan.lb_off;
+  uint16_t* stage = reinterpret_cast<uint16_t*>(smem + plan.st_off);
+  uint64_t* x_full = reinterpret_cast<uint64_t*>(smem + plan.bar_off);
+  uint64_t* x_empty = x_full + SX;
+  uint64_t* c_full = x_empty + SX;
+  uint64_t* c_empty = c_full + SC;
+  uint64_t* a_full = c_empty + SC;
+  uint64_t* a_empty = a_full + SA;
+  uint64_t* lora_full = a_empty + SA;
+  uint64_t* lora_empty = lora_full + 1;
+  uint64_t* acc_full = lora_empty + 1;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain_bar = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto act_tile = [&](int s) { return smem + s * plan.stage_bytes; };
-  auto a_tile = [&](int s) { return smem + s * plan.stage_bytes + BN * 128; };
-  auto code_tile = [&](int s) { return smem + s * plan.stage_bytes + BN * 128 + kATileBytes; };
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  auto x_tile = [&](int s) { return smem + s * plan.x_bytes; };
+  auto a_tile = [&](int s) { return smem + plan.a_off + s * kATileBytes; };
+  auto c_tile = [&](int s) { return smem + plan.c_off + s * kCodeBytes; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&deq[s], 128);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < SX; ++s) {
+      mbar_init(&x_full[s], 1);
+      mbar_init(&x_empty[s], 1);
     }
-    mbar_init(lora_bar, 1);
-    mbar_init(acc_bar, 1);
+    for (int s = 0; s < SC; ++s) {
+      mbar_init(&c_full[s], 1);
+      mbar_init(&c_empty[s], 128);
+    }
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(&a_full[s], 128);
+      mbar_init(&a_empty[s], 1);
+    }
+    mbar_init(lora_full, 1);
+    mbar_init(lora_empty, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 128);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
-    tmem_alloc(tmem_slot, static_cast<uint32_t>(p.tmem_cols));
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_slot, static_cast<uint32_t>(P.tmem_cols));
     tmem_relinquish();
   }
   tc_fence_before();
@@ -130,173 +201,325 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // idesc: M = 128, N = BN; fwd A is K-major, dx A is MN-major; B K-major.
-  const uint32_t idesc = make_idesc_bf16(kTileM, BN, MODE == kGemmDx ? 1 : 0, 0);
-
-  int issued_phase[8];  // producer: parity of the last load issued per stage (-1 none)
+  int last_x = -1, last_c = -1, last_l = -1;  // producers: last issued sequence numbers
   bool mma_started = false;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ producer
+  if (warp == kWarpProdX) {
+    // -------------------------------------------------- activations + rank-r operands
     if (lane == 0) {
-      for (int s = 0; s < 8; ++s) issued_phase[s] = -1;
-      tma_prefetch_desc(&p.map_act);
-      tma_prefetch_desc(&p.map_codes);
-      mbar_arrive_expect_tx(lora_bar,
-                            static_cast<uint32_t>(plan.lora_a_bytes + plan.lora_b_bytes));
-      if (MODE == kGemmFwd) {
-        for (int j = 0; j < slices; ++j)
-          tma_load_2d(lora_a + j * 4096, &p.map_lo_a, lora_bar, j * 16, m0);
-      } else {
-        for (int h = 0; h < 2; ++h)
-          tma_load_2d(lora_a + h * p.r_pad * 128, &p.map_lo_a, lora_bar, m0 + h * 64, 0);
-      }
-      for (int j = 0; j < slices; ++j)
-        tma_load_2d(lora_b + j * BN * 32, &p.map_lo_b, lora_bar, j * 16, t0);
-      const uint32_t stage_tx = static_cast<uint32_t>(BN * 128 + kCodeBytes);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % S, round = kb / S;
-        if (kb >= S && !mbar_wait(&empty[s], (round - 1) & 1, abort_flag, &g_gemm_flags,
-                                  kFlagProducer))
+      int g = 0, lu = 0;
+      const uint32_t lora_tx = static_cast<uint32_t>(plan.st_off - plan.la_off);
+      bool ok = true;
+      for (int ui = u_begin; ui < u_end && ok; ++ui, ++lu) {
+        const Unit U = unpack_unit(P, P.units[ui]);
+        const GemmProblem& pr = P.prob[U.p];
+        const int m0 = U.mt * kTileM, t0 = U.tt * BN;
+        for (int kb = U.kb0; kb < U.kb1; ++kb, ++g) {
+          const int s = g % SX;
+          if (g >= SX && !mbar_wait(&x_empty[s], ((g / SX) - 1) & 1, abort_flag, &g_gemm_flags,
+                                    kFlagProducer)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&x_full[s], static_cast<uint32_t>(BN * 128));
+          for (int h = 0; h * box_rows < BN; ++h)
+            tma_load_2d(x_tile(s) + h * box_rows * 128, &pr.map_act, &x_full[s], kb * kStepK,
+                        t0 + h * box_rows);
+          last_x = g;
+        }
+        if (!ok) break;
+        // rank-r operands after the unit's activation tiles: the previous
+        // unit's rank-r slice has long been consumed by then
+        if (lu > 0 && !mbar_wait(lora_empty, (lu - 1) & 1, abort_flag, &g_gemm_flags,
+                                 kFlagProducer))
           break;
-        mbar_arrive_expect_tx(&full[s], stage_tx);
-        tma_load_2d(act_tile(s), &p.map_act, &full[s], kb * kStepK, t0);
-        if (MODE == kGemmFwd)
-          tma_load_2d(code_tile(s), &p.map_codes, &full[s], kb * 32, m0);
-        else
-          tma_load_2d(code_tile(s), &p.map_codes, &full[s], m0 / 2, kb * kStepK);
-        issued_phase[s] = round & 1;
+        mbar_arrive_expect_tx(lora_full, lora_tx);
+        if (MODE == kGemmFwd) {
+          for (int j = 0; j < slices; ++j)
+            tma_load_2d(lora_a + j * 4096, &pr.map_lo_a, lora_full, j * 16, m0);
+        } else {
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(lora_a + h * P.r_pad * 128, &pr.map_lo_a, lora_full, m0 + h * 64, 0);
+        }
+        for (int j = 0; j < slices; ++j)
+          for (int h = 0; h * box_rows < BN; ++h)
+            tma_load_2d(lora_b + j * BN * 32 + h * box_rows * 32, &pr.map_lo_b, lora_full, j * 16,
+                        t0 + h * box_rows);
+        last_l = lu;
       }
     }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ UMMA issuer
+  } else if (warp == kWarpProdC) {
+    // -------------------------------------------------- raw code tiles
     if (lane == 0) {
+      int g = 0;
       bool ok = true;
-      for (int kb = 0; kb < nk && ok; ++kb) {
-        const int s = kb % S, ph = (kb / S) & 1;
-        ok = mbar_wait(&full[s], ph, abort_flag, &g_gemm_flags, kFlagMma) &&
-             mbar_wait(&deq[s], ph, abort_flag, &g_gemm_flags, kFlagMma);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t a_base = smem_u32(a_tile(s));
-        const uint32_t b_base = smem_u32(act_tile(s));
-#pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16) {
-          // fwd A: 128 rows x 128 B lines (K-major, 8-row groups 1024 B apart);
-          //        a 16-wide K step is 32 B further along each line.
-          // dx  A: two 64-column atoms 8 KiB apart (LBO), 8-row groups 1 KiB
-          //        apart (SBO); a 16-row K step is 2 KiB further.
-          const uint64_t adesc =
-              (MODE == kGemmFwd)
-                  ? make_sdesc(a_base + k16 * 32, 16, 1024, kLayoutSw128)
-                  : make_sdesc(a_base + k16 * 2048, 64 * 128, 1024, kLayoutSw128);
-          const uint64_t bdesc = make_sdesc(b_base + k16 * 32, 16, 1024, kLayoutSw128);
-          umma_bf16(tmem, adesc, bdesc, idesc, (kb > 0 || k16 > 0) ? 1u : 0u);
+      for (int ui = u_begin; ui < u_end && ok; ++ui) {
+        const Unit U = unpack_unit(P, P.units[ui]);
+        const GemmProblem& pr = P.prob[U.p];
+        const int m0 = U.mt * kTileM;
+        for (int kb = U.kb0; kb < U.kb1; ++kb, ++g) {
+          const int s = g % SC;
+          if (g >= SC && !mbar_wait(&c_empty[s], ((g / SC) - 1) & 1, abort_flag, &g_gemm_flags,
+                                    kFlagProducer)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&c_full[s], static_cast<uint32_t>(kCodeBytes));
+          if (MODE == kGemmFwd)
+            tma_load_2d(c_tile(s), &pr.map_codes, &c_full[s], kb * 32, m0);
+          else
+            tma_load_2d(c_tile(s), &pr.map_codes, &c_full[s], m0 / 2, kb * kStepK);
+          last_c = g;
         }
-        mma_started = true;
-        umma_commit(&empty[s]);
       }
-      if (ok && mbar_wait(lora_bar, 0, abort_flag, &g_gemm_flags, kFlagLora)) {
-        tc_fence_after();
-        const uint32_t la = smem_u32(lora_a), lb = smem_u32(lora_b);
-        for (int j = 0; j < slices; ++j) {
-          const uint64_t adesc =
-              (MODE == kGemmFwd)
-                  ? make_sdesc(la + j * 4096, 16, 256, kLayoutSw32)
-                  : make_sdesc(la + j * 2048, p.r_pad * 128, 1024, kLayoutSw128);
-          const uint64_t bdesc = make_sdesc(lb + j * BN * 32, 16, 256, kLayoutSw32);
-          umma_bf16(tmem, adesc, bdesc, idesc, 1u);
+    }
+  } else if (warp == kWarpMma) {
+    // -------------------------------------------------- UMMA issuer
+    if (lane == 0) {
+      int g = 0, lu = 0;
+      bool ok = true;
+      for (int ui = u_begin; ui < u_end && ok; ++ui, ++lu) {
+        const Unit U = unpack_unit(P, P.units[ui]);
+        if (lu > 0) {
+          ok = mbar_wait(acc_empty, (lu - 1) & 1, abort_flag, &g_gemm_flags, kFlagMma);
+          if (!ok) break;
+          tc_fence_after();
         }
-        mma_started = true;
-        umma_commit(acc_bar);
+        for (int kb = U.kb0; kb < U.kb1; ++kb, ++g) {
+          const int sx = g % SX, sa = g % SA;
+          ok = mbar_wait(&x_full[sx], (g / SX) & 1, abort_flag, &g_gemm_flags, kFlagMma) &&
+               mbar_wait(&a_full[sa], (g / SA) & 1, abort_flag, &g_gemm_flags, kFlagMma);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(a_tile(sa));
+          const uint32_t b_base = smem_u32(x_tile(sx));
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16) {
+            // fwd A: 128 rows x 128 B lines (K-major, 8-row groups 1 KiB apart);
+            //        a 16-wide K step is 32 B further along each line.
+            // dx  A: two 64-column atoms 8 KiB apart (LBO), 8-row groups 1 KiB
+            //        apart (SBO); a 16-row K step is 2 KiB further.
+            const uint64_t adesc =
+                (MODE == kGemmFwd)
+                    ? make_sdesc(a_base + k16 * 32, 16, 1024, kLayoutSw128)
+                    : make_sdesc(a_base + k16 * 2048, 64 * 128, 1024, kLayoutSw128);
+            for (int h = 0; h < P.n_acc; ++h) {
+              const int n = (BN - h * 256) < 256 ? (BN - h * 256) : 256;
+              const uint64_t bdesc =
+                  make_sdesc(b_base + h * 256 * 128 + k16 * 32, 16, 1024, kLayoutSw128);
+              umma_bf16(tmem + h * 256, adesc, bdesc,
+                        make_idesc_bf16(kTileM, n, MODE == kGemmDx ? 1 : 0, 0),
+                        (kb > U.kb0 || k16 > 0) ? 1u : 0u);
+            }
+          }
+          mma_started = true;
+          umma_commit(&x_empty[sx]);
+          umma_commit(&a_empty[sa]);
+        }
+        if (!ok) break;
+        ok = mbar_wait(lora_full, lu & 1, abort_flag, &g_gemm_flags, kFlagLora);
+        if (!ok) break;
+        if (U.split == 0) {  // the rank-r slice is added once, by split 0
+          tc_fence_after();
+          const uint32_t la = smem_u32(lora_a), lb = smem_u32(lora_b);
+          for (int j = 0; j < slices; ++j) {
+            const uint64_t adesc =
+                (MODE == kGemmFwd) ? make_sdesc(la + j * 4096, 16, 256, kLayoutSw32)
+                                   : make_sdesc(la + j * 2048, P.r_pad * 128, 1024, kLayoutSw128);
+            for (int h = 0; h < P.n_acc; ++h) {
+              const int n = (BN - h * 256) < 256 ? (BN - h * 256) : 256;
+              const uint64_t bdesc =
+                  make_sdesc(lb + j * BN * 32 + h * 256 * 32, 16, 256, kLayoutSw32);
+              umma_bf16(tmem + h * 256, adesc, bdesc,
+                        make_idesc_bf16(kTileM, n, MODE == kGemmDx ? 1 : 0, 0), 1u);
+            }
+          }
+          mma_started = true;
+        }
+        umma_commit(lora_empty);
+        umma_commit(acc_full);
+      }
+    }
+  } else if (warp < kWarpEpi) {
+    // -------------------------------------------------- dequant (two warpgroups)
+    const int grp = warp >> 2;        // 0 or 1: takes the K steps with g % 2 == grp
+    const int i = threadIdx.x & 127;  // this thread's line of the A tile
+    const int line = (MODE == kGemmFwd) ? i : ((i >> 6) * 64 + (i & 63));
+    const int code_off = (MODE == kGemmFwd) ? i * 32 : (i & 63) * 64 + (i >> 6) * 32;
+    int g = 0;
+    bool ok = true;
+    for (int ui = u_begin; ui < u_end && ok; ++ui) {
+      const Unit U = unpack_unit(P, P.units[ui]);
+      const GemmProblem& pr = P.prob[U.p];
+      const int m0 = U.mt * kTileM;
+      for (int kb = U.kb0; kb < U.kb1; ++kb, ++g) {
+        if ((g & 1) != grp) continue;
+        const int sc = g % SC, sa = g % SA;
+        float a;
+        if (MODE == kGemmFwd) {
+          const int row = m0 + i;
+          a = (row < pr.n_out)
+                  ? __ldg(pr.absmax + static_cast<int64_t>(row) * pr.kblocks + kb)
+                  : 0.0f;
+        } else {
+          const int row = kb * kStepK + (i & 63);
+          const int kblk = m0 / 64 + (i >> 6);
+          a = (kblk < pr.kblocks)
+                  ? __ldg(pr.absmax + static_cast<int64_t>(row) * pr.kblocks + kblk)
+                  : 0.0f;
+        }
+        if (!mbar_wait(&c_full[sc], (g / SC) & 1, abort_flag, &g_gemm_flags, kFlagDequant)) {
+          ok = false;
+          break;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(c_tile(sc) + code_off);
+        const uint4 c0 = src[0], c1 = src[1];
+        mbar_arrive(&c_empty[sc]);
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const Nf4Table tab = nf4_make_table(P.cb, a);
+        if (g >= SA && !mbar_wait(&a_empty[sa], ((g / SA) - 1) & 1, abort_flag, &g_gemm_flags,
+                                  kFlagDequant)) {
+          ok = false;
+          break;
+        }
+        uint8_t* dst = a_tile(sa) + line * 128;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          const uint4 v = nf4_dequant8(words[w], tab);
+          *reinterpret_cast<uint4*>(dst + ((w ^ (line & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&a_full[sa]);
       }
     }
   } else {
-    // ------------------------------------------------------------ dequant
-    const int i = threadIdx.x;  // 0..127
-    const int line = (MODE == kGemmFwd) ? i : ((i >> 6) * 64 + (i & 63));
-    const int code_off = (MODE == kGemmFwd) ? i * 32 : (i & 63) * 64 + (i >> 6) * 32;
-    bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % S, ph = (kb / S) & 1;
-      float a;
-      if (MODE == kGemmFwd) {
-        const int row = m0 + i;
-        a = (row < p.n_out) ? __ldg(p.absmax + static_cast<int64_t>(row) * kblocks + kb) : 0.0f;
-      } else {
-        const int row = kb * kStepK + (i & 63);
-        const int kblk = m0 / 64 + (i >> 6);
-        a = (kblk < kblocks) ? __ldg(p.absmax + static_cast<int64_t>(row) * kblocks + kblk)
-                             : 0.0f;
-      }
-      if (!mbar_wait(&full[s], ph, abort_flag, &g_gemm_flags, kFlagDequant)) {
-        ok = false;
-        break;
-      }
-      const uint4* src = reinterpret_cast<const uint4*>(code_tile(s) + code_off);
-      const uint4 c0 = src[0], c1 = src[1];
-      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-      const Nf4Table tab = nf4_make_table(p.cb, a);
-      uint8_t* dst = a_tile(s) + line * 128;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        const uint4 v = nf4_dequant8(words[w], tab);
-        *reinterpret_cast<uint4*>(dst + ((w ^ (line & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&deq[s]);
-    }
-    // ------------------------------------------------------------ epilogue
-    // tcgen05.ld is warp-collective: decide per warp, never per lane.
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_bar, 0, abort_flag, &g_gemm_flags,
-                                                   kFlagEpilogue));
-    if (ok) {
+    // -------------------------------------------------- epilogue (warps 8..11)
+    const int q = warp - kWarpEpi;              // TMEM lane quarter
+    const int i = threadIdx.x - kWarpEpi * 32;  // 0..127: TMEM lane = tile row
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    int lu = 0;
+    for (int ui = u_begin; ui < u_end; ++ui, ++lu) {
+      const Unit U = unpack_unit(P, P.units[ui]);
+      const GemmProblem& pr = P.prob[U.p];
+      const int m0 = U.mt * kTileM, t0 = U.tt * BN;
+      const int M = pr.m_total;
+      bool ok = mbar_wait(acc_full, lu & 1, abort_flag, &g_gemm_flags, kFlagEpilogue);
+      ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld is warp-collective
+      if (!ok) break;
       tc_fence_after();
-      const int M = (MODE == kGemmFwd) ? p.n_out : p.k_in;
-      const int row = m0 + warp * 32 + lane;
-      for (int c = 0; c < BN; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c), v);
-        tmem_wait_ld();
-        if (row < M) {
+      const int tile = U.tt * pr.m_tiles + U.mt;
+      const bool split = pr.splits > 1;
+      float* tile_part = split ? pr.partial + static_cast<int64_t>(tile) * pr.splits * kTileM * BN
+                               : nullptr;
+      bool reduce = !split;
+      if (split) {
+        // this split's fp32 tile -> workspace, row i = TMEM lane
+        float* mine = tile_part + static_cast<int64_t>(U.split) * kTileM * BN +
+                      static_cast<int64_t>(i) * BN;
+        for (int c = 0; c < BN; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c), v);
+          tmem_wait_ld();
+          float4* dst = reinterpret_cast<float4*>(mine + c);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            __stcg(dst + j, make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                        __uint_as_float(v[4 * j + 2]),
+                                        __uint_as_float(v[4 * j + 3])));
+        }
+        // the accumulator is free for the next unit now
+        tc_fence_before();
+        mbar_arrive(acc_empty);
+        __threadfence();
+        named_sync(1, 128);
+        if (i == 0) {
+          const unsigned int old = atomicAdd(pr.counter + tile, 1u);
+          const int last = (old == static_cast<unsigned int>(pr.splits - 1)) ? 1 : 0;
+          if (last) pr.counter[tile] = 0u;  // leave the counter ready for reuse
+          *last_flag = last;
+        }
+        named_sync(1, 128);
+        reduce = *last_flag != 0;
+        if (reduce) __threadfence();
+      }
+      if (reduce) {
+        for (int c = 0; c < BN; c += 16) {
+          float f[16];
+          if (split) {
+            // add the splits' tiles in split order 0, 1, ..., S-1
+            const float* base = tile_part + static_cast<int64_t>(i) * BN + c;
+            for (int s = 0; s < pr.splits; ++s) {
+              const float4* src =
+                  reinterpret_cast<const float4*>(base + static_cast<int64_t>(s) * kTileM * BN);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float4 x = __ldcg(src + j);
+                if (s == 0) {
+                  f[4 * j] = x.x, f[4 * j + 1] = x.y, f[4 * j + 2] = x.z, f[4 * j + 3] = x.w;
+                } else {
+                  f[4 * j] += x.x, f[4 * j + 1] += x.y, f[4 * j + 2] += x.z, f[4 * j + 3] += x.w;
+                }
+              }
+            }
+          } else {
+            uint32_t v[16];
+            tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(v[j]);
+          }
+          // transpose through smem: sb[token j][row i], double-buffered
+          uint16_t* sb = stage + ((c >> 4) & 1) * kStageElems;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int t = t0 + c + j;
-            if (t < p.T) {
-              const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[j]));
-              p.out[static_cast<int64_t>(t) * M + row] = *reinterpret_cast<const uint16_t*>(&b);
+            const __nv_bfloat16 b = __float2bfloat16_rn(f[j]);
+            sb[j * kTileM + i] = *reinterpret_cast<const uint16_t*>(&b);
+          }
+          named_sync(1, 128);
+          // 16 token rows x 256 B of output: 256 chunks of 16 B, two per thread
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int chunk = i + h * 128;
+            const int j = chunk >> 4, col = (chunk & 15) * 8;
+            const int t = t0 + c + j, row = m0 + col;
+            if (t < P.T && row < M) {
+              const uint4 val = *reinterpret_cast<const uint4*>(sb + j * kTileM + col);
+              *reinterpret_cast<uint4*>(pr.out + static_cast<int64_t>(t) * M + row) = val;
             }
           }
         }
       }
+      if (!split) {
+        tc_fence_before();
+        mbar_arrive(acc_empty);
+      }
     }
   }
 
-  // ------------------------------------------------------------ teardown
+  // -------------------------------------------------- teardown
   __syncthreads();
   if (*abort_flag) {
-    // Drain what this CTA started before its shared memory and TMEM go away.
-    if (warp == 4 && lane == 0) {
-      for (int s = 0; s < S && s < 8; ++s)
-        if (issued_phase[s] >= 0) {
-          volatile int never = 0;
-          if (!mbar_wait(&full[s], static_cast<uint32_t>(issued_phase[s]), &never,
-                         &g_gemm_flags, kFlagDrain))
-            break;
-        }
+    // drain what this CTA started before its shared memory and TMEM go away
+    volatile int never = 0;
+    if (warp == kWarpProdX && lane == 0) {
+      for (int g = (last_x - SX + 1 > 0 ? last_x - SX + 1 : 0); g <= last_x; ++g)
+        if (!mbar_wait(&x_full[g % SX], (g / SX) & 1, &never, &g_gemm_flags, kFlagDrain)) break;
+      if (last_l >= 0) mbar_wait(lora_full, last_l & 1, &never, &g_gemm_flags, kFlagDrain);
     }
-    if (warp == 5 && lane == 0 && mma_started) {
+    if (warp == kWarpProdC && lane == 0) {
+      for (int g = (last_c - SC + 1 > 0 ? last_c - SC + 1 : 0); g <= last_c; ++g)
+        if (!mbar_wait(&c_full[g % SC], (g / SC) & 1, &never, &g_gemm_flags, kFlagDrain)) break;
+    }
+    if (warp == kWarpMma && lane == 0 && mma_started) {
       umma_commit(drain_bar);
-      volatile int never = 0;
       mbar_wait(drain_bar, 0, &never, &g_gemm_flags, kFlagDrain);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tc_fence_after();
-    tmem_dealloc(tmem, static_cast<uint32_t>(p.tmem_cols));
+    tmem_dealloc(tmem, static_cast<uint32_t>(P.tmem_cols));
   }
 }
 
@@ -361,64 +584,231 @@ static int configure_once() {
   return rc;
 }
 
-int launch_lora_gemm(GemmMode mode, const hsnf4_nf4_weight* W, const void* act, int64_t T,
-                     const void* lo_a, int r, int r_pad, const void* lo_b, void* out,
-                     cudaStream_t st) {
-  const int64_t n_out = W->n_out, k_in = W->k_in;
-  GemmParams p;
-  memset(&p, 0, sizeof p);
-  const int64_t bn16 = (T + 15) / 16 * 16;
-  p.BN = static_cast<int>(bn16 < 256 ? bn16 : 256);
-  p.T = static_cast<int>(T);
-  p.n_out = static_cast<int>(n_out);
-  p.k_in = static_cast<int>(k_in);
-  p.r_pad = r_pad;
-  p.absmax = W->absmax;
-  p.out = static_cast<uint16_t*>(out);
-  p.cb = codebook();
-  int tc = 32;
-  while (tc < p.BN) tc <<= 1;
-  p.tmem_cols = tc;
-  int stages = 4;
-  while (stages > 2 && smem_plan(mode, p.BN, stages, r_pad).total + 1024 > kMaxSmem) --stages;
-  p.stages = stages;
-  const int smem = smem_plan(mode, p.BN, stages, r_pad).total + 1024;
-  if (smem > kMaxSmem) return fail(HSNF4_ERR_INVALID, "lora gemm: shared memory plan %d B too large", smem);
+static int sm_count() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
 
-  const int64_t contraction = (mode == kGemmFwd) ? k_in : n_out;
-  bool ok = encode_2d(&p.map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, contraction, T,
-                      contraction * 2, 64, p.BN, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (mode == kGemmFwd) {
-    ok = ok && encode_2d(&p.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, k_in / 2, n_out,
-                         k_in / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
-    ok = ok && encode_2d(&p.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lo_a, r, n_out, r * 2, 16,
-                         128, CU_TENSOR_MAP_SWIZZLE_32B);
-  } else {
-    ok = ok && encode_2d(&p.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, k_in / 2, n_out,
-                         k_in / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
-    ok = ok && encode_2d(&p.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lo_a, k_in, r, k_in * 2,
-                         64, r_pad, CU_TENSOR_MAP_SWIZZLE_128B);
+struct Tiling {
+  int BN, sx, sc, sa;
+};
+
+// Token tile (<= 256 and a multiple of 16, or 512) and ring depths that fit
+// in shared memory.
+static bool choose_tiling(GemmMode mode, int64_t T, int r_pad, Tiling* t) {
+  const int64_t t16 = (T + 15) / 16 * 16;
+  const int first = t16 > 256 ? 512 : static_cast<int>(t16);
+  for (int bn : {first, 256}) {
+    if (bn > first) continue;
+    for (int x : {4, 3, 2}) {
+      if (smem_plan(mode, bn, x, 4, 3, r_pad).total + 1024 <= kMaxSmem) {
+        *t = {bn, x, 4, 3};
+        return true;
+      }
+    }
   }
-  ok = ok && encode_2d(&p.map_lo_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lo_b, r_pad, T, r_pad * 2,
-                       16, p.BN, CU_TENSOR_MAP_SWIZZLE_32B);
+  return false;
+}
+
+// K splits per problem: problems whose units are few and long are split so
+// that no unit is much longer than the group's balanced per-SM load, while
+// every piece keeps at least 16 K steps.
+static void plan_splits(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int BN,
+                        int sms, std::vector<int>* splits) {
+  splits->assign(n, 1);
+  double total = 0;
+  std::vector<int64_t> nk(n);
+  for (int p = 0; p < n; ++p) {
+    const int64_t mdim = (mode == kGemmFwd) ? probs[p].n_out : probs[p].k_in;
+    const int64_t contraction = (mode == kGemmFwd) ? probs[p].k_in : probs[p].n_out;
+    const int64_t tiles = ((mdim + kTileM - 1) / kTileM) * ((T + BN - 1) / BN);
+    nk[p] = contraction / kStepK;
+    total += static_cast<double>(tiles) * nk[p];
+  }
+  const double avg = total / sms;
+  for (int p = 0; p < n; ++p) {
+    int s = 1;
+    while (s < 16 && nk[p] / (s + 1) >= 16 && static_cast<double>(nk[p]) / s > 1.15 * avg) ++s;
+    (*splits)[p] = s;
+  }
+}
+
+struct SplitLayout {
+  std::vector<int> splits;
+  std::vector<size_t> part_base, cnt_base;
+  size_t cnt_off = 0, cnt_bytes = 0, need = 0;
+};
+
+static void split_layout(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int BN,
+                         SplitLayout* L) {
+  plan_splits(mode, probs, n, T, BN, sm_count(), &L->splits);
+  L->part_base.assign(n, 0);
+  L->cnt_base.assign(n, 0);
+  size_t part = 0, cnt = 0;
+  const int64_t t_tiles = (T + BN - 1) / BN;
+  for (int p = 0; p < n; ++p) {
+    if (L->splits[p] <= 1) continue;
+    const int64_t mdim = (mode == kGemmFwd) ? probs[p].n_out : probs[p].k_in;
+    const int64_t tiles = ((mdim + kTileM - 1) / kTileM) * t_tiles;
+    L->part_base[p] = part;
+    part += static_cast<size_t>(tiles) * L->splits[p] * kTileM * BN * 4;
+    L->cnt_base[p] = cnt;
+    cnt += static_cast<size_t>(tiles) * 4;
+  }
+  L->cnt_off = round_up(part, 256);
+  L->cnt_bytes = cnt;
+  L->need = part ? L->cnt_off + round_up(cnt, 256) : 0;
+}
+
+size_t gemm_workspace_bytes(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r) {
+  Tiling tl;
+  if (!choose_tiling(mode, T, (r + 15) / 16 * 16, &tl)) return 0;
+  SplitLayout L;
+  split_layout(mode, probs, n, T, tl.BN, &L);
+  return L.need;
+}
+
+int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r,
+                           void* workspace, size_t ws_bytes, cudaStream_t st) {
+  if (n < 1 || n > kMaxProblems)
+    return fail(HSNF4_ERR_INVALID, "lora gemm: 1..%d problems per launch (got %d)", kMaxProblems,
+                n);
+  static GemmParams P;  // large: built on the host, copied into the launch
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  memset(&P, 0, offsetof(GemmParams, units));
+  const int r_pad = (r + 15) / 16 * 16;
+  Tiling tl;
+  if (!choose_tiling(mode, T, r_pad, &tl))
+    return fail(HSNF4_ERR_INVALID, "lora gemm: no tiling fits shared memory (T=%lld, r=%d)",
+                (long long)T, r);
+  const int BN = tl.BN;
+  const int t_tiles = static_cast<int>((T + BN - 1) / BN);
+  if (t_tiles > 64)
+    return fail(HSNF4_ERR_INVALID, "lora gemm: T=%lld exceeds %d tokens per launch",
+                (long long)T, 64 * BN);
+  P.T = static_cast<int>(T);
+  P.BN = BN;
+  P.r_pad = r_pad;
+  P.n_acc = (BN + 255) / 256;
+  P.sx = tl.sx;
+  P.sc = tl.sc;
+  P.sa = tl.sa;
+  P.cb = codebook();
+  int tc = 32;
+  while (tc < BN) tc <<= 1;
+  P.tmem_cols = tc;
+  const int sms = sm_count();
+  SplitLayout L;
+  split_layout(mode, probs, n, T, BN, &L);
+  if (L.need > ws_bytes || (L.need && !workspace))
+    return fail(HSNF4_ERR_OOM, "lora gemm: workspace too small: need %zu bytes, given %zu",
+                L.need, ws_bytes);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  // units, longest first, each to the least loaded CTA so far
+  struct U {
+    int64_t cost;
+    uint32_t code;
+  };
+  std::vector<U> units;
+  for (int p = 0; p < n; ++p) {
+    const GemmProblemDesc& d = probs[p];
+    const int64_t mdim = (mode == kGemmFwd) ? d.n_out : d.k_in;
+    const int64_t nk = ((mode == kGemmFwd) ? d.k_in : d.n_out) / kStepK;
+    const int mt_n = static_cast<int>((mdim + kTileM - 1) / kTileM);
+    if (mt_n > (1 << 18))
+      return fail(HSNF4_ERR_INVALID, "lora gemm: %lld rows exceed the tile index range",
+                  (long long)mdim);
+    const int S = L.splits[p];
+    for (int s = 0; s < S; ++s) {
+      const int64_t cost = (s + 1) * nk / S - s * nk / S;
+      for (int tt = 0; tt < t_tiles; ++tt)
+        for (int mt = 0; mt < mt_n; ++mt) units.push_back({cost + 8, pack_unit(p, s, tt, mt)});
+    }
+  }
+  if (units.size() > static_cast<size_t>(kMaxUnits))
+    return fail(HSNF4_ERR_INVALID, "lora gemm: %zu work units exceed the per-launch limit %d",
+                units.size(), kMaxUnits);
+  std::stable_sort(units.begin(), units.end(),
+                   [](const U& a, const U& b) { return a.cost > b.cost; });
+  const int G = static_cast<int>(std::min<size_t>(units.size(), std::min(sms, kMaxCtas)));
+  std::vector<std::vector<uint32_t>> per(G);
+  using Load = std::pair<int64_t, int>;
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int c = 0; c < G; ++c) heap.push({0, c});
+  for (const U& u : units) {
+    Load top = heap.top();
+    heap.pop();
+    per[top.second].push_back(u.code);
+    heap.push({top.first + u.cost, top.second});
+  }
+  int k = 0;
+  for (int c = 0; c < G; ++c) {
+    P.cta_off[c] = static_cast<uint16_t>(k);
+    for (uint32_t code : per[c]) P.units[k++] = code;
+  }
+  P.cta_off[G] = static_cast<uint16_t>(k);
+
+  bool ok = true;
+  const int box_rows = BN < 256 ? BN : 256;
+  for (int p = 0; p < n; ++p) {
+    const GemmProblemDesc& d = probs[p];
+    GemmProblem& g = P.prob[p];
+    const int64_t contraction = (mode == kGemmFwd) ? d.k_in : d.n_out;
+    g.absmax = d.absmax;
+    g.out = static_cast<uint16_t*>(d.out);
+    g.n_out = static_cast<int>(d.n_out);
+    g.k_in = static_cast<int>(d.k_in);
+    g.m_total = static_cast<int>((mode == kGemmFwd) ? d.n_out : d.k_in);
+    g.nk = static_cast<int>(contraction / kStepK);
+    g.kblocks = static_cast<int>(d.k_in / 64);
+    g.m_tiles = (g.m_total + kTileM - 1) / kTileM;
+    g.splits = L.splits[p];
+    if (g.splits > 1) {
+      g.partial = reinterpret_cast<float*>(ws + L.part_base[p]);
+      g.counter = reinterpret_cast<unsigned int*>(ws + L.cnt_off + L.cnt_base[p]);
+    }
+    ok = ok && encode_2d(&g.map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.act, contraction, T,
+                         contraction * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (mode == kGemmFwd) {
+      ok = ok && encode_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
+                           d.n_out, d.k_in / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+      ok = ok && encode_2d(&g.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_a, r, d.n_out,
+                           r * 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
+    } else {
+      ok = ok && encode_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
+                           d.n_out, d.k_in / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+      ok = ok && encode_2d(&g.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_a, d.k_in, r,
+                           d.k_in * 2, 64, r_pad, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    ok = ok && encode_2d(&g.map_lo_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_b, r_pad, T,
+                         r_pad * 2, 16, box_rows, CU_TENSOR_MAP_SWIZZLE_32B);
+  }
   if (!ok) return fail(HSNF4_ERR_CUDA, "lora gemm: cuTensorMapEncodeTiled failed");
 
-  const int64_t mdim = (mode == kGemmFwd) ? n_out : k_in;
-  dim3 grid(static_cast<unsigned>((mdim + kTileM - 1) / kTileM),
-            static_cast<unsigned>((T + p.BN - 1) / p.BN));
-  cudaError_t e;
+  if (L.need) {
+    int rc = cuda_status(cudaMemsetAsync(ws + L.cnt_off, 0, L.cnt_bytes, st),
+                         "lora gemm: clear split counters");
+    if (rc) return rc;
+  }
   if (configure_once<kGemmFwd>() != 0 || configure_once<kGemmDx>() != 0)
     return fail(HSNF4_ERR_CUDA, "lora gemm: smem attribute");
+  const int smem = smem_plan(mode, BN, tl.sx, tl.sc, tl.sa, r_pad).total + 1024;
   void* prof = prof_begin(st);
   if (mode == kGemmFwd)
-    lora_gemm_kernel<kGemmFwd><<<grid, kThreads, smem, st>>>(p);
+    lora_gemm_kernel<kGemmFwd><<<G, kThreads, smem, st>>>(P);
   else
-    lora_gemm_kernel<kGemmDx><<<grid, kThreads, smem, st>>>(p);
-  e = cudaGetLastError();
+    lora_gemm_kernel<kGemmDx><<<G, kThreads, smem, st>>>(P);
+  const cudaError_t e = cudaGetLastError();
   if (prof) {
-    // algorithmic FLOPs: the base product plus the rank-r slice
-    const double flops = (mode == kGemmFwd) ? 2.0 * T * n_out * (k_in + r)
-                                            : 2.0 * T * k_in * (n_out + r);
+    // algorithmic FLOPs: the base products plus the rank-r slices
+    double flops = 0;
+    for (int p = 0; p < n; ++p)
+      flops += (mode == kGemmFwd) ? 2.0 * T * probs[p].n_out * (probs[p].k_in + r)
+                                  : 2.0 * T * probs[p].k_in * (probs[p].n_out + r);
     prof_end(prof, mode == kGemmFwd ? kProfGemmFwd : kProfGemmDx, flops, st);
   }
   return cuda_status(e, "lora gemm launch");

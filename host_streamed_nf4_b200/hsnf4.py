@@ -25,6 +25,17 @@ class Nf4WeightC(Structure):
     _fields_ = [("codes", c_void_p), ("absmax", c_void_p), ("n_out", c_int64), ("k_in", c_int64)]
 
 
+class FwdArgs(Structure):
+    _fields_ = [("W", Nf4WeightC), ("X", c_void_p), ("A", c_void_p), ("B", c_void_p),
+                ("Y", c_void_p), ("t_save", c_void_p)]
+
+
+class BwdArgs(Structure):
+    _fields_ = [("W", Nf4WeightC), ("X", c_void_p), ("t_save", c_void_p), ("A", c_void_p),
+                ("B", c_void_p), ("dY", c_void_p), ("dX", c_void_p), ("dA", c_void_p),
+                ("dB", c_void_p)]
+
+
 class LayerDesc(Structure):
     _fields_ = [("n_proj", c_int), ("n_out", c_int64 * MAX_PROJ), ("k_in", c_int64 * MAX_PROJ)]
 
@@ -71,6 +82,12 @@ _SIGS = {
     "lora_linear_bwd": ([POINTER(Nf4WeightC), c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_int,
                          c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                          c_void_p], c_int),
+    "lora_group_fwd_workspace": ([POINTER(FwdArgs), c_int, c_int64, c_int], c_size_t),
+    "lora_group_bwd_workspace": ([POINTER(BwdArgs), c_int, c_int64, c_int], c_size_t),
+    "lora_group_fwd": ([POINTER(FwdArgs), c_int, c_int64, c_int, c_float, c_void_p, c_size_t,
+                        c_void_p], c_int),
+    "lora_group_bwd": ([POINTER(BwdArgs), c_int, c_int64, c_int, c_float, c_void_p, c_size_t,
+                        c_void_p], c_int),
     "stream_layer_bytes": ([POINTER(LayerDesc), POINTER(c_size_t)], c_int),
     "stream_layer_offsets": ([POINTER(LayerDesc), c_int, POINTER(c_size_t), POINTER(c_size_t)], c_int),
     "stream_slab_bytes": ([POINTER(LayerDesc), c_int, POINTER(c_size_t)], c_int),
@@ -259,6 +276,46 @@ def lora_linear_bwd(W, X, t_save, A, B, dY, alpha: float, dX=None, dA=None, dB=N
                                  float(alpha), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB),
                                  _ptr(workspace), workspace.numel(), _stream(stream)))
     return dX, dA, dB
+
+
+def _wc(W):
+    return W.c() if isinstance(W, Nf4Weight) else W
+
+
+def _p(t):
+    return None if t is None else t.data_ptr()
+
+
+def fwd_args(W, X, A, B, Y, t_save=None) -> FwdArgs:
+    """One problem of a grouped forward (tensors are kept alive by the caller)."""
+    return FwdArgs(_wc(W), _p(X), _p(A), _p(B), _p(Y), _p(t_save))
+
+
+def bwd_args(W, X, t_save, A, B, dY, dX, dA, dB) -> BwdArgs:
+    return BwdArgs(_wc(W), _p(X), _p(t_save), _p(A), _p(B), _p(dY), _p(dX), _p(dA), _p(dB))
+
+
+def group_fwd_workspace_bytes(args, T, r) -> int:
+    arr = (FwdArgs * len(args))(*args)
+    return int(lib().lora_group_fwd_workspace(arr, len(args), T, r))
+
+
+def group_bwd_workspace_bytes(args, T, r) -> int:
+    arr = (BwdArgs * len(args))(*args)
+    return int(lib().lora_group_bwd_workspace(arr, len(args), T, r))
+
+
+def lora_group_fwd(args, T: int, r: int, alpha: float, workspace: torch.Tensor, stream=None):
+    """Forward of len(args) independent LoRA linears in one grouped call."""
+    arr = (FwdArgs * len(args))(*args)
+    _check(lib().lora_group_fwd(arr, len(args), T, r, float(alpha), _ptr(workspace),
+                                workspace.numel(), _stream(stream)))
+
+
+def lora_group_bwd(args, T: int, r: int, alpha: float, workspace: torch.Tensor, stream=None):
+    arr = (BwdArgs * len(args))(*args)
+    _check(lib().lora_group_bwd(arr, len(args), T, r, float(alpha), _ptr(workspace),
+                                workspace.numel(), _stream(stream)))
 
 
 # ------------------------------------------------------------------ streamer

@@ -29,6 +29,18 @@ from . import hsnf4, synth
 
 INPUT_OF = {"q": "h", "k": "h", "v": "h", "o": "o", "gate": "h", "up": "h", "down": "i"}
 
+# How a layer's 7 projections are batched into grouped launches.
+#   decoder: what a decoder layer's data dependencies allow -- q/k/v share
+#            their input, o needs attention, gate/up share their input, down
+#            needs the MLP activation (the backward runs the groups reversed);
+#   layer:   all 7 in one group (they are independent in this stack);
+#   none:    one launch sequence per projection.
+GROUPINGS = {
+    "decoder": [[0, 1, 2], [3], [4, 5], [6]],
+    "layer": [[0, 1, 2, 3, 4, 5, 6]],
+    "none": [[0], [1], [2], [3], [4], [5], [6]],
+}
+
 
 def _randn_bf16(shape, std, gen, device):
     return (torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * std).to(
@@ -43,7 +55,7 @@ class LayerStack:
     def __init__(self, family: synth.Family, n_layers: int, T: int, *, block_size: int = 4,
                  streamed: bool = True, reuse_resident: bool = True, enable_prefetch: bool = True,
                  poison_on_release: bool = False, r: int = synth.RANK, alpha: float = synth.ALPHA,
-                 seed: int = 42, device=None):
+                 seed: int = 42, device=None, grouping: str = "decoder"):
         self.device = torch.device(device) if device is not None else torch.device(
             "cuda", torch.cuda.current_device())
         dev = self.device
@@ -51,6 +63,7 @@ class LayerStack:
         self.block_size, self.streamed = block_size, streamed
         self.projs = family.projections()
         self.P = len(self.projs)
+        self.groups = GROUPINGS[grouping]
         self.desc = hsnf4.layer_desc([(n, k) for _, n, k in self.projs])
         self.descs = [self.desc] * n_layers
         self.layer_bytes = hsnf4.layer_bytes(self.desc)
@@ -92,8 +105,17 @@ class LayerStack:
                             for _, n, _ in self.projs])
         self.Y = [torch.empty(T, n, dtype=torch.bfloat16, device=dev) for _, n, _ in self.projs]
         self.dX = [torch.empty(T, k, dtype=torch.bfloat16, device=dev) for _, _, k in self.projs]
-        ws_f = max(hsnf4.fwd_workspace_bytes(T, n, k, r) for _, n, k in self.projs)
-        ws_b = max(hsnf4.bwd_workspace_bytes(T, n, k, r) for _, n, k in self.projs)
+        # workspaces: the largest any group needs (addresses do not matter here)
+        dummy = hsnf4.Nf4WeightC(0, 0, 0, 0)
+        ws_f = ws_b = 256
+        for grp in self.groups:
+            fa = [hsnf4.FwdArgs(hsnf4.Nf4WeightC(0, 0, self.projs[p][1], self.projs[p][2]), 0, 0, 0,
+                                0, 1) for p in grp]
+            ba = [hsnf4.BwdArgs(hsnf4.Nf4WeightC(0, 0, self.projs[p][1], self.projs[p][2]),
+                                0, 0, 0, 0, 0, 0, 0, 0) for p in grp]
+            ws_f = max(ws_f, hsnf4.group_fwd_workspace_bytes(fa, T, r))
+            ws_b = max(ws_b, hsnf4.group_bwd_workspace_bytes(ba, T, r))
+        del dummy
         self.ws_f = torch.empty(ws_f, dtype=torch.uint8, device=dev)
         self.ws_b = torch.empty(ws_b, dtype=torch.uint8, device=dev)
         self._prefetched = False
@@ -143,25 +165,30 @@ class LayerStack:
 
     def _fwd_block(self, ws, b, record):
         for i, l in enumerate(self.block_layers(b)):
-            for p, (name, _, _) in enumerate(self.projs):
-                hsnf4.lora_linear_fwd(ws[i * self.P + p], self.X[INPUT_OF[name]], self.A[l][p],
-                                      self.B[l][p], self.alpha, Y=self.Y[p], t_save=self.t[l][p],
-                                      workspace=self.ws_f, stream=self.compute)
+            for grp in self.groups:
+                args = [hsnf4.fwd_args(ws[i * self.P + p], self.X[INPUT_OF[self.projs[p][0]]],
+                                       self.A[l][p], self.B[l][p], self.Y[p], self.t[l][p])
+                        for p in grp]
+                hsnf4.lora_group_fwd(args, self.T, self.r, self.alpha, self.ws_f,
+                                     stream=self.compute)
                 if record is not None:
-                    record(l, p, "Y", self.Y[p])
+                    for p in grp:
+                        record(l, p, "Y", self.Y[p])
 
     def _bwd_block(self, ws, b, record):
         layers = list(self.block_layers(b))
         for i in reversed(range(len(layers))):
             l = layers[i]
-            for p in reversed(range(self.P)):
-                name = self.projs[p][0]
-                hsnf4.lora_linear_bwd(ws[i * self.P + p], self.X[INPUT_OF[name]], self.t[l][p],
-                                      self.A[l][p], self.B[l][p], self.dY[p], self.alpha,
-                                      dX=self.dX[p], dA=self.dA[l][p], dB=self.dB[l][p],
-                                      workspace=self.ws_b, stream=self.compute)
+            for grp in reversed(self.groups):
+                args = [hsnf4.bwd_args(ws[i * self.P + p], self.X[INPUT_OF[self.projs[p][0]]],
+                                       self.t[l][p], self.A[l][p], self.B[l][p], self.dY[p],
+                                       self.dX[p], self.dA[l][p], self.dB[l][p])
+                        for p in grp]
+                hsnf4.lora_group_bwd(args, self.T, self.r, self.alpha, self.ws_b,
+                                     stream=self.compute)
                 if record is not None:
-                    record(l, p, "dX", self.dX[p])
+                    for p in grp:
+                        record(l, p, "dX", self.dX[p])
 
     def forward(self, record=None):
         nb = self.n_blocks
@@ -225,8 +252,10 @@ class LayerStack:
             - self.block_bytes(0) - self.block_bytes(1)
 
     def kernels_per_step(self) -> int:
-        # forward: rank-r projection + fused GEMM; backward: projection, GEMM, dB, dA
-        return self.L * self.P * (2 + 4)
+        """Library kernels one step launches: per group, the forward runs the
+        rank-r projection (2 kernels) and the fused GEMM (1); the backward the
+        projection (2), the GEMM (1) and the adapter gradients (1)."""
+        return self.L * len(self.groups) * (3 + 4)
 
     def tokens_per_step(self) -> int:
         return self.T

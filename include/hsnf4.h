@@ -157,8 +157,9 @@ int nf4_dequant(const void *codes, const float *absmax, int64_t n_out,
 /* a ring slot or in a resident buffer -- the result is bitwise the same)  */
 /* ----------------------------------------------------------------------- */
 
-/* Limits: 8 <= r <= 64 and r % 8 == 0; T >= 1; n_out, k_in multiples of
- * 64.  alpha is any finite float; the scale is s = alpha / r (fp32). */
+/* Limits: 8 <= r <= 64 and r % 8 == 0; 1 <= T <= 32768; n_out, k_in
+ * multiples of 64.  alpha is any finite float; the scale is s = alpha / r
+ * (fp32).  Workspace needs depend on the shapes and the device's SM count. */
 
 /* Workspace bytes lora_linear_fwd needs for these sizes. */
 size_t lora_linear_fwd_workspace(int64_t T, int64_t n_out, int64_t k_in, int r);
@@ -193,6 +194,47 @@ int lora_linear_bwd(const hsnf4_nf4_weight *W, const void *X,
                     const void *B, int r, float alpha, const void *dY,
                     void *dX, float *dA, float *dB, void *workspace,
                     size_t ws_bytes, void *stream);
+
+/* Grouped forms: n (1..8) independent LoRA linears that share T, r and
+ * alpha, run as ONE rank-r projection pass, ONE persistent fused-GEMM
+ * launch whose CTAs take the group's tiles longest-first (with a K split,
+ * reduced in fixed order, for problems whose tiles are few and long), and
+ * in the backward ONE adapter-gradient launch.  A problem's K split (and so
+ * its fp32 summation order) depends on the whole group's shapes and the
+ * device's SM count, so its result can differ from the single-problem call
+ * in the last bits; it never depends on timing or on buffer addresses.  Per
+ * problem the arguments mean exactly what they mean for lora_linear_fwd /
+ * lora_linear_bwd. */
+typedef struct {
+  hsnf4_nf4_weight W;
+  const void *X;   /* bf16 [T, k_in] */
+  const void *A;   /* bf16 [r, k_in] */
+  const void *B;   /* bf16 [n_out, r] */
+  void *Y;         /* bf16 [T, n_out] */
+  float *t_save;   /* fp32 [T, r] or NULL */
+} hsnf4_lora_fwd_args;
+
+typedef struct {
+  hsnf4_nf4_weight W;
+  const void *X;        /* bf16 [T, k_in] */
+  const float *t_save;  /* fp32 [T, r] */
+  const void *A;        /* bf16 [r, k_in] */
+  const void *B;        /* bf16 [n_out, r] */
+  const void *dY;       /* bf16 [T, n_out] */
+  void *dX;             /* bf16 [T, k_in] */
+  float *dA;            /* fp32 [r, k_in] */
+  float *dB;            /* fp32 [n_out, r] */
+} hsnf4_lora_bwd_args;
+
+/* Workspace bytes of a grouped call (depends on the shapes and on the
+ * current device's SM count). */
+size_t lora_group_fwd_workspace(const hsnf4_lora_fwd_args *probs, int n, int64_t T, int r);
+size_t lora_group_bwd_workspace(const hsnf4_lora_bwd_args *probs, int n, int64_t T, int r);
+
+int lora_group_fwd(const hsnf4_lora_fwd_args *probs, int n, int64_t T, int r, float alpha,
+                   void *workspace, size_t ws_bytes, void *stream);
+int lora_group_bwd(const hsnf4_lora_bwd_args *probs, int n, int64_t T, int r, float alpha,
+                   void *workspace, size_t ws_bytes, void *stream);
 
 /* ----------------------------------------------------------------------- */
 /* Host-pinned NF4 base -> VRAM ring streamer                              */
