@@ -82,6 +82,8 @@ _SIGS = {
     "lora_linear_bwd": ([POINTER(Nf4WeightC), c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_int,
                          c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                          c_void_p], c_int),
+    "lora_linear_fwd_noalloc": ([POINTER(Nf4WeightC), c_void_p, c_int64, c_void_p, c_void_p, c_int,
+                                 c_float, c_void_p, c_void_p, c_void_p], c_int),
     "lora_group_fwd_workspace": ([POINTER(FwdArgs), c_int, c_int64, c_int], c_size_t),
     "lora_group_bwd_workspace": ([POINTER(BwdArgs), c_int, c_int64, c_int], c_size_t),
     "lora_group_fwd": ([POINTER(FwdArgs), c_int, c_int64, c_int, c_float, c_void_p, c_size_t,
@@ -254,6 +256,22 @@ def lora_linear_fwd(W, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha:
     _check(lib().lora_linear_fwd(_weight_arg(W), _ptr(X), T, _ptr(A), _ptr(B), r, float(alpha),
                                  _ptr(Y), _ptr(t_save), _ptr(workspace), workspace.numel(),
                                  _stream(stream)))
+    return Y, t_save
+
+
+def lora_linear_fwd_noalloc(W, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                            Y=None, t_save=None, stream=None):
+    """The forward without a workspace argument, for callers that cannot
+    allocate device memory: the library's built-in 64 MiB scratch is used.
+    (The output buffers passed here may be preallocated by the caller.)"""
+    n_out = W.n_out
+    T, r = X.shape[0], A.shape[0]
+    if Y is None:
+        Y = torch.empty(T, n_out, dtype=torch.bfloat16, device=X.device)
+    if t_save is None:
+        t_save = torch.empty(T, r, dtype=torch.float32, device=X.device)
+    _check(lib().lora_linear_fwd_noalloc(_weight_arg(W), _ptr(X), T, _ptr(A), _ptr(B), r,
+                                         float(alpha), _ptr(Y), _ptr(t_save), _stream(stream)))
     return Y, t_save
 
 

@@ -179,6 +179,28 @@ int lora_linear_fwd(const hsnf4_nf4_weight *W, const void *X, int64_t T,
                     float *t_save, void *workspace, size_t ws_bytes,
                     void *stream);
 
+/* The same forward for callers that cannot allocate device memory (a
+ * runtime that reserves its whole device-memory budget at start-up and
+ * forbids later allocations, a plugin or callback that may not call the
+ * allocator): no workspace argument; the scratch is a 64 MiB array compiled
+ * into the library, which every GPU that loads the library holds until the
+ * process exits.  This entry point has no counterpart in the paper; it is a
+ * convenience of this library.
+ *   - Sizes whose scratch need (lora_linear_fwd_workspace) exceeds 64 MiB
+ *     are rejected with HSNF4_ERR_INVALID before anything touches the GPU.
+ *   - It allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ *     library routine.  The first call on each device looks up the array's
+ *     device address (cudaGetSymbolAddress, with that device current) and
+ *     caches it; make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents
+ *     (what must start at zero is cleared by each call).  Calls whose GPU
+ *     work overlaps -- other streams, other host threads -- race on it;
+ *     serialize them.
+ * Arguments, results and errors are otherwise those of lora_linear_fwd. */
+int lora_linear_fwd_noalloc(const hsnf4_nf4_weight *W, const void *X, int64_t T,
+                            const void *A, const void *B, int r, float alpha, void *Y,
+                            float *t_save, void *stream);
+
 /* Workspace bytes lora_linear_bwd needs for these sizes. */
 size_t lora_linear_bwd_workspace(int64_t T, int64_t n_out, int64_t k_in, int r);
 
