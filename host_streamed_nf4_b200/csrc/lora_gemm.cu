@@ -276,6 +276,27 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
   } else if (warp == kWarpMma) {
     // -------------------------------------------------- UMMA issuer
     if (lane == 0) {
+      // All descriptors are computed once: per stage and per 16-wide K step
+      // only the start-address field changes (in 16-byte units; shared
+      // addresses stay below 256 KiB, so the 14-bit field never carries).
+      //   fwd A: 128 rows x 128 B lines (K-major, 8-row groups 1 KiB apart);
+      //          a 16-wide K step is 32 B further along each line.
+      //   dx  A: two 64-column atoms 8 KiB apart (LBO), 8-row groups 1 KiB
+      //          apart (SBO); a 16-row K step is 2 KiB further.
+      //   B (activations): K-major, 8-row groups 1 KiB apart; accumulator
+      //          h reads rows h*256.. (32 KiB further).
+      const uint64_t a_desc0 =
+          (MODE == kGemmFwd) ? make_sdesc(smem_u32(a_tile(0)), 16, 1024, kLayoutSw128)
+                             : make_sdesc(smem_u32(a_tile(0)), 64 * 128, 1024, kLayoutSw128);
+      const uint64_t b_desc0 = make_sdesc(smem_u32(x_tile(0)), 16, 1024, kLayoutSw128);
+      const uint32_t a_k16 = (MODE == kGemmFwd) ? (32 >> 4) : (2048 >> 4);
+      const uint32_t a_stage = kATileBytes >> 4, b_stage = plan.x_bytes >> 4;
+      const uint32_t b_half = (256 * 128) >> 4;
+      const int n0 = BN < 256 ? BN : 256;
+      const uint32_t idesc0 = make_idesc_bf16(kTileM, n0, MODE == kGemmDx ? 1 : 0, 0);
+      const uint32_t idesc1 =
+          make_idesc_bf16(kTileM, BN > 256 ? BN - 256 : 16, MODE == kGemmDx ? 1 : 0, 0);
+      const bool two = P.n_acc > 1;
       int g = 0, lu = 0;
       bool ok = true;
       for (int ui = u_begin; ui < u_end && ok; ++ui, ++lu) {
@@ -291,26 +312,14 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
                mbar_wait(&a_full[sa], (g / SA) & 1, abort_flag, &g_gemm_flags, kFlagMma);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t a_base = smem_u32(a_tile(sa));
-          const uint32_t b_base = smem_u32(x_tile(sx));
+          const uint64_t ad = a_desc0 + static_cast<uint64_t>(sa * a_stage);
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>(sx * b_stage);
+          const uint32_t first = (kb > U.kb0) ? 1u : 0u;
 #pragma unroll
           for (int k16 = 0; k16 < 4; ++k16) {
-            // fwd A: 128 rows x 128 B lines (K-major, 8-row groups 1 KiB apart);
-            //        a 16-wide K step is 32 B further along each line.
-            // dx  A: two 64-column atoms 8 KiB apart (LBO), 8-row groups 1 KiB
-            //        apart (SBO); a 16-row K step is 2 KiB further.
-            const uint64_t adesc =
-                (MODE == kGemmFwd)
-                    ? make_sdesc(a_base + k16 * 32, 16, 1024, kLayoutSw128)
-                    : make_sdesc(a_base + k16 * 2048, 64 * 128, 1024, kLayoutSw128);
-            for (int h = 0; h < P.n_acc; ++h) {
-              const int n = (BN - h * 256) < 256 ? (BN - h * 256) : 256;
-              const uint64_t bdesc =
-                  make_sdesc(b_base + h * 256 * 128 + k16 * 32, 16, 1024, kLayoutSw128);
-              umma_bf16(tmem + h * 256, adesc, bdesc,
-                        make_idesc_bf16(kTileM, n, MODE == kGemmDx ? 1 : 0, 0),
-                        (kb > U.kb0 || k16 > 0) ? 1u : 0u);
-            }
+            const uint32_t acc = (k16 > 0) ? 1u : first;
+            umma_bf16(tmem, ad + k16 * a_k16, bd + k16 * 2, idesc0, acc);
+            if (two) umma_bf16(tmem + 256, ad + k16 * a_k16, bd + b_half + k16 * 2, idesc1, acc);
           }
           mma_started = true;
           umma_commit(&x_empty[sx]);
@@ -326,13 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
             const uint64_t adesc =
                 (MODE == kGemmFwd) ? make_sdesc(la + j * 4096, 16, 256, kLayoutSw32)
                                    : make_sdesc(la + j * 2048, P.r_pad * 128, 1024, kLayoutSw128);
-            for (int h = 0; h < P.n_acc; ++h) {
-              const int n = (BN - h * 256) < 256 ? (BN - h * 256) : 256;
-              const uint64_t bdesc =
-                  make_sdesc(lb + j * BN * 32 + h * 256 * 32, 16, 256, kLayoutSw32);
-              umma_bf16(tmem + h * 256, adesc, bdesc,
-                        make_idesc_bf16(kTileM, n, MODE == kGemmDx ? 1 : 0, 0), 1u);
-            }
+            const uint64_t bdesc = make_sdesc(lb + j * BN * 32, 16, 256, kLayoutSw32);
+            umma_bf16(tmem, adesc, bdesc, idesc0, 1u);
+            if (two) umma_bf16(tmem + 256, adesc, bdesc + ((256 * 32) >> 4), idesc1, 1u);
           }
           mma_started = true;
         }
