@@ -52,14 +52,15 @@ WORKLOADS = {
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qwen2.5-7b-layer")
     ap.add_argument("--mode", choices=["streamed", "resident"], default=None)
     ap.add_argument("--block-size", type=int, default=None)
+    ap.add_argument("--slots", type=int, default=2, help="ring slots (2 = prefetch one ahead)")
     ap.add_argument("--seq", type=int, default=512)
-    ap.add_argument("--grouping", choices=["decoder", "layer", "none"], default="decoder",
+    ap.add_argument("--grouping", choices=["decoder", "layer", "none"], default="layer",
                     help="how a layer's projections are batched into grouped launches")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -99,73 +100,93 @@ def barrier(ws):
         dist.barrier()
 
 
-def max_over_ranks(ws, x: float) -> float:
-    if ws == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
 # ---------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons sampled every 10 ms during the timed
+    region (NVML; nvidia-smi as a fallback)."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(self.cuda_index)
+        bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+
+    def _run_nvml(self, nv, h):
+        self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+            mask = get_reasons(h)
+            for bit, name in self.REASONS.items():
+                if mask & bit:
+                    self.reasons.add(name)
+            self._stop.wait(0.01)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-i", str(self.index), "-lms", "200"], stdout=subprocess.PIPE,
-                stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except OSError:
-            self.proc = None
+            nv, h = self._nvml_handle()
+            self._thread = threading.Thread(target=self._run_nvml, args=(nv, h), daemon=True)
+            self._thread.start()
+        except Exception:
+            self._start_smi()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _start_smi(self):
+        q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self._proc = None
+            return
+
+        def read():
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for line in self._proc.stdout:
+                f = [x.strip() for x in line.split(",")]
+                try:
+                    self.samples.append(float(f[0]))
+                    self.max_mhz = float(f[1])
+                except (ValueError, IndexError):
+                    continue
+                for n, v in zip(names, f[2:6]):
+                    if v.lower() == "active":
+                        self.reasons.add(n)
+        self._thread = threading.Thread(target=read, daemon=True)
+        self._thread.start()
 
     def __exit__(self, *exc):
-        if self.proc:
-            self.proc.terminate()
+        self._stop.set()
+        if self._proc:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.t.join(timeout=2)
+                self._proc.kill()
+        if self._thread:
+            self._thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 # ---------------------------------------------------------------------- peaks
@@ -209,6 +230,7 @@ def run_ours(args, ws, rank, local):
     import numpy as np
     import torch
 
+    from host_streamed_nf4_b200 import dist as hdist
     from host_streamed_nf4_b200 import hsnf4, synth
     from host_streamed_nf4_b200.stack import LayerStack
 
@@ -222,7 +244,7 @@ def run_ours(args, ws, rank, local):
     # compute); a stack reuses the blocks still resident at each turn-around.
     stack = LayerStack(fam, args.layers, args.seq, block_size=args.block_size, streamed=streamed,
                        reuse_resident=not single, seed=42 + rank, device=dev,
-                       grouping=args.grouping)
+                       grouping=args.grouping, n_slots=args.slots)
     compute = stack.compute
 
     def one_step():
@@ -230,6 +252,8 @@ def run_ours(args, ws, rank, local):
             stack.step_single_block()
         else:
             stack.step()
+        # data parallel: the adapter gradients are summed over ranks each step
+        hdist.allreduce_grads(stack.grad_flat)
 
     def drain_copies():
         # make the compute stream wait for the copy stream, so that an
@@ -248,7 +272,7 @@ def run_ours(args, ws, rank, local):
     # ------------------------------------------------ device-timed region
     K = args.steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clocks:
+    with ClockSampler(local) as clocks:
         barrier(ws)
         torch.cuda.synchronize(dev)
         e0.record(compute)
@@ -258,10 +282,10 @@ def run_ours(args, ws, rank, local):
         e1.record(compute)
         torch.cuda.synchronize(dev)
         barrier(ws)
-    ms_total = max_over_ranks(ws, e0.elapsed_time(e1))
+    ms_total = hdist.max_over_ranks(e0.elapsed_time(e1))
     ms_step = ms_total / K
     tokens_per_step = stack.tokens_per_step()
-    value = ws * tokens_per_step * K / (ms_total / 1e3)
+    value = hdist.job_throughput(tokens_per_step, K, ms_total, ws)
     h2d_step = 0
     if streamed:
         st1 = stack.streamer.stats()
@@ -320,9 +344,10 @@ def run_ours(args, ws, rank, local):
         "config": {"workload": args.workload, "family": args.family, "layers": args.layers,
                    "tokens": args.seq, "batch": 1, "mode": args.mode,
                    "block_size": args.block_size, "rank": stack.r, "alpha": stack.alpha,
-                   "grouping": args.grouping,
+                   "grouping": args.grouping, "ring_slots": args.slots,
                    "projections": [p[0] for p in fam.projections()],
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "single",
+                   "parallelism": (f"dp{ws} (per-rank tokens, adapter-gradient all-reduce per "
+                                   f"step)" if ws > 1 else "single"),
                    "l2": "no flush: every step reads > 126 MB L2 (NF4 weights + activations)"},
         "roofline": roofline, "step_roofline": step_roofline, "e2e": e2e,
         "gpu_launches": K * stack.kernels_per_step(),
@@ -345,7 +370,7 @@ def run_e2e(args, stack, one_step, drain_copies, ws, dev):
         host_in[k].copy_(v)
     for h, v in zip(host_dy, stack.dY):
         h.copy_(v)
-    grads = [g for l in range(stack.L) for g in (stack.dA[l] + stack.dB[l])]
+    grads = [stack.grad_flat]  # every dA/dB of the stack, summed over ranks
     host_grads = [torch.empty_like(g, device="cpu").pin_memory() for g in grads]
     h2d = sum(t.numel() * t.element_size() for t in list(host_in.values()) + host_dy)
     d2h = sum(t.numel() * t.element_size() for t in host_grads)
@@ -374,8 +399,10 @@ def run_e2e(args, stack, one_step, drain_copies, ws, dev):
     e1.record(compute)
     torch.cuda.synchronize(dev)
     barrier(ws)
-    ms = max_over_ranks(ws, e0.elapsed_time(e1))
-    return {"value": round(ws * stack.tokens_per_step() * K / (ms / 1e3), 1), "unit": "tokens/s",
+    from host_streamed_nf4_b200 import dist as hdist
+    ms = hdist.max_over_ranks(e0.elapsed_time(e1))
+    return {"value": round(hdist.job_throughput(stack.tokens_per_step(), K, ms, ws), 1),
+            "unit": "tokens/s",
             "ms_per_step": round(ms / K, 4), "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h)}
 

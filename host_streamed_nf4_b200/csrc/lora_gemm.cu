@@ -39,7 +39,9 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <climits>
 #include <cstddef>
+#include <map>
 #include <mutex>
 #include <queue>
 #include <vector>
@@ -77,8 +79,7 @@ struct GemmProblem {
   CUtensorMap map_lo_b;   // s*t or s*u: bf16 [T, r_pad], box {16, min(BN,256)}, 32B swizzle
   const float* absmax;
   uint16_t* out;          // bf16 [T, m_total]
-  float* partial;         // split-K partial tiles (fp32 [128][BN] each), or null
-  unsigned int* counter;  // split-K arrival counters, one per (row tile, token tile)
+  float* partial;         // split-K partial tiles (fp32 [BN tokens][128 rows] each), or null
   int n_out, k_in, m_total, nk, kblocks, m_tiles, splits;
 };
 
@@ -166,7 +167,6 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
   uint64_t* drain_bar = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   auto x_tile = [&](int s) { return smem + s * plan.x_bytes; };
   auto a_tile = [&](int s) { return smem + plan.a_off + s * kATileBytes; };
   auto c_tile = [&](int s) { return smem + plan.c_off + s * kCodeBytes; };
@@ -413,91 +413,50 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       if (!ok) break;
       tc_fence_after();
       const int tile = U.tt * pr.m_tiles + U.mt;
-      const bool split = pr.splits > 1;
-      float* tile_part = split ? pr.partial + static_cast<int64_t>(tile) * pr.splits * kTileM * BN
-                               : nullptr;
-      bool reduce = !split;
-      if (split) {
-        // this split's fp32 tile -> workspace, row i = TMEM lane
-        float* mine = tile_part + static_cast<int64_t>(U.split) * kTileM * BN +
-                      static_cast<int64_t>(i) * BN;
+      if (pr.splits > 1) {
+        // this split's fp32 tile -> workspace, token-major ([BN][128]) so that a
+        // warp's 32 rows of one token are 128 contiguous bytes; the splits are
+        // added in split order by lora_splitk_reduce after this kernel
+        float* mine = pr.partial +
+                      (static_cast<int64_t>(tile) * pr.splits + U.split) * kTileM * BN + i;
         for (int c = 0; c < BN; c += 16) {
           uint32_t v[16];
           tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c), v);
           tmem_wait_ld();
-          float4* dst = reinterpret_cast<float4*>(mine + c);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            __stcg(dst + j, make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                        __uint_as_float(v[4 * j + 2]),
-                                        __uint_as_float(v[4 * j + 3])));
+          for (int j = 0; j < 16; ++j)
+            __stcg(mine + static_cast<int64_t>(c + j) * kTileM, __uint_as_float(v[j]));
         }
-        // the accumulator is free for the next unit now
         tc_fence_before();
         mbar_arrive(acc_empty);
-        __threadfence();
-        named_sync(1, 128);
-        if (i == 0) {
-          const unsigned int old = atomicAdd(pr.counter + tile, 1u);
-          const int last = (old == static_cast<unsigned int>(pr.splits - 1)) ? 1 : 0;
-          if (last) pr.counter[tile] = 0u;  // leave the counter ready for reuse
-          *last_flag = last;
+        continue;
+      }
+      for (int c = 0; c < BN; c += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c), v);
+        tmem_wait_ld();
+        // transpose through smem: sb[token j][row i], double-buffered
+        uint16_t* sb = stage + ((c >> 4) & 1) * kStageElems;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[j]));
+          sb[j * kTileM + i] = *reinterpret_cast<const uint16_t*>(&b);
         }
         named_sync(1, 128);
-        reduce = *last_flag != 0;
-        if (reduce) __threadfence();
-      }
-      if (reduce) {
-        for (int c = 0; c < BN; c += 16) {
-          float f[16];
-          if (split) {
-            // add the splits' tiles in split order 0, 1, ..., S-1
-            const float* base = tile_part + static_cast<int64_t>(i) * BN + c;
-            for (int s = 0; s < pr.splits; ++s) {
-              const float4* src =
-                  reinterpret_cast<const float4*>(base + static_cast<int64_t>(s) * kTileM * BN);
+        // 16 token rows x 256 B of output: 256 chunks of 16 B, two per thread
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float4 x = __ldcg(src + j);
-                if (s == 0) {
-                  f[4 * j] = x.x, f[4 * j + 1] = x.y, f[4 * j + 2] = x.z, f[4 * j + 3] = x.w;
-                } else {
-                  f[4 * j] += x.x, f[4 * j + 1] += x.y, f[4 * j + 2] += x.z, f[4 * j + 3] += x.w;
-                }
-              }
-            }
-          } else {
-            uint32_t v[16];
-            tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c), v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(v[j]);
-          }
-          // transpose through smem: sb[token j][row i], double-buffered
-          uint16_t* sb = stage + ((c >> 4) & 1) * kStageElems;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const __nv_bfloat16 b = __float2bfloat16_rn(f[j]);
-            sb[j * kTileM + i] = *reinterpret_cast<const uint16_t*>(&b);
-          }
-          named_sync(1, 128);
-          // 16 token rows x 256 B of output: 256 chunks of 16 B, two per thread
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int chunk = i + h * 128;
-            const int j = chunk >> 4, col = (chunk & 15) * 8;
-            const int t = t0 + c + j, row = m0 + col;
-            if (t < P.T && row < M) {
-              const uint4 val = *reinterpret_cast<const uint4*>(sb + j * kTileM + col);
-              *reinterpret_cast<uint4*>(pr.out + static_cast<int64_t>(t) * M + row) = val;
-            }
+        for (int h = 0; h < 2; ++h) {
+          const int chunk = i + h * 128;
+          const int j = chunk >> 4, col = (chunk & 15) * 8;
+          const int t = t0 + c + j, row = m0 + col;
+          if (t < P.T && row < M) {
+            const uint4 val = *reinterpret_cast<const uint4*>(sb + j * kTileM + col);
+            *reinterpret_cast<uint4*>(pr.out + static_cast<int64_t>(t) * M + row) = val;
           }
         }
       }
-      if (!split) {
-        tc_fence_before();
-        mbar_arrive(acc_empty);
-      }
+      tc_fence_before();
+      mbar_arrive(acc_empty);
     }
   }
 
@@ -544,6 +503,45 @@ __global__ void selftest_stall_kernel() {
 cudaError_t launch_selftest_stall(cudaStream_t st) {
   selftest_stall_kernel<<<1, 32, 0, st>>>();
   return cudaGetLastError();
+}
+
+// Adds the K-split partial tiles of every split problem in split order and
+// writes the bf16 outputs.  One CTA per (problem tile, 8-token slice);
+// thread i owns row pair (2i, 2i+1) of the tile.
+struct ReduceTile {
+  const float* part;  // [splits][BN][128] of this tile
+  uint16_t* out;      // output base
+  int m0, t0, M, splits;
+};
+
+constexpr int kReduceTok = 8;
+constexpr int kMaxReduceTiles = 768;  // 32 B each: the parameter block stays < 32 KiB
+
+struct ReduceParams {
+  ReduceTile tile[kMaxReduceTiles];
+  int n_tiles, BN, T;
+};
+
+__global__ void __launch_bounds__(64) lora_splitk_reduce(const __grid_constant__ ReduceParams R) {
+  const int slices = R.BN / kReduceTok;
+  const int tix = blockIdx.x / slices, slice = blockIdx.x % slices;
+  const ReduceTile& tl = R.tile[tix];
+  const int i = threadIdx.x * 2;  // rows i, i+1
+  const int row = tl.m0 + i;
+  for (int jj = 0; jj < kReduceTok; ++jj) {
+    const int c = slice * kReduceTok + jj;
+    const int t = tl.t0 + c;
+    if (t >= R.T || row >= tl.M) continue;
+    float2 acc = __ldcg(reinterpret_cast<const float2*>(tl.part + static_cast<int64_t>(c) * kTileM + i));
+    for (int s = 1; s < tl.splits; ++s) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(
+          tl.part + (static_cast<int64_t>(s) * R.BN + c) * kTileM + i));
+      acc.x += v.x;
+      acc.y += v.y;
+    }
+    const __nv_bfloat162 b = __floats2bfloat162_rn(acc.x, acc.y);
+    *reinterpret_cast<__nv_bfloat162*>(tl.out + static_cast<int64_t>(t) * tl.M + row) = b;
+  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -617,54 +615,128 @@ static bool choose_tiling(GemmMode mode, int64_t T, int r_pad, Tiling* t) {
   return false;
 }
 
-// K splits per problem: problems whose units are few and long are split so
-// that no unit is much longer than the group's balanced per-SM load, while
-// every piece keeps at least 16 K steps.
+// Cost model of a unit in K steps: its K steps plus a fixed overhead (the
+// epilogue and the pipeline refill), plus the fp32 partial-tile write when
+// the tile is split along K.
+constexpr int64_t kUnitOverhead = 8;
+constexpr int64_t kSplitOverhead = 4;
+
+static int64_t unit_cost(int64_t ksteps, int splits) {
+  return ksteps + kUnitOverhead + (splits > 1 ? kSplitOverhead : 0);
+}
+
+// Makespan of the longest-first assignment of these units to `sms` CTAs.
+static int64_t lpt_makespan(std::vector<int64_t>& costs, int sms) {
+  std::sort(costs.begin(), costs.end(), std::greater<int64_t>());
+  std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> heap;
+  const size_t G = std::min<size_t>(costs.size(), static_cast<size_t>(sms));
+  for (size_t c = 0; c < G; ++c) heap.push(0);
+  int64_t mk = 0;
+  for (int64_t c : costs) {
+    int64_t l = heap.top();
+    heap.pop();
+    l += c;
+    mk = std::max(mk, l);
+    heap.push(l);
+  }
+  return mk;
+}
+
+// K splits per problem.  Objective: the simulated makespan of the
+// longest-first schedule (in K steps) plus the split-K reduce pass, whose
+// partial reads are charged at ~16 KiB per K step per SM.  Search: starting
+// from no splits, repeatedly add one split to the problem holding the
+// longest unit (pieces of at least 16 K steps, at most 8 splits), keeping
+// the best objective seen.  Deterministic in the shapes and the SM count.
 static void plan_splits(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int BN,
                         int sms, std::vector<int>* splits) {
-  splits->assign(n, 1);
-  double total = 0;
-  std::vector<int64_t> nk(n);
+  std::vector<int64_t> tiles(n), nk(n);
   for (int p = 0; p < n; ++p) {
     const int64_t mdim = (mode == kGemmFwd) ? probs[p].n_out : probs[p].k_in;
     const int64_t contraction = (mode == kGemmFwd) ? probs[p].k_in : probs[p].n_out;
-    const int64_t tiles = ((mdim + kTileM - 1) / kTileM) * ((T + BN - 1) / BN);
+    tiles[p] = ((mdim + kTileM - 1) / kTileM) * ((T + BN - 1) / BN);
     nk[p] = contraction / kStepK;
-    total += static_cast<double>(tiles) * nk[p];
   }
-  const double avg = total / sms;
-  for (int p = 0; p < n; ++p) {
-    int s = 1;
-    while (s < 16 && nk[p] / (s + 1) >= 16 && static_cast<double>(nk[p]) / s > 1.15 * avg) ++s;
-    (*splits)[p] = s;
+  auto objective = [&](const std::vector<int>& sp) -> int64_t {
+    std::vector<int64_t> costs;
+    double reduce_bytes = 0;
+    for (int p = 0; p < n; ++p) {
+      for (int s = 0; s < sp[p]; ++s) {
+        const int64_t ks = (s + 1) * nk[p] / sp[p] - s * nk[p] / sp[p];
+        costs.insert(costs.end(), static_cast<size_t>(tiles[p]), unit_cost(ks, sp[p]));
+      }
+      if (sp[p] > 1) reduce_bytes += static_cast<double>(tiles[p]) * sp[p] * kTileM * BN * 4;
+    }
+    if (costs.size() > static_cast<size_t>(3072)) return INT64_MAX;  // over the unit limit
+    const int64_t reduce = reduce_bytes > 0
+                               ? 4 + static_cast<int64_t>(reduce_bytes / (16384.0 * sms))
+                               : 0;
+    return lpt_makespan(costs, sms) + reduce;
+  };
+  std::vector<int> cur(n, 1);
+  *splits = cur;
+  int64_t best = objective(cur);
+  for (int it = 0; it < 24; ++it) {
+    int worst = -1;
+    int64_t worst_cost = -1;
+    for (int p = 0; p < n; ++p) {
+      const int64_t c = unit_cost(nk[p] / cur[p] + (nk[p] % cur[p] ? 1 : 0), cur[p]);
+      if (c > worst_cost && cur[p] < 8 && nk[p] / (cur[p] + 1) >= 16) {
+        worst = p;
+        worst_cost = c;
+      }
+    }
+    if (worst < 0) break;
+    cur[worst] += 1;
+    const int64_t obj = objective(cur);
+    if (obj < best) {
+      best = obj;
+      *splits = cur;
+    }
   }
 }
 
 struct SplitLayout {
   std::vector<int> splits;
-  std::vector<size_t> part_base, cnt_base;
-  size_t cnt_off = 0, cnt_bytes = 0, need = 0;
+  std::vector<size_t> part_base;
+  size_t need = 0;
 };
+
+// plan_splits results, cached by (mode, T, BN, SM count, shapes)
+static std::vector<int> cached_splits(GemmMode mode, const GemmProblemDesc* probs, int n,
+                                      int64_t T, int BN) {
+  static std::mutex mu;
+  static std::map<std::vector<int64_t>, std::vector<int>> cache;
+  const int sms = sm_count();
+  std::vector<int64_t> key = {static_cast<int64_t>(mode), T, BN, sms};
+  for (int p = 0; p < n; ++p) {
+    key.push_back(probs[p].n_out);
+    key.push_back(probs[p].k_in);
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  std::vector<int> sp;
+  plan_splits(mode, probs, n, T, BN, sms, &sp);
+  if (cache.size() > 4096) cache.clear();
+  cache.emplace(key, sp);
+  return sp;
+}
 
 static void split_layout(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int BN,
                          SplitLayout* L) {
-  plan_splits(mode, probs, n, T, BN, sm_count(), &L->splits);
+  L->splits = cached_splits(mode, probs, n, T, BN);
   L->part_base.assign(n, 0);
-  L->cnt_base.assign(n, 0);
-  size_t part = 0, cnt = 0;
+  size_t part = 0;
   const int64_t t_tiles = (T + BN - 1) / BN;
   for (int p = 0; p < n; ++p) {
     if (L->splits[p] <= 1) continue;
     const int64_t mdim = (mode == kGemmFwd) ? probs[p].n_out : probs[p].k_in;
     const int64_t tiles = ((mdim + kTileM - 1) / kTileM) * t_tiles;
     L->part_base[p] = part;
-    part += static_cast<size_t>(tiles) * L->splits[p] * kTileM * BN * 4;
-    L->cnt_base[p] = cnt;
-    cnt += static_cast<size_t>(tiles) * 4;
+    part += round_up(static_cast<size_t>(tiles) * L->splits[p] * kTileM * BN * 4, 256);
   }
-  L->cnt_off = round_up(part, 256);
-  L->cnt_bytes = cnt;
-  L->need = part ? L->cnt_off + round_up(cnt, 256) : 0;
+  L->need = part;
 }
 
 size_t gemm_workspace_bytes(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r) {
@@ -729,9 +801,9 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
                   (long long)mdim);
     const int S = L.splits[p];
     for (int s = 0; s < S; ++s) {
-      const int64_t cost = (s + 1) * nk / S - s * nk / S;
+      const int64_t cost = unit_cost((s + 1) * nk / S - s * nk / S, S);
       for (int tt = 0; tt < t_tiles; ++tt)
-        for (int mt = 0; mt < mt_n; ++mt) units.push_back({cost + 8, pack_unit(p, s, tt, mt)});
+        for (int mt = 0; mt < mt_n; ++mt) units.push_back({cost, pack_unit(p, s, tt, mt)});
     }
   }
   if (units.size() > static_cast<size_t>(kMaxUnits))
@@ -772,10 +844,7 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     g.kblocks = static_cast<int>(d.k_in / 64);
     g.m_tiles = (g.m_total + kTileM - 1) / kTileM;
     g.splits = L.splits[p];
-    if (g.splits > 1) {
-      g.partial = reinterpret_cast<float*>(ws + L.part_base[p]);
-      g.counter = reinterpret_cast<unsigned int*>(ws + L.cnt_off + L.cnt_base[p]);
-    }
+    if (g.splits > 1) g.partial = reinterpret_cast<float*>(ws + L.part_base[p]);
     ok = ok && encode_2d(&g.map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.act, contraction, T,
                          contraction * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
     if (mode == kGemmFwd) {
@@ -794,11 +863,6 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
   }
   if (!ok) return fail(HSNF4_ERR_CUDA, "lora gemm: cuTensorMapEncodeTiled failed");
 
-  if (L.need) {
-    int rc = cuda_status(cudaMemsetAsync(ws + L.cnt_off, 0, L.cnt_bytes, st),
-                         "lora gemm: clear split counters");
-    if (rc) return rc;
-  }
   if (configure_once<kGemmFwd>() != 0 || configure_once<kGemmDx>() != 0)
     return fail(HSNF4_ERR_CUDA, "lora gemm: smem attribute");
   const int smem = smem_plan(mode, BN, tl.sx, tl.sc, tl.sa, r_pad).total + 1024;
@@ -807,7 +871,30 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     lora_gemm_kernel<kGemmFwd><<<G, kThreads, smem, st>>>(P);
   else
     lora_gemm_kernel<kGemmDx><<<G, kThreads, smem, st>>>(P);
-  const cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess && L.need) {
+    // add the K-split partials in split order and write the bf16 outputs
+    static ReduceParams R;
+    R.n_tiles = 0;
+    R.BN = BN;
+    R.T = static_cast<int>(T);
+    for (int p = 0; p < n; ++p) {
+      const GemmProblem& g = P.prob[p];
+      if (g.splits <= 1) continue;
+      for (int tt = 0; tt < t_tiles; ++tt)
+        for (int mt = 0; mt < g.m_tiles; ++mt) {
+          if (R.n_tiles == kMaxReduceTiles) {
+            lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 64, 0, st>>>(R);
+            R.n_tiles = 0;
+          }
+          const int tile = tt * g.m_tiles + mt;
+          R.tile[R.n_tiles++] = {g.partial + static_cast<int64_t>(tile) * g.splits * kTileM * BN,
+                                 g.out, mt * kTileM, tt * BN, g.m_total, g.splits};
+        }
+    }
+    if (R.n_tiles) lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 64, 0, st>>>(R);
+    e = cudaGetLastError();
+  }
   if (prof) {
     // algorithmic FLOPs: the base products plus the rank-r slices
     double flops = 0;

@@ -88,7 +88,7 @@ struct hsnf4_streamer {
   size_t slot_bytes = 0;
   cudaStream_t copy = nullptr;
   int n_blocks = 0;
-  Slot slots[2];
+  std::vector<Slot> slots;
   uint64_t seq = 0;
   hsnf4_stream_stats stats{};
   std::mutex mu;
@@ -105,7 +105,7 @@ struct hsnf4_streamer {
   }
   // Slot holding block b in `state`, or -1.
   int find(int b, SlotState state) const {
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < static_cast<int>(slots.size()); ++i)
       if (slots[i].block == b && slots[i].state == state) return i;
     return -1;
   }
@@ -152,19 +152,35 @@ int enqueue_copy(hsnf4_streamer* s, int i, int b, cudaStream_t after) {
   return HSNF4_OK;
 }
 
-// Pick the slot a new copy of block b goes to, or -1 (detail set).
-int choose_slot(hsnf4_streamer* s, int b) {
-  int best = -1;
-  for (int i = 0; i < 2; ++i) {
+// Pick the slot a new copy of block b goes to: an empty slot, else a
+// released slot -- the one whose block is needed furthest in the future
+// according to `upcoming` (blocks not listed count as never needed; ties go
+// to the least recently used).  Returns -1 (detail set unless quiet) if
+// every slot holds a block that is prefetched or in use.
+int choose_slot(hsnf4_streamer* s, int b, const int* upcoming = nullptr, int n_up = 0,
+                bool quiet = false) {
+  int best = -1, best_next = -1;
+  for (int i = 0; i < static_cast<int>(s->slots.size()); ++i) {
     const Slot& sl = s->slots[i];
     if (sl.state == kEmpty) return i;
-    if (sl.state == kReleased && (best < 0 || sl.last_use < s->slots[best].last_use)) best = i;
+    if (sl.state != kReleased) continue;
+    int next = 1 << 30;  // not needed within the window
+    for (int k = 0; k < n_up; ++k)
+      if (upcoming[k] == sl.block) {
+        next = k;
+        break;
+      }
+    if (best < 0 || next > best_next ||
+        (next == best_next && sl.last_use < s->slots[best].last_use)) {
+      best = i;
+      best_next = next;
+    }
   }
-  if (best < 0)
+  if (best < 0 && !quiet)
     fail(HSNF4_ERR_STATE,
-         "prefetch(%d): no free slot -- both slots hold blocks (%d, %d) that are prefetched or "
+         "prefetch(%d): no free slot -- all %zu slots hold blocks that are prefetched or "
          "acquired and not released; release before prefetching further ahead",
-         b, s->slots[0].block, s->slots[1].block);
+         b, s->slots.size());
   return best;
 }
 
@@ -212,6 +228,15 @@ int stream_slab_bytes(const hsnf4_layer_desc* layers, int n_layers, size_t* out_
   return HSNF4_OK;
 }
 
+int stream_slot_bytes(const hsnf4_layer_desc* layers, int n_layers, int block_size,
+                      size_t* out_bytes) {
+  size_t ring = 0;
+  int rc = stream_ring_bytes(layers, n_layers, block_size, &ring);
+  if (rc) return rc;
+  *out_bytes = ring / 2;
+  return HSNF4_OK;
+}
+
 int stream_ring_bytes(const hsnf4_layer_desc* layers, int n_layers, int block_size,
                       size_t* out_bytes) {
   if (!layers || n_layers < 1 || !out_bytes || block_size < 1)
@@ -242,19 +267,25 @@ int stream_create(const void* pinned_slab, size_t slab_bytes, const hsnf4_layer_
     return fail(HSNF4_ERR_INVALID, "%s: block_size must be >= 1 (got %d)", fn, cfg->block_size);
   if (reinterpret_cast<uintptr_t>(ring_dev) % kAlign)
     return fail(HSNF4_ERR_INVALID, "%s: ring must be %zu-byte aligned", fn, kAlign);
+  const int n_slots = cfg->n_slots == 0 ? 2 : cfg->n_slots;
+  if (n_slots < 2 || n_slots > HSNF4_MAX_SLOTS)
+    return fail(HSNF4_ERR_INVALID, "%s: n_slots must be 0 (= 2) or in [2, %d] (got %d)", fn,
+                HSNF4_MAX_SLOTS, cfg->n_slots);
   size_t need_slab = 0, need_ring = 0;
   int rc = stream_slab_bytes(layers, n_layers, &need_slab);
   if (rc) return rc;
-  rc = stream_ring_bytes(layers, n_layers, cfg->block_size, &need_ring);
+  rc = stream_slot_bytes(layers, n_layers, cfg->block_size, &need_ring);
   if (rc) return rc;
+  const size_t slot_bytes = need_ring;
+  need_ring *= static_cast<size_t>(n_slots);
   if (slab_bytes < need_slab)
     return fail(HSNF4_ERR_OOM, "%s: pinned slab too small: need %zu bytes, given %zu", fn,
                 need_slab, slab_bytes);
   if (ring_bytes < need_ring)
     return fail(HSNF4_ERR_OOM,
-                "%s: ring too small for block_size=%d: need %zu bytes, given %zu (lower "
-                "block_size to shrink the ring)",
-                fn, cfg->block_size, need_ring, ring_bytes);
+                "%s: ring too small for block_size=%d and %d slots: need %zu bytes, given %zu "
+                "(lower block_size to shrink the ring)",
+                fn, cfg->block_size, n_slots, need_ring, ring_bytes);
   auto* s = new (std::nothrow) hsnf4_streamer();
   if (!s) return fail(HSNF4_ERR_OOM, "%s: host allocation failed", fn);
   s->slab = static_cast<const uint8_t*>(pinned_slab);
@@ -269,7 +300,8 @@ int stream_create(const void* pinned_slab, size_t slab_bytes, const hsnf4_layer_
   s->cfg = *cfg;
   if (s->cfg.poison_on_release) s->cfg.reuse_resident = 0;  // poisoned data is never reused
   s->ring = static_cast<uint8_t*>(ring_dev);
-  s->slot_bytes = need_ring / 2;
+  s->slot_bytes = slot_bytes;
+  s->slots.resize(static_cast<size_t>(n_slots));
   s->copy = static_cast<cudaStream_t>(copy_stream);
   s->n_blocks = (n_layers + cfg->block_size - 1) / cfg->block_size;
   for (auto& sl : s->slots) {
@@ -313,6 +345,37 @@ int stream_block_prefetch(hsnf4_streamer* s, int block) {
   const int i = choose_slot(s, block);
   if (i < 0) return HSNF4_ERR_STATE;
   return enqueue_copy(s, i, block, nullptr);
+}
+
+int stream_prefetch_ahead(hsnf4_streamer* s, const int* upcoming, int n, int* issued) {
+  if (issued) *issued = 0;
+  if (!s || (!upcoming && n > 0) || n < 0)
+    return fail(HSNF4_ERR_INVALID, "stream_prefetch_ahead: NULL streamer or list");
+  for (int k = 0; k < n; ++k) {
+    int rc = check_block("stream_prefetch_ahead", s, upcoming[k]);
+    if (rc) return rc;
+  }
+  std::lock_guard<std::mutex> lk(s->mu);
+  for (int k = 0; k < n; ++k) {
+    const int b = upcoming[k];
+    if (s->find(b, kLoaded) >= 0) continue;
+    if (s->cfg.reuse_resident) {
+      if (s->find(b, kAcquired) >= 0) continue;  // in use now and still resident then
+      const int rel = s->find(b, kReleased);
+      if (rel >= 0) {  // keep it: it is needed soon
+        s->slots[rel].state = kLoaded;
+        s->stats.reuses += 1;
+        continue;
+      }
+    }
+    if (!s->cfg.enable_prefetch) break;
+    const int i = choose_slot(s, b, upcoming + k + 1, n - k - 1, /*quiet=*/true);
+    if (i < 0) break;  // the ring is full of blocks still needed: stop here
+    int rc = enqueue_copy(s, i, b, nullptr);
+    if (rc) return rc;
+    if (issued) ++*issued;
+  }
+  return HSNF4_OK;
 }
 
 int stream_block_acquire(hsnf4_streamer* s, int block, void* compute_stream,
@@ -427,7 +490,7 @@ int stream_stats(const hsnf4_streamer* s, hsnf4_stream_stats* out) {
 int stream_destroy(hsnf4_streamer* s) {
   if (!s) return HSNF4_OK;
   int rc = HSNF4_OK;
-  if (s->copy || s->slots[0].ready)
+  if (s->copy || (!s->slots.empty() && s->slots[0].ready))
     rc = cuda_status(cudaStreamSynchronize(s->copy), "stream_destroy: synchronize copy stream");
   for (auto& sl : s->slots) {
     if (sl.ready) cudaEventDestroy(sl.ready);

@@ -42,7 +42,7 @@ class LayerDesc(Structure):
 
 class StreamConfig(Structure):
     _fields_ = [("block_size", c_int), ("enable_prefetch", c_int), ("reuse_resident", c_int),
-                ("poison_on_release", c_int)]
+                ("poison_on_release", c_int), ("n_slots", c_int)]
 
 
 class StreamStats(Structure):
@@ -94,6 +94,8 @@ _SIGS = {
     "stream_layer_offsets": ([POINTER(LayerDesc), c_int, POINTER(c_size_t), POINTER(c_size_t)], c_int),
     "stream_slab_bytes": ([POINTER(LayerDesc), c_int, POINTER(c_size_t)], c_int),
     "stream_ring_bytes": ([POINTER(LayerDesc), c_int, c_int, POINTER(c_size_t)], c_int),
+    "stream_slot_bytes": ([POINTER(LayerDesc), c_int, c_int, POINTER(c_size_t)], c_int),
+    "stream_prefetch_ahead": ([c_void_p, POINTER(c_int), c_int, POINTER(c_int)], c_int),
     "stream_create": ([c_void_p, c_size_t, POINTER(LayerDesc), c_int, POINTER(StreamConfig), c_void_p,
                        c_size_t, c_void_p, POINTER(c_void_p)], c_int),
     "stream_num_blocks": ([c_void_p], c_int),
@@ -371,10 +373,10 @@ def slab_bytes(descs) -> int:
     return out.value
 
 
-def ring_bytes(descs, block_size: int) -> int:
+def ring_bytes(descs, block_size: int, n_slots: int = 2) -> int:
     out = c_size_t(0)
-    _check(lib().stream_ring_bytes(_desc_array(descs), len(descs), block_size, ctypes.byref(out)))
-    return out.value
+    _check(lib().stream_slot_bytes(_desc_array(descs), len(descs), block_size, ctypes.byref(out)))
+    return out.value * n_slots
 
 
 class Streamer:
@@ -382,7 +384,7 @@ class Streamer:
 
     def __init__(self, slab: torch.Tensor, descs, block_size: int, ring: torch.Tensor,
                  copy_stream: torch.cuda.Stream, enable_prefetch=True, reuse_resident=True,
-                 poison_on_release=False):
+                 poison_on_release=False, n_slots=2):
         _need(slab, "slab", torch.uint8, device=False)
         if not slab.is_pinned():
             raise ValueError("slab must be page-locked (pin_memory)")
@@ -390,7 +392,8 @@ class Streamer:
         self.descs = list(descs)
         self._arr = _desc_array(self.descs)
         cfg = StreamConfig(block_size, int(bool(enable_prefetch)), int(bool(reuse_resident)),
-                           int(bool(poison_on_release)))
+                           int(bool(poison_on_release)), int(n_slots))
+        self.n_slots = n_slots
         h = c_void_p()
         _check(lib().stream_create(_ptr(slab), slab.numel(), self._arr, len(self.descs),
                                    ctypes.byref(cfg), _ptr(ring), ring.numel(),
@@ -402,6 +405,12 @@ class Streamer:
 
     def prefetch(self, b: int):
         _check(lib().stream_block_prefetch(self._h, b))
+
+    def prefetch_ahead(self, upcoming) -> int:
+        arr = (c_int * len(upcoming))(*upcoming)
+        issued = c_int(0)
+        _check(lib().stream_prefetch_ahead(self._h, arr, len(upcoming), ctypes.byref(issued)))
+        return issued.value
 
     def acquire(self, b: int, stream=None):
         first = b * self.block_size

@@ -55,7 +55,7 @@ class LayerStack:
     def __init__(self, family: synth.Family, n_layers: int, T: int, *, block_size: int = 4,
                  streamed: bool = True, reuse_resident: bool = True, enable_prefetch: bool = True,
                  poison_on_release: bool = False, r: int = synth.RANK, alpha: float = synth.ALPHA,
-                 seed: int = 42, device=None, grouping: str = "decoder"):
+                 seed: int = 42, device=None, grouping: str = "layer", n_slots: int = 2):
         self.device = torch.device(device) if device is not None else torch.device(
             "cuda", torch.cuda.current_device())
         dev = self.device
@@ -74,13 +74,13 @@ class LayerStack:
 
         self.compute = torch.cuda.current_stream(dev)
         if streamed:
-            self.ring = torch.empty(hsnf4.ring_bytes(self.descs, block_size), dtype=torch.uint8,
-                                    device=dev)
+            self.ring = torch.empty(hsnf4.ring_bytes(self.descs, block_size, n_slots),
+                                    dtype=torch.uint8, device=dev)
             self.copy_stream = torch.cuda.Stream(dev)
             self.streamer = hsnf4.Streamer(self.slab, self.descs, block_size, self.ring,
                                            self.copy_stream, enable_prefetch=enable_prefetch,
                                            reuse_resident=reuse_resident,
-                                           poison_on_release=poison_on_release)
+                                           poison_on_release=poison_on_release, n_slots=n_slots)
         else:
             self.dev_slab = self.slab.to(dev)
             self.streamer = None
@@ -93,16 +93,26 @@ class LayerStack:
                   "i": _randn_bf16((T, family.inter), 1.0, g, dev)}
         self.dY = [_randn_bf16((T, n), 1.0, g, dev) for _, n, _ in self.projs]
         # adapters (always resident) and per-(layer, projection) outputs kept for the backward
+        # every adapter gradient lives in one flat fp32 buffer (dA then dB per
+        # layer and projection), so that data-parallel ranks can sum them with
+        # one all-reduce
+        per_layer = sum(r * k + n * r for _, n, k in self.projs)
+        self.grad_flat = torch.empty(n_layers * per_layer, dtype=torch.float32, device=dev)
         self.A, self.B, self.t, self.dA, self.dB = [], [], [], [], []
+        off = 0
         for l in range(n_layers):
             ga = _gen(dev, seed, 2_000_000 + l)
             self.A.append([_randn_bf16((r, k), synth.A_STD, ga, dev) for _, _, k in self.projs])
             self.B.append([_randn_bf16((n, r), synth.B_STD, ga, dev) for _, n, _ in self.projs])
             self.t.append([torch.empty(T, r, dtype=torch.float32, device=dev) for _ in self.projs])
-            self.dA.append([torch.empty(r, k, dtype=torch.float32, device=dev)
-                            for _, _, k in self.projs])
-            self.dB.append([torch.empty(n, r, dtype=torch.float32, device=dev)
-                            for _, n, _ in self.projs])
+            dA, dB = [], []
+            for _, n, k in self.projs:
+                dA.append(self.grad_flat[off: off + r * k].view(r, k))
+                off += r * k
+                dB.append(self.grad_flat[off: off + n * r].view(n, r))
+                off += n * r
+            self.dA.append(dA)
+            self.dB.append(dB)
         self.Y = [torch.empty(T, n, dtype=torch.bfloat16, device=dev) for _, n, _ in self.projs]
         self.dX = [torch.empty(T, k, dtype=torch.bfloat16, device=dev) for _, _, k in self.projs]
         # workspaces: the largest any group needs (addresses do not matter here)
@@ -212,9 +222,31 @@ class LayerStack:
             self._bwd_block(ws, b, record)
             self._release(b)
 
+    def visits(self):
+        """One step's block visits: forward in order, then backward reversed."""
+        nb = self.n_blocks
+        return [(b, True) for b in range(nb)] + [(b, False) for b in reversed(range(nb))]
+
     def step(self, record=None):
-        self.forward(record)
-        self.backward(record)
+        """One training step.  Streamed: at each visit the block is acquired,
+        the upcoming visits (wrapping into the next step) are prefetched as
+        far as the ring allows, the block is computed and released."""
+        V = self.visits()
+        if not self.streamed:
+            for b, fwd in V:
+                ws = self._weights(b)
+                (self._fwd_block if fwd else self._bwd_block)(ws, b, record)
+            return
+        n = len(V)
+        look = 2 * self.streamer.n_slots
+        if not self._prefetched:
+            self.streamer.prefetch_ahead([V[0][0]])
+            self._prefetched = True
+        for i, (b, fwd) in enumerate(V):
+            ws = self.streamer.acquire(b, self.compute)
+            self.streamer.prefetch_ahead([V[(i + j) % n][0] for j in range(1, look + 1)])
+            (self._fwd_block if fwd else self._bwd_block)(ws, b, record)
+            self.streamer.release(b, self.compute)
 
     def step_single_block(self, record=None):
         """A one-block stack whose block is re-streamed every step: acquire the
@@ -237,19 +269,20 @@ class LayerStack:
     def block_bytes(self, b: int) -> int:
         return len(self.block_layers(b)) * self.layer_bytes
 
-    def steady_h2d_bytes_per_step(self, reuse_resident: bool = True) -> int:
+    def steady_h2d_bytes_per_step(self, reuse_resident: bool = True, n_slots: int = 2) -> int:
         """Bytes one steady-state step copies host -> device.  Without reuse
-        every block crosses once per pass; with reuse the two blocks resident
-        at each turn-around (forward -> backward and backward -> the next
-        forward) are not copied again."""
+        every block crosses once per pass.  With reuse, the blocks still
+        resident at each of the two turn-arounds (forward -> backward and
+        backward -> next forward) are not copied again: the n_slots blocks
+        nearest the turn-around."""
         nb = self.n_blocks
         total = 2 * sum(self.block_bytes(b) for b in range(nb))
         if not reuse_resident:
             return total
-        if nb <= 2:
-            return 0
-        return total - self.block_bytes(nb - 1) - self.block_bytes(nb - 2) \
-            - self.block_bytes(0) - self.block_bytes(1)
+        k = min(n_slots, nb)
+        reused = sum(self.block_bytes(nb - 1 - j) for j in range(k)) + \
+            sum(self.block_bytes(j) for j in range(k))
+        return max(total - reused, 0)
 
     def kernels_per_step(self) -> int:
         """Library kernels one step launches: per group, the forward runs the

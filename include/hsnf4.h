@@ -272,7 +272,8 @@ int lora_group_bwd(const hsnf4_lora_bwd_args *probs, int n, int64_t T, int r, fl
  * codes then its absmax, each starting on a 1 KiB boundary
  * (stream_layer_offsets).  A block is block_size consecutive layers (the
  * last block may be shorter) and is one contiguous byte range of the slab.
- * The ring holds 2 block slots in caller-provided device memory.
+ * The ring holds n_slots (default 2) block slots in caller-provided device
+ * memory.
  *
  * Protocol for block b (prefetch one ahead):
  *   acquire(b) -> prefetch(next) -> compute on b -> release(b)
@@ -284,6 +285,7 @@ int lora_group_bwd(const hsnf4_lora_bwd_args *probs, int n, int64_t T, int r, fl
  * unless reuse is disabled. */
 
 #define HSNF4_MAX_PROJ 8
+#define HSNF4_MAX_SLOTS 8
 
 typedef struct {
   int n_proj;
@@ -299,6 +301,9 @@ typedef struct {
                           0: only a copy not yet acquired satisfies it, so
                           every pass re-streams its blocks */
   int poison_on_release; /* debug: fill a released slot with 0xFF bytes */
+  int n_slots;         /* block slots in the ring: 0 (= 2, prefetch one
+                          ahead) or 2..HSNF4_MAX_SLOTS; more slots reuse
+                          more blocks at each forward/backward turn-around */
 } hsnf4_stream_config;
 
 typedef struct {
@@ -321,8 +326,13 @@ int stream_layer_offsets(const hsnf4_layer_desc *layer, int proj,
 int stream_slab_bytes(const hsnf4_layer_desc *layers, int n_layers,
                       size_t *out_bytes);
 
-/* Device bytes the 2-slot ring needs for this stack and block_size. */
+/* Device bytes the default 2-slot ring needs for this stack and block_size. */
 int stream_ring_bytes(const hsnf4_layer_desc *layers, int n_layers,
+                      int block_size, size_t *out_bytes);
+
+/* Bytes of one block slot (the largest block); a ring of n_slots needs
+ * n_slots times this. */
+int stream_slot_bytes(const hsnf4_layer_desc *layers, int n_layers,
                       int block_size, size_t *out_bytes);
 
 /* Create a streamer.  pinned_slab: HOST pointer to page-locked memory of
@@ -342,6 +352,15 @@ int stream_num_blocks(const hsnf4_streamer *s);
 /* Enqueue block b's H2D copy into a free slot (asynchronous).  STATE if the
  * only candidate slot holds a block that was acquired and not released. */
 int stream_block_prefetch(hsnf4_streamer *s, int block);
+
+/* Prefetch along the upcoming visit order (upcoming[0] first): blocks
+ * already copied (or, with reuse_resident, in use or still resident) are
+ * kept, and the next blocks that are not resident are copied into free
+ * slots, evicting the released block needed furthest in the future, until
+ * every slot holds a block that is copied, kept or in use.  *issued
+ * (optional) receives the number of copies enqueued.  With 2 slots this is
+ * prefetch-one-ahead. */
+int stream_prefetch_ahead(hsnf4_streamer *s, const int *upcoming, int n, int *issued);
 
 /* Make `compute_stream` wait for block b and return its weights:
  * out[i*n_proj + p] for layer (first layer of b) + i, projection p;

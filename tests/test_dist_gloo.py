@@ -1,0 +1,69 @@
+"""The multi-rank host logic on CPU: two gloo ranks on 127.0.0.1.
+
+Covers what `bench.py --gpus N` relies on besides the GPU: the slowest
+rank's time, the whole-job throughput, and the adapter-gradient all-reduce
+(the data-parallel exchange step) over a flat buffer with per-layer views.
+"""
+import os
+import socket
+
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from host_streamed_nf4_b200 import dist as hdist
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, ws, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        # each rank "took" a different time; the job time is the max
+        ms = 10.0 + 5.0 * rank
+        ms_max = hdist.max_over_ranks(ms)
+        value = hdist.job_throughput(512, 20, ms_max, ws)
+        # flat gradient buffer with views, as the stack lays out dA/dB
+        flat = torch.zeros(3 * 4 + 5 * 4)
+        dA, dB = flat[:12].view(3, 4), flat[12:].view(5, 4)
+        dA.fill_(rank + 1.0)
+        dB.copy_(torch.arange(20, dtype=torch.float32).view(5, 4) * (rank + 1))
+        hdist.allreduce_grads(flat)
+        q.put((rank, ms_max, value, dA.clone(), dB.clone()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_max_time_throughput_and_grad_allreduce():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ms_max, value, dA, dB in results:
+        assert ms_max == 15.0
+        assert abs(value - 2 * 512 * 20 / 0.015) < 1e-6 * value
+        assert torch.equal(dA, torch.full((3, 4), 3.0))  # 1 + 2
+        assert torch.equal(dB, torch.arange(20, dtype=torch.float32).view(5, 4) * 3)
+
+
+def test_single_rank_is_identity():
+    assert hdist.world() == (1, 0)
+    assert hdist.max_over_ranks(7.5) == 7.5
+    flat = torch.ones(4)
+    hdist.allreduce_grads(flat)
+    assert torch.equal(flat, torch.ones(4))
+    assert hdist.job_throughput(512, 10, 1000.0, 1) == 5120.0

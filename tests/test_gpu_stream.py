@@ -51,9 +51,9 @@ def resident6():
     return rec
 
 
-@pytest.mark.parametrize("bs", [1, 2, 4])
-def test_streamed_equals_resident_bitwise(resident6, bs):
-    s = LayerStack(TINY, 6, 96, block_size=bs, streamed=True)
+@pytest.mark.parametrize("bs,slots", [(1, 2), (2, 2), (4, 2), (1, 3), (2, 4)])
+def test_streamed_equals_resident_bitwise(resident6, bs, slots):
+    s = LayerStack(TINY, 6, 96, block_size=bs, streamed=True, n_slots=slots)
     rec = _run(s)
     s.close()
     _assert_bitwise(rec, resident6)
@@ -69,16 +69,19 @@ def test_partial_last_block_bitwise():
         s.close()
 
 
-@pytest.mark.parametrize("bs,reuse", [(1, True), (2, True), (4, True), (1, False), (2, False)])
-def test_h2d_bytes_match_the_schedule(bs, reuse):
-    s = LayerStack(TINY, 6, 32, block_size=bs, streamed=True, reuse_resident=reuse)
+@pytest.mark.parametrize("bs,reuse,slots", [(1, True, 2), (2, True, 2), (4, True, 2),
+                                             (1, False, 2), (2, False, 2), (1, True, 3),
+                                             (1, True, 4), (2, True, 3)])
+def test_h2d_bytes_match_the_schedule(bs, reuse, slots):
+    s = LayerStack(TINY, 6, 32, block_size=bs, streamed=True, reuse_resident=reuse, n_slots=slots)
+    s.step()
     s.step()
     before = s.streamer.stats()
     s.step()
     torch.cuda.synchronize()
     after = s.streamer.stats()
     moved = after["h2d_bytes"] - before["h2d_bytes"]
-    assert moved == s.steady_h2d_bytes_per_step(reuse_resident=reuse)
+    assert moved == s.steady_h2d_bytes_per_step(reuse_resident=reuse, n_slots=slots)
     assert after["acquires"] - before["acquires"] == 2 * s.n_blocks
     assert after["releases"] - before["releases"] == 2 * s.n_blocks
     s.close()
@@ -100,12 +103,12 @@ def test_no_prefetch_mode_bitwise(resident6):
 
 # ---------------------------------------------------------------- protocol
 
-def _small_streamer(reuse=True, n_layers=4, bs=1):
+def _small_streamer(reuse=True, n_layers=4, bs=1, slots=2):
     descs = [hsnf4.layer_desc([(128, 256), (64, 128)])] * n_layers
     slab = torch.zeros(hsnf4.slab_bytes(descs), dtype=torch.uint8, pin_memory=True)
-    ring = torch.empty(hsnf4.ring_bytes(descs, bs), dtype=torch.uint8, device="cuda")
+    ring = torch.empty(hsnf4.ring_bytes(descs, bs, slots), dtype=torch.uint8, device="cuda")
     cs = torch.cuda.Stream()
-    return hsnf4.Streamer(slab, descs, bs, ring, cs, reuse_resident=reuse), cs
+    return hsnf4.Streamer(slab, descs, bs, ring, cs, reuse_resident=reuse, n_slots=slots), cs
 
 
 def _status(fn):
@@ -175,3 +178,15 @@ def test_device_bounded_wait_gives_up_and_context_survives():
     assert hsnf4.device_status() == 0  # reading clears
     x = torch.arange(10, device="cuda").sum().item()
     assert x == 45
+
+
+def test_prefetch_ahead_fills_free_slots_in_visit_order():
+    st, _ = _small_streamer(n_layers=6)  # 2 slots
+    assert st.prefetch_ahead([0, 1, 2]) == 2   # two free slots: blocks 0 and 1
+    st.acquire(0)
+    assert st.prefetch_ahead([1, 2, 3]) == 0   # 1 is already there; no free slot for 2
+    st.release(0)
+    assert st.prefetch_ahead([1, 2, 3]) == 1   # block 0's slot takes block 2
+    torch.cuda.synchronize()
+    assert st.stats()["copies"] == 3
+    st.close()
