@@ -317,6 +317,10 @@ def run_ours(args, ws, rank, local):
                                     "achieved": round(v["work"] / (v["total_ms"] / 1e3) / 1e12, 1)}
                                 for k, v in gemms.items()}}
 
+    # standalone NF4 dequant on the layer's largest weight (HBM-bound; the
+    # output, 2 B per element, is far larger than L2)
+    dequant = dequant_roofline(stack, fam, dev)
+
     # step-level binding roofline: max(PCIe bytes / link rate, FLOPs / tensor peak)
     flops_step = sum(2.0 * args.seq * n * k * 2 for _, n, k in fam.projections()) * args.layers
     flops_step += sum(2.0 * args.seq * stack.r * (2 * k + 2 * n) + 2.0 * args.seq * stack.r * (k + n)
@@ -349,7 +353,7 @@ def run_ours(args, ws, rank, local):
                    "parallelism": (f"dp{ws} (per-rank tokens, adapter-gradient all-reduce per "
                                    f"step)" if ws > 1 else "single"),
                    "l2": "no flush: every step reads > 126 MB L2 (NF4 weights + activations)"},
-        "roofline": roofline, "step_roofline": step_roofline, "e2e": e2e,
+        "roofline": roofline, "step_roofline": step_roofline, "dequant": dequant, "e2e": e2e,
         "gpu_launches": K * stack.kernels_per_step(),
         "clocks": clocks.summary(),
     }
@@ -357,6 +361,39 @@ def run_ours(args, ws, rank, local):
         out["cpu_baseline"] = cpu_baseline(args, fam)
     stack.close()
     return out
+
+
+def dequant_roofline(stack, fam, dev):
+    """nf4_dequant of the layer's largest projection, timed with CUDA events
+    (library-side, on the launch stream) against the measured HBM copy rate."""
+    import torch
+
+    from host_streamed_nf4_b200 import hsnf4
+    p = max(range(len(stack.projs)), key=lambda i: stack.projs[i][1] * stack.projs[i][2])
+    _, n, k = stack.projs[p]
+    co, ao = stack.offs[p]
+    codes = torch.empty(n * k // 2, dtype=torch.uint8, device=dev)
+    absmax = torch.empty(n * k // 64, dtype=torch.float32, device=dev)
+    codes.copy_(stack.slab[co: co + n * k // 2])
+    absmax.copy_(stack.slab[ao: ao + n * k // 16].view(torch.float32))
+    W = hsnf4.Nf4Weight(codes, absmax, n, k)
+    out = torch.empty(n, k, dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        hsnf4.nf4_dequant(W, out)
+    torch.cuda.synchronize(dev)
+    hsnf4.profile(True)
+    for _ in range(10):
+        hsnf4.nf4_dequant(W, out)
+    torch.cuda.synchronize(dev)
+    d = hsnf4.profile_read()["nf4_dequant"]
+    hsnf4.profile(False)
+    hbm, _, _, src = measured_peaks()
+    gbs = d["work"] / (d["total_ms"] / 1e3) / 1e9
+    return {"bound": "hbm", "shape": [n, k], "achieved": round(gbs, 1), "peak": hbm,
+            "unit": "GB/s", "frac": round(gbs / hbm, 4),
+            "bytes_per_launch": int(d["work"] / d["launches"]),
+            "avg_launch_us": round(d["total_ms"] / d["launches"] * 1e3, 2),
+            "peak_source": f"{src} hbm_gbs (copy read+write)"}
 
 
 def run_e2e(args, stack, one_step, drain_copies, ws, dev):
