@@ -10,9 +10,11 @@
 //
 // project multiplies exact bf16 inputs on the tensor cores (mma.sync
 // m16n8k16, fp32 accumulate) over 64-token x 128-column chunks and writes a
-// partial per chunk; a second pass adds the chunks in chunk order.  grad keeps
-// V in fp32 and runs on the CUDA cores with 4 x 4 register tiles; each output
-// is a fixed-order sum.  Both are bound by reading Z once.
+// partial per chunk; a second pass adds the chunks in chunk order.  grad also
+// runs on mma.sync: Z is exact in bf16 and the fp32 V is split into
+// V = hi + lo (two bf16 numbers, |lo| <= 2^-9 |V|), both multiplied, so each
+// product keeps ~16 significant bits and accumulates in fp32, in a fixed
+// token order.  Both are bound by reading Z once.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -22,10 +24,19 @@ namespace hsnf4 {
 constexpr int kMaxAux = 16;
 
 // ---------------------------------------------------------------- project
+// CTA = 64 tokens x one chunk of the contraction (128 to 1024 columns),
+// walked in 128-column sub-chunks; the next sub-chunk is loaded into
+// registers while the current one is multiplied.  Warp tiles of 16 tokens x
+// 8 rank columns keep their accumulators across the sub-chunks; one fp32
+// partial per chunk.  The launch takes the widest chunk that still gives
+// every SM two CTAs, so short token counts keep the grid wide and long ones
+// keep the partial sums few.
 
-constexpr int kPrjTok = 64;   // tokens per chunk
-constexpr int kPrjCols = 128; // contraction columns per chunk
-constexpr int kPrjLd = kPrjCols + 8;  // padded smem row (bf16): conflict-free fragment loads
+constexpr int kPrjTok = 64;          // tokens per CTA
+constexpr int kPrjSub = 128;         // columns per sub-chunk (staged in smem)
+constexpr int kPrjColsMax = 1024;    // widest chunk
+constexpr int kPrjColsMin = kPrjSub; // narrowest chunk (sizes the workspace)
+constexpr int kPrjLd = kPrjSub + 8;  // padded smem row (bf16): conflict-free fragment loads
 
 struct PrjProblem {
   const uint16_t* Z;
@@ -39,7 +50,7 @@ struct PrjProblem {
 
 struct PrjParams {
   PrjProblem p[kMaxAux];
-  int n, T, r, r_pad, t_tiles;
+  int n, T, r, r_pad, t_tiles, cols;  // cols: chunk width
   float s;
 };
 
@@ -58,9 +69,75 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Register staging of one sub-chunk: the Z tile (64 x 128 bf16 = 1024 16-byte
+// pieces, 4 per thread) and the adapter tile (R x 128 bf16, R <= 64: up to
+// 1024 pieces, 4 per thread).
+struct PrjStage {
+  uint4 z[4];
+  uint4 a[4];
+};
+
+__device__ __forceinline__ void prj_load(const PrjParams& P, const PrjProblem& pr, int t0,
+                                         int64_t c0, PrjStage& st) {
+  const int tid = threadIdx.x, R = P.r_pad;
+  const int width = static_cast<int>((pr.C - c0) < kPrjSub ? (pr.C - c0) : kPrjSub);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int v = tid + k * 256;
+    const int row = v >> 4, col = (v & 15) * 8;
+    st.z[k] = make_uint4(0, 0, 0, 0);
+    if (t0 + row < P.T && col < width)
+      st.z[k] = __ldg(reinterpret_cast<const uint4*>(pr.Z + static_cast<int64_t>(t0 + row) * pr.C +
+                                                     c0 + col));
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int v = tid + k * 256;
+    st.a[k] = make_uint4(0, 0, 0, 0);
+    if (pr.r_major) {
+      const int j = v >> 4, col = (v & 15) * 8;  // A [r, C]: row j, 8 columns
+      if (j < P.r && col < width)
+        st.a[k] = __ldg(reinterpret_cast<const uint4*>(pr.adp + static_cast<int64_t>(j) * pr.C +
+                                                       c0 + col));
+    } else {
+      const int c = v / (R / 8), jq = (v % (R / 8)) * 8;  // B [C, r]: column c, 8 ranks
+      if (c < kPrjSub && c < width && jq < P.r)
+        st.a[k] = __ldg(reinterpret_cast<const uint4*>(pr.adp + (c0 + c) * P.r) + jq / 8);
+    }
+  }
+}
+
+__device__ __forceinline__ void prj_store(const PrjParams& P, const PrjProblem& pr,
+                                          const PrjStage& st, uint16_t* zt, uint16_t* at) {
+  const int tid = threadIdx.x, R = P.r_pad;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int v = tid + k * 256;
+    *reinterpret_cast<uint4*>(zt + (v >> 4) * kPrjLd + (v & 15) * 8) = st.z[k];
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int v = tid + k * 256;
+    if (pr.r_major) {
+      const int j = v >> 4;
+      if (j < R) *reinterpret_cast<uint4*>(at + j * kPrjLd + (v & 15) * 8) = st.a[k];
+    } else {
+      const int c = v / (R / 8), jq = (v % (R / 8)) * 8;
+      if (c < kPrjSub) {
+        const uint32_t w[4] = {st.a[k].x, st.a[k].y, st.a[k].z, st.a[k].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          at[(jq + 2 * e) * kPrjLd + c] = static_cast<uint16_t>(w[e] & 0xFFFFu);
+          at[(jq + 2 * e + 1) * kPrjLd + c] = static_cast<uint16_t>(w[e] >> 16);
+        }
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) lora_project_chunks(const __grid_constant__ PrjParams P) {
-  __shared__ __align__(16) uint16_t zs_tile[kPrjTok * kPrjLd];
-  __shared__ __align__(16) uint16_t ad_tile[64 * kPrjLd];
+  __shared__ __align__(16) uint16_t zt[kPrjTok * kPrjLd];
+  __shared__ __align__(16) uint16_t at[64 * kPrjLd];
   int item0[kMaxAux];
 #pragma unroll
   for (int q = 0; q < kMaxAux; ++q) item0[q] = q < P.n ? P.p[q].item0 : 0x7fffffff;
@@ -69,73 +146,56 @@ __global__ void __launch_bounds__(256) lora_project_chunks(const __grid_constant
   const int local = blockIdx.x - pr.item0;
   const int tt = local % P.t_tiles, chunk = local / P.t_tiles;
   const int t0 = tt * kPrjTok;
-  const int64_t c0 = static_cast<int64_t>(chunk) * kPrjCols;
+  const int64_t cb = static_cast<int64_t>(chunk) * P.cols;
+  const int64_t ce = (cb + P.cols) < pr.C ? (cb + P.cols) : pr.C;
   const int R = P.r_pad;
-  const int tid = threadIdx.x;
-
-  // Z chunk: 64 rows x 128 columns, 16-byte loads (C % 64 == 0, so a chunk is
-  // 64 or 128 columns wide)
-  const int width = static_cast<int>((pr.C - c0) < kPrjCols ? (pr.C - c0) : kPrjCols);
-  for (int v = tid; v < kPrjTok * (kPrjCols / 8); v += 256) {
-    const int row = v / (kPrjCols / 8), col = (v % (kPrjCols / 8)) * 8;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (t0 + row < P.T && col < width)
-      val = __ldg(reinterpret_cast<const uint4*>(pr.Z + static_cast<int64_t>(t0 + row) * pr.C +
-                                                 c0 + col));
-    *reinterpret_cast<uint4*>(zs_tile + row * kPrjLd + col) = val;
-  }
-  // adapter chunk as [j][c] (bf16), rows j >= r zero
-  if (pr.r_major) {
-    for (int v = tid; v < R * (kPrjCols / 8); v += 256) {
-      const int j = v / (kPrjCols / 8), col = (v % (kPrjCols / 8)) * 8;
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (j < P.r && col < width)
-        val = __ldg(reinterpret_cast<const uint4*>(pr.adp + static_cast<int64_t>(j) * pr.C + c0 +
-                                                   col));
-      *reinterpret_cast<uint4*>(ad_tile + j * kPrjLd + col) = val;
-    }
-  } else {
-    // B is [C, r]: each 16-byte load holds 8 consecutive j of one column c
-    const int per_row = P.r / 8;
-    for (int v = tid; v < kPrjCols * (R / 8); v += 256) {
-      const int c = v / (R / 8), jq = (v % (R / 8)) * 8;
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (c < width && jq < P.r)
-        val = __ldg(reinterpret_cast<const uint4*>(pr.adp + (c0 + c) * P.r) + jq / 8);
-      (void)per_row;
-      const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, qd = lane & 3;
+  const int n_tiles = (kPrjTok / 16) * (R / 8);  // 8 .. 32 warp tiles
+  float acc[4][4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        ad_tile[(jq + 2 * e) * kPrjLd + c] = static_cast<uint16_t>(w[e] & 0xFFFFu);
-        ad_tile[(jq + 2 * e + 1) * kPrjLd + c] = static_cast<uint16_t>(w[e] >> 16);
+  for (int w = 0; w < 4; ++w)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[w][e] = 0.0f;
+
+  PrjStage st;
+  prj_load(P, pr, t0, cb, st);
+  for (int64_t c0 = cb; c0 < ce; c0 += kPrjSub) {
+    __syncthreads();
+    prj_store(P, pr, st, zt, at);
+    __syncthreads();
+    if (c0 + kPrjSub < ce) prj_load(P, pr, t0, c0 + kPrjSub, st);  // overlaps the MMAs below
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int wt = warp + 8 * w;
+      if (wt >= n_tiles) break;
+      const int m0 = (wt % (kPrjTok / 16)) * 16, n0 = (wt / (kPrjTok / 16)) * 8;
+#pragma unroll
+      for (int k0 = 0; k0 < kPrjSub; k0 += 16) {
+        const uint16_t* ar = zt + (m0 + g) * kPrjLd + k0 + 2 * qd;
+        const uint16_t* br = at + (n0 + g) * kPrjLd + k0 + 2 * qd;
+        mma_bf16_16816(acc[w], *reinterpret_cast<const uint32_t*>(ar),
+                       *reinterpret_cast<const uint32_t*>(ar + 8 * kPrjLd),
+                       *reinterpret_cast<const uint32_t*>(ar + 8),
+                       *reinterpret_cast<const uint32_t*>(ar + 8 * kPrjLd + 8),
+                       *reinterpret_cast<const uint32_t*>(br),
+                       *reinterpret_cast<const uint32_t*>(br + 8));
       }
     }
   }
-  __syncthreads();
-
-  // warp tiles: 16 tokens x 8 rank columns over the chunk's 128 columns
-  const int warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, qd = lane & 3;
-  const int n_tiles = (kPrjTok / 16) * (R / 8);
-  for (int wt = warp; wt < n_tiles; wt += 8) {
-    const int m0 = (wt % (kPrjTok / 16)) * 16, n0 = (wt / (kPrjTok / 16)) * 8;
-    float c[4] = {0.f, 0.f, 0.f, 0.f};
+  float* part = pr.partial + static_cast<int64_t>(chunk) * P.T * R;
 #pragma unroll
-    for (int k0 = 0; k0 < kPrjCols; k0 += 16) {
-      const uint16_t* ar = zs_tile + (m0 + g) * kPrjLd + k0 + 2 * qd;
-      const uint16_t* br = ad_tile + (n0 + g) * kPrjLd + k0 + 2 * qd;
-      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(ar);
-      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(ar + 8 * kPrjLd);
-      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(ar + 8);
-      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(ar + 8 * kPrjLd + 8);
-      const uint32_t b0 = *reinterpret_cast<const uint32_t*>(br);
-      const uint32_t b1 = *reinterpret_cast<const uint32_t*>(br + 8);
-      mma_bf16_16816(c, a0, a1, a2, a3, b0, b1);
-    }
-    float* part = pr.partial + static_cast<int64_t>(chunk) * P.T * R;
+  for (int w = 0; w < 4; ++w) {
+    const int wt = warp + 8 * w;
+    if (wt >= n_tiles) break;
+    const int m0 = (wt % (kPrjTok / 16)) * 16, n0 = (wt / (kPrjTok / 16)) * 8;
     const int ta = t0 + m0 + g, tb = ta + 8, j = n0 + 2 * qd;
-    if (ta < P.T) *reinterpret_cast<float2*>(part + static_cast<int64_t>(ta) * R + j) = make_float2(c[0], c[1]);
-    if (tb < P.T) *reinterpret_cast<float2*>(part + static_cast<int64_t>(tb) * R + j) = make_float2(c[2], c[3]);
+    if (ta < P.T)
+      *reinterpret_cast<float2*>(part + static_cast<int64_t>(ta) * R + j) =
+          make_float2(acc[w][0], acc[w][1]);
+    if (tb < P.T)
+      *reinterpret_cast<float2*>(part + static_cast<int64_t>(tb) * R + j) =
+          make_float2(acc[w][2], acc[w][3]);
   }
 }
 
@@ -149,8 +209,18 @@ __global__ void __launch_bounds__(256) lora_project_sum(const __grid_constant__ 
   const int t = e / P.r_pad, j = e % P.r_pad;
   uint16_t out = 0;
   if (j < P.r) {
+    // loads run ahead in batches of 8; the adds stay in chunk order
     float v = 0.0f;
-    for (int ch = 0; ch < pr.chunks; ++ch) v += __ldg(pr.partial + static_cast<int64_t>(ch) * per + e);
+    const float* src = pr.partial + e;
+    int ch = 0;
+    for (; ch + 8 <= pr.chunks; ch += 8) {
+      float x[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = __ldg(src + static_cast<int64_t>(ch + k) * per);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v += x[k];
+    }
+    for (; ch < pr.chunks; ++ch) v += __ldg(src + static_cast<int64_t>(ch) * per);
     pr.t_out[static_cast<int64_t>(t) * P.r + j] = v;
     const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(P.s, v));
     out = *reinterpret_cast<const uint16_t*>(&b);
@@ -162,7 +232,7 @@ size_t project_workspace_bytes(const ProjectDesc* d, int n, int64_t T, int r) {
   const int r_pad = (r + 15) / 16 * 16;
   size_t total = 0;
   for (int q = 0; q < n; ++q) {
-    const int64_t chunks = (d[q].C + kPrjCols - 1) / kPrjCols;
+    const int64_t chunks = (d[q].C + kPrjColsMin - 1) / kPrjColsMin;
     total += round_up(static_cast<size_t>(chunks) * T * r_pad * 4, 256);
   }
   return total;
@@ -179,6 +249,16 @@ cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, in
   P.r_pad = (r + 15) / 16 * 16;
   P.s = s;
   P.t_tiles = static_cast<int>((T + kPrjTok - 1) / kPrjTok);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  auto grid_for = [&](int cols) {
+    int64_t items = 0;
+    for (int q = 0; q < n; ++q) items += (d[q].C + cols - 1) / cols * P.t_tiles;
+    return items;
+  };
+  P.cols = kPrjColsMax;
+  while (P.cols > kPrjColsMin && grid_for(P.cols) < 2 * sms) P.cols /= 2;
   uint8_t* w = static_cast<uint8_t*>(ws);
   int items = 0;
   for (int q = 0; q < n; ++q) {
@@ -189,7 +269,7 @@ cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, in
     p.zs = static_cast<uint16_t*>(d[q].zs);
     p.C = d[q].C;
     p.r_major = d[q].r_major ? 1 : 0;
-    p.chunks = static_cast<int>((d[q].C + kPrjCols - 1) / kPrjCols);
+    p.chunks = static_cast<int>((d[q].C + P.cols - 1) / P.cols);
     p.partial = reinterpret_cast<float*>(w);
     w += round_up(static_cast<size_t>(p.chunks) * T * P.r_pad * 4, 256);
     p.item0 = items;
@@ -204,12 +284,16 @@ cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, in
 }
 
 // ---------------------------------------------------------------- grad
-// CTA = 64 columns.  Thread (cq, jq, tg): columns 4cq..4cq+3, rank indices
-// 4jq..4jq+3 of the current 16-block, tokens t = tg (mod 4) in increasing
-// order; the 4 token groups are then added in group order.
+// out[c, j] = s * sum_t Z[t, c] V[t, j] as D = A B with A = Z^T (16 columns
+// c x 16 tokens per mma) and B = V (16 tokens x 8 rank indices).  A CTA owns
+// 64 columns and one 16-wide rank block: 8 warps, each a 16 x 8 output tile,
+// over all tokens in chunks of 64 (Z chunk staged row-major and read with
+// ldmatrix.trans; V staged transposed as bf16 hi and lo parts).
 
 constexpr int kGrdCols = 64;
 constexpr int kGrdTok = 64;
+constexpr int kGrdLdZ = kGrdCols + 8;   // padded Z row (bf16): conflict-free ldmatrix
+constexpr int kGrdLdV = kGrdTok + 8;    // padded V^T row (bf16)
 
 struct GrdProblem {
   const uint16_t* Z;
@@ -221,85 +305,110 @@ struct GrdProblem {
 
 struct GrdParams {
   GrdProblem p[kMaxAux];
-  int n, T, r;
+  int n, T, r, jblocks;
   float s;
 };
 
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&d)[4], const void* smem_row) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_row))));
+}
+
 __global__ void __launch_bounds__(256) lora_grad_group(const __grid_constant__ GrdParams P) {
-  __shared__ __align__(16) uint16_t zt[kGrdTok * kGrdCols];
-  __shared__ __align__(16) float vt[kGrdTok * 16];
-  __shared__ __align__(16) float red[4][kGrdCols][16 + 1];
+  __shared__ __align__(16) uint16_t zt[kGrdTok * kGrdLdZ];
+  __shared__ __align__(16) uint16_t vhi[16 * kGrdLdV];
+  __shared__ __align__(16) uint16_t vlo[16 * kGrdLdV];
   int item0[kMaxAux];
 #pragma unroll
   for (int q = 0; q < kMaxAux; ++q) item0[q] = q < P.n ? P.p[q].item0 : 0x7fffffff;
   const int q = find_problem(item0, P.n, blockIdx.x);
   const GrdProblem& pr = P.p[q];
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x - pr.item0) * kGrdCols;
-  const int tid = threadIdx.x;
-  const int cq = tid & 15, jq = (tid >> 4) & 3, tg = tid >> 6;
+  const int local = blockIdx.x - pr.item0;
+  const int jb = (local % P.jblocks) * 16;
+  const int64_t c0 = static_cast<int64_t>(local / P.jblocks) * kGrdCols;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, qd = lane & 3;
+  const int mt = (warp & 3) * 16, nt = (warp >> 2) * 8;  // this warp's 16 columns, 8 ranks
   const int width = static_cast<int>((pr.C - c0) < kGrdCols ? (pr.C - c0) : kGrdCols);
+  const int jn = (P.r - jb) < 16 ? (P.r - jb) : 16;
 
-  for (int jb = 0; jb < P.r; jb += 16) {
-    const int jn = (P.r - jb) < 16 ? (P.r - jb) : 16;  // 8 or 16
-    float acc[4][4];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // register staging of one token chunk: Z 64 x 64 bf16 (2 x 16 B per
+  // thread) and V 64 x 16 fp32 (4 per thread); the next chunk is loaded
+  // while the current one is multiplied
+  uint4 zr[2];
+  float vr[4];
+  auto load = [&](int tc) {
+    const int nt_tok = (P.T - tc) < kGrdTok ? (P.T - tc) : kGrdTok;
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-    for (int tc = 0; tc < P.T; tc += kGrdTok) {
-      const int nt = (P.T - tc) < kGrdTok ? (P.T - tc) : kGrdTok;
-      __syncthreads();
-      for (int v = tid; v < kGrdTok * (kGrdCols / 8); v += 256) {
-        const int row = v / (kGrdCols / 8), col = (v % (kGrdCols / 8)) * 8;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (row < nt && col < width)
-          val = __ldg(reinterpret_cast<const uint4*>(pr.Z + static_cast<int64_t>(tc + row) * pr.C +
+    for (int k = 0; k < 2; ++k) {
+      const int v = tid + k * 256;
+      const int row = v >> 3, col = (v & 7) * 8;
+      zr[k] = make_uint4(0, 0, 0, 0);
+      if (row < nt_tok && col < width)
+        zr[k] = __ldg(reinterpret_cast<const uint4*>(pr.Z + static_cast<int64_t>(tc + row) * pr.C +
                                                      c0 + col));
-        *reinterpret_cast<uint4*>(zt + row * kGrdCols + col) = val;
-      }
-      for (int v = tid; v < kGrdTok * 16; v += 256) {
-        const int row = v >> 4, j = v & 15;
-        vt[v] = (row < nt && j < jn) ? __ldg(pr.V + static_cast<int64_t>(tc + row) * P.r + jb + j)
-                                     : 0.0f;
-      }
-      __syncthreads();
-      for (int i = tg; i < nt; i += 4) {
-        const uint2 zz = *reinterpret_cast<const uint2*>(zt + i * kGrdCols + cq * 4);
-        const float z[4] = {__uint_as_float(zz.x << 16), __uint_as_float(zz.x & 0xFFFF0000u),
-                            __uint_as_float(zz.y << 16), __uint_as_float(zz.y & 0xFFFF0000u)};
-        const float4 vv = *reinterpret_cast<const float4*>(vt + i * 16 + jq * 4);
-        const float w[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(z[a], w[b], acc[a][b]);
-      }
     }
-    // token groups 0..3 added in order
-    for (int g = 0; g < 4; ++g) {
-      if (tg == g) {
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            float& dst = red[0][cq * 4 + a][jq * 4 + b];
-            dst = (g == 0) ? acc[a][b] : dst + acc[a][b];
-          }
-      }
-      __syncthreads();
+    for (int k = 0; k < 4; ++k) {
+      const int v = tid + k * 256;
+      const int row = v >> 4, j = v & 15;
+      vr[k] = (row < nt_tok && j < jn) ? __ldg(pr.V + static_cast<int64_t>(tc + row) * P.r + jb + j)
+                                      : 0.0f;
     }
-    for (int v = tid; v < kGrdCols * 16; v += 256) {
-      const int cl = v >> 4, j = v & 15;
-      if (cl < width && j < jn) {
-        const float val = __fmul_rn(P.s, red[0][cl][j]);
-        const int64_t c = c0 + cl;
-        if (pr.c_major)
-          pr.out[c * P.r + jb + j] = val;
-        else
-          pr.out[static_cast<int64_t>(jb + j) * pr.C + c] = val;
-      }
+  };
+  load(0);
+  for (int tc = 0; tc < P.T; tc += kGrdTok) {
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int v = tid + k * 256;
+      *reinterpret_cast<uint4*>(zt + (v >> 3) * kGrdLdZ + (v & 7) * 8) = zr[k];
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int v = tid + k * 256;
+      const int row = v >> 4, j = v & 15;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(vr[k]);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(vr[k], __bfloat162float(hi)));
+      vhi[j * kGrdLdV + row] = *reinterpret_cast<const uint16_t*>(&hi);
+      vlo[j * kGrdLdV + row] = *reinterpret_cast<const uint16_t*>(&lo);
     }
     __syncthreads();
+    if (tc + kGrdTok < P.T) load(tc + kGrdTok);
+#pragma unroll
+    for (int k0 = 0; k0 < kGrdTok; k0 += 16) {
+      // A = Z^T: submatrices (c 0-7 | 8-15) x (t 0-7 | 8-15), each the transpose
+      // of an 8 x 8 block of the row-major Z chunk
+      uint32_t a[4];
+      const int mrow = lane & 7, which = lane >> 3;  // which: 0..3 -> (c+0,t+0) (c+8,t+0) (c+0,t+8) (c+8,t+8)
+      const uint16_t* src = zt + (k0 + mrow + (which >> 1) * 8) * kGrdLdZ + mt + (which & 1) * 8;
+      ldmatrix_x4_trans(a, src);
+      const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(vhi + (nt + g) * kGrdLdV + k0 + 2 * qd);
+      const uint32_t bh1 = *reinterpret_cast<const uint32_t*>(vhi + (nt + g) * kGrdLdV + k0 + 8 + 2 * qd);
+      const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(vlo + (nt + g) * kGrdLdV + k0 + 2 * qd);
+      const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(vlo + (nt + g) * kGrdLdV + k0 + 8 + 2 * qd);
+      mma_bf16_16816(acc, a[0], a[1], a[2], a[3], bh0, bh1);
+      mma_bf16_16816(acc, a[0], a[1], a[2], a[3], bl0, bl1);
+    }
+  }
+  // acc: (c = mt+g, j = nt+2qd, +1) and (c = mt+g+8, same j)
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int cl = mt + g + 8 * h;
+    if (cl >= width) continue;
+    const int64_t c = c0 + cl;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int j = nt + 2 * qd + e;
+      if (j >= jn) continue;
+      const float val = __fmul_rn(P.s, acc[2 * h + e]);
+      if (pr.c_major)
+        pr.out[c * P.r + jb + j] = val;
+      else
+        pr.out[static_cast<int64_t>(jb + j) * pr.C + c] = val;
+    }
   }
 }
 
@@ -312,6 +421,7 @@ cudaError_t launch_lora_grad_group(const GradDesc* d, int n, int64_t T, int r, f
   P.T = static_cast<int>(T);
   P.r = r;
   P.s = s;
+  P.jblocks = (r + 15) / 16;
   int items = 0;
   for (int q = 0; q < n; ++q) {
     GrdProblem& p = P.p[q];
@@ -321,7 +431,7 @@ cudaError_t launch_lora_grad_group(const GradDesc* d, int n, int64_t T, int r, f
     p.C = d[q].C;
     p.c_major = d[q].c_major ? 1 : 0;
     p.item0 = items;
-    items += static_cast<int>((d[q].C + kGrdCols - 1) / kGrdCols);
+    items += static_cast<int>((d[q].C + kGrdCols - 1) / kGrdCols) * P.jblocks;
   }
   lora_grad_group<<<items, 256, 0, st>>>(P);
   return cudaGetLastError();

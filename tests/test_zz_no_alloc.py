@@ -44,8 +44,10 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     """Checked from the shapes alone: the call fails before touching memory."""
     L = hsnf4.lib()
     fake = 0x10000
-    W = hsnf4.Nf4WeightC(fake, fake, 3584, 18944)
-    rc = L.lora_linear_fwd_noalloc(ctypes.byref(W), fake, 16384, fake, fake, 16, 32.0, fake,
+    # r = 64 over a 32768-wide contraction at 16384 tokens: the rank-r
+    # projection's partial sums alone need 128 MiB
+    W = hsnf4.Nf4WeightC(fake, fake, 4096, 32768)
+    rc = L.lora_linear_fwd_noalloc(ctypes.byref(W), fake, 16384, fake, fake, 64, 128.0, fake,
                                    fake, None)
     assert rc == hsnf4.ERR_INVALID
     msg = hsnf4.last_error()
