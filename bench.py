@@ -325,6 +325,10 @@ def run_ours(args, ws, rank, local):
     flops_step = sum(2.0 * args.seq * n * k * 2 for _, n, k in fam.projections()) * args.layers
     flops_step += sum(2.0 * args.seq * stack.r * (2 * k + 2 * n) + 2.0 * args.seq * stack.r * (k + n)
                       for _, n, k in fam.projections()) * args.layers
+    link = link_probe(stack, dev) if streamed else None
+    roofline["cublas_same_shapes"] = cublas_probe(fam, args.seq, dom, dev)
+    roofline["frac_vs_cublas_same_shapes"] = round(
+        achieved_tflops / roofline["cublas_same_shapes"]["tflops"], 4)
     t_pcie = h2d_step / (PCIE_GEN5_X16_GBPS * 1e9)
     t_tensor = flops_step / (bf16_sus * 1e12)
     t_bound = max(t_pcie, t_tensor)
@@ -334,6 +338,10 @@ def run_ours(args, ws, rank, local):
                      "h2d_bytes_per_step": int(h2d_step),
                      "h2d_GBps": round(h2d_step / (ms_step / 1e3) / 1e9, 2) if streamed else None,
                      "pcie_peak_GBps": PCIE_GEN5_X16_GBPS, "flops_per_step": flops_step}
+    if link:
+        step_roofline["pcie_link"] = link
+        step_roofline["frac_vs_probe"] = round(
+            (h2d_step / (ms_step / 1e3) / 1e9) / link["probe_GBps"], 4)
 
     # ------------------------------------------------ end to end through the API
     e2e = None
@@ -394,6 +402,75 @@ def dequant_roofline(stack, fam, dev):
             "bytes_per_launch": int(d["work"] / d["launches"]),
             "avg_launch_us": round(d["total_ms"] / d["launches"] * 1e3, 2),
             "peak_source": f"{src} hbm_gbs (copy read+write)"}
+
+
+def pcie_link_info(dev):
+    """Current and maximum PCIe generation and width of the device (NVML)."""
+    try:
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(dev)
+        h = pynvml.nvmlDeviceGetHandleByPciBusId(
+            f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0")
+        return {"gen": pynvml.nvmlDeviceGetCurrPcieLinkGeneration(h),
+                "width": pynvml.nvmlDeviceGetCurrPcieLinkWidth(h),
+                "max_gen": pynvml.nvmlDeviceGetMaxPcieLinkGeneration(h),
+                "max_width": pynvml.nvmlDeviceGetMaxPcieLinkWidth(h)}
+    except Exception as e:  # NVML missing or not permitted: report why
+        return {"error": type(e).__name__}
+
+
+def link_probe(stack, dev, reps=8):
+    """A plain pinned-host -> device cudaMemcpyAsync of one ring slot's bytes
+    (the streamer's copy size), repeated on a side stream and timed with CUDA
+    events: the practical rate of this link, beside the theoretical 63 GB/s."""
+    import torch
+    nbytes = min(stack.slab.numel(), stack.ring.numel() // max(1, stack.streamer.n_slots))
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    src = stack.slab[:nbytes]
+    s = torch.cuda.Stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        dst.copy_(src, non_blocking=True)
+        e0.record(s)
+        for _ in range(reps):
+            dst.copy_(src, non_blocking=True)
+        e1.record(s)
+    torch.cuda.synchronize(dev)
+    gbs = nbytes * reps / (e0.elapsed_time(e1) / 1e3) / 1e9
+    out = {"probe_GBps": round(gbs, 2), "probe_bytes": int(nbytes), "probe_copies": reps}
+    out.update(pcie_link_info(dev))
+    del dst
+    return out
+
+
+def cublas_probe(fam, T, kernel, dev, reps=10):
+    """cuBLAS bf16 GEMMs of the same shapes as the dominant grouped kernel
+    (torch.mm; fwd: [T,K] x [K,N] per projection, dx: [T,N] x [N,K]), timed
+    with CUDA events: a same-shape library reference for the tensor peak."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(7)
+    pairs = []
+    for _, n, k in fam.projections():
+        a_rows, inner, outer = (T, k, n) if kernel == "lora_gemm_fwd" else (T, n, k)
+        a = torch.randn(a_rows, inner, generator=g, device=dev, dtype=torch.bfloat16)
+        b = torch.randn(inner, outer, generator=g, device=dev, dtype=torch.bfloat16)
+        pairs.append((a, b, 2.0 * a_rows * inner * outer))
+    for a, b, _ in pairs:
+        torch.mm(a, b)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        for a, b, _ in pairs:
+            torch.mm(a, b)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    sec = e0.elapsed_time(e1) / 1e3
+    flops = reps * sum(f for _, _, f in pairs)
+    return {"tflops": round(flops / sec / 1e12, 1), "gemms_per_pass": len(pairs),
+            "us_per_pass": round(sec / reps * 1e6, 2)}
 
 
 def run_e2e(args, stack, one_step, drain_copies, ws, dev):
@@ -517,7 +594,8 @@ def cpu_baseline(args, family):
     value = tokens / (per_layer * args.layers)
     return {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{tokens} tokens x 1 layer of {family.name} (7 projections, fwd+bwd, "
-                      f"median of {len(times)} runs), scaled to {args.layers} layer(s)"}
+                      f"median of {len(times)} runs), scaled to {args.layers} layer(s)",
+            "extrapolated": args.layers > 1 or tokens < args.seq}
 
 
 def run_reference(args, ws, rank):

@@ -9,13 +9,15 @@
 //             dB = s dY^T t  ([n_out, r]),   dA = s u^T X  ([r, k_in])
 //
 // project multiplies exact bf16 inputs on the tensor cores (mma.sync
-// m16n8k16, fp32 accumulate) over 64-token x 128-column chunks and writes a
-// partial per chunk; a second pass adds the chunks in chunk order.  grad also
+// m16n8k16, fp32 accumulate) over 64-token x 128..1024-column chunks and
+// writes a partial per chunk; a second pass adds the chunks in chunk order.  grad also
 // runs on mma.sync: Z is exact in bf16 and the fp32 V is split into
 // V = hi + lo (two bf16 numbers, |lo| <= 2^-9 |V|), both multiplied, so each
 // product keeps ~16 significant bits and accumulates in fp32, in a fixed
 // token order.  Both are bound by reading Z once.
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 #include "internal.h"
 
@@ -25,18 +27,25 @@ constexpr int kMaxAux = 16;
 
 // ---------------------------------------------------------------- project
 // CTA = 64 tokens x one chunk of the contraction (128 to 1024 columns),
-// walked in 128-column sub-chunks; the next sub-chunk is loaded into
-// registers while the current one is multiplied.  Warp tiles of 16 tokens x
-// 8 rank columns keep their accumulators across the sub-chunks; one fp32
-// partial per chunk.  The launch takes the widest chunk that still gives
-// every SM two CTAs, so short token counts keep the grid wide and long ones
-// keep the partial sums few.
+// walked in 128-column sub-chunks through a 3-stage cp.async ring in shared
+// memory, so two sub-chunks are in flight while one is multiplied.  Warp
+// tiles of 16 tokens x 8 rank columns keep their accumulators across the
+// sub-chunks; one fp32 partial per chunk.  The launch takes the widest chunk
+// that still gives every SM four CTAs (two resident, two waves), so short
+// token counts keep the grid wide and long ones keep the partial sums few.
 
 constexpr int kPrjTok = 64;          // tokens per CTA
-constexpr int kPrjSub = 128;         // columns per sub-chunk (staged in smem)
+constexpr int kPrjSub = 128;         // columns per sub-chunk (one ring stage)
 constexpr int kPrjColsMax = 1024;    // widest chunk
 constexpr int kPrjColsMin = kPrjSub; // narrowest chunk (sizes the workspace)
 constexpr int kPrjLd = kPrjSub + 8;  // padded smem row (bf16): conflict-free fragment loads
+constexpr int kPrjStages = 3;
+constexpr int kPrjZBytes = kPrjTok * kPrjLd * 2;   // Z tile [64][136]
+// adapter tile: A [r, C] staged [j][136] (<= 64 rows), B [C, r] staged [c][R + 8]
+constexpr int kPrjABytes = (64 * kPrjLd * 2) > (kPrjSub * 72 * 2) ? (64 * kPrjLd * 2)
+                                                                 : (kPrjSub * 72 * 2);
+constexpr int kPrjStageBytes = kPrjZBytes + kPrjABytes;
+constexpr int kPrjSmem = kPrjStages * kPrjStageBytes;
 
 struct PrjProblem {
   const uint16_t* Z;
@@ -54,9 +63,12 @@ struct PrjParams {
   float s;
 };
 
-__device__ __forceinline__ int find_problem(const int* item0, int n, int item) {
+// index of the problem whose CTA range holds `item` (problems are laid out
+// back to back; the scan reads the kernel parameters in place)
+template <typename Prob>
+__device__ __forceinline__ int find_problem(const Prob* p, int n, int item) {
   int q = 0;
-  while (q + 1 < n && item >= item0[q + 1]) ++q;
+  while (q + 1 < n && item >= p[q + 1].item0) ++q;
   return q;
 }
 
@@ -69,102 +81,107 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Register staging of one sub-chunk: the Z tile (64 x 128 bf16 = 1024 16-byte
-// pieces, 4 per thread) and the adapter tile (R x 128 bf16, R <= 64: up to
-// 1024 pieces, 4 per thread).
-struct PrjStage {
-  uint4 z[4];
-  uint4 a[4];
-};
+// 16-byte global -> shared copy; src_bytes 0 writes zeros and reads nothing
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
-__device__ __forceinline__ void prj_load(const PrjParams& P, const PrjProblem& pr, int t0,
-                                         int64_t c0, PrjStage& st) {
+__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t& d0, uint32_t& d1, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+               : "=r"(d0), "=r"(d1)
+               : "r"(addr));
+}
+
+// Issue the copies of one sub-chunk [c0, c0 + 128) into a ring stage: the Z
+// tile (64 x 128 bf16 = 1024 16-byte pieces, 4 per thread) and the adapter
+// tile (at most 1024 pieces, 4 per thread).  Rows past T, columns past C and
+// rank indices past r are written as zeros.
+__device__ __forceinline__ void prj_issue(const PrjParams& P, const PrjProblem& pr, int t0,
+                                          int64_t c0, uint32_t stage) {
   const int tid = threadIdx.x, R = P.r_pad;
   const int width = static_cast<int>((pr.C - c0) < kPrjSub ? (pr.C - c0) : kPrjSub);
+  const uint32_t zt = stage, at = stage + kPrjZBytes;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int v = tid + k * 256;
     const int row = v >> 4, col = (v & 15) * 8;
-    st.z[k] = make_uint4(0, 0, 0, 0);
-    if (t0 + row < P.T && col < width)
-      st.z[k] = __ldg(reinterpret_cast<const uint4*>(pr.Z + static_cast<int64_t>(t0 + row) * pr.C +
-                                                     c0 + col));
+    const bool ok = t0 + row < P.T && col < width;
+    const uint16_t* src = ok ? pr.Z + static_cast<int64_t>(t0 + row) * pr.C + c0 + col : pr.Z;
+    cp_async16(zt + (row * kPrjLd + col) * 2, src, ok ? 16 : 0);
   }
+  if (pr.r_major) {  // A [r, C]: stage row j holds A[j, c0 .. c0 + 127]
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int v = tid + k * 256;
-    st.a[k] = make_uint4(0, 0, 0, 0);
-    if (pr.r_major) {
-      const int j = v >> 4, col = (v & 15) * 8;  // A [r, C]: row j, 8 columns
-      if (j < P.r && col < width)
-        st.a[k] = __ldg(reinterpret_cast<const uint4*>(pr.adp + static_cast<int64_t>(j) * pr.C +
-                                                       c0 + col));
-    } else {
-      const int c = v / (R / 8), jq = (v % (R / 8)) * 8;  // B [C, r]: column c, 8 ranks
-      if (c < kPrjSub && c < width && jq < P.r)
-        st.a[k] = __ldg(reinterpret_cast<const uint4*>(pr.adp + (c0 + c) * P.r) + jq / 8);
+    for (int k = 0; k < 4; ++k) {
+      const int v = tid + k * 256;
+      const int j = v >> 4, col = (v & 15) * 8;
+      if (j < R) {
+        const bool ok = j < P.r && col < width;
+        const uint16_t* src = ok ? pr.adp + static_cast<int64_t>(j) * pr.C + c0 + col : pr.adp;
+        cp_async16(at + (j * kPrjLd + col) * 2, src, ok ? 16 : 0);
+      }
     }
-  }
-}
-
-__device__ __forceinline__ void prj_store(const PrjParams& P, const PrjProblem& pr,
-                                          const PrjStage& st, uint16_t* zt, uint16_t* at) {
-  const int tid = threadIdx.x, R = P.r_pad;
+  } else {  // B [C, r]: stage row c holds B[c0 + c, 0 .. R - 1]
+    const int per_row = R / 8;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int v = tid + k * 256;
-    *reinterpret_cast<uint4*>(zt + (v >> 4) * kPrjLd + (v & 15) * 8) = st.z[k];
-  }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int v = tid + k * 256;
-    if (pr.r_major) {
-      const int j = v >> 4;
-      if (j < R) *reinterpret_cast<uint4*>(at + j * kPrjLd + (v & 15) * 8) = st.a[k];
-    } else {
-      const int c = v / (R / 8), jq = (v % (R / 8)) * 8;
+    for (int k = 0; k < 4; ++k) {
+      const int v = tid + k * 256;
+      const int c = v / per_row, jq = (v % per_row) * 8;
       if (c < kPrjSub) {
-        const uint32_t w[4] = {st.a[k].x, st.a[k].y, st.a[k].z, st.a[k].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          at[(jq + 2 * e) * kPrjLd + c] = static_cast<uint16_t>(w[e] & 0xFFFFu);
-          at[(jq + 2 * e + 1) * kPrjLd + c] = static_cast<uint16_t>(w[e] >> 16);
-        }
+        const bool ok = c < width && jq < P.r;
+        const uint16_t* src = ok ? pr.adp + (c0 + c) * P.r + jq : pr.adp;
+        cp_async16(at + (c * (R + 8) + jq) * 2, src, ok ? 16 : 0);
       }
     }
   }
 }
 
-__global__ void __launch_bounds__(256) lora_project_chunks(const __grid_constant__ PrjParams P) {
-  __shared__ __align__(16) uint16_t zt[kPrjTok * kPrjLd];
-  __shared__ __align__(16) uint16_t at[64 * kPrjLd];
-  int item0[kMaxAux];
-#pragma unroll
-  for (int q = 0; q < kMaxAux; ++q) item0[q] = q < P.n ? P.p[q].item0 : 0x7fffffff;
-  const int q = find_problem(item0, P.n, blockIdx.x);
+__global__ void __launch_bounds__(256, 2) lora_project_chunks(const __grid_constant__ PrjParams P) {
+  extern __shared__ __align__(128) uint8_t prj_smem[];
+  const int q = find_problem(P.p, P.n, blockIdx.x);
   const PrjProblem& pr = P.p[q];
   const int local = blockIdx.x - pr.item0;
   const int tt = local % P.t_tiles, chunk = local / P.t_tiles;
   const int t0 = tt * kPrjTok;
   const int64_t cb = static_cast<int64_t>(chunk) * P.cols;
   const int64_t ce = (cb + P.cols) < pr.C ? (cb + P.cols) : pr.C;
+  const int n_sub = static_cast<int>((ce - cb + kPrjSub - 1) / kPrjSub);
   const int R = P.r_pad;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, qd = lane & 3;
   const int n_tiles = (kPrjTok / 16) * (R / 8);  // 8 .. 32 warp tiles
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(prj_smem));
   float acc[4][4];
 #pragma unroll
   for (int w = 0; w < 4; ++w)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[w][e] = 0.0f;
 
-  PrjStage st;
-  prj_load(P, pr, t0, cb, st);
-  for (int64_t c0 = cb; c0 < ce; c0 += kPrjSub) {
-    __syncthreads();
-    prj_store(P, pr, st, zt, at);
-    __syncthreads();
-    if (c0 + kPrjSub < ce) prj_load(P, pr, t0, c0 + kPrjSub, st);  // overlaps the MMAs below
+#pragma unroll
+  for (int i = 0; i < kPrjStages - 1; ++i) {
+    if (i < n_sub) prj_issue(P, pr, t0, cb + static_cast<int64_t>(i) * kPrjSub,
+                             base + i * kPrjStageBytes);
+    cp_async_commit();
+  }
+  for (int i = 0; i < n_sub; ++i) {
+    cp_async_wait<kPrjStages - 2>();  // this thread's copies of sub-chunk i landed
+    __syncthreads();                  // everyone's did; stage (i - 1) is free again
+    const int nx = i + kPrjStages - 1;
+    if (nx < n_sub) prj_issue(P, pr, t0, cb + static_cast<int64_t>(nx) * kPrjSub,
+                              base + (nx % kPrjStages) * kPrjStageBytes);
+    cp_async_commit();
+    const uint8_t* stage = prj_smem + (i % kPrjStages) * kPrjStageBytes;
+    const uint16_t* zt = reinterpret_cast<const uint16_t*>(stage);
+    const uint16_t* at = reinterpret_cast<const uint16_t*>(stage + kPrjZBytes);
+    const uint32_t at_u32 = base + (i % kPrjStages) * kPrjStageBytes + kPrjZBytes;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const int wt = warp + 8 * w;
@@ -173,16 +190,22 @@ __global__ void __launch_bounds__(256) lora_project_chunks(const __grid_constant
 #pragma unroll
       for (int k0 = 0; k0 < kPrjSub; k0 += 16) {
         const uint16_t* ar = zt + (m0 + g) * kPrjLd + k0 + 2 * qd;
-        const uint16_t* br = at + (n0 + g) * kPrjLd + k0 + 2 * qd;
+        uint32_t b0, b1;
+        if (pr.r_major) {
+          const uint16_t* br = at + (n0 + g) * kPrjLd + k0 + 2 * qd;
+          b0 = *reinterpret_cast<const uint32_t*>(br);
+          b1 = *reinterpret_cast<const uint32_t*>(br + 8);
+        } else {  // rows k0 .. k0 + 15 of the [c][R + 8] tile, columns n0 .. n0 + 7
+          ldmatrix_x2_trans(b0, b1, at_u32 + ((k0 + (lane & 15)) * (R + 8) + n0) * 2);
+        }
         mma_bf16_16816(acc[w], *reinterpret_cast<const uint32_t*>(ar),
                        *reinterpret_cast<const uint32_t*>(ar + 8 * kPrjLd),
                        *reinterpret_cast<const uint32_t*>(ar + 8),
-                       *reinterpret_cast<const uint32_t*>(ar + 8 * kPrjLd + 8),
-                       *reinterpret_cast<const uint32_t*>(br),
-                       *reinterpret_cast<const uint32_t*>(br + 8));
+                       *reinterpret_cast<const uint32_t*>(ar + 8 * kPrjLd + 8), b0, b1);
       }
     }
   }
+  cp_async_wait<0>();
   float* part = pr.partial + static_cast<int64_t>(chunk) * P.T * R;
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
@@ -258,7 +281,7 @@ cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, in
     return items;
   };
   P.cols = kPrjColsMax;
-  while (P.cols > kPrjColsMin && grid_for(P.cols) < 2 * sms) P.cols /= 2;
+  while (P.cols > kPrjColsMin && grid_for(P.cols) < 4 * sms) P.cols /= 2;
   uint8_t* w = static_cast<uint8_t*>(ws);
   int items = 0;
   for (int q = 0; q < n; ++q) {
@@ -275,7 +298,14 @@ cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, in
     p.item0 = items;
     items += p.chunks * P.t_tiles;
   }
-  lora_project_chunks<<<items, 256, 0, st>>>(P);
+  static cudaError_t smem_rc = cudaSuccess;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    smem_rc = cudaFuncSetAttribute(lora_project_chunks,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kPrjSmem);
+  });
+  if (smem_rc != cudaSuccess) return smem_rc;
+  lora_project_chunks<<<items, 256, kPrjSmem, st>>>(P);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t outs = static_cast<int64_t>(n) * T * P.r_pad;
@@ -319,10 +349,7 @@ __global__ void __launch_bounds__(256) lora_grad_group(const __grid_constant__ G
   __shared__ __align__(16) uint16_t zt[kGrdTok * kGrdLdZ];
   __shared__ __align__(16) uint16_t vhi[16 * kGrdLdV];
   __shared__ __align__(16) uint16_t vlo[16 * kGrdLdV];
-  int item0[kMaxAux];
-#pragma unroll
-  for (int q = 0; q < kMaxAux; ++q) item0[q] = q < P.n ? P.p[q].item0 : 0x7fffffff;
-  const int q = find_problem(item0, P.n, blockIdx.x);
+  const int q = find_problem(P.p, P.n, blockIdx.x);
   const GrdProblem& pr = P.p[q];
   const int local = blockIdx.x - pr.item0;
   const int jb = (local % P.jblocks) * 16;
