@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--seq", type=int, default=512)
     ap.add_argument("--grouping", choices=["decoder", "layer", "none"], default="layer",
                     help="how a layer's projections are batched into grouped launches")
+    ap.add_argument("--base", choices=["nf4", "bf16"], default="nf4",
+                    help="frozen base format: NF4 (default) or dense bf16 (bf16_bitwise)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=4.0,
@@ -244,7 +246,7 @@ def run_ours(args, ws, rank, local):
     # compute); a stack reuses the blocks still resident at each turn-around.
     stack = LayerStack(fam, args.layers, args.seq, block_size=args.block_size, streamed=streamed,
                        reuse_resident=not single, seed=42 + rank, device=dev,
-                       grouping=args.grouping, n_slots=args.slots)
+                       grouping=args.grouping, n_slots=args.slots, base=args.base)
     compute = stack.compute
 
     def one_step():
@@ -275,11 +277,13 @@ def run_ours(args, ws, rank, local):
     with ClockSampler(local) as clocks:
         barrier(ws)
         torch.cuda.synchronize(dev)
+        launches0 = hsnf4.kernel_launches()
         e0.record(compute)
         for _ in range(K):
             one_step()
         drain_copies()
         e1.record(compute)
+        launches = hsnf4.kernel_launches() - launches0
         torch.cuda.synchronize(dev)
         barrier(ws)
     ms_total = hdist.max_over_ranks(e0.elapsed_time(e1))
@@ -319,7 +323,8 @@ def run_ours(args, ws, rank, local):
 
     # standalone NF4 dequant on the layer's largest weight (HBM-bound; the
     # output, 2 B per element, is far larger than L2)
-    dequant = dequant_roofline(stack, fam, dev)
+    dequant = dequant_roofline(stack, fam, dev) if args.base == "nf4" else None
+    merge = merge_roofline(stack, dev)
 
     # step-level binding roofline: max(PCIe bytes / link rate, FLOPs / tensor peak)
     flops_step = sum(2.0 * args.seq * n * k * 2 for _, n, k in fam.projections()) * args.layers
@@ -354,15 +359,16 @@ def run_ours(args, ws, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded normal weights/activations; no dataset)",
         "config": {"workload": args.workload, "family": args.family, "layers": args.layers,
-                   "tokens": args.seq, "batch": 1, "mode": args.mode,
+                   "tokens": args.seq, "batch": 1, "mode": args.mode, "base": args.base,
                    "block_size": args.block_size, "rank": stack.r, "alpha": stack.alpha,
                    "grouping": args.grouping, "ring_slots": args.slots,
                    "projections": [p[0] for p in fam.projections()],
                    "parallelism": (f"dp{ws} (per-rank tokens, adapter-gradient all-reduce per "
                                    f"step)" if ws > 1 else "single"),
                    "l2": "no flush: every step reads > 126 MB L2 (NF4 weights + activations)"},
-        "roofline": roofline, "step_roofline": step_roofline, "dequant": dequant, "e2e": e2e,
-        "gpu_launches": K * stack.kernels_per_step(),
+        "roofline": roofline, "step_roofline": step_roofline, "dequant": dequant, "merge": merge,
+        "peak_vram_GB": round(torch.cuda.max_memory_allocated(dev) / 1e9, 3), "e2e": e2e,
+        "gpu_launches": launches,  # counted by the library over the timed region
         "clocks": clocks.summary(),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -473,6 +479,46 @@ def cublas_probe(fam, T, kernel, dev, reps=10):
             "us_per_pass": round(sec / reps * 1e6, 2)}
 
 
+def merge_roofline(stack, dev):
+    """lora_merge (merge_and_unload) of the layer's largest projection, timed
+    with CUDA events on the launch stream, against the measured HBM copy
+    rate: algorithmic bytes are the base read plus the bf16 W' written."""
+    import torch
+
+    from host_streamed_nf4_b200 import hsnf4
+    p = max(range(len(stack.projs)), key=lambda i: stack.projs[i][1] * stack.projs[i][2])
+    _, n, k = stack.projs[p]
+    W = stack.layer_weights(0)[p] if not stack.streamed else None
+    keep = None
+    if W is None:  # streamed stack: copy the projection's slab range to the device
+        co, ao = stack.offs[p]
+        nbytes = (ao - co) + n * k // 16 if stack.base == "nf4" else n * k * 2
+        keep = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        keep.copy_(stack.slab[co: co + nbytes])
+        W = hsnf4.Nf4WeightC(keep.data_ptr(), keep.data_ptr() + (ao - co), n, k,
+                             hsnf4.BASE_NF4, 0) if stack.base == "nf4" else \
+            hsnf4.Nf4WeightC(keep.data_ptr(), None, n, k, hsnf4.BASE_BF16, 0)
+    A, B = stack.A[0][p], stack.B[0][p]
+    out = torch.empty(n, k, dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        hsnf4.lora_merge(W, A, B, stack.alpha, out=out)
+    torch.cuda.synchronize(dev)
+    hsnf4.profile(True)
+    for _ in range(10):
+        hsnf4.lora_merge(W, A, B, stack.alpha, out=out)
+    torch.cuda.synchronize(dev)
+    d = hsnf4.profile_read()["lora_merge"]
+    hsnf4.profile(False)
+    hbm, _, _, src = measured_peaks()
+    gbs = d["work"] / (d["total_ms"] / 1e3) / 1e9
+    del keep, out
+    return {"bound": "hbm", "shape": [n, k], "base": stack.base, "achieved": round(gbs, 1),
+            "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+            "bytes_per_launch": int(d["work"] / d["launches"]),
+            "avg_launch_us": round(d["total_ms"] / d["launches"] * 1e3, 2),
+            "peak_source": f"{src} hbm_gbs (copy read+write)"}
+
+
 def run_e2e(args, stack, one_step, drain_copies, ws, dev):
     """Same step through the public API with host buffers: each step copies
     its activations and upstream gradients from pinned host memory and reads
@@ -526,25 +572,28 @@ def run_e2e(args, stack, one_step, drain_copies, ws, dev):
 _ORACLE_W = {}
 
 
-def oracle_sample(family, tokens: int, seed: int = 7):
+def oracle_sample(family, tokens: int, seed: int = 7, base: str = "nf4"):
     """Inputs for `tokens` tokens through one layer of `family` (host arrays);
-    the layer's NF4 weights are drawn and quantized once per family."""
+    the layer's weights are drawn (and, for an NF4 base, quantized) once per
+    family.  A dense base is carried as (bf16 bits, absmax None)."""
     import numpy as np
 
     import oracle
     from host_streamed_nf4_b200 import synth
-    if family.name not in _ORACLE_W:
+    key = (family.name, base)
+    if key not in _ORACLE_W:
         rng = np.random.default_rng(seed)
         ws = []
         for name, n, k in family.projections():
-            codes, absmax = oracle.quantize(synth.normal_bf16(rng, (n, k), synth.W_STD))
+            w = synth.normal_bf16(rng, (n, k), synth.W_STD)
+            codes, absmax = oracle.quantize(w) if base == "nf4" else (w, None)
             ws.append((n, k, codes, absmax,
                        synth.normal_bf16(rng, (synth.RANK, k), synth.A_STD),
                        synth.normal_bf16(rng, (n, synth.RANK), synth.B_STD)))
-        _ORACLE_W[family.name] = ws
+        _ORACLE_W[key] = ws
     rng = np.random.default_rng(seed + tokens)
     cases = []
-    for n, k, codes, absmax, A, B in _ORACLE_W[family.name]:
+    for n, k, codes, absmax, A, B in _ORACLE_W[key]:
         cases.append((n, k, codes, absmax, synth.normal_bf16(rng, (tokens, k), 1.0), A, B,
                       synth.normal_bf16(rng, (tokens, n), 1.0)))
     return cases
@@ -553,18 +602,24 @@ def oracle_sample(family, tokens: int, seed: int = 7):
 def oracle_step(cases, threads):
     import oracle
     for n, k, codes, absmax, X, A, B, dY in cases:
-        oracle.lora_fwd(codes, absmax, n, k, X, A, B, 32.0, n_threads=threads)
+        if absmax is None:
+            oracle.lora_fwd_bf16w(codes, X, A, B, 32.0, n_threads=threads)
+        else:
+            oracle.lora_fwd(codes, absmax, n, k, X, A, B, 32.0, n_threads=threads)
     for n, k, codes, absmax, X, A, B, dY in reversed(cases):
-        oracle.lora_bwd(codes, absmax, n, k, X, A, B, dY, 32.0, n_threads=threads)
+        if absmax is None:
+            oracle.lora_bwd_bf16w(codes, X, A, B, dY, 32.0, n_threads=threads)
+        else:
+            oracle.lora_bwd(codes, absmax, n, k, X, A, B, dY, 32.0, n_threads=threads)
 
 
-def calibrate_tokens(family, target_s, threads):
+def calibrate_tokens(family, target_s, threads, base="nf4"):
     """Largest sample (in tokens) whose oracle step stays near target_s."""
-    cases = oracle_sample(family, 1)
+    cases = oracle_sample(family, 1, base=base)
     t = time.perf_counter()
     oracle_step(cases, threads)
     one = time.perf_counter() - t
-    cases = oracle_sample(family, 2)
+    cases = oracle_sample(family, 2, base=base)
     t = time.perf_counter()
     oracle_step(cases, threads)
     two = time.perf_counter() - t
@@ -580,8 +635,8 @@ def cpu_baseline(args, family):
     import oracle
     oracle.build()
     threads = os.cpu_count() or 1
-    tokens = calibrate_tokens(family, 2.0, threads)
-    cases = oracle_sample(family, tokens)
+    tokens = calibrate_tokens(family, 2.0, threads, args.base)
+    cases = oracle_sample(family, tokens, base=args.base)
     times = []
     t_end = time.perf_counter() + 15.0
     while time.perf_counter() < t_end or len(times) < 2:
@@ -606,8 +661,8 @@ def run_reference(args, ws, rank):
     oracle.build()
     family = synth.FAMILIES[args.family]
     threads = os.cpu_count() or 1
-    tokens = calibrate_tokens(family, args.ref_seconds, threads)
-    cases = oracle_sample(family, tokens)
+    tokens = calibrate_tokens(family, args.ref_seconds, threads, args.base)
+    cases = oracle_sample(family, tokens, base=args.base)
     for _ in range(args.warmup):
         oracle_step(cases, threads)
     t = time.perf_counter()
@@ -621,7 +676,8 @@ def run_reference(args, ws, rank):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": args.workload, "family": args.family, "layers": args.layers,
-                       "tokens": args.seq, "batch": 1, "mode": "cpu-oracle"},
+                       "tokens": args.seq, "batch": 1, "mode": "cpu-oracle",
+                       "base": args.base},
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,
                              "kind": "oracle",
                              "sample": f"{tokens} tokens x 1 layer per step, scaled to "

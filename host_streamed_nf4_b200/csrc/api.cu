@@ -209,6 +209,23 @@ static int check_weight(const char* fn, int i, const hsnf4_nf4_weight& W) {
                 fn, i, (long long)W.n_out, (long long)W.k_in);
   if (W.n_out > (1 << 30) || W.k_in > (1 << 30))
     return fail(HSNF4_ERR_INVALID, "%s: problem %d: weight dimension too large", fn, i);
+  if (W.format == HSNF4_BASE_NF4)
+    return check_ptrs(fn, {{W.codes, "W.codes"}, {W.absmax, "W.absmax"}});
+  if (W.format == HSNF4_BASE_BF16) {
+    if (W.absmax)
+      return fail(HSNF4_ERR_INVALID, "%s: problem %d: a BF16 base weight takes absmax = NULL",
+                  fn, i);
+    return check_ptrs(fn, {{W.codes, "W.codes (bf16 weight)"}});
+  }
+  return fail(HSNF4_ERR_INVALID, "%s: problem %d: unknown base format %d", fn, i, W.format);
+}
+
+// one base format per group (the fused GEMM reads all its problems one way)
+static int check_one_format(const char* fn, int n, const int32_t* formats) {
+  for (int i = 1; i < n; ++i)
+    if (formats[i] != formats[0])
+      return fail(HSNF4_ERR_INVALID, "%s: problem %d has base format %d, problem 0 has %d; a "
+                  "group takes one format", fn, i, formats[i], formats[0]);
   return HSNF4_OK;
 }
 
@@ -246,7 +263,7 @@ static void fwd_layout(const hsnf4_lora_fwd_args* p, int n, int64_t T, int r, Fw
   for (int i = 0; i < n; ++i) {
     pd[i] = {p[i].X, p[i].W.k_in, p[i].A, true, nullptr, nullptr};
     gd[i] = {p[i].W.codes, p[i].W.absmax, p[i].W.n_out, p[i].W.k_in, p[i].X, p[i].B, nullptr,
-             p[i].Y};
+             p[i].Y, p[i].W.format == HSNF4_BASE_BF16};
   }
   L->prj = off;
   off += project_workspace_bytes(pd, n, T, r);
@@ -278,7 +295,7 @@ static void bwd_layout(const hsnf4_lora_bwd_args* p, int n, int64_t T, int r, Bw
   for (int i = 0; i < n; ++i) {
     pd[i] = {p[i].dY, p[i].W.n_out, p[i].B, false, nullptr, nullptr};
     gd[i] = {p[i].W.codes, p[i].W.absmax, p[i].W.n_out, p[i].W.k_in, p[i].dY, p[i].A, nullptr,
-             p[i].dX};
+             p[i].dX, p[i].W.format == HSNF4_BASE_BF16};
   }
   L->prj = off;
   off += project_workspace_bytes(pd, n, T, r);
@@ -320,11 +337,15 @@ int lora_group_fwd(const hsnf4_lora_fwd_args* probs, int n, int64_t T, int r, fl
   for (int i = 0; i < n; ++i) {
     const hsnf4_lora_fwd_args& p = probs[i];
     rc = check_weight(fn, i, p.W);
-    if (!rc)
-      rc = check_ptrs(fn, {{p.W.codes, "W.codes"}, {p.W.absmax, "W.absmax"}, {p.X, "X"},
-                           {p.A, "A"}, {p.B, "B"}, {p.Y, "Y"}});
+    if (!rc) rc = check_ptrs(fn, {{p.X, "X"}, {p.A, "A"}, {p.B, "B"}, {p.Y, "Y"}});
     if (!rc && p.t_save && !aligned16(p.t_save))
       rc = fail(HSNF4_ERR_INVALID, "%s: problem %d: t_save misaligned", fn, i);
+    if (rc) return rc;
+  }
+  {
+    int32_t formats[8];
+    for (int i = 0; i < n; ++i) formats[i] = probs[i].W.format;
+    rc = check_one_format(fn, n, formats);
     if (rc) return rc;
   }
   FwdLayout L;
@@ -340,7 +361,8 @@ int lora_group_fwd(const hsnf4_lora_fwd_args* probs, int n, int64_t T, int r, fl
     const hsnf4_lora_fwd_args& p = probs[i];
     float* t_out = p.t_save ? p.t_save : reinterpret_cast<float*>(ws + L.tscratch[i]);
     pd[i] = {p.X, p.W.k_in, p.A, true, t_out, ws + L.zs[i]};
-    gd[i] = {p.W.codes, p.W.absmax, p.W.n_out, p.W.k_in, p.X, p.B, ws + L.zs[i], p.Y};
+    gd[i] = {p.W.codes, p.W.absmax, p.W.n_out, p.W.k_in, p.X, p.B, ws + L.zs[i], p.Y,
+             p.W.format == HSNF4_BASE_BF16};
   }
   rc = cuda_status(launch_lora_project_group(pd, n, T, r, s, ws + L.prj, st),
                    "lora_group_fwd: projection launch");
@@ -358,9 +380,14 @@ int lora_group_bwd(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r, fl
     const hsnf4_lora_bwd_args& p = probs[i];
     rc = check_weight(fn, i, p.W);
     if (!rc)
-      rc = check_ptrs(fn, {{p.W.codes, "W.codes"}, {p.W.absmax, "W.absmax"}, {p.X, "X"},
-                           {p.t_save, "t_save"}, {p.A, "A"}, {p.B, "B"}, {p.dY, "dY"},
-                           {p.dX, "dX"}, {p.dA, "dA"}, {p.dB, "dB"}});
+      rc = check_ptrs(fn, {{p.X, "X"}, {p.t_save, "t_save"}, {p.A, "A"}, {p.B, "B"},
+                           {p.dY, "dY"}, {p.dX, "dX"}, {p.dA, "dA"}, {p.dB, "dB"}});
+    if (rc) return rc;
+  }
+  {
+    int32_t formats[8];
+    for (int i = 0; i < n; ++i) formats[i] = probs[i].W.format;
+    rc = check_one_format(fn, n, formats);
     if (rc) return rc;
   }
   BwdLayout L;
@@ -377,7 +404,8 @@ int lora_group_bwd(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r, fl
     const hsnf4_lora_bwd_args& p = probs[i];
     float* u = reinterpret_cast<float*>(ws + L.u[i]);
     pd[i] = {p.dY, p.W.n_out, p.B, false, u, ws + L.su[i]};
-    gd[i] = {p.W.codes, p.W.absmax, p.W.n_out, p.W.k_in, p.dY, p.A, ws + L.su[i], p.dX};
+    gd[i] = {p.W.codes, p.W.absmax, p.W.n_out, p.W.k_in, p.dY, p.A, ws + L.su[i], p.dX,
+             p.W.format == HSNF4_BASE_BF16};
     grd[2 * i] = {p.dY, p.W.n_out, p.t_save, p.dB, true};  // dB = s dY^T t  [n_out, r]
     grd[2 * i + 1] = {p.X, p.W.k_in, u, p.dA, false};      // dA = s u^T X   [r, k_in]
   }
@@ -388,6 +416,25 @@ int lora_group_bwd(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r, fl
   if (rc) return rc;
   return cuda_status(launch_lora_grad_group(grd, 2 * n, T, r, s, st),
                      "lora_group_bwd: gradient launch");
+}
+
+int lora_merge(const hsnf4_nf4_weight* W, const void* A, const void* B, int r, float alpha,
+               void* W_out, void* stream) {
+  static const char* fn = "lora_merge";
+  if (!W) return fail(HSNF4_ERR_INVALID, "%s: W is NULL", fn);
+  int rc = check_weight(fn, 0, *W);
+  if (rc) return rc;
+  if (r < 8 || r > 64 || r % 8)
+    return fail(HSNF4_ERR_INVALID, "%s: rank must be a multiple of 8 in [8, 64] (got %d)", fn, r);
+  if (!isfinite(alpha)) return fail(HSNF4_ERR_INVALID, "%s: alpha is not finite", fn);
+  rc = check_ptrs(fn, {{A, "A"}, {B, "B"}, {W_out, "W_out"}});
+  if (rc) return rc;
+  if (W_out == W->codes) return fail(HSNF4_ERR_INVALID, "%s: W_out aliases the base", fn);
+  return cuda_status(launch_lora_merge(W->codes, W->absmax, W->format == HSNF4_BASE_BF16,
+                                       W->n_out, W->k_in, A, B, r,
+                                       alpha / static_cast<float>(r), W_out,
+                                       static_cast<cudaStream_t>(stream)),
+                     "lora_merge launch");
 }
 
 static hsnf4_lora_fwd_args one_fwd(const hsnf4_nf4_weight* W, const void* X, const void* A,
@@ -403,7 +450,7 @@ static hsnf4_lora_fwd_args one_fwd(const hsnf4_nf4_weight* W, const void* X, con
 }
 
 size_t lora_linear_fwd_workspace(int64_t T, int64_t n_out, int64_t k_in, int r) {
-  hsnf4_nf4_weight W = {nullptr, nullptr, n_out, k_in};
+  hsnf4_nf4_weight W = {nullptr, nullptr, n_out, k_in, HSNF4_BASE_NF4, 0};
   hsnf4_lora_fwd_args a = one_fwd(&W, nullptr, nullptr, nullptr, nullptr, nullptr);
   return lora_group_fwd_workspace(&a, 1, T, r);
 }

@@ -76,6 +76,7 @@ struct GemmProblemDesc {
   const void* lo_a;
   const void* lo_b;
   void* out;
+  bool dense;  // codes is a bf16 [n_out, k_in] weight (no absmax, no dequant)
 };
 size_t gemm_workspace_bytes(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r);
 int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r,
@@ -83,8 +84,16 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
 
 cudaError_t launch_selftest_stall(cudaStream_t st);
 
+// W' = deq(W) + s B A -> bf16 [N, K] (dense: base is a bf16 weight)
+cudaError_t launch_lora_merge(const void* base, const float* absmax, bool dense, int64_t N,
+                              int64_t K, const void* A, const void* B, int r, float s, void* out,
+                              cudaStream_t st);
+
+// Process-wide count of kernels this library launched (hsnf4_kernel_launches).
+void count_launch();
+
 // Kernel timing (hsnf4_profile): bracket a launch with prof_begin/prof_end.
-enum ProfKind { kProfGemmFwd = 0, kProfGemmDx = 1, kProfDequant = 2, kProfKinds = 3 };
+enum ProfKind { kProfGemmFwd = 0, kProfGemmDx = 1, kProfDequant = 2, kProfMerge = 3, kProfKinds = 4 };
 bool profiling();
 void* prof_begin(cudaStream_t st);
 void prof_end(void* token, int kind, double work, cudaStream_t st);

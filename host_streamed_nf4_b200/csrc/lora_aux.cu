@@ -305,10 +305,12 @@ cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, in
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kPrjSmem);
   });
   if (smem_rc != cudaSuccess) return smem_rc;
+  count_launch();
   lora_project_chunks<<<items, 256, kPrjSmem, st>>>(P);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t outs = static_cast<int64_t>(n) * T * P.r_pad;
+  count_launch();
   lora_project_sum<<<static_cast<unsigned>((outs + 255) / 256), 256, 0, st>>>(P);
   return cudaGetLastError();
 }
@@ -460,6 +462,7 @@ cudaError_t launch_lora_grad_group(const GradDesc* d, int n, int64_t T, int r, f
     p.item0 = items;
     items += static_cast<int>((d[q].C + kGrdCols - 1) / kGrdCols) * P.jblocks;
   }
+  count_launch();
   lora_grad_group<<<items, 256, 0, st>>>(P);
   return cudaGetLastError();
 }

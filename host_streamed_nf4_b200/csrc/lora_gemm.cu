@@ -74,7 +74,8 @@ constexpr int kWarpEpi = 8, kWarpProdX = 12, kWarpProdC = 13, kWarpMma = 14;
 
 struct GemmProblem {
   CUtensorMap map_act;    // X / dY: bf16 [T, contraction], box {64, min(BN,256)}, 128B swizzle
-  CUtensorMap map_codes;  // uint8 [n_out, k_in/2]; box {32, 128} fwd, {64, 64} dx
+  CUtensorMap map_codes;  // uint8 [n_out, k_in/2]; box {32, 128} fwd, {64, 64} dx; dense:
+                          // bf16 [n_out, k_in], box {64, 128} fwd, {64, 64} dx, 128B swizzle
   CUtensorMap map_lo_a;   // fwd: B [n_out, r] box {16, 128} 32B; dx: A [r, k_in] box {64, r_pad} 128B
   CUtensorMap map_lo_b;   // s*t or s*u: bf16 [T, r_pad], box {16, min(BN,256)}, 32B swizzle
   const float* absmax;
@@ -91,6 +92,7 @@ struct GemmParams {
   GemmProblem prob[kMaxProblems];
   Nf4Codebook cb;
   int T, BN, r_pad, n_acc, sx, sc, sa, tmem_cols;
+  int dense;  // 1: map_codes is the bf16 weight, TMA-loaded straight into the A ring
   uint16_t cta_off[kMaxCtas + 1];
   uint32_t units[kMaxUnits];  // problem(3) | split(5) | token tile(6) | row tile(18)
 };
@@ -181,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       mbar_init(&c_empty[s], 128);
     }
     for (int s = 0; s < SA; ++s) {
-      mbar_init(&a_full[s], 128);
+      mbar_init(&a_full[s], P.dense ? 1 : 128);  // TMA (dense) or one dequant warpgroup
       mbar_init(&a_empty[s], 1);
     }
     mbar_init(lora_full, 1);
@@ -249,7 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       }
     }
   } else if (warp == kWarpProdC) {
-    // -------------------------------------------------- raw code tiles
+    // -------------------------------------------------- raw code tiles, or (dense base) the
+    // bf16 weight tiles straight into the A ring: the 128B-swizzled TMA box is
+    // the UMMA operand layout the dequant warps would have written
     if (lane == 0) {
       int g = 0;
       bool ok = true;
@@ -258,6 +262,24 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
         const GemmProblem& pr = P.prob[U.p];
         const int m0 = U.mt * kTileM;
         for (int kb = U.kb0; kb < U.kb1; ++kb, ++g) {
+          if (P.dense) {
+            const int s = g % SA;
+            if (g >= SA && !mbar_wait(&a_empty[s], ((g / SA) - 1) & 1, abort_flag, &g_gemm_flags,
+                                      kFlagProducer)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&a_full[s], static_cast<uint32_t>(kATileBytes));
+            if (MODE == kGemmFwd) {
+              tma_load_2d(a_tile(s), &pr.map_codes, &a_full[s], kb * kStepK, m0);
+            } else {
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d(a_tile(s) + h * (kATileBytes / 2), &pr.map_codes, &a_full[s],
+                            m0 + h * 64, kb * kStepK);
+            }
+            last_c = g;
+            continue;
+          }
           const int s = g % SC;
           if (g >= SC && !mbar_wait(&c_empty[s], ((g / SC) - 1) & 1, abort_flag, &g_gemm_flags,
                                     kFlagProducer)) {
@@ -345,6 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
         umma_commit(acc_full);
       }
     }
+  } else if (warp < kWarpEpi && P.dense) {
+    // dense base: the weight arrives as bf16, the dequant warps have no work
   } else if (warp < kWarpEpi) {
     // -------------------------------------------------- dequant (two warpgroups)
     const int grp = warp >> 2;        // 0 or 1: takes the K steps with g % 2 == grp
@@ -471,8 +495,10 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       if (last_l >= 0) mbar_wait(lora_full, last_l & 1, &never, &g_gemm_flags, kFlagDrain);
     }
     if (warp == kWarpProdC && lane == 0) {
-      for (int g = (last_c - SC + 1 > 0 ? last_c - SC + 1 : 0); g <= last_c; ++g)
-        if (!mbar_wait(&c_full[g % SC], (g / SC) & 1, &never, &g_gemm_flags, kFlagDrain)) break;
+      const int S = P.dense ? SA : SC;
+      uint64_t* full = P.dense ? a_full : c_full;
+      for (int g = (last_c - S + 1 > 0 ? last_c - S + 1 : 0); g <= last_c; ++g)
+        if (!mbar_wait(&full[g % S], (g / S) & 1, &never, &g_gemm_flags, kFlagDrain)) break;
     }
     if (warp == kWarpMma && lane == 0 && mma_started) {
       umma_commit(drain_bar);
@@ -501,6 +527,7 @@ __global__ void selftest_stall_kernel() {
 }
 
 cudaError_t launch_selftest_stall(cudaStream_t st) {
+  count_launch();
   selftest_stall_kernel<<<1, 32, 0, st>>>();
   return cudaGetLastError();
 }
@@ -774,6 +801,10 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
   P.sc = tl.sc;
   P.sa = tl.sa;
   P.cb = codebook();
+  P.dense = probs[0].dense ? 1 : 0;
+  for (int p = 1; p < n; ++p)
+    if (probs[p].dense != probs[0].dense)
+      return fail(HSNF4_ERR_INVALID, "lora gemm: a group takes one base format");
   int tc = 32;
   while (tc < BN) tc <<= 1;
   P.tmem_cols = tc;
@@ -847,14 +878,20 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     if (g.splits > 1) g.partial = reinterpret_cast<float*>(ws + L.part_base[p]);
     ok = ok && encode_2d(&g.map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.act, contraction, T,
                          contraction * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (d.dense)  // bf16 [n_out, k_in]: 64 k x (128 rows fwd | 64 rows dx), 128B swizzle
+      ok = ok && encode_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.codes, d.k_in,
+                           d.n_out, d.k_in * 2, 64, mode == kGemmFwd ? 128 : 64,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
     if (mode == kGemmFwd) {
-      ok = ok && encode_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
-                           d.n_out, d.k_in / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (!d.dense)
+        ok = ok && encode_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
+                             d.n_out, d.k_in / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
       ok = ok && encode_2d(&g.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_a, r, d.n_out,
                            r * 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
     } else {
-      ok = ok && encode_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
-                           d.n_out, d.k_in / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (!d.dense)
+        ok = ok && encode_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
+                             d.n_out, d.k_in / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
       ok = ok && encode_2d(&g.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_a, d.k_in, r,
                            d.k_in * 2, 64, r_pad, CU_TENSOR_MAP_SWIZZLE_128B);
     }
@@ -867,6 +904,7 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     return fail(HSNF4_ERR_CUDA, "lora gemm: smem attribute");
   const int smem = smem_plan(mode, BN, tl.sx, tl.sc, tl.sa, r_pad).total + 1024;
   void* prof = prof_begin(st);
+  count_launch();
   if (mode == kGemmFwd)
     lora_gemm_kernel<kGemmFwd><<<G, kThreads, smem, st>>>(P);
   else
@@ -884,6 +922,7 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
       for (int tt = 0; tt < t_tiles; ++tt)
         for (int mt = 0; mt < g.m_tiles; ++mt) {
           if (R.n_tiles == kMaxReduceTiles) {
+            count_launch();
             lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 64, 0, st>>>(R);
             R.n_tiles = 0;
           }
@@ -892,7 +931,10 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
                                  g.out, mt * kTileM, tt * BN, g.m_total, g.splits};
         }
     }
-    if (R.n_tiles) lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 64, 0, st>>>(R);
+    if (R.n_tiles) {
+      count_launch();
+      lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 64, 0, st>>>(R);
+    }
     e = cudaGetLastError();
   }
   if (prof) {

@@ -84,6 +84,7 @@ cudaError_t launch_nf4_quantize(const void* w, int64_t n_out, int64_t k_in, void
   // The last pair may hold a single block: give the kernel an even-sized
   // view only when the element count allows it (n_blocks even), otherwise
   // the guarded lanes skip the missing half.
+  count_launch();
   nf4_quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(
       static_cast<const uint2*>(w), static_cast<uint16_t*>(codes), absmax, n_pairs, n_blocks,
       codebook());
@@ -120,6 +121,7 @@ cudaError_t launch_nf4_dequant(const void* codes, const float* absmax, int64_t n
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   void* prof = prof_begin(st);
+  count_launch();
   nf4_dequant_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(
       static_cast<const uint32_t*>(codes), absmax, static_cast<uint4*>(out), n_groups,
       codebook());

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -23,9 +24,14 @@ std::mutex g_mu;
 bool g_on = false;
 std::vector<Rec> g_recs;
 
-const char* kKindName[kProfKinds] = {"lora_gemm_fwd", "lora_gemm_dx", "nf4_dequant"};
+const char* kKindName[kProfKinds] = {"lora_gemm_fwd", "lora_gemm_dx", "nf4_dequant",
+                                      "lora_merge"};
 
 }  // namespace
+
+std::atomic<uint64_t> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 bool profiling() { return g_on; }
 
@@ -62,6 +68,8 @@ static void clear_locked() {
 using namespace hsnf4;
 
 extern "C" {
+
+uint64_t hsnf4_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int hsnf4_profile(int enable) {
   std::lock_guard<std::mutex> lk(g_mu);

@@ -38,12 +38,22 @@ size_t proj_codes_bytes(const hsnf4_layer_desc& d, int p) {
 size_t proj_absmax_bytes(const hsnf4_layer_desc& d, int p) {
   return static_cast<size_t>(d.n_out[p]) * static_cast<size_t>(d.k_in[p]) / 64 * 4;
 }
+// slab bytes of projection p: NF4 codes then absmax, or the dense bf16
+// weight, each range starting on a 1 KiB boundary
+size_t proj_bytes(const hsnf4_layer_desc& d, int p) {
+  if (d.base_format == HSNF4_BASE_BF16)
+    return round_up(static_cast<size_t>(d.n_out[p]) * static_cast<size_t>(d.k_in[p]) * 2, kAlign);
+  return round_up(proj_codes_bytes(d, p), kAlign) + round_up(proj_absmax_bytes(d, p), kAlign);
+}
 
 int check_layer(const char* fn, const hsnf4_layer_desc* d) {
   if (!d) return fail(HSNF4_ERR_INVALID, "%s: layer descriptor is NULL", fn);
   if (d->n_proj < 1 || d->n_proj > HSNF4_MAX_PROJ)
     return fail(HSNF4_ERR_INVALID, "%s: n_proj must be in [1, %d] (got %d)", fn, HSNF4_MAX_PROJ,
                 d->n_proj);
+  if (d->base_format != HSNF4_BASE_NF4 && d->base_format != HSNF4_BASE_BF16)
+    return fail(HSNF4_ERR_INVALID, "%s: base_format must be HSNF4_BASE_NF4 or HSNF4_BASE_BF16 "
+                "(got %d)", fn, d->base_format);
   for (int p = 0; p < d->n_proj; ++p)
     if (d->n_out[p] < 1 || d->k_in[p] < 64 || d->k_in[p] % 64)
       return fail(HSNF4_ERR_INVALID, "%s: projection %d has invalid shape %lld x %lld", fn, p,
@@ -53,17 +63,15 @@ int check_layer(const char* fn, const hsnf4_layer_desc* d) {
 
 size_t layer_bytes(const hsnf4_layer_desc& d) {
   size_t b = 0;
-  for (int p = 0; p < d.n_proj; ++p)
-    b += round_up(proj_codes_bytes(d, p), kAlign) + round_up(proj_absmax_bytes(d, p), kAlign);
+  for (int p = 0; p < d.n_proj; ++p) b += proj_bytes(d, p);
   return b;
 }
 
 void layer_offsets(const hsnf4_layer_desc& d, int proj, size_t* co, size_t* ao) {
   size_t off = 0;
-  for (int p = 0; p < proj; ++p)
-    off += round_up(proj_codes_bytes(d, p), kAlign) + round_up(proj_absmax_bytes(d, p), kAlign);
+  for (int p = 0; p < proj; ++p) off += proj_bytes(d, p);
   *co = off;
-  *ao = off + round_up(proj_codes_bytes(d, proj), kAlign);
+  *ao = (d.base_format == HSNF4_BASE_BF16) ? off : off + round_up(proj_codes_bytes(d, proj), kAlign);
 }
 
 enum SlotState { kEmpty = 0, kLoaded = 1, kAcquired = 2, kReleased = 3 };
@@ -416,9 +424,13 @@ int stream_block_acquire(hsnf4_streamer* s, int block, void* compute_stream,
       size_t co, ao;
       layer_offsets(d, p, &co, &ao);
       out[k].codes = base + lo + co;
-      out[k].absmax = reinterpret_cast<const float*>(base + lo + ao);
+      out[k].absmax = (d.base_format == HSNF4_BASE_BF16)
+                          ? nullptr
+                          : reinterpret_cast<const float*>(base + lo + ao);
       out[k].n_out = d.n_out[p];
       out[k].k_in = d.k_in[p];
+      out[k].format = d.base_format;
+      out[k].reserved = 0;
       ++k;
     }
   }

@@ -19,10 +19,12 @@ LIB_PATH = os.path.join(_HERE, "libhsnf4.so")
 MAX_PROJ = 8
 
 OK, ERR_INVALID, ERR_OOM, ERR_CUDA, ERR_TIMEOUT, ERR_STATE, ERR_DEVICE = range(7)
+BASE_NF4, BASE_BF16 = 0, 1  # formats of the frozen base weight
 
 
 class Nf4WeightC(Structure):
-    _fields_ = [("codes", c_void_p), ("absmax", c_void_p), ("n_out", c_int64), ("k_in", c_int64)]
+    _fields_ = [("codes", c_void_p), ("absmax", c_void_p), ("n_out", c_int64), ("k_in", c_int64),
+                ("format", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class FwdArgs(Structure):
@@ -37,7 +39,8 @@ class BwdArgs(Structure):
 
 
 class LayerDesc(Structure):
-    _fields_ = [("n_proj", c_int), ("n_out", c_int64 * MAX_PROJ), ("k_in", c_int64 * MAX_PROJ)]
+    _fields_ = [("n_proj", c_int), ("n_out", c_int64 * MAX_PROJ), ("k_in", c_int64 * MAX_PROJ),
+                ("base_format", c_int)]
 
 
 class StreamConfig(Structure):
@@ -71,10 +74,13 @@ _SIGS = {
     "hsnf4_inject_fault": ([c_char_p], c_int),
     "hsnf4_selftest_stall": ([c_void_p], c_int),
     "hsnf4_profile": ([c_int], c_int),
+    "hsnf4_kernel_launches": ([], c_uint64),
     "hsnf4_profile_read": ([POINTER(KernelTime), c_int], c_int),
     "nf4_codebook": ([POINTER(c_float)], c_int),
     "nf4_quantize_pack": ([c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p], c_int),
     "nf4_dequant": ([c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p], c_int),
+    "lora_merge": ([POINTER(Nf4WeightC), c_void_p, c_void_p, c_int, c_float, c_void_p, c_void_p],
+                   c_int),
     "lora_linear_fwd_workspace": ([c_int64, c_int64, c_int64, c_int], c_size_t),
     "lora_linear_bwd_workspace": ([c_int64, c_int64, c_int64, c_int], c_size_t),
     "lora_linear_fwd": ([POINTER(Nf4WeightC), c_void_p, c_int64, c_void_p, c_void_p, c_int, c_float,
@@ -168,6 +174,11 @@ def device_status(stream=None) -> int:
     return int(flags.value)
 
 
+def kernel_launches() -> int:
+    """Kernels this library has launched in this process so far."""
+    return int(lib().hsnf4_kernel_launches())
+
+
 def profile(enable: bool):
     _check(lib().hsnf4_profile(int(bool(enable))))
 
@@ -207,7 +218,27 @@ class Nf4Weight:
     k_in: int
 
     def c(self) -> Nf4WeightC:
-        return Nf4WeightC(self.codes.data_ptr(), self.absmax.data_ptr(), self.n_out, self.k_in)
+        return Nf4WeightC(self.codes.data_ptr(), self.absmax.data_ptr(), self.n_out, self.k_in,
+                          BASE_NF4, 0)
+
+
+@dataclass
+class Bf16Weight:
+    """A dense bf16 base weight [n_out, k_in] in device memory (the
+    quantization="bf16_bitwise" base: streamed, never dequantized)."""
+    w: torch.Tensor
+
+    @property
+    def n_out(self) -> int:
+        return self.w.shape[0]
+
+    @property
+    def k_in(self) -> int:
+        return self.w.shape[1]
+
+    def c(self) -> Nf4WeightC:
+        _need(self.w, "w", torch.bfloat16)
+        return Nf4WeightC(self.w.data_ptr(), None, self.n_out, self.k_in, BASE_BF16, 0)
 
 
 def nf4_quantize_pack(w: torch.Tensor, codes=None, absmax=None, stream=None) -> Nf4Weight:
@@ -229,6 +260,17 @@ def nf4_dequant(W: Nf4Weight, out=None, stream=None) -> torch.Tensor:
     return out
 
 
+def lora_merge(W, A: torch.Tensor, B: torch.Tensor, alpha: float, out=None, stream=None):
+    """W' = deq(W) + (alpha/r) B A as a bf16 [n_out, k_in] tensor (merge_and_unload)."""
+    r = A.shape[0]
+    dev = A.device
+    if out is None:
+        out = torch.empty(W.n_out, W.k_in, dtype=torch.bfloat16, device=dev)
+    _check(lib().lora_merge(_weight_arg(W), _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
+                            _stream(stream)))
+    return out
+
+
 # ------------------------------------------------------------------ LoRA linear
 
 def fwd_workspace_bytes(T, n_out, k_in, r) -> int:
@@ -240,7 +282,7 @@ def bwd_workspace_bytes(T, n_out, k_in, r) -> int:
 
 
 def _weight_arg(W):
-    return ctypes.byref(W.c() if isinstance(W, Nf4Weight) else W)
+    return ctypes.byref(_wc(W))
 
 
 def lora_linear_fwd(W, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
@@ -299,7 +341,7 @@ def lora_linear_bwd(W, X, t_save, A, B, dY, alpha: float, dX=None, dA=None, dB=N
 
 
 def _wc(W):
-    return W.c() if isinstance(W, Nf4Weight) else W
+    return W.c() if isinstance(W, (Nf4Weight, Bf16Weight)) else W
 
 
 def _p(t):
@@ -340,10 +382,12 @@ def lora_group_bwd(args, T: int, r: int, alpha: float, workspace: torch.Tensor, 
 
 # ------------------------------------------------------------------ streamer
 
-def layer_desc(shapes) -> LayerDesc:
-    """shapes: [(n_out, k_in), ...] of one layer's projections."""
+def layer_desc(shapes, base_format: int = 0) -> LayerDesc:
+    """shapes: [(n_out, k_in), ...] of one layer's projections; base_format
+    BASE_NF4 (codes + absmax) or BASE_BF16 (dense bf16 weights)."""
     d = LayerDesc()
     d.n_proj = len(shapes)
+    d.base_format = base_format
     for i, (n, k) in enumerate(shapes):
         d.n_out[i] = n
         d.k_in[i] = k

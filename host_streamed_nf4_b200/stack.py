@@ -1,5 +1,9 @@
 """A stack of NF4 LoRA layers driven through the C ABI, streamed or resident.
 
+base="bf16" holds the frozen base as dense bf16 instead (the
+quantization="bf16_bitwise" base of the Poros API reference: 3.56x the
+bytes per weight, the same ring, no dequantization).
+
 Each layer has the 7 LoRA-targeted projections of its model family.  The
 frozen NF4 base of the whole stack lives in one pinned host slab (quantized
 on the GPU, layer by layer, and copied down -- the bounded-residency load
@@ -55,7 +59,8 @@ class LayerStack:
     def __init__(self, family: synth.Family, n_layers: int, T: int, *, block_size: int = 4,
                  streamed: bool = True, reuse_resident: bool = True, enable_prefetch: bool = True,
                  poison_on_release: bool = False, r: int = synth.RANK, alpha: float = synth.ALPHA,
-                 seed: int = 42, device=None, grouping: str = "layer", n_slots: int = 2):
+                 seed: int = 42, device=None, grouping: str = "layer", n_slots: int = 2,
+                 base: str = "nf4"):
         self.device = torch.device(device) if device is not None else torch.device(
             "cuda", torch.cuda.current_device())
         dev = self.device
@@ -64,7 +69,11 @@ class LayerStack:
         self.projs = family.projections()
         self.P = len(self.projs)
         self.groups = GROUPINGS[grouping]
-        self.desc = hsnf4.layer_desc([(n, k) for _, n, k in self.projs])
+        if base not in ("nf4", "bf16"):
+            raise ValueError(f"base must be 'nf4' or 'bf16' (got {base!r})")
+        self.base = base
+        self.base_format = hsnf4.BASE_BF16 if base == "bf16" else hsnf4.BASE_NF4
+        self.desc = hsnf4.layer_desc([(n, k) for _, n, k in self.projs], self.base_format)
         self.descs = [self.desc] * n_layers
         self.layer_bytes = hsnf4.layer_bytes(self.desc)
         self.offs = [hsnf4.layer_offsets(self.desc, p) for p in range(self.P)]
@@ -139,8 +148,12 @@ class LayerStack:
             base = l * self.layer_bytes
             for p, (_, n, k) in enumerate(self.projs):
                 w = _randn_bf16((n, k), synth.W_STD, _gen(dev, seed, l, p), dev)
-                W = hsnf4.nf4_quantize_pack(w)
                 co, ao = self.offs[p]
+                if self.base_format == hsnf4.BASE_BF16:
+                    self.slab[base + co: base + co + n * k * 2].copy_(w.view(torch.uint8).flatten())
+                    del w
+                    continue
+                W = hsnf4.nf4_quantize_pack(w)
                 self.slab[base + co: base + co + n * k // 2].copy_(W.codes)
                 self.slab[base + ao: base + ao + n * k // 16].view(torch.float32).copy_(W.absmax)
                 del w, W
@@ -152,8 +165,13 @@ class LayerStack:
         out = []
         for p, (_, n, k) in enumerate(self.projs):
             co, ao = self.offs[p]
-            out.append(hsnf4.Nf4WeightC(self.dev_slab.data_ptr() + base + co,
-                                        self.dev_slab.data_ptr() + base + ao, n, k))
+            if self.base_format == hsnf4.BASE_BF16:
+                out.append(hsnf4.Nf4WeightC(self.dev_slab.data_ptr() + base + co, None, n, k,
+                                            hsnf4.BASE_BF16, 0))
+            else:
+                out.append(hsnf4.Nf4WeightC(self.dev_slab.data_ptr() + base + co,
+                                            self.dev_slab.data_ptr() + base + ao, n, k,
+                                            hsnf4.BASE_NF4, 0))
         return out
 
     def block_layers(self, b: int):

@@ -73,11 +73,24 @@ typedef enum {
   HSNF4_ERR_DEVICE = 6   /* a kernel recorded a failed (timed-out) wait */
 } hsnf4_status;
 
-/* One NF4 weight as the kernels consume it (device pointers). */
+/* Formats of the frozen base weight (Poros API reference, the
+ * `quantization` knob: "nf4", the default, and "bf16_bitwise", the dense
+ * 16-bit base that still streams and keeps bitwise resident parity). */
+#define HSNF4_BASE_NF4 0  /* codes + absmax, 0.5625 bytes per weight */
+#define HSNF4_BASE_BF16 1 /* dense bf16, 2 bytes per weight */
+
+/* One frozen base weight as the kernels consume it (device pointers).
+ * format HSNF4_BASE_NF4 (0, what a zero-initialised struct holds): codes
+ * and absmax as below.  format HSNF4_BASE_BF16: codes points to the dense
+ * bf16 [n_out, k_in] row-major weight and absmax must be NULL.  Every LoRA
+ * entry point takes either format; a group call takes one format for all
+ * its problems. */
 typedef struct {
-  const void *codes;    /* uint8 [n_out*k_in/2] */
-  const float *absmax;  /* fp32 [n_out*k_in/64] */
+  const void *codes;    /* NF4: uint8 [n_out*k_in/2]; BF16: bf16 [n_out, k_in] */
+  const float *absmax;  /* NF4: fp32 [n_out*k_in/64]; BF16: NULL */
   int64_t n_out, k_in;
+  int32_t format;       /* HSNF4_BASE_NF4 or HSNF4_BASE_BF16 */
+  int32_t reserved;     /* 0 */
 } hsnf4_nf4_weight;
 
 /* ----------------------------------------------------------------------- */
@@ -121,6 +134,12 @@ typedef struct {
 int hsnf4_profile(int enable);
 int hsnf4_profile_read(hsnf4_kernel_time *out, int max_out);
 
+/* Number of kernels this library has launched in this process (every
+ * entry point counts each launch it makes, on any device or stream).  Read
+ * it before and after a region to count the region's launches.  No counterpart
+ * in the paper; a measurement aid. */
+uint64_t hsnf4_kernel_launches(void);
+
 /* Host-side fault injection for failure-path tests: the next call that
  * reaches `site` fails with HSNF4_ERR_CUDA without calling CUDA.  Sites:
  * "copy_enqueue" (the streamer's H2D copy), "event_record" (streamer event
@@ -151,6 +170,16 @@ int nf4_quantize_pack(const void *w_bf16, int64_t n_out, int64_t k_in,
  * absmax[e/64])), bit-exact by construction.  Same errors as above. */
 int nf4_dequant(const void *codes, const float *absmax, int64_t n_out,
                 int64_t k_in, void *w_bf16_out, void *stream);
+
+/* Merge the adapter into the base (Poros API reference,
+ * PorosModel.merge_and_unload): W' = deq(W) + s B A, s = alpha / r, each
+ * element computed in fp32 (the rank-r sum on the tensor cores, then
+ * scaled, added to the bf16 value of deq(W)) and rounded once to bf16.
+ * W: NF4 or BF16 base [n_out, k_in]; A bf16 [r, k_in]; B bf16 [n_out, r];
+ * W_out bf16 [n_out, k_in] (may not alias the inputs).  Rank limits as for
+ * the LoRA linear below.  Errors: INVALID (sizes, rank, pointers). */
+int lora_merge(const hsnf4_nf4_weight *W, const void *A, const void *B, int r,
+               float alpha, void *W_out, void *stream);
 
 /* ----------------------------------------------------------------------- */
 /* LoRA linear forward / backward (north of the ring: weights may live in  */
@@ -269,8 +298,8 @@ int lora_group_bwd(const hsnf4_lora_bwd_args *probs, int n, int64_t T, int r, fl
  *
  * Layout: a stack is n_layers layers; layer l has n_proj projections.  The
  * pinned slab holds the layers back to back; inside a layer, projection p's
- * codes then its absmax, each starting on a 1 KiB boundary
- * (stream_layer_offsets).  A block is block_size consecutive layers (the
+ * codes then its absmax (or its dense bf16 weight), each starting on a
+ * 1 KiB boundary (stream_layer_offsets).  A block is block_size consecutive layers (the
  * last block may be shorter) and is one contiguous byte range of the slab.
  * The ring holds n_slots (default 2) block slots in caller-provided device
  * memory.
@@ -291,6 +320,10 @@ typedef struct {
   int n_proj;
   int64_t n_out[HSNF4_MAX_PROJ];
   int64_t k_in[HSNF4_MAX_PROJ];
+  int base_format;  /* HSNF4_BASE_NF4 (0) or HSNF4_BASE_BF16, for every
+                       projection of the layer: with BF16 a projection's
+                       slab range is its bf16 [n_out, k_in] weight (1 KiB
+                       aligned) and acquire returns it with format BF16 */
 } hsnf4_layer_desc;
 
 typedef struct {
@@ -318,7 +351,8 @@ typedef struct hsnf4_streamer hsnf4_streamer;
 /* Bytes of one layer in the slab (multiple of 1 KiB). */
 int stream_layer_bytes(const hsnf4_layer_desc *layer, size_t *out_bytes);
 
-/* Byte offsets of projection p's codes and absmax inside its layer. */
+/* Byte offsets of projection p's codes and absmax inside its layer (for a
+ * BF16 layer: the weight's offset, twice). */
 int stream_layer_offsets(const hsnf4_layer_desc *layer, int proj,
                          size_t *codes_off, size_t *absmax_off);
 

@@ -71,7 +71,14 @@ def lib():
                                    ctypes.c_float, i64p, i64, f32p, f32p, i32]
         L.orc_lora_bwd.argtypes = [u8p, f32p, i64, i64, u16p, i64, u16p, u16p, i32,
                                    ctypes.c_float, u16p, i64p, i64, f32p, f32p, f32p, i32]
-        for fn in ("orc_nf4_quantize", "orc_nf4_dequant", "orc_lora_fwd", "orc_lora_bwd"):
+        L.orc_lora_fwd_bf16w.argtypes = [u16p, i64, i64, u16p, i64, u16p, u16p, i32,
+                                         ctypes.c_float, i64p, i64, f32p, f32p, i32]
+        L.orc_lora_bwd_bf16w.argtypes = [u16p, i64, i64, u16p, i64, u16p, u16p, i32,
+                                         ctypes.c_float, u16p, i64p, i64, f32p, f32p, f32p, i32]
+        L.orc_lora_merge.argtypes = [u8p, f32p, u16p, i64, i64, u16p, u16p, i32,
+                                     ctypes.c_float, u16p]
+        for fn in ("orc_nf4_quantize", "orc_nf4_dequant", "orc_lora_fwd", "orc_lora_bwd",
+                   "orc_lora_fwd_bf16w", "orc_lora_bwd_bf16w", "orc_lora_merge"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -207,3 +214,62 @@ def lora_bwd(codes, absmax, N, K, X, A, B, dY, alpha, rows=None, n_threads=None)
     if rc != 0:
         raise ValueError("orc_lora_bwd rejected its arguments")
     return dX, dA, dB
+
+
+def lora_fwd_bf16w(W, X, A, B, alpha, rows=None, n_threads=None):
+    """Forward with a dense bf16 base W (uint16 bits [N, K]).  Returns (Y, t) as lora_fwd."""
+    W, X, A, B = (_c(a, np.uint16) for a in (W, X, A, B))
+    N, K = W.shape
+    T, r = X.shape[0], A.shape[0]
+    if rows is not None:
+        rows = _c(np.asarray(rows, np.int64), np.int64)
+    nr = T if rows is None else rows.shape[0]
+    Y = np.zeros((nr, N), np.float32)
+    t = np.zeros((T, r), np.float32)
+    u16 = ctypes.c_uint16
+    rc = lib().orc_lora_fwd_bf16w(_p(W, u16), N, K, _p(X, u16), T, _p(A, u16), _p(B, u16), r,
+                                  float(alpha), _p(rows, ctypes.c_int64), nr,
+                                  _p(Y, ctypes.c_float), _p(t, ctypes.c_float),
+                                  n_threads or default_threads())
+    if rc != 0:
+        raise ValueError("orc_lora_fwd_bf16w rejected its arguments")
+    return Y, t
+
+
+def lora_bwd_bf16w(W, X, A, B, dY, alpha, rows=None, n_threads=None):
+    """Backward with a dense bf16 base W.  Returns (dX, dA, dB) as lora_bwd."""
+    W, X, A, B, dY = (_c(a, np.uint16) for a in (W, X, A, B, dY))
+    N, K = W.shape
+    T, r = X.shape[0], A.shape[0]
+    if rows is not None:
+        rows = _c(np.asarray(rows, np.int64), np.int64)
+    nr = T if rows is None else rows.shape[0]
+    dX = np.zeros((nr, K), np.float32)
+    dA = np.zeros((r, K), np.float32)
+    dB = np.zeros((N, r), np.float32)
+    u16, f = ctypes.c_uint16, ctypes.c_float
+    rc = lib().orc_lora_bwd_bf16w(_p(W, u16), N, K, _p(X, u16), T, _p(A, u16), _p(B, u16), r,
+                                  float(alpha), _p(dY, u16), _p(rows, ctypes.c_int64), nr,
+                                  _p(dX, f), _p(dA, f), _p(dB, f), n_threads or default_threads())
+    if rc != 0:
+        raise ValueError("orc_lora_bwd_bf16w rejected its arguments")
+    return dX, dA, dB
+
+
+def lora_merge(A, B, alpha, codes=None, absmax=None, W=None, N=None, K=None):
+    """merge_and_unload: bf16 bits [N, K] of deq(W) + (alpha/r) B A, one rounding.
+    The base is NF4 (codes, absmax, N, K) or dense bf16 (W bits [N, K])."""
+    A, B = _c(A, np.uint16), _c(B, np.uint16)
+    r = A.shape[0]
+    if W is not None:
+        W = _c(W, np.uint16)
+        N, K = W.shape
+    else:
+        codes, absmax = _c(codes, np.uint8), _c(absmax, np.float32)
+    out = np.zeros((N, K), np.uint16)
+    rc = lib().orc_lora_merge(_p(codes, ctypes.c_uint8), _p(absmax, ctypes.c_float),
+                              _p(W, ctypes.c_uint16), N, K, _p(A, ctypes.c_uint16),
+                              _p(B, ctypes.c_uint16), r, float(alpha), _p(out, ctypes.c_uint16))
+    if rc != 0:
+        raise ValueError("orc_lora_merge rejected its arguments")
+    return out

@@ -231,7 +231,8 @@ static void parallel_for(int64_t n, int n_threads, range_fn fn, void *ctx) {
 
 /* A source of rows of W, as doubles, for columns [k0, k1). */
 typedef struct {
-  const double *dense; /* [N,K] or NULL */
+  const double *dense;   /* [N,K] or NULL */
+  const uint16_t *wbf16; /* [N,K] bf16 bit patterns or NULL */
   const uint8_t *codes;
   const float *absmax;
   float cb[16];
@@ -242,6 +243,11 @@ static void w_row(const wsrc *w, int64_t n, int64_t k0, int64_t k1,
                   double *out) {
   if (w->dense) {
     for (int64_t k = k0; k < k1; ++k) out[k - k0] = w->dense[n * w->K + k];
+    return;
+  }
+  if (w->wbf16) {
+    for (int64_t k = k0; k < k1; ++k)
+      out[k - k0] = (double)orc_bf16_to_f32(w->wbf16[n * w->K + k]);
     return;
   }
   for (int64_t k = k0; k < k1; ++k) {
@@ -426,19 +432,14 @@ static int lora_args_ok(int64_t N, int64_t K, int64_t T, int r,
   return 1;
 }
 
-int orc_lora_fwd(const uint8_t *codes, const float *absmax, int64_t N,
-                 int64_t K, const uint16_t *X, int64_t T, const uint16_t *A,
-                 const uint16_t *B, int r, float alpha, const int64_t *rows,
-                 int64_t n_rows, float *Y, float *t_out, int n_threads) {
+static int lora_fwd_src(const wsrc *wp, int64_t N, int64_t K, const uint16_t *X,
+                        int64_t T, const uint16_t *A, const uint16_t *B, int r,
+                        float alpha, const int64_t *rows, int64_t n_rows, float *Y,
+                        float *t_out, int n_threads) {
   if (!lora_args_ok(N, K, T, r, rows, n_rows)) return -1;
   if (!rows) n_rows = T;
   const double s = (double)alpha / (double)r;
-  wsrc w;
-  memset(&w, 0, sizeof w);
-  w.codes = codes;
-  w.absmax = absmax;
-  w.K = K;
-  orc_nf4_codebook(w.cb);
+  const wsrc w = *wp;
 
   double *Xd = widen_bf16(X, T * K);
   double *Ad = widen_bf16(A, (int64_t)r * K);
@@ -473,20 +474,15 @@ done:
   return rc;
 }
 
-int orc_lora_bwd(const uint8_t *codes, const float *absmax, int64_t N,
-                 int64_t K, const uint16_t *X, int64_t T, const uint16_t *A,
-                 const uint16_t *B, int r, float alpha, const uint16_t *dY,
-                 const int64_t *rows, int64_t n_rows, float *dX, float *dA,
-                 float *dB, int n_threads) {
+static int lora_bwd_src(const wsrc *wp, int64_t N, int64_t K, const uint16_t *X,
+                        int64_t T, const uint16_t *A, const uint16_t *B, int r,
+                        float alpha, const uint16_t *dY, const int64_t *rows,
+                        int64_t n_rows, float *dX, float *dA, float *dB,
+                        int n_threads) {
   if (!lora_args_ok(N, K, T, r, rows, n_rows)) return -1;
   if (!rows) n_rows = T;
   const double s = (double)alpha / (double)r;
-  wsrc w;
-  memset(&w, 0, sizeof w);
-  w.codes = codes;
-  w.absmax = absmax;
-  w.K = K;
-  orc_nf4_codebook(w.cb);
+  const wsrc w = *wp;
 
   double *Xd = widen_bf16(X, T * K);
   double *Ad = widen_bf16(A, (int64_t)r * K);
@@ -529,4 +525,103 @@ done:
   free(dYs);
   free(us);
   return rc;
+}
+
+static wsrc nf4_src(const uint8_t *codes, const float *absmax, int64_t K) {
+  wsrc w;
+  memset(&w, 0, sizeof w);
+  w.codes = codes;
+  w.absmax = absmax;
+  w.K = K;
+  orc_nf4_codebook(w.cb);
+  return w;
+}
+
+static wsrc bf16_src(const uint16_t *W, int64_t K) {
+  wsrc w;
+  memset(&w, 0, sizeof w);
+  w.wbf16 = W;
+  w.K = K;
+  return w;
+}
+
+int orc_lora_fwd(const uint8_t *codes, const float *absmax, int64_t N,
+                 int64_t K, const uint16_t *X, int64_t T, const uint16_t *A,
+                 const uint16_t *B, int r, float alpha, const int64_t *rows,
+                 int64_t n_rows, float *Y, float *t_out, int n_threads) {
+  const wsrc w = nf4_src(codes, absmax, K);
+  return lora_fwd_src(&w, N, K, X, T, A, B, r, alpha, rows, n_rows, Y, t_out, n_threads);
+}
+
+int orc_lora_bwd(const uint8_t *codes, const float *absmax, int64_t N,
+                 int64_t K, const uint16_t *X, int64_t T, const uint16_t *A,
+                 const uint16_t *B, int r, float alpha, const uint16_t *dY,
+                 const int64_t *rows, int64_t n_rows, float *dX, float *dA,
+                 float *dB, int n_threads) {
+  const wsrc w = nf4_src(codes, absmax, K);
+  return lora_bwd_src(&w, N, K, X, T, A, B, r, alpha, dY, rows, n_rows, dX, dA, dB,
+                      n_threads);
+}
+
+int orc_lora_fwd_bf16w(const uint16_t *W, int64_t N, int64_t K, const uint16_t *X,
+                       int64_t T, const uint16_t *A, const uint16_t *B, int r,
+                       float alpha, const int64_t *rows, int64_t n_rows, float *Y,
+                       float *t_out, int n_threads) {
+  const wsrc w = bf16_src(W, K);
+  return lora_fwd_src(&w, N, K, X, T, A, B, r, alpha, rows, n_rows, Y, t_out, n_threads);
+}
+
+int orc_lora_bwd_bf16w(const uint16_t *W, int64_t N, int64_t K, const uint16_t *X,
+                       int64_t T, const uint16_t *A, const uint16_t *B, int r,
+                       float alpha, const uint16_t *dY, const int64_t *rows,
+                       int64_t n_rows, float *dX, float *dA, float *dB, int n_threads) {
+  const wsrc w = bf16_src(W, K);
+  return lora_bwd_src(&w, N, K, X, T, A, B, r, alpha, dY, rows, n_rows, dX, dA, dB,
+                      n_threads);
+}
+
+/* ---- merge_and_unload (Poros API reference, PorosModel.merge_and_unload):
+ * the adapter folded into the base, W' = deq(W) + (alpha/r) B A, in the
+ * compute dtype bf16.  Each element: the exact bf16 value of the base plus
+ * the rank-r sum accumulated in double, rounded ONCE to bf16 (nearest,
+ * ties to even). ---- */
+
+/* double -> bf16, one rounding (nearest, ties to even).  A double that is
+ * not a float first goes to the float of the same sign nearer to zero
+ * (truncation), with the discarded part recorded as a sticky bit in the
+ * float's last place, so that the float -> bf16 rounding below sees a tie
+ * only for values exactly halfway between two bf16 numbers. */
+static uint16_t bf16_from_double(double v) {
+  if (v != v) return 0x7FC0u;
+  float f = (float)v;
+  if ((double)f != v && isfinite(f)) {
+    /* truncate toward zero, then set the sticky bit */
+    if (fabs((double)f) > fabs(v)) f = nextafterf(f, 0.0f);
+    uint32_t b;
+    memcpy(&b, &f, sizeof b);
+    b |= 1u;
+    memcpy(&f, &b, sizeof b);
+  }
+  return orc_f32_to_bf16(f);
+}
+
+int orc_lora_merge(const uint8_t *codes, const float *absmax, const uint16_t *Wbf16,
+                   int64_t N, int64_t K, const uint16_t *A, const uint16_t *B, int r,
+                   float alpha, uint16_t *out) {
+  if (!shape_ok(N, K) || r <= 0 || (!Wbf16 && (!codes || !absmax))) return -1;
+  const double s = (double)alpha / (double)r;
+  wsrc w = Wbf16 ? bf16_src(Wbf16, K) : nf4_src(codes, absmax, K);
+  double *row = (double *)malloc(sizeof(double) * (size_t)K);
+  if (!row) return -1;
+  for (int64_t n = 0; n < N; ++n) {
+    w_row(&w, n, 0, K, row);
+    for (int64_t k = 0; k < K; ++k) {
+      double acc = 0.0;
+      for (int j = 0; j < r; ++j)
+        acc += (double)orc_bf16_to_f32(B[n * r + j]) * (double)orc_bf16_to_f32(A[(int64_t)j * K + k]);
+      out[n * K + k] = bf16_from_double(row[k] + s * acc);
+    }
+  }
+  free(row);
+  return 0;
 }

@@ -97,6 +97,26 @@ int orc_lora_bwd(const uint8_t *codes, const float *absmax, int64_t N,
                  const int64_t *rows, int64_t n_rows, float *dX, float *dA,
                  float *dB, int n_threads);
 
+/* The same forward / backward with a dense bf16 base W [N,K] (bf16 bit
+ * patterns) in place of NF4 -- the quantization="bf16_bitwise" base of the
+ * Poros API reference.  Same conventions and returns as above. */
+int orc_lora_fwd_bf16w(const uint16_t *W, int64_t N, int64_t K, const uint16_t *X,
+                       int64_t T, const uint16_t *A, const uint16_t *B, int r,
+                       float alpha, const int64_t *rows, int64_t n_rows, float *Y,
+                       float *t_out, int n_threads);
+int orc_lora_bwd_bf16w(const uint16_t *W, int64_t N, int64_t K, const uint16_t *X,
+                       int64_t T, const uint16_t *A, const uint16_t *B, int r,
+                       float alpha, const uint16_t *dY, const int64_t *rows,
+                       int64_t n_rows, float *dX, float *dA, float *dB, int n_threads);
+
+/* merge_and_unload: out[n,k] = bf16_rne(deq(W)[n,k] + (alpha/r) sum_j B[n,j]
+ * A[j,k]), the sum in double, ONE rounding to bf16.  The base is NF4
+ * (codes, absmax; Wbf16 NULL) or dense bf16 (Wbf16 [N,K]; codes, absmax
+ * ignored).  A bf16 [r,K], B bf16 [N,r], out bf16 [N,K].  0 or -1. */
+int orc_lora_merge(const uint8_t *codes, const float *absmax, const uint16_t *Wbf16,
+                   int64_t N, int64_t K, const uint16_t *A, const uint16_t *B, int r,
+                   float alpha, uint16_t *out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -16,7 +16,7 @@ HEADER = os.path.join(ROOT, "include", "hsnf4.h")
 def _declared():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char)\s*\**\s*([a-z0-9_]+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char|uint64_t)\s*\**\s*([a-z0-9_]+)\s*\(",
                                  src, flags=re.M)))
 
 
@@ -129,3 +129,65 @@ def test_host_fault_injection_sites():
     hsnf4.inject_fault(None)
     with pytest.raises(hsnf4.HsNf4Error):
         hsnf4.inject_fault("kernel_trap")
+
+
+# ---------------------------------------------------------------- dense bf16 base, merge
+
+def test_base_format_validation_before_cuda():
+    import ctypes
+    L = hsnf4.lib()
+    fake = 0x10000
+    call = lambda W: L.lora_linear_fwd(ctypes.byref(W), fake, 64, fake, fake, 16, 32.0, fake,
+                                       fake, fake, 1 << 20, None)
+    # a BF16 base takes absmax = NULL
+    assert call(hsnf4.Nf4WeightC(fake, fake, 128, 256, hsnf4.BASE_BF16, 0)) == hsnf4.ERR_INVALID
+    assert "absmax = NULL" in hsnf4.last_error()
+    # an NF4 base needs absmax
+    assert call(hsnf4.Nf4WeightC(fake, None, 128, 256, hsnf4.BASE_NF4, 0)) == hsnf4.ERR_INVALID
+    assert "absmax" in hsnf4.last_error()
+    # unknown format
+    assert call(hsnf4.Nf4WeightC(fake, fake, 128, 256, 7, 0)) == hsnf4.ERR_INVALID
+    assert "format" in hsnf4.last_error()
+    # one format per group
+    Wq = hsnf4.Nf4WeightC(fake, fake, 128, 256, hsnf4.BASE_NF4, 0)
+    Wd = hsnf4.Nf4WeightC(fake, None, 128, 256, hsnf4.BASE_BF16, 0)
+    arr = (hsnf4.FwdArgs * 2)(hsnf4.FwdArgs(Wq, fake, fake, fake, fake, None),
+                              hsnf4.FwdArgs(Wd, fake, fake, fake, fake, None))
+    assert L.lora_group_fwd(arr, 2, 64, 16, 32.0, fake, 1 << 30, None) == hsnf4.ERR_INVALID
+    assert "one format" in hsnf4.last_error()
+
+
+def test_merge_validates_before_cuda():
+    import ctypes
+    L = hsnf4.lib()
+    fake = 0x10000
+    W = hsnf4.Nf4WeightC(fake, fake, 128, 256, hsnf4.BASE_NF4, 0)
+    assert L.lora_merge(ctypes.byref(W), fake, fake, 4, 32.0, fake + 0x1000, None) == \
+        hsnf4.ERR_INVALID
+    assert "rank" in hsnf4.last_error()
+    assert L.lora_merge(ctypes.byref(W), fake, fake, 16, 32.0, fake, None) == hsnf4.ERR_INVALID
+    assert "aliases" in hsnf4.last_error()
+    assert L.lora_merge(ctypes.byref(W), fake, None, 16, 32.0, fake + 0x1000, None) == \
+        hsnf4.ERR_INVALID
+    Wbad = hsnf4.Nf4WeightC(fake, fake, 96, 256, hsnf4.BASE_NF4, 0)
+    assert L.lora_merge(ctypes.byref(Wbad), fake, fake, 16, 32.0, fake + 0x1000, None) == \
+        hsnf4.ERR_INVALID
+
+
+def test_bf16_layer_layout():
+    shapes = [(n, k) for _, n, k in synth.FAMILIES["qwen2.5-7b"].projections()]
+    d = hsnf4.layer_desc(shapes, hsnf4.BASE_BF16)
+    total = hsnf4.layer_bytes(d)
+    spans = []
+    for p, (n, k) in enumerate(shapes):
+        co, ao = hsnf4.layer_offsets(d, p)
+        assert co == ao and co % 1024 == 0
+        spans.append((co, co + n * k * 2))
+    assert spans[0][0] == 0 and all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+    payload = sum(2 * n * k for n, k in shapes)
+    assert payload <= total < payload + 7 * 1024
+    # 2 B per weight vs 0.5625 B: the pages' 3.56x
+    nf4 = hsnf4.layer_bytes(hsnf4.layer_desc(shapes))
+    assert abs(total / nf4 - 2 / 0.5625) < 1e-3
+    with pytest.raises(hsnf4.HsNf4Error):
+        hsnf4.layer_bytes(hsnf4.layer_desc(shapes, 2))

@@ -349,3 +349,104 @@ def test_bf16_wrapper_equals_fp32_rounding_of_double_core(orc):
     assert np.array_equal(dX, dXd.astype(np.float32))
     assert np.array_equal(dA, dAd.astype(np.float32))
     assert np.array_equal(dB, dBd.astype(np.float32))
+
+
+# ---------------------------------------------------------------- dense bf16 base
+
+def test_dense_base_equals_nf4_path_on_its_dequantized_weight(orc):
+    """The dense-bf16-base entry points on W = deq(codes) give exactly what the
+    (FD- and closed-form-pinned) NF4 entry points give on the codes."""
+    c = synth.linear_case(21, 6, 128, 192, r=8)
+    codes, absmax = orc.quantize(c.W)
+    Wd = orc.dequant(codes, absmax, 128, 192)
+    Y, t = orc.lora_fwd(codes, absmax, 128, 192, c.X, c.A, c.B, 16.0)
+    Yd, td = orc.lora_fwd_bf16w(Wd, c.X, c.A, c.B, 16.0)
+    assert np.array_equal(Y, Yd) and np.array_equal(t, td)
+    dX, dA, dB = orc.lora_bwd(codes, absmax, 128, 192, c.X, c.A, c.B, c.dY, 16.0)
+    dXd, dAd, dBd = orc.lora_bwd_bf16w(Wd, c.X, c.A, c.B, c.dY, 16.0)
+    assert np.array_equal(dX, dXd) and np.array_equal(dA, dAd) and np.array_equal(dB, dBd)
+
+
+def test_dense_base_reads_the_weight_not_a_quantized_copy(orc):
+    """A dense weight with values NF4 cannot hold (3/8, 5/8 of the absmax)
+    must come through exactly: W = diag(w_i), B = 0  =>  Y[:, i] = w_i X[:, i]."""
+    rng = np.random.default_rng(22)
+    T, N = 4, 64
+    w = np.where(np.arange(N) % 2 == 0, 0.375, 0.625).astype(np.float32)
+    W = np.diag(w)
+    X = synth.normal_bf16(rng, (T, N), 1.0)
+    A = synth.normal_bf16(rng, (8, N), 0.1)
+    Y, _ = orc.lora_fwd_bf16w(synth.to_bf16_bits(W), X, A, np.zeros((N, 8), np.uint16), 16.0)
+    ref = synth.bits_to_f32(X).astype(np.float64) * w[None, :]
+    assert np.array_equal(Y, ref.astype(np.float32))
+
+
+# ---------------------------------------------------------------- merge_and_unload
+
+def _bf16_of_fraction(q):
+    """Exact round-to-nearest-even of a rational to bf16 bits (normal range),
+    by integer arithmetic only -- independent of any float rounding."""
+    from fractions import Fraction
+    if q == 0:
+        return 0
+    sign = 0x8000 if q < 0 else 0
+    a = abs(Fraction(q))
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    m = a / Fraction(2) ** (e - 7)          # 128 <= m < 256
+    fl = m.numerator // m.denominator
+    rem = m - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    if fl == 256:
+        fl, e = 128, e + 1
+    return sign | ((e + 127) << 7) | (fl - 128)
+
+
+def test_merge_zero_adapter_is_dequant(orc):
+    c = synth.linear_case(23, 1, 128, 256, r=16)
+    codes, absmax = orc.quantize(c.W)
+    out = orc.lora_merge(c.A, np.zeros_like(c.B), 32.0, codes=codes, absmax=absmax, N=128, K=256)
+    assert np.array_equal(out, orc.dequant(codes, absmax, 128, 256))
+    Wd = orc.dequant(codes, absmax, 128, 256)
+    assert np.array_equal(orc.lora_merge(c.A, np.zeros_like(c.B), 32.0, W=Wd), Wd)
+
+
+def test_merge_exact_rational_bruteforce(orc):
+    """Every element against exact rational arithmetic rounded once: catches a
+    transposed operand, a wrong scale, a missing base term or a double
+    rounding."""
+    from fractions import Fraction
+    rng = np.random.default_rng(24)
+    N, K, r, alpha = 64, 64, 8, 16.0
+    c = synth.linear_case(24, 1, N, K, r=r)
+    codes, absmax = orc.quantize(c.W)
+    deq = synth.bits_to_f32(orc.dequant(codes, absmax, N, K))
+    A = synth.normal_bf16(rng, (r, K), 0.5)
+    B = synth.normal_bf16(rng, (N, r), 0.5)
+    Af, Bf = synth.bits_to_f32(A), synth.bits_to_f32(B)
+    out = orc.lora_merge(A, B, alpha, codes=codes, absmax=absmax, N=N, K=K)
+    s = Fraction(alpha) / r
+    for n in range(N):
+        for k in range(K):
+            acc = sum(Fraction(float(Bf[n, j])) * Fraction(float(Af[j, k])) for j in range(r))
+            assert out[n, k] == _bf16_of_fraction(Fraction(float(deq[n, k])) + s * acc), (n, k)
+
+
+def test_merge_rounds_once_at_a_bf16_midpoint(orc):
+    """1 + 2^-8 is exactly halfway between bf16 1.0 and 1 + 2^-7: ties go to
+    even (1.0).  1 + 2^-8 + 2^-30 is above halfway: it must round up, which
+    a float32 intermediate (2^-30 lost) would get wrong."""
+    N, K, r = 64, 64, 8
+    W = np.full((N, K), 1.0, np.float32)
+    A = np.zeros((r, K), np.float32)
+    B = np.zeros((N, r), np.float32)
+    A[0, :] = 1.0
+    A[1, :] = 2.0 ** -24
+    B[:, 0] = 2.0 ** -8 / 2.0        # s = 16/8 = 2
+    B[: N // 2, 1] = 2.0 ** -7        # rows 0..31: + 2 * 2^-7 * 2^-24 = 2^-30
+    out = orc.lora_merge(synth.to_bf16_bits(A), synth.to_bf16_bits(B), 16.0,
+                         W=synth.to_bf16_bits(W))
+    assert np.all(out[N // 2:] == 0x3F80)   # tie -> even
+    assert np.all(out[: N // 2] == 0x3F81)  # just above the tie -> up
