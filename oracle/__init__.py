@@ -77,8 +77,24 @@ def lib():
                                          ctypes.c_float, u16p, i64p, i64, f32p, f32p, f32p, i32]
         L.orc_lora_merge.argtypes = [u8p, f32p, u16p, i64, i64, u16p, u16p, i32,
                                      ctypes.c_float, u16p]
+        u32p, u64 = ctypes.POINTER(ctypes.c_uint32), ctypes.c_uint64
+        L.orc_philox4x32_10.argtypes = [u32p, u32p, u32p]
+        L.orc_dropout_keep.argtypes = [u64, u64, ctypes.c_float, i64, i64, u8p]
+        L.orc_dropout_apply.argtypes = [u16p, i64, i64, u64, u64, ctypes.c_float, u16p]
+        L.orc_lora_fwd_f64m.argtypes = [f64p, f64p, f64p, f64p, f64p, i64, i64, i64, i32,
+                                        ctypes.c_double, f64p, f64p]
+        L.orc_lora_bwd_f64m.argtypes = [f64p, f64p, f64p, f64p, f64p, f64p, i64, i64, i64, i32,
+                                        ctypes.c_double, f64p, f64p, f64p]
+        L.orc_lora_fwd_drop.argtypes = [u8p, f32p, i64, i64, u16p, i64, u16p, u16p, i32,
+                                        ctypes.c_float, ctypes.c_float, u64, u64, i64p, i64,
+                                        f32p, f32p, i32]
+        L.orc_lora_bwd_drop.argtypes = [u8p, f32p, i64, i64, u16p, i64, u16p, u16p, i32,
+                                        ctypes.c_float, ctypes.c_float, u64, u64, u16p, i64p,
+                                        i64, f32p, f32p, f32p, i32]
         for fn in ("orc_nf4_quantize", "orc_nf4_dequant", "orc_lora_fwd", "orc_lora_bwd",
-                   "orc_lora_fwd_bf16w", "orc_lora_bwd_bf16w", "orc_lora_merge"):
+                   "orc_lora_fwd_bf16w", "orc_lora_bwd_bf16w", "orc_lora_merge",
+                   "orc_dropout_keep", "orc_dropout_apply", "orc_lora_fwd_drop",
+                   "orc_lora_bwd_drop"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -273,3 +289,100 @@ def lora_merge(A, B, alpha, codes=None, absmax=None, W=None, N=None, K=None):
     if rc != 0:
         raise ValueError("orc_lora_merge rejected its arguments")
     return out
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32-10 of a 4-word counter under a 2-word key -> 4 words."""
+    c = np.ascontiguousarray(ctr, np.uint32)
+    k = np.ascontiguousarray(key, np.uint32)
+    out = np.zeros(4, np.uint32)
+    lib().orc_philox4x32_10(_p(c, ctypes.c_uint32), _p(k, ctypes.c_uint32),
+                            _p(out, ctypes.c_uint32))
+    return out
+
+
+def dropout_keep(seed: int, offset: int, p: float, T: int, K: int) -> np.ndarray:
+    keep = np.zeros((T, K), np.uint8)
+    if lib().orc_dropout_keep(seed, offset, p, T, K, _p(keep, ctypes.c_uint8)) != 0:
+        raise ValueError("orc_dropout_keep rejected its arguments")
+    return keep
+
+
+def dropout_apply(X, seed: int, offset: int, p: float) -> np.ndarray:
+    X = _c(X, np.uint16)
+    T, K = X.shape
+    out = np.zeros((T, K), np.uint16)
+    if lib().orc_dropout_apply(_p(X, ctypes.c_uint16), T, K, seed, offset, p,
+                               _p(out, ctypes.c_uint16)) != 0:
+        raise ValueError("orc_dropout_apply rejected its arguments")
+    return out
+
+
+def lora_fwd_f64m(W, X, Xl, A, B, s):
+    W, X, Xl, A, B = (_c(np.asarray(a, np.float64), np.float64) for a in (W, X, Xl, A, B))
+    T, K = X.shape
+    N, r = W.shape[0], A.shape[0]
+    Y = np.zeros((T, N), np.float64)
+    t = np.zeros((T, r), np.float64)
+    f = ctypes.c_double
+    lib().orc_lora_fwd_f64m(_p(W, f), _p(X, f), _p(Xl, f), _p(A, f), _p(B, f), T, N, K, r,
+                            float(s), _p(Y, f), _p(t, f))
+    return Y, t
+
+
+def lora_bwd_f64m(W, Xl, g, A, B, dY, s):
+    W, Xl, A, B, dY = (_c(np.asarray(a, np.float64), np.float64) for a in (W, Xl, A, B, dY))
+    g = None if g is None else _c(np.asarray(g, np.float64), np.float64)
+    T, K = Xl.shape
+    N, r = W.shape[0], A.shape[0]
+    dX = np.zeros((T, K), np.float64)
+    dA = np.zeros((r, K), np.float64)
+    dB = np.zeros((N, r), np.float64)
+    f = ctypes.c_double
+    lib().orc_lora_bwd_f64m(_p(W, f), _p(Xl, f), _p(g, f), _p(A, f), _p(B, f), _p(dY, f), T, N,
+                            K, r, float(s), _p(dX, f), _p(dA, f), _p(dB, f))
+    return dX, dA, dB
+
+
+def lora_fwd_drop(codes, absmax, N, K, X, A, B, alpha, p, seed, offset, rows=None,
+                  n_threads=None):
+    """lora_fwd with dropout p under (seed, offset) on the adapter branch."""
+    codes, absmax = _c(codes, np.uint8), _c(absmax, np.float32)
+    X, A, B = _c(X, np.uint16), _c(A, np.uint16), _c(B, np.uint16)
+    T, r = X.shape[0], A.shape[0]
+    if rows is not None:
+        rows = _c(np.asarray(rows, np.int64), np.int64)
+    nr = T if rows is None else rows.shape[0]
+    Y = np.zeros((nr, N), np.float32)
+    t = np.zeros((T, r), np.float32)
+    u16 = ctypes.c_uint16
+    rc = lib().orc_lora_fwd_drop(_p(codes, ctypes.c_uint8), _p(absmax, ctypes.c_float), N, K,
+                                 _p(X, u16), T, _p(A, u16), _p(B, u16), r, float(alpha),
+                                 float(p), seed, offset, _p(rows, ctypes.c_int64), nr,
+                                 _p(Y, ctypes.c_float), _p(t, ctypes.c_float),
+                                 n_threads or default_threads())
+    if rc != 0:
+        raise ValueError("orc_lora_fwd_drop rejected its arguments")
+    return Y, t
+
+
+def lora_bwd_drop(codes, absmax, N, K, X, A, B, dY, alpha, p, seed, offset, rows=None,
+                  n_threads=None):
+    """lora_bwd with dropout p under (seed, offset) on the adapter branch."""
+    codes, absmax = _c(codes, np.uint8), _c(absmax, np.float32)
+    X, A, B, dY = (_c(a, np.uint16) for a in (X, A, B, dY))
+    T, r = X.shape[0], A.shape[0]
+    if rows is not None:
+        rows = _c(np.asarray(rows, np.int64), np.int64)
+    nr = T if rows is None else rows.shape[0]
+    dX = np.zeros((nr, K), np.float32)
+    dA = np.zeros((r, K), np.float32)
+    dB = np.zeros((N, r), np.float32)
+    u16, f = ctypes.c_uint16, ctypes.c_float
+    rc = lib().orc_lora_bwd_drop(_p(codes, ctypes.c_uint8), _p(absmax, f), N, K, _p(X, u16), T,
+                                 _p(A, u16), _p(B, u16), r, float(alpha), float(p), seed, offset,
+                                 _p(dY, u16), _p(rows, ctypes.c_int64), nr, _p(dX, f), _p(dA, f),
+                                 _p(dB, f), n_threads or default_threads())
+    if rc != 0:
+        raise ValueError("orc_lora_bwd_drop rejected its arguments")
+    return dX, dA, dB

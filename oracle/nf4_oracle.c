@@ -308,6 +308,7 @@ typedef struct {
   int r;
   double s;
   double *dX; /* [n_rows, K] */
+  const double *g; /* [n_rows, K] multiplier of the LoRA term (dropout), or NULL */
 } dx_ctx;
 
 static void dx_cols(void *p, int64_t lo, int64_t hi) {
@@ -333,6 +334,7 @@ static void dx_cols(void *p, int64_t lo, int64_t hi) {
     for (int64_t k = lo; k < hi; ++k) {
       double lora = 0.0;
       for (int j = 0; j < c->r; ++j) lora += c->u[i * c->r + j] * c->A[j * c->K + k];
+      if (c->g) lora *= c->g[i * c->K + k];
       c->dX[i * c->K + k] = acc[i * width + (k - lo)] + c->s * lora;
     }
   free(row);
@@ -371,11 +373,17 @@ static void lora_up_t(const double *dY, const double *B, int64_t T, int64_t N,
 void orc_lora_fwd_f64(const double *W, const double *X, const double *A,
                       const double *B, int64_t T, int64_t N, int64_t K, int r,
                       double s, double *Y, double *t) {
+  orc_lora_fwd_f64m(W, X, X, A, B, T, N, K, r, s, Y, t);
+}
+
+void orc_lora_fwd_f64m(const double *W, const double *X, const double *Xl,
+                       const double *A, const double *B, int64_t T, int64_t N,
+                       int64_t K, int r, double s, double *Y, double *t) {
   wsrc w;
   memset(&w, 0, sizeof w);
   w.dense = W;
   w.K = K;
-  lora_down(X, A, T, K, r, t);
+  lora_down(Xl, A, T, K, r, t);
   fwd_ctx c = {&w, X, t, B, T, N, K, r, s, Y};
   fwd_cols(&c, 0, N);
 }
@@ -384,6 +392,14 @@ void orc_lora_bwd_f64(const double *W, const double *X, const double *A,
                       const double *B, const double *dY, int64_t T, int64_t N,
                       int64_t K, int r, double s, double *dX, double *dA,
                       double *dB) {
+  orc_lora_bwd_f64m(W, X, NULL, A, B, dY, T, N, K, r, s, dX, dA, dB);
+}
+
+void orc_lora_bwd_f64m(const double *W, const double *Xl, const double *g,
+                       const double *A, const double *B, const double *dY,
+                       int64_t T, int64_t N, int64_t K, int r, double s,
+                       double *dX, double *dA, double *dB) {
+  const double *X = Xl;
   wsrc w;
   memset(&w, 0, sizeof w);
   w.dense = W;
@@ -397,11 +413,132 @@ void orc_lora_bwd_f64(const double *W, const double *X, const double *A,
   }
   lora_down(X, A, T, K, r, t);
   lora_up_t(dY, B, T, N, r, u);
-  dx_ctx c = {&w, dY, u, A, T, N, K, r, s, dX};
+  dx_ctx c = {&w, dY, u, A, T, N, K, r, s, dX, g};
   dx_cols(&c, 0, K);
   lora_grads(X, dY, t, u, T, N, K, r, s, dA, dB);
   free(t);
   free(u);
+}
+
+/* ---- counter-based RNG: Philox4x32-10 (Salmon, Moraes, Dror, Shaw,
+ * "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011), from its
+ * published definition: a 4 x 32-bit counter and a 2 x 32-bit key; each of
+ * 10 rounds multiplies counter words 0 and 2 by the two round multipliers
+ * (full 64-bit products split into high and low halves) and mixes the high
+ * halves with the other two words and the key; between rounds the key is
+ * bumped by the two Weyl constants. ---- */
+
+void orc_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2],
+                       uint32_t out[4]) {
+  uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+  uint32_t k0 = key_in[0], k1 = key_in[1];
+  for (int round = 0; round < 10; ++round) {
+    if (round > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+    const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+    const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  out[0] = c0;
+  out[1] = c1;
+  out[2] = c2;
+  out[3] = c3;
+}
+
+/* ---- LoRA dropout (Poros API reference: lora_dropout, default 0.05; the
+ * dropout sits on the adapter branch's input).  The mask of element e of a
+ * row-major [T,K] input (e = t*K + k) under (seed, offset):
+ *   q = e / 4;  w = Philox4x32-10(ctr = {lo(q), hi(q), lo(offset), hi(offset)},
+ *                                 key = {lo(seed), hi(seed)})[e % 4]
+ *   keep  <=>  (w >> 8) >= floor(p * 2^24)   (p * 2^24 formed in fp32)
+ * and the kept value is bf16_rne(fp32(x) * scale), scale = fp32(1 / fp32(1 - p)).
+ * The caller picks the offset per (step, layer, projection) so that the
+ * backward (and any recompute) draws the same mask. ---- */
+
+static uint32_t drop_threshold(float p) { return (uint32_t)(p * 16777216.0f); }
+
+static float drop_scale(float p) {
+  volatile float one_minus = 1.0f - p; /* fp32 rounding of each step */
+  return 1.0f / one_minus;
+}
+
+int orc_dropout_keep(uint64_t seed, uint64_t offset, float p, int64_t T, int64_t K,
+                     uint8_t *keep) {
+  if (T < 0 || K < 0 || !(p >= 0.0f && p < 1.0f)) return -1;
+  const uint32_t thr = drop_threshold(p);
+  const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  const int64_t n = T * K;
+  for (int64_t e = 0; e < n; ++e) {
+    const uint64_t q = (uint64_t)e >> 2;
+    const uint32_t ctr[4] = {(uint32_t)q, (uint32_t)(q >> 32), (uint32_t)offset,
+                             (uint32_t)(offset >> 32)};
+    uint32_t w[4];
+    orc_philox4x32_10(ctr, key, w);
+    keep[e] = (w[e & 3] >> 8) >= thr ? 1 : 0;
+  }
+  return 0;
+}
+
+int orc_dropout_apply(const uint16_t *X, int64_t T, int64_t K, uint64_t seed,
+                      uint64_t offset, float p, uint16_t *out) {
+  uint8_t *keep = (uint8_t *)malloc((size_t)(T * K > 0 ? T * K : 1));
+  if (!keep) return -1;
+  if (orc_dropout_keep(seed, offset, p, T, K, keep) != 0) {
+    free(keep);
+    return -1;
+  }
+  const float scale = drop_scale(p);
+  for (int64_t e = 0; e < T * K; ++e) {
+    volatile float v = orc_bf16_to_f32(X[e]) * scale;
+    out[e] = keep[e] ? orc_f32_to_bf16(v) : 0;
+  }
+  free(keep);
+  return 0;
+}
+
+/* dropout of one problem: NULL = none */
+typedef struct {
+  float p;
+  uint64_t seed, offset;
+} drop_cfg;
+
+/* the adapter branch's input (bf16 X_d, widened) and the dX multiplier
+ * keep * scale, or NULLs when there is no dropout */
+static int drop_inputs(const drop_cfg *d, const uint16_t *X, int64_t T, int64_t K,
+                       double **Xl, double **g) {
+  *Xl = NULL;
+  *g = NULL;
+  if (!d) return 0;
+  uint16_t *xd = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(T * K > 0 ? T * K : 1));
+  uint8_t *keep = (uint8_t *)malloc((size_t)(T * K > 0 ? T * K : 1));
+  *Xl = (double *)malloc(sizeof(double) * (size_t)(T * K > 0 ? T * K : 1));
+  *g = (double *)malloc(sizeof(double) * (size_t)(T * K > 0 ? T * K : 1));
+  int rc = -1;
+  if (xd && keep && *Xl && *g && orc_dropout_apply(X, T, K, d->seed, d->offset, d->p, xd) == 0 &&
+      orc_dropout_keep(d->seed, d->offset, d->p, T, K, keep) == 0) {
+    const double scale = (double)drop_scale(d->p);
+    for (int64_t e = 0; e < T * K; ++e) {
+      (*Xl)[e] = (double)orc_bf16_to_f32(xd[e]);
+      (*g)[e] = keep[e] ? scale : 0.0;
+    }
+    rc = 0;
+  }
+  free(xd);
+  free(keep);
+  if (rc) {
+    free(*Xl);
+    free(*g);
+    *Xl = *g = NULL;
+  }
+  return rc;
 }
 
 /* ---- the method's data types ---- */
@@ -432,14 +569,16 @@ static int lora_args_ok(int64_t N, int64_t K, int64_t T, int r,
   return 1;
 }
 
-static int lora_fwd_src(const wsrc *wp, int64_t N, int64_t K, const uint16_t *X,
-                        int64_t T, const uint16_t *A, const uint16_t *B, int r,
-                        float alpha, const int64_t *rows, int64_t n_rows, float *Y,
+static int lora_fwd_src(const wsrc *wp, const drop_cfg *drop, int64_t N, int64_t K,
+                        const uint16_t *X, int64_t T, const uint16_t *A, const uint16_t *B,
+                        int r, float alpha, const int64_t *rows, int64_t n_rows, float *Y,
                         float *t_out, int n_threads) {
   if (!lora_args_ok(N, K, T, r, rows, n_rows)) return -1;
   if (!rows) n_rows = T;
   const double s = (double)alpha / (double)r;
   const wsrc w = *wp;
+  double *Xl = NULL, *g = NULL; /* adapter-branch input after dropout */
+  if (drop_inputs(drop, X, T, K, &Xl, &g) != 0) return -1;
 
   double *Xd = widen_bf16(X, T * K);
   double *Ad = widen_bf16(A, (int64_t)r * K);
@@ -449,7 +588,7 @@ static int lora_fwd_src(const wsrc *wp, int64_t N, int64_t K, const uint16_t *X,
   double *Xs = NULL, *ts = NULL;
   int rc = -1;
   if (!Xd || !Ad || !Bd || !t || !Yd) goto done;
-  lora_down(Xd, Ad, T, K, r, t);
+  lora_down(Xl ? Xl : Xd, Ad, T, K, r, t);
   if (rows) {
     Xs = gather_rows(Xd, K, rows, n_rows);
     ts = gather_rows(t, r, rows, n_rows);
@@ -464,6 +603,8 @@ static int lora_fwd_src(const wsrc *wp, int64_t N, int64_t K, const uint16_t *X,
     for (int64_t i = 0; i < T * r; ++i) t_out[i] = (float)t[i];
   rc = 0;
 done:
+  free(Xl);
+  free(g);
   free(Xd);
   free(Ad);
   free(Bd);
@@ -474,15 +615,17 @@ done:
   return rc;
 }
 
-static int lora_bwd_src(const wsrc *wp, int64_t N, int64_t K, const uint16_t *X,
-                        int64_t T, const uint16_t *A, const uint16_t *B, int r,
-                        float alpha, const uint16_t *dY, const int64_t *rows,
+static int lora_bwd_src(const wsrc *wp, const drop_cfg *drop, int64_t N, int64_t K,
+                        const uint16_t *X, int64_t T, const uint16_t *A, const uint16_t *B,
+                        int r, float alpha, const uint16_t *dY, const int64_t *rows,
                         int64_t n_rows, float *dX, float *dA, float *dB,
                         int n_threads) {
   if (!lora_args_ok(N, K, T, r, rows, n_rows)) return -1;
   if (!rows) n_rows = T;
   const double s = (double)alpha / (double)r;
   const wsrc w = *wp;
+  double *Xl = NULL, *g = NULL, *gs = NULL; /* adapter-branch input, dX multiplier */
+  if (drop_inputs(drop, X, T, K, &Xl, &g) != 0) return -1;
 
   double *Xd = widen_bf16(X, T * K);
   double *Ad = widen_bf16(A, (int64_t)r * K);
@@ -496,23 +639,28 @@ static int lora_bwd_src(const wsrc *wp, int64_t N, int64_t K, const uint16_t *X,
   double *dYs = NULL, *us = NULL;
   int rc = -1;
   if (!Xd || !Ad || !Bd || !dYd || !t || !u || !dXd || !dAd || !dBd) goto done;
-  lora_down(Xd, Ad, T, K, r, t);
+  lora_down(Xl ? Xl : Xd, Ad, T, K, r, t);
   lora_up_t(dYd, Bd, T, N, r, u);
   if (rows) {
     dYs = gather_rows(dYd, N, rows, n_rows);
     us = gather_rows(u, r, rows, n_rows);
     if (!dYs || !us) goto done;
+    if (g && !(gs = gather_rows(g, K, rows, n_rows))) goto done;
   }
   {
-    dx_ctx c = {&w, rows ? dYs : dYd, rows ? us : u, Ad, n_rows, N, K, r, s, dXd};
+    dx_ctx c = {&w, rows ? dYs : dYd, rows ? us : u, Ad, n_rows, N, K, r, s, dXd,
+                rows ? gs : g};
     parallel_for(K, n_threads, dx_cols, &c);
   }
-  lora_grads(Xd, dYd, t, u, T, N, K, r, s, dAd, dBd);
+  lora_grads(Xl ? Xl : Xd, dYd, t, u, T, N, K, r, s, dAd, dBd);
   for (int64_t i = 0; i < n_rows * K; ++i) dX[i] = (float)dXd[i];
   for (int64_t i = 0; i < (int64_t)r * K; ++i) dA[i] = (float)dAd[i];
   for (int64_t i = 0; i < N * r; ++i) dB[i] = (float)dBd[i];
   rc = 0;
 done:
+  free(Xl);
+  free(g);
+  free(gs);
   free(Xd);
   free(Ad);
   free(Bd);
@@ -550,7 +698,7 @@ int orc_lora_fwd(const uint8_t *codes, const float *absmax, int64_t N,
                  const uint16_t *B, int r, float alpha, const int64_t *rows,
                  int64_t n_rows, float *Y, float *t_out, int n_threads) {
   const wsrc w = nf4_src(codes, absmax, K);
-  return lora_fwd_src(&w, N, K, X, T, A, B, r, alpha, rows, n_rows, Y, t_out, n_threads);
+  return lora_fwd_src(&w, NULL, N, K, X, T, A, B, r, alpha, rows, n_rows, Y, t_out, n_threads);
 }
 
 int orc_lora_bwd(const uint8_t *codes, const float *absmax, int64_t N,
@@ -559,7 +707,7 @@ int orc_lora_bwd(const uint8_t *codes, const float *absmax, int64_t N,
                  const int64_t *rows, int64_t n_rows, float *dX, float *dA,
                  float *dB, int n_threads) {
   const wsrc w = nf4_src(codes, absmax, K);
-  return lora_bwd_src(&w, N, K, X, T, A, B, r, alpha, dY, rows, n_rows, dX, dA, dB,
+  return lora_bwd_src(&w, NULL, N, K, X, T, A, B, r, alpha, dY, rows, n_rows, dX, dA, dB,
                       n_threads);
 }
 
@@ -568,7 +716,7 @@ int orc_lora_fwd_bf16w(const uint16_t *W, int64_t N, int64_t K, const uint16_t *
                        float alpha, const int64_t *rows, int64_t n_rows, float *Y,
                        float *t_out, int n_threads) {
   const wsrc w = bf16_src(W, K);
-  return lora_fwd_src(&w, N, K, X, T, A, B, r, alpha, rows, n_rows, Y, t_out, n_threads);
+  return lora_fwd_src(&w, NULL, N, K, X, T, A, B, r, alpha, rows, n_rows, Y, t_out, n_threads);
 }
 
 int orc_lora_bwd_bf16w(const uint16_t *W, int64_t N, int64_t K, const uint16_t *X,
@@ -576,7 +724,7 @@ int orc_lora_bwd_bf16w(const uint16_t *W, int64_t N, int64_t K, const uint16_t *
                        float alpha, const uint16_t *dY, const int64_t *rows,
                        int64_t n_rows, float *dX, float *dA, float *dB, int n_threads) {
   const wsrc w = bf16_src(W, K);
-  return lora_bwd_src(&w, N, K, X, T, A, B, r, alpha, dY, rows, n_rows, dX, dA, dB,
+  return lora_bwd_src(&w, NULL, N, K, X, T, A, B, r, alpha, dY, rows, n_rows, dX, dA, dB,
                       n_threads);
 }
 
@@ -624,4 +772,29 @@ int orc_lora_merge(const uint8_t *codes, const float *absmax, const uint16_t *Wb
   }
   free(row);
   return 0;
+}
+
+/* The NF4 LoRA linear with dropout p (seed, offset) on the adapter branch:
+ *   X_d = dropout(X);  t = X_d A^T;  Y = X W^T + s t B^T
+ *   u = dY B;  dX = dY W + (s u A) * keep * scale;  dB = s dY^T t;  dA = s u^T X_d
+ * p = 0 gives exactly orc_lora_fwd / orc_lora_bwd. */
+int orc_lora_fwd_drop(const uint8_t *codes, const float *absmax, int64_t N, int64_t K,
+                      const uint16_t *X, int64_t T, const uint16_t *A, const uint16_t *B,
+                      int r, float alpha, float p, uint64_t seed, uint64_t offset,
+                      const int64_t *rows, int64_t n_rows, float *Y, float *t_out,
+                      int n_threads) {
+  const wsrc w = nf4_src(codes, absmax, K);
+  const drop_cfg d = {p, seed, offset};
+  return lora_fwd_src(&w, &d, N, K, X, T, A, B, r, alpha, rows, n_rows, Y, t_out, n_threads);
+}
+
+int orc_lora_bwd_drop(const uint8_t *codes, const float *absmax, int64_t N, int64_t K,
+                      const uint16_t *X, int64_t T, const uint16_t *A, const uint16_t *B,
+                      int r, float alpha, float p, uint64_t seed, uint64_t offset,
+                      const uint16_t *dY, const int64_t *rows, int64_t n_rows, float *dX,
+                      float *dA, float *dB, int n_threads) {
+  const wsrc w = nf4_src(codes, absmax, K);
+  const drop_cfg d = {p, seed, offset};
+  return lora_bwd_src(&w, &d, N, K, X, T, A, B, r, alpha, dY, rows, n_rows, dX, dA, dB,
+                      n_threads);
 }

@@ -78,6 +78,35 @@ void orc_lora_bwd_f64(const double *W, const double *X, const double *A,
                       int64_t K, int r, double s, double *dX, double *dA,
                       double *dB);
 
+/* Masked variants of the double core (dropout on the adapter branch):
+ * fwd: t = Xl A^T with Xl the adapter branch's input, Y = X W^T + s t B^T;
+ * bwd: t = Xl A^T, u = dY B, dX = dY W + (s u A) * g (elementwise; g NULL
+ * = 1), dB = s dY^T t, dA = s u^T Xl.  The unmasked functions above are
+ * these with Xl = X and g = NULL. */
+void orc_lora_fwd_f64m(const double *W, const double *X, const double *Xl,
+                       const double *A, const double *B, int64_t T, int64_t N,
+                       int64_t K, int r, double s, double *Y, double *t);
+void orc_lora_bwd_f64m(const double *W, const double *Xl, const double *g,
+                       const double *A, const double *B, const double *dY,
+                       int64_t T, int64_t N, int64_t K, int r, double s,
+                       double *dX, double *dA, double *dB);
+
+/* ---- counter-based RNG and LoRA dropout ----
+ * Philox4x32-10 as published (Salmon et al., SC 2011): out = the 10-round
+ * bijection of the 128-bit counter under the 64-bit key. */
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+
+/* Dropout mask of a row-major [T,K] input: keep[e] for e = t*K + k, from
+ * word e%4 of Philox(ctr = {lo(e/4), hi(e/4), lo(offset), hi(offset)},
+ * key = {lo(seed), hi(seed)}): keep <=> (word >> 8) >= floor(p * 2^24).
+ * 0 <= p < 1.  Returns 0 or -1. */
+int orc_dropout_keep(uint64_t seed, uint64_t offset, float p, int64_t T, int64_t K,
+                     uint8_t *keep);
+
+/* X_d = keep ? bf16_rne(fp32(x) * scale) : +0,  scale = fp32(1 / fp32(1 - p)). */
+int orc_dropout_apply(const uint16_t *X, int64_t T, int64_t K, uint64_t seed,
+                      uint64_t offset, float p, uint16_t *out);
+
 /* ---- LoRA linear on the method's data types ----
  * W given as NF4 codes + absmax; X, A, B, dY as bf16 bit patterns; every
  * input is widened exactly, every sum is accumulated in double and rounded
@@ -96,6 +125,23 @@ int orc_lora_bwd(const uint8_t *codes, const float *absmax, int64_t N,
                  const uint16_t *B, int r, float alpha, const uint16_t *dY,
                  const int64_t *rows, int64_t n_rows, float *dX, float *dA,
                  float *dB, int n_threads);
+
+/* The NF4 LoRA linear with dropout p under (seed, offset) on the adapter
+ * branch (Poros API reference, lora_dropout):
+ *   X_d = dropout(X);  t = X_d A^T;  Y = X deq(W)^T + s t B^T;
+ *   u = dY B;  dX = dY deq(W) + (s u A) * keep * scale;
+ *   dB = s dY^T t;  dA = s u^T X_d.
+ * Conventions as orc_lora_fwd / orc_lora_bwd (which are p = 0). */
+int orc_lora_fwd_drop(const uint8_t *codes, const float *absmax, int64_t N, int64_t K,
+                      const uint16_t *X, int64_t T, const uint16_t *A, const uint16_t *B,
+                      int r, float alpha, float p, uint64_t seed, uint64_t offset,
+                      const int64_t *rows, int64_t n_rows, float *Y, float *t_out,
+                      int n_threads);
+int orc_lora_bwd_drop(const uint8_t *codes, const float *absmax, int64_t N, int64_t K,
+                      const uint16_t *X, int64_t T, const uint16_t *A, const uint16_t *B,
+                      int r, float alpha, float p, uint64_t seed, uint64_t offset,
+                      const uint16_t *dY, const int64_t *rows, int64_t n_rows, float *dX,
+                      float *dA, float *dB, int n_threads);
 
 /* The same forward / backward with a dense bf16 base W [N,K] (bf16 bit
  * patterns) in place of NF4 -- the quantization="bf16_bitwise" base of the

@@ -450,3 +450,135 @@ def test_merge_rounds_once_at_a_bf16_midpoint(orc):
                          W=synth.to_bf16_bits(W))
     assert np.all(out[N // 2:] == 0x3F80)   # tie -> even
     assert np.all(out[: N // 2] == 0x3F81)  # just above the tie -> up
+
+
+# ---------------------------------------------------------------- LoRA dropout
+
+def test_philox_known_answer_vectors(orc):
+    kat = json.load(open(os.path.join(GOLDEN, "philox4x32_10_kat.json")))
+    for v in kat["vectors"]:
+        got = orc.philox4x32_10([int(x, 16) for x in v["ctr"]], [int(x, 16) for x in v["key"]])
+        assert [f"{int(x):08x}" for x in got] == v["out"]
+
+
+def test_dropout_mask_follows_its_definition(orc):
+    """keep[t, k] from word (e % 4) of the Philox block of e // 4 (e = t K + k)
+    and the 24-bit threshold floor(p 2^24); checked on scattered elements with
+    the KAT-pinned generator."""
+    seed, offset, p, T, K = 0x1234_5678_9ABC_DEF0, (7 << 32) | 3, 0.3, 37, 192
+    keep = orc.dropout_keep(seed, offset, p, T, K)
+    thr = int(np.float32(p) * np.float32(2.0 ** 24))
+    rng = np.random.default_rng(30)
+    for _ in range(200):
+        t, k = int(rng.integers(T)), int(rng.integers(K))
+        e = t * K + k
+        q = e >> 2
+        w = orc.philox4x32_10([q & 0xFFFFFFFF, q >> 32, offset & 0xFFFFFFFF, offset >> 32],
+                              [seed & 0xFFFFFFFF, seed >> 32])[e & 3]
+        assert keep[t, k] == int((int(w) >> 8) >= thr), (t, k)
+
+
+@pytest.mark.parametrize("p", [0.0, 0.05, 0.5, 0.9])
+def test_dropout_keep_rate(orc, p):
+    T, K = 1024, 1024
+    keep = orc.dropout_keep(11, 5, p, T, K)
+    n = T * K
+    rate = keep.mean()
+    sigma = np.sqrt(p * (1 - p) / n)
+    assert abs(rate - (1 - p)) <= 6 * sigma + 1e-12
+    if p == 0.0:
+        assert keep.all()
+
+
+def test_dropout_masks_differ_across_offsets_and_seeds(orc):
+    """Independent streams agree on about p^2 + (1-p)^2 of the elements."""
+    p, T, K = 0.5, 512, 512
+    a = orc.dropout_keep(1, 0, p, T, K)
+    b = orc.dropout_keep(1, 1, p, T, K)
+    c = orc.dropout_keep(2, 0, p, T, K)
+    for x, y in ((a, b), (a, c), (b, c)):
+        agree = (x == y).mean()
+        assert abs(agree - 0.5) < 0.01
+    assert np.array_equal(a, orc.dropout_keep(1, 0, p, T, K))  # reproducible
+
+
+def test_dropout_apply_values(orc):
+    """Dropped -> +0; kept -> bf16_rne(fp32(x * scale)) with scale =
+    fp32(1 / fp32(1 - p)), rounded exactly (rational arithmetic); p = 0 ->
+    the input unchanged."""
+    from fractions import Fraction
+    rng = np.random.default_rng(31)
+    T, K, p = 16, 128, 0.05
+    X = synth.normal_bf16(rng, (T, K), 1.0)
+    assert np.array_equal(orc.dropout_apply(X, 3, 4, 0.0), X)
+    out = orc.dropout_apply(X, 3, 4, p)
+    keep = orc.dropout_keep(3, 4, p, T, K)
+    scale = np.float32(1.0) / (np.float32(1.0) - np.float32(p))
+    xf = synth.bits_to_f32(X)
+    for t in range(T):
+        for k in range(K):
+            if not keep[t, k]:
+                assert out[t, k] == 0
+            else:
+                prod = np.float32(xf[t, k]) * scale  # IEEE fp32 multiply (RN)
+                assert out[t, k] == _bf16_of_fraction(Fraction(float(prod))), (t, k)
+
+
+def test_dropout_zero_p_equals_plain_lora(orc):
+    c = synth.linear_case(32, 8, 128, 192, r=8)
+    codes, absmax = orc.quantize(c.W)
+    Y, t = orc.lora_fwd(codes, absmax, 128, 192, c.X, c.A, c.B, 16.0)
+    Yd, td = orc.lora_fwd_drop(codes, absmax, 128, 192, c.X, c.A, c.B, 16.0, 0.0, 9, 9)
+    assert np.array_equal(Y, Yd) and np.array_equal(t, td)
+    g = orc.lora_bwd(codes, absmax, 128, 192, c.X, c.A, c.B, c.dY, 16.0)
+    gd = orc.lora_bwd_drop(codes, absmax, 128, 192, c.X, c.A, c.B, c.dY, 16.0, 0.0, 9, 9)
+    for a, b in zip(g, gd):
+        assert np.array_equal(a, b)
+
+
+def test_dropout_gradient_matches_finite_differences(orc):
+    """With the mask m fixed, Y(X) = X W^T + s ((X * m) A^T) B^T: the loss
+    <G, Y> is linear in X, so central differences give dX exactly up to
+    rounding -- pinning the masked dX term and dA = s u^T (X * m)."""
+    W, X, A, B, G = _fd_case(33, T=4, N=64, K=64, r=2)
+    rng = np.random.default_rng(34)
+    m = np.where(rng.random(X.shape) < 0.3, 0.0, 1.0 / 0.7)
+    s = 2.0
+    dX, dA, dB = orc.lora_bwd_f64m(W, X * m, m, A, B, G, s)
+
+    def loss(X_, A_, B_):
+        Y, _ = orc.lora_fwd_f64m(W, X_, X_ * m, A_, B_, s)
+        return float(np.sum(G * Y))
+
+    h = 0.5
+    for name, M, grad in (("X", X, dX), ("A", A, dA), ("B", B, dB)):
+        for _ in range(12):
+            idx = tuple(int(rng.integers(0, d)) for d in M.shape)
+            P, Mm = M.copy(), M.copy()
+            P[idx] += h
+            Mm[idx] -= h
+            ap = {"X": (P, A, B), "A": (X, P, B), "B": (X, A, P)}[name]
+            am = {"X": (Mm, A, B), "A": (X, Mm, B), "B": (X, A, Mm)}[name]
+            fd = (loss(*ap) - loss(*am)) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-9 * max(1.0, abs(fd)), (name, idx, fd, grad[idx])
+
+
+def test_dropout_wrapper_is_the_masked_core(orc):
+    """The bf16 entry points with dropout are the FD-pinned masked core on
+    X_d = dropout_apply(X) and g = keep * scale, rounded once to fp32."""
+    c = synth.linear_case(35, 8, 64, 128, r=4)
+    p, seed, off = 0.25, 77, 12
+    codes, absmax = orc.quantize(c.W)
+    Wd = synth.bits_to_f32(orc.dequant(codes, absmax, 64, 128)).astype(np.float64)
+    f = lambda a: synth.bits_to_f32(a).astype(np.float64)
+    Xd = f(orc.dropout_apply(c.X, seed, off, p))
+    g = orc.dropout_keep(seed, off, p, 8, 128) * float(np.float32(1) / (np.float32(1) - np.float32(p)))
+    s = 32.0 / 4
+    Y, t = orc.lora_fwd_drop(codes, absmax, 64, 128, c.X, c.A, c.B, 32.0, p, seed, off)
+    Yc, tc = orc.lora_fwd_f64m(Wd, f(c.X), Xd, f(c.A), f(c.B), s)
+    assert np.array_equal(Y, Yc.astype(np.float32)) and np.array_equal(t, tc.astype(np.float32))
+    dX, dA, dB = orc.lora_bwd_drop(codes, absmax, 64, 128, c.X, c.A, c.B, c.dY, 32.0, p, seed, off)
+    dXc, dAc, dBc = orc.lora_bwd_f64m(Wd, Xd, g, f(c.A), f(c.B), f(c.dY), s)
+    assert np.array_equal(dX, dXc.astype(np.float32))
+    assert np.array_equal(dA, dAc.astype(np.float32))
+    assert np.array_equal(dB, dBc.astype(np.float32))
