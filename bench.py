@@ -64,6 +64,8 @@ def parse():
                     help="how a layer's projections are batched into grouped launches")
     ap.add_argument("--base", choices=["nf4", "bf16"], default="nf4",
                     help="frozen base format: NF4 (default) or dense bf16 (bf16_bitwise)")
+    ap.add_argument("--dropout", type=float, default=0.0,
+                    help="LoRA dropout on the adapter branch (the configs use 0)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=4.0,
@@ -246,7 +248,8 @@ def run_ours(args, ws, rank, local):
     # compute); a stack reuses the blocks still resident at each turn-around.
     stack = LayerStack(fam, args.layers, args.seq, block_size=args.block_size, streamed=streamed,
                        reuse_resident=not single, seed=42 + rank, device=dev,
-                       grouping=args.grouping, n_slots=args.slots, base=args.base)
+                       grouping=args.grouping, n_slots=args.slots, base=args.base,
+                       dropout=args.dropout)
     compute = stack.compute
 
     def one_step():
@@ -360,6 +363,7 @@ def run_ours(args, ws, rank, local):
         "data": "synthetic (seeded normal weights/activations; no dataset)",
         "config": {"workload": args.workload, "family": args.family, "layers": args.layers,
                    "tokens": args.seq, "batch": 1, "mode": args.mode, "base": args.base,
+                   "dropout": args.dropout,
                    "block_size": args.block_size, "rank": stack.r, "alpha": stack.alpha,
                    "grouping": args.grouping, "ring_slots": args.slots,
                    "projections": [p[0] for p in fam.projections()],

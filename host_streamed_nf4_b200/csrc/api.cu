@@ -229,6 +229,13 @@ static int check_one_format(const char* fn, int n, const int32_t* formats) {
   return HSNF4_OK;
 }
 
+static int check_dropout(const char* fn, int i, float p) {
+  if (!(p >= 0.0f && p < 1.0f))
+    return fail(HSNF4_ERR_INVALID, "%s: problem %d: dropout_p must be in [0, 1) (got %g)", fn, i,
+                static_cast<double>(p));
+  return HSNF4_OK;
+}
+
 static int check_group(const char* fn, int n, int64_t T, int r, float alpha) {
   if (n < 1 || n > 8)
     return fail(HSNF4_ERR_INVALID, "%s: 1..8 problems per call (got %d)", fn, n);
@@ -242,9 +249,10 @@ static int check_group(const char* fn, int n, int64_t T, int r, float alpha) {
 
 // Workspace layout of a forward group:
 //   [s*t bf16 [T, r_pad] per problem][t fp32 [T, r] per problem without t_save]
+//   [X_d bf16 [T, k_in] per problem with dropout]
 //   [projection partials][GEMM split-K partials + counters]
 struct FwdLayout {
-  size_t zs[8], tscratch[8], prj, gemm, total;
+  size_t zs[8], tscratch[8], xd[8], prj, gemm, total;
 };
 
 static void fwd_layout(const hsnf4_lora_fwd_args* p, int n, int64_t T, int r, FwdLayout* L) {
@@ -257,6 +265,10 @@ static void fwd_layout(const hsnf4_lora_fwd_args* p, int n, int64_t T, int r, Fw
   for (int i = 0; i < n; ++i) {
     L->tscratch[i] = off;
     if (!p[i].t_save) off += round_up(static_cast<size_t>(T) * r * 4, 256);
+  }
+  for (int i = 0; i < n; ++i) {
+    L->xd[i] = off;
+    if (p[i].dropout_p > 0.0f) off += round_up(static_cast<size_t>(T) * p[i].W.k_in * 2, 256);
   }
   ProjectDesc pd[8];
   GemmProblemDesc gd[8];
@@ -274,9 +286,10 @@ static void fwd_layout(const hsnf4_lora_fwd_args* p, int n, int64_t T, int r, Fw
 
 // Workspace layout of a backward group:
 //   [s*u bf16 [T, r_pad] per problem][u fp32 [T, r] per problem]
+//   [X_d bf16 [T, k_in] per problem with dropout]
 //   [projection partials][GEMM split-K partials + counters]
 struct BwdLayout {
-  size_t su[8], u[8], prj, gemm, total;
+  size_t su[8], u[8], xd[8], prj, gemm, total;
 };
 
 static void bwd_layout(const hsnf4_lora_bwd_args* p, int n, int64_t T, int r, BwdLayout* L) {
@@ -289,6 +302,10 @@ static void bwd_layout(const hsnf4_lora_bwd_args* p, int n, int64_t T, int r, Bw
   for (int i = 0; i < n; ++i) {
     L->u[i] = off;
     off += round_up(static_cast<size_t>(T) * r * 4, 256);
+  }
+  for (int i = 0; i < n; ++i) {
+    L->xd[i] = off;
+    if (p[i].dropout_p > 0.0f) off += round_up(static_cast<size_t>(T) * p[i].W.k_in * 2, 256);
   }
   ProjectDesc pd[8];
   GemmProblemDesc gd[8];
@@ -340,6 +357,7 @@ int lora_group_fwd(const hsnf4_lora_fwd_args* probs, int n, int64_t T, int r, fl
     if (!rc) rc = check_ptrs(fn, {{p.X, "X"}, {p.A, "A"}, {p.B, "B"}, {p.Y, "Y"}});
     if (!rc && p.t_save && !aligned16(p.t_save))
       rc = fail(HSNF4_ERR_INVALID, "%s: problem %d: t_save misaligned", fn, i);
+    if (!rc) rc = check_dropout(fn, i, p.dropout_p);
     if (rc) return rc;
   }
   {
@@ -357,12 +375,25 @@ int lora_group_fwd(const hsnf4_lora_fwd_args* probs, int n, int64_t T, int r, fl
   const float s = alpha / static_cast<float>(r);
   ProjectDesc pd[8];
   GemmProblemDesc gd[8];
+  DropDesc dd[8];
+  int nd = 0;
   for (int i = 0; i < n; ++i) {
     const hsnf4_lora_fwd_args& p = probs[i];
     float* t_out = p.t_save ? p.t_save : reinterpret_cast<float*>(ws + L.tscratch[i]);
-    pd[i] = {p.X, p.W.k_in, p.A, true, t_out, ws + L.zs[i]};
+    // with dropout the adapter branch reads X_d = dropout(X); the base reads X
+    const void* xl = p.X;
+    if (p.dropout_p > 0.0f) {
+      xl = ws + L.xd[i];
+      dd[nd++] = {p.X, ws + L.xd[i], nullptr, nullptr, p.W.k_in, p.dropout_p, p.dropout_seed,
+                  p.dropout_offset};
+    }
+    pd[i] = {xl, p.W.k_in, p.A, true, t_out, ws + L.zs[i]};
     gd[i] = {p.W.codes, p.W.absmax, p.W.n_out, p.W.k_in, p.X, p.B, ws + L.zs[i], p.Y,
              p.W.format == HSNF4_BASE_BF16};
+  }
+  if (nd) {
+    rc = cuda_status(launch_dropout_apply(dd, nd, T, st), "lora_group_fwd: dropout launch");
+    if (rc) return rc;
   }
   rc = cuda_status(launch_lora_project_group(pd, n, T, r, s, ws + L.prj, st),
                    "lora_group_fwd: projection launch");
@@ -382,6 +413,7 @@ int lora_group_bwd(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r, fl
     if (!rc)
       rc = check_ptrs(fn, {{p.X, "X"}, {p.t_save, "t_save"}, {p.A, "A"}, {p.B, "B"},
                            {p.dY, "dY"}, {p.dX, "dX"}, {p.dA, "dA"}, {p.dB, "dB"}});
+    if (!rc) rc = check_dropout(fn, i, p.dropout_p);
     if (rc) return rc;
   }
   {
@@ -400,20 +432,42 @@ int lora_group_bwd(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r, fl
   ProjectDesc pd[8];
   GemmProblemDesc gd[8];
   GradDesc grd[16];
+  DropDesc dd[8], da[8];
+  int nd = 0;
   for (int i = 0; i < n; ++i) {
     const hsnf4_lora_bwd_args& p = probs[i];
     float* u = reinterpret_cast<float*>(ws + L.u[i]);
-    pd[i] = {p.dY, p.W.n_out, p.B, false, u, ws + L.su[i]};
+    const bool drop = p.dropout_p > 0.0f;
+    // with dropout: X_d recomputed from the forward's (seed, offset) feeds
+    // dA; the GEMM's rank-r slice is zero and the masked adapter term of dX
+    // is added after it
+    const void* xl = drop ? static_cast<const void*>(ws + L.xd[i]) : p.X;
+    if (drop) {
+      dd[nd] = {p.X, ws + L.xd[i], nullptr, nullptr, p.W.k_in, p.dropout_p, p.dropout_seed,
+                p.dropout_offset};
+      da[nd] = {nullptr, p.dX, u, p.A, p.W.k_in, p.dropout_p, p.dropout_seed, p.dropout_offset};
+      ++nd;
+    }
+    pd[i] = {p.dY, p.W.n_out, p.B, false, u, ws + L.su[i], drop};
     gd[i] = {p.W.codes, p.W.absmax, p.W.n_out, p.W.k_in, p.dY, p.A, ws + L.su[i], p.dX,
              p.W.format == HSNF4_BASE_BF16};
-    grd[2 * i] = {p.dY, p.W.n_out, p.t_save, p.dB, true};  // dB = s dY^T t  [n_out, r]
-    grd[2 * i + 1] = {p.X, p.W.k_in, u, p.dA, false};      // dA = s u^T X   [r, k_in]
+    grd[2 * i] = {p.dY, p.W.n_out, p.t_save, p.dB, true};  // dB = s dY^T t    [n_out, r]
+    grd[2 * i + 1] = {xl, p.W.k_in, u, p.dA, false};       // dA = s u^T X(_d) [r, k_in]
+  }
+  if (nd) {
+    rc = cuda_status(launch_dropout_apply(dd, nd, T, st), "lora_group_bwd: dropout launch");
+    if (rc) return rc;
   }
   rc = cuda_status(launch_lora_project_group(pd, n, T, r, s, ws + L.prj, st),
                    "lora_group_bwd: projection launch");
   if (rc) return rc;
   rc = launch_lora_gemm_group(kGemmDx, gd, n, T, r, ws + L.gemm, L.total - L.gemm, st);
   if (rc) return rc;
+  if (nd) {
+    rc = cuda_status(launch_dx_dropout_add(da, nd, T, r, s, st),
+                     "lora_group_bwd: dropout dX launch");
+    if (rc) return rc;
+  }
   return cuda_status(launch_lora_grad_group(grd, 2 * n, T, r, s, st),
                      "lora_group_bwd: gradient launch");
 }
@@ -437,9 +491,22 @@ int lora_merge(const hsnf4_nf4_weight* W, const void* A, const void* B, int r, f
                      "lora_merge launch");
 }
 
+int lora_dropout_apply(const void* X, int64_t T, int64_t k_in, float p, uint64_t seed,
+                       uint64_t offset, void* X_d, void* stream) {
+  static const char* fn = "lora_dropout_apply";
+  int rc = check_nf4_shape(fn, T, k_in);
+  if (!rc) rc = check_dropout(fn, 0, p);
+  if (!rc) rc = check_ptrs(fn, {{X, "X"}, {X_d, "X_d"}});
+  if (rc) return rc;
+  DropDesc d = {X, X_d, nullptr, nullptr, k_in, p, seed, offset};
+  return cuda_status(launch_dropout_apply(&d, 1, T, static_cast<cudaStream_t>(stream)),
+                     "lora_dropout_apply launch");
+}
+
 static hsnf4_lora_fwd_args one_fwd(const hsnf4_nf4_weight* W, const void* X, const void* A,
                                    const void* B, void* Y, float* t_save) {
   hsnf4_lora_fwd_args a;
+  memset(&a, 0, sizeof a);  // no dropout
   a.W = *W;
   a.X = X;
   a.A = A;
@@ -476,6 +543,7 @@ int lora_linear_bwd(const hsnf4_nf4_weight* W, const void* X, const float* t_sav
                     float* dA, float* dB, void* workspace, size_t ws_bytes, void* stream) {
   if (!W) return fail(HSNF4_ERR_INVALID, "lora_linear_bwd: W is NULL");
   hsnf4_lora_bwd_args a;
+  memset(&a, 0, sizeof a);  // no dropout
   a.W = *W;
   a.X = X;
   a.t_save = t_save;

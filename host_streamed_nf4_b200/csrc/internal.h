@@ -45,6 +45,7 @@ struct ProjectDesc {
   bool r_major;
   float* t_out;
   void* zs;
+  bool zero_zs = false;  // write zs = 0 (the GEMM's rank-r slice then adds nothing)
 };
 size_t project_workspace_bytes(const ProjectDesc* d, int n, int64_t T, int r);
 cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, int r, float s,
@@ -91,6 +92,21 @@ cudaError_t launch_lora_merge(const void* base, const float* absmax, bool dense,
 
 // Process-wide count of kernels this library launched (hsnf4_kernel_launches).
 void count_launch();
+
+// ---- LoRA dropout, grouped (lora_dropout.cu): apply writes out = X_d;
+// dx add updates out = dX += keep * scale * s * (u A).
+struct DropDesc {
+  const void* X;
+  void* out;
+  const float* u;
+  const void* A;
+  int64_t K;
+  float p;
+  uint64_t seed, offset;
+};
+cudaError_t launch_dropout_apply(const DropDesc* d, int n, int64_t T, cudaStream_t st);
+cudaError_t launch_dx_dropout_add(const DropDesc* d, int n, int64_t T, int r, float s,
+                                  cudaStream_t st);
 
 // Kernel timing (hsnf4_profile): bracket a launch with prof_begin/prof_end.
 enum ProfKind { kProfGemmFwd = 0, kProfGemmDx = 1, kProfDequant = 2, kProfMerge = 3, kProfKinds = 4 };

@@ -55,6 +55,7 @@ struct PrjProblem {
   float* partial;  // [chunks][T][r_pad]
   int64_t C;
   int r_major, chunks, item0;  // item0: first CTA index of this problem
+  int zero_zs;
 };
 
 struct PrjParams {
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(256) lora_project_sum(const __grid_constant__ 
     for (; ch < pr.chunks; ++ch) v += __ldg(src + static_cast<int64_t>(ch) * per);
     pr.t_out[static_cast<int64_t>(t) * P.r + j] = v;
     const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(P.s, v));
-    out = *reinterpret_cast<const uint16_t*>(&b);
+    out = pr.zero_zs ? 0 : *reinterpret_cast<const uint16_t*>(&b);
   }
   pr.zs[static_cast<int64_t>(t) * P.r_pad + j] = out;
 }
@@ -292,6 +293,7 @@ cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, in
     p.zs = static_cast<uint16_t*>(d[q].zs);
     p.C = d[q].C;
     p.r_major = d[q].r_major ? 1 : 0;
+    p.zero_zs = d[q].zero_zs ? 1 : 0;
     p.chunks = static_cast<int>((d[q].C + P.cols - 1) / P.cols);
     p.partial = reinterpret_cast<float*>(w);
     w += round_up(static_cast<size_t>(p.chunks) * T * P.r_pad * 4, 256);

@@ -28,6 +28,8 @@
 
 #include <mutex>
 
+#include <cstring>
+
 #include "internal.h"
 
 namespace hsnf4 {
@@ -78,6 +80,7 @@ extern "C" int lora_linear_fwd_noalloc(const hsnf4_nf4_weight* W, const void* X,
   static const char* fn = "lora_linear_fwd_noalloc";
   if (!W) return fail(HSNF4_ERR_INVALID, "%s: W is NULL", fn);
   hsnf4_lora_fwd_args a;
+  memset(&a, 0, sizeof a);  // no dropout
   a.W = *W;
   a.X = X;
   a.A = A;

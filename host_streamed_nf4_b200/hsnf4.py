@@ -27,15 +27,19 @@ class Nf4WeightC(Structure):
                 ("format", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
+_DROPOUT_FIELDS = [("dropout_p", c_float), ("reserved", ctypes.c_uint32),
+                   ("dropout_seed", c_uint64), ("dropout_offset", c_uint64)]
+
+
 class FwdArgs(Structure):
     _fields_ = [("W", Nf4WeightC), ("X", c_void_p), ("A", c_void_p), ("B", c_void_p),
-                ("Y", c_void_p), ("t_save", c_void_p)]
+                ("Y", c_void_p), ("t_save", c_void_p)] + _DROPOUT_FIELDS
 
 
 class BwdArgs(Structure):
     _fields_ = [("W", Nf4WeightC), ("X", c_void_p), ("t_save", c_void_p), ("A", c_void_p),
                 ("B", c_void_p), ("dY", c_void_p), ("dX", c_void_p), ("dA", c_void_p),
-                ("dB", c_void_p)]
+                ("dB", c_void_p)] + _DROPOUT_FIELDS
 
 
 class LayerDesc(Structure):
@@ -81,6 +85,8 @@ _SIGS = {
     "nf4_dequant": ([c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p], c_int),
     "lora_merge": ([POINTER(Nf4WeightC), c_void_p, c_void_p, c_int, c_float, c_void_p, c_void_p],
                    c_int),
+    "lora_dropout_apply": ([c_void_p, c_int64, c_int64, c_float, c_uint64, c_uint64, c_void_p,
+                            c_void_p], c_int),
     "lora_linear_fwd_workspace": ([c_int64, c_int64, c_int64, c_int], c_size_t),
     "lora_linear_bwd_workspace": ([c_int64, c_int64, c_int64, c_int], c_size_t),
     "lora_linear_fwd": ([POINTER(Nf4WeightC), c_void_p, c_int64, c_void_p, c_void_p, c_int, c_float,
@@ -348,13 +354,29 @@ def _p(t):
     return None if t is None else t.data_ptr()
 
 
-def fwd_args(W, X, A, B, Y, t_save=None) -> FwdArgs:
-    """One problem of a grouped forward (tensors are kept alive by the caller)."""
-    return FwdArgs(_wc(W), _p(X), _p(A), _p(B), _p(Y), _p(t_save))
+def fwd_args(W, X, A, B, Y, t_save=None, dropout=None) -> FwdArgs:
+    """One problem of a grouped forward (tensors are kept alive by the caller).
+    dropout: (p, seed, offset) for the adapter branch, or None."""
+    p, seed, off = dropout or (0.0, 0, 0)
+    return FwdArgs(_wc(W), _p(X), _p(A), _p(B), _p(Y), _p(t_save), p, 0, seed, off)
 
 
-def bwd_args(W, X, t_save, A, B, dY, dX, dA, dB) -> BwdArgs:
-    return BwdArgs(_wc(W), _p(X), _p(t_save), _p(A), _p(B), _p(dY), _p(dX), _p(dA), _p(dB))
+def bwd_args(W, X, t_save, A, B, dY, dX, dA, dB, dropout=None) -> BwdArgs:
+    p, seed, off = dropout or (0.0, 0, 0)
+    return BwdArgs(_wc(W), _p(X), _p(t_save), _p(A), _p(B), _p(dY), _p(dX), _p(dA), _p(dB),
+                   p, 0, seed, off)
+
+
+def lora_dropout_apply(X: torch.Tensor, p: float, seed: int, offset: int, out=None,
+                       stream=None) -> torch.Tensor:
+    """X_d = dropout(X) on the adapter branch's definition (bf16 [T, K])."""
+    _need(X, "X", torch.bfloat16)
+    T, K = X.shape
+    if out is None:
+        out = torch.empty_like(X)
+    _check(lib().lora_dropout_apply(_ptr(X), T, K, float(p), seed, offset, _ptr(out),
+                                    _stream(stream)))
+    return out
 
 
 def group_fwd_workspace_bytes(args, T, r) -> int:

@@ -60,7 +60,7 @@ class LayerStack:
                  streamed: bool = True, reuse_resident: bool = True, enable_prefetch: bool = True,
                  poison_on_release: bool = False, r: int = synth.RANK, alpha: float = synth.ALPHA,
                  seed: int = 42, device=None, grouping: str = "layer", n_slots: int = 2,
-                 base: str = "nf4"):
+                 base: str = "nf4", dropout: float = 0.0):
         self.device = torch.device(device) if device is not None else torch.device(
             "cuda", torch.cuda.current_device())
         dev = self.device
@@ -73,6 +73,10 @@ class LayerStack:
             raise ValueError(f"base must be 'nf4' or 'bf16' (got {base!r})")
         self.base = base
         self.base_format = hsnf4.BASE_BF16 if base == "bf16" else hsnf4.BASE_NF4
+        # LoRA dropout on the adapter branch: the mask of (step, layer,
+        # projection) is drawn from a counter-based generator, so the backward
+        # re-draws exactly the forward's mask
+        self.dropout, self.seed, self.step_idx = float(dropout), int(seed), 0
         self.desc = hsnf4.layer_desc([(n, k) for _, n, k in self.projs], self.base_format)
         self.descs = [self.desc] * n_layers
         self.layer_bytes = hsnf4.layer_bytes(self.desc)
@@ -129,9 +133,9 @@ class LayerStack:
         ws_f = ws_b = 256
         for grp in self.groups:
             fa = [hsnf4.FwdArgs(hsnf4.Nf4WeightC(0, 0, self.projs[p][1], self.projs[p][2]), 0, 0, 0,
-                                0, 1) for p in grp]
+                                0, 1, self.dropout) for p in grp]
             ba = [hsnf4.BwdArgs(hsnf4.Nf4WeightC(0, 0, self.projs[p][1], self.projs[p][2]),
-                                0, 0, 0, 0, 0, 0, 0, 0) for p in grp]
+                                0, 0, 0, 0, 0, 0, 0, 0, self.dropout) for p in grp]
             ws_f = max(ws_f, hsnf4.group_fwd_workspace_bytes(fa, T, r))
             ws_b = max(ws_b, hsnf4.group_bwd_workspace_bytes(ba, T, r))
         del dummy
@@ -191,11 +195,19 @@ class LayerStack:
         if self.streamed:
             self.streamer.release(b, self.compute)
 
+    def dropout_of(self, l: int, p: int):
+        """(p, seed, offset) of layer l, projection p in the current step, or
+        None: the offset packs (step, layer, projection)."""
+        if self.dropout <= 0.0:
+            return None
+        return (self.dropout, self.seed, (self.step_idx << 32) | (l << 4) | p)
+
     def _fwd_block(self, ws, b, record):
         for i, l in enumerate(self.block_layers(b)):
             for grp in self.groups:
                 args = [hsnf4.fwd_args(ws[i * self.P + p], self.X[INPUT_OF[self.projs[p][0]]],
-                                       self.A[l][p], self.B[l][p], self.Y[p], self.t[l][p])
+                                       self.A[l][p], self.B[l][p], self.Y[p], self.t[l][p],
+                                       self.dropout_of(l, p))
                         for p in grp]
                 hsnf4.lora_group_fwd(args, self.T, self.r, self.alpha, self.ws_f,
                                      stream=self.compute)
@@ -210,7 +222,8 @@ class LayerStack:
             for grp in reversed(self.groups):
                 args = [hsnf4.bwd_args(ws[i * self.P + p], self.X[INPUT_OF[self.projs[p][0]]],
                                        self.t[l][p], self.A[l][p], self.B[l][p], self.dY[p],
-                                       self.dX[p], self.dA[l][p], self.dB[l][p])
+                                       self.dX[p], self.dA[l][p], self.dB[l][p],
+                                       self.dropout_of(l, p))
                         for p in grp]
                 hsnf4.lora_group_bwd(args, self.T, self.r, self.alpha, self.ws_b,
                                      stream=self.compute)
@@ -254,6 +267,7 @@ class LayerStack:
             for b, fwd in V:
                 ws = self._weights(b)
                 (self._fwd_block if fwd else self._bwd_block)(ws, b, record)
+            self.step_idx += 1
             return
         n = len(V)
         look = 2 * self.streamer.n_slots
@@ -265,6 +279,7 @@ class LayerStack:
             self.streamer.prefetch_ahead([V[(i + j) % n][0] for j in range(1, look + 1)])
             (self._fwd_block if fwd else self._bwd_block)(ws, b, record)
             self.streamer.release(b, self.compute)
+        self.step_idx += 1
 
     def step_single_block(self, record=None):
         """A one-block stack whose block is re-streamed every step: acquire the
@@ -281,6 +296,7 @@ class LayerStack:
         self._fwd_block(ws, 0, record)
         self._bwd_block(ws, 0, record)
         self.streamer.release(0, self.compute)
+        self.step_idx += 1
 
     # ------------------------------------------------------------------ accounting
 

@@ -263,6 +263,17 @@ typedef struct {
   const void *B;   /* bf16 [n_out, r] */
   void *Y;         /* bf16 [T, n_out] */
   float *t_save;   /* fp32 [T, r] or NULL */
+  /* LoRA dropout on the adapter branch (Poros API reference, lora_dropout):
+   * t = dropout(X) A^T.  p in [0, 1), 0 = none (a zero-initialised struct
+   * has none).  The mask of X[t, k] comes from Philox4x32-10 keyed by
+   * dropout_seed at counter {(t*k_in + k)/4, dropout_offset}: word
+   * (t*k_in + k) % 4 kept iff its top 24 bits >= floor(p * 2^24); kept
+   * values are bf16_rne(x * fp32(1 / (1 - p))).  The backward of the same
+   * step must pass the same seed and offset (it recomputes the mask). */
+  float dropout_p;
+  uint32_t reserved;
+  uint64_t dropout_seed;
+  uint64_t dropout_offset;
 } hsnf4_lora_fwd_args;
 
 typedef struct {
@@ -275,10 +286,24 @@ typedef struct {
   void *dX;             /* bf16 [T, k_in] */
   float *dA;            /* fp32 [r, k_in] */
   float *dB;            /* fp32 [n_out, r] */
+  /* dropout as in the forward (same p, seed, offset): dA = s u^T dropout(X)
+   * and dX's adapter term is (s u A) * keep / (1 - p), added in fp32 to the
+   * bf16 dY deq(W) and rounded again (two roundings of dX when p > 0). */
+  float dropout_p;
+  uint32_t reserved;
+  uint64_t dropout_seed;
+  uint64_t dropout_offset;
 } hsnf4_lora_bwd_args;
 
-/* Workspace bytes of a grouped call (depends on the shapes and on the
- * current device's SM count). */
+/* The dropout of the adapter branch on its own: X_d = dropout(X) as defined
+ * at hsnf4_lora_fwd_args (X, X_d bf16 [T, k_in], k_in a multiple of 64,
+ * 0 <= p < 1).  The grouped calls apply it internally; this entry point
+ * exposes the mask for checking and reuse.  Errors: INVALID. */
+int lora_dropout_apply(const void *X, int64_t T, int64_t k_in, float p, uint64_t seed,
+                       uint64_t offset, void *X_d, void *stream);
+
+/* Workspace bytes of a grouped call (depends on the shapes, on which
+ * problems use dropout and on the current device's SM count). */
 size_t lora_group_fwd_workspace(const hsnf4_lora_fwd_args *probs, int n, int64_t T, int r);
 size_t lora_group_bwd_workspace(const hsnf4_lora_bwd_args *probs, int n, int64_t T, int r);
 

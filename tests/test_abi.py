@@ -191,3 +191,24 @@ def test_bf16_layer_layout():
     assert abs(total / nf4 - 2 / 0.5625) < 1e-3
     with pytest.raises(hsnf4.HsNf4Error):
         hsnf4.layer_bytes(hsnf4.layer_desc(shapes, 2))
+
+
+def test_dropout_validation_before_cuda():
+    import ctypes
+    L = hsnf4.lib()
+    fake = 0x10000
+    W = hsnf4.Nf4WeightC(fake, fake, 128, 256, hsnf4.BASE_NF4, 0)
+    for p in (1.0, -0.25, float("nan")):
+        arr = (hsnf4.FwdArgs * 1)(hsnf4.FwdArgs(W, fake, fake, fake, fake, None, p, 0, 1, 2))
+        assert L.lora_group_fwd(arr, 1, 64, 16, 32.0, fake, 1 << 30, None) == hsnf4.ERR_INVALID
+        assert "dropout_p" in hsnf4.last_error()
+        barr = (hsnf4.BwdArgs * 1)(hsnf4.BwdArgs(W, fake, fake, fake, fake, fake, fake, fake, fake,
+                                                 p, 0, 1, 2))
+        assert L.lora_group_bwd(barr, 1, 64, 16, 32.0, fake, 1 << 30, None) == hsnf4.ERR_INVALID
+        assert L.lora_dropout_apply(fake, 64, 256, p, 1, 2, fake, None) == hsnf4.ERR_INVALID
+    assert L.lora_dropout_apply(fake, 64, 100, 0.1, 1, 2, fake, None) == hsnf4.ERR_INVALID
+    # a forward with dropout needs room for X_d [T, k_in] in its workspace
+    plain = hsnf4.FwdArgs(hsnf4.Nf4WeightC(0, 0, 128, 256), 0, 0, 0, 0, 1)
+    drop = hsnf4.FwdArgs(hsnf4.Nf4WeightC(0, 0, 128, 256), 0, 0, 0, 0, 1, 0.1, 0, 1, 2)
+    assert hsnf4.group_fwd_workspace_bytes([drop], 64, 16) >= \
+        hsnf4.group_fwd_workspace_bytes([plain], 64, 16) + 64 * 256 * 2
