@@ -66,6 +66,9 @@ def parse():
                     help="frozen base format: NF4 (default) or dense bf16 (bf16_bitwise)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="LoRA dropout on the adapter branch (the configs use 0)")
+    ap.add_argument("--no-shard-h2d", dest="shard_h2d", action="store_false",
+                    help="with N > 1 GPUs every rank streams whole blocks (default: each "
+                         "streams 1/N and the ranks all-gather)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=4.0,
@@ -246,8 +249,14 @@ def run_ours(args, ws, rank, local):
     # A one-layer workload re-streams its layer every step (the layer's bytes
     # cross PCIe once per step, the next copy overlapping this step's
     # compute); a stack reuses the blocks still resident at each turn-around.
+    # data-parallel ranks share the frozen base and the adapters (seed 42)
+    # and see their own tokens (data_seed); with N > 1 the ranks share the
+    # stream too: each copies 1/N of every block and an NCCL all-gather on
+    # the copy stream rebuilds the block in every ring
+    shard = (rank, ws, hdist.ring_gather) if (streamed and ws > 1 and args.shard_h2d) else None
     stack = LayerStack(fam, args.layers, args.seq, block_size=args.block_size, streamed=streamed,
-                       reuse_resident=not single, seed=42 + rank, device=dev,
+                       reuse_resident=not single, seed=42, data_seed=42 + rank, device=dev,
+                       shard=shard,
                        grouping=args.grouping, n_slots=args.slots, base=args.base,
                        dropout=args.dropout)
     compute = stack.compute
@@ -368,7 +377,8 @@ def run_ours(args, ws, rank, local):
                    "grouping": args.grouping, "ring_slots": args.slots,
                    "projections": [p[0] for p in fam.projections()],
                    "parallelism": (f"dp{ws} (per-rank tokens, adapter-gradient all-reduce per "
-                                   f"step)" if ws > 1 else "single"),
+                                   f"step" + (", sharded H2D + per-block all-gather)"
+                                              if shard else ")") if ws > 1 else "single"),
                    "l2": "no flush: every step reads > 126 MB L2 (NF4 weights + activations)"},
         "roofline": roofline, "step_roofline": step_roofline, "dequant": dequant, "merge": merge,
         "peak_vram_GB": round(torch.cuda.max_memory_allocated(dev) / 1e9, 3), "e2e": e2e,

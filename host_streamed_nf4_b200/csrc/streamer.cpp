@@ -146,16 +146,37 @@ int enqueue_copy(hsnf4_streamer* s, int i, int b, cudaStream_t after) {
   if (take_fault(kFaultCopyEnqueue))
     return fail(HSNF4_ERR_CUDA, "prefetch: injected fault at copy_enqueue (block %d)", b);
   const size_t bytes = s->block_bytes(b);
-  rc = cuda_status(cudaMemcpyAsync(s->ring + static_cast<size_t>(i) * s->slot_bytes,
-                                   s->slab + s->block_off(b), bytes, cudaMemcpyHostToDevice,
-                                   s->copy),
-                   "prefetch: cudaMemcpyAsync H2D");
-  if (rc) return rc;
+  uint8_t* slot = s->ring + static_cast<size_t>(i) * s->slot_bytes;
+  size_t copied = bytes;
+  if (s->cfg.gather) {
+    // sharded: this rank's shard over its own link, then the gather fills
+    // the other ranks' shards, in copy-stream order before `ready`
+    const int world = s->cfg.shard_world > 1 ? s->cfg.shard_world : 1;
+    size_t S = 0, off = 0, len = 0;
+    stream_shard_range(bytes, world, s->cfg.shard_rank, &S, &off, &len);
+    if (len) {
+      rc = cuda_status(cudaMemcpyAsync(slot + off, s->slab + s->block_off(b) + off, len,
+                                       cudaMemcpyHostToDevice, s->copy),
+                       "prefetch: cudaMemcpyAsync H2D (shard)");
+      if (rc) return rc;
+    }
+    const int g = s->cfg.gather(slot, S, world, b, s->copy, s->cfg.gather_user);
+    if (g != 0)
+      return fail(HSNF4_ERR_CUDA, "prefetch: gather of block %d failed (callback returned %d)",
+                  b, g);
+    s->stats.gathers += 1;
+    copied = len;
+  } else {
+    rc = cuda_status(cudaMemcpyAsync(slot, s->slab + s->block_off(b), bytes,
+                                     cudaMemcpyHostToDevice, s->copy),
+                     "prefetch: cudaMemcpyAsync H2D");
+    if (rc) return rc;
+  }
   rc = record(sl.ready, s->copy, "prefetch: record ready");
   if (rc) return rc;
   sl.block = b;
   sl.state = kLoaded;
-  s->stats.h2d_bytes += bytes;
+  s->stats.h2d_bytes += copied;
   s->stats.copies += 1;
   return HSNF4_OK;
 }
@@ -245,6 +266,40 @@ int stream_slot_bytes(const hsnf4_layer_desc* layers, int n_layers, int block_si
   return HSNF4_OK;
 }
 
+int stream_shard_range(size_t block_bytes, int world, int rank, size_t* shard_bytes,
+                       size_t* off, size_t* len) {
+  if (world < 1 || rank < 0 || rank >= world || !shard_bytes || !off || !len)
+    return fail(HSNF4_ERR_INVALID, "stream_shard_range: need 0 <= rank < world and outputs "
+                "(world=%d rank=%d)", world, rank);
+  const size_t S = round_up((block_bytes + world - 1) / world, kAlign);
+  const size_t o = S * static_cast<size_t>(rank);
+  *shard_bytes = S;
+  *off = o;
+  *len = o >= block_bytes ? 0 : (block_bytes - o < S ? block_bytes - o : S);
+  return HSNF4_OK;
+}
+
+int stream_slot_bytes_sharded(const hsnf4_layer_desc* layers, int n_layers, int block_size,
+                              int world, size_t* out_bytes) {
+  if (!layers || n_layers < 1 || !out_bytes || block_size < 1 || world < 1)
+    return fail(HSNF4_ERR_INVALID, "stream_slot_bytes_sharded: need layers, n_layers >= 1, "
+                "block_size >= 1, world >= 1, out_bytes");
+  size_t slot = 0;
+  for (int first = 0; first < n_layers; first += block_size) {
+    size_t b = 0;
+    for (int l = first; l < n_layers && l < first + block_size; ++l) {
+      int rc = check_layer("stream_slot_bytes_sharded", &layers[l]);
+      if (rc) return rc;
+      b += layer_bytes(layers[l]);
+    }
+    size_t S = 0, off = 0, len = 0;
+    stream_shard_range(b, world, 0, &S, &off, &len);
+    if (S * world > slot) slot = S * world;
+  }
+  *out_bytes = slot;
+  return HSNF4_OK;
+}
+
 int stream_ring_bytes(const hsnf4_layer_desc* layers, int n_layers, int block_size,
                       size_t* out_bytes) {
   if (!layers || n_layers < 1 || !out_bytes || block_size < 1)
@@ -279,10 +334,19 @@ int stream_create(const void* pinned_slab, size_t slab_bytes, const hsnf4_layer_
   if (n_slots < 2 || n_slots > HSNF4_MAX_SLOTS)
     return fail(HSNF4_ERR_INVALID, "%s: n_slots must be 0 (= 2) or in [2, %d] (got %d)", fn,
                 HSNF4_MAX_SLOTS, cfg->n_slots);
+  const int world = cfg->shard_world > 1 ? cfg->shard_world : 1;
+  if (cfg->shard_world < 0 || cfg->shard_rank < 0 || cfg->shard_rank >= world)
+    return fail(HSNF4_ERR_INVALID, "%s: need 0 <= shard_rank < shard_world (got rank %d of %d)",
+                fn, cfg->shard_rank, cfg->shard_world);
+  if (world > 1 && !cfg->gather)
+    return fail(HSNF4_ERR_INVALID, "%s: a stream sharded over %d ranks needs a gather callback",
+                fn, world);
   size_t need_slab = 0, need_ring = 0;
   int rc = stream_slab_bytes(layers, n_layers, &need_slab);
   if (rc) return rc;
-  rc = stream_slot_bytes(layers, n_layers, cfg->block_size, &need_ring);
+  rc = cfg->gather
+           ? stream_slot_bytes_sharded(layers, n_layers, cfg->block_size, world, &need_ring)
+           : stream_slot_bytes(layers, n_layers, cfg->block_size, &need_ring);
   if (rc) return rc;
   const size_t slot_bytes = need_ring;
   need_ring *= static_cast<size_t>(n_slots);

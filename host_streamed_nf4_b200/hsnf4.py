@@ -47,14 +47,19 @@ class LayerDesc(Structure):
                 ("base_format", c_int)]
 
 
+# int gather(void *slot, size_t shard_bytes, int world, int block, void *copy_stream, void *user)
+GATHER_FN = ctypes.CFUNCTYPE(c_int, c_void_p, c_size_t, c_int, c_int, c_void_p, c_void_p)
+
+
 class StreamConfig(Structure):
     _fields_ = [("block_size", c_int), ("enable_prefetch", c_int), ("reuse_resident", c_int),
-                ("poison_on_release", c_int), ("n_slots", c_int)]
+                ("poison_on_release", c_int), ("n_slots", c_int), ("shard_world", c_int),
+                ("shard_rank", c_int), ("gather", GATHER_FN), ("gather_user", c_void_p)]
 
 
 class StreamStats(Structure):
     _fields_ = [("h2d_bytes", c_uint64), ("copies", c_uint64), ("reuses", c_uint64),
-                ("acquires", c_uint64), ("releases", c_uint64)]
+                ("acquires", c_uint64), ("releases", c_uint64), ("gathers", c_uint64)]
 
 
 class KernelTime(Structure):
@@ -108,6 +113,10 @@ _SIGS = {
     "stream_ring_bytes": ([POINTER(LayerDesc), c_int, c_int, POINTER(c_size_t)], c_int),
     "stream_slot_bytes": ([POINTER(LayerDesc), c_int, c_int, POINTER(c_size_t)], c_int),
     "stream_prefetch_ahead": ([c_void_p, POINTER(c_int), c_int, POINTER(c_int)], c_int),
+    "stream_shard_range": ([c_size_t, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t),
+                            POINTER(c_size_t)], c_int),
+    "stream_slot_bytes_sharded": ([POINTER(LayerDesc), c_int, c_int, c_int, POINTER(c_size_t)],
+                                  c_int),
     "stream_create": ([c_void_p, c_size_t, POINTER(LayerDesc), c_int, POINTER(StreamConfig), c_void_p,
                        c_size_t, c_void_p, POINTER(c_void_p)], c_int),
     "stream_num_blocks": ([c_void_p], c_int),
@@ -439,18 +448,37 @@ def slab_bytes(descs) -> int:
     return out.value
 
 
-def ring_bytes(descs, block_size: int, n_slots: int = 2) -> int:
+def ring_bytes(descs, block_size: int, n_slots: int = 2, shard_world: int = 0) -> int:
+    """Device bytes of an n_slots ring; shard_world >= 1: of a sharded stream."""
     out = c_size_t(0)
-    _check(lib().stream_slot_bytes(_desc_array(descs), len(descs), block_size, ctypes.byref(out)))
+    if shard_world >= 1:
+        _check(lib().stream_slot_bytes_sharded(_desc_array(descs), len(descs), block_size,
+                                               shard_world, ctypes.byref(out)))
+    else:
+        _check(lib().stream_slot_bytes(_desc_array(descs), len(descs), block_size,
+                                       ctypes.byref(out)))
     return out.value * n_slots
 
 
+def shard_range(block_bytes: int, world: int, rank: int):
+    """(stride S, offset, length) of rank's shard of a block shared by world ranks."""
+    S, off, n = c_size_t(0), c_size_t(0), c_size_t(0)
+    _check(lib().stream_shard_range(block_bytes, world, rank, ctypes.byref(S), ctypes.byref(off),
+                                    ctypes.byref(n)))
+    return S.value, off.value, n.value
+
+
 class Streamer:
-    """Pinned-host NF4 stack -> 2-slot VRAM ring, prefetched one block ahead."""
+    """Pinned-host NF4 stack -> 2-slot VRAM ring, prefetched one block ahead.
+
+    shard=(rank, world, gather): stream 1/world of every block over this
+    rank's link; gather(slot_offset, shard_bytes, world, block) must enqueue,
+    on the current CUDA stream (the copy stream), the in-place all-gather of
+    the ring bytes [slot_offset, slot_offset + world * shard_bytes)."""
 
     def __init__(self, slab: torch.Tensor, descs, block_size: int, ring: torch.Tensor,
                  copy_stream: torch.cuda.Stream, enable_prefetch=True, reuse_resident=True,
-                 poison_on_release=False, n_slots=2):
+                 poison_on_release=False, n_slots=2, shard=None):
         _need(slab, "slab", torch.uint8, device=False)
         if not slab.is_pinned():
             raise ValueError("slab must be page-locked (pin_memory)")
@@ -459,6 +487,24 @@ class Streamer:
         self._arr = _desc_array(self.descs)
         cfg = StreamConfig(block_size, int(bool(enable_prefetch)), int(bool(reuse_resident)),
                            int(bool(poison_on_release)), int(n_slots))
+        self._gather_error = None
+        self._gather_cb = None
+        if shard is not None:
+            rank, world, fn = shard
+            base = ring.data_ptr()
+
+            def _cb(slot, shard_bytes, world_, block, stream, user):
+                try:
+                    with torch.cuda.stream(copy_stream):
+                        fn(slot - base, shard_bytes, world_, block)
+                    return 0
+                except Exception as e:  # reported through the library's status
+                    self._gather_error = e
+                    return 1
+
+            self._gather_cb = GATHER_FN(_cb)
+            cfg.shard_world, cfg.shard_rank = world, rank
+            cfg.gather = self._gather_cb
         self.n_slots = n_slots
         h = c_void_p()
         _check(lib().stream_create(_ptr(slab), slab.numel(), self._arr, len(self.descs),
@@ -469,20 +515,26 @@ class Streamer:
         self.block_size = block_size
         self.n_blocks = lib().stream_num_blocks(h)
 
+    def _check(self, rc: int):
+        err, self._gather_error = self._gather_error, None
+        if rc != 0 and err is not None:
+            raise HsNf4Error(rc, f"{last_error()} ({type(err).__name__}: {err})") from err
+        _check(rc)
+
     def prefetch(self, b: int):
-        _check(lib().stream_block_prefetch(self._h, b))
+        self._check(lib().stream_block_prefetch(self._h, b))
 
     def prefetch_ahead(self, upcoming) -> int:
         arr = (c_int * len(upcoming))(*upcoming)
         issued = c_int(0)
-        _check(lib().stream_prefetch_ahead(self._h, arr, len(upcoming), ctypes.byref(issued)))
+        self._check(lib().stream_prefetch_ahead(self._h, arr, len(upcoming), ctypes.byref(issued)))
         return issued.value
 
     def acquire(self, b: int, stream=None):
         first = b * self.block_size
         n = sum(d.n_proj for d in self.descs[first:first + self.block_size])
         out = (Nf4WeightC * n)()
-        _check(lib().stream_block_acquire(self._h, b, _stream(stream), out, n))
+        self._check(lib().stream_block_acquire(self._h, b, _stream(stream), out, n))
         return list(out)
 
     def acquire_host(self, b: int, timeout_ms: int):

@@ -60,7 +60,12 @@ class LayerStack:
                  streamed: bool = True, reuse_resident: bool = True, enable_prefetch: bool = True,
                  poison_on_release: bool = False, r: int = synth.RANK, alpha: float = synth.ALPHA,
                  seed: int = 42, device=None, grouping: str = "layer", n_slots: int = 2,
-                 base: str = "nf4", dropout: float = 0.0):
+                 base: str = "nf4", dropout: float = 0.0, data_seed=None, shard=None):
+        """shard = (rank, world, gather_factory): stream 1/world of every
+        block (sharded stream); gather_factory(ring) returns the streamer's
+        gather callback (dist.ring_gather).  data_seed: seed of the
+        activations and upstream gradients (default: seed); the weights and
+        adapters always come from seed, as data-parallel ranks share them."""
         self.device = torch.device(device) if device is not None else torch.device(
             "cuda", torch.cuda.current_device())
         dev = self.device
@@ -86,21 +91,25 @@ class LayerStack:
         self._fill_slab(seed)
 
         self.compute = torch.cuda.current_stream(dev)
+        self.shard = shard
         if streamed:
-            self.ring = torch.empty(hsnf4.ring_bytes(self.descs, block_size, n_slots),
+            world = shard[1] if shard else 0
+            self.ring = torch.empty(hsnf4.ring_bytes(self.descs, block_size, n_slots, world),
                                     dtype=torch.uint8, device=dev)
             self.copy_stream = torch.cuda.Stream(dev)
+            sh = (shard[0], shard[1], shard[2](self.ring)) if shard else None
             self.streamer = hsnf4.Streamer(self.slab, self.descs, block_size, self.ring,
                                            self.copy_stream, enable_prefetch=enable_prefetch,
                                            reuse_resident=reuse_resident,
-                                           poison_on_release=poison_on_release, n_slots=n_slots)
+                                           poison_on_release=poison_on_release, n_slots=n_slots,
+                                           shard=sh)
         else:
             self.dev_slab = self.slab.to(dev)
             self.streamer = None
 
         # activations and upstream gradients (shared by all layers)
         h, d = family.hidden, family.head_dim
-        g = _gen(dev, seed, 1_000_001)
+        g = _gen(dev, seed if data_seed is None else data_seed, 1_000_001)
         self.X = {"h": _randn_bf16((T, h), 1.0, g, dev),
                   "o": _randn_bf16((T, family.heads * d), 1.0, g, dev),
                   "i": _randn_bf16((T, family.inter), 1.0, g, dev)}
@@ -310,13 +319,20 @@ class LayerStack:
         backward -> next forward) are not copied again: the n_slots blocks
         nearest the turn-around."""
         nb = self.n_blocks
-        total = 2 * sum(self.block_bytes(b) for b in range(nb))
+        total = 2 * sum(self.copied_bytes(b) for b in range(nb))
         if not reuse_resident:
             return total
         k = min(n_slots, nb)
-        reused = sum(self.block_bytes(nb - 1 - j) for j in range(k)) + \
-            sum(self.block_bytes(j) for j in range(k))
+        reused = sum(self.copied_bytes(nb - 1 - j) for j in range(k)) + \
+            sum(self.copied_bytes(j) for j in range(k))
         return max(total - reused, 0)
+
+    def copied_bytes(self, b: int) -> int:
+        """Bytes this rank copies host -> device for block b: the whole block,
+        or its shard of it in a sharded stream."""
+        if not self.shard:
+            return self.block_bytes(b)
+        return hsnf4.shard_range(self.block_bytes(b), self.shard[1], self.shard[0])[2]
 
     def kernels_per_step(self) -> int:
         """Library kernels one step launches: per group, the forward runs the

@@ -351,6 +351,26 @@ typedef struct {
                        aligned) and acquire returns it with format BF16 */
 } hsnf4_layer_desc;
 
+/* Sharded streaming across the GPUs of one node (data-parallel ranks that
+ * stream the same stack).  No counterpart in the pages, which describe one
+ * GPU: each of `world` ranks copies 1/world of every block over its own
+ * PCIe link, then a gather enqueued on the copy stream rebuilds the whole
+ * block in every rank's slot over NVLink, so per-GPU PCIe bytes fall
+ * world-fold.  Block b of B bytes is cut into world shards of
+ * S = round_up(ceil(B / world), 1 KiB) bytes (the last ones shorter or
+ * empty); rank j's shard is bytes [j*S, min((j+1)*S, B)) and lands at the
+ * same offset of the slot.  The gather callback (block = the block being
+ * fetched, for the caller's bookkeeping) is called, with the
+ * streamer's lock held, right after this rank's shard copy is enqueued on
+ * copy_stream; it must enqueue on copy_stream the in-place all-gather that
+ * makes slot[j*S, (j+1)*S) hold rank j's shard for every j (for example
+ * NCCL all-gather with sendbuff = slot + rank*S, recvbuff = slot, count S),
+ * and return 0, or nonzero on failure (prefetch then fails with
+ * HSNF4_ERR_CUDA).  Every rank must make the same prefetch calls in the
+ * same order, since each one issues a collective. */
+typedef int (*hsnf4_gather_fn)(void *slot, size_t shard_bytes, int world, int block,
+                               void *copy_stream, void *user);
+
 typedef struct {
   int block_size;      /* layers per block, >= 1 */
   int enable_prefetch; /* 0: acquire() issues the copy itself (no overlap) */
@@ -362,6 +382,11 @@ typedef struct {
   int n_slots;         /* block slots in the ring: 0 (= 2, prefetch one
                           ahead) or 2..HSNF4_MAX_SLOTS; more slots reuse
                           more blocks at each forward/backward turn-around */
+  int shard_world;     /* ranks sharing the stream: 0 or 1 = not sharded
+                          (unless gather is set: then 1 rank, one shard) */
+  int shard_rank;      /* this rank, in [0, shard_world) */
+  hsnf4_gather_fn gather; /* required when shard_world >= 2; NULL otherwise */
+  void *gather_user;   /* passed to gather */
 } hsnf4_stream_config;
 
 typedef struct {
@@ -369,6 +394,7 @@ typedef struct {
   uint64_t copies;     /* H2D copies issued */
   uint64_t reuses;     /* prefetches satisfied by a resident block */
   uint64_t acquires, releases;
+  uint64_t gathers;    /* gather callbacks made (sharded streams) */
 } hsnf4_stream_stats;
 
 typedef struct hsnf4_streamer hsnf4_streamer;
@@ -393,6 +419,18 @@ int stream_ring_bytes(const hsnf4_layer_desc *layers, int n_layers,
  * n_slots times this. */
 int stream_slot_bytes(const hsnf4_layer_desc *layers, int n_layers,
                       int block_size, size_t *out_bytes);
+
+/* This rank's shard of a block of block_bytes bytes shared by world ranks:
+ * *shard_bytes = S (the stride), *off and *len the rank's byte range
+ * (len may be 0).  Pure host arithmetic. */
+int stream_shard_range(size_t block_bytes, int world, int rank, size_t *shard_bytes,
+                       size_t *off, size_t *len);
+
+/* Bytes of one block slot of a stream sharded over `world` ranks (the
+ * largest block rounded up to world * S); a ring of n_slots needs n_slots
+ * times this.  world 1 gives stream_slot_bytes rounded up to 1 KiB. */
+int stream_slot_bytes_sharded(const hsnf4_layer_desc *layers, int n_layers, int block_size,
+                              int world, size_t *out_bytes);
 
 /* Create a streamer.  pinned_slab: HOST pointer to page-locked memory of
  * slab_bytes holding the stack; ring_dev: device memory of ring_bytes

@@ -67,3 +67,56 @@ def test_single_rank_is_identity():
     hdist.allreduce_grads(flat)
     assert torch.equal(flat, torch.ones(4))
     assert hdist.job_throughput(512, 10, 1000.0, 1) == 5120.0
+
+
+# ---------------------------------------------------------------- sharded stream
+
+def test_shard_ranges_tile_every_block():
+    from host_streamed_nf4_b200 import hsnf4
+    for B in (1, 500, 1024, 1025, 5000, 131088384, 3 * 1024 * 1024 + 7):
+        for world in (1, 2, 3, 4, 8):
+            spans = [hsnf4.shard_range(B, world, r) for r in range(world)]
+            S = spans[0][0]
+            assert S % 1024 == 0 and world * S >= B and (S - 1024) * world < B
+            covered = 0
+            for r, (s_, off, n) in enumerate(spans):
+                assert s_ == S and off == r * S
+                assert n == max(0, min(S, B - off))
+                covered += n
+            assert covered == B
+
+
+def _gather_worker(rank, ws, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        from host_streamed_nf4_b200 import hsnf4
+        g = torch.Generator().manual_seed(5)
+        slab = torch.randint(0, 256, (20000,), dtype=torch.uint8, generator=g)  # same on all ranks
+        results = []
+        for B, slot_off in ((5000, 0), (500, 8192), (20000, 0)):
+            S, off, n = hsnf4.shard_range(B, ws, rank)
+            ring = torch.zeros(2 * ws * S + 8192, dtype=torch.uint8)
+            # this rank's shard lands at its offset, as the streamer's copy puts it
+            ring[slot_off + off: slot_off + off + n] = slab[off: off + n]
+            hdist.ring_gather(ring)(slot_off, S, ws, 0)
+            results.append(bool(torch.equal(ring[slot_off: slot_off + B], slab[:B])))
+        q.put((rank, results))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ring_gather_rebuilds_the_block_on_every_rank():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ok in results:
+        assert all(ok), (rank, ok)

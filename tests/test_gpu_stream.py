@@ -190,3 +190,57 @@ def test_prefetch_ahead_fills_free_slots_in_visit_order():
     torch.cuda.synchronize()
     assert st.stats()["copies"] == 3
     st.close()
+
+
+# ---------------------------------------------------------------- sharded stream, one GPU
+
+def _emulated_peers(holder):
+    """Gather factory that stands in for the other ranks on one GPU: it fills
+    their shards of the slot from the pinned slab (what their own PCIe copies
+    would have brought), enqueued on the copy stream like the all-gather."""
+    def factory(ring):
+        def gather(slot_off, S, world, block):
+            st = holder[0]
+            B = st.block_bytes(block)
+            base = block * st.block_size * st.layer_bytes
+            for j in range(world):
+                off = j * S
+                n = max(0, min(S, B - off))
+                if j != st.shard[0] and n:
+                    ring[slot_off + off: slot_off + off + n].copy_(
+                        st.slab[base + off: base + off + n], non_blocking=True)
+        return gather
+    return factory
+
+
+@pytest.mark.parametrize("world,rank,bs", [(2, 0, 1), (2, 1, 2), (4, 3, 1), (4, 2, 4)])
+def test_sharded_stream_equals_resident_bitwise(resident6, world, rank, bs):
+    holder = []
+    s = LayerStack(TINY, 6, 96, block_size=bs, streamed=True, shard=(rank, world,
+                                                                       _emulated_peers(holder)))
+    holder.append(s)
+    _assert_bitwise(_run(s), resident6)
+    st = s.streamer.stats()
+    assert st["gathers"] == st["copies"] > 0
+    # this rank's link moved only its shards
+    before = s.streamer.stats()["h2d_bytes"]
+    s.step()
+    torch.cuda.synchronize()
+    assert s.streamer.stats()["h2d_bytes"] - before == s.steady_h2d_bytes_per_step()
+    # about 1/world of the unsharded bytes (shards are 1 KiB-rounded)
+    full = sum(2 * s.block_bytes(b) for b in range(s.n_blocks))
+    assert s.steady_h2d_bytes_per_step() <= full / world + 2 * s.n_blocks * 1024
+    s.close()
+
+
+def test_gather_failure_is_reported():
+    def factory(ring):
+        def gather(slot_off, S, world, block):
+            raise RuntimeError("peer went away")
+        return gather
+    s = LayerStack(TINY, 2, 32, block_size=1, streamed=True, shard=(0, 2, factory))
+    with pytest.raises(hsnf4.HsNf4Error) as e:
+        s.step()
+    assert e.value.status == hsnf4.ERR_CUDA and "peer went away" in str(e.value)
+    torch.cuda.synchronize()
+    s.close()
