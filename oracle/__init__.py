@@ -91,6 +91,14 @@ def lib():
         L.orc_lora_bwd_drop.argtypes = [u8p, f32p, i64, i64, u16p, i64, u16p, u16p, i32,
                                         ctypes.c_float, ctypes.c_float, u64, u64, u16p, i64p,
                                         i64, f32p, f32p, f32p, i32]
+        L.orc_rmsnorm_fwd.argtypes = [f64p, f64p, i64, i64, ctypes.c_double, f64p]
+        L.orc_rmsnorm_bwd.argtypes = [f64p, f64p, f64p, i64, i64, ctypes.c_double, f64p]
+        L.orc_silu_mul_fwd.argtypes = [f64p, f64p, i64, f64p]
+        L.orc_silu_mul_bwd.argtypes = [f64p, f64p, f64p, i64, f64p, f64p]
+        L.orc_attention_fwd.argtypes = [f64p, f64p, f64p, i64, i32, i32, i32, ctypes.c_double,
+                                        f64p, f64p]
+        L.orc_attention_bwd.argtypes = [f64p, f64p, f64p, f64p, i64, i32, i32, i32,
+                                        ctypes.c_double, f64p, f64p, f64p]
         for fn in ("orc_nf4_quantize", "orc_nf4_dequant", "orc_lora_fwd", "orc_lora_bwd",
                    "orc_lora_fwd_bf16w", "orc_lora_bwd_bf16w", "orc_lora_merge",
                    "orc_dropout_keep", "orc_dropout_apply", "orc_lora_fwd_drop",
@@ -386,3 +394,64 @@ def lora_bwd_drop(codes, absmax, N, K, X, A, B, dY, alpha, p, seed, offset, rows
     if rc != 0:
         raise ValueError("orc_lora_bwd_drop rejected its arguments")
     return dX, dA, dB
+
+
+# ---------------------------------------------------------------- decoder glue
+
+def _d(a):
+    return _c(np.asarray(a, np.float64), np.float64)
+
+
+def rmsnorm_fwd(x, g, eps):
+    x, g = _d(x), _d(g)
+    T, n = x.shape
+    y = np.zeros_like(x)
+    f = ctypes.c_double
+    lib().orc_rmsnorm_fwd(_p(x, f), _p(g, f), T, n, float(eps), _p(y, f))
+    return y
+
+
+def rmsnorm_bwd(x, g, dy, eps):
+    x, g, dy = _d(x), _d(g), _d(dy)
+    T, n = x.shape
+    dx = np.zeros_like(x)
+    f = ctypes.c_double
+    lib().orc_rmsnorm_bwd(_p(x, f), _p(g, f), _p(dy, f), T, n, float(eps), _p(dx, f))
+    return dx
+
+
+def silu_mul_fwd(a, b):
+    a, b = _d(a), _d(b)
+    m = np.zeros_like(a)
+    f = ctypes.c_double
+    lib().orc_silu_mul_fwd(_p(a, f), _p(b, f), a.size, _p(m, f))
+    return m
+
+
+def silu_mul_bwd(a, b, dm):
+    a, b, dm = _d(a), _d(b), _d(dm)
+    da, db = np.zeros_like(a), np.zeros_like(a)
+    f = ctypes.c_double
+    lib().orc_silu_mul_bwd(_p(a, f), _p(b, f), _p(dm, f), a.size, _p(da, f), _p(db, f))
+    return da, db
+
+
+def attention_fwd(q, k, v, H, KV, d, scale):
+    q, k, v = _d(q), _d(k), _d(v)
+    T = q.shape[0]
+    o = np.zeros_like(q)
+    lse = np.zeros((H, T), np.float64)
+    f = ctypes.c_double
+    lib().orc_attention_fwd(_p(q, f), _p(k, f), _p(v, f), T, H, KV, d, float(scale), _p(o, f),
+                            _p(lse, f))
+    return o, lse
+
+
+def attention_bwd(q, k, v, do, H, KV, d, scale):
+    q, k, v, do = _d(q), _d(k), _d(v), _d(do)
+    T = q.shape[0]
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    f = ctypes.c_double
+    lib().orc_attention_bwd(_p(q, f), _p(k, f), _p(v, f), _p(do, f), T, H, KV, d, float(scale),
+                            _p(dq, f), _p(dk, f), _p(dv, f))
+    return dq, dk, dv

@@ -798,3 +798,147 @@ int orc_lora_bwd_drop(const uint8_t *codes, const float *absmax, int64_t N, int6
   return lora_bwd_src(&w, &d, N, K, X, T, A, B, r, alpha, dY, rows, n_rows, dX, dA, dB,
                       n_threads);
 }
+
+/* ======================================================================
+ * Decoder-layer glue around the seven projections (the pages train LoRA
+ * on Qwen2.5 / Llama-3.1 decoder layers and rematerialize each block in
+ * the backward -- Poros on consumer GPUs, "OOM playbook": activation
+ * memory at the rematerialization boundary).  Plain double arithmetic,
+ * row-major tensors; these are the textbook definitions.
+ * ====================================================================== */
+
+/* RMSNorm: y[t,i] = x[t,i] * g[i] / sqrt(mean_i x[t,i]^2 + eps) */
+void orc_rmsnorm_fwd(const double *x, const double *g, int64_t T, int64_t n, double eps,
+                     double *y) {
+  for (int64_t t = 0; t < T; ++t) {
+    double ss = 0.0;
+    for (int64_t i = 0; i < n; ++i) ss += x[t * n + i] * x[t * n + i];
+    const double r = 1.0 / sqrt(ss / (double)n + eps);
+    for (int64_t i = 0; i < n; ++i) y[t * n + i] = x[t * n + i] * r * g[i];
+  }
+}
+
+/* dx of RMSNorm (g frozen): with r = (mean x^2 + eps)^-1/2 and w = g * dy,
+ * dx_i = r w_i - r^3 x_i (sum_j w_j x_j) / n */
+void orc_rmsnorm_bwd(const double *x, const double *g, const double *dy, int64_t T,
+                     int64_t n, double eps, double *dx) {
+  for (int64_t t = 0; t < T; ++t) {
+    double ss = 0.0, wx = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+      ss += x[t * n + i] * x[t * n + i];
+      wx += g[i] * dy[t * n + i] * x[t * n + i];
+    }
+    const double r = 1.0 / sqrt(ss / (double)n + eps);
+    for (int64_t i = 0; i < n; ++i)
+      dx[t * n + i] = r * g[i] * dy[t * n + i] - r * r * r * x[t * n + i] * wx / (double)n;
+  }
+}
+
+/* SwiGLU gate: m = silu(a) * b, silu(a) = a / (1 + e^-a) */
+static double silu_d(double a) { return a / (1.0 + exp(-a)); }
+
+void orc_silu_mul_fwd(const double *a, const double *b, int64_t n, double *m) {
+  for (int64_t i = 0; i < n; ++i) m[i] = silu_d(a[i]) * b[i];
+}
+
+/* da = dm * b * silu'(a), silu'(a) = s (1 + a (1 - s)), s = 1/(1+e^-a); db = dm * silu(a) */
+void orc_silu_mul_bwd(const double *a, const double *b, const double *dm, int64_t n,
+                      double *da, double *db) {
+  for (int64_t i = 0; i < n; ++i) {
+    const double s = 1.0 / (1.0 + exp(-a[i]));
+    da[i] = dm[i] * b[i] * s * (1.0 + a[i] * (1.0 - s));
+    db[i] = dm[i] * a[i] * s;
+  }
+}
+
+/* Causal scaled dot-product attention with grouped KV heads.
+ * q [T, H*d], k and v [T, KV*d] (head h reads KV head h / (H/KV));
+ * o [T, H*d]; lse [H, T] = log sum_j exp(scale q_i . k_j) over j <= i. */
+void orc_attention_fwd(const double *q, const double *k, const double *v, int64_t T, int H,
+                       int KV, int d, double scale, double *o, double *lse) {
+  const int grp = H / KV;
+  double *p = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+  if (!p) return;
+  for (int h = 0; h < H; ++h) {
+    const int kh = h / grp;
+    for (int64_t i = 0; i < T; ++i) {
+      double mx = -INFINITY;
+      for (int64_t j = 0; j <= i; ++j) {
+        double s = 0.0;
+        for (int c = 0; c < d; ++c)
+          s += q[i * H * d + h * d + c] * k[j * KV * d + kh * d + c];
+        p[j] = s * scale;
+        if (p[j] > mx) mx = p[j];
+      }
+      double sum = 0.0;
+      for (int64_t j = 0; j <= i; ++j) {
+        p[j] = exp(p[j] - mx);
+        sum += p[j];
+      }
+      lse[(int64_t)h * T + i] = mx + log(sum);
+      for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int64_t j = 0; j <= i; ++j) acc += p[j] * v[j * KV * d + kh * d + c];
+        o[i * H * d + h * d + c] = acc / sum;
+      }
+    }
+  }
+  free(p);
+}
+
+/* Its gradients: with P the attention probabilities,
+ *   dV = P^T dO, dP = dO V^T, dS = P * (dP - rowsum(P * dP)),
+ *   dQ = scale dS K, dK = scale dS^T Q, summed over the query heads that
+ * share a KV head. */
+void orc_attention_bwd(const double *q, const double *k, const double *v, const double *dout,
+                       int64_t T, int H, int KV, int d, double scale, double *dq, double *dk,
+                       double *dv) {
+  const int grp = H / KV;
+  double *p = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+  double *dp = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+  if (!p || !dp) {
+    free(p);
+    free(dp);
+    return;
+  }
+  memset(dq, 0, sizeof(double) * (size_t)(T * H * d));
+  memset(dk, 0, sizeof(double) * (size_t)(T * KV * d));
+  memset(dv, 0, sizeof(double) * (size_t)(T * KV * d));
+  for (int h = 0; h < H; ++h) {
+    const int kh = h / grp;
+    for (int64_t i = 0; i < T; ++i) {
+      double mx = -INFINITY;
+      for (int64_t j = 0; j <= i; ++j) {
+        double s = 0.0;
+        for (int c = 0; c < d; ++c)
+          s += q[i * H * d + h * d + c] * k[j * KV * d + kh * d + c];
+        p[j] = s * scale;
+        if (p[j] > mx) mx = p[j];
+      }
+      double sum = 0.0;
+      for (int64_t j = 0; j <= i; ++j) {
+        p[j] = exp(p[j] - mx);
+        sum += p[j];
+      }
+      double pdp = 0.0;
+      for (int64_t j = 0; j <= i; ++j) {
+        p[j] /= sum;
+        double s = 0.0;
+        for (int c = 0; c < d; ++c)
+          s += dout[i * H * d + h * d + c] * v[j * KV * d + kh * d + c];
+        dp[j] = s;
+        pdp += p[j] * s;
+      }
+      for (int64_t j = 0; j <= i; ++j) {
+        const double ds = p[j] * (dp[j] - pdp);
+        for (int c = 0; c < d; ++c) {
+          dv[j * KV * d + kh * d + c] += p[j] * dout[i * H * d + h * d + c];
+          dq[i * H * d + h * d + c] += scale * ds * k[j * KV * d + kh * d + c];
+          dk[j * KV * d + kh * d + c] += scale * ds * q[i * H * d + h * d + c];
+        }
+      }
+    }
+  }
+  free(p);
+  free(dp);
+}

@@ -163,6 +163,24 @@ int orc_lora_merge(const uint8_t *codes, const float *absmax, const uint16_t *Wb
                    int64_t N, int64_t K, const uint16_t *A, const uint16_t *B, int r,
                    float alpha, uint16_t *out);
 
+/* ---- decoder-layer glue (double, row-major; textbook definitions) ---- */
+/* RMSNorm y = x g / sqrt(mean x^2 + eps) over rows of n; and its dx (g frozen). */
+void orc_rmsnorm_fwd(const double *x, const double *g, int64_t T, int64_t n, double eps,
+                     double *y);
+void orc_rmsnorm_bwd(const double *x, const double *g, const double *dy, int64_t T,
+                     int64_t n, double eps, double *dx);
+/* SwiGLU gate m = silu(a) b, and its gradients. */
+void orc_silu_mul_fwd(const double *a, const double *b, int64_t n, double *m);
+void orc_silu_mul_bwd(const double *a, const double *b, const double *dm, int64_t n,
+                      double *da, double *db);
+/* Causal SDPA, H query heads sharing KV heads in groups of H/KV: q [T,H*d],
+ * k, v [T,KV*d], o [T,H*d], lse [H,T]; and its gradients. */
+void orc_attention_fwd(const double *q, const double *k, const double *v, int64_t T, int H,
+                       int KV, int d, double scale, double *o, double *lse);
+void orc_attention_bwd(const double *q, const double *k, const double *v, const double *dout,
+                       int64_t T, int H, int KV, int d, double scale, double *dq, double *dk,
+                       double *dv);
+
 #ifdef __cplusplus
 }
 #endif

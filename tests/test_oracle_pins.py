@@ -582,3 +582,125 @@ def test_dropout_wrapper_is_the_masked_core(orc):
     assert np.array_equal(dX, dXc.astype(np.float32))
     assert np.array_equal(dA, dAc.astype(np.float32))
     assert np.array_equal(dB, dBc.astype(np.float32))
+
+
+# ---------------------------------------------------------------- decoder glue
+
+def _fd_check(f, x, grad, n=10, h=1e-4, seed=0, tol=1e-6):
+    """Central differences of the scalar f at n random entries of x."""
+    rng = np.random.default_rng(seed)
+    for _ in range(n):
+        idx = tuple(int(rng.integers(0, s)) for s in x.shape)
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += h
+        xm[idx] -= h
+        fd = (f(xp) - f(xm)) / (2 * h)
+        assert abs(fd - grad[idx]) <= tol * max(1.0, abs(fd)), (idx, fd, grad[idx])
+
+
+def test_rmsnorm_unit_rms_scale_invariance_and_gradient(orc):
+    rng = np.random.default_rng(40)
+    x = rng.standard_normal((5, 64))
+    y = orc.rmsnorm_fwd(x, np.ones(64), 0.0)
+    assert np.allclose(np.mean(y * y, axis=1), 1.0, rtol=0, atol=1e-12)
+    assert np.allclose(orc.rmsnorm_fwd(7.5 * x, np.ones(64), 0.0), y, rtol=0, atol=1e-12)
+    g = rng.standard_normal(64)
+    assert np.allclose(orc.rmsnorm_fwd(x, g, 0.0), y * g[None, :], rtol=0, atol=1e-12)
+    G = rng.standard_normal((5, 64))
+    dx = orc.rmsnorm_bwd(x, g, G, 1e-6)
+    _fd_check(lambda x_: float(np.sum(G * orc.rmsnorm_fwd(x_, g, 1e-6))), x, dx, seed=41)
+
+
+def test_silu_mul_closed_forms_and_gradient(orc):
+    a = np.array([0.0, 30.0, -30.0, 1.0])
+    b = np.array([2.0, 1.0, 1.0, 1.0])
+    m = orc.silu_mul_fwd(a, b)
+    assert m[0] == 0.0 and abs(m[1] - 30.0) < 1e-9 and abs(m[2]) < 1e-9
+    assert abs(m[3] - 1.0 / (1.0 + np.exp(-1.0))) < 1e-15
+    da, db = orc.silu_mul_bwd(a, b, np.ones(4))
+    assert da[0] == 0.5 * 2.0 and db[0] == 0.0  # silu'(0) = 1/2, silu(0) = 0
+    rng = np.random.default_rng(42)
+    A, B, G = (rng.standard_normal((6, 8)) for _ in range(3))
+    dA, dB = orc.silu_mul_bwd(A, B, G)
+    _fd_check(lambda a_: float(np.sum(G * orc.silu_mul_fwd(a_, B))), A, dA, seed=43)
+    _fd_check(lambda b_: float(np.sum(G * orc.silu_mul_fwd(A, b_))), B, dB, seed=44)
+
+
+def test_attention_special_cases(orc):
+    rng = np.random.default_rng(45)
+    T, H, KV, d = 6, 4, 2, 8
+    q, k, v = (rng.standard_normal((T, n * d)) for n in (H, KV, KV))
+    # one token: each head returns its KV head's value
+    o1, lse1 = orc.attention_fwd(q[:1], k[:1], v[:1], H, KV, d, 0.3)
+    for h in range(H):
+        kh = h // (H // KV)
+        assert np.allclose(o1[0, h * d:(h + 1) * d], v[0, kh * d:(kh + 1) * d], rtol=0, atol=1e-15)
+    # zero queries: uniform weights over the causal prefix -> running mean of v
+    o0, lse0 = orc.attention_fwd(np.zeros_like(q), k, v, H, KV, d, 0.3)
+    for h in range(H):
+        kh = h // (H // KV)
+        vh = v[:, kh * d:(kh + 1) * d]
+        ref = np.cumsum(vh, axis=0) / np.arange(1, T + 1)[:, None]
+        assert np.allclose(o0[:, h * d:(h + 1) * d], ref, rtol=0, atol=1e-13)
+        assert np.allclose(lse0[h], np.log(np.arange(1, T + 1)), rtol=0, atol=1e-13)
+    # causality: the first i rows do not see tokens after i
+    o, _ = orc.attention_fwd(q, k, v, H, KV, d, 0.3)
+    k2, v2 = k.copy(), v.copy()
+    k2[4:] += 5.0
+    v2[4:] -= 3.0
+    o2, _ = orc.attention_fwd(q, k2, v2, H, KV, d, 0.3)
+    assert np.array_equal(o[:4], o2[:4]) and not np.allclose(o[4:], o2[4:])
+
+
+def test_attention_gradient_matches_finite_differences(orc):
+    rng = np.random.default_rng(46)
+    T, H, KV, d, sc = 5, 4, 2, 8, 0.35
+    q, k, v = (rng.standard_normal((T, n * d)) for n in (H, KV, KV))
+    G = rng.standard_normal((T, H * d))
+    dq, dk, dv = orc.attention_bwd(q, k, v, G, H, KV, d, sc)
+    loss = lambda q_, k_, v_: float(np.sum(G * orc.attention_fwd(q_, k_, v_, H, KV, d, sc)[0]))
+    _fd_check(lambda x: loss(x, k, v), q, dq, seed=47)
+    _fd_check(lambda x: loss(q, x, v), k, dk, seed=48)
+    _fd_check(lambda x: loss(q, k, x), v, dv, seed=49)
+
+
+def test_decoder_layer_wiring_matches_finite_differences(orc):
+    """The layer composition with exact arithmetic (no bf16 rounding, dense
+    double projections) against central differences of <G, h2>: dh0 and
+    the adapter gradients of every projection."""
+    from oracle import decoder as dec
+    rng = np.random.default_rng(50)
+    T, hid, H, KV, d, inter, r = 5, 16, 4, 2, 4, 24, 2
+    shapes = {"q": (H * d, hid), "k": (KV * d, hid), "v": (KV * d, hid), "o": (hid, H * d),
+              "gate": (inter, hid), "up": (inter, hid), "down": (hid, inter)}
+    lin = {n: dec.Linear(N, K, A=rng.standard_normal((r, K)) * 0.3,
+                         B=rng.standard_normal((N, r)) * 0.3,
+                         W=rng.standard_normal((N, K)) / np.sqrt(K))
+           for n, (N, K) in shapes.items()}
+    layer = dec.Layer(H=H, KV=KV, d=d, g1=1 + 0.1 * rng.standard_normal(hid),
+                      g2=1 + 0.1 * rng.standard_normal(hid), lin=lin, alpha=4.0)
+    ident = lambda x: x
+    h0 = rng.standard_normal((T, hid))
+    G = rng.standard_normal((T, hid))
+    s = dec.layer_forward(layer, h0, rnd=ident)
+    dh0, grads = dec.layer_backward(layer, s, G, rnd=ident)
+    loss = lambda: float(np.sum(G * dec.layer_forward(layer, h0_[0], rnd=ident)["h2"]))
+    h0_ = [h0]
+
+    def f_h0(x):
+        h0_[0] = x
+        return loss()
+    _fd_check(f_h0, h0, dh0, n=12, seed=51)
+    h0_[0] = h0
+    for name in dec.PROJ:
+        dA, dB = grads[name]
+        L = lin[name]
+        for M, g in ((L.A, dA), (L.B, dB)):
+            base = M.copy()
+
+            def f(x, M=M, base=base):
+                M[...] = x
+                out = loss()
+                M[...] = base
+                return out
+            _fd_check(f, base, g, n=4, seed=52)
