@@ -27,7 +27,7 @@ CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-Wall",
           "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr"]
 SOURCES = ["api.cu", "nf4_codec.cu", "lora_aux.cu", "lora_gemm.cu", "streamer.cpp", "profile.cpp",
            "noalloc.cu", "lora_merge.cu",
-           "lora_dropout.cu"]
+           "lora_dropout.cu", "glue.cu", "attention.cu"]
 
 
 def _headers_mtime() -> float:

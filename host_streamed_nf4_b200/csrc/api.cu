@@ -503,6 +503,117 @@ int lora_dropout_apply(const void* X, int64_t T, int64_t k_in, float p, uint64_t
                      "lora_dropout_apply launch");
 }
 
+// ---------------------------------------------------------------- decoder glue
+
+static int check_rows(const char* fn, int64_t T, int64_t n) {
+  if (T < 1 || n < 8 || n % 8 || T > (int64_t(1) << 31) || n > (int64_t(1) << 30))
+    return fail(HSNF4_ERR_INVALID, "%s: need T >= 1 and n a positive multiple of 8 (got T=%lld, "
+                "n=%lld)", fn, (long long)T, (long long)n);
+  return HSNF4_OK;
+}
+
+static int check_elems(const char* fn, int64_t n) {
+  if (n < 8 || n % 8)
+    return fail(HSNF4_ERR_INVALID, "%s: need a positive multiple of 8 elements (got %lld)", fn,
+                (long long)n);
+  return HSNF4_OK;
+}
+
+static int check_opt(const char* fn, const void* p, const char* name) {
+  if (p && !aligned16(p)) return fail(HSNF4_ERR_INVALID, "%s: %s is not 16-byte aligned", fn, name);
+  return HSNF4_OK;
+}
+
+int decoder_rmsnorm_fwd(const void* xa, const void* xb, const void* g, void* h_out, void* y,
+                        int64_t T, int64_t n, float eps, void* stream) {
+  static const char* fn = "decoder_rmsnorm_fwd";
+  int rc = check_rows(fn, T, n);
+  if (!rc) rc = check_ptrs(fn, {{xa, "xa"}, {g, "g"}, {y, "y"}});
+  if (!rc) rc = check_opt(fn, xb, "xb");
+  if (!rc && xb) rc = check_ptrs(fn, {{h_out, "h_out"}});
+  if (!rc && !(eps >= 0.0f)) rc = fail(HSNF4_ERR_INVALID, "%s: eps must be >= 0", fn);
+  if (rc) return rc;
+  return cuda_status(launch_rmsnorm_fwd(xa, xb, g, h_out, y, T, n, eps,
+                                        static_cast<cudaStream_t>(stream)),
+                     "decoder_rmsnorm_fwd launch");
+}
+
+int decoder_rmsnorm_bwd(const void* x, const void* g, const void* dy1, const void* dy2,
+                        const void* dy3, const void* dres, void* dx, int64_t T, int64_t n,
+                        float eps, void* stream) {
+  static const char* fn = "decoder_rmsnorm_bwd";
+  int rc = check_rows(fn, T, n);
+  if (!rc) rc = check_ptrs(fn, {{x, "x"}, {g, "g"}, {dy1, "dy1"}, {dx, "dx"}});
+  if (!rc) rc = check_opt(fn, dy2, "dy2");
+  if (!rc) rc = check_opt(fn, dy3, "dy3");
+  if (!rc) rc = check_opt(fn, dres, "dres");
+  if (!rc && !(eps >= 0.0f)) rc = fail(HSNF4_ERR_INVALID, "%s: eps must be >= 0", fn);
+  if (rc) return rc;
+  return cuda_status(launch_rmsnorm_bwd(x, g, dy1, dy2, dy3, dres, dx, T, n, eps,
+                                        static_cast<cudaStream_t>(stream)),
+                     "decoder_rmsnorm_bwd launch");
+}
+
+int decoder_swiglu_fwd(const void* a, const void* b, void* m, int64_t n, void* stream) {
+  static const char* fn = "decoder_swiglu_fwd";
+  int rc = check_elems(fn, n);
+  if (!rc) rc = check_ptrs(fn, {{a, "a"}, {b, "b"}, {m, "m"}});
+  if (rc) return rc;
+  return cuda_status(launch_silu_mul_fwd(a, b, m, n, static_cast<cudaStream_t>(stream)),
+                     "decoder_swiglu_fwd launch");
+}
+
+int decoder_swiglu_bwd(const void* a, const void* b, const void* dm, void* da, void* db, int64_t n,
+                       void* stream) {
+  static const char* fn = "decoder_swiglu_bwd";
+  int rc = check_elems(fn, n);
+  if (!rc) rc = check_ptrs(fn, {{a, "a"}, {b, "b"}, {dm, "dm"}, {da, "da"}, {db, "db"}});
+  if (rc) return rc;
+  return cuda_status(launch_silu_mul_bwd(a, b, dm, da, db, n, static_cast<cudaStream_t>(stream)),
+                     "decoder_swiglu_bwd launch");
+}
+
+int decoder_add(const void* x, const void* y, void* out, int64_t n, void* stream) {
+  static const char* fn = "decoder_add";
+  int rc = check_elems(fn, n);
+  if (!rc) rc = check_ptrs(fn, {{x, "x"}, {y, "y"}, {out, "out"}});
+  if (rc) return rc;
+  return cuda_status(launch_add(x, y, out, n, static_cast<cudaStream_t>(stream)),
+                     "decoder_add launch");
+}
+
+static int check_attn(const char* fn, int64_t T, int H, int KV) {
+  if (T < 1 || T > 32768 || H < 1 || KV < 1 || H % KV)
+    return fail(HSNF4_ERR_INVALID, "%s: need 1 <= T <= 32768 and H a multiple of KV (got T=%lld, "
+                "H=%d, KV=%d)", fn, (long long)T, H, KV);
+  return HSNF4_OK;
+}
+
+int decoder_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int64_t T, int H, int KV, void* stream) {
+  static const char* fn = "decoder_attention_fwd";
+  int rc = check_attn(fn, T, H, KV);
+  if (!rc) rc = check_ptrs(fn, {{q, "q"}, {k, "k"}, {v, "v"}, {o, "o"}, {lse, "lse"}});
+  if (rc) return rc;
+  return cuda_status(launch_attention_fwd(q, k, v, o, lse, T, H, KV, 1.0f / sqrtf(128.0f),
+                                          static_cast<cudaStream_t>(stream)),
+                     "decoder_attention_fwd launch");
+}
+
+int decoder_attention_bwd(const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                          float* scratch, int64_t T, int H, int KV, void* stream) {
+  static const char* fn = "decoder_attention_bwd";
+  int rc = check_attn(fn, T, H, KV);
+  if (!rc)
+    rc = check_ptrs(fn, {{q, "q"}, {k, "k"}, {v, "v"}, {o, "o"}, {lse, "lse"}, {dout, "dout"},
+                         {dq, "dq"}, {dk, "dk"}, {dv, "dv"}, {scratch, "scratch"}});
+  if (rc) return rc;
+  return cuda_status(launch_attention_bwd(q, k, v, o, lse, dout, dq, dk, dv, scratch, T, H, KV,
+                                          1.0f / sqrtf(128.0f), static_cast<cudaStream_t>(stream)),
+                     "decoder_attention_bwd launch");
+}
+
 static hsnf4_lora_fwd_args one_fwd(const hsnf4_nf4_weight* W, const void* X, const void* A,
                                    const void* B, void* Y, float* t_save) {
   hsnf4_lora_fwd_args a;

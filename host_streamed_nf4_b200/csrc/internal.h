@@ -108,6 +108,24 @@ cudaError_t launch_dropout_apply(const DropDesc* d, int n, int64_t T, cudaStream
 cudaError_t launch_dx_dropout_add(const DropDesc* d, int n, int64_t T, int r, float s,
                                   cudaStream_t st);
 
+// ---- decoder glue (glue.cu, attention.cu)
+cudaError_t launch_rmsnorm_fwd(const void* xa, const void* xb, const void* g, void* h_out,
+                               void* y, int64_t T, int64_t n, float eps, cudaStream_t st);
+cudaError_t launch_rmsnorm_bwd(const void* x, const void* g, const void* dy1, const void* dy2,
+                               const void* dy3, const void* dres, void* dx, int64_t T, int64_t n,
+                               float eps, cudaStream_t st);
+cudaError_t launch_silu_mul_fwd(const void* a, const void* b, void* m, int64_t n,
+                                cudaStream_t st);
+cudaError_t launch_silu_mul_bwd(const void* a, const void* b, const void* dm, void* da, void* db,
+                                int64_t n, cudaStream_t st);
+cudaError_t launch_add(const void* x, const void* y, void* out, int64_t n, cudaStream_t st);
+cudaError_t launch_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 int64_t T, int H, int KV, float scale, cudaStream_t st);
+cudaError_t launch_attention_bwd(const void* q, const void* k, const void* v, const void* o,
+                                 const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                 float* D, int64_t T, int H, int KV, float scale,
+                                 cudaStream_t st);
+
 // Kernel timing (hsnf4_profile): bracket a launch with prof_begin/prof_end.
 enum ProfKind { kProfGemmFwd = 0, kProfGemmDx = 1, kProfDequant = 2, kProfMerge = 3, kProfKinds = 4 };
 bool profiling();

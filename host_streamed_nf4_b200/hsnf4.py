@@ -90,6 +90,19 @@ _SIGS = {
     "nf4_dequant": ([c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p], c_int),
     "lora_merge": ([POINTER(Nf4WeightC), c_void_p, c_void_p, c_int, c_float, c_void_p, c_void_p],
                    c_int),
+    "decoder_rmsnorm_fwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64,
+                             c_float, c_void_p], c_int),
+    "decoder_rmsnorm_bwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                             c_int64, c_int64, c_float, c_void_p], c_int),
+    "decoder_swiglu_fwd": ([c_void_p, c_void_p, c_void_p, c_int64, c_void_p], c_int),
+    "decoder_swiglu_bwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_void_p],
+                           c_int),
+    "decoder_add": ([c_void_p, c_void_p, c_void_p, c_int64, c_void_p], c_int),
+    "decoder_attention_fwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int,
+                               c_int, c_void_p], c_int),
+    "decoder_attention_bwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                               c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int, c_int,
+                               c_void_p], c_int),
     "lora_dropout_apply": ([c_void_p, c_int64, c_int64, c_float, c_uint64, c_uint64, c_void_p,
                             c_void_p], c_int),
     "lora_linear_fwd_workspace": ([c_int64, c_int64, c_int64, c_int], c_size_t),
@@ -284,6 +297,79 @@ def lora_merge(W, A: torch.Tensor, B: torch.Tensor, alpha: float, out=None, stre
     _check(lib().lora_merge(_weight_arg(W), _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
                             _stream(stream)))
     return out
+
+
+# ------------------------------------------------------------------ decoder glue
+
+def _pp(t):
+    return None if t is None else _ptr(t)
+
+
+def rmsnorm_fwd(x, g, eps, res=None, h_out=None, y=None, stream=None):
+    """y = rmsnorm(x [+ res]) (bf16 [T, n]); with res, h_out receives x + res."""
+    T, n = x.shape
+    if y is None:
+        y = torch.empty_like(x)
+    if res is not None and h_out is None:
+        h_out = torch.empty_like(x)
+    _check(lib().decoder_rmsnorm_fwd(_ptr(x), _pp(res), _ptr(g), _pp(h_out), _ptr(y), T, n,
+                                     float(eps), _stream(stream)))
+    return (y, h_out) if res is not None else y
+
+
+def rmsnorm_bwd(x, g, dys, eps, dres=None, dx=None, stream=None):
+    """dx = dres + drmsnorm(x)/dx . sum(dys) (1..3 bf16 branch gradients)."""
+    T, n = x.shape
+    if dx is None:
+        dx = torch.empty_like(x)
+    d = list(dys) + [None] * (3 - len(dys))
+    _check(lib().decoder_rmsnorm_bwd(_ptr(x), _ptr(g), _ptr(d[0]), _pp(d[1]), _pp(d[2]), _pp(dres),
+                                     _ptr(dx), T, n, float(eps), _stream(stream)))
+    return dx
+
+
+def swiglu_fwd(a, b, m=None, stream=None):
+    if m is None:
+        m = torch.empty_like(a)
+    _check(lib().decoder_swiglu_fwd(_ptr(a), _ptr(b), _ptr(m), a.numel(), _stream(stream)))
+    return m
+
+
+def swiglu_bwd(a, b, dm, da=None, db=None, stream=None):
+    da = torch.empty_like(a) if da is None else da
+    db = torch.empty_like(a) if db is None else db
+    _check(lib().decoder_swiglu_bwd(_ptr(a), _ptr(b), _ptr(dm), _ptr(da), _ptr(db), a.numel(),
+                                    _stream(stream)))
+    return da, db
+
+
+def add(x, y, out=None, stream=None):
+    out = torch.empty_like(x) if out is None else out
+    _check(lib().decoder_add(_ptr(x), _ptr(y), _ptr(out), x.numel(), _stream(stream)))
+    return out
+
+
+def attention_fwd(q, k, v, H, KV, o=None, lse=None, stream=None):
+    T = q.shape[0]
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty(H, T, dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(lib().decoder_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), T, H, KV,
+                                       _stream(stream)))
+    return o, lse
+
+
+def attention_bwd(q, k, v, o, lse, dout, H, KV, dq=None, dk=None, dv=None, scratch=None,
+                  stream=None):
+    T = q.shape[0]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if scratch is None:
+        scratch = torch.empty(H, T, dtype=torch.float32, device=q.device)
+    _check(lib().decoder_attention_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                       _ptr(dq), _ptr(dk), _ptr(dv), _ptr(scratch), T, H, KV,
+                                       _stream(stream)))
+    return dq, dk, dv
 
 
 # ------------------------------------------------------------------ LoRA linear

@@ -313,6 +313,53 @@ int lora_group_bwd(const hsnf4_lora_bwd_args *probs, int n, int64_t T, int r, fl
                    void *workspace, size_t ws_bytes, void *stream);
 
 /* ----------------------------------------------------------------------- */
+/* Decoder-layer glue around the projections                               */
+/* ----------------------------------------------------------------------- */
+/* The pages train LoRA on Qwen2.5 / Llama-3.1 decoder layers and recompute
+ * each block's forward inside its backward (Poros on consumer GPUs, "OOM
+ * playbook": activation memory at the rematerialization boundary; Poros API
+ * reference, patch_hf_model).  These are the layer's other pieces: pre-norm
+ * RMSNorm, causal grouped-query SDPA (head_dim 128, no rotary embedding),
+ * the SwiGLU gate and the residual adds.  Tensors are row-major bf16 [T, n]
+ * device arrays, 16-byte aligned, n a multiple of 8; every output is rounded
+ * once to bf16 from fp32 arithmetic; results do not depend on timing.
+ * Errors: INVALID (sizes, pointers), CUDA. */
+
+/* y = x g / sqrt(mean x^2 + eps) per row, x = xa, or x = bf16(xa + xb)
+ * (written to h_out) when xb is not NULL -- the residual add fused in front
+ * of the norm.  g bf16 [n]. */
+int decoder_rmsnorm_fwd(const void *xa, const void *xb, const void *g, void *h_out, void *y,
+                        int64_t T, int64_t n, float eps, void *stream);
+
+/* dx = bf16(dres + dRMSNorm/dx . (dy1 + dy2 + dy3)) with x the norm's input
+ * (g frozen: no dg); dy2, dy3, dres may be NULL.  The branch gradients are
+ * summed in fp32. */
+int decoder_rmsnorm_bwd(const void *x, const void *g, const void *dy1, const void *dy2,
+                        const void *dy3, const void *dres, void *dx, int64_t T, int64_t n,
+                        float eps, void *stream);
+
+/* m = silu(a) b (n elements); da = dm b silu'(a), db = dm silu(a). */
+int decoder_swiglu_fwd(const void *a, const void *b, void *m, int64_t n, void *stream);
+int decoder_swiglu_bwd(const void *a, const void *b, const void *dm, void *da, void *db,
+                       int64_t n, void *stream);
+
+/* out = x + y (n elements; out may alias x or y). */
+int decoder_add(const void *x, const void *y, void *out, int64_t n, void *stream);
+
+/* Causal SDPA with H query heads over KV heads (H % KV == 0; head h reads
+ * KV head h / (H / KV)), head_dim 128, scale 1/sqrt(128):  q, o [T, H*128],
+ * k, v [T, KV*128]; lse fp32 [H, T] (log-sum-exp of the scaled scores, kept
+ * for the backward). */
+int decoder_attention_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                          int64_t T, int H, int KV, void *stream);
+
+/* Its gradients from the forward's o and lse:  dq [T, H*128], dk, dv
+ * [T, KV*128] (overwritten); scratch fp32 [H, T] (caller-owned). */
+int decoder_attention_bwd(const void *q, const void *k, const void *v, const void *o,
+                          const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                          float *scratch, int64_t T, int H, int KV, void *stream);
+
+/* ----------------------------------------------------------------------- */
 /* Host-pinned NF4 base -> VRAM ring streamer                              */
 /* ----------------------------------------------------------------------- */
 /* HN comment: the base sits in host RAM and streams into a small pool of

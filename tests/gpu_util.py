@@ -26,7 +26,7 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def assert_lora_close(got, ref, what=""):
+def assert_lora_close(got, ref, what="", max_rel=MAX_REL, fro_rel=FRO_REL):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
@@ -34,6 +34,6 @@ def assert_lora_close(got, ref, what=""):
     d = np.abs(got - ref)
     scale = np.abs(ref).max()
     fro = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
-    assert d.max() <= MAX_REL * scale, f"{what}: max|d| {d.max():.3e} > {MAX_REL} * {scale:.3e}"
-    assert fro <= FRO_REL, f"{what}: rel Frobenius {fro:.3e} > {FRO_REL}"
+    assert d.max() <= max_rel * scale, f"{what}: max|d| {d.max():.3e} > {max_rel} * {scale:.3e}"
+    assert fro <= fro_rel, f"{what}: rel Frobenius {fro:.3e} > {fro_rel}"
     return (d.max() / scale if scale > 0 else 0.0), fro

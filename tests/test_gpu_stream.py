@@ -244,3 +244,50 @@ def test_gather_failure_is_reported():
     assert e.value.status == hsnf4.ERR_CUDA and "peer went away" in str(e.value)
     torch.cuda.synchronize()
     s.close()
+
+
+_NCCL_CHILD = r"""
+import os, sys, datetime, torch
+import torch.distributed as dist
+sys.path.insert(0, os.environ["REPO"])
+from host_streamed_nf4_b200 import dist as hdist, synth
+from host_streamed_nf4_b200.stack import LayerStack
+dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                        init_method="tcp://127.0.0.1:%s" % os.environ["PORT"],
+                        device_id=torch.device("cuda", 0))
+fam = synth.Family("tiny", hidden=256, inter=640, heads=2, kv_heads=1, head_dim=128, layers=4)
+def run(st):
+    out = []
+    for _ in range(2):
+        st.step()
+    torch.cuda.synchronize()
+    return [t.clone() for t in [st.grad_flat] + st.Y + st.dX]
+ref = LayerStack(fam, 4, 64, streamed=False)
+a = run(ref)
+ref.close()
+sh = LayerStack(fam, 4, 64, block_size=2, streamed=True, shard=(0, 1, hdist.ring_gather))
+b = run(sh)
+gathers = sh.streamer.stats()["gathers"]
+sh.close()
+ok = all(torch.equal(x, y) for x, y in zip(a, b)) and gathers > 0
+dist.destroy_process_group()
+print("NCCL_GATHER_OK" if ok else "NCCL_GATHER_MISMATCH")
+"""
+
+
+def test_nccl_ring_gather_on_one_rank():
+    """The real NCCL gather path (in-place all_gather_into_tensor on the copy
+    stream, called back from the streamer) with a one-rank process group."""
+    import os
+    import socket
+    import subprocess
+    import sys
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    repo = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, REPO=repo, PORT=str(port), NCCL_NVLS_ENABLE="0")
+    r = subprocess.run([sys.executable, "-c", _NCCL_CHILD], env=env, capture_output=True,
+                       text=True, timeout=300)
+    assert "NCCL_GATHER_OK" in r.stdout, (r.stdout[-2000:], r.stderr[-2000:])
