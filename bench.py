@@ -64,6 +64,10 @@ def parse():
                     help="how a layer's projections are batched into grouped launches")
     ap.add_argument("--base", choices=["nf4", "bf16"], default="nf4",
                     help="frozen base format: NF4 (default) or dense bf16 (bf16_bitwise)")
+    ap.add_argument("--model", choices=["projections", "decoder"], default="projections",
+                    help="projections: the 7 LoRA linears per layer on seeded inputs; decoder: "
+                         "full decoder layers (norms, attention, SwiGLU, residuals) with "
+                         "per-block rematerialization")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="LoRA dropout on the adapter branch (the configs use 0)")
     ap.add_argument("--no-shard-h2d", dest="shard_h2d", action="store_false",
@@ -254,7 +258,11 @@ def run_ours(args, ws, rank, local):
     # stream too: each copies 1/N of every block and an NCCL all-gather on
     # the copy stream rebuilds the block in every ring
     shard = (rank, ws, hdist.ring_gather) if (streamed and ws > 1 and args.shard_h2d) else None
-    stack = LayerStack(fam, args.layers, args.seq, block_size=args.block_size, streamed=streamed,
+    from host_streamed_nf4_b200.decoder import DecoderStack
+    cls = DecoderStack if args.model == "decoder" else LayerStack
+    if args.model == "decoder":
+        args.grouping = "decoder"
+    stack = cls(fam, args.layers, args.seq, block_size=args.block_size, streamed=streamed,
                        reuse_resident=not single, seed=42, data_seed=42 + rank, device=dev,
                        shard=shard,
                        grouping=args.grouping, n_slots=args.slots, base=args.base,
@@ -342,6 +350,13 @@ def run_ours(args, ws, rank, local):
     flops_step = sum(2.0 * args.seq * n * k * 2 for _, n, k in fam.projections()) * args.layers
     flops_step += sum(2.0 * args.seq * stack.r * (2 * k + 2 * n) + 2.0 * args.seq * stack.r * (k + n)
                       for _, n, k in fam.projections()) * args.layers
+    if args.model == "decoder":
+        # the backward recomputes each block's forward: the projections' forward
+        # again, plus causal attention (forward, its recompute, backward ~3.5x)
+        flops_step += sum(2.0 * args.seq * n * (k + stack.r) + 2.0 * args.seq * stack.r * k
+                          for _, n, k in fam.projections()) * args.layers
+        attn_fwd = 2.0 * args.seq * args.seq * fam.head_dim * fam.heads
+        flops_step += (2 * attn_fwd + 3.5 * attn_fwd) * args.layers
     link = link_probe(stack, dev) if streamed else None
     roofline["cublas_same_shapes"] = cublas_probe(fam, args.seq, dom, dev)
     roofline["frac_vs_cublas_same_shapes"] = round(
@@ -370,7 +385,8 @@ def run_ours(args, ws, rank, local):
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded normal weights/activations; no dataset)",
-        "config": {"workload": args.workload, "family": args.family, "layers": args.layers,
+        "config": {"workload": args.workload + ("-decoder" if args.model == "decoder" else ""),
+                   "model": args.model, "family": args.family, "layers": args.layers,
                    "tokens": args.seq, "batch": 1, "mode": args.mode, "base": args.base,
                    "dropout": args.dropout,
                    "block_size": args.block_size, "rank": stack.r, "alpha": stack.alpha,
@@ -538,22 +554,18 @@ def run_e2e(args, stack, one_step, drain_copies, ws, dev):
     its activations and upstream gradients from pinned host memory and reads
     the layer stack's adapter gradients back (device-timed)."""
     import torch
-    host_in = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in stack.X.items()}
-    host_dy = [torch.empty_like(v, device="cpu").pin_memory() for v in stack.dY]
-    for k, v in stack.X.items():
-        host_in[k].copy_(v)
-    for h, v in zip(host_dy, stack.dY):
+    dev_in = stack.step_inputs()  # the tensors a step reads from the host
+    host_in = [torch.empty_like(v, device="cpu").pin_memory() for v in dev_in]
+    for h, v in zip(host_in, dev_in):
         h.copy_(v)
     grads = [stack.grad_flat]  # every dA/dB of the stack, summed over ranks
     host_grads = [torch.empty_like(g, device="cpu").pin_memory() for g in grads]
-    h2d = sum(t.numel() * t.element_size() for t in list(host_in.values()) + host_dy)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_grads)
     compute = stack.compute
 
     def step_e2e():
-        for k, v in stack.X.items():
-            v.copy_(host_in[k], non_blocking=True)
-        for d, h in zip(stack.dY, host_dy):
+        for d, h in zip(dev_in, host_in):
             d.copy_(h, non_blocking=True)
         one_step()
         for h, g in zip(host_grads, grads):
@@ -613,8 +625,34 @@ def oracle_sample(family, tokens: int, seed: int = 7, base: str = "nf4"):
     return cases
 
 
+def oracle_decoder_sample(family, tokens: int, seed: int = 7):
+    """One decoder layer of `family` on the oracle (NF4 weights drawn once per
+    family, unit norm gains) and `tokens` tokens of input and output gradient."""
+    import numpy as np
+
+    from host_streamed_nf4_b200 import synth
+    from oracle import decoder as odec
+    cases = oracle_sample(family, 1, seed)
+    lin = {}
+    for name, (n, k, codes, absmax, _, A, B, _) in zip(synth.PROJ_NAMES, cases):
+        lin[name] = odec.Linear(n, k, A=A, B=B, codes=codes, absmax=absmax)
+    layer = odec.Layer(H=family.heads, KV=family.kv_heads, d=family.head_dim,
+                       g1=np.ones(family.hidden), g2=np.ones(family.hidden), lin=lin)
+    rng = np.random.default_rng(seed + tokens)
+    h0 = odec.bits_f64(synth.normal_bf16(rng, (tokens, family.hidden), 1.0))
+    dh = odec.bits_f64(synth.normal_bf16(rng, (tokens, family.hidden), 1.0))
+    return ("decoder", layer, h0, dh)
+
+
 def oracle_step(cases, threads):
     import oracle
+    if isinstance(cases, tuple) and cases[0] == "decoder":
+        # forward, its recompute in the backward visit, then the backward
+        from oracle import decoder as odec
+        _, layer, h0, dh = cases
+        odec.layer_forward(layer, h0)
+        odec.layer_backward(layer, odec.layer_forward(layer, h0), dh)
+        return
     for n, k, codes, absmax, X, A, B, dY in cases:
         if absmax is None:
             oracle.lora_fwd_bf16w(codes, X, A, B, 32.0, n_threads=threads)
@@ -627,13 +665,19 @@ def oracle_step(cases, threads):
             oracle.lora_bwd(codes, absmax, n, k, X, A, B, dY, 32.0, n_threads=threads)
 
 
-def calibrate_tokens(family, target_s, threads, base="nf4"):
+def _sample(family, tokens, base="nf4", model="projections"):
+    if model == "decoder":
+        return oracle_decoder_sample(family, tokens)
+    return oracle_sample(family, tokens, base=base)
+
+
+def calibrate_tokens(family, target_s, threads, base="nf4", model="projections"):
     """Largest sample (in tokens) whose oracle step stays near target_s."""
-    cases = oracle_sample(family, 1, base=base)
+    cases = _sample(family, 1, base, model)
     t = time.perf_counter()
     oracle_step(cases, threads)
     one = time.perf_counter() - t
-    cases = oracle_sample(family, 2, base=base)
+    cases = _sample(family, 2, base, model)
     t = time.perf_counter()
     oracle_step(cases, threads)
     two = time.perf_counter() - t
@@ -649,8 +693,8 @@ def cpu_baseline(args, family):
     import oracle
     oracle.build()
     threads = os.cpu_count() or 1
-    tokens = calibrate_tokens(family, 2.0, threads, args.base)
-    cases = oracle_sample(family, tokens, base=args.base)
+    tokens = calibrate_tokens(family, 2.0, threads, args.base, args.model)
+    cases = _sample(family, tokens, args.base, args.model)
     times = []
     t_end = time.perf_counter() + 15.0
     while time.perf_counter() < t_end or len(times) < 2:
@@ -662,8 +706,10 @@ def cpu_baseline(args, family):
     per_layer = statistics.median(times)
     value = tokens / (per_layer * args.layers)
     return {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{tokens} tokens x 1 layer of {family.name} (7 projections, fwd+bwd, "
-                      f"median of {len(times)} runs), scaled to {args.layers} layer(s)",
+            "sample": f"{tokens} tokens x 1 layer of {family.name} ("
+                      + ("decoder layer: fwd, recomputed fwd, bwd" if args.model == "decoder"
+                         else "7 projections, fwd+bwd")
+                      + f", median of {len(times)} runs), scaled to {args.layers} layer(s)",
             "extrapolated": args.layers > 1 or tokens < args.seq}
 
 
@@ -675,8 +721,8 @@ def run_reference(args, ws, rank):
     oracle.build()
     family = synth.FAMILIES[args.family]
     threads = os.cpu_count() or 1
-    tokens = calibrate_tokens(family, args.ref_seconds, threads, args.base)
-    cases = oracle_sample(family, tokens, base=args.base)
+    tokens = calibrate_tokens(family, args.ref_seconds, threads, args.base, args.model)
+    cases = _sample(family, tokens, args.base, args.model)
     for _ in range(args.warmup):
         oracle_step(cases, threads)
     t = time.perf_counter()
@@ -689,7 +735,8 @@ def run_reference(args, ws, rank):
             "ms_per_step": round(dt * args.layers * 1e3 * (args.seq / tokens), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": args.workload, "family": args.family, "layers": args.layers,
+            "config": {"workload": args.workload + ("-decoder" if args.model == "decoder" else ""),
+                       "model": args.model, "family": args.family, "layers": args.layers,
                        "tokens": args.seq, "batch": 1, "mode": "cpu-oracle",
                        "base": args.base},
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,

@@ -176,5 +176,8 @@ class DecoderStack(LayerStack):
                 record(l, -1, "dh_in", nxt)
             self.dh_cur = nxt
 
+    def step_inputs(self):
+        return [self.h_in, self.dh_top]
+
     def kernels_per_step(self) -> int:
         return -1  # counted by the library (hsnf4.kernel_launches)

@@ -340,6 +340,11 @@ class LayerStack:
         projection (2), the GEMM (1) and the adapter gradients (1)."""
         return self.L * len(self.groups) * (3 + 4)
 
+    def step_inputs(self):
+        """The device tensors a step reads that come from outside (the
+        activations and upstream gradients), for end-to-end timing."""
+        return list(self.X.values()) + list(self.dY)
+
     def tokens_per_step(self) -> int:
         return self.T
 
