@@ -600,6 +600,12 @@ int decoder_attention_fwd(const void* q, const void* k, const void* v, void* o, 
                      "decoder_attention_fwd launch");
 }
 
+size_t decoder_attention_scratch_bytes(int64_t T, int H) {
+  if (T < 1 || H < 1) return 0;
+  // row dots [H, T] (rounded up to 64 floats), then fp32 dK, dV partials [2H][T][128]
+  return (static_cast<size_t>(T) * H + 63) / 64 * 64 * 4 + static_cast<size_t>(T) * H * 2 * 128 * 4;
+}
+
 int decoder_attention_bwd(const void* q, const void* k, const void* v, const void* o,
                           const float* lse, const void* dout, void* dq, void* dk, void* dv,
                           float* scratch, int64_t T, int H, int KV, void* stream) {

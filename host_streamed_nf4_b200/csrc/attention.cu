@@ -9,9 +9,10 @@
 // 64-key tiles, 4 warps of 16 rows, online softmax in registers (exp2 with
 // the scale folded into log2 units); the probabilities are rounded to bf16
 // for the P.V product.  Backward in two kernels without atomics, so results
-// are run-to-run identical: dQ per (query tile, head) over its key tiles,
-// dK and dV per (key tile, KV head) over the query tiles and the query heads
-// of the group, with D_i = sum_c dO_ic O_ic precomputed.
+// are run-to-run identical: dQ per (query tile, head) over its key tiles;
+// dK and dV per (key tile, query head) over the query tiles, as fp32
+// partials that a last kernel adds over the query heads of each KV group in
+// head order; D_i = sum_c dO_ic O_ic precomputed.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -40,6 +41,7 @@ struct AttnArgs {
   uint16_t* dv;
   float* lse;         // [H, T]
   const float* D;     // [H, T]
+  float* part;        // backward: per-head fp32 dK, dV partials [2H][T][128]
   int T, H, KV;
   float scale;
 };
@@ -305,7 +307,9 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(const __grid_constant_
 }
 
 // ---------------------------------------------------------------- dK, dV
-// Per warp 16 keys; S^T = K Q^T (keys x queries), P^T from the saved lse.
+// Per CTA one key tile and one QUERY head: S^T = K Q^T (keys x queries), P^T
+// from the saved lse, 16 keys per warp; the head's fp32 dK, dV partials go to
+// scratch and a second kernel adds the heads of each KV group in head order.
 __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const __grid_constant__ AttnArgs P) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
@@ -314,7 +318,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const __grid_constan
   uint16_t* dOs = Qs + 64 * kLd;
   float* lse_s = reinterpret_cast<float*>(dOs + 64 * kLd);  // [64] in log2 units
   float* D_s = lse_s + 64;
-  const int kt = blockIdx.x, kh = blockIdx.y, grp = P.H / P.KV;
+  const int kt = blockIdx.x, h = blockIdx.y, kh = h / (P.H / P.KV);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, qd = lane & 3;
   const int m0 = warp * 16;
   const int64_t qs = static_cast<int64_t>(P.H) * kD, ks = static_cast<int64_t>(P.KV) * kD;
@@ -328,53 +332,76 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const __grid_constan
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.0f;
   const int q_tiles = (P.T + kBM - 1) / kBM;
-  for (int hh = 0; hh < grp; ++hh) {
-    const int h = kh * grp + hh;
-    for (int qt = kt; qt < q_tiles; ++qt) {
-      __syncthreads();
-      load_tile(Qs, P.q, qt * kBM, P.T, qs, h * kD);
-      load_tile(dOs, P.dout, qt * kBM, P.T, qs, h * kD);
-      for (int i = threadIdx.x; i < 64; i += blockDim.x) {
-        const int row = qt * kBM + i;
-        lse_s[i] = row < P.T ? P.lse[static_cast<int64_t>(h) * P.T + row] * kLog2e : 0.0f;
-        D_s[i] = row < P.T ? P.D[static_cast<int64_t>(h) * P.T + row] : 0.0f;
-      }
-      __syncthreads();
-      float s[8][4];
-      gemm_xyt(s, Ks, m0, Qs);  // S^T = K Q^T
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int hr = e >> 1, qi = j * 8 + 2 * qd + (e & 1), row = qt * kBM + qi;
-          const bool on = keys[hr] <= row && row < P.T && keys[hr] < P.T;
-          s[j][e] = on ? exp2f(s[j][e] * c - lse_s[qi]) : 0.0f;  // P^T
-        }
-      gemm_py(dv, s, dOs);  // dV += P^T dO
-      float dp[8][4];
-      gemm_xyt(dp, Vs, m0, dOs);  // dP^T = V dO^T
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int qi = j * 8 + 2 * qd + (e & 1);
-          s[j][e] = s[j][e] * (dp[j][e] - D_s[qi]);  // dS^T
-        }
-      gemm_py(dk, s, Qs);  // dK += dS^T Q
+  for (int qt = kt; qt < q_tiles; ++qt) {
+    __syncthreads();
+    load_tile(Qs, P.q, qt * kBM, P.T, qs, h * kD);
+    load_tile(dOs, P.dout, qt * kBM, P.T, qs, h * kD);
+    for (int i = threadIdx.x; i < 64; i += blockDim.x) {
+      const int row = qt * kBM + i;
+      lse_s[i] = row < P.T ? P.lse[static_cast<int64_t>(h) * P.T + row] * kLog2e : 0.0f;
+      D_s[i] = row < P.T ? P.D[static_cast<int64_t>(h) * P.T + row] : 0.0f;
     }
+    __syncthreads();
+    float s[8][4];
+    gemm_xyt(s, Ks, m0, Qs);  // S^T = K Q^T
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int hr = e >> 1, qi = j * 8 + 2 * qd + (e & 1), row = qt * kBM + qi;
+        const bool on = keys[hr] <= row && row < P.T && keys[hr] < P.T;
+        s[j][e] = on ? exp2f(s[j][e] * c - lse_s[qi]) : 0.0f;  // P^T
+      }
+    gemm_py(dv, s, dOs);  // dV += P^T dO
+    float dp[8][4];
+    gemm_xyt(dp, Vs, m0, dOs);  // dP^T = V dO^T
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int qi = j * 8 + 2 * qd + (e & 1);
+        s[j][e] = s[j][e] * (dp[j][e] - D_s[qi]);  // dS^T
+      }
+    gemm_py(dk, s, Qs);  // dK += dS^T Q
   }
+  // this head's partials: part[h][key][c] (dK unscaled), part[H + h][key][c] (dV)
 #pragma unroll
   for (int hr = 0; hr < 2; ++hr) {
     if (keys[hr] >= P.T) continue;
-    uint16_t* dkd = P.dk + static_cast<int64_t>(keys[hr]) * ks + kh * kD;
-    uint16_t* dvd = P.dv + static_cast<int64_t>(keys[hr]) * ks + kh * kD;
+    float* pk = P.part + (static_cast<int64_t>(h) * P.T + keys[hr]) * kD;
+    float* pv = P.part + (static_cast<int64_t>(P.H + h) * P.T + keys[hr]) * kD;
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
-      *reinterpret_cast<uint32_t*>(dkd + n * 8 + 2 * qd) =
-          pack_bf16(dk[n][2 * hr] * P.scale, dk[n][2 * hr + 1] * P.scale);
-      *reinterpret_cast<uint32_t*>(dvd + n * 8 + 2 * qd) =
-          pack_bf16(dv[n][2 * hr], dv[n][2 * hr + 1]);
+      *reinterpret_cast<float2*>(pk + n * 8 + 2 * qd) = make_float2(dk[n][2 * hr], dk[n][2 * hr + 1]);
+      *reinterpret_cast<float2*>(pv + n * 8 + 2 * qd) = make_float2(dv[n][2 * hr], dv[n][2 * hr + 1]);
     }
+  }
+}
+
+// dK[key, kh] = scale sum_{h in group kh} part_k[h][key], dV likewise (head order)
+__global__ void __launch_bounds__(256) attn_bwd_kv_reduce_kernel(const __grid_constant__ AttnArgs P) {
+  const int grp = P.H / P.KV;
+  const int64_t n4 = static_cast<int64_t>(P.T) * P.KV * (kD / 4);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * 256) {
+    const int c4 = static_cast<int>(i % (kD / 4));
+    const int64_t rk = i / (kD / 4);
+    const int kh = static_cast<int>(rk % P.KV);
+    const int64_t key = rk / P.KV;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    for (int hh = 0; hh < grp; ++hh) {
+      const int h = kh * grp + hh;
+      const float4 x = *reinterpret_cast<const float4*>(
+          P.part + (static_cast<int64_t>(h) * P.T + key) * kD + c4 * 4);
+      const float4 y = *reinterpret_cast<const float4*>(
+          P.part + (static_cast<int64_t>(P.H + h) * P.T + key) * kD + c4 * 4);
+      a.x += x.x, a.y += x.y, a.z += x.z, a.w += x.w;
+      b.x += y.x, b.y += y.y, b.z += y.z, b.w += y.w;
+    }
+    const int64_t o = key * P.KV * kD + kh * kD + c4 * 4;
+    *reinterpret_cast<uint2*>(P.dk + o) =
+        make_uint2(pack_bf16(a.x * P.scale, a.y * P.scale), pack_bf16(a.z * P.scale, a.w * P.scale));
+    *reinterpret_cast<uint2*>(P.dv + o) = make_uint2(pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
   }
 }
 
@@ -433,6 +460,8 @@ cudaError_t launch_attention_bwd(const void* q, const void* k, const void* v, co
   P.H = H;
   P.KV = KV;
   P.scale = scale;
+  // partials after the row dots, on a 256-byte boundary (float4 loads)
+  P.part = D + (static_cast<int64_t>(H) * T + 63) / 64 * 64;
   const int64_t warps = T * H;
   count_launch();
   attn_bwd_dot_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(P);
@@ -444,7 +473,16 @@ cudaError_t launch_attention_bwd(const void* q, const void* k, const void* v, co
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   count_launch();
-  attn_bwd_dkdv_kernel<<<dim3(tiles, KV), 128, smem_kv, st>>>(P);
+  attn_bwd_dkdv_kernel<<<dim3(tiles, H), 128, smem_kv, st>>>(P);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t grid = (T * KV * (kD / 4) + 255) / 256;
+  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
+  count_launch();
+  attn_bwd_kv_reduce_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(P);
   return cudaGetLastError();
 }
 

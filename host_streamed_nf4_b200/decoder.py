@@ -79,7 +79,8 @@ class DecoderStack(LayerStack):
                    "db_u": bf(T, h), "dh1": bf(T, h), "datt": bf(T, H * d), "dq": bf(T, H * d),
                    "dk": bf(T, KV * d), "dv": bf(T, KV * d), "da_q": bf(T, h), "da_k": bf(T, h),
                    "da_v": bf(T, h), "dh_a": bf(T, h), "dh_b": bf(T, h),
-                   "scratch": torch.empty(H, T, dtype=torch.float32, device=dev)}
+                   "scratch": torch.empty(hsnf4.attention_scratch_bytes(T, H), dtype=torch.uint8,
+                                          device=dev)}
         torch.cuda.synchronize(dev)
 
     # ------------------------------------------------------------ one layer

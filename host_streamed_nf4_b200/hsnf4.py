@@ -100,6 +100,7 @@ _SIGS = {
     "decoder_add": ([c_void_p, c_void_p, c_void_p, c_int64, c_void_p], c_int),
     "decoder_attention_fwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int,
                                c_int, c_void_p], c_int),
+    "decoder_attention_scratch_bytes": ([c_int64, c_int], c_size_t),
     "decoder_attention_bwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int, c_int,
                                c_void_p], c_int),
@@ -358,6 +359,10 @@ def attention_fwd(q, k, v, H, KV, o=None, lse=None, stream=None):
     return o, lse
 
 
+def attention_scratch_bytes(T: int, H: int) -> int:
+    return int(lib().decoder_attention_scratch_bytes(T, H))
+
+
 def attention_bwd(q, k, v, o, lse, dout, H, KV, dq=None, dk=None, dv=None, scratch=None,
                   stream=None):
     T = q.shape[0]
@@ -365,7 +370,7 @@ def attention_bwd(q, k, v, o, lse, dout, H, KV, dq=None, dk=None, dv=None, scrat
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     if scratch is None:
-        scratch = torch.empty(H, T, dtype=torch.float32, device=q.device)
+        scratch = torch.empty(attention_scratch_bytes(T, H), dtype=torch.uint8, device=q.device)
     _check(lib().decoder_attention_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
                                        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(scratch), T, H, KV,
                                        _stream(stream)))

@@ -354,7 +354,10 @@ int decoder_attention_fwd(const void *q, const void *k, const void *v, void *o, 
                           int64_t T, int H, int KV, void *stream);
 
 /* Its gradients from the forward's o and lse:  dq [T, H*128], dk, dv
- * [T, KV*128] (overwritten); scratch fp32 [H, T] (caller-owned). */
+ * [T, KV*128] (overwritten); scratch: caller-owned device memory of
+ * decoder_attention_scratch_bytes(T, H) bytes (the row dots and per-head
+ * fp32 partials of dk and dv, added over each KV group in head order). */
+size_t decoder_attention_scratch_bytes(int64_t T, int H);
 int decoder_attention_bwd(const void *q, const void *k, const void *v, const void *o,
                           const float *lse, const void *dout, void *dq, void *dk, void *dv,
                           float *scratch, int64_t T, int H, int KV, void *stream);
