@@ -383,51 +383,73 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
     const int i = threadIdx.x & 127;  // this thread's line of the A tile
     const int line = (MODE == kGemmFwd) ? i : ((i >> 6) * 64 + (i & 63));
     const int code_off = (MODE == kGemmFwd) ? i * 32 : (i & 63) * 64 + (i >> 6) * 32;
-    int g = 0;
-    bool ok = true;
-    for (int ui = u_begin; ui < u_end && ok; ++ui) {
-      const Unit U = unpack_unit(P, P.units[ui]);
+    // this thread's absmax for K step kb of unit U (0 past the weight's edge)
+    auto absmax_at = [&](const Unit& U, int kb) -> float {
       const GemmProblem& pr = P.prob[U.p];
       const int m0 = U.mt * kTileM;
-      for (int kb = U.kb0; kb < U.kb1; ++kb, ++g) {
-        if ((g & 1) != grp) continue;
-        const int sc = g % SC, sa = g % SA;
-        float a;
-        if (MODE == kGemmFwd) {
-          const int row = m0 + i;
-          a = (row < pr.n_out)
-                  ? __ldg(pr.absmax + static_cast<int64_t>(row) * pr.kblocks + kb)
-                  : 0.0f;
-        } else {
-          const int row = kb * kStepK + (i & 63);
-          const int kblk = m0 / 64 + (i >> 6);
-          a = (kblk < pr.kblocks)
-                  ? __ldg(pr.absmax + static_cast<int64_t>(row) * pr.kblocks + kblk)
-                  : 0.0f;
-        }
-        if (!mbar_wait(&c_full[sc], (g / SC) & 1, abort_flag, &g_gemm_flags, kFlagDequant)) {
-          ok = false;
-          break;
-        }
-        const uint4* src = reinterpret_cast<const uint4*>(c_tile(sc) + code_off);
-        const uint4 c0 = src[0], c1 = src[1];
-        mbar_arrive(&c_empty[sc]);
-        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const Nf4Table tab = nf4_make_table(P.cb, a);
-        if (g >= SA && !mbar_wait(&a_empty[sa], ((g / SA) - 1) & 1, abort_flag, &g_gemm_flags,
-                                  kFlagDequant)) {
-          ok = false;
-          break;
-        }
-        uint8_t* dst = a_tile(sa) + line * 128;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          const uint4 v = nf4_dequant8(words[w], tab);
-          *reinterpret_cast<uint4*>(dst + ((w ^ (line & 7)) << 4)) = v;
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&a_full[sa]);
+      if (MODE == kGemmFwd) {
+        const int row = m0 + i;
+        return row < pr.n_out ? __ldg(pr.absmax + static_cast<int64_t>(row) * pr.kblocks + kb)
+                              : 0.0f;
       }
+      const int row = kb * kStepK + (i & 63);
+      const int kblk = m0 / 64 + (i >> 6);
+      return kblk < pr.kblocks ? __ldg(pr.absmax + static_cast<int64_t>(row) * pr.kblocks + kblk)
+                               : 0.0f;
+    };
+    // advance (ui, kb, U) by `steps` K steps of this CTA's sequence; false at its end
+    auto advance = [&](int& ui, int& kb, Unit& U, int steps) -> bool {
+      kb += steps;
+      while (kb >= U.kb1) {
+        const int over = kb - U.kb1;
+        if (++ui >= u_end) return false;
+        U = unpack_unit(P, P.units[ui]);
+        kb = U.kb0 + over;
+      }
+      return true;
+    };
+    // This warpgroup's K steps are g = grp, grp + 2, ...  The absmax of the
+    // next one is loaded while the current one waits and expands, so the
+    // global-load latency is off the per-step path.
+    int ui = u_begin, kb = 0, g = grp;
+    Unit U{};
+    bool have = ui < u_end;
+    if (have) {
+      U = unpack_unit(P, P.units[ui]);
+      kb = U.kb0;
+      have = advance(ui, kb, U, grp);
+    }
+    float a_next = have ? absmax_at(U, kb) : 0.0f;
+    bool ok = true;
+    while (have && ok) {
+      const float a = a_next;
+      const int gc = g;
+      have = advance(ui, kb, U, 2);
+      g += 2;
+      if (have) a_next = absmax_at(U, kb);
+      const int sc = gc % SC, sa = gc % SA;
+      if (!mbar_wait(&c_full[sc], (gc / SC) & 1, abort_flag, &g_gemm_flags, kFlagDequant)) {
+        ok = false;
+        break;
+      }
+      const uint4* src = reinterpret_cast<const uint4*>(c_tile(sc) + code_off);
+      const uint4 c0 = src[0], c1 = src[1];
+      mbar_arrive(&c_empty[sc]);
+      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      const Nf4Table tab = nf4_make_table(P.cb, a);
+      if (gc >= SA && !mbar_wait(&a_empty[sa], ((gc / SA) - 1) & 1, abort_flag, &g_gemm_flags,
+                                 kFlagDequant)) {
+        ok = false;
+        break;
+      }
+      uint8_t* dst = a_tile(sa) + line * 128;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const uint4 v = nf4_dequant8(words[w], tab);
+        *reinterpret_cast<uint4*>(dst + ((w ^ (line & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&a_full[sa]);
     }
   } else {
     // -------------------------------------------------- epilogue (warps 8..11)
