@@ -10,8 +10,9 @@
 //            (the GEMM's rank-r slice is zero in this mode).
 //
 // The mask is recomputed, never stored: element e = t K + k takes word e % 4
-// of the Philox block of e / 4 (philox.cuh).  A thread owns 8 consecutive
-// elements of one row (16 bytes of bf16, two Philox blocks).  Both kernels
+// of the Philox block of e / 4 (philox.cuh).  An apply thread owns 8
+// consecutive elements of one row (16 bytes of bf16, two Philox blocks); a
+// dx-add thread the same 8 columns of 4 consecutive rows.  Both kernels
 // are HBM-bound elementwise passes: apply reads 2 B and writes 2 B per
 // element, dx add reads 2 B and writes 2 B (u and A are re-read from L2).
 #include <cuda_bf16.h>
@@ -28,7 +29,7 @@ struct DropProblem {
   uint16_t* out;       // apply: X_d [T, K];    dx add: dX [T, K] (read and written)
   const float* u;      // dx add: u fp32 [T, r]
   const uint16_t* A;   // dx add: A bf16 [r, K]
-  int64_t groups;      // T * K / 8
+  int64_t groups;      // work items: T * K / 8 (apply), ceil(T / 4) * K / 8 (dx add)
   int64_t g0;          // first group index of this problem in the launch
   int64_t K;
   uint64_t seed, offset;
@@ -38,9 +39,9 @@ struct DropProblem {
 
 struct DropParams {
   DropProblem p[kMaxDrop];
-  int n, r;
+  int n, r, T;
   float s;
-  int64_t total;  // groups over all problems
+  int64_t total;  // work items over all problems
 };
 
 __device__ __forceinline__ int drop_problem(const DropParams& P, int64_t g) {
@@ -86,45 +87,72 @@ __global__ void __launch_bounds__(256) lora_dropout_apply(const __grid_constant_
   }
 }
 
+// dx add: a thread owns 8 consecutive columns of 4 consecutive tokens, so
+// each 16-byte row of A serves 32 elements
 __global__ void __launch_bounds__(256) lora_dx_dropout_add(const __grid_constant__ DropParams P) {
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < P.total;
        g += stride) {
     const DropProblem& pr = P.p[drop_problem(P, g)];
     const int64_t lg = g - pr.g0;
-    const int64_t e0 = lg * 8;
-    const int64_t t = e0 / pr.K, k0 = e0 - t * pr.K;
-    const uint32_t keep = keep8(pr, lg);
-    // adapter term of the 8 elements: sum_j u[t, j] A[j, k0 + i]
-    float lora[8];
+    const int64_t k8 = pr.K / 8;
+    const int64_t t0 = (lg / k8) * 4, k0 = (lg % k8) * 8;
+    const int nt = static_cast<int>((P.T - t0) < 4 ? (P.T - t0) : 4);
+    // adapter term: lora[tt][i] = sum_j u[t0 + tt, j] A[j, k0 + i]
+    float lora[4][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) lora[i] = 0.0f;
-    const float* ur = pr.u + t * P.r;
-    for (int j = 0; j < P.r; ++j) {
-      const float uj = __ldg(ur + j);
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(pr.A + j * pr.K + k0));
-      const uint32_t as[4] = {a.x, a.y, a.z, a.w};
+    for (int tt = 0; tt < 4; ++tt)
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        lora[2 * h] = __fmaf_rn(uj, __uint_as_float(as[h] << 16), lora[2 * h]);
-        lora[2 * h + 1] = __fmaf_rn(uj, __uint_as_float(as[h] & 0xFFFF0000u), lora[2 * h + 1]);
+      for (int i = 0; i < 8; ++i) lora[tt][i] = 0.0f;
+    for (int j0 = 0; j0 < P.r; j0 += 4) {  // r % 8 == 0
+      // four rows of A and the four tokens' u[j0 .. j0 + 3], all loads first
+      uint4 a[4];
+      float4 uq[4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+        a[jj] = __ldg(reinterpret_cast<const uint4*>(pr.A + (j0 + jj) * pr.K + k0));
+#pragma unroll
+      for (int tt = 0; tt < 4; ++tt)
+        uq[tt] = tt < nt ? __ldg(reinterpret_cast<const float4*>(pr.u + (t0 + tt) * P.r + j0))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const uint32_t as[4] = {a[jj].x, a[jj].y, a[jj].z, a[jj].w};
+        float af[8];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          af[2 * h] = __uint_as_float(as[h] << 16);
+          af[2 * h + 1] = __uint_as_float(as[h] & 0xFFFF0000u);
+        }
+#pragma unroll
+        for (int tt = 0; tt < 4; ++tt) {
+          const float uj = jj == 0 ? uq[tt].x : jj == 1 ? uq[tt].y : jj == 2 ? uq[tt].z : uq[tt].w;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) lora[tt][i] = __fmaf_rn(uj, af[i], lora[tt][i]);
+        }
       }
     }
-    uint4* dst = reinterpret_cast<uint4*>(pr.out) + lg;
-    const uint4 d = *dst;
-    const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
-    uint32_t o[4];
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      float lo = __uint_as_float(ds[h] << 16), hi = __uint_as_float(ds[h] & 0xFFFF0000u);
-      if ((keep >> (2 * h)) & 1u)
-        lo = __fadd_rn(lo, __fmul_rn(__fmul_rn(P.s, lora[2 * h]), pr.scale));
-      if ((keep >> (2 * h + 1)) & 1u)
-        hi = __fadd_rn(hi, __fmul_rn(__fmul_rn(P.s, lora[2 * h + 1]), pr.scale));
-      const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-      o[h] = *reinterpret_cast<const uint32_t*>(&v);
+    for (int tt = 0; tt < 4; ++tt) {
+      if (tt >= nt) break;
+      const int64_t e8 = ((t0 + tt) * pr.K + k0) / 8;  // this row segment's 8-element group
+      const uint32_t keep = keep8(pr, e8);
+      uint4* dst = reinterpret_cast<uint4*>(pr.out) + e8;
+      const uint4 d = *dst;
+      const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        float lo = __uint_as_float(ds[h] << 16), hi = __uint_as_float(ds[h] & 0xFFFF0000u);
+        if ((keep >> (2 * h)) & 1u)
+          lo = __fadd_rn(lo, __fmul_rn(__fmul_rn(P.s, lora[tt][2 * h]), pr.scale));
+        if ((keep >> (2 * h + 1)) & 1u)
+          hi = __fadd_rn(hi, __fmul_rn(__fmul_rn(P.s, lora[tt][2 * h + 1]), pr.scale));
+        const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        o[h] = *reinterpret_cast<const uint32_t*>(&v);
+      }
+      *dst = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    *dst = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -135,6 +163,7 @@ static cudaError_t launch_drop(bool dx, const DropDesc* d, int n, int64_t T, int
   memset(&P, 0, sizeof P);
   P.n = n;
   P.r = r;
+  P.T = static_cast<int>(T);
   P.s = s;
   int64_t g = 0;
   for (int q = 0; q < n; ++q) {
@@ -145,7 +174,8 @@ static cudaError_t launch_drop(bool dx, const DropDesc* d, int n, int64_t T, int
     pr.u = d[q].u;
     pr.A = static_cast<const uint16_t*>(d[q].A);
     pr.K = d[q].K;
-    pr.groups = T * d[q].K / 8;
+    // apply: one item per 8 elements; dx add: 8 columns x 4 tokens
+    pr.groups = dx ? (T + 3) / 4 * (d[q].K / 8) : T * d[q].K / 8;
     pr.g0 = g;
     pr.seed = dp.seed;
     pr.offset = dp.offset;

@@ -58,6 +58,27 @@ __global__ void __launch_bounds__(256) lora_merge_kernel(const __grid_constant__
   const int64_t n0 = static_cast<int64_t>(blockIdx.x / P.col_tiles) * kMrgRows;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x % P.col_tiles) * kMrgCols;
 
+  // ---- the base bytes of this thread's two 8-element groups, loaded first so
+  // that their DRAM latency overlaps the staging and the product below
+  uint4 wraw[2];
+  float wabs[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int v = tid + i * 256;
+    const int row = v >> 4, col = (v & 15) * 8;
+    wraw[i] = make_uint4(0, 0, 0, 0);
+    wabs[i] = 0.0f;
+    if (k0 + col >= P.K) continue;
+    const int64_t e = (n0 + row) * P.K + k0 + col;
+    if (P.dense) {
+      wraw[i] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(P.base) + e));
+    } else {
+      wraw[i].x = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(P.base) +
+                                                          e / 2));
+      wabs[i] = __ldg(P.absmax + e / 64);
+    }
+  }
+
   // ---- stage B rows n0.. (j < r, zeros up to R) and A columns k0.. (rows j < r)
   for (int v = tid; v < kMrgRows * (R / 8); v += 256) {
     const int row = v / (R / 8), jq = (v % (R / 8)) * 8;
@@ -107,12 +128,9 @@ __global__ void __launch_bounds__(256) lora_merge_kernel(const __grid_constant__
     const int64_t e = (n0 + row) * P.K + k0 + col;  // first element of the group
     uint32_t wv[4];
     if (P.dense) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(P.base) + e));
-      wv[0] = w.x, wv[1] = w.y, wv[2] = w.z, wv[3] = w.w;
+      wv[0] = wraw[i].x, wv[1] = wraw[i].y, wv[2] = wraw[i].z, wv[3] = wraw[i].w;
     } else {
-      const uint32_t cw = __ldg(reinterpret_cast<const uint32_t*>(
-          static_cast<const uint8_t*>(P.base) + e / 2));
-      const uint4 w = nf4_dequant8(cw, nf4_make_table(P.cb, __ldg(P.absmax + e / 64)));
+      const uint4 w = nf4_dequant8(wraw[i].x, nf4_make_table(P.cb, wabs[i]));
       wv[0] = w.x, wv[1] = w.y, wv[2] = w.z, wv[3] = w.w;
     }
     const float* pr = ps + row * kMrgLdS + col;
