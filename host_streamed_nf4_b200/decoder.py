@@ -179,6 +179,3 @@ class DecoderStack(LayerStack):
 
     def step_inputs(self):
         return [self.h_in, self.dh_top]
-
-    def kernels_per_step(self) -> int:
-        return -1  # counted by the library (hsnf4.kernel_launches)

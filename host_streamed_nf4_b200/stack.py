@@ -334,12 +334,6 @@ class LayerStack:
             return self.block_bytes(b)
         return hsnf4.shard_range(self.block_bytes(b), self.shard[1], self.shard[0])[2]
 
-    def kernels_per_step(self) -> int:
-        """Library kernels one step launches: per group, the forward runs the
-        rank-r projection (2 kernels) and the fused GEMM (1); the backward the
-        projection (2), the GEMM (1) and the adapter gradients (1)."""
-        return self.L * len(self.groups) * (3 + 4)
-
     def step_inputs(self):
         """The device tensors a step reads that come from outside (the
         activations and upstream gradients), for end-to-end timing."""
