@@ -6,7 +6,8 @@
 //   keys/values of KV head h / (H / KV);  lse_i = log sum_{j <= i} e^{scale q_i.k_j}
 //
 // Tensor cores via mma.sync m16n8k16 (bf16 in, fp32 accumulate), 64-query x
-// 64-key tiles, 4 warps of 16 rows, online softmax in registers (exp2 with
+// 64-key tiles double-buffered through cp.async (the next tile loads while
+// this one is multiplied), 4 warps of 16 rows, online softmax in registers (exp2 with
 // the scale folded into log2 units); the probabilities are rounded to bf16
 // for the P.V product.  Backward in two kernels without atomics, so results
 // are run-to-run identical: dQ per (query tile, head) over its key tiles;
@@ -76,17 +77,29 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // 64 rows x 128 columns of a row-major [T, stride] bf16 tensor (rows from
-// r0, columns from c0) into a padded smem tile; rows past T are zeros.
-__device__ __forceinline__ void load_tile(uint16_t* dst, const uint16_t* src, int r0, int T,
-                                          int64_t stride, int c0) {
+// r0, columns from c0) into a padded smem tile with cp.async; rows past T
+// are written as zeros.
+__device__ __forceinline__ void load_tile_async(uint16_t* dst, const uint16_t* src, int r0, int T,
+                                                int64_t stride, int c0) {
   for (int v = threadIdx.x; v < 64 * 16; v += blockDim.x) {
     const int row = v >> 4, col = (v & 15) * 8;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (r0 + row < T)
-      val = __ldg(reinterpret_cast<const uint4*>(src + static_cast<int64_t>(r0 + row) * stride +
-                                                 c0 + col));
-    *reinterpret_cast<uint4*>(dst + row * kLd + col) = val;
+    const bool in = r0 + row < T;
+    const uint16_t* s = in ? src + static_cast<int64_t>(r0 + row) * stride + c0 + col : src;
+    cp_async16(su32(dst + row * kLd + col), s, in ? 16 : 0);
   }
 }
 
@@ -156,13 +169,15 @@ __device__ __forceinline__ void gemm_py(float (&acc)[16][4], const float (&p)[8]
 __global__ void __launch_bounds__(128) attn_fwd_kernel(const __grid_constant__ AttnArgs P) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint16_t* Qs = reinterpret_cast<uint16_t*>(smem);
-  uint16_t* Ks = Qs + 64 * kLd;
-  uint16_t* Vs = Ks + 64 * kLd;
+  uint16_t* KV = Qs + 64 * kLd;  // K0 V0 K1 V1: the next tile loads during this one
   const int qt = blockIdx.x, h = blockIdx.y, kh = h / (P.H / P.KV);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, qd = lane & 3;
   const int m0 = warp * 16;
   const int64_t qs = static_cast<int64_t>(P.H) * kD, ks = static_cast<int64_t>(P.KV) * kD;
-  load_tile(Qs, P.q, qt * kBM, P.T, qs, h * kD);
+  load_tile_async(Qs, P.q, qt * kBM, P.T, qs, h * kD);
+  load_tile_async(KV, P.k, 0, P.T, ks, kh * kD);
+  load_tile_async(KV + 64 * kLd, P.v, 0, P.T, ks, kh * kD);
+  cp_async_commit();
   const float c = P.scale * kLog2e;
   float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
   float acc[16][4];
@@ -172,9 +187,15 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const __grid_constant__ A
     for (int e = 0; e < 4; ++e) acc[n][e] = 0.0f;
   const int rows[2] = {qt * kBM + m0 + g, qt * kBM + m0 + g + 8};
   for (int kt = 0; kt <= qt; ++kt) {
-    __syncthreads();
-    load_tile(Ks, P.k, kt * kBN, P.T, ks, kh * kD);
-    load_tile(Vs, P.v, kt * kBN, P.T, ks, kh * kD);
+    const uint16_t* Ks = KV + ((kt & 1) * 2) * 64 * kLd;
+    const uint16_t* Vs = Ks + 64 * kLd;
+    if (kt < qt) {  // the other buffer was released at the end of the previous tile
+      uint16_t* Kn = KV + (((kt + 1) & 1) * 2) * 64 * kLd;
+      load_tile_async(Kn, P.k, (kt + 1) * kBN, P.T, ks, kh * kD);
+      load_tile_async(Kn + 64 * kLd, P.v, (kt + 1) * kBN, P.T, ks, kh * kD);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();  // everything but the group just committed: tile kt is in
     __syncthreads();
     float s[8][4];
     gemm_xyt(s, Qs, m0, Ks);
@@ -215,6 +236,7 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const __grid_constant__ A
       }
     }
     gemm_py(acc, s, Vs);
+    __syncthreads();  // this buffer is refilled by the next iteration's prefetch
   }
   // normalize and write o (bf16) and lse (natural log)
 #pragma unroll
@@ -254,14 +276,16 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(const __grid_constant_
   extern __shared__ __align__(16) uint8_t smem[];
   uint16_t* Qs = reinterpret_cast<uint16_t*>(smem);
   uint16_t* dOs = Qs + 64 * kLd;
-  uint16_t* Ks = dOs + 64 * kLd;
-  uint16_t* Vs = Ks + 64 * kLd;
+  uint16_t* KV = dOs + 64 * kLd;  // K0 V0 K1 V1
   const int qt = blockIdx.x, h = blockIdx.y, kh = h / (P.H / P.KV);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, qd = lane & 3;
   const int m0 = warp * 16;
   const int64_t qs = static_cast<int64_t>(P.H) * kD, ks = static_cast<int64_t>(P.KV) * kD;
-  load_tile(Qs, P.q, qt * kBM, P.T, qs, h * kD);
-  load_tile(dOs, P.dout, qt * kBM, P.T, qs, h * kD);
+  load_tile_async(Qs, P.q, qt * kBM, P.T, qs, h * kD);
+  load_tile_async(dOs, P.dout, qt * kBM, P.T, qs, h * kD);
+  load_tile_async(KV, P.k, 0, P.T, ks, kh * kD);
+  load_tile_async(KV + 64 * kLd, P.v, 0, P.T, ks, kh * kD);
+  cp_async_commit();
   const float c = P.scale * kLog2e;
   const int rows[2] = {qt * kBM + m0 + g, qt * kBM + m0 + g + 8};
   float lse2[2], Dr[2];
@@ -277,9 +301,15 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(const __grid_constant_
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[n][e] = 0.0f;
   for (int kt = 0; kt <= qt; ++kt) {
-    __syncthreads();
-    load_tile(Ks, P.k, kt * kBN, P.T, ks, kh * kD);
-    load_tile(Vs, P.v, kt * kBN, P.T, ks, kh * kD);
+    const uint16_t* Ks = KV + ((kt & 1) * 2) * 64 * kLd;
+    const uint16_t* Vs = Ks + 64 * kLd;
+    if (kt < qt) {
+      uint16_t* Kn = KV + (((kt + 1) & 1) * 2) * 64 * kLd;
+      load_tile_async(Kn, P.k, (kt + 1) * kBN, P.T, ks, kh * kD);
+      load_tile_async(Kn + 64 * kLd, P.v, (kt + 1) * kBN, P.T, ks, kh * kD);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();
     __syncthreads();
     float s[8][4], dp[8][4];
     gemm_xyt(s, Qs, m0, Ks);    // S = Q K^T
@@ -294,6 +324,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(const __grid_constant_
         s[j][e] = p * (dp[j][e] - Dr[hr]);  // dS
       }
     gemm_py(acc, s, Ks);  // dQ += dS K
+    __syncthreads();
   }
 #pragma unroll
   for (int hr = 0; hr < 2; ++hr) {
@@ -314,16 +345,26 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const __grid_constan
   extern __shared__ __align__(16) uint8_t smem[];
   uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
   uint16_t* Vs = Ks + 64 * kLd;
-  uint16_t* Qs = Vs + 64 * kLd;
-  uint16_t* dOs = Qs + 64 * kLd;
-  float* lse_s = reinterpret_cast<float*>(dOs + 64 * kLd);  // [64] in log2 units
-  float* D_s = lse_s + 64;
+  uint16_t* QD = Vs + 64 * kLd;  // Q0 dO0 Q1 dO1: the next query tile loads during this one
+  float* LD = reinterpret_cast<float*>(QD + 4 * 64 * kLd);  // per buffer: lse [64], D [64]
   const int kt = blockIdx.x, h = blockIdx.y, kh = h / (P.H / P.KV);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, qd = lane & 3;
   const int m0 = warp * 16;
   const int64_t qs = static_cast<int64_t>(P.H) * kD, ks = static_cast<int64_t>(P.KV) * kD;
-  load_tile(Ks, P.k, kt * kBN, P.T, ks, kh * kD);
-  load_tile(Vs, P.v, kt * kBN, P.T, ks, kh * kD);
+  auto stage = [&](int qt, int b) {  // query tile qt into buffer b
+    uint16_t* q = QD + (b * 2) * 64 * kLd;
+    load_tile_async(q, P.q, qt * kBM, P.T, qs, h * kD);
+    load_tile_async(q + 64 * kLd, P.dout, qt * kBM, P.T, qs, h * kD);
+    for (int i = threadIdx.x; i < 64; i += blockDim.x) {
+      const int row = qt * kBM + i;
+      LD[b * 128 + i] = row < P.T ? P.lse[static_cast<int64_t>(h) * P.T + row] * kLog2e : 0.0f;
+      LD[b * 128 + 64 + i] = row < P.T ? P.D[static_cast<int64_t>(h) * P.T + row] : 0.0f;
+    }
+  };
+  load_tile_async(Ks, P.k, kt * kBN, P.T, ks, kh * kD);
+  load_tile_async(Vs, P.v, kt * kBN, P.T, ks, kh * kD);
+  stage(kt, 0);
+  cp_async_commit();
   const float c = P.scale * kLog2e;
   const int keys[2] = {kt * kBN + m0 + g, kt * kBN + m0 + g + 8};
   float dk[16][4], dv[16][4];
@@ -333,14 +374,14 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const __grid_constan
     for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.0f;
   const int q_tiles = (P.T + kBM - 1) / kBM;
   for (int qt = kt; qt < q_tiles; ++qt) {
-    __syncthreads();
-    load_tile(Qs, P.q, qt * kBM, P.T, qs, h * kD);
-    load_tile(dOs, P.dout, qt * kBM, P.T, qs, h * kD);
-    for (int i = threadIdx.x; i < 64; i += blockDim.x) {
-      const int row = qt * kBM + i;
-      lse_s[i] = row < P.T ? P.lse[static_cast<int64_t>(h) * P.T + row] * kLog2e : 0.0f;
-      D_s[i] = row < P.T ? P.D[static_cast<int64_t>(h) * P.T + row] : 0.0f;
-    }
+    const int b = (qt - kt) & 1;
+    const uint16_t* Qs = QD + (b * 2) * 64 * kLd;
+    const uint16_t* dOs = Qs + 64 * kLd;
+    const float* lse_s = LD + b * 128;
+    const float* D_s = lse_s + 64;
+    if (qt + 1 < q_tiles) stage(qt + 1, b ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
     __syncthreads();
     float s[8][4];
     gemm_xyt(s, Ks, m0, Qs);  // S^T = K Q^T
@@ -363,6 +404,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const __grid_constan
         s[j][e] = s[j][e] * (dp[j][e] - D_s[qi]);  // dS^T
       }
     gemm_py(dk, s, Qs);  // dK += dS^T Q
+    __syncthreads();
   }
   // this head's partials: part[h][key][c] (dK unscaled), part[H + h][key][c] (dV)
 #pragma unroll
@@ -419,7 +461,7 @@ cudaError_t launch_attention_fwd(const void* q, const void* k, const void* v, vo
                                  int64_t T, int H, int KV, float scale, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t rc = cudaSuccess;
-  const int smem = 3 * kTileBytes;
+  const int smem = 5 * kTileBytes;  // Q + double-buffered K, V
   if (set_smem(attn_fwd_kernel, smem, once, rc) != cudaSuccess) return rc;
   AttnArgs P{};
   P.q = static_cast<const uint16_t*>(q);
@@ -442,7 +484,7 @@ cudaError_t launch_attention_bwd(const void* q, const void* k, const void* v, co
                                  cudaStream_t st) {
   static std::once_flag once_q, once_kv;
   static cudaError_t rc_q = cudaSuccess, rc_kv = cudaSuccess;
-  const int smem_q = 4 * kTileBytes, smem_kv = 4 * kTileBytes + 2 * 64 * 4;
+  const int smem_q = 6 * kTileBytes, smem_kv = 6 * kTileBytes + 2 * 2 * 64 * 4;
   if (set_smem(attn_bwd_dq_kernel, smem_q, once_q, rc_q) != cudaSuccess) return rc_q;
   if (set_smem(attn_bwd_dkdv_kernel, smem_kv, once_kv, rc_kv) != cudaSuccess) return rc_kv;
   AttnArgs P{};
