@@ -212,3 +212,24 @@ def test_dropout_validation_before_cuda():
     drop = hsnf4.FwdArgs(hsnf4.Nf4WeightC(0, 0, 128, 256), 0, 0, 0, 0, 1, 0.1, 0, 1, 2)
     assert hsnf4.group_fwd_workspace_bytes([drop], 64, 16) >= \
         hsnf4.group_fwd_workspace_bytes([plain], 64, 16) + 64 * 256 * 2
+
+
+@pytest.mark.slow
+def test_bench_reference_arm_prints_its_json_line():
+    """`bench.py --impl reference` (the oracle on the host cores) runs on CPU
+    and prints one JSON line with the contract's keys."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3", "--ref-seconds", "0.2"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = [l for l in r.stdout.splitlines() if l.startswith("{")][-1]
+    d = json.loads(line)
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["config"]["workload"] == "qwen2.5-7b-layer"
