@@ -182,10 +182,10 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
     }
     for (int s = 0; s < SC; ++s) {
       mbar_init(&c_full[s], 1);
-      mbar_init(&c_empty[s], 128);
+      mbar_init(&c_empty[s], 4);  // one arrival per warp of the consuming warpgroup
     }
     for (int s = 0; s < SA; ++s) {
-      mbar_init(&a_full[s], P.dense ? 1 : 128);  // TMA (dense) or one dequant warpgroup
+      mbar_init(&a_full[s], P.dense ? 1 : 4);  // TMA (dense) or the 4 warps of a warpgroup
       mbar_init(&a_empty[s], 1);
     }
     mbar_init(lora_full, 1);
@@ -434,7 +434,8 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       }
       const uint4* src = reinterpret_cast<const uint4*>(c_tile(sc) + code_off);
       const uint4 c0 = src[0], c1 = src[1];
-      mbar_arrive(&c_empty[sc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c_empty[sc]);
       const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
       const Nf4Table tab = nf4_make_table(P.cb, a);
       if (gc >= SA && !mbar_wait(&a_empty[sa], ((gc / SA) - 1) & 1, abort_flag, &g_gemm_flags,
@@ -448,8 +449,9 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
         const uint4 v = nf4_dequant8(words[w], tab);
         *reinterpret_cast<uint4*>(dst + ((w ^ (line & 7)) << 4)) = v;
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&a_full[sa]);
+      fence_proxy_async_smem();  // each thread's tile writes -> visible to the MMA (async proxy)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[sa]);
     }
   } else {
     // -------------------------------------------------- epilogue (warps 8..11)
