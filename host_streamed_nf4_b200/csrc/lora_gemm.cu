@@ -143,6 +143,22 @@ __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// named barrier that also ANDs a predicate over its n threads: every thread
+// leaves with the same answer, so a group that leaves its loop on a failed
+// wait leaves it together and never strands the others at a barrier
+__device__ __forceinline__ bool named_sync_and(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_constant__ GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -467,10 +483,11 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       const int NB = P.n_buf;
       const int buf = NB > 1 ? (lu & 1) : 0;
       const uint32_t acc0 = tmem + static_cast<uint32_t>(buf * 256) + lane_base;
-      bool ok = mbar_wait(&acc_full[buf], (lu / NB) & 1, abort_flag, &g_gemm_flags,
-                          kFlagEpilogue);
-      ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld is warp-collective
-      if (!ok) break;
+      const bool ok = mbar_wait(&acc_full[buf], (lu / NB) & 1, abort_flag, &g_gemm_flags,
+                                kFlagEpilogue);
+      // all four warps go on or stop together (the tile loop below meets at
+      // a named barrier; tcgen05.ld is warp-collective)
+      if (!named_sync_and(1, 128, ok)) break;
       tc_fence_after();
       const int tile = U.tt * pr.m_tiles + U.mt;
       if (pr.splits > 1) {
