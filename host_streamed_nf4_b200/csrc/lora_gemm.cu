@@ -159,6 +159,28 @@ __device__ __forceinline__ bool named_sync_and(int id, int n, bool v) {
   return r != 0;
 }
 
+// Position in a ring of n stages: the stage and the parity of the phase in
+// which it is filled this round.  Stepping it costs a compare, where
+// g % n and g / n by a run-time n would cost a division on every K step of
+// the critical path.
+struct Ring {
+  int s = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ void step(int n) {
+    if (++s == n) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+  __device__ __forceinline__ void step2(int n) {  // two stages at once (n >= 2)
+    s += 2;
+    if (s >= n) {
+      s -= n;
+      ph ^= 1u;
+    }
+  }
+};
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_constant__ GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -230,15 +252,16 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
     // -------------------------------------------------- activations + rank-r operands
     if (lane == 0) {
       int g = 0, lu = 0;
+      Ring xr;
       const uint32_t lora_tx = static_cast<uint32_t>(plan.st_off - plan.la_off);
       bool ok = true;
       for (int ui = u_begin; ui < u_end && ok; ++ui, ++lu) {
         const Unit U = unpack_unit(P, P.units[ui]);
         const GemmProblem& pr = P.prob[U.p];
         const int m0 = U.mt * kTileM, t0 = U.tt * BN;
-        for (int kb = U.kb0; kb < U.kb1; ++kb, ++g) {
-          const int s = g % SX;
-          if (g >= SX && !mbar_wait(&x_empty[s], ((g / SX) - 1) & 1, abort_flag, &g_gemm_flags,
+        for (int kb = U.kb0; kb < U.kb1; ++kb, ++g, xr.step(SX)) {
+          const int s = xr.s;
+          if (g >= SX && !mbar_wait(&x_empty[s], xr.ph ^ 1u, abort_flag, &g_gemm_flags,
                                     kFlagProducer)) {
             ok = false;
             break;
@@ -276,15 +299,17 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
     // the UMMA operand layout the dequant warps would have written
     if (lane == 0) {
       int g = 0;
+      Ring cr;  // over the A ring (dense base) or the code ring
+      const int CS = P.dense ? SA : SC;
       bool ok = true;
       for (int ui = u_begin; ui < u_end && ok; ++ui) {
         const Unit U = unpack_unit(P, P.units[ui]);
         const GemmProblem& pr = P.prob[U.p];
         const int m0 = U.mt * kTileM;
-        for (int kb = U.kb0; kb < U.kb1; ++kb, ++g) {
+        for (int kb = U.kb0; kb < U.kb1; ++kb, ++g, cr.step(CS)) {
           if (P.dense) {
-            const int s = g % SA;
-            if (g >= SA && !mbar_wait(&a_empty[s], ((g / SA) - 1) & 1, abort_flag, &g_gemm_flags,
+            const int s = cr.s;
+            if (g >= SA && !mbar_wait(&a_empty[s], cr.ph ^ 1u, abort_flag, &g_gemm_flags,
                                       kFlagProducer)) {
               ok = false;
               break;
@@ -300,8 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
             last_c = g;
             continue;
           }
-          const int s = g % SC;
-          if (g >= SC && !mbar_wait(&c_empty[s], ((g / SC) - 1) & 1, abort_flag, &g_gemm_flags,
+          const int s = cr.s;
+          if (g >= SC && !mbar_wait(&c_empty[s], cr.ph ^ 1u, abort_flag, &g_gemm_flags,
                                     kFlagProducer)) {
             ok = false;
             break;
@@ -340,7 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
           make_idesc_bf16(kTileM, BN > 256 ? BN - 256 : 16, MODE == kGemmDx ? 1 : 0, 0);
       const bool two = P.n_acc > 1;
       const int NB = P.n_buf;
-      int g = 0, lu = 0;
+      int lu = 0;
+      Ring xr, ar;
       bool ok = true;
       for (int ui = u_begin; ui < u_end && ok; ++ui, ++lu) {
         const Unit U = unpack_unit(P, P.units[ui]);
@@ -352,10 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
           if (!ok) break;
           tc_fence_after();
         }
-        for (int kb = U.kb0; kb < U.kb1; ++kb, ++g) {
-          const int sx = g % SX, sa = g % SA;
-          ok = mbar_wait(&x_full[sx], (g / SX) & 1, abort_flag, &g_gemm_flags, kFlagMma) &&
-               mbar_wait(&a_full[sa], (g / SA) & 1, abort_flag, &g_gemm_flags, kFlagMma);
+        for (int kb = U.kb0; kb < U.kb1; ++kb, xr.step(SX), ar.step(SA)) {
+          const int sx = xr.s, sa = ar.s;
+          ok = mbar_wait(&x_full[sx], xr.ph, abort_flag, &g_gemm_flags, kFlagMma) &&
+               mbar_wait(&a_full[sa], ar.ph, abort_flag, &g_gemm_flags, kFlagMma);
           if (!ok) break;
           tc_fence_after();
           const uint64_t ad = a_desc0 + static_cast<uint64_t>(sa * a_stage);
@@ -437,14 +463,20 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
     }
     float a_next = have ? absmax_at(U, kb) : 0.0f;
     bool ok = true;
+    Ring cr, ar;  // this warpgroup's stages: grp, grp + 2, ... (both rings hold >= 2)
+    cr.s = grp;
+    ar.s = grp;
     while (have && ok) {
       const float a = a_next;
       const int gc = g;
       have = advance(ui, kb, U, 2);
       g += 2;
       if (have) a_next = absmax_at(U, kb);
-      const int sc = gc % SC, sa = gc % SA;
-      if (!mbar_wait(&c_full[sc], (gc / SC) & 1, abort_flag, &g_gemm_flags, kFlagDequant)) {
+      const int sc = cr.s, sa = ar.s;
+      const uint32_t phc = cr.ph, pha = ar.ph;
+      cr.step2(SC);
+      ar.step2(SA);
+      if (!mbar_wait(&c_full[sc], phc, abort_flag, &g_gemm_flags, kFlagDequant)) {
         ok = false;
         break;
       }
@@ -454,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       if (lane == 0) mbar_arrive(&c_empty[sc]);
       const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
       const Nf4Table tab = nf4_make_table(P.cb, a);
-      if (gc >= SA && !mbar_wait(&a_empty[sa], ((gc / SA) - 1) & 1, abort_flag, &g_gemm_flags,
+      if (gc >= SA && !mbar_wait(&a_empty[sa], pha ^ 1u, abort_flag, &g_gemm_flags,
                                  kFlagDequant)) {
         ok = false;
         break;
