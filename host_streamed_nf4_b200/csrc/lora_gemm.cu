@@ -9,20 +9,30 @@
 //     dX[T, k_in] = dY[T, n_out] deq(W) + (s u)[T, r] A[r, k_in]
 //
 // Both are computed transposed, with the weight on the MMA's M side so that
-// a CTA dequantizes each 128-row slab of W once for up to 512 tokens:
+// each 128-row slab of W is dequantized once for up to 512 tokens:
 //     fwd: D[n, t] = sum_k deq(W)[n, k] X[t, k]      (A operand K-major)
 //     dx : D[k, t] = sum_n deq(W)[n, k] dY[t, n]     (A operand MN-major)
 // The rank-r term is one more K-slice of the same accumulator:
 //     fwd: D[n, t] += sum_j B[n, j] (s t)[t, j]
 //     dx : D[k, t] += sum_j A[j, k] (s u)[t, j]
 //
-// Work units are (problem, 128-row tile, token tile, K split).  The host
-// assigns them to persistent CTAs longest-first (static, deterministic).
-// A problem whose units are long and few is split along K: each split
-// writes its fp32 tile to workspace and the last split to arrive adds them
+// The kernel runs as clusters of two CTAs on neighbouring SMs that share
+// every MMA (tcgen05 cta_group::2, M = 256): each CTA dequantizes its own
+// 128 rows of the 256-row tile and holds half of each token block, and the
+// even CTA issues one instruction for both.  Per SM that halves the MMA
+// instructions and the activation bytes staged per K step.  Each CTA fills
+// its own rings with its own barriers; the odd CTA's otherwise idle MMA
+// warp forwards "my half of stage g is ready" (and "my epilogue drained
+// the accumulator") to the even CTA's pair barriers, and the MMA
+// completion is committed to the matching barriers of both CTAs.
+//
+// Work units are (problem, 256-row tile, token tile, K split).  The host
+// assigns them to persistent CTA pairs longest-first (static,
+// deterministic).  A problem whose units are long and few is split along K:
+// each split writes its fp32 tile to workspace and a second pass adds them
 // in split order, so the sum does not depend on timing.
 //
-// CTA roles (15 warps):
+// CTA roles (15 warps, the same in both CTAs of a pair):
 //   warps 0-3, 4-7   two dequant warpgroups taking alternate K steps: raw
 //                    codes (smem) -> bf16 A tile in the UMMA 128B-swizzled
 //                    layout, one 64-element block (one 128-byte line) per
@@ -31,7 +41,8 @@
 //                    coalesced bf16 rows of the output (or fp32 partials);
 //   warp 12          TMA producer of the activation tiles and rank-r operands;
 //   warp 13          TMA producer of the raw code tiles;
-//   warp 14          TMEM owner and UMMA issuer (one elected thread).
+//   warp 14          TMEM owner; UMMA issuer of the pair (even CTA) or the
+//                    forwarder of the odd CTA's ready signals.
 // Every wait is bounded (ptx.cuh); a timed-out wait records a flag in
 // g_gemm_flags, the CTA drains what it started and exits.
 #include <cuda.h>
@@ -63,7 +74,8 @@ enum : unsigned int {
   kFlagSelftest = 64u,
 };
 
-constexpr int kTileM = 128;                    // rows of the MMA (W rows or k_in columns)
+constexpr int kTileM = 128;                    // rows of one CTA (W rows or k_in columns)
+constexpr int kPairM = 2 * kTileM;             // rows of the pair's MMA (one unit)
 constexpr int kStepK = 64;                     // contraction per pipeline step
 constexpr int kCodeBytes = 4096;               // raw codes of one step (128 x 64 / 2)
 constexpr int kATileBytes = kTileM * 128;      // dequantized bf16 A tile
@@ -73,19 +85,19 @@ constexpr int kThreads = 15 * 32;
 constexpr int kWarpEpi = 8, kWarpProdX = 12, kWarpProdC = 13, kWarpMma = 14;
 
 struct GemmProblem {
-  CUtensorMap map_act;    // X / dY: bf16 [T, contraction], box {64, min(BN,256)}, 128B swizzle
+  CUtensorMap map_act;    // X / dY: bf16 [T, contraction], box {64, min(BN/2,128)}, 128B swizzle
   CUtensorMap map_codes;  // uint8 [n_out, k_in/2]; box {32, 128} fwd, {64, 64} dx; dense:
                           // bf16 [n_out, k_in], box {64, 128} fwd, {64, 64} dx, 128B swizzle
   CUtensorMap map_lo_a;   // fwd: B [n_out, r] box {16, 128} 32B; dx: A [r, k_in] box {64, r_pad} 128B
-  CUtensorMap map_lo_b;   // s*t or s*u: bf16 [T, r_pad], box {16, min(BN,256)}, 32B swizzle
+  CUtensorMap map_lo_b;   // s*t or s*u: bf16 [T, r_pad], box {16, min(BN/2,128)}, 32B swizzle
   const float* absmax;
   uint16_t* out;          // bf16 [T, m_total]
   float* partial;         // split-K partial tiles (fp32 [BN tokens][128 rows] each), or null
-  int n_out, k_in, m_total, nk, kblocks, m_tiles, splits;
+  int n_out, k_in, m_total, nk, kblocks, m_tiles, splits;  // m_tiles: 256-row tiles
 };
 
 constexpr int kMaxProblems = 8;
-constexpr int kMaxCtas = 160;
+constexpr int kMaxPairs = 80;
 constexpr int kMaxUnits = 3072;
 
 struct GemmParams {
@@ -95,7 +107,7 @@ struct GemmParams {
   int n_buf;  // TMEM accumulator buffers: 2 (BN <= 256: the epilogue of a unit
               // overlaps the next unit's MMAs) or 1 (BN = 512 fills TMEM)
   int dense;  // 1: map_codes is the bf16 weight, TMA-loaded straight into the A ring
-  uint16_t cta_off[kMaxCtas + 1];
+  uint16_t pair_off[kMaxPairs + 1];  // units of pair c: units[pair_off[c] .. pair_off[c+1])
   uint32_t units[kMaxUnits];  // problem(3) | split(5) | token tile(6) | row tile(18)
 };
 
@@ -127,15 +139,15 @@ struct SmemPlan {
 __host__ __device__ inline SmemPlan smem_plan(int mode, int BN, int sx, int sc, int sa, int r_pad) {
   SmemPlan p;
   const int slices = r_pad / 16;
-  p.x_bytes = BN * 128;
+  p.x_bytes = (BN / 2) * 128;  // this CTA's half of the token block
   p.a_off = sx * p.x_bytes;
   p.c_off = p.a_off + sa * kATileBytes;
   p.la_off = p.c_off + sc * kCodeBytes;
   const int la = (mode == kGemmFwd) ? slices * 4096 : 2 * r_pad * 128;
   p.lb_off = p.la_off + la;
-  p.st_off = p.lb_off + slices * BN * 32;
+  p.st_off = p.lb_off + slices * (BN / 2) * 32;
   p.bar_off = p.st_off + 2 * kStageElems * 2;
-  p.total = p.bar_off + (2 * sx + 2 * sc + 2 * sa + 8) * 8 + 32;
+  p.total = p.bar_off + (2 * sx + 2 * sc + 2 * sa + 16) * 8 + 32;
   return p;
 }
 
@@ -182,7 +194,8 @@ struct Ring {
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_constant__ GemmParams P) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    lora_gemm_kernel(const __grid_constant__ GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -190,8 +203,15 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
   const SmemPlan plan = smem_plan(MODE, BN, SX, SC, SA, P.r_pad);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slices = P.r_pad / 16;
-  const int u_begin = P.cta_off[blockIdx.x], u_end = P.cta_off[blockIdx.x + 1];
-  const int box_rows = BN < 256 ? BN : 256;  // TMA boxes of activations / rank-r factor
+  const uint32_t crank = cluster_ctarank();  // 0: issues the pair's MMAs; 1: forwards
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int u_begin = P.pair_off[pair], u_end = P.pair_off[pair + 1];
+  // This CTA's share of a token block: per accumulator h (tokens t0 + 256 h
+  // .. + min(256, BN - 256 h)) the half starting crank * box_rows further,
+  // staged as rows h * box_rows .. of the X tile and of each rank-r slice.
+  const int half_rows = BN / 2;
+  const int box_rows = half_rows < 128 ? half_rows : 128;
+  const int row0 = static_cast<int>(crank) * kTileM;  // this CTA's rows within a unit
 
   uint8_t* lora_a = smem + plan.la_off;
   uint8_t* lora_b = smem + plan.lb_off;
@@ -207,7 +227,12 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
   uint64_t* acc_full = lora_empty + 1;  // [2]
   uint64_t* acc_empty = acc_full + 2;   // [2]
   uint64_t* drain_bar = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  // the even CTA's view of the odd CTA (arrived on by its forwarder)
+  uint64_t* pair_full = drain_bar + 1;  // [4]: both halves of K step g staged (ring of SP)
+  uint64_t* pair_lora = pair_full + 4;  // the odd CTA's rank-r operands staged
+  uint64_t* pair_acc = pair_lora + 1;   // [2]: the odd CTA's epilogue drained buffer b
+  const int SP = SX < SA ? SX : SA;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pair_acc + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto x_tile = [&](int s) { return smem + s * plan.x_bytes; };
   auto a_tile = [&](int s) { return smem + plan.a_off + s * kATileBytes; };
@@ -233,15 +258,18 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       mbar_init(&acc_empty[b], 128);
     }
     mbar_init(drain_bar, 1);
+    for (int s = 0; s < 4; ++s) mbar_init(&pair_full[s], 1);
+    mbar_init(pair_lora, 1);
+    for (int b = 0; b < 2; ++b) mbar_init(&pair_acc[b], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kWarpMma) {
-    tmem_alloc(tmem_slot, static_cast<uint32_t>(P.tmem_cols));
-    tmem_relinquish();
+  if (warp == kWarpMma) {  // both CTAs: one allocation of the same columns in each TMEM
+    tmem_alloc_pair(tmem_slot, static_cast<uint32_t>(P.tmem_cols));
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised before any cross-CTA arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -258,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       for (int ui = u_begin; ui < u_end && ok; ++ui, ++lu) {
         const Unit U = unpack_unit(P, P.units[ui]);
         const GemmProblem& pr = P.prob[U.p];
-        const int m0 = U.mt * kTileM, t0 = U.tt * BN;
+        const int m0 = U.mt * kPairM + row0, t0 = U.tt * BN;
         for (int kb = U.kb0; kb < U.kb1; ++kb, ++g, xr.step(SX)) {
           const int s = xr.s;
           if (g >= SX && !mbar_wait(&x_empty[s], xr.ph ^ 1u, abort_flag, &g_gemm_flags,
@@ -266,10 +294,10 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&x_full[s], static_cast<uint32_t>(BN * 128));
-          for (int h = 0; h * box_rows < BN; ++h)
+          mbar_arrive_expect_tx(&x_full[s], static_cast<uint32_t>(half_rows * 128));
+          for (int h = 0; h < P.n_acc; ++h)
             tma_load_2d(x_tile(s) + h * box_rows * 128, &pr.map_act, &x_full[s], kb * kStepK,
-                        t0 + h * box_rows);
+                        t0 + h * 256 + static_cast<int>(crank) * box_rows);
           last_x = g;
         }
         if (!ok) break;
@@ -287,9 +315,9 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
             tma_load_2d(lora_a + h * P.r_pad * 128, &pr.map_lo_a, lora_full, m0 + h * 64, 0);
         }
         for (int j = 0; j < slices; ++j)
-          for (int h = 0; h * box_rows < BN; ++h)
-            tma_load_2d(lora_b + j * BN * 32 + h * box_rows * 32, &pr.map_lo_b, lora_full, j * 16,
-                        t0 + h * box_rows);
+          for (int h = 0; h < P.n_acc; ++h)
+            tma_load_2d(lora_b + j * half_rows * 32 + h * box_rows * 32, &pr.map_lo_b, lora_full,
+                        j * 16, t0 + h * 256 + static_cast<int>(crank) * box_rows);
         last_l = lu;
       }
     }
@@ -305,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       for (int ui = u_begin; ui < u_end && ok; ++ui) {
         const Unit U = unpack_unit(P, P.units[ui]);
         const GemmProblem& pr = P.prob[U.p];
-        const int m0 = U.mt * kTileM;
+        const int m0 = U.mt * kPairM + row0;
         for (int kb = U.kb0; kb < U.kb1; ++kb, ++g, cr.step(CS)) {
           if (P.dense) {
             const int s = cr.s;
@@ -340,48 +368,84 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
         }
       }
     }
+  } else if (warp == kWarpMma && crank == 1) {
+    // -------------------------------------------------- forwarder (odd CTA)
+    // Mirrors the issuer's order: before a unit, "my epilogue drained this
+    // buffer"; per K step, "my X and A halves of step g are staged"; after
+    // the unit's K steps, "my rank-r operands are staged".
+    if (lane == 0) {
+      const int NB = P.n_buf;
+      int lu = 0;
+      Ring xr, ar, pr_;
+      bool ok = true;
+      for (int ui = u_begin; ui < u_end && ok; ++ui, ++lu) {
+        const Unit U = unpack_unit(P, P.units[ui]);
+        const int buf = NB > 1 ? (lu & 1) : 0;
+        if (lu >= NB) {
+          if (!mbar_wait(&acc_empty[buf], ((lu / NB) - 1) & 1, abort_flag, &g_gemm_flags,
+                         kFlagMma))
+            break;
+          mbar_arrive_cluster(&pair_acc[buf], 0);
+        }
+        for (int kb = U.kb0; kb < U.kb1; ++kb, xr.step(SX), ar.step(SA), pr_.step(SP)) {
+          ok = mbar_wait(&x_full[xr.s], xr.ph, abort_flag, &g_gemm_flags, kFlagMma) &&
+               mbar_wait(&a_full[ar.s], ar.ph, abort_flag, &g_gemm_flags, kFlagMma);
+          if (!ok) break;
+          mbar_arrive_cluster(&pair_full[pr_.s], 0);
+        }
+        if (!ok) break;
+        if (!mbar_wait(lora_full, lu & 1, abort_flag, &g_gemm_flags, kFlagLora)) break;
+        mbar_arrive_cluster(pair_lora, 0);
+      }
+    }
   } else if (warp == kWarpMma) {
-    // -------------------------------------------------- UMMA issuer
+    // -------------------------------------------------- UMMA issuer of the pair (even CTA)
     if (lane == 0) {
       // All descriptors are computed once: per stage and per 16-wide K step
       // only the start-address field changes (in 16-byte units; shared
       // addresses stay below 256 KiB, so the 14-bit field never carries).
+      // They address this CTA's shared memory; the odd CTA's operands sit
+      // at the same offsets in its own.
       //   fwd A: 128 rows x 128 B lines (K-major, 8-row groups 1 KiB apart);
       //          a 16-wide K step is 32 B further along each line.
       //   dx  A: two 64-column atoms 8 KiB apart (LBO), 8-row groups 1 KiB
       //          apart (SBO); a 16-row K step is 2 KiB further.
       //   B (activations): K-major, 8-row groups 1 KiB apart; accumulator
-      //          h reads rows h*256.. (32 KiB further).
+      //          h reads this CTA's rows h*128.. (16 KiB further).
       const uint64_t a_desc0 =
           (MODE == kGemmFwd) ? make_sdesc(smem_u32(a_tile(0)), 16, 1024, kLayoutSw128)
                              : make_sdesc(smem_u32(a_tile(0)), 64 * 128, 1024, kLayoutSw128);
       const uint64_t b_desc0 = make_sdesc(smem_u32(x_tile(0)), 16, 1024, kLayoutSw128);
       const uint32_t a_k16 = (MODE == kGemmFwd) ? (32 >> 4) : (2048 >> 4);
       const uint32_t a_stage = kATileBytes >> 4, b_stage = plan.x_bytes >> 4;
-      const uint32_t b_half = (256 * 128) >> 4;
+      const uint32_t b_half = static_cast<uint32_t>(box_rows * 128) >> 4;
+      const uint32_t lb_half = static_cast<uint32_t>(box_rows * 32) >> 4;
       const int n0 = BN < 256 ? BN : 256;
-      const uint32_t idesc0 = make_idesc_bf16(kTileM, n0, MODE == kGemmDx ? 1 : 0, 0);
+      const uint32_t idesc0 = make_idesc_bf16(kPairM, n0, MODE == kGemmDx ? 1 : 0, 0);
       const uint32_t idesc1 =
-          make_idesc_bf16(kTileM, BN > 256 ? BN - 256 : 16, MODE == kGemmDx ? 1 : 0, 0);
+          make_idesc_bf16(kPairM, BN > 256 ? BN - 256 : 16, MODE == kGemmDx ? 1 : 0, 0);
       const bool two = P.n_acc > 1;
       const int NB = P.n_buf;
+      constexpr uint16_t kBoth = 3;  // commit to the barriers of both CTAs
       int lu = 0;
-      Ring xr, ar;
+      Ring xr, ar, pr_;
       bool ok = true;
       for (int ui = u_begin; ui < u_end && ok; ++ui, ++lu) {
         const Unit U = unpack_unit(P, P.units[ui]);
         const int buf = NB > 1 ? (lu & 1) : 0;
         const uint32_t acc0 = tmem + static_cast<uint32_t>(buf * 256);
-        if (lu >= NB) {  // the epilogue has drained this buffer's previous unit
-          ok = mbar_wait(&acc_empty[buf], ((lu / NB) - 1) & 1, abort_flag, &g_gemm_flags,
-                         kFlagMma);
+        if (lu >= NB) {  // both epilogues have drained this buffer's previous unit
+          const uint32_t ph = ((lu / NB) - 1) & 1;
+          ok = mbar_wait(&acc_empty[buf], ph, abort_flag, &g_gemm_flags, kFlagMma) &&
+               mbar_wait(&pair_acc[buf], ph, abort_flag, &g_gemm_flags, kFlagMma);
           if (!ok) break;
           tc_fence_after();
         }
-        for (int kb = U.kb0; kb < U.kb1; ++kb, xr.step(SX), ar.step(SA)) {
+        for (int kb = U.kb0; kb < U.kb1; ++kb, xr.step(SX), ar.step(SA), pr_.step(SP)) {
           const int sx = xr.s, sa = ar.s;
           ok = mbar_wait(&x_full[sx], xr.ph, abort_flag, &g_gemm_flags, kFlagMma) &&
-               mbar_wait(&a_full[sa], ar.ph, abort_flag, &g_gemm_flags, kFlagMma);
+               mbar_wait(&a_full[sa], ar.ph, abort_flag, &g_gemm_flags, kFlagMma) &&
+               mbar_wait(&pair_full[pr_.s], pr_.ph, abort_flag, &g_gemm_flags, kFlagMma);
           if (!ok) break;
           tc_fence_after();
           const uint64_t ad = a_desc0 + static_cast<uint64_t>(sa * a_stage);
@@ -390,15 +454,17 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
 #pragma unroll
           for (int k16 = 0; k16 < 4; ++k16) {
             const uint32_t acc = (k16 > 0) ? 1u : first;
-            umma_bf16(acc0, ad + k16 * a_k16, bd + k16 * 2, idesc0, acc);
-            if (two) umma_bf16(acc0 + 256, ad + k16 * a_k16, bd + b_half + k16 * 2, idesc1, acc);
+            umma_bf16_pair(acc0, ad + k16 * a_k16, bd + k16 * 2, idesc0, acc);
+            if (two)
+              umma_bf16_pair(acc0 + 256, ad + k16 * a_k16, bd + b_half + k16 * 2, idesc1, acc);
           }
           mma_started = true;
-          umma_commit(&x_empty[sx]);
-          umma_commit(&a_empty[sa]);
+          umma_commit_pair(&x_empty[sx], kBoth);
+          umma_commit_pair(&a_empty[sa], kBoth);
         }
         if (!ok) break;
-        ok = mbar_wait(lora_full, lu & 1, abort_flag, &g_gemm_flags, kFlagLora);
+        ok = mbar_wait(lora_full, lu & 1, abort_flag, &g_gemm_flags, kFlagLora) &&
+             mbar_wait(pair_lora, lu & 1, abort_flag, &g_gemm_flags, kFlagLora);
         if (!ok) break;
         if (U.split == 0) {  // the rank-r slice is added once, by split 0
           tc_fence_after();
@@ -407,14 +473,14 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
             const uint64_t adesc =
                 (MODE == kGemmFwd) ? make_sdesc(la + j * 4096, 16, 256, kLayoutSw32)
                                    : make_sdesc(la + j * 2048, P.r_pad * 128, 1024, kLayoutSw128);
-            const uint64_t bdesc = make_sdesc(lb + j * BN * 32, 16, 256, kLayoutSw32);
-            umma_bf16(acc0, adesc, bdesc, idesc0, 1u);
-            if (two) umma_bf16(acc0 + 256, adesc, bdesc + ((256 * 32) >> 4), idesc1, 1u);
+            const uint64_t bdesc = make_sdesc(lb + j * half_rows * 32, 16, 256, kLayoutSw32);
+            umma_bf16_pair(acc0, adesc, bdesc, idesc0, 1u);
+            if (two) umma_bf16_pair(acc0 + 256, adesc, bdesc + lb_half, idesc1, 1u);
           }
           mma_started = true;
         }
-        umma_commit(lora_empty);
-        umma_commit(&acc_full[buf]);
+        umma_commit_pair(lora_empty, kBoth);
+        umma_commit_pair(&acc_full[buf], kBoth);
       }
     }
   } else if (warp < kWarpEpi && P.dense) {
@@ -428,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
     // this thread's absmax for K step kb of unit U (0 past the weight's edge)
     auto absmax_at = [&](const Unit& U, int kb) -> float {
       const GemmProblem& pr = P.prob[U.p];
-      const int m0 = U.mt * kTileM;
+      const int m0 = U.mt * kPairM + row0;
       if (MODE == kGemmFwd) {
         const int row = m0 + i;
         return row < pr.n_out ? __ldg(pr.absmax + static_cast<int64_t>(row) * pr.kblocks + kb)
@@ -510,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
     for (int ui = u_begin; ui < u_end; ++ui, ++lu) {
       const Unit U = unpack_unit(P, P.units[ui]);
       const GemmProblem& pr = P.prob[U.p];
-      const int m0 = U.mt * kTileM, t0 = U.tt * BN;
+      const int m0 = U.mt * kPairM + row0, t0 = U.tt * BN;
       const int M = pr.m_total;
       const int NB = P.n_buf;
       const int buf = NB > 1 ? (lu & 1) : 0;
@@ -521,7 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       // a named barrier; tcgen05.ld is warp-collective)
       if (!named_sync_and(1, 128, ok)) break;
       tc_fence_after();
-      const int tile = U.tt * pr.m_tiles + U.mt;
+      // this CTA's 128-row half of the unit's tile
+      const int tile = (U.tt * pr.m_tiles + U.mt) * 2 + static_cast<int>(crank);
       if (pr.splits > 1) {
         // this split's fp32 tile -> workspace, token-major ([BN][128]) so that a
         // warp's 32 rows of one token are 128 contiguous bytes; the splits are
@@ -585,16 +652,18 @@ __global__ void __launch_bounds__(kThreads, 1) lora_gemm_kernel(const __grid_con
       for (int g = (last_c - S + 1 > 0 ? last_c - S + 1 : 0); g <= last_c; ++g)
         if (!mbar_wait(&full[g % S], (g / S) & 1, &never, &g_gemm_flags, kFlagDrain)) break;
     }
-    if (warp == kWarpMma && lane == 0 && mma_started) {
-      umma_commit(drain_bar);
+    if (warp == kWarpMma && lane == 0 && mma_started) {  // the even CTA's issued MMAs
+      umma_commit_pair(drain_bar, 1);
       mbar_wait(drain_bar, 0, &never, &g_gemm_flags, kFlagDrain);
     }
   }
   tc_fence_before();
-  __syncthreads();
+  // neither CTA leaves while the pair's MMAs may still read its shared memory
+  // or a forwarder may still arrive on the even CTA's barriers
+  cluster_sync();
   if (warp == kWarpMma) {
     tc_fence_after();
-    tmem_dealloc(tmem, static_cast<uint32_t>(P.tmem_cols));
+    tmem_dealloc_pair(tmem, static_cast<uint32_t>(P.tmem_cols));
   }
 }
 
@@ -768,7 +837,7 @@ static void plan_splits(GemmMode mode, const GemmProblemDesc* probs, int n, int6
   for (int p = 0; p < n; ++p) {
     const int64_t mdim = (mode == kGemmFwd) ? probs[p].n_out : probs[p].k_in;
     const int64_t contraction = (mode == kGemmFwd) ? probs[p].k_in : probs[p].n_out;
-    tiles[p] = ((mdim + kTileM - 1) / kTileM) * ((T + BN - 1) / BN);
+    tiles[p] = ((mdim + kPairM - 1) / kPairM) * ((T + BN - 1) / BN);
     nk[p] = contraction / kStepK;
   }
   auto objective = [&](const std::vector<int>& sp) -> int64_t {
@@ -779,13 +848,13 @@ static void plan_splits(GemmMode mode, const GemmProblemDesc* probs, int n, int6
         const int64_t ks = (s + 1) * nk[p] / sp[p] - s * nk[p] / sp[p];
         costs.insert(costs.end(), static_cast<size_t>(tiles[p]), unit_cost(ks, sp[p]));
       }
-      if (sp[p] > 1) reduce_bytes += static_cast<double>(tiles[p]) * sp[p] * kTileM * BN * 4;
+      if (sp[p] > 1) reduce_bytes += static_cast<double>(tiles[p]) * sp[p] * kPairM * BN * 4;
     }
     if (costs.size() > static_cast<size_t>(3072)) return INT64_MAX;  // over the unit limit
     const int64_t reduce = reduce_bytes > 0
                                ? 4 + static_cast<int64_t>(reduce_bytes / (16384.0 * sms))
                                : 0;
-    return lpt_makespan(costs, sms) + reduce;
+    return lpt_makespan(costs, sms / 2) + reduce;  // units run on CTA pairs
   };
   std::vector<int> cur(n, 1);
   *splits = cur;
@@ -846,9 +915,9 @@ static void split_layout(GemmMode mode, const GemmProblemDesc* probs, int n, int
   for (int p = 0; p < n; ++p) {
     if (L->splits[p] <= 1) continue;
     const int64_t mdim = (mode == kGemmFwd) ? probs[p].n_out : probs[p].k_in;
-    const int64_t tiles = ((mdim + kTileM - 1) / kTileM) * t_tiles;
+    const int64_t tiles = ((mdim + kPairM - 1) / kPairM) * t_tiles;
     L->part_base[p] = part;
-    part += round_up(static_cast<size_t>(tiles) * L->splits[p] * kTileM * BN * 4, 256);
+    part += round_up(static_cast<size_t>(tiles) * L->splits[p] * kPairM * BN * 4, 256);
   }
   L->need = part;
 }
@@ -914,7 +983,7 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     const GemmProblemDesc& d = probs[p];
     const int64_t mdim = (mode == kGemmFwd) ? d.n_out : d.k_in;
     const int64_t nk = ((mode == kGemmFwd) ? d.k_in : d.n_out) / kStepK;
-    const int mt_n = static_cast<int>((mdim + kTileM - 1) / kTileM);
+    const int mt_n = static_cast<int>((mdim + kPairM - 1) / kPairM);
     if (mt_n > (1 << 18))
       return fail(HSNF4_ERR_INVALID, "lora gemm: %lld rows exceed the tile index range",
                   (long long)mdim);
@@ -930,7 +999,8 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
                 units.size(), kMaxUnits);
   std::stable_sort(units.begin(), units.end(),
                    [](const U& a, const U& b) { return a.cost > b.cost; });
-  const int G = static_cast<int>(std::min<size_t>(units.size(), std::min(sms, kMaxCtas)));
+  // persistent CTA pairs: one per two SMs
+  const int G = static_cast<int>(std::min<size_t>(units.size(), std::min(sms / 2, kMaxPairs)));
   std::vector<std::vector<uint32_t>> per(G);
   using Load = std::pair<int64_t, int>;
   std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
@@ -943,13 +1013,14 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
   }
   int k = 0;
   for (int c = 0; c < G; ++c) {
-    P.cta_off[c] = static_cast<uint16_t>(k);
+    P.pair_off[c] = static_cast<uint16_t>(k);
     for (uint32_t code : per[c]) P.units[k++] = code;
   }
-  P.cta_off[G] = static_cast<uint16_t>(k);
+  P.pair_off[G] = static_cast<uint16_t>(k);
 
   bool ok = true;
-  const int box_rows = BN < 256 ? BN : 256;
+  // each CTA of a pair stages half of every 256-token accumulator block
+  const int box_rows = BN / 2 < 128 ? BN / 2 : 128;
   for (int p = 0; p < n; ++p) {
     const GemmProblemDesc& d = probs[p];
     GemmProblem& g = P.prob[p];
@@ -961,7 +1032,7 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     g.m_total = static_cast<int>((mode == kGemmFwd) ? d.n_out : d.k_in);
     g.nk = static_cast<int>(contraction / kStepK);
     g.kblocks = static_cast<int>(d.k_in / 64);
-    g.m_tiles = (g.m_total + kTileM - 1) / kTileM;
+    g.m_tiles = (g.m_total + kPairM - 1) / kPairM;
     g.splits = L.splits[p];
     if (g.splits > 1) g.partial = reinterpret_cast<float*>(ws + L.part_base[p]);
     ok = ok && encode_2d(&g.map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.act, contraction, T,
@@ -994,9 +1065,9 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
   void* prof = prof_begin(st);
   count_launch();
   if (mode == kGemmFwd)
-    lora_gemm_kernel<kGemmFwd><<<G, kThreads, smem, st>>>(P);
+    lora_gemm_kernel<kGemmFwd><<<2 * G, kThreads, smem, st>>>(P);  // G clusters of 2
   else
-    lora_gemm_kernel<kGemmDx><<<G, kThreads, smem, st>>>(P);
+    lora_gemm_kernel<kGemmDx><<<2 * G, kThreads, smem, st>>>(P);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess && L.need) {
     // add the K-split partials in split order and write the bf16 outputs
@@ -1008,16 +1079,19 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
       const GemmProblem& g = P.prob[p];
       if (g.splits <= 1) continue;
       for (int tt = 0; tt < t_tiles; ++tt)
-        for (int mt = 0; mt < g.m_tiles; ++mt) {
-          if (R.n_tiles == kMaxReduceTiles) {
-            count_launch();
-            lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 64, 0, st>>>(R);
-            R.n_tiles = 0;
+        for (int mt = 0; mt < g.m_tiles; ++mt)
+          for (int c = 0; c < 2; ++c) {  // the two 128-row halves of the pair's tile
+            const int m0 = mt * kPairM + c * kTileM;
+            if (m0 >= g.m_total) continue;
+            if (R.n_tiles == kMaxReduceTiles) {
+              count_launch();
+              lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 64, 0, st>>>(R);
+              R.n_tiles = 0;
+            }
+            const int tile = (tt * g.m_tiles + mt) * 2 + c;
+            R.tile[R.n_tiles++] = {g.partial + static_cast<int64_t>(tile) * g.splits * kTileM * BN,
+                                   g.out, m0, tt * BN, g.m_total, g.splits};
           }
-          const int tile = tt * g.m_tiles + mt;
-          R.tile[R.n_tiles++] = {g.partial + static_cast<int64_t>(tile) * g.splits * kTileM * BN,
-                                 g.out, mt * kTileM, tt * BN, g.m_total, g.splits};
-        }
     }
     if (R.n_tiles) {
       count_launch();
