@@ -552,35 +552,63 @@ def merge_roofline(stack, dev):
 def run_e2e(args, stack, one_step, drain_copies, ws, dev):
     """Same step through the public API with host buffers: each step copies
     its activations and upstream gradients from pinned host memory and reads
-    the layer stack's adapter gradients back (device-timed)."""
+    the layer stack's adapter gradients back (device-timed).
+
+    The next step's inputs are copied on their own stream into one of two
+    device staging sets while the current step computes (its weights stream
+    on the copy stream meanwhile), and moved into the stack's input tensors
+    with one on-device copy at the start of the step, so the host link is
+    not left idle while a step's kernels run."""
     import torch
     dev_in = stack.step_inputs()  # the tensors a step reads from the host
     host_in = [torch.empty_like(v, device="cpu").pin_memory() for v in dev_in]
     for h, v in zip(host_in, dev_in):
         h.copy_(v)
+    stage = [[torch.empty_like(v) for v in dev_in] for _ in range(2)]
     grads = [stack.grad_flat]  # every dA/dB of the stack, summed over ranks
     host_grads = [torch.empty_like(g, device="cpu").pin_memory() for g in grads]
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_grads)
     compute = stack.compute
+    in_stream = torch.cuda.Stream(dev)
+    ready = [torch.cuda.Event() for _ in range(2)]
+    free = [torch.cuda.Event() for _ in range(2)]
 
-    def step_e2e():
-        for d, h in zip(dev_in, host_in):
-            d.copy_(h, non_blocking=True)
-        one_step()
-        for h, g in zip(host_grads, grads):
-            h.copy_(g, non_blocking=True)
+    def prefetch(buf, after=None):
+        # host -> staging set `buf`, once the compute stream is done with it
+        if after is not None:
+            in_stream.wait_event(after)
+        in_stream.wait_event(free[buf])
+        with torch.cuda.stream(in_stream):
+            for d, h in zip(stage[buf], host_in):
+                d.copy_(h, non_blocking=True)
+        ready[buf].record(in_stream)
 
-    for _ in range(2):
-        step_e2e()
+    def run(n, start=None):
+        for b in range(2):
+            free[b].record(compute)
+        prefetch(0, start)
+        for i in range(n):
+            buf = i % 2
+            compute.wait_event(ready[buf])
+            for d, st in zip(dev_in, stage[buf]):
+                d.copy_(st, non_blocking=True)
+            free[buf].record(compute)
+            if i + 1 < n:
+                prefetch(1 - buf)
+            one_step()
+            for h, g in zip(host_grads, grads):
+                h.copy_(g, non_blocking=True)
+
+    run(2)
     torch.cuda.synchronize(dev)
     K = args.steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(ws)
     torch.cuda.synchronize(dev)
     e0.record(compute)
-    for _ in range(K):
-        step_e2e()
+    run(K, start=e0)
+    compute.wait_stream(in_stream)
     drain_copies()
     e1.record(compute)
     torch.cuda.synchronize(dev)
