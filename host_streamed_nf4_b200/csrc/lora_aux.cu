@@ -365,49 +365,49 @@ __global__ void __launch_bounds__(256) lora_grad_group(const __grid_constant__ G
   const int jn = (P.r - jb) < 16 ? (P.r - jb) : 16;
 
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  // register staging of one token chunk: Z 64 x 64 bf16 (2 x 16 B per
-  // thread) and V 64 x 16 fp32 (4 per thread); the next chunk is loaded
-  // while the current one is multiplied
-  uint4 zr[2];
-  float vr[4];
-  auto load = [&](int tc) {
+  // register staging of token chunks: Z 64 x 64 bf16 (2 x 16 B per thread)
+  // and V 64 x 16 fp32 (4 per thread).  Two sets, so that the loads of the
+  // next two chunks are in flight while one is multiplied.
+  uint4 zr[2][2];
+  float vr[2][4];
+  auto load = [&](int set, int tc) {
     const int nt_tok = (P.T - tc) < kGrdTok ? (P.T - tc) : kGrdTok;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int v = tid + k * 256;
       const int row = v >> 3, col = (v & 7) * 8;
-      zr[k] = make_uint4(0, 0, 0, 0);
+      zr[set][k] = make_uint4(0, 0, 0, 0);
       if (row < nt_tok && col < width)
-        zr[k] = __ldg(reinterpret_cast<const uint4*>(pr.Z + static_cast<int64_t>(tc + row) * pr.C +
-                                                     c0 + col));
+        zr[set][k] = __ldg(reinterpret_cast<const uint4*>(
+            pr.Z + static_cast<int64_t>(tc + row) * pr.C + c0 + col));
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int v = tid + k * 256;
       const int row = v >> 4, j = v & 15;
-      vr[k] = (row < nt_tok && j < jn) ? __ldg(pr.V + static_cast<int64_t>(tc + row) * P.r + jb + j)
-                                      : 0.0f;
+      vr[set][k] = (row < nt_tok && j < jn)
+                       ? __ldg(pr.V + static_cast<int64_t>(tc + row) * P.r + jb + j)
+                       : 0.0f;
     }
   };
-  load(0);
-  for (int tc = 0; tc < P.T; tc += kGrdTok) {
+  auto chunk = [&](int set, int tc) {
     __syncthreads();
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int v = tid + k * 256;
-      *reinterpret_cast<uint4*>(zt + (v >> 3) * kGrdLdZ + (v & 7) * 8) = zr[k];
+      *reinterpret_cast<uint4*>(zt + (v >> 3) * kGrdLdZ + (v & 7) * 8) = zr[set][k];
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int v = tid + k * 256;
       const int row = v >> 4, j = v & 15;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(vr[k]);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(vr[k], __bfloat162float(hi)));
+      const __nv_bfloat16 hi = __float2bfloat16_rn(vr[set][k]);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(vr[set][k], __bfloat162float(hi)));
       vhi[j * kGrdLdV + row] = *reinterpret_cast<const uint16_t*>(&hi);
       vlo[j * kGrdLdV + row] = *reinterpret_cast<const uint16_t*>(&lo);
     }
     __syncthreads();
-    if (tc + kGrdTok < P.T) load(tc + kGrdTok);
+    if (tc + 2 * kGrdTok < P.T) load(set, tc + 2 * kGrdTok);  // refill the set just staged
 #pragma unroll
     for (int k0 = 0; k0 < kGrdTok; k0 += 16) {
       // A = Z^T: submatrices (c 0-7 | 8-15) x (t 0-7 | 8-15), each the transpose
@@ -423,6 +423,12 @@ __global__ void __launch_bounds__(256) lora_grad_group(const __grid_constant__ G
       mma_bf16_16816(acc, a[0], a[1], a[2], a[3], bh0, bh1);
       mma_bf16_16816(acc, a[0], a[1], a[2], a[3], bl0, bl1);
     }
+  };
+  load(0, 0);
+  if (kGrdTok < P.T) load(1, kGrdTok);
+  for (int tc = 0; tc < P.T; tc += 2 * kGrdTok) {  // chunk order (and sum order) unchanged
+    chunk(0, tc);
+    if (tc + kGrdTok < P.T) chunk(1, tc + kGrdTok);
   }
   // acc: (c = mt+g, j = nt+2qd, +1) and (c = mt+g+8, same j)
 #pragma unroll
