@@ -18,7 +18,10 @@ forward keeps only each block's input; the backward of a block recomputes
 its layers' forward from that input with the same weights (the block is in
 its ring slot for the backward visit anyway) and the same dropout masks (the
 counter-based generator is keyed by step, layer and projection), then runs
-the layers' backward in reverse.  Every step of the path runs in the
+the layers' backward in reverse.  The last block is the exception: its
+backward visit follows its forward visit at once, so its forward keeps
+every layer's activations (the buffers a recompute would fill) and its
+backward uses them as they are; the activation memory is still one block's.  Every step of the path runs in the
 library's kernels; this module only sequences the calls and owns buffers.
 
 Synthetic data: the stack's input h0 [T, hidden] and the gradient arriving
@@ -74,6 +77,7 @@ class DecoderStack(LayerStack):
         self.h_cur = bf(T, h)  # running hidden state (forward output of the last layer)
         self.rec_out = [bf(T, h) for _ in range(max(bs, 2))]  # layer outputs inside a block
         self.dh_cur = None
+        self._kept = None  # block whose forward activations are still in self.act
         # backward scratch, shared by the layers
         self.gs = {"dm": bf(T, I), "dgate": bf(T, I), "dup": bf(T, I), "db_g": bf(T, h),
                    "db_u": bf(T, h), "dh1": bf(T, h), "datt": bf(T, H * d), "dq": bf(T, H * d),
@@ -141,31 +145,41 @@ class DecoderStack(LayerStack):
     def _fwd_block(self, ws, b, record):
         """Forward through block b from its input; the last layer writes the
         next block's saved input (the rematerialization boundary), the others
-        ping-pong between two buffers: nothing else is kept."""
+        ping-pong between two buffers: nothing else is kept.  The stack's last
+        block instead keeps each layer's activations and outputs, for the
+        backward visit that comes next."""
         layers = list(self.block_layers(b))
+        keep = b == self.n_blocks - 1
         h = self.block_input(b)
         for i, l in enumerate(layers):
             last = i == len(layers) - 1
-            if last:
-                out = self.saved[b + 1] if b + 1 < self.n_blocks else self.h_cur
+            if keep:
+                out, s = (self.h_cur if last else self.rec_out[i]), self.act[i]
+            elif last:
+                out, s = self.saved[b + 1], self.act[0]
             else:
-                out = self.rec_out[i % 2] if self.block_size > 1 else self.h_cur
-            self.layer_forward(ws[i * self.P:(i + 1) * self.P], l, h, out, self.act[0])
+                out, s = (self.rec_out[i % 2] if self.block_size > 1 else self.h_cur), self.act[0]
+            self.layer_forward(ws[i * self.P:(i + 1) * self.P], l, h, out, s)
             if record is not None:
                 record(l, -1, "h_out", out)
             h = out
+        self._kept = b if keep else None
 
     def _bwd_block(self, ws, b, record):
         """Recompute block b's forward from its saved input, keeping every
-        layer's activations, then back-propagate through its layers."""
+        layer's activations (unless its forward kept them), then
+        back-propagate through its layers."""
         layers = list(self.block_layers(b))
-        h = self.block_input(b)
-        for i, l in enumerate(layers):
-            out = self.rec_out[i]
-            self.layer_forward(ws[i * self.P:(i + 1) * self.P], l, h, out, self.act[i])
-            if record is not None:
-                record(l, -1, "h_out_recomputed", out)
-            h = out
+        if self._kept == b:
+            self._kept = None  # the forward just left these activations in self.act
+        else:
+            h = self.block_input(b)
+            for i, l in enumerate(layers):
+                out = self.rec_out[i]
+                self.layer_forward(ws[i * self.P:(i + 1) * self.P], l, h, out, self.act[i])
+                if record is not None:
+                    record(l, -1, "h_out_recomputed", out)
+                h = out
         if b == self.n_blocks - 1:
             self.dh_cur = self.dh_top  # gradient arriving at the stack output
         for i in reversed(range(len(layers))):
