@@ -286,10 +286,11 @@ static void fwd_layout(const hsnf4_lora_fwd_args* p, int n, int64_t T, int r, Fw
 
 // Workspace layout of a backward group:
 //   [s*u bf16 [T, r_pad] per problem][u fp32 [T, r] per problem]
-//   [X_d bf16 [T, k_in] per problem with dropout]
+//   [X_d bf16 [T, k_in] and its keep-mask bytes [T, k_in / 8] per problem
+//    with dropout]
 //   [projection partials][GEMM split-K partials + counters]
 struct BwdLayout {
-  size_t su[8], u[8], xd[8], prj, gemm, total;
+  size_t su[8], u[8], xd[8], bits[8], prj, gemm, total;
 };
 
 static void bwd_layout(const hsnf4_lora_bwd_args* p, int n, int64_t T, int r, BwdLayout* L) {
@@ -306,6 +307,8 @@ static void bwd_layout(const hsnf4_lora_bwd_args* p, int n, int64_t T, int r, Bw
   for (int i = 0; i < n; ++i) {
     L->xd[i] = off;
     if (p[i].dropout_p > 0.0f) off += round_up(static_cast<size_t>(T) * p[i].W.k_in * 2, 256);
+    L->bits[i] = off;
+    if (p[i].dropout_p > 0.0f) off += round_up(static_cast<size_t>(T) * p[i].W.k_in / 8, 256);
   }
   ProjectDesc pd[8];
   GemmProblemDesc gd[8];
@@ -443,9 +446,11 @@ int lora_group_bwd(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r, fl
     // is added after it
     const void* xl = drop ? static_cast<const void*>(ws + L.xd[i]) : p.X;
     if (drop) {
+      // the apply pass records the keep mask; the dX pass reads it back
       dd[nd] = {p.X, ws + L.xd[i], nullptr, nullptr, p.W.k_in, p.dropout_p, p.dropout_seed,
-                p.dropout_offset};
-      da[nd] = {nullptr, p.dX, u, p.A, p.W.k_in, p.dropout_p, p.dropout_seed, p.dropout_offset};
+                p.dropout_offset, ws + L.bits[i]};
+      da[nd] = {nullptr, p.dX, u, p.A, p.W.k_in, p.dropout_p, p.dropout_seed, p.dropout_offset,
+                ws + L.bits[i]};
       ++nd;
     }
     pd[i] = {p.dY, p.W.n_out, p.B, false, u, ws + L.su[i], drop};

@@ -103,6 +103,9 @@ struct DropDesc {
   int64_t K;
   float p;
   uint64_t seed, offset;
+  // optional keep mask, one byte per 8 consecutive elements (bit i: element
+  // 8g + i): apply writes it, dx add reads it instead of re-running Philox
+  uint8_t* bits = nullptr;
 };
 cudaError_t launch_dropout_apply(const DropDesc* d, int n, int64_t T, cudaStream_t st);
 cudaError_t launch_dx_dropout_add(const DropDesc* d, int n, int64_t T, int r, float s,

@@ -9,8 +9,11 @@
 //            elementwise, added after the fused GEMM has written dY deq(W)
 //            (the GEMM's rank-r slice is zero in this mode).
 //
-// The mask is recomputed, never stored: element e = t K + k takes word e % 4
-// of the Philox block of e / 4 (philox.cuh).  An apply thread owns 8
+// The mask is recomputed from (seed, offset), never kept across calls:
+// element e = t K + k takes word e % 4 of the Philox block of e / 4
+// (philox.cuh).  Within one backward call the apply pass also writes the
+// mask as one byte per 8 elements to workspace, and the dx add that follows
+// reads those bytes instead of running Philox a second time.  An apply thread owns 8
 // consecutive elements of one row (16 bytes of bf16, two Philox blocks); a
 // dx-add thread the same 8 columns of 4 consecutive rows.  Both kernels
 // are HBM-bound elementwise passes: apply reads 2 B and writes 2 B per
@@ -29,6 +32,7 @@ struct DropProblem {
   uint16_t* out;       // apply: X_d [T, K];    dx add: dX [T, K] (read and written)
   const float* u;      // dx add: u fp32 [T, r]
   const uint16_t* A;   // dx add: A bf16 [r, K]
+  uint8_t* bits;       // keep mask bytes [T * K / 8], or null (apply: written; dx add: read)
   int64_t groups;      // work items: T * K / 8 (apply), ceil(T / 4) * K / 8 (dx add)
   int64_t g0;          // first group index of this problem in the launch
   int64_t K;
@@ -70,6 +74,7 @@ __global__ void __launch_bounds__(256) lora_dropout_apply(const __grid_constant_
     const DropProblem& pr = P.p[drop_problem(P, g)];
     const int64_t lg = g - pr.g0;
     const uint32_t keep = keep8(pr, lg);
+    if (pr.bits) pr.bits[lg] = static_cast<uint8_t>(keep);
     const uint4 x = __ldg(reinterpret_cast<const uint4*>(pr.X) + lg);
     const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
     uint32_t o[4];
@@ -87,72 +92,96 @@ __global__ void __launch_bounds__(256) lora_dropout_apply(const __grid_constant_
   }
 }
 
-// dx add: a thread owns 8 consecutive columns of 4 consecutive tokens, so
-// each 16-byte row of A serves 32 elements
+// dx add: a CTA owns a tile of 32 tokens x 256 columns of one problem.  It
+// stages the tile's slice of A ([r, 256] bf16) and of u ([32, r] fp32) in
+// shared memory once, while each thread's dX rows and mask bytes are already
+// in flight; thread (token group w, column group l) then forms its 4 tokens
+// x 8 columns of u A from shared memory and updates dX.
+constexpr int kDxTok = 32, kDxCols = 256, kDxMaxR = 64;
+
 __global__ void __launch_bounds__(256) lora_dx_dropout_add(const __grid_constant__ DropParams P) {
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < P.total;
-       g += stride) {
-    const DropProblem& pr = P.p[drop_problem(P, g)];
-    const int64_t lg = g - pr.g0;
-    const int64_t k8 = pr.K / 8;
-    const int64_t t0 = (lg / k8) * 4, k0 = (lg % k8) * 8;
-    const int nt = static_cast<int>((P.T - t0) < 4 ? (P.T - t0) : 4);
-    // adapter term: lora[tt][i] = sum_j u[t0 + tt, j] A[j, k0 + i]
-    float lora[4][8];
+  __shared__ __align__(16) uint16_t a_s[kDxMaxR * kDxCols];  // A[j][c], this tile's columns
+  __shared__ __align__(16) float u_s[kDxTok * kDxMaxR];      // u[t][j], this tile's tokens
+  const int q = drop_problem(P, blockIdx.x);
+  const DropProblem& pr = P.p[q];
+  const int64_t local = static_cast<int64_t>(blockIdx.x) - pr.g0;
+  const int64_t col_tiles = (pr.K + kDxCols - 1) / kDxCols;
+  const int tt0 = static_cast<int>(local / col_tiles) * kDxTok;
+  const int64_t c0 = (local % col_tiles) * kDxCols;
+  const int width = static_cast<int>((pr.K - c0) < kDxCols ? (pr.K - c0) : kDxCols);
+  const int tid = threadIdx.x, l = tid & 31, w = tid >> 5;
+  const int r = P.r;
+  const int t0 = tt0 + w * 4, k0 = l * 8;  // this thread's tokens and columns (tile-relative)
+  const bool col_ok = k0 < width;
+
+  // this thread's dX rows and mask bytes first: their latency overlaps the staging
+  uint4 d[4];
+  uint32_t keep[4];
 #pragma unroll
-    for (int tt = 0; tt < 4; ++tt)
+  for (int tt = 0; tt < 4; ++tt) {
+    d[tt] = make_uint4(0, 0, 0, 0);
+    keep[tt] = 0;
+    if (col_ok && t0 + tt < P.T) {
+      const int64_t e8 = (static_cast<int64_t>(t0 + tt) * pr.K + c0 + k0) / 8;
+      d[tt] = reinterpret_cast<const uint4*>(pr.out)[e8];
+      keep[tt] = pr.bits ? static_cast<uint32_t>(__ldg(pr.bits + e8)) : keep8(pr, e8);
+    }
+  }
+  // stage A[:, c0 .. c0 + 255] (16-byte pieces) and u[tt0 .. tt0 + 31, :]
+  for (int v = tid; v < r * (kDxCols / 8); v += 256) {
+    const int j = v / (kDxCols / 8), cc = (v % (kDxCols / 8)) * 8;
+    uint4 x = make_uint4(0, 0, 0, 0);
+    if (cc < width) x = __ldg(reinterpret_cast<const uint4*>(pr.A + static_cast<int64_t>(j) * pr.K +
+                                                             c0 + cc));
+    *reinterpret_cast<uint4*>(a_s + j * kDxCols + cc) = x;
+  }
+  for (int v = tid; v < kDxTok * r / 4; v += 256) {
+    const int t = v / (r / 4), jq = (v % (r / 4)) * 4;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tt0 + t < P.T) x = __ldg(reinterpret_cast<const float4*>(pr.u + static_cast<int64_t>(tt0 + t) * r + jq));
+    *reinterpret_cast<float4*>(u_s + t * r + jq) = x;
+  }
+  __syncthreads();
+  if (!col_ok) return;
+  // adapter term: lora[tt][i] = sum_j u[t0 + tt, j] A[j, k0 + i], in j order
+  float lora[4][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) lora[tt][i] = 0.0f;
-    for (int j0 = 0; j0 < P.r; j0 += 4) {  // r % 8 == 0
-      // four rows of A and the four tokens' u[j0 .. j0 + 3], all loads first
-      uint4 a[4];
-      float4 uq[4];
+  for (int tt = 0; tt < 4; ++tt)
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-        a[jj] = __ldg(reinterpret_cast<const uint4*>(pr.A + (j0 + jj) * pr.K + k0));
+    for (int i = 0; i < 8; ++i) lora[tt][i] = 0.0f;
+  for (int j = 0; j < r; ++j) {
+    const uint4 a = *reinterpret_cast<const uint4*>(a_s + j * kDxCols + k0);
+    const uint32_t as[4] = {a.x, a.y, a.z, a.w};
+    float af[8];
 #pragma unroll
-      for (int tt = 0; tt < 4; ++tt)
-        uq[tt] = tt < nt ? __ldg(reinterpret_cast<const float4*>(pr.u + (t0 + tt) * P.r + j0))
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const uint32_t as[4] = {a[jj].x, a[jj].y, a[jj].z, a[jj].w};
-        float af[8];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          af[2 * h] = __uint_as_float(as[h] << 16);
-          af[2 * h + 1] = __uint_as_float(as[h] & 0xFFFF0000u);
-        }
-#pragma unroll
-        for (int tt = 0; tt < 4; ++tt) {
-          const float uj = jj == 0 ? uq[tt].x : jj == 1 ? uq[tt].y : jj == 2 ? uq[tt].z : uq[tt].w;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) lora[tt][i] = __fmaf_rn(uj, af[i], lora[tt][i]);
-        }
-      }
+    for (int h = 0; h < 4; ++h) {
+      af[2 * h] = __uint_as_float(as[h] << 16);
+      af[2 * h + 1] = __uint_as_float(as[h] & 0xFFFF0000u);
     }
 #pragma unroll
     for (int tt = 0; tt < 4; ++tt) {
-      if (tt >= nt) break;
-      const int64_t e8 = ((t0 + tt) * pr.K + k0) / 8;  // this row segment's 8-element group
-      const uint32_t keep = keep8(pr, e8);
-      uint4* dst = reinterpret_cast<uint4*>(pr.out) + e8;
-      const uint4 d = *dst;
-      const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
-      uint32_t o[4];
+      const float uj = u_s[(w * 4 + tt) * r + j];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        float lo = __uint_as_float(ds[h] << 16), hi = __uint_as_float(ds[h] & 0xFFFF0000u);
-        if ((keep >> (2 * h)) & 1u)
-          lo = __fadd_rn(lo, __fmul_rn(__fmul_rn(P.s, lora[tt][2 * h]), pr.scale));
-        if ((keep >> (2 * h + 1)) & 1u)
-          hi = __fadd_rn(hi, __fmul_rn(__fmul_rn(P.s, lora[tt][2 * h + 1]), pr.scale));
-        const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-        o[h] = *reinterpret_cast<const uint32_t*>(&v);
-      }
-      *dst = make_uint4(o[0], o[1], o[2], o[3]);
+      for (int i = 0; i < 8; ++i) lora[tt][i] = __fmaf_rn(uj, af[i], lora[tt][i]);
     }
+  }
+#pragma unroll
+  for (int tt = 0; tt < 4; ++tt) {
+    if (t0 + tt >= P.T) break;
+    const int64_t e8 = (static_cast<int64_t>(t0 + tt) * pr.K + c0 + k0) / 8;
+    const uint32_t ds[4] = {d[tt].x, d[tt].y, d[tt].z, d[tt].w};
+    uint32_t o[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float lo = __uint_as_float(ds[h] << 16), hi = __uint_as_float(ds[h] & 0xFFFF0000u);
+      if ((keep[tt] >> (2 * h)) & 1u)
+        lo = __fadd_rn(lo, __fmul_rn(__fmul_rn(P.s, lora[tt][2 * h]), pr.scale));
+      if ((keep[tt] >> (2 * h + 1)) & 1u)
+        hi = __fadd_rn(hi, __fmul_rn(__fmul_rn(P.s, lora[tt][2 * h + 1]), pr.scale));
+      const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+      o[h] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    reinterpret_cast<uint4*>(pr.out)[e8] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -173,9 +202,11 @@ static cudaError_t launch_drop(bool dx, const DropDesc* d, int n, int64_t T, int
     pr.out = static_cast<uint16_t*>(d[q].out);
     pr.u = d[q].u;
     pr.A = static_cast<const uint16_t*>(d[q].A);
+    pr.bits = d[q].bits;
     pr.K = d[q].K;
-    // apply: one item per 8 elements; dx add: 8 columns x 4 tokens
-    pr.groups = dx ? (T + 3) / 4 * (d[q].K / 8) : T * d[q].K / 8;
+    // apply: one item per 8 elements; dx add: one CTA per 32 tokens x 256 columns
+    pr.groups = dx ? (T + kDxTok - 1) / kDxTok * ((d[q].K + kDxCols - 1) / kDxCols)
+                   : T * d[q].K / 8;
     pr.g0 = g;
     pr.seed = dp.seed;
     pr.offset = dp.offset;
@@ -189,6 +220,7 @@ static cudaError_t launch_drop(bool dx, const DropDesc* d, int n, int64_t T, int
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int64_t grid = (g + 255) / 256;
   if (grid > static_cast<int64_t>(sms) * 16) grid = static_cast<int64_t>(sms) * 16;
+  if (dx) grid = g;  // one CTA per tile
   if (grid < 1) grid = 1;
   count_launch();
   if (dx)

@@ -696,6 +696,7 @@ struct ReduceTile {
 };
 
 constexpr int kReduceTok = 8;
+constexpr int kMaxSplits = 8;  // the split planner's limit
 constexpr int kMaxReduceTiles = 768;  // 32 B each: the parameter block stays < 32 KiB
 
 struct ReduceParams {
@@ -703,25 +704,44 @@ struct ReduceParams {
   int n_tiles, BN, T;
 };
 
-__global__ void __launch_bounds__(64) lora_splitk_reduce(const __grid_constant__ ReduceParams R) {
+__global__ void __launch_bounds__(128) lora_splitk_reduce(const __grid_constant__ ReduceParams R) {
+  // CTA: one tile, 8 tokens; warp w the tokens 2w, 2w + 1 of them; lane l
+  // rows 4l .. 4l + 3 (one 16-byte piece of each partial, 512 contiguous
+  // bytes per token across the warp).  All of a token's split loads are in
+  // flight before the adds, which stay in split order.
   const int slices = R.BN / kReduceTok;
   const int tix = blockIdx.x / slices, slice = blockIdx.x % slices;
   const ReduceTile& tl = R.tile[tix];
-  const int i = threadIdx.x * 2;  // rows i, i+1
-  const int row = tl.m0 + i;
-  for (int jj = 0; jj < kReduceTok; ++jj) {
-    const int c = slice * kReduceTok + jj;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int i = lane * 4;
+  const int row = tl.m0 + i;  // m_total is a multiple of 64: rows i .. i + 3 are all in or out
+  if (row >= tl.M) return;
+#pragma unroll
+  for (int jj = 0; jj < 2; ++jj) {
+    const int c = slice * kReduceTok + w * 2 + jj;
     const int t = tl.t0 + c;
-    if (t >= R.T || row >= tl.M) continue;
-    float2 acc = __ldcg(reinterpret_cast<const float2*>(tl.part + static_cast<int64_t>(c) * kTileM + i));
-    for (int s = 1; s < tl.splits; ++s) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(
-          tl.part + (static_cast<int64_t>(s) * R.BN + c) * kTileM + i));
-      acc.x += v.x;
-      acc.y += v.y;
-    }
-    const __nv_bfloat162 b = __floats2bfloat162_rn(acc.x, acc.y);
-    *reinterpret_cast<__nv_bfloat162*>(tl.out + static_cast<int64_t>(t) * tl.M + row) = b;
+    if (t >= R.T) continue;
+    float4 v[kMaxSplits];
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s)
+      if (s < tl.splits)
+        v[s] = __ldcg(reinterpret_cast<const float4*>(
+            tl.part + (static_cast<int64_t>(s) * R.BN + c) * kTileM + i));
+    float4 acc = v[0];
+#pragma unroll
+    for (int s = 1; s < kMaxSplits; ++s)
+      if (s < tl.splits) {
+        acc.x += v[s].x;
+        acc.y += v[s].y;
+        acc.z += v[s].z;
+        acc.w += v[s].w;
+      }
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&lo);
+    o.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(tl.out + static_cast<int64_t>(t) * tl.M + row) = o;
   }
 }
 
@@ -864,7 +884,7 @@ static void plan_splits(GemmMode mode, const GemmProblemDesc* probs, int n, int6
     int64_t worst_cost = -1;
     for (int p = 0; p < n; ++p) {
       const int64_t c = unit_cost(nk[p] / cur[p] + (nk[p] % cur[p] ? 1 : 0), cur[p]);
-      if (c > worst_cost && cur[p] < 8 && nk[p] / (cur[p] + 1) >= 16) {
+      if (c > worst_cost && cur[p] < kMaxSplits && nk[p] / (cur[p] + 1) >= 16) {
         worst = p;
         worst_cost = c;
       }
@@ -1085,7 +1105,7 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
             if (m0 >= g.m_total) continue;
             if (R.n_tiles == kMaxReduceTiles) {
               count_launch();
-              lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 64, 0, st>>>(R);
+              lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 128, 0, st>>>(R);
               R.n_tiles = 0;
             }
             const int tile = (tt * g.m_tiles + mt) * 2 + c;
@@ -1095,7 +1115,7 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     }
     if (R.n_tiles) {
       count_launch();
-      lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 64, 0, st>>>(R);
+      lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 128, 0, st>>>(R);
     }
     e = cudaGetLastError();
   }
