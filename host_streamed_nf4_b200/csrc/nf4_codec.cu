@@ -92,39 +92,78 @@ cudaError_t launch_nf4_quantize(const void* w, int64_t n_out, int64_t k_in, void
 }
 
 // ---------------------------------------------------------------- dequant
-// A lane expands 8 elements (4 code bytes -> 16 output bytes); 8 lanes cover
-// one 64-element block and build that block's bf16 table.  A warp therefore
-// reads 128 contiguous code bytes and writes 512 contiguous output bytes.
+// A lane expands 32 elements per step: one 16-byte code load (half a
+// 64-element block), one absmax, one bf16 table, 64 output bytes.  The
+// warp's 2 KiB of output for the step goes through a per-warp shared-memory
+// stage, so that every global store instruction writes 512 contiguous bytes
+// (lane l stores the 16-byte pieces l, l + 32, l + 64, l + 96); the stage
+// slots are XOR-swizzled so both the writes and the reads are free of bank
+// conflicts.  Each lane has the code loads of two steps in flight.
 
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t* __restrict__ codes,
+__device__ __forceinline__ int dq_slot(int s) { return s ^ ((s >> 3) & 7); }
+
+__device__ __forceinline__ void dq_step(const uint4 cw, const float a, bool active,
+                                        const Nf4Codebook& cb, uint4* __restrict__ stage,
+                                        uint4* __restrict__ out, int64_t qw, int64_t n_quads,
+                                        int lane) {
+  if (active) {
+    const Nf4Table t = nf4_make_table(cb, a);
+    stage[dq_slot(4 * lane + 0)] = nf4_dequant8(cw.x, t);
+    stage[dq_slot(4 * lane + 1)] = nf4_dequant8(cw.y, t);
+    stage[dq_slot(4 * lane + 2)] = nf4_dequant8(cw.z, t);
+    stage[dq_slot(4 * lane + 3)] = nf4_dequant8(cw.w, t);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int sl = lane + 32 * j;  // the warp's 16-byte piece sl: quad qw + sl / 4
+    if (qw + (sl >> 2) < n_quads) out[4 * qw + sl] = stage[dq_slot(sl)];
+  }
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4* __restrict__ codes,
                                                           const float* __restrict__ absmax,
                                                           uint4* __restrict__ out,
-                                                          int64_t n_groups, Nf4Codebook cb) {
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t g = tid; g < n_groups; g += stride) {  // g = group of 8 elements
-    const uint32_t cw = __ldg(codes + g);
-    const float a = __ldg(absmax + (g >> 3));
-    const Nf4Table t = nf4_make_table(cb, a);
-    out[g] = nf4_dequant8(cw, t);
+                                                          int64_t n_quads, Nf4Codebook cb) {
+  __shared__ uint4 stage_all[8][128];  // per warp: 32 lanes x 4 pieces
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint4* stage = stage_all[warp];
+  const int64_t step = static_cast<int64_t>(gridDim.x) * 256;  // quads per grid-wide step
+  // qw: first quad of this warp's step (warp-uniform, so the loop is too)
+  int64_t qw = static_cast<int64_t>(blockIdx.x) * 256 + warp * 32;
+  for (; qw < n_quads; qw += 2 * step) {
+    const int64_t q0 = qw + lane, q1 = qw + step + lane;
+    const bool a0 = q0 < n_quads, a1 = q1 < n_quads;
+    uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
+    float m0 = 0.0f, m1 = 0.0f;
+    if (a0) {
+      c0 = __ldg(codes + q0);
+      m0 = __ldg(absmax + (q0 >> 1));
+    }
+    if (a1) {
+      c1 = __ldg(codes + q1);
+      m1 = __ldg(absmax + (q1 >> 1));
+    }
+    dq_step(c0, m0, a0, cb, stage, out, qw, n_quads, lane);
+    if (qw + step < n_quads) dq_step(c1, m1, a1, cb, stage, out, qw + step, n_quads, lane);
   }
 }
 
 cudaError_t launch_nf4_dequant(const void* codes, const float* absmax, int64_t n_out,
                                int64_t k_in, void* out, cudaStream_t st) {
-  const int64_t n_groups = n_out * k_in / 8;
+  const int64_t n_quads = n_out * k_in / 32;  // k_in % 64 == 0
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t grid = (n_groups + 255) / 256;
-  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  int64_t grid = (n_quads + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sms) * 4;  // resident at 52 registers: one wave
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   void* prof = prof_begin(st);
   count_launch();
   nf4_dequant_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(
-      static_cast<const uint32_t*>(codes), absmax, static_cast<uint4*>(out), n_groups,
-      codebook());
+      static_cast<const uint4*>(codes), absmax, static_cast<uint4*>(out), n_quads, codebook());
   const cudaError_t e = cudaGetLastError();
   // algorithmic bytes: 0.5 B codes + 4/64 B absmax read, 2 B written per element
   if (prof) prof_end(prof, kProfDequant, 2.5625 * static_cast<double>(n_out) * k_in, st);
