@@ -136,8 +136,8 @@ int hsnf4_profile_read(hsnf4_kernel_time *out, int max_out);
 
 /* Number of kernels this library has launched in this process (every
  * entry point counts each launch it makes, on any device or stream).  Read
- * it before and after a region to count the region's launches.  No counterpart
- * in the paper; a measurement aid. */
+ * it before and after a region to count the region's launches.  The method
+ * has no counterpart to it; it is a measurement aid. */
 uint64_t hsnf4_kernel_launches(void);
 
 /* Host-side fault injection for failure-path tests: the next call that
@@ -213,8 +213,8 @@ int lora_linear_fwd(const hsnf4_nf4_weight *W, const void *X, int64_t T,
  * forbids later allocations, a plugin or callback that may not call the
  * allocator): no workspace argument; the scratch is a 64 MiB array compiled
  * into the library, which every GPU that loads the library holds until the
- * process exits.  This entry point has no counterpart in the paper; it is a
- * convenience of this library.
+ * process exits.  The method has no counterpart to this entry point; it
+ * is a convenience of this library.
  *   - Sizes whose scratch need (lora_linear_fwd_workspace) exceeds 64 MiB
  *     are rejected with HSNF4_ERR_INVALID before anything touches the GPU.
  *   - It allocates nothing: no cudaMalloc, no cudaFree, no allocating
