@@ -125,6 +125,7 @@ class ClockSampler:
         self._stop = threading.Event()
         self._thread = None
         self._proc = None
+        self._nv = self._h = None
 
     def _nvml_handle(self):
         import pynvml
@@ -134,24 +135,46 @@ class ClockSampler:
         bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
         return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
 
-    def _run_nvml(self, nv, h):
-        self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+    def _sample(self):
+        nv, h = self._nv, self._h
         get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
             nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+        mask = get_reasons(h)
+        for bit, name in self.REASONS.items():
+            if mask & bit:
+                self.reasons.add(name)
+
+    def _run_nvml(self):
         while not self._stop.is_set():
-            self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
-            mask = get_reasons(h)
-            for bit, name in self.REASONS.items():
-                if mask & bit:
-                    self.reasons.add(name)
+            try:
+                self._sample()
+            except Exception:
+                return
             self._stop.wait(0.01)
+
+    def sample_while(self, busy, limit_s: float = 600.0):
+        """Also sample from the calling thread while busy() holds (the GPU is
+        still working through the timed region's queued steps), so that a
+        short region still gets samples.  NVML only; never raises."""
+        if self._nv is None:
+            return
+        t0 = time.monotonic()
+        try:
+            while busy() and time.monotonic() - t0 < limit_s:
+                self._sample()
+                time.sleep(0.002)
+        except Exception:
+            return
 
     def __enter__(self):
         try:
-            nv, h = self._nvml_handle()
-            self._thread = threading.Thread(target=self._run_nvml, args=(nv, h), daemon=True)
+            self._nv, self._h = self._nvml_handle()
+            self.max_mhz = self._nv.nvmlDeviceGetMaxClockInfo(self._h, self._nv.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run_nvml, daemon=True)
             self._thread.start()
         except Exception:
+            self._nv = self._h = None
             self._start_smi()
         return self
 
@@ -304,6 +327,7 @@ def run_ours(args, ws, rank, local):
         drain_copies()
         e1.record(compute)
         launches = hsnf4.kernel_launches() - launches0
+        clocks.sample_while(lambda: not e1.query())  # the GPU is still inside the region
         torch.cuda.synchronize(dev)
         barrier(ws)
     ms_total = hdist.max_over_ranks(e0.elapsed_time(e1))
