@@ -39,51 +39,24 @@ bool take_fault(FaultSite site) {
 }
 
 // ---------------------------------------------------------------- codebook
-// NormalFloat-4 (the "nf4" type of the Poros API reference; values from the
-// published construction): standard-normal quantiles at probabilities
-// delta - j (delta - 1/2) / 8, j = 0..7 (positive side) and
-// delta - j (delta - 1/2) / 7, j = 0..6 (negative side, mirrored), plus 0,
-// divided by the quantile at delta = 1 - (1/32 + 1/30) / 2.
-// The quantile is found by Newton's method on Phi(x) - p with
-// Phi(x) = erfc(-x / sqrt 2) / 2 and Phi'(x) = exp(-x^2 / 2) / sqrt(2 pi),
-// iterated to a fixed point in double; each ratio is rounded once to fp32.
+// NormalFloat-4, the "nf4" type of the Poros API reference: the 16 float32
+// values of the data type as QLoRA (Dettmers et al. 2023) prints them in its
+// Appendix E, as IEEE-754 bit patterns, code 0 (-1) up to code 15 (+1).  They
+// are standard-normal quantiles at evenly spaced probabilities plus an exact
+// zero, normalised to [-1, 1] (the paper's "4-bit NormalFloat Quantization").
 
-static double newton_quantile(double p) {
-  const double inv_sqrt2 = 0.70710678118654752440;
-  const double inv_sqrt_2pi = 0.39894228040143267794;
-  double x = 0.0;
-  for (int it = 0; it < 200; ++it) {
-    const double f = 0.5 * erfc(-x * inv_sqrt2) - p;
-    const double d = inv_sqrt_2pi * exp(-0.5 * x * x);
-    const double nx = x - f / d;
-    if (nx == x) break;
-    if (it > 60 && fabs(nx - x) <= 4e-16 * fabs(x)) {  // settled to rounding noise
-      x = 0.5 * (x + nx);
-      break;
-    }
-    x = nx;
-  }
-  return x;
-}
-
-static Nf4Codebook derive_codebook() {
-  Nf4Codebook cb;
-  const double delta = 1.0 - 0.5 * (1.0 / 32.0 + 1.0 / 30.0);
-  const double top = newton_quantile(delta);
-  for (int j = 0; j < 7; ++j)
-    cb.v[j] = static_cast<float>(-newton_quantile(delta - j * (delta - 0.5) / 7.0) / top);
-  cb.v[7] = 0.0f;
-  for (int j = 0; j < 8; ++j)
-    cb.v[15 - j] = static_cast<float>(newton_quantile(delta - j * (delta - 0.5) / 8.0) / top);
-  cb.v[0] = -1.0f;
-  cb.v[15] = 1.0f;
-  return cb;
-}
+static const uint32_t kNf4Bits[16] = {
+    0xbf800000u, 0xbf3239b1u, 0xbf066b30u, 0xbeca32a0u, 0xbe91a24du, 0xbe3d353fu,
+    0xbdba7871u, 0x00000000u, 0x3da2faffu, 0x3e24cae3u, 0x3e7c04ddu, 0x3ead033au,
+    0x3ee1a4b8u, 0x3f1007abu, 0x3f3913b3u, 0x3f800000u,
+};
 
 const Nf4Codebook& codebook() {
-  static Nf4Codebook cb;
-  static std::once_flag once;
-  std::call_once(once, [] { cb = derive_codebook(); });
+  static const Nf4Codebook cb = [] {
+    Nf4Codebook c;
+    memcpy(c.v, kNf4Bits, sizeof c.v);
+    return c;
+  }();
   return cb;
 }
 

@@ -17,7 +17,7 @@ int fail(int status, const char* fmt, ...) __attribute__((format(printf, 2, 3)))
 // Map a CUDA error to HSNF4_ERR_CUDA with the call's name, or HSNF4_OK.
 int cuda_status(cudaError_t e, const char* what);
 
-// The NormalFloat-4 codebook the kernels use (derived once, in double).
+// The NormalFloat-4 codebook the kernels use (the published NF4 values).
 const Nf4Codebook& codebook();
 
 // Host-side fault injection sites (hsnf4_inject_fault).

@@ -155,6 +155,13 @@ class LayerStack:
 
     # ------------------------------------------------------------------ setup
 
+    def base_weight_bf16(self, l: int, p: int) -> torch.Tensor:
+        """The seeded bf16 weight [n_out, k_in] of layer l, projection p that
+        the slab holds (quantized, for an NF4 base), drawn again on the
+        device: lets a checker quantize it independently."""
+        _, n, k = self.projs[p]
+        return _randn_bf16((n, k), synth.W_STD, _gen(self.device, self.seed, l, p), self.device)
+
     def _fill_slab(self, seed: int):
         dev = self.device
         for l in range(self.L):

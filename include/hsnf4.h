@@ -150,10 +150,13 @@ int hsnf4_inject_fault(const char *site);
 /* NF4 quantize / dequantize                                               */
 /* ----------------------------------------------------------------------- */
 
-/* The 16 fp32 codebook values the kernels use, ascending (host out[16]).
- * NormalFloat construction: standard-normal quantiles at probabilities
+/* The 16 fp32 codebook values the kernels use, ascending (host out[16]):
+ * the NormalFloat-4 data type exactly as QLoRA (Dettmers et al. 2023)
+ * prints it in Appendix E -- standard-normal quantiles at probabilities
  * evenly spaced from 1 - (1/32 + 1/30)/2 down to 1/2 (8 positive, 7
- * negative, plus 0), divided by the largest; derived once in double. */
+ * negative, plus 0), divided by the largest.  Codes and dequantized values
+ * are therefore those of any NF4 implementation that uses the published
+ * table.  Errors: INVALID if out is NULL. */
 int nf4_codebook(float *out);
 
 /* Quantize + pack a bf16 weight (Poros API reference: quantization="nf4").

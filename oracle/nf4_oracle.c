@@ -39,19 +39,44 @@ uint16_t orc_f32_to_bf16(float f) {
 /* NormalFloat-4 codebook                                                   */
 /* ------------------------------------------------------------------------ */
 /* The pages name the data type (4-bit NF4, Poros API reference,
- * PorosTrainer.from_pretrained "quantization") but print no values.  The
- * plainest reading is the published NormalFloat construction (QLoRA,
- * Dettmers et al. 2023, section "4-bit NormalFloat Quantization"):
- * standard-normal quantiles at probabilities spaced evenly from
- * delta = 1 - (1/32 + 1/30)/2 down to 1/2 -- eight on the positive side
- * (the 1/2 end excluded), seven mirrored on the negative side (likewise),
- * plus an exact zero -- all divided by the largest magnitude, so that the
- * ends are exactly -1 and +1.  The probabilities are formed as exact
- * rationals, the quantiles in double, and each ratio is rounded once to
- * fp32. */
+ * PorosTrainer.from_pretrained "quantization") but print no values.  NF4 is
+ * a fixed published data type: QLoRA (Dettmers et al. 2023), Appendix E
+ * "NormalFloat 4-bit data type", prints its 16 values, and those exact
+ * float32 numbers are what this oracle uses.
+ *
+ * Where they come from (section "4-bit NormalFloat Quantization" of the same
+ * paper): standard-normal quantiles at probabilities spaced evenly from
+ * delta = 1 - (1/32 + 1/30)/2 down to 1/2 -- eight on the positive side and
+ * seven mirrored on the negative side, the 1/2 end excluded -- plus an exact
+ * zero, all divided by the largest magnitude so that the ends are -1 and +1.
+ * The printed values carry that construction with the probabilities and the
+ * final division in single precision, so they sit a few float32 ulps away
+ * from the same construction in exact arithmetic; orc_normal_quantile below
+ * lets the tests check that distance. */
+
+static const float kNf4Published[16] = {
+    -1.0f,
+    -0.6961928009986877f,
+    -0.5250730514526367f,
+    -0.39491748809814453f,
+    -0.28444138169288635f,
+    -0.18477343022823334f,
+    -0.09105003625154495f,
+    0.0f,
+    0.07958029955625534f,
+    0.16093020141124725f,
+    0.24611230194568634f,
+    0.33791524171829224f,
+    0.44070982933044434f,
+    0.5626170039176941f,
+    0.7229568362236023f,
+    1.0f,
+};
 
 static double normal_cdf(double x) { return 0.5 * erfc(-x / sqrt(2.0)); }
 
+/* Inverse standard-normal CDF by bisection on erfc (used only by the tests'
+ * check of the construction above). */
 double orc_normal_quantile(double p) {
   double lo = -40.0, hi = 40.0;
   for (int it = 0; it < 4000; ++it) {
@@ -66,23 +91,7 @@ double orc_normal_quantile(double p) {
 }
 
 void orc_nf4_codebook(float out[16]) {
-  /* delta = 1 - (1/32 + 1/30)/2 = 929/960. */
-  const double top = orc_normal_quantile(929.0 / 960.0);
-  /* negative side: p_j = delta + j (1/2 - delta) / 7, j = 0..6
-   *              = (929*7 - 449 j) / 6720                                  */
-  for (int j = 0; j < 7; ++j) {
-    double p = (929.0 * 7.0 - 449.0 * j) / 6720.0;
-    out[j] = (float)(-orc_normal_quantile(p) / top);
-  }
-  out[7] = 0.0f;
-  /* positive side: p_j = delta + j (1/2 - delta) / 8, j = 0..7
-   *              = (929*8 - 449 j) / 7680; largest first, stored ascending */
-  for (int j = 0; j < 8; ++j) {
-    double p = (929.0 * 8.0 - 449.0 * j) / 7680.0;
-    out[15 - j] = (float)(orc_normal_quantile(p) / top);
-  }
-  out[0] = -1.0f; /* the j = 0 ratios are x/x = 1 exactly */
-  out[15] = 1.0f;
+  for (int i = 0; i < 16; ++i) out[i] = kNf4Published[i];
 }
 
 /* Nearest codebook entry by a linear scan of fp32 distances |x - c_i|.

@@ -33,11 +33,13 @@
 extern "C" {
 #endif
 
-/* NormalFloat-4 codebook, 16 ascending fp32 values, derived in double. */
+/* NormalFloat-4 codebook: the 16 ascending fp32 values QLoRA (Dettmers et
+ * al. 2023) prints in its Appendix E. */
 void orc_nf4_codebook(float out[16]);
 
 /* Standard normal quantile by bisection on erfc (double).  Exposed so the
- * tests can compare it to an independent inverse-CDF algorithm. */
+ * tests can compare it to an independent inverse-CDF algorithm and check the
+ * published codebook against the construction it comes from. */
 double orc_normal_quantile(double p);
 
 /* Index of the codebook entry nearest to x (fp32 distances, ties -> lower). */

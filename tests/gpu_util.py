@@ -22,6 +22,16 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+def oracle_nf4_weight(orc, w_bits: np.ndarray):
+    """Quantize a bf16 weight (uint16 bits [N, K]) with the oracle and upload
+    its codes and absmax, so that a LoRA check does not depend on the GPU
+    quantizer (which the codec tests check separately)."""
+    from host_streamed_nf4_b200 import hsnf4
+    n, k = w_bits.shape
+    codes, absmax = orc.quantize(w_bits)
+    return hsnf4.Nf4Weight(torch.from_numpy(codes).cuda(), torch.from_numpy(absmax).cuda(), n, k)
+
+
 def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 

@@ -113,8 +113,10 @@ def test_attention_deterministic():
 TINY = synth.Family("tiny", hidden=256, inter=640, heads=2, kv_heads=1, head_dim=128, layers=2)
 
 
-def _oracle_layers(st, dropout=None, step=0):
-    """The stack's weights as oracle layers (NF4 codes/absmax from the slab)."""
+def _oracle_layers(orc, st, dropout=None, step=0):
+    """The stack's weights as oracle layers: the oracle quantizes the seeded
+    bf16 weights itself, and the slab the GPU filled must hold those exact
+    codes and absmax values."""
     layers = []
     slab = st.slab.numpy()
     for l in range(st.L):
@@ -122,8 +124,10 @@ def _oracle_layers(st, dropout=None, step=0):
         base = l * st.layer_bytes
         for p, (name, n, k) in enumerate(st.projs):
             co, ao = st.offs[p]
-            codes = slab[base + co: base + co + n * k // 2]
-            absmax = slab[base + ao: base + ao + n * k // 16].view(np.float32)
+            codes, absmax = orc.quantize(bf16_bits(st.base_weight_bf16(l, p)))
+            assert np.array_equal(slab[base + co: base + co + n * k // 2], codes), (l, name)
+            assert np.array_equal(slab[base + ao: base + ao + n * k // 16].view(np.float32),
+                                  absmax), (l, name)
             drop = (dropout, st.seed, (step << 32) | (l << 4) | p) if dropout else None
             lin[name] = odec.Linear(n, k, A=bf16_bits(st.A[l][p]), B=bf16_bits(st.B[l][p]),
                                     codes=codes, absmax=absmax, dropout=drop)
@@ -147,12 +151,12 @@ def _stack_close(got, ref, what):
 
 
 @pytest.mark.parametrize("T,dropout", [(96, 0.0), (64, 0.1)])
-def test_decoder_stack_vs_oracle(T, dropout):
+def test_decoder_stack_vs_oracle(orc, T, dropout):
     st = DecoderStack(TINY, 2, T, streamed=False, block_size=2, dropout=dropout)
     st.step()
     torch.cuda.synchronize()
     assert hsnf4.device_status() == 0
-    layers = _oracle_layers(st, dropout or None, step=0)
+    layers = _oracle_layers(orc, st, dropout or None, step=0)
     h = bf16_to_f64(st.h_in)
     acts = []
     for L in layers:

@@ -17,7 +17,7 @@ import torch
 
 from host_streamed_nf4_b200 import hsnf4, synth
 from host_streamed_nf4_b200.stack import LayerStack
-from gpu_util import assert_lora_close, bf16_bits, bf16_to_f64, to_dev_bf16
+from gpu_util import assert_lora_close, bf16_bits, bf16_to_f64, oracle_nf4_weight, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -126,7 +126,7 @@ def test_merge_vs_oracle(orc, N, K, r, alpha, base):
     case = synth.linear_case(4000 + N + K + r, 1, N, K, r=r, alpha=alpha, b_std=0.05)
     A, B = to_dev_bf16(case.A), to_dev_bf16(case.B)
     if base == "nf4":
-        W = hsnf4.nf4_quantize_pack(to_dev_bf16(case.W))
+        W = oracle_nf4_weight(orc, case.W)
         ref = orc.lora_merge(case.A, case.B, alpha, codes=W.codes.cpu().numpy(),
                              absmax=W.absmax.cpu().numpy(), N=N, K=K)
     else:

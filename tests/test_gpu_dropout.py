@@ -8,7 +8,7 @@ import torch
 
 from host_streamed_nf4_b200 import hsnf4, synth
 from host_streamed_nf4_b200.stack import LayerStack
-from gpu_util import assert_lora_close, bf16_bits, bf16_to_f64, to_dev_bf16
+from gpu_util import assert_lora_close, bf16_bits, bf16_to_f64, oracle_nf4_weight, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -28,11 +28,12 @@ def test_dropout_apply_bitwise(orc, T, K, p, seed, offset):
     assert np.array_equal(got, ref)
 
 
-def _group(cases, T, r, alpha, drops):
-    """One grouped forward + backward; drops[i] = (p, seed, offset) or None."""
+def _group(orc, cases, T, r, alpha, drops):
+    """One grouped forward + backward on the oracle's NF4 codes;
+    drops[i] = (p, seed, offset) or None."""
     Ws, outs, fa, ba = [], [], [], []
     for c, d in zip(cases, drops):
-        W = hsnf4.nf4_quantize_pack(to_dev_bf16(c.W))
+        W = oracle_nf4_weight(orc, c.W)
         X, A, B, dY = (to_dev_bf16(a) for a in (c.X, c.A, c.B, c.dY))
         N, K = c.W.shape
         Y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
@@ -61,7 +62,7 @@ def test_group_with_dropout_vs_oracle(orc, T, p):
              for i, (N, K) in enumerate(shapes)]
     # one problem without dropout in the same group
     drops = [(p, 1234, (5 << 32) | i) if i != 1 else None for i in range(len(cases))]
-    Ws, outs = _group(cases, T, r, alpha, drops)
+    Ws, outs = _group(orc, cases, T, r, alpha, drops)
     for c, d, (W, *_), (Y, t, dX, dA, dB) in zip(cases, drops, Ws, outs):
         N, K = c.W.shape
         codes, absmax = W.codes.cpu().numpy(), W.absmax.cpu().numpy()
@@ -77,12 +78,12 @@ def test_group_with_dropout_vs_oracle(orc, T, p):
         assert_lora_close(dB.cpu().numpy(), dBr, what + " dB")
 
 
-def test_dropout_changes_the_adapter_path_and_is_reproducible():
+def test_dropout_changes_the_adapter_path_and_is_reproducible(orc):
     T, r = 128, 16
     c = [synth.linear_case(9100, T, 256, 512, r=r, b_std=0.05)]
-    _, a = _group(c, T, r, 32.0, [(0.5, 9, 1)])
-    _, b = _group(c, T, r, 32.0, [(0.5, 9, 1)])
-    _, o = _group(c, T, r, 32.0, [(0.5, 9, 2)])
+    _, a = _group(orc, c, T, r, 32.0, [(0.5, 9, 1)])
+    _, b = _group(orc, c, T, r, 32.0, [(0.5, 9, 1)])
+    _, o = _group(orc, c, T, r, 32.0, [(0.5, 9, 2)])
     for x, y in zip(a[0], b[0]):
         assert torch.equal(x, y)                    # same (seed, offset): same bits
     assert not torch.equal(a[0][1], o[0][1])        # another offset: another t

@@ -5,14 +5,15 @@ import pytest
 import torch
 
 from host_streamed_nf4_b200 import hsnf4, synth
-from gpu_util import assert_lora_close, bf16_to_f64, to_dev_bf16
+from gpu_util import assert_lora_close, bf16_to_f64, oracle_nf4_weight, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
 
-def _run(case, rows=None):
+def _run(orc, case):
+    """The GPU forward and backward on the oracle's NF4 codes of case.W."""
     T, N, K, r = case.shape
-    W = hsnf4.nf4_quantize_pack(to_dev_bf16(case.W))
+    W = oracle_nf4_weight(orc, case.W)
     X, A, B, dY = (to_dev_bf16(a) for a in (case.X, case.A, case.B, case.dY))
     Y, t = hsnf4.lora_linear_fwd(W, X, A, B, case.alpha)
     dX, dA, dB = hsnf4.lora_linear_bwd(W, X, t, A, B, dY, case.alpha)
@@ -54,13 +55,13 @@ CASES = [
 @pytest.mark.parametrize("T,N,K,r,alpha", CASES)
 def test_lora_fwd_bwd_vs_oracle(orc, T, N, K, r, alpha):
     case = synth.linear_case(1000 + T + N + K + r, T, N, K, r=r, alpha=alpha)
-    _check(orc, case, _run(case), what=f"T{T} N{N} K{K} r{r}")
+    _check(orc, case, _run(orc, case), what=f"T{T} N{N} K{K} r{r}")
 
 
-def test_deterministic_bitwise():
+def test_deterministic_bitwise(orc):
     case = synth.linear_case(5, 300, 384, 640, r=16)
-    a = _run(case)
-    b = _run(case)
+    a = _run(orc, case)
+    b = _run(orc, case)
     for x, y in zip(a[1:], b[1:]):
         assert torch.equal(x, y)
 
@@ -69,7 +70,7 @@ def test_zero_adapter_B_gives_base_only(orc):
     """B = 0: Y is the plain NF4 matmul; dA = 0 exactly."""
     case = synth.linear_case(6, 128, 256, 512)
     case.B[:] = 0
-    got = _run(case)
+    got = _run(orc, case)
     _check(orc, case, got, what="B=0")
     assert torch.count_nonzero(got[4]) == 0
 
@@ -83,7 +84,7 @@ def test_full_size_qwen7b_projection_sampled(orc, name):
     _, N, K = fam.projections()[idx]
     case = synth.linear_case(synth.sub_seed(42, 0, idx) % (2**31), 512, N, K)
     rows = np.array([0, 1, 127, 128, 255, 256, 400, 511])
-    _check(orc, case, _run(case), rows=rows, what=name)
+    _check(orc, case, _run(orc, case), rows=rows, what=name)
 
 
 # ---------------------------------------------------------------- grouped launches
@@ -93,11 +94,11 @@ GROUP = [  # (N, K): mixed shapes, one long-K problem (split along K), ragged N
 ]
 
 
-def _group_run(cases, T, r, alpha):
+def _group_run(orc, cases, T, r, alpha):
     Ws, ins, outs = [], [], []
     fa, ba = [], []
     for c in cases:
-        W = hsnf4.nf4_quantize_pack(to_dev_bf16(c.W))
+        W = oracle_nf4_weight(orc, c.W)
         X, A, B, dY = (to_dev_bf16(a) for a in (c.X, c.A, c.B, c.dY))
         N, K = c.W.shape
         Y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
@@ -124,16 +125,16 @@ def test_group_fwd_bwd_vs_oracle(orc, T):
     r, alpha = 16, 32.0
     cases = [synth.linear_case(7000 + i + T, T, N, K, r=r, alpha=alpha)
              for i, (N, K) in enumerate(GROUP)]
-    Ws, outs = _group_run(cases, T, r, alpha)
+    Ws, outs = _group_run(orc, cases, T, r, alpha)
     for c, W, (Y, t, dX, dA, dB) in zip(cases, Ws, outs):
         _check(orc, c, (W, Y, t, dX, dA, dB), what=f"group T{T} {c.W.shape}")
 
 
-def test_group_deterministic_bitwise():
+def test_group_deterministic_bitwise(orc):
     T, r = 512, 16
     cases = [synth.linear_case(8000 + i, T, N, K, r=r) for i, (N, K) in enumerate(GROUP)]
-    _, a = _group_run(cases, T, r, 32.0)
-    _, b = _group_run(cases, T, r, 32.0)
+    _, a = _group_run(orc, cases, T, r, 32.0)
+    _, b = _group_run(orc, cases, T, r, 32.0)
     for xa, xb in zip(a, b):
         for u, v in zip(xa, xb):
             assert torch.equal(u, v)

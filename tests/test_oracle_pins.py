@@ -28,10 +28,22 @@ def test_codebook_structure(orc):
     assert (cb < 0).sum() == 7 and (cb > 0).sum() == 8
 
 
-def _independent_codebook():
-    """NormalFloat construction with Python's own inverse normal CDF
-    (statistics.NormalDist, a rational-approximation algorithm unrelated to
-    the oracle's bisection on erfc)."""
+def _published_codebook():
+    """The NF4 values QLoRA prints (Appendix E), from the golden fixture,
+    as float32; the decimal strings and the bit patterns must agree."""
+    g = json.load(open(os.path.join(GOLDEN, "nf4_codebook.json")))
+    vals = np.array([float(v) for v in g["values"]], np.float64)
+    f32 = vals.astype(np.float32)
+    assert np.array_equal(f32.astype(np.float64), vals), "every printed value is a float32"
+    bits = np.array([int(b, 16) for b in g["f32_bits"]], np.uint32)
+    assert np.array_equal(f32.view(np.uint32), bits)
+    return f32
+
+
+def _construction_codebook():
+    """The NormalFloat construction in exact arithmetic, with Python's own
+    inverse normal CDF (statistics.NormalDist, a rational-approximation
+    algorithm unrelated to the oracle's bisection on erfc)."""
     nd = statistics.NormalDist()
     delta = 1.0 - 0.5 * (1.0 / 32.0 + 1.0 / 30.0)
     top = nd.inv_cdf(delta)
@@ -40,14 +52,33 @@ def _independent_codebook():
     return np.array(sorted(neg + [0.0] + pos), np.float64)
 
 
-def test_codebook_matches_independent_quantiles(orc):
-    cb = orc.codebook().astype(np.float64)
-    ref = _independent_codebook()
-    # equal to within one fp32 ulp of the value (the two double quantile
-    # algorithms agree to ~1e-15; fp32 rounding can differ only at a tie)
+def test_codebook_is_the_published_table(orc):
+    """Bitwise the 16 float32 values of the NF4 data type as published."""
+    assert np.array_equal(orc.codebook().view(np.uint32), _published_codebook().view(np.uint32))
+
+
+def test_published_codebook_follows_the_construction():
+    """The published values are the NormalFloat construction carried with the
+    probabilities and the last division in single precision: within a few
+    float32 ulps (at most 9 here) of the same construction in exact
+    arithmetic.  A wrong probability grid, a missing normalisation or a
+    swapped side would be off by far more."""
+    pub = _published_codebook().astype(np.float64)
+    ref = _construction_codebook()
     ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
-    assert np.all(np.abs(cb - ref) <= ulp)
-    assert np.array_equal(cb.astype(np.float32), ref.astype(np.float32))
+    ulp[7] = np.spacing(np.float32(0))
+    assert np.all(np.abs(pub - ref) <= 10 * ulp), (pub - ref) / ulp
+    assert np.max(np.abs(pub - ref)) < 5e-7
+
+
+def test_oracle_quantile_reproduces_the_construction(orc):
+    """The oracle's own quantile routine gives the same construction."""
+    delta = 1.0 - 0.5 * (1.0 / 32.0 + 1.0 / 30.0)
+    top = orc.normal_quantile(delta)
+    pos = [orc.normal_quantile(delta + j * (0.5 - delta) / 8.0) / top for j in range(8)]
+    neg = [-orc.normal_quantile(delta + j * (0.5 - delta) / 7.0) / top for j in range(7)]
+    got = np.array(sorted(neg + [0.0] + pos), np.float64)
+    assert np.allclose(got, _construction_codebook(), rtol=0, atol=1e-13)
 
 
 def test_normal_quantile_against_stdlib(orc):
@@ -127,9 +158,9 @@ def test_roundtrip_codebook_exact_blocks(orc):
 
 
 def test_dequant_code_sweep_is_bf16_of_codebook(orc):
-    """codes 0..15 at absmax 1 dequantize to bf16 of the independently
-    derived codebook, in order (pins the lookup and the nibble order)."""
-    ref = _independent_codebook().astype(np.float32)
+    """codes 0..15 at absmax 1 dequantize to bf16 of the published codebook,
+    in order (pins the lookup and the nibble order)."""
+    ref = _published_codebook()
     seq = np.tile(np.arange(16), 4)                  # 64 elements
     packed = ((seq[0::2] << 4) | seq[1::2]).astype(np.uint8)
     out = orc.dequant(packed, np.ones(1, np.float32), 1, 64)
