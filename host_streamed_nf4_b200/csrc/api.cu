@@ -223,7 +223,10 @@ static int check_group(const char* fn, int n, int64_t T, int r, float alpha) {
 // Workspace layout of a forward group:
 //   [s*t bf16 [T, r_pad] per problem][t fp32 [T, r] per problem without t_save]
 //   [X_d bf16 [T, k_in] per problem with dropout]
-//   [projection partials][GEMM split-K partials + counters]
+//   [projection partials][GEMM split-K partial tiles]
+// Every byte of it that a call reads was written earlier in the same call
+// (the split-K partials are summed by a separate reduce kernel, not through
+// counters), so nothing in it needs clearing between calls.
 struct FwdLayout {
   size_t zs[8], tscratch[8], xd[8], prj, gemm, total;
 };
@@ -261,7 +264,8 @@ static void fwd_layout(const hsnf4_lora_fwd_args* p, int n, int64_t T, int r, Fw
 //   [s*u bf16 [T, r_pad] per problem][u fp32 [T, r] per problem]
 //   [X_d bf16 [T, k_in] and its keep-mask bytes [T, k_in / 8] per problem
 //    with dropout]
-//   [projection partials][GEMM split-K partials + counters]
+//   [projection partials][GEMM split-K partial tiles]
+// As for the forward, every byte read was written earlier in the same call.
 struct BwdLayout {
   size_t su[8], u[8], xd[8], bits[8], prj, gemm, total;
 };
@@ -326,6 +330,7 @@ int lora_group_fwd(const hsnf4_lora_fwd_args* probs, int n, int64_t T, int r, fl
   static const char* fn = "lora_group_fwd";
   if (!probs) return fail(HSNF4_ERR_INVALID, "%s: probs is NULL", fn);
   int rc = check_group(fn, n, T, r, alpha);
+  if (!rc) rc = check_gemm_tokens(kGemmFwd, T, r);
   if (rc) return rc;
   for (int i = 0; i < n; ++i) {
     const hsnf4_lora_fwd_args& p = probs[i];
@@ -382,6 +387,7 @@ int lora_group_bwd(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r, fl
   static const char* fn = "lora_group_bwd";
   if (!probs) return fail(HSNF4_ERR_INVALID, "%s: probs is NULL", fn);
   int rc = check_group(fn, n, T, r, alpha);
+  if (!rc) rc = check_gemm_tokens(kGemmDx, T, r);
   if (rc) return rc;
   for (int i = 0; i < n; ++i) {
     const hsnf4_lora_bwd_args& p = probs[i];

@@ -80,6 +80,10 @@ struct GemmProblemDesc {
   bool dense;  // codes is a bf16 [n_out, k_in] weight (no absmax, no dequant)
 };
 size_t gemm_workspace_bytes(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r);
+// HSNF4_OK if the fused GEMM takes T tokens at rank r in this mode (a tiling
+// fits shared memory and T spans at most 64 token tiles); else the error,
+// recorded.  Needs only the sizes, so callers check it before any launch.
+int check_gemm_tokens(GemmMode mode, int64_t T, int r);
 int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r,
                            void* workspace, size_t ws_bytes, cudaStream_t st);
 

@@ -950,6 +950,17 @@ size_t gemm_workspace_bytes(GemmMode mode, const GemmProblemDesc* probs, int n, 
   return L.need;
 }
 
+int check_gemm_tokens(GemmMode mode, int64_t T, int r) {
+  Tiling tl;
+  if (!choose_tiling(mode, T, (r + 15) / 16 * 16, &tl))
+    return fail(HSNF4_ERR_INVALID, "lora gemm: no tiling fits shared memory (T=%lld, r=%d)",
+                (long long)T, r);
+  if ((T + tl.BN - 1) / tl.BN > 64)
+    return fail(HSNF4_ERR_INVALID, "lora gemm: T=%lld exceeds %d tokens per launch",
+                (long long)T, 64 * tl.BN);
+  return HSNF4_OK;
+}
+
 int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r,
                            void* workspace, size_t ws_bytes, cudaStream_t st) {
   if (n < 1 || n > kMaxProblems)

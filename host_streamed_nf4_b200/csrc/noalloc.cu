@@ -2,8 +2,8 @@
 // memory.
 //
 // lora_linear_fwd needs scratch (the scaled rank-r factor, the projection's
-// chunk partials and, for long-K shapes, split-K partial tiles and their
-// counters) and expects the caller to hand it in.  Some callers have no way
+// chunk partials and, for long-K shapes, split-K partial tiles) and expects
+// the caller to hand it in.  Some callers have no way
 // to obtain device memory at the point where they run the layer: a runtime
 // that reserves its whole device-memory budget at start-up and treats any
 // later allocation as an error, a plugin or host callback that is not
@@ -16,14 +16,19 @@
 // code cannot use the array's name as a device address (on the host it names
 // a stand-in object), so the first call on each device looks the address up
 // with cudaGetSymbolAddress while that device is current, checks the result
-// and caches it; later calls reuse the cached address.  That first call
-// should therefore come before any stream capture.
+// and caches it, keyed by the current context's unique ID; later calls in
+// the same context reuse it.  That first call should therefore come before
+// any stream capture.  A new context on the device (after cudaDeviceReset,
+// say) has a new ID, so its first call looks the address up again instead
+// of using one from the old context.
 //
 // Every call shares the one array and the array keeps the last call's
-// contents; what must start at zero (the split-K arrival counters) is
-// cleared on the stream by each call.  Calls whose work overlaps on the GPU
-// -- on different streams, or from different host threads -- race on the
-// scratch; serialize them.
+// contents.  Nothing needs clearing: every scratch byte a call reads was
+// written earlier in that same call (split-K partial tiles are summed by a
+// separate reduce kernel, with no counters).  Calls whose work overlaps on
+// the GPU -- on different streams, or from different host threads -- race
+// on the scratch; serialize them.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -40,11 +45,40 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes]
 
 constexpr int kMaxDevices = 64;
 
-// Device address of g_noalloc_scratch on the current device (looked up once
-// per device), or nullptr with the error recorded.
+// The current context's process-unique ID, through driver entry points the
+// runtime hands out (no link against the driver library): 0 if no context
+// is current or the entry points are missing.
+static unsigned long long current_context_id() {
+  using CtxGetCurrent = CUresult (*)(CUcontext*);
+  using CtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+  static CtxGetCurrent get_current = nullptr;
+  static CtxGetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetId>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch in the current context (looked up once
+// per device and context), or nullptr with the error recorded.
 static void* scratch_on_current_device() {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
+  static unsigned long long ctx_id[kMaxDevices] = {};
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
@@ -57,7 +91,8 @@ static void* scratch_on_current_device() {
     return nullptr;
   }
   std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
+  const unsigned long long id = current_context_id();
+  if (!addr[dev] || id == 0 || id != ctx_id[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) {
@@ -66,6 +101,9 @@ static void* scratch_on_current_device() {
       return nullptr;
     }
     addr[dev] = p;
+    // the lookup makes the device's context current if none was: read the
+    // ID again, so the next call in this context reuses the address
+    ctx_id[dev] = current_context_id();
   }
   return addr[dev];
 }

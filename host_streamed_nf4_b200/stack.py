@@ -60,12 +60,16 @@ class LayerStack:
                  streamed: bool = True, reuse_resident: bool = True, enable_prefetch: bool = True,
                  poison_on_release: bool = False, r: int = synth.RANK, alpha: float = synth.ALPHA,
                  seed: int = 42, device=None, grouping: str = "layer", n_slots: int = 2,
-                 base: str = "nf4", dropout: float = 0.0, data_seed=None, shard=None):
+                 base: str = "nf4", dropout: float = 0.0, data_seed=None, shard=None,
+                 slab=None):
         """shard = (rank, world, gather_factory): stream 1/world of every
         block (sharded stream); gather_factory(ring) returns the streamer's
         gather callback (dist.ring_gather).  data_seed: seed of the
         activations and upstream gradients (default: seed); the weights and
-        adapters always come from seed, as data-parallel ranks share them."""
+        adapters always come from seed, as data-parallel ranks share them.
+        slab: an already filled pinned slab of a stack with the same family,
+        layer count, base and seed (e.g. another stack's .slab), used as is
+        instead of drawing and quantizing the base again."""
         self.device = torch.device(device) if device is not None else torch.device(
             "cuda", torch.cuda.current_device())
         dev = self.device
@@ -87,8 +91,15 @@ class LayerStack:
         self.layer_bytes = hsnf4.layer_bytes(self.desc)
         self.offs = [hsnf4.layer_offsets(self.desc, p) for p in range(self.P)]
         self.n_blocks = (n_layers + block_size - 1) // block_size
-        self.slab = torch.empty(hsnf4.slab_bytes(self.descs), dtype=torch.uint8, pin_memory=True)
-        self._fill_slab(seed)
+        if slab is not None:
+            if slab.dtype != torch.uint8 or slab.numel() != hsnf4.slab_bytes(self.descs) or \
+                    not slab.is_pinned():
+                raise ValueError("slab: expected a pinned uint8 tensor of this stack's slab size")
+            self.slab = slab
+        else:
+            self.slab = torch.empty(hsnf4.slab_bytes(self.descs), dtype=torch.uint8,
+                                    pin_memory=True)
+            self._fill_slab(seed)
 
         self.compute = torch.cuda.current_stream(dev)
         self.shard = shard

@@ -223,11 +223,14 @@ int lora_linear_fwd(const hsnf4_nf4_weight *W, const void *X, int64_t T,
  *   - It allocates nothing: no cudaMalloc, no cudaFree, no allocating
  *     library routine.  The first call on each device looks up the array's
  *     device address (cudaGetSymbolAddress, with that device current) and
- *     caches it; make that first call before any stream capture.
- *   - All calls share the one array, which keeps the last call's contents
- *     (what must start at zero is cleared by each call).  Calls whose GPU
- *     work overlaps -- other streams, other host threads -- race on it;
- *     serialize them.
+ *     caches it for the device's current context; make that first call
+ *     before any stream capture.  A later context on the device (after
+ *     cudaDeviceReset, for one) looks the address up again on its first
+ *     call, which then likewise belongs before any capture.
+ *   - All calls share the one array, which keeps the last call's contents.
+ *     Nothing in it needs clearing: every byte a call reads was written
+ *     earlier in the same call.  Calls whose GPU work overlaps -- other
+ *     streams, other host threads -- race on it; serialize them.
  * Arguments, results and errors are otherwise those of lora_linear_fwd. */
 int lora_linear_fwd_noalloc(const hsnf4_nf4_weight *W, const void *X, int64_t T,
                             const void *A, const void *B, int r, float alpha, void *Y,

@@ -11,8 +11,33 @@
 
 #include <math.h>
 #include <pthread.h>
+#include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* allocation                                                               */
+/* ------------------------------------------------------------------------ */
+/* A checker must fail loudly: an allocation the oracle cannot make ends the
+ * process with a message rather than leaving outputs unwritten. */
+
+static void *xmalloc(size_t n) {
+  void *p = malloc(n ? n : 1);
+  if (!p) {
+    fprintf(stderr, "nf4 oracle: out of memory allocating %zu bytes\n", n);
+    abort();
+  }
+  return p;
+}
+
+static void *xcalloc(size_t n, size_t size) {
+  void *p = calloc(n ? n : 1, size ? size : 1);
+  if (!p) {
+    fprintf(stderr, "nf4 oracle: out of memory allocating %zu x %zu bytes\n", n, size);
+    abort();
+  }
+  return p;
+}
 
 /* ------------------------------------------------------------------------ */
 /* bf16 <-> fp32                                                            */
@@ -280,7 +305,7 @@ typedef struct {
 
 static void fwd_cols(void *p, int64_t lo, int64_t hi) {
   fwd_ctx *c = (fwd_ctx *)p;
-  double *row = (double *)malloc(sizeof(double) * (size_t)c->K);
+  double *row = (double *)xmalloc(sizeof(double) * (size_t)c->K);
   if (!row) return;
   for (int64_t n = lo; n < hi; ++n) {
     w_row(c->w, n, 0, c->K, row);
@@ -324,8 +349,8 @@ static void dx_cols(void *p, int64_t lo, int64_t hi) {
   dx_ctx *c = (dx_ctx *)p;
   int64_t width = hi - lo;
   if (width <= 0) return;
-  double *row = (double *)malloc(sizeof(double) * (size_t)width);
-  double *acc = (double *)calloc((size_t)(c->n_rows * width), sizeof(double));
+  double *row = (double *)xmalloc(sizeof(double) * (size_t)width);
+  double *acc = (double *)xcalloc((size_t)(c->n_rows * width), sizeof(double));
   if (!row || !acc) {
     free(row);
     free(acc);
@@ -413,8 +438,8 @@ void orc_lora_bwd_f64m(const double *W, const double *Xl, const double *g,
   memset(&w, 0, sizeof w);
   w.dense = W;
   w.K = K;
-  double *t = (double *)malloc(sizeof(double) * (size_t)(T * r));
-  double *u = (double *)malloc(sizeof(double) * (size_t)(T * r));
+  double *t = (double *)xmalloc(sizeof(double) * (size_t)(T * r));
+  double *u = (double *)xmalloc(sizeof(double) * (size_t)(T * r));
   if (!t || !u) {
     free(t);
     free(u);
@@ -498,7 +523,7 @@ int orc_dropout_keep(uint64_t seed, uint64_t offset, float p, int64_t T, int64_t
 
 int orc_dropout_apply(const uint16_t *X, int64_t T, int64_t K, uint64_t seed,
                       uint64_t offset, float p, uint16_t *out) {
-  uint8_t *keep = (uint8_t *)malloc((size_t)(T * K > 0 ? T * K : 1));
+  uint8_t *keep = (uint8_t *)xmalloc((size_t)(T * K > 0 ? T * K : 1));
   if (!keep) return -1;
   if (orc_dropout_keep(seed, offset, p, T, K, keep) != 0) {
     free(keep);
@@ -526,10 +551,10 @@ static int drop_inputs(const drop_cfg *d, const uint16_t *X, int64_t T, int64_t 
   *Xl = NULL;
   *g = NULL;
   if (!d) return 0;
-  uint16_t *xd = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(T * K > 0 ? T * K : 1));
-  uint8_t *keep = (uint8_t *)malloc((size_t)(T * K > 0 ? T * K : 1));
-  *Xl = (double *)malloc(sizeof(double) * (size_t)(T * K > 0 ? T * K : 1));
-  *g = (double *)malloc(sizeof(double) * (size_t)(T * K > 0 ? T * K : 1));
+  uint16_t *xd = (uint16_t *)xmalloc(sizeof(uint16_t) * (size_t)(T * K > 0 ? T * K : 1));
+  uint8_t *keep = (uint8_t *)xmalloc((size_t)(T * K > 0 ? T * K : 1));
+  *Xl = (double *)xmalloc(sizeof(double) * (size_t)(T * K > 0 ? T * K : 1));
+  *g = (double *)xmalloc(sizeof(double) * (size_t)(T * K > 0 ? T * K : 1));
   int rc = -1;
   if (xd && keep && *Xl && *g && orc_dropout_apply(X, T, K, d->seed, d->offset, d->p, xd) == 0 &&
       orc_dropout_keep(d->seed, d->offset, d->p, T, K, keep) == 0) {
@@ -553,7 +578,7 @@ static int drop_inputs(const drop_cfg *d, const uint16_t *X, int64_t T, int64_t 
 /* ---- the method's data types ---- */
 
 static double *widen_bf16(const uint16_t *src, int64_t n) {
-  double *d = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+  double *d = (double *)xmalloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
   if (!d) return NULL;
   for (int64_t i = 0; i < n; ++i) d[i] = (double)orc_bf16_to_f32(src[i]);
   return d;
@@ -561,7 +586,7 @@ static double *widen_bf16(const uint16_t *src, int64_t n) {
 
 static double *gather_rows(const double *M, int64_t cols, const int64_t *rows,
                            int64_t n_rows) {
-  double *d = (double *)malloc(sizeof(double) * (size_t)(n_rows * cols > 0 ? n_rows * cols : 1));
+  double *d = (double *)xmalloc(sizeof(double) * (size_t)(n_rows * cols > 0 ? n_rows * cols : 1));
   if (!d) return NULL;
   for (int64_t i = 0; i < n_rows; ++i)
     memcpy(d + i * cols, M + rows[i] * cols, sizeof(double) * (size_t)cols);
@@ -592,8 +617,8 @@ static int lora_fwd_src(const wsrc *wp, const drop_cfg *drop, int64_t N, int64_t
   double *Xd = widen_bf16(X, T * K);
   double *Ad = widen_bf16(A, (int64_t)r * K);
   double *Bd = widen_bf16(B, N * r);
-  double *t = (double *)malloc(sizeof(double) * (size_t)(T * r));
-  double *Yd = (double *)malloc(sizeof(double) * (size_t)(n_rows * N > 0 ? n_rows * N : 1));
+  double *t = (double *)xmalloc(sizeof(double) * (size_t)(T * r));
+  double *Yd = (double *)xmalloc(sizeof(double) * (size_t)(n_rows * N > 0 ? n_rows * N : 1));
   double *Xs = NULL, *ts = NULL;
   int rc = -1;
   if (!Xd || !Ad || !Bd || !t || !Yd) goto done;
@@ -640,11 +665,11 @@ static int lora_bwd_src(const wsrc *wp, const drop_cfg *drop, int64_t N, int64_t
   double *Ad = widen_bf16(A, (int64_t)r * K);
   double *Bd = widen_bf16(B, N * r);
   double *dYd = widen_bf16(dY, T * N);
-  double *t = (double *)malloc(sizeof(double) * (size_t)(T * r));
-  double *u = (double *)malloc(sizeof(double) * (size_t)(T * r));
-  double *dXd = (double *)malloc(sizeof(double) * (size_t)(n_rows * K > 0 ? n_rows * K : 1));
-  double *dAd = (double *)malloc(sizeof(double) * (size_t)(r * K));
-  double *dBd = (double *)malloc(sizeof(double) * (size_t)(N * r));
+  double *t = (double *)xmalloc(sizeof(double) * (size_t)(T * r));
+  double *u = (double *)xmalloc(sizeof(double) * (size_t)(T * r));
+  double *dXd = (double *)xmalloc(sizeof(double) * (size_t)(n_rows * K > 0 ? n_rows * K : 1));
+  double *dAd = (double *)xmalloc(sizeof(double) * (size_t)(r * K));
+  double *dBd = (double *)xmalloc(sizeof(double) * (size_t)(N * r));
   double *dYs = NULL, *us = NULL;
   int rc = -1;
   if (!Xd || !Ad || !Bd || !dYd || !t || !u || !dXd || !dAd || !dBd) goto done;
@@ -768,7 +793,7 @@ int orc_lora_merge(const uint8_t *codes, const float *absmax, const uint16_t *Wb
   if (!shape_ok(N, K) || r <= 0 || (!Wbf16 && (!codes || !absmax))) return -1;
   const double s = (double)alpha / (double)r;
   wsrc w = Wbf16 ? bf16_src(Wbf16, K) : nf4_src(codes, absmax, K);
-  double *row = (double *)malloc(sizeof(double) * (size_t)K);
+  double *row = (double *)xmalloc(sizeof(double) * (size_t)K);
   if (!row) return -1;
   for (int64_t n = 0; n < N; ++n) {
     w_row(&w, n, 0, K, row);
@@ -866,7 +891,7 @@ void orc_silu_mul_bwd(const double *a, const double *b, const double *dm, int64_
 void orc_attention_fwd(const double *q, const double *k, const double *v, int64_t T, int H,
                        int KV, int d, double scale, double *o, double *lse) {
   const int grp = H / KV;
-  double *p = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+  double *p = (double *)xmalloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
   if (!p) return;
   for (int h = 0; h < H; ++h) {
     const int kh = h / grp;
@@ -903,8 +928,8 @@ void orc_attention_bwd(const double *q, const double *k, const double *v, const 
                        int64_t T, int H, int KV, int d, double scale, double *dq, double *dk,
                        double *dv) {
   const int grp = H / KV;
-  double *p = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
-  double *dp = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+  double *p = (double *)xmalloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+  double *dp = (double *)xmalloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
   if (!p || !dp) {
     free(p);
     free(dp);
