@@ -377,6 +377,16 @@ def run_ours(args, ws, rank, local):
                                     "achieved": round(v["work"] / (v["total_ms"] / 1e3) / 1e12, 1)}
                                 for k, v in gemms.items()}}
 
+    # the rank-r kernels (HBM-bound: each reads its activation operand once)
+    hbm_peak, _, _, hbm_src = measured_peaks()
+    rank_r = {k: {"launches": v["launches"],
+                  "avg_us": round(v["total_ms"] / v["launches"] * 1e3, 2),
+                  "bytes_per_launch": int(v["work"] / v["launches"]),
+                  "achieved_GBps": round(v["work"] / (v["total_ms"] / 1e3) / 1e9, 1),
+                  "frac": round(v["work"] / (v["total_ms"] / 1e3) / 1e9 / hbm_peak, 4),
+                  "peak_GBps": hbm_peak, "peak_source": f"{hbm_src} hbm_gbs"}
+              for k, v in kt.items() if k in ("lora_project", "lora_grad")}
+
     # standalone NF4 dequant on the layer's largest weight (HBM-bound; the
     # output, 2 B per element, is far larger than L2)
     dequant = dequant_roofline(stack, fam, dev) if args.base == "nf4" else None
@@ -432,8 +442,12 @@ def run_ours(args, ws, rank, local):
                                    f"step" + (", sharded H2D + per-block all-gather)"
                                               if shard else ")") if ws > 1 else "single"),
                    "l2": "no flush: every step reads > 126 MB L2 (NF4 weights + activations)"},
-        "roofline": roofline, "step_roofline": step_roofline, "dequant": dequant, "merge": merge,
+        "roofline": roofline, "step_roofline": step_roofline, "rank_r": rank_r,
+        "dequant": dequant, "merge": merge,
         "peak_vram_GB": round(torch.cuda.max_memory_allocated(dev) / 1e9, 3), "e2e": e2e,
+        # page-locked host bytes of the frozen base on this rank (a sharded
+        # stream pins only the rank's shards)
+        "pinned_host_GB_per_rank": round(stack.pinned_bytes() / 1e9, 3),
         "gpu_launches": launches,  # counted by the library over the timed region
         "clocks": clock_summary,
     }
@@ -465,18 +479,15 @@ def dequant_roofline(stack, fam, dev):
     from host_streamed_nf4_b200 import hsnf4
     p = max(range(len(stack.projs)), key=lambda i: stack.projs[i][1] * stack.projs[i][2])
     _, n, k = stack.projs[p]
-    co, ao = stack.offs[p]
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     set_bytes = n * k * 2 + n * k // 2 + n * k // 16
     n_sets = max(2, math.ceil(4 * l2 / set_bytes))
+    W0 = stack.device_weight(0, p)
     sets = []
     for _ in range(n_sets):
-        codes = torch.empty(n * k // 2, dtype=torch.uint8, device=dev)
-        absmax = torch.empty(n * k // 64, dtype=torch.float32, device=dev)
-        codes.copy_(stack.slab[co: co + n * k // 2])
-        absmax.copy_(stack.slab[ao: ao + n * k // 16].view(torch.float32))
-        sets.append((hsnf4.Nf4Weight(codes, absmax, n, k),
+        sets.append((hsnf4.Nf4Weight(W0.codes.clone(), W0.absmax.clone(), n, k),
                      torch.empty(n, k, dtype=torch.bfloat16, device=dev)))
+    del W0
     for W, out in sets:
         hsnf4.nf4_dequant(W, out)
     torch.cuda.synchronize(dev)
@@ -578,16 +589,7 @@ def merge_roofline(stack, dev):
     from host_streamed_nf4_b200 import hsnf4
     p = max(range(len(stack.projs)), key=lambda i: stack.projs[i][1] * stack.projs[i][2])
     _, n, k = stack.projs[p]
-    W = stack.layer_weights(0)[p] if not stack.streamed else None
-    keep = None
-    if W is None:  # streamed stack: copy the projection's slab range to the device
-        co, ao = stack.offs[p]
-        nbytes = (ao - co) + n * k // 16 if stack.base == "nf4" else n * k * 2
-        keep = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-        keep.copy_(stack.slab[co: co + nbytes])
-        W = hsnf4.Nf4WeightC(keep.data_ptr(), keep.data_ptr() + (ao - co), n, k,
-                             hsnf4.BASE_NF4, 0) if stack.base == "nf4" else \
-            hsnf4.Nf4WeightC(keep.data_ptr(), None, n, k, hsnf4.BASE_BF16, 0)
+    keep = W = stack.device_weight(0, p)
     A, B = stack.A[0][p], stack.B[0][p]
     out = torch.empty(n, k, dtype=torch.bfloat16, device=dev)
     for _ in range(3):

@@ -91,6 +91,7 @@ struct hsnf4_streamer {
   size_t slab_bytes = 0;
   std::vector<hsnf4_layer_desc> layers;
   std::vector<size_t> layer_off, layer_size;
+  std::vector<size_t> shard_off;  // shard_slab: where block b's shard sits in the slab
   hsnf4_stream_config cfg{};
   uint8_t* ring = nullptr;
   size_t slot_bytes = 0;
@@ -155,8 +156,10 @@ int enqueue_copy(hsnf4_streamer* s, int i, int b, cudaStream_t after) {
     size_t S = 0, off = 0, len = 0;
     stream_shard_range(bytes, world, s->cfg.shard_rank, &S, &off, &len);
     if (len) {
-      rc = cuda_status(cudaMemcpyAsync(slot + off, s->slab + s->block_off(b) + off, len,
-                                       cudaMemcpyHostToDevice, s->copy),
+      // the whole stack in the slab, or (shard_slab) only this rank's shards
+      const uint8_t* src =
+          s->cfg.shard_slab ? s->slab + s->shard_off[b] : s->slab + s->block_off(b) + off;
+      rc = cuda_status(cudaMemcpyAsync(slot + off, src, len, cudaMemcpyHostToDevice, s->copy),
                        "prefetch: cudaMemcpyAsync H2D (shard)");
       if (rc) return rc;
     }
@@ -300,6 +303,38 @@ int stream_slot_bytes_sharded(const hsnf4_layer_desc* layers, int n_layers, int 
   return HSNF4_OK;
 }
 
+int stream_shard_slab_layout(const hsnf4_layer_desc* layers, int n_layers, int block_size,
+                             int world, int rank, int block, size_t* block_off, size_t* len,
+                             size_t* total_bytes) {
+  static const char* fn = "stream_shard_slab_layout";
+  if (!layers || n_layers < 1 || block_size < 1 || world < 1 || rank < 0 || rank >= world)
+    return fail(HSNF4_ERR_INVALID, "%s: need layers, n_layers >= 1, block_size >= 1 and "
+                "0 <= rank < world (got rank %d of %d)", fn, rank, world);
+  const int n_blocks = (n_layers + block_size - 1) / block_size;
+  if (block < -1 || block >= n_blocks)
+    return fail(HSNF4_ERR_INVALID, "%s: block %d outside [-1, %d)", fn, block, n_blocks);
+  size_t at = 0, found_off = 0, found_len = 0;
+  for (int b = 0; b < n_blocks; ++b) {
+    size_t bytes = 0;
+    for (int l = b * block_size; l < n_layers && l < (b + 1) * block_size; ++l) {
+      int rc = check_layer(fn, &layers[l]);
+      if (rc) return rc;
+      bytes += layer_bytes(layers[l]);
+    }
+    size_t S = 0, off = 0, n = 0;
+    stream_shard_range(bytes, world, rank, &S, &off, &n);
+    if (b == block) {
+      found_off = at;
+      found_len = n;
+    }
+    at += n;
+  }
+  if (block_off) *block_off = found_off;
+  if (len) *len = found_len;
+  if (total_bytes) *total_bytes = at;
+  return HSNF4_OK;
+}
+
 int stream_ring_bytes(const hsnf4_layer_desc* layers, int n_layers, int block_size,
                       size_t* out_bytes) {
   if (!layers || n_layers < 1 || !out_bytes || block_size < 1)
@@ -341,8 +376,14 @@ int stream_create(const void* pinned_slab, size_t slab_bytes, const hsnf4_layer_
   if (world > 1 && !cfg->gather)
     return fail(HSNF4_ERR_INVALID, "%s: a stream sharded over %d ranks needs a gather callback",
                 fn, world);
+  if (cfg->shard_slab && !cfg->gather)
+    return fail(HSNF4_ERR_INVALID, "%s: shard_slab needs a sharded stream (a gather callback)",
+                fn);
   size_t need_slab = 0, need_ring = 0;
-  int rc = stream_slab_bytes(layers, n_layers, &need_slab);
+  int rc = cfg->shard_slab
+               ? stream_shard_slab_layout(layers, n_layers, cfg->block_size, world,
+                                          cfg->shard_rank, -1, nullptr, nullptr, &need_slab)
+               : stream_slab_bytes(layers, n_layers, &need_slab);
   if (rc) return rc;
   rc = cfg->gather
            ? stream_slot_bytes_sharded(layers, n_layers, cfg->block_size, world, &need_ring)
@@ -371,6 +412,15 @@ int stream_create(const void* pinned_slab, size_t slab_bytes, const hsnf4_layer_
   }
   s->cfg = *cfg;
   if (s->cfg.poison_on_release) s->cfg.reuse_resident = 0;  // poisoned data is never reused
+  if (cfg->shard_slab) {
+    const int nb = (n_layers + cfg->block_size - 1) / cfg->block_size;
+    for (int b = 0; b < nb; ++b) {
+      size_t o = 0;
+      stream_shard_slab_layout(layers, n_layers, cfg->block_size, world, cfg->shard_rank, b, &o,
+                               nullptr, nullptr);
+      s->shard_off.push_back(o);
+    }
+  }
   s->ring = static_cast<uint8_t*>(ring_dev);
   s->slot_bytes = slot_bytes;
   s->slots.resize(static_cast<size_t>(n_slots));

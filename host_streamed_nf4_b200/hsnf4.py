@@ -54,7 +54,8 @@ GATHER_FN = ctypes.CFUNCTYPE(c_int, c_void_p, c_size_t, c_int, c_int, c_void_p, 
 class StreamConfig(Structure):
     _fields_ = [("block_size", c_int), ("enable_prefetch", c_int), ("reuse_resident", c_int),
                 ("poison_on_release", c_int), ("n_slots", c_int), ("shard_world", c_int),
-                ("shard_rank", c_int), ("gather", GATHER_FN), ("gather_user", c_void_p)]
+                ("shard_rank", c_int), ("gather", GATHER_FN), ("gather_user", c_void_p),
+                ("shard_slab", c_int)]
 
 
 class StreamStats(Structure):
@@ -129,6 +130,8 @@ _SIGS = {
     "stream_prefetch_ahead": ([c_void_p, POINTER(c_int), c_int, POINTER(c_int)], c_int),
     "stream_shard_range": ([c_size_t, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t),
                             POINTER(c_size_t)], c_int),
+    "stream_shard_slab_layout": ([POINTER(LayerDesc), c_int, c_int, c_int, c_int, c_int,
+                                  POINTER(c_size_t), POINTER(c_size_t), POINTER(c_size_t)], c_int),
     "stream_slot_bytes_sharded": ([POINTER(LayerDesc), c_int, c_int, c_int, POINTER(c_size_t)],
                                   c_int),
     "stream_create": ([c_void_p, c_size_t, POINTER(LayerDesc), c_int, POINTER(StreamConfig), c_void_p,
@@ -559,17 +562,34 @@ def shard_range(block_bytes: int, world: int, rank: int):
     return S.value, off.value, n.value
 
 
+def shard_slab_layout(descs, block_size: int, world: int, rank: int):
+    """Rank's shard slab: ([(offset in the shard slab, length) per block], total bytes)."""
+    arr = _desc_array(descs)
+    total = c_size_t(0)
+    _check(lib().stream_shard_slab_layout(arr, len(descs), block_size, world, rank, -1, None,
+                                          None, ctypes.byref(total)))
+    n_blocks = (len(descs) + block_size - 1) // block_size
+    out = []
+    for b in range(n_blocks):
+        off, n = c_size_t(0), c_size_t(0)
+        _check(lib().stream_shard_slab_layout(arr, len(descs), block_size, world, rank, b,
+                                              ctypes.byref(off), ctypes.byref(n), None))
+        out.append((off.value, n.value))
+    return out, total.value
+
+
 class Streamer:
     """Pinned-host NF4 stack -> 2-slot VRAM ring, prefetched one block ahead.
 
     shard=(rank, world, gather): stream 1/world of every block over this
     rank's link; gather(slot_offset, shard_bytes, world, block) must enqueue,
     on the current CUDA stream (the copy stream), the in-place all-gather of
-    the ring bytes [slot_offset, slot_offset + world * shard_bytes)."""
+    the ring bytes [slot_offset, slot_offset + world * shard_bytes).
+    shard_slab: the slab holds only this rank's shards (shard_slab_layout)."""
 
     def __init__(self, slab: torch.Tensor, descs, block_size: int, ring: torch.Tensor,
                  copy_stream: torch.cuda.Stream, enable_prefetch=True, reuse_resident=True,
-                 poison_on_release=False, n_slots=2, shard=None):
+                 poison_on_release=False, n_slots=2, shard=None, shard_slab=False):
         _need(slab, "slab", torch.uint8, device=False)
         if not slab.is_pinned():
             raise ValueError("slab must be page-locked (pin_memory)")
@@ -596,6 +616,7 @@ class Streamer:
             self._gather_cb = GATHER_FN(_cb)
             cfg.shard_world, cfg.shard_rank = world, rank
             cfg.gather = self._gather_cb
+            cfg.shard_slab = int(bool(shard_slab))
         self.n_slots = n_slots
         h = c_void_p()
         _check(lib().stream_create(_ptr(slab), slab.numel(), self._arr, len(self.descs),

@@ -61,7 +61,7 @@ class LayerStack:
                  poison_on_release: bool = False, r: int = synth.RANK, alpha: float = synth.ALPHA,
                  seed: int = 42, device=None, grouping: str = "layer", n_slots: int = 2,
                  base: str = "nf4", dropout: float = 0.0, data_seed=None, shard=None,
-                 slab=None):
+                 slab=None, shard_slab: bool = True):
         """shard = (rank, world, gather_factory): stream 1/world of every
         block (sharded stream); gather_factory(ring) returns the streamer's
         gather callback (dist.ring_gather).  data_seed: seed of the
@@ -69,7 +69,10 @@ class LayerStack:
         adapters always come from seed, as data-parallel ranks share them.
         slab: an already filled pinned slab of a stack with the same family,
         layer count, base and seed (e.g. another stack's .slab), used as is
-        instead of drawing and quantizing the base again."""
+        instead of drawing and quantizing the base again.
+        shard_slab (sharded streams): pin only this rank's shards of every
+        block, about 1/world of the base, so that the ranks of a node hold
+        one copy of it between them; False pins the whole base per rank."""
         self.device = torch.device(device) if device is not None else torch.device(
             "cuda", torch.cuda.current_device())
         dev = self.device
@@ -91,7 +94,15 @@ class LayerStack:
         self.layer_bytes = hsnf4.layer_bytes(self.desc)
         self.offs = [hsnf4.layer_offsets(self.desc, p) for p in range(self.P)]
         self.n_blocks = (n_layers + block_size - 1) // block_size
-        if slab is not None:
+        self.shard_slab = bool(shard) and streamed and shard_slab
+        if self.shard_slab:
+            if slab is not None:
+                raise ValueError("slab: a shard slab is filled by the stack itself")
+            self.shard_layout, total = hsnf4.shard_slab_layout(self.descs, block_size, shard[1],
+                                                               shard[0])
+            self.slab = torch.empty(max(total, 1), dtype=torch.uint8, pin_memory=True)
+            self._fill_shard_slab(seed, shard[0], shard[1])
+        elif slab is not None:
             if slab.dtype != torch.uint8 or slab.numel() != hsnf4.slab_bytes(self.descs) or \
                     not slab.is_pinned():
                 raise ValueError("slab: expected a pinned uint8 tensor of this stack's slab size")
@@ -113,7 +124,7 @@ class LayerStack:
                                            self.copy_stream, enable_prefetch=enable_prefetch,
                                            reuse_resident=reuse_resident,
                                            poison_on_release=poison_on_release, n_slots=n_slots,
-                                           shard=sh)
+                                           shard=sh, shard_slab=self.shard_slab)
         else:
             self.dev_slab = self.slab.to(dev)
             self.streamer = None
@@ -172,6 +183,49 @@ class LayerStack:
         device: lets a checker quantize it independently."""
         _, n, k = self.projs[p]
         return _randn_bf16((n, k), synth.W_STD, _gen(self.device, self.seed, l, p), self.device)
+
+    def _layer_into(self, buf: torch.Tensor, l: int, seed: int):
+        """Write layer l's slab bytes (drawn and quantized on the device)
+        into the device byte buffer buf [layer_bytes]."""
+        dev = self.device
+        for p, (_, n, k) in enumerate(self.projs):
+            w = _randn_bf16((n, k), synth.W_STD, _gen(dev, seed, l, p), dev)
+            co, ao = self.offs[p]
+            if self.base_format == hsnf4.BASE_BF16:
+                buf[co: co + n * k * 2].copy_(w.view(torch.uint8).flatten())
+                continue
+            W = hsnf4.nf4_quantize_pack(w)
+            buf[co: co + n * k // 2].copy_(W.codes)
+            buf[ao: ao + n * k // 16].copy_(W.absmax.view(torch.uint8))
+
+    def _fill_shard_slab(self, seed: int, rank: int, world: int):
+        """This rank's shard of every block, block after block: each block is
+        built on the device and only the rank's byte range copied down."""
+        dev = self.device
+        block = torch.zeros(self.block_size * self.layer_bytes, dtype=torch.uint8, device=dev)
+        for b in range(self.n_blocks):
+            layers = list(self.block_layers(b))
+            for i, l in enumerate(layers):
+                self._layer_into(block[i * self.layer_bytes: (i + 1) * self.layer_bytes], l, seed)
+            _, off, n = hsnf4.shard_range(len(layers) * self.layer_bytes, world, rank)
+            at, n2 = self.shard_layout[b]
+            assert n2 == n
+            if n:
+                self.slab[at: at + n].copy_(block[off: off + n])
+        torch.cuda.synchronize(dev)
+        del block
+
+    def device_weight(self, l: int, p: int):
+        """Layer l, projection p of the frozen base on the device, drawn and
+        quantized again (independent of where the slab keeps it)."""
+        w = self.base_weight_bf16(l, p)
+        if self.base_format == hsnf4.BASE_BF16:
+            return hsnf4.Bf16Weight(w)
+        return hsnf4.nf4_quantize_pack(w)
+
+    def pinned_bytes(self) -> int:
+        """Page-locked host bytes this stack holds for the frozen base."""
+        return self.slab.numel()
 
     def _fill_slab(self, seed: int):
         dev = self.device

@@ -443,6 +443,12 @@ typedef struct {
   int shard_rank;      /* this rank, in [0, shard_world) */
   hsnf4_gather_fn gather; /* required when shard_world >= 2; NULL otherwise */
   void *gather_user;   /* passed to gather */
+  int shard_slab;      /* sharded streams only.  0: pinned_slab holds the
+                          whole stack; 1: it holds only this rank's shards,
+                          block after block, laid out as
+                          stream_shard_slab_layout gives -- about 1/world of
+                          the stack, so that the node's ranks together pin
+                          one copy of the base */
 } hsnf4_stream_config;
 
 typedef struct {
@@ -482,6 +488,17 @@ int stream_slot_bytes(const hsnf4_layer_desc *layers, int n_layers,
 int stream_shard_range(size_t block_bytes, int world, int rank, size_t *shard_bytes,
                        size_t *off, size_t *len);
 
+/* Layout of a shard slab (hsnf4_stream_config.shard_slab): rank `rank`'s
+ * shards of every block (stream_shard_range of the block's bytes), packed
+ * block after block in block order.  For block >= 0, *block_off and *len
+ * (either may be NULL) receive where that block's shard starts in the shard
+ * slab and its length; *total_bytes (may be NULL) the size of the whole
+ * shard slab.  block = -1 asks for the total only.  Pure host arithmetic.
+ * Errors: INVALID (layers, sizes, rank or block out of range). */
+int stream_shard_slab_layout(const hsnf4_layer_desc *layers, int n_layers, int block_size,
+                             int world, int rank, int block, size_t *block_off, size_t *len,
+                             size_t *total_bytes);
+
 /* Bytes of one block slot of a stream sharded over `world` ranks (the
  * largest block rounded up to world * S); a ring of n_slots needs n_slots
  * times this.  world 1 gives stream_slot_bytes rounded up to 1 KiB. */
@@ -489,7 +506,8 @@ int stream_slot_bytes_sharded(const hsnf4_layer_desc *layers, int n_layers, int 
                               int world, size_t *out_bytes);
 
 /* Create a streamer.  pinned_slab: HOST pointer to page-locked memory of
- * slab_bytes holding the stack; ring_dev: device memory of ring_bytes
+ * slab_bytes holding the stack (or, with cfg->shard_slab, this rank's
+ * shards of it); ring_dev: device memory of ring_bytes
  * (>= stream_ring_bytes(), 1 KiB aligned); copy_stream: the dedicated H2D
  * stream.  The caller keeps all three alive until stream_destroy.  Errors:
  * INVALID, OOM (ring or slab too small: needed vs given), CUDA. */

@@ -86,6 +86,31 @@ def test_shard_ranges_tile_every_block():
             assert covered == B
 
 
+def test_shard_slabs_hold_exactly_each_ranks_shards():
+    """The shard slabs of a node's ranks, between them, hold every byte of the
+    stack exactly once: each rank's slab is its shard of every block, packed
+    block after block."""
+    from host_streamed_nf4_b200 import hsnf4
+    descs = [hsnf4.layer_desc([(896, 1024), (128, 1024), (1024, 1536), (1024, 512)])] * 7
+    full = hsnf4.slab_bytes(descs)
+    layer = hsnf4.layer_bytes(descs[0])
+    for bs in (1, 2, 3, 4, 7):
+        n_blocks = (7 + bs - 1) // bs
+        for world in (1, 2, 3, 4, 8):
+            totals = 0
+            for rank in range(world):
+                layout, total = hsnf4.shard_slab_layout(descs, bs, world, rank)
+                assert len(layout) == n_blocks
+                at = 0
+                for b, (off, n) in enumerate(layout):
+                    B = (min(7, (b + 1) * bs) - b * bs) * layer
+                    assert (off, n) == (at, hsnf4.shard_range(B, world, rank)[2])
+                    at += n
+                assert at == total
+                totals += total
+            assert totals == full, (bs, world)
+
+
 def _gather_worker(rank, ws, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=ws,
@@ -102,6 +127,25 @@ def _gather_worker(rank, ws, port, q):
             ring[slot_off + off: slot_off + off + n] = slab[off: off + n]
             hdist.ring_gather(ring)(slot_off, S, ws, 0)
             results.append(bool(torch.equal(ring[slot_off: slot_off + B], slab[:B])))
+        # a stack whose ranks each hold only their shard slab: every block
+        # rebuilt through the gather equals the block of the whole stack
+        descs = [hsnf4.layer_desc([(384, 512), (128, 512)])] * 5
+        full = torch.randint(0, 256, (hsnf4.slab_bytes(descs),), dtype=torch.uint8, generator=g)
+        layer = hsnf4.layer_bytes(descs[0])
+        bs = 2
+        layout, total = hsnf4.shard_slab_layout(descs, bs, ws, rank)
+        mine = torch.empty(total, dtype=torch.uint8)
+        for b, (at, n) in enumerate(layout):
+            B = (min(5, (b + 1) * bs) - b * bs) * layer
+            _, off, n2 = hsnf4.shard_range(B, ws, rank)
+            mine[at: at + n] = full[b * bs * layer + off: b * bs * layer + off + n2]
+        for b, (at, n) in enumerate(layout):
+            B = (min(5, (b + 1) * bs) - b * bs) * layer
+            S, off, _ = hsnf4.shard_range(B, ws, rank)
+            ring = torch.zeros(ws * S, dtype=torch.uint8)
+            ring[off: off + n] = mine[at: at + n]
+            hdist.ring_gather(ring)(0, S, ws, b)
+            results.append(bool(torch.equal(ring[:B], full[b * bs * layer: b * bs * layer + B])))
         q.put((rank, results))
     finally:
         dist.destroy_process_group()

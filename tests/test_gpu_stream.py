@@ -194,10 +194,11 @@ def test_prefetch_ahead_fills_free_slots_in_visit_order():
 
 # ---------------------------------------------------------------- sharded stream, one GPU
 
-def _emulated_peers(holder):
+def _emulated_peers(holder, full_slab):
     """Gather factory that stands in for the other ranks on one GPU: it fills
-    their shards of the slot from the pinned slab (what their own PCIe copies
-    would have brought), enqueued on the copy stream like the all-gather."""
+    their shards of the slot from the whole stack's pinned slab (what their
+    own PCIe copies would have brought), enqueued on the copy stream like the
+    all-gather."""
     def factory(ring):
         def gather(slot_off, S, world, block):
             st = holder[0]
@@ -208,17 +209,30 @@ def _emulated_peers(holder):
                 n = max(0, min(S, B - off))
                 if j != st.shard[0] and n:
                     ring[slot_off + off: slot_off + off + n].copy_(
-                        st.slab[base + off: base + off + n], non_blocking=True)
+                        full_slab[base + off: base + off + n], non_blocking=True)
         return gather
     return factory
 
 
-@pytest.mark.parametrize("world,rank,bs", [(2, 0, 1), (2, 1, 2), (4, 3, 1), (4, 2, 4)])
-def test_sharded_stream_equals_resident_bitwise(resident6, world, rank, bs):
+@pytest.fixture(scope="module")
+def tiny6_slab():
+    s = LayerStack(TINY, 6, 96, streamed=False)
+    slab = s.slab
+    s.close()
+    return slab
+
+
+@pytest.mark.parametrize("world,rank,bs,shard_slab", [(2, 0, 1, True), (2, 1, 2, True),
+                                                      (4, 3, 1, True), (4, 2, 4, True),
+                                                      (2, 1, 2, False), (4, 2, 4, False)])
+def test_sharded_stream_equals_resident_bitwise(resident6, tiny6_slab, world, rank, bs,
+                                                shard_slab):
     holder = []
-    s = LayerStack(TINY, 6, 96, block_size=bs, streamed=True, shard=(rank, world,
-                                                                       _emulated_peers(holder)))
+    s = LayerStack(TINY, 6, 96, block_size=bs, streamed=True,
+                   shard=(rank, world, _emulated_peers(holder, tiny6_slab)), shard_slab=shard_slab)
     holder.append(s)
+    if shard_slab:  # this rank pins only its shards: about 1/world of the stack
+        assert s.pinned_bytes() < tiny6_slab.numel() / world + s.n_blocks * 1024
     _assert_bitwise(_run(s), resident6)
     st = s.streamer.stats()
     assert st["gathers"] == st["copies"] > 0
