@@ -232,4 +232,5 @@ def test_bench_reference_arm_prints_its_json_line():
               "cpu_baseline", "e2e"):
         assert k in d, k
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
-    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["config"]["workload"] == "qwen2.5-7b-layer"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["config"]["workload"] == "qwen2.5-72b-stack"
+    assert d["config"]["layers"] == 80 and "one layer x 80, extrapolated" in d["cpu_baseline"]["sample"]
