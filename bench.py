@@ -2,8 +2,8 @@
 """Benchmark of the host-streamed NF4 LoRA hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload qwen2.5-7b-layer|llama-3.1-8b-stack|qwen2.5-32b-stack|
-                                qwen2.5-72b-stack]
+                    [--workload qwen2.5-72b-stack|qwen2.5-72b-layer|qwen2.5-7b-layer|
+                                llama-3.1-8b-stack|qwen2.5-32b-stack]
                     [--mode streamed|resident] [--block-size B] [--seq T]
 
 One step = forward + backward of every LoRA-targeted projection (q, k, v,
@@ -45,6 +45,8 @@ PCIE_GEN5_X16_GBPS = 63.0  # per direction, theoretical (32 GT/s x 16 lanes, 128
 WORKLOADS = {
     # name: (family, layers, default block size, default mode)
     "qwen2.5-7b-layer": ("qwen2.5-7b", 1, 1, "streamed"),
+    # one layer of the 72B stack: the same grouped launches, small enough to profile
+    "qwen2.5-72b-layer": ("qwen2.5-72b", 1, 1, "streamed"),
     "llama-3.1-8b-stack": ("llama-3.1-8b", 32, 4, "streamed"),
     "qwen2.5-32b-stack": ("qwen2.5-32b", 64, 4, "streamed"),
     "qwen2.5-72b-stack": ("qwen2.5-72b", 80, 4, "streamed"),
@@ -421,6 +423,21 @@ def run_ours(args, ws, rank, local):
         step_roofline["frac_vs_probe"] = round(
             (h2d_step / (ms_step / 1e3) / 1e9) / link["probe_GBps"], 4)
 
+    # ------------------------------------------------ result check
+    # one more step (no gradient exchange), then layers 0 and L-1 recomputed
+    # from weights drawn afresh and held in VRAM: their outputs and adapter
+    # gradients must equal the streamed step's bit for bit
+    check = None
+    if args.model == "projections":
+        if streamed and single:
+            stack.step_single_block()
+        else:
+            stack.step()
+        res = stack.resident_check()
+        check = {"layers": {str(k): v for k, v in res.items()}, "bitwise": all(res.values()),
+                 "what": "t, dA, dB of layers 0 and L-1, Y of layer L-1, dX of layer 0, vs a "
+                         "resident recomputation"}
+
     # ------------------------------------------------ end to end through the API
     e2e = None
     if not args.no_e2e:
@@ -443,6 +460,7 @@ def run_ours(args, ws, rank, local):
                                               if shard else ")") if ws > 1 else "single"),
                    "l2": "no flush: every step reads > 126 MB L2 (NF4 weights + activations)"},
         "roofline": roofline, "step_roofline": step_roofline, "rank_r": rank_r,
+        "resident_check": check,
         "dequant": dequant, "merge": merge,
         "peak_vram_GB": round(torch.cuda.max_memory_allocated(dev) / 1e9, 3), "e2e": e2e,
         # page-locked host bytes of the frozen base on this rank (a sharded

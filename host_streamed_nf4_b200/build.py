@@ -25,7 +25,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-Wall",
           "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr"]
-SOURCES = ["api.cu", "nf4_codec.cu", "lora_aux.cu", "lora_gemm.cu", "streamer.cpp", "profile.cpp",
+SOURCES = ["api.cu", "nf4_codec.cu", "lora_rank.cu", "lora_gemm.cu", "streamer.cpp", "profile.cpp",
            "noalloc.cu", "lora_merge.cu",
            "lora_dropout.cu", "glue.cu", "attention.cu"]
 

@@ -94,9 +94,12 @@ int hsnf4_device_status(void* stream, uint32_t* flags) {
   int rc = cuda_status(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)),
                        "hsnf4_device_status: cudaStreamSynchronize");
   if (rc) return rc;
-  uint32_t f = 0;
+  uint32_t f = 0, fr = 0, fm = 0;
   rc = cuda_status(read_gemm_flags(&f), "hsnf4_device_status: read flags");
+  if (!rc) rc = cuda_status(read_rank_flags(&fr), "hsnf4_device_status: read flags");
+  if (!rc) rc = cuda_status(read_merge_flags(&fm), "hsnf4_device_status: read flags");
   if (rc) return rc;
+  f |= fr | fm;
   *flags = f;
   if (f) return fail(HSNF4_ERR_DEVICE, "a kernel wait gave up (flags 0x%x)", f);
   return HSNF4_OK;
@@ -262,12 +265,14 @@ static void fwd_layout(const hsnf4_lora_fwd_args* p, int n, int64_t T, int r, Fw
 
 // Workspace layout of a backward group:
 //   [s*u bf16 [T, r_pad] per problem][u fp32 [T, r] per problem]
+//   [u and t as two bf16 parts each, 4 x [T, r_pad] per problem: the
+//    adapter-gradient operands]
 //   [X_d bf16 [T, k_in] and its keep-mask bytes [T, k_in / 8] per problem
 //    with dropout]
 //   [projection partials][GEMM split-K partial tiles]
 // As for the forward, every byte read was written earlier in the same call.
 struct BwdLayout {
-  size_t su[8], u[8], xd[8], bits[8], prj, gemm, total;
+  size_t su[8], u[8], parts[8], xd[8], bits[8], prj, gemm, total;
 };
 
 static void bwd_layout(const hsnf4_lora_bwd_args* p, int n, int64_t T, int r, BwdLayout* L) {
@@ -280,6 +285,10 @@ static void bwd_layout(const hsnf4_lora_bwd_args* p, int n, int64_t T, int r, Bw
   for (int i = 0; i < n; ++i) {
     L->u[i] = off;
     off += round_up(static_cast<size_t>(T) * r * 4, 256);
+  }
+  for (int i = 0; i < n; ++i) {
+    L->parts[i] = off;
+    off += 4 * round_up(static_cast<size_t>(T) * rp * 2, 256);
   }
   for (int i = 0; i < n; ++i) {
     L->xd[i] = off;
@@ -432,11 +441,18 @@ int lora_group_bwd(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r, fl
                 ws + L.bits[i]};
       ++nd;
     }
-    pd[i] = {p.dY, p.W.n_out, p.B, false, u, ws + L.su[i], drop};
+    // u and the forward's t as two bf16 parts each: the gradient kernel's operands
+    const size_t part = round_up(static_cast<size_t>(T) * r_padded(r) * 2, 256);
+    uint8_t* u_hi = ws + L.parts[i];
+    uint8_t* u_lo = u_hi + part;
+    uint8_t* t_hi = u_lo + part;
+    uint8_t* t_lo = t_hi + part;
+    pd[i] = {p.dY, p.W.n_out, p.B, false, u, ws + L.su[i], drop, u_hi, u_lo, p.t_save, t_hi,
+             t_lo};
     gd[i] = {p.W.codes, p.W.absmax, p.W.n_out, p.W.k_in, p.dY, p.A, ws + L.su[i], p.dX,
              p.W.format == HSNF4_BASE_BF16};
-    grd[2 * i] = {p.dY, p.W.n_out, p.t_save, p.dB, true};  // dB = s dY^T t    [n_out, r]
-    grd[2 * i + 1] = {xl, p.W.k_in, u, p.dA, false};       // dA = s u^T X(_d) [r, k_in]
+    grd[2 * i] = {p.dY, p.W.n_out, t_hi, t_lo, p.dB, true};  // dB = s dY^T t    [n_out, r]
+    grd[2 * i + 1] = {xl, p.W.k_in, u_hi, u_lo, p.dA, false};  // dA = s u^T X(_d) [r, k_in]
   }
   if (nd) {
     rc = cuda_status(launch_dropout_apply(dd, nd, T, st), "lora_group_bwd: dropout launch");

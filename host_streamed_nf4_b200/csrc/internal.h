@@ -2,6 +2,7 @@
 // units (not part of the public ABI; see include/hsnf4.h for that).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -35,9 +36,11 @@ cudaError_t launch_nf4_quantize(const void* w, int64_t n_out, int64_t k_in, void
 cudaError_t launch_nf4_dequant(const void* codes, const float* absmax, int64_t n_out,
                                int64_t k_in, void* out, cudaStream_t st);
 
-// ---- rank-r projections, grouped: t_q = Z_q Adp_q^T (fp32 [T, r]) and
-// zs_q = bf16(s * t_q) ([T, r_pad], pad columns 0).  Adp is A [r, C]
-// (r_major) or B [C, r].  Workspace: project_workspace_bytes().
+// ---- rank-r projections, grouped (lora_rank.cu): t_q = Z_q Adp_q^T (fp32
+// [T, r]) and zs_q = bf16(s * t_q) ([T, r_pad], pad columns 0).  Adp is
+// A [r, C] (r_major, forward) or B [C, r] (backward).  Optional outputs:
+// hi/lo, the two bf16 parts of t_q ([T, r_pad] each); split_hi/lo, the two
+// bf16 parts of split_src (fp32 [T, r]).  No workspace.
 struct ProjectDesc {
   const void* Z;
   int64_t C;
@@ -46,22 +49,37 @@ struct ProjectDesc {
   float* t_out;
   void* zs;
   bool zero_zs = false;  // write zs = 0 (the GEMM's rank-r slice then adds nothing)
+  void* hi = nullptr;
+  void* lo = nullptr;
+  const float* split_src = nullptr;
+  void* split_hi = nullptr;
+  void* split_lo = nullptr;
 };
 size_t project_workspace_bytes(const ProjectDesc* d, int n, int64_t T, int r);
 cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, int r, float s,
                                       void* ws, cudaStream_t st);
 
-// ---- adapter gradients, grouped: out_q = s Z_q^T V_q, Z bf16 [T, C],
-// V fp32 [T, r]; out is [C, r] (c_major, dB) or [r, C] (dA).
+// ---- adapter gradients, grouped (lora_rank.cu): out_q = s Z_q^T V_q, Z
+// bf16 [T, C], V = V_hi + V_lo (bf16 [T, r_pad] each); out is [C, r]
+// (c_major, dB) or [r, C] (dA).
 struct GradDesc {
   const void* Z;
   int64_t C;
-  const float* V;
+  const void* V_hi;
+  const void* V_lo;
   float* out;
   bool c_major;
 };
 cudaError_t launch_lora_grad_group(const GradDesc* d, int n, int64_t T, int r, float s,
                                    cudaStream_t st);
+cudaError_t read_rank_flags(uint32_t* flags);
+cudaError_t read_merge_flags(uint32_t* flags);
+
+// 2-D TMA descriptor of a row-major tensor [outer][inner] (row_bytes apart)
+// with a box of box_inner x box_outer elements; false if the driver refuses.
+bool encode_tma_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle sw);
 
 enum GemmMode { kGemmFwd = 0, kGemmDx = 1 };
 
@@ -134,7 +152,15 @@ cudaError_t launch_attention_bwd(const void* q, const void* k, const void* v, co
                                  cudaStream_t st);
 
 // Kernel timing (hsnf4_profile): bracket a launch with prof_begin/prof_end.
-enum ProfKind { kProfGemmFwd = 0, kProfGemmDx = 1, kProfDequant = 2, kProfMerge = 3, kProfKinds = 4 };
+enum ProfKind {
+  kProfGemmFwd = 0,
+  kProfGemmDx = 1,
+  kProfDequant = 2,
+  kProfMerge = 3,
+  kProfProject = 4,
+  kProfGrad = 5,
+  kProfKinds = 6
+};
 bool profiling();
 void* prof_begin(cudaStream_t st);
 void prof_end(void* token, int kind, double work, cudaStream_t st);

@@ -80,6 +80,7 @@ constexpr int kStepK = 64;                     // contraction per pipeline step
 constexpr int kCodeBytes = 4096;               // raw codes of one step (128 x 64 / 2)
 constexpr int kATileBytes = kTileM * 128;      // dequantized bf16 A tile
 constexpr int kStageElems = 16 * kTileM;       // epilogue transpose buffer: 16 tokens x 128 rows
+constexpr int kStageBufs = 4;                  // ... a ring of 4: two per 32-token step
 constexpr int kMaxSmem = 232448;               // 227 KiB opt-in per block
 constexpr int kThreads = 15 * 32;
 constexpr int kWarpEpi = 8, kWarpProdX = 12, kWarpProdC = 13, kWarpMma = 14;
@@ -90,6 +91,7 @@ struct GemmProblem {
                           // bf16 [n_out, k_in], box {64, 128} fwd, {64, 64} dx, 128B swizzle
   CUtensorMap map_lo_a;   // fwd: B [n_out, r] box {16, 128} 32B; dx: A [r, k_in] box {64, r_pad} 128B
   CUtensorMap map_lo_b;   // s*t or s*u: bf16 [T, r_pad], box {16, min(BN/2,128)}, 32B swizzle
+  CUtensorMap map_out;    // output bf16 [T, m_total], box {128 rows, 16 tokens}, no swizzle
   const float* absmax;
   uint16_t* out;          // bf16 [T, m_total]
   float* partial;         // split-K partial tiles (fp32 [BN tokens][128 rows] each), or null
@@ -146,7 +148,7 @@ __host__ __device__ inline SmemPlan smem_plan(int mode, int BN, int sx, int sc, 
   const int la = (mode == kGemmFwd) ? slices * 4096 : 2 * r_pad * 128;
   p.lb_off = p.la_off + la;
   p.st_off = p.lb_off + slices * (BN / 2) * 32;
-  p.bar_off = p.st_off + 2 * kStageElems * 2;
+  p.bar_off = p.st_off + kStageBufs * kStageElems * 2;
   p.total = p.bar_off + (2 * sx + 2 * sc + 2 * sa + 16) * 8 + 32;
   return p;
 }
@@ -573,6 +575,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int i = threadIdx.x - kWarpEpi * 32;  // 0..127: TMEM lane = tile row
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     int lu = 0;
+    int epi_step = 0;  // 32-token output steps so far (picks the staging buffer pair)
     for (int ui = u_begin; ui < u_end; ++ui, ++lu) {
       const Unit U = unpack_unit(P, P.units[ui]);
       const GemmProblem& pr = P.prob[U.p];
@@ -607,33 +610,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_arrive(&acc_empty[buf]);
         continue;
       }
-      for (int c = 0; c < BN; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(acc0 + static_cast<uint32_t>(c), v);
+      // 32 tokens per step: one TMEM load, a transpose into two 16-token x
+      // 128-row bf16 buffers (sb[token j][row i]) of a ring of four, and two
+      // TMA tile stores issued by thread 0 (rows and tokens past the output's
+      // edge are not written).  Buffers alternate in pairs: before the step's
+      // barrier thread 0 waits until the previous step's stores have read
+      // their buffers, which the next step overwrites.
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(acc0 + static_cast<uint32_t>(c), v);
         tmem_wait_ld();
-        // transpose through smem: sb[token j][row i], double-buffered
-        uint16_t* sb = stage + ((c >> 4) & 1) * kStageElems;
+        uint16_t* sb = stage + (epi_step & 1) * 2 * kStageElems;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 32; ++j) {
           const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[j]));
           sb[j * kTileM + i] = *reinterpret_cast<const uint16_t*>(&b);
         }
+        fence_proxy_async_smem();
+        if (i == 0) bulk_wait_group_read<0>();
         named_sync(1, 128);
-        // 16 token rows x 256 B of output: 256 chunks of 16 B, two per thread
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int chunk = i + h * 128;
-          const int j = chunk >> 4, col = (chunk & 15) * 8;
-          const int t = t0 + c + j, row = m0 + col;
-          if (t < P.T && row < M) {
-            const uint4 val = *reinterpret_cast<const uint4*>(sb + j * kTileM + col);
-            *reinterpret_cast<uint4*>(pr.out + static_cast<int64_t>(t) * M + row) = val;
-          }
+        if (i == 0) {
+          for (int h = 0; h < 2; ++h)
+            if (t0 + c + 16 * h < P.T)
+              tma_store_2d(&pr.map_out, sb + h * kStageElems, m0, t0 + c + 16 * h);
+          bulk_commit_group();
         }
+        ++epi_step;
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
     }
+    if (i == 0) bulk_wait_group_all();  // the output stores are done before smem goes away
   }
 
   // -------------------------------------------------- teardown
@@ -761,9 +768,9 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-static bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
-                      uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                      CUtensorMapSwizzle sw) {
+bool encode_tma_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle sw) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -1066,27 +1073,30 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     g.m_tiles = (g.m_total + kPairM - 1) / kPairM;
     g.splits = L.splits[p];
     if (g.splits > 1) g.partial = reinterpret_cast<float*>(ws + L.part_base[p]);
-    ok = ok && encode_2d(&g.map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.act, contraction, T,
+    ok = ok && encode_tma_2d(&g.map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.act, contraction, T,
                          contraction * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
     if (d.dense)  // bf16 [n_out, k_in]: 64 k x (128 rows fwd | 64 rows dx), 128B swizzle
-      ok = ok && encode_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.codes, d.k_in,
+      ok = ok && encode_tma_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.codes, d.k_in,
                            d.n_out, d.k_in * 2, 64, mode == kGemmFwd ? 128 : 64,
                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (mode == kGemmFwd) {
       if (!d.dense)
-        ok = ok && encode_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
+        ok = ok && encode_tma_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
                              d.n_out, d.k_in / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
-      ok = ok && encode_2d(&g.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_a, r, d.n_out,
+      ok = ok && encode_tma_2d(&g.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_a, r, d.n_out,
                            r * 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
     } else {
       if (!d.dense)
-        ok = ok && encode_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
+        ok = ok && encode_tma_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
                              d.n_out, d.k_in / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
-      ok = ok && encode_2d(&g.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_a, d.k_in, r,
+      ok = ok && encode_tma_2d(&g.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_a, d.k_in, r,
                            d.k_in * 2, 64, r_pad, CU_TENSOR_MAP_SWIZZLE_128B);
     }
-    ok = ok && encode_2d(&g.map_lo_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_b, r_pad, T,
+    ok = ok && encode_tma_2d(&g.map_lo_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_b, r_pad, T,
                          r_pad * 2, 16, box_rows, CU_TENSOR_MAP_SWIZZLE_32B);
+    ok = ok && encode_tma_2d(&g.map_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.out, g.m_total, T,
+                             static_cast<uint64_t>(g.m_total) * 2, kTileM, 16,
+                             CU_TENSOR_MAP_SWIZZLE_NONE);
   }
   if (!ok) return fail(HSNF4_ERR_CUDA, "lora gemm: cuTensorMapEncodeTiled failed");
 

@@ -25,7 +25,7 @@ bool g_on = false;
 std::vector<Rec> g_recs;
 
 const char* kKindName[kProfKinds] = {"lora_gemm_fwd", "lora_gemm_dx", "nf4_dequant",
-                                      "lora_merge"};
+                                      "lora_merge",    "lora_project", "lora_grad"};
 
 }  // namespace
 

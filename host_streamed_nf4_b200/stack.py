@@ -379,6 +379,52 @@ class LayerStack:
         self.streamer.release(0, self.compute)
         self.step_idx += 1
 
+    # ------------------------------------------------------------------ checks
+
+    def resident_check(self) -> dict:
+        """Bitwise check of the last step against a resident recomputation:
+        layers 0 and L-1 are run again from weights drawn and quantized
+        afresh on the device (not from the ring), with the step's inputs, and
+        their t, dA, dB -- plus Y of layer L-1 (the forward's last output)
+        and dX of layer 0 (the backward's last output) -- must equal what
+        the step left behind.  Call right after step(); returns the
+        comparison per layer."""
+        dev, T, r = self.device, self.T, self.r
+        step = self.step_idx - 1  # the step whose outputs are checked
+        out = {}
+        for l in sorted({0, self.L - 1}):
+            ws = [self.device_weight(l, p) for p in range(self.P)]
+            Y = [torch.empty(T, n, dtype=torch.bfloat16, device=dev) for _, n, _ in self.projs]
+            t = [torch.empty(T, r, dtype=torch.float32, device=dev) for _ in self.projs]
+            dX = [torch.empty(T, k, dtype=torch.bfloat16, device=dev) for _, _, k in self.projs]
+            dA = [torch.empty(r, k, dtype=torch.float32, device=dev) for _, _, k in self.projs]
+            dB = [torch.empty(n, r, dtype=torch.float32, device=dev) for _, n, _ in self.projs]
+
+            def drop(p, l=l):
+                if self.dropout <= 0.0:
+                    return None
+                return (self.dropout, self.seed, (step << 32) | (l << 4) | p)
+
+            for grp in self.groups:
+                args = [hsnf4.fwd_args(ws[p], self.X[INPUT_OF[self.projs[p][0]]], self.A[l][p],
+                                       self.B[l][p], Y[p], t[p], drop(p)) for p in grp]
+                hsnf4.lora_group_fwd(args, T, r, self.alpha, self.ws_f, stream=self.compute)
+            for grp in reversed(self.groups):
+                args = [hsnf4.bwd_args(ws[p], self.X[INPUT_OF[self.projs[p][0]]], t[p],
+                                       self.A[l][p], self.B[l][p], self.dY[p], dX[p], dA[p],
+                                       dB[p], drop(p)) for p in grp]
+                hsnf4.lora_group_bwd(args, T, r, self.alpha, self.ws_b, stream=self.compute)
+            torch.cuda.synchronize(dev)
+            eq = all(torch.equal(t[p], self.t[l][p]) and torch.equal(dA[p], self.dA[l][p]) and
+                     torch.equal(dB[p], self.dB[l][p]) for p in range(self.P))
+            if l == self.L - 1:
+                eq = eq and all(torch.equal(Y[p], self.Y[p]) for p in range(self.P))
+            if l == 0:
+                eq = eq and all(torch.equal(dX[p], self.dX[p]) for p in range(self.P))
+            out[l] = bool(eq)
+            del ws, Y, t, dX, dA, dB
+        return out
+
     # ------------------------------------------------------------------ accounting
 
     def block_bytes(self, b: int) -> int:

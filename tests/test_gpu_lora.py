@@ -94,12 +94,19 @@ GROUP = [  # (N, K): mixed shapes, one long-K problem (split along K), ragged N
 ]
 
 
-def _group_run(orc, cases, T, r, alpha):
+def _group_run(orc, cases, T, r, alpha, share_x=False):
+    """One grouped forward + backward.  share_x: problems whose X is the same
+    host array get the same device tensor (one pointer, as in a layer)."""
     Ws, ins, outs = [], [], []
     fa, ba = [], []
+    dev_x = {}
     for c in cases:
         W = oracle_nf4_weight(orc, c.W)
-        X, A, B, dY = (to_dev_bf16(a) for a in (c.X, c.A, c.B, c.dY))
+        A, B, dY = (to_dev_bf16(a) for a in (c.A, c.B, c.dY))
+        if share_x:
+            X = dev_x.setdefault(id(c.X), to_dev_bf16(c.X))
+        else:
+            X = to_dev_bf16(c.X)
         N, K = c.W.shape
         Y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
         t = torch.empty(T, r, dtype=torch.float32, device="cuda")
@@ -128,6 +135,25 @@ def test_group_fwd_bwd_vs_oracle(orc, T):
     Ws, outs = _group_run(orc, cases, T, r, alpha)
     for c, W, (Y, t, dX, dA, dB) in zip(cases, Ws, outs):
         _check(orc, c, (W, Y, t, dX, dA, dB), what=f"group T{T} {c.W.shape}")
+
+
+@pytest.mark.parametrize("T,r", [(512, 16), (300, 8), (129, 64), (64, 24)])
+def test_group_sharing_one_input_vs_oracle(orc, T, r):
+    """Problems that read the same X (as q, k, v, gate and up do) are stacked
+    on one read of X by the rank-r kernels; each must still match the
+    oracle.  Their upstream gradients differ, and one problem reads another X."""
+    alpha = 2.0 * r
+    K = 640
+    shared = synth.linear_case(9500 + T + r, T, 64, K, r=r, alpha=alpha)
+    cases = []
+    for i, N in enumerate([384, 128, 128, 1152, 1152]):
+        c = synth.linear_case(9600 + 17 * i + T + r, T, N, K, r=r, alpha=alpha)
+        c.X = shared.X  # the same input tensor for all five
+        cases.append(c)
+    cases.append(synth.linear_case(9700 + T + r, T, 512, 1152, r=r, alpha=alpha))
+    Ws, outs = _group_run(orc, cases, T, r, alpha, share_x=True)
+    for c, W, (Y, t, dX, dA, dB) in zip(cases, Ws, outs):
+        _check(orc, c, (W, Y, t, dX, dA, dB), what=f"shared-X group T{T} r{r} {c.W.shape}")
 
 
 def test_group_deterministic_bitwise(orc):

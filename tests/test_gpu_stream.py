@@ -305,3 +305,15 @@ def test_nccl_ring_gather_on_one_rank():
     r = subprocess.run([sys.executable, "-c", _NCCL_CHILD], env=env, capture_output=True,
                        text=True, timeout=300)
     assert "NCCL_GATHER_OK" in r.stdout, (r.stdout[-2000:], r.stderr[-2000:])
+
+
+@pytest.mark.parametrize("bs,dropout", [(2, 0.0), (4, 0.1)])
+def test_resident_check_of_a_streamed_step(bs, dropout):
+    """The bench's result check: layers 0 and L-1 recomputed from freshly
+    drawn weights in VRAM equal the streamed step bit for bit."""
+    s = LayerStack(TINY, 6, 96, block_size=bs, streamed=True, dropout=dropout)
+    s.step()
+    s.step()
+    res = s.resident_check()
+    s.close()
+    assert res == {0: True, 5: True}

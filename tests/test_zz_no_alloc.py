@@ -71,10 +71,11 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     """Checked from the shapes alone: the call fails before touching memory."""
     L = hsnf4.lib()
     fake = 0x10000
-    # r = 64 over a 32768-wide contraction at 16384 tokens: the rank-r
-    # projection's partial sums alone need 128 MiB
-    W = hsnf4.Nf4WeightC(fake, fake, 4096, 32768)
-    rc = L.lora_linear_fwd_noalloc(ctypes.byref(W), fake, 16384, fake, fake, 64, 128.0, fake,
+    # a 128 x 131072 weight at 32768 tokens: few, very long tiles, so the GEMM
+    # splits the contraction and its fp32 partial tiles need ~259 MiB
+    assert L.lora_linear_fwd_workspace(32768, 128, 131072, 16) > 64 << 20
+    W = hsnf4.Nf4WeightC(fake, fake, 128, 131072)
+    rc = L.lora_linear_fwd_noalloc(ctypes.byref(W), fake, 32768, fake, fake, 16, 32.0, fake,
                                    fake, None)
     assert rc == hsnf4.ERR_INVALID
     msg = hsnf4.last_error()
