@@ -252,7 +252,11 @@ static void fwd_layout(const hsnf4_lora_fwd_args* p, int n, int64_t T, int r, Fw
   ProjectDesc pd[8];
   GemmProblemDesc gd[8];
   for (int i = 0; i < n; ++i) {
-    pd[i] = {p[i].X, p[i].W.k_in, p[i].A, true, nullptr, nullptr};
+    // with dropout the projection reads this problem's own X_d: a distinct
+    // input, as the launch will see it (only equality of inputs matters here)
+    const void* z = p[i].dropout_p > 0.0f ? reinterpret_cast<const void*>(uintptr_t(16) * (i + 1))
+                                          : p[i].X;
+    pd[i] = {z, p[i].W.k_in, p[i].A, true, nullptr, nullptr};
     gd[i] = {p[i].W.codes, p[i].W.absmax, p[i].W.n_out, p[i].W.k_in, p[i].X, p[i].B, nullptr,
              p[i].Y, p[i].W.format == HSNF4_BASE_BF16};
   }

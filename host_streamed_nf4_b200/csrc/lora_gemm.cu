@@ -640,7 +640,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
     }
-    if (i == 0) bulk_wait_group_all();  // the output stores are done before smem goes away
+    if (i == 0) bulk_wait_group_read<0>();  // the output stores have read smem before it goes away
   }
 
   // -------------------------------------------------- teardown

@@ -19,6 +19,7 @@
 // once plus W' written once; several CTAs per SM keep loads in flight.
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "internal.h"
@@ -37,6 +38,25 @@ enum : unsigned int {
 
 constexpr int kMrgTile = 128;
 
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// named barrier that also ANDs a predicate over its n threads, so that a
+// group leaving its loop on a failed wait leaves it together
+__device__ __forceinline__ bool named_sync_and_mrg(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
 struct MergeParams {
   CUtensorMap map_base;  // NF4: codes uint8 [N, K/2], box {64, 128}, 64B swizzle
                          // dense: bf16 [N, K], box {64, 128}, 128B swizzle (two per tile)
@@ -45,48 +65,63 @@ struct MergeParams {
   CUtensorMap map_out;   // W' bf16 [N, K], box {64, 128}, 128B swizzle
   const float* absmax;   // NF4 only: fp32 [N, K/64]
   int64_t N, K;
-  int r_pad, dense, col_tiles;
+  int r_pad, dense, col_tiles, row_tiles;
   float s;
   Nf4Codebook cb;
 };
 
-// shared-memory plan of a tile (offsets from a 1 KiB-aligned base)
+// shared-memory plan (offsets from a 1 KiB-aligned base): two load stages
+// (base tile, B slices, A atoms) and two output staging tiles
 struct MergeSmem {
-  int base, b, a, out, total;
+  int b, a, stage, out, total;  // b, a: offsets inside a stage
 };
 
 __host__ __device__ inline MergeSmem merge_smem(int dense, int r_pad) {
   MergeSmem m;
-  m.base = 0;
   m.b = dense ? 32768 : 8192;        // base tile: 128 x 128 bf16, or 128 x 64 code bytes
   m.a = m.b + (r_pad / 16) * 4096;   // B: r_pad / 16 slices of 128 rows x 32 B
-  m.out = m.a + 2 * r_pad * 128;     // A: two 64-column atoms of r_pad rows x 128 B
-  m.total = m.out + 2 * 16384;       // W': two 64-column boxes of 128 rows x 128 B
+  m.stage = m.a + 2 * r_pad * 128;   // A: two 64-column atoms of r_pad rows x 128 B
+  m.out = 2 * m.stage;               // W': per buffer two 64-column boxes of 128 rows x 128 B
+  m.total = m.out + 2 * 32768;
   return m;
 }
 
-__global__ void __launch_bounds__(128) lora_merge_kernel(const __grid_constant__ MergeParams P) {
+constexpr int kMrgThreads = 320;  // producer, MMA issuer, two expanding warpgroups
+constexpr int kMrgExpand = kMrgThreads - 64;  // the expanding threads (warps 2..9)
+static_assert(kMrgExpand == 256, "two warpgroups expand the tile");
+
+// Persistent: CTA b takes tiles b, b + gridDim.x, ...  Warp 0 loads the next
+// tile into the other stage while the current one is processed; warp 1
+// issues each tile's r/16 MMAs into one of two TMEM accumulators; warps 2..5
+// (one row of the tile per thread) read the product row back 32 columns at a
+// time, expand the matching base bytes, add, round and write the bf16 row
+// into one of two staging tiles, which one thread stores with TMA while the
+// next tile is expanded.
+__global__ void __launch_bounds__(kMrgThreads, 2) lora_merge_kernel(const __grid_constant__ MergeParams P) {
   extern __shared__ uint8_t mrg_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(mrg_smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t loaded, done, drain;
+  __shared__ uint64_t st_full[2], st_empty[2], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   const MergeSmem L = merge_smem(P.dense, P.r_pad);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int n0 = static_cast<int>(blockIdx.x / P.col_tiles) * kMrgTile;
-  const int k0 = static_cast<int>(blockIdx.x % P.col_tiles) * kMrgTile;
-  const int n = n0 + tid;  // this thread's row
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = P.row_tiles * P.col_tiles;
+  const int slices = P.r_pad / 16;
 
-  if (tid == 0) {
-    mbar_init(&loaded, 1);
-    mbar_init(&done, 1);
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&st_full[b], 1);
+      mbar_init(&st_empty[b], 1 + kMrgExpand);  // the MMAs (commit) and the expanding threads
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kMrgExpand);
+    }
     mbar_init(&drain, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_slot, kMrgTile);
+    tmem_alloc(&tmem_slot, 2 * kMrgTile);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -94,129 +129,175 @@ __global__ void __launch_bounds__(128) lora_merge_kernel(const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_p = &abort_flag;
-  bool issued_load = false, issued_mma = false;
+  int last_load = -1;
+  bool mma_issued = false;
 
-  // this thread's two absmax values (blocks k0/64 and k0/64 + 1 of row n),
-  // loaded first so that their latency overlaps the tile loads
-  float am[2] = {0.f, 0.f};
-  if (!P.dense && n < P.N)
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-      if (k0 + 64 * h < P.K) am[h] = __ldg(P.absmax + static_cast<int64_t>(n) * (P.K / 64) + k0 / 64 + h);
-
-  if (tid == 0) {
-    const int slices = P.r_pad / 16;
-    const uint32_t bytes = static_cast<uint32_t>(L.total - 2 * 16384);
-    mbar_arrive_expect_tx(&loaded, bytes);
-    if (P.dense) {
-      tma_load_2d(smem, &P.map_base, &loaded, k0, n0);
-      tma_load_2d(smem + 16384, &P.map_base, &loaded, k0 + 64, n0);
-    } else {
-      tma_load_2d(smem, &P.map_base, &loaded, k0 / 2, n0);
+  if (warp == 0) {
+    // ---------------------------------------------- TMA loads of each tile
+    if (lane == 0) {
+      const uint32_t bytes = static_cast<uint32_t>(L.stage);
+      int li = 0;
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++li) {
+        const int s = li & 1;
+        if (li >= 2 && !mbar_wait(&st_empty[s], ((li >> 1) - 1) & 1, abort_p, &g_merge_flags,
+                                  kMrgFlagLoad))
+          break;
+        const int n0 = (tile / P.col_tiles) * kMrgTile, k0 = (tile % P.col_tiles) * kMrgTile;
+        uint8_t* st = smem + s * L.stage;
+        mbar_arrive_expect_tx(&st_full[s], bytes);
+        if (P.dense) {
+          tma_load_2d(st, &P.map_base, &st_full[s], k0, n0);
+          tma_load_2d(st + 16384, &P.map_base, &st_full[s], k0 + 64, n0);
+        } else {
+          tma_load_2d(st, &P.map_base, &st_full[s], k0 / 2, n0);
+        }
+        for (int j = 0; j < slices; ++j)
+          tma_load_2d(st + L.b + j * 4096, &P.map_b, &st_full[s], 16 * j, n0);
+        for (int h = 0; h < 2; ++h)
+          tma_load_2d(st + L.a + h * P.r_pad * 128, &P.map_a, &st_full[s], k0 + 64 * h, 0);
+        last_load = li;
+      }
     }
-    for (int j = 0; j < slices; ++j) tma_load_2d(smem + L.b + j * 4096, &P.map_b, &loaded, 16 * j, n0);
-    for (int h = 0; h < 2; ++h)
-      tma_load_2d(smem + L.a + h * P.r_pad * 128, &P.map_a, &loaded, k0 + 64 * h, 0);
-    issued_load = true;
-    if (mbar_wait(&loaded, 0, abort_p, &g_merge_flags, kMrgFlagLoad)) {
-      tc_fence_after();
-      // D[n, k] = sum_j B[n, j] A[j, k]: A operand = B slice j (K-major,
-      // 32B swizzle, 8-row groups 256 B apart); B operand = rows 16j.. of A
-      // (MN-major, 128B swizzle: 64-column atoms r_pad * 128 B apart,
-      // 8-rank groups 1 KiB apart, 16 ranks = 2 KiB per slice)
+  } else if (warp == 1) {
+    // ---------------------------------------------- MMA issuer
+    if (lane == 0) {
+      // D[n, k] = sum_j B[n, j] A[j, k]: A operand = B slice j (K-major, 32B
+      // swizzle, 8-row groups 256 B apart); B operand = rows 16j.. of A
+      // (MN-major, 128B swizzle: 64-column atoms r_pad * 128 B apart, 8-rank
+      // groups 1 KiB apart, 16 ranks = 2 KiB per slice)
       const uint32_t idesc = make_idesc_bf16(kMrgTile, kMrgTile, 0, 1);
-      for (int j = 0; j < slices; ++j) {
-        const uint64_t ad = make_sdesc(smem_u32(smem + L.b + j * 4096), 16, 256, kLayoutSw32);
-        const uint64_t bd =
-            make_sdesc(smem_u32(smem + L.a + j * 2048), P.r_pad * 128, 1024, kLayoutSw128);
-        umma_bf16(tmem, ad, bd, idesc, j > 0 ? 1u : 0u);
+      int li = 0;
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++li) {
+        const int s = li & 1, b = li & 1;
+        if (!mbar_wait(&st_full[s], (li >> 1) & 1, abort_p, &g_merge_flags, kMrgFlagMma)) break;
+        if (li >= 2 && !mbar_wait(&acc_empty[b], ((li >> 1) - 1) & 1, abort_p, &g_merge_flags,
+                                  kMrgFlagMma))
+          break;
+        tc_fence_after();
+        const uint8_t* st = smem + s * L.stage;
+        for (int j = 0; j < slices; ++j) {
+          const uint64_t ad = make_sdesc(smem_u32(st + L.b + j * 4096), 16, 256, kLayoutSw32);
+          const uint64_t bd =
+              make_sdesc(smem_u32(st + L.a + j * 2048), P.r_pad * 128, 1024, kLayoutSw128);
+          umma_bf16(tmem + static_cast<uint32_t>(b * kMrgTile), ad, bd, idesc, j > 0 ? 1u : 0u);
+        }
+        mma_issued = true;
+        umma_commit(&acc_full[b]);
+        umma_commit(&st_empty[s]);  // B and A of this stage are read
       }
-      issued_mma = true;
-      umma_commit(&done);
     }
+  } else {
+    // ---------------------------------------------- expand, add, round, store
+    // warpgroup h (warps 2..5 or 6..9) takes columns 64 h .. 64 h + 63, one
+    // row of the tile per thread, and stores its own 64-column box
+    const int h = (warp - 2) >> 2;
+    const int q4 = warp & 3;           // TMEM lane quarter of this warp
+    const int tid = q4 * 32 + lane;    // this thread's row of the tile
+    const int et = (threadIdx.x - 64) & 127;  // 0 issues the warpgroup's stores
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    // this row's absmax for the warpgroup's block of a tile, loaded one tile ahead
+    auto absmax_of = [&](int tile) -> float {
+      if (P.dense || tile >= n_tiles) return 0.f;
+      const int n = (tile / P.col_tiles) * kMrgTile + tid, k0 = (tile % P.col_tiles) * kMrgTile;
+      if (n >= P.N || k0 + 64 * h >= P.K) return 0.f;
+      return __ldg(P.absmax + static_cast<int64_t>(n) * (P.K / 64) + k0 / 64 + h);
+    };
+    float am_next = absmax_of(blockIdx.x);
+    int li = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++li) {
+      const int s = li & 1, b = li & 1;
+      const float am = am_next;
+      am_next = absmax_of(tile + gridDim.x);
+      const int n0 = (tile / P.col_tiles) * kMrgTile, k0 = (tile % P.col_tiles) * kMrgTile;
+      ok = mbar_wait(&st_full[s], (li >> 1) & 1, abort_p, &g_merge_flags, kMrgFlagMma) &&
+           mbar_wait(&acc_full[b], (li >> 1) & 1, abort_p, &g_merge_flags, kMrgFlagMma);
+      // the staging box written two tiles ago has been read by its store
+      if (et == 0) bulk_wait_group_read<1>();
+      if (!named_sync_and_mrg(1 + h, 128, ok)) break;
+      tc_fence_after();
+      const uint8_t* st = smem + s * L.stage;
+      uint8_t* out_box = smem + L.out + b * 32768 + h * 16384;
+      Nf4Table tab;
+      if (!P.dense) tab = nf4_make_table(P.cb, am);
+#pragma unroll
+      for (int cc = 0; cc < 64; cc += 32) {
+        const int c = 64 * h + cc;
+        uint32_t v[32];
+        tmem_ld32(tmem + static_cast<uint32_t>(b * kMrgTile) + lane_base + static_cast<uint32_t>(c), v);
+        tmem_wait_ld();
+        // the base's 32 bf16 values of this row, columns c .. c + 31
+        uint32_t w[16];
+        if (P.dense) {
+          const uint8_t* row = st + h * 16384 + tid * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = (cc / 8 + q) ^ (tid & 7);
+            const uint4 x = *reinterpret_cast<const uint4*>(row + chunk * 16);
+            w[4 * q] = x.x, w[4 * q + 1] = x.y, w[4 * q + 2] = x.z, w[4 * q + 3] = x.w;
+          }
+        } else {
+          // 64-byte code rows, 64B swizzle: 16-byte chunk q of row i sits at
+          // chunk q ^ ((i >> 1) & 3)
+          const int chunk = (c / 32) ^ ((tid >> 1) & 3);
+          const uint4 x = *reinterpret_cast<const uint4*>(st + tid * 64 + chunk * 16);
+          const uint32_t cw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 d = nf4_dequant8(cw[q], tab);
+            w[4 * q] = d.x, w[4 * q + 1] = d.y, w[4 * q + 2] = d.z, w[4 * q + 3] = d.w;
+          }
+        }
+        uint32_t o[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+          const __nv_bfloat162 m =
+              __floats2bfloat162_rn(__fadd_rn(lo, __fmul_rn(P.s, __uint_as_float(v[2 * e]))),
+                                    __fadd_rn(hi, __fmul_rn(P.s, __uint_as_float(v[2 * e + 1]))));
+          o[e] = *reinterpret_cast<const uint32_t*>(&m);
+        }
+        // row of the 128B-swizzled output box: 16-byte chunk q of row i at
+        // chunk q ^ (i & 7)
+        uint8_t* orow = out_box + tid * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = (cc / 8 + q) ^ (tid & 7);
+          *reinterpret_cast<uint4*>(orow + chunk * 16) =
+              make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[b]);  // the accumulator is read
+      mbar_arrive(&st_empty[s]);   // and this row of the base
+      fence_proxy_async_smem();
+      named_sync(1 + h, 128);
+      if (et == 0) {
+        if (k0 + 64 * h < P.K) tma_store_2d(&P.map_out, out_box, k0 + 64 * h, n0);
+        bulk_commit_group();
+      }
+    }
+    if (et == 0) bulk_wait_group_read<0>();  // the stores have read their staging boxes
   }
-  __syncwarp();
 
-  const bool ok = mbar_wait(&done, 0, abort_p, &g_merge_flags, kMrgFlagMma);
-  if (ok) {
-    tc_fence_after();
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    Nf4Table tab[2];
-    if (!P.dense) {
-      tab[0] = nf4_make_table(P.cb, am[0]);
-      tab[1] = nf4_make_table(P.cb, am[1]);
-    }
-    uint8_t* out_row = smem + L.out;
-#pragma unroll
-    for (int c = 0; c < kMrgTile; c += 32) {
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c), v);
-      tmem_wait_ld();
-      // the base's 32 bf16 values of row n, columns c .. c + 31
-      uint32_t w[16];
-      if (P.dense) {
-        const uint8_t* row = smem + (c / 64) * 16384 + tid * 128;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = ((c % 64) / 8 + q) ^ (tid & 7);
-          const uint4 x = *reinterpret_cast<const uint4*>(row + chunk * 16);
-          w[4 * q] = x.x, w[4 * q + 1] = x.y, w[4 * q + 2] = x.z, w[4 * q + 3] = x.w;
-        }
-      } else {
-        // 64-byte code rows, 64B swizzle: 16-byte chunk q of row i sits at
-        // chunk q ^ ((i >> 1) & 3)
-        const int chunk = (c / 32) ^ ((tid >> 1) & 3);
-        const uint4 x = *reinterpret_cast<const uint4*>(smem + tid * 64 + chunk * 16);
-        const Nf4Table& t = tab[c / 64];
-        const uint32_t cw[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 d = nf4_dequant8(cw[q], t);
-          w[4 * q] = d.x, w[4 * q + 1] = d.y, w[4 * q + 2] = d.z, w[4 * q + 3] = d.w;
-        }
-      }
-      uint32_t o[16];
-#pragma unroll
-      for (int h = 0; h < 16; ++h) {
-        const float lo = __uint_as_float(w[h] << 16), hi = __uint_as_float(w[h] & 0xFFFF0000u);
-        const __nv_bfloat162 m =
-            __floats2bfloat162_rn(__fadd_rn(lo, __fmul_rn(P.s, __uint_as_float(v[2 * h]))),
-                                  __fadd_rn(hi, __fmul_rn(P.s, __uint_as_float(v[2 * h + 1]))));
-        o[h] = *reinterpret_cast<const uint32_t*>(&m);
-      }
-      // row n of the 128B-swizzled output box c / 64: 16-byte chunk q of
-      // row i at chunk q ^ (i & 7)
-      uint8_t* orow = out_row + (c / 64) * 16384 + tid * 128;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int chunk = ((c % 64) / 8 + q) ^ (tid & 7);
-        *reinterpret_cast<uint4*>(orow + chunk * 16) =
-            make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-      }
-    }
-    fence_proxy_async_smem();
-  }
-  __syncthreads();
-  if (tid == 0 && ok && !*abort_p) {
-    for (int h = 0; h < 2; ++h)
-      if (k0 + 64 * h < P.K) tma_store_2d(&P.map_out, smem + L.out + h * 16384, k0 + 64 * h, n0);
-    bulk_commit_group();
-    bulk_wait_group_all();
-  }
-  if (*abort_p && tid == 0) {
+  __syncthreads();  // every thread sees the final abort word
+  if (*abort_p && threadIdx.x == 0) {
     // drain what this CTA started before its shared memory and TMEM go away
     volatile int never = 0;
-    if (issued_load) mbar_wait(&loaded, 0, &never, &g_merge_flags, kMrgFlagDrain);
-    if (issued_mma) {
-      umma_commit(&drain);
-      mbar_wait(&drain, 0, &never, &g_merge_flags, kMrgFlagDrain);
-    }
+    for (int li = (last_load - 1 > 0 ? last_load - 1 : 0); li <= last_load; ++li)
+      if (!mbar_wait(&st_full[li & 1], (li >> 1) & 1, &never, &g_merge_flags, kMrgFlagDrain))
+        break;
+  }
+  if (*abort_p && warp == 1 && lane == 0 && mma_issued) {
+    volatile int never = 0;
+    umma_commit(&drain);
+    mbar_wait(&drain, 0, &never, &g_merge_flags, kMrgFlagDrain);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kMrgTile);
+    tmem_dealloc(tmem, 2 * kMrgTile);
   }
 }
 
@@ -254,11 +335,17 @@ cudaError_t launch_lora_merge(const void* base, const float* absmax, bool dense,
                                    merge_smem(1, 64).total + 1024);
   });
   if (attr_rc != cudaSuccess) return attr_rc;
-  const int64_t grid = ((N + kMrgTile - 1) / kMrgTile) * P.col_tiles;
-  if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  P.row_tiles = static_cast<int>((N + kMrgTile - 1) / kMrgTile);
+  const int64_t tiles = static_cast<int64_t>(P.row_tiles) * P.col_tiles;
+  if (tiles > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int per_sm = std::max(1, std::min(2, (227 * 1024) / smem));  // TMEM: 2 x 256 columns
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, static_cast<int64_t>(per_sm) * sms));
   void* prof = prof_begin(st);
   count_launch();
-  lora_merge_kernel<<<static_cast<unsigned>(grid), 128, smem, st>>>(P);
+  lora_merge_kernel<<<grid, kMrgThreads, smem, st>>>(P);
   const cudaError_t e = cudaGetLastError();
   // algorithmic bytes per element: the base read (0.5625 B NF4, 2 B dense) + 2 B written
   if (prof) prof_end(prof, kProfMerge, (dense ? 4.0 : 2.5625) * static_cast<double>(N) * K, st);

@@ -17,19 +17,21 @@
 // the same Z (q, k, v, gate and up share their input) are stacked along the
 // MMA's N side, so their shared input is read once for all of them.
 //
-// project: a CTA takes 128 tokens x one slice of the contraction.  Warp 0
-// streams 64-column steps of Z and of the stacked adapters through a ring of
-// shared-memory stages (TMA, 128B swizzle), warp 1 issues
-// tcgen05.mma.cta_group::1 (M = 128 tokens, N = stacked ranks, bf16 in,
-// fp32 accumulate in TMEM).  The CS CTAs of a thread-block cluster split the
-// contraction of one token tile; each writes its fp32 partial to its own
-// shared memory and the cluster adds the CS partials through distributed
-// shared memory in slice order, so the sum never depends on timing and no
-// second pass or atomic is needed.
+// project: two passes.  Pass 1 is persistent: an item is one group's 128
+// tokens x one slice of the contraction (slices sized so that every SM gets
+// a few items); warp 0 streams 64-column steps of Z and of the stacked
+// adapters through a ring of shared-memory stages (TMA, 128B swizzle; B read
+// MN-major with a 32B swizzle) without pausing between items, warp 1 issues
+// tcgen05.mma.cta_group::1 (M = 128 tokens, N = stacked ranks) into one of
+// two TMEM accumulators, and four warps write the other accumulator to the
+// item's fp32 partial meanwhile.  Pass 2 adds each token's partials, a warp
+// per token, in an order fixed by the sizes (deterministic, no atomics) and
+// writes the outputs.
 //
-// grad: a CTA takes 128 columns c of Z and every token: D[c, j] =
-// sum_t Z[t, c] V[t, j] with Z read MN-major (the same shared-memory tile a
-// K-major read would use, another descriptor) and V MN-major.  The fp32
+// grad (persistent, same roles): an item is 128 columns c of Z over every
+// token, D[c, j] = sum_t Z[t, c] V[t, j], with Z read MN-major (the same
+// shared-memory tile a K-major read would use, another descriptor) and V
+// MN-major.  The fp32
 // factor V enters as two exact bf16 parts, both multiplied, so every
 // product keeps ~16 significant bits and accumulates in fp32 in token order.
 //
@@ -40,10 +42,9 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
-#include <map>
 #include <mutex>
-#include <tuple>
 #include <utility>
+#include <vector>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -59,30 +60,10 @@ enum : unsigned int {
   kRkFlagDrain = 1u << 11,
 };
 
-constexpr int kRkThreads = 128;   // 4 warps: TMEM lanes 0..127 = tile rows
-constexpr int kRkStages = 4;
 constexpr int kRkMaxGroups = 8;
 constexpr int kRkMaxProbs = 8;
-constexpr int kRkMaxN = 128;      // stacked ranks per item (the partial tile fits the ring)
+constexpr int kRkMaxN = 128;      // stacked ranks per item (two TMEM accumulators fit)
 constexpr int kRkZBytes = 128 * 128;  // 128 rows x 64 bf16
-
-__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t local_addr, uint32_t rank) {
-  float4 v;
-  asm volatile(
-      "{\n\t.reg .b32 ra;\n\t"
-      "mapa.shared::cluster.u32 ra, %4, %5;\n\t"
-      "ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [ra];\n\t}"
-      : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-      : "r"(local_addr), "r"(rank)
-      : "memory");
-  return v;
-}
-
-__device__ __forceinline__ uint32_t cluster_nctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-  return r;
-}
 
 __device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
   const __nv_bfloat16 b = __float2bfloat16_rn(x);
@@ -121,56 +102,71 @@ struct RkProjProb {
 
 struct RkProjGroup {
   CUtensorMap map_z;  // Z bf16 [T, C], box {64, 128}, 128B swizzle
+  float* part;        // fp32 partials [t_tiles * 128][chunks][N] of this group
   int nk;             // 64-column steps of the contraction
+  int chunks;         // slices of the contraction (ceil(nk / L))
   int n_prob;         // problems stacked on this Z (N = n_prob * r_pad)
   int prob[kRkMaxProbs];
-  int cluster0;       // first cluster of this group (t_tiles clusters each)
+  int item0;          // first item of this group (t_tiles * chunks items)
+  int out0;           // first thread of this group in the reduce pass
 };
+
+constexpr int kPrjStagesMax = 8;
+constexpr int kPrjThreads = 192;
 
 struct RkProjParams {
   RkProjGroup g[kRkMaxGroups];
   RkProjProb p[kRkMaxProbs];
-  int n_groups, T, r, r_pad, t_tiles, bwd;
+  int n_groups, n_items, n_out, T, r, r_pad, bwd, max_n, stages, tmem_cols, L;
   float s;
 };
 
-__global__ void __launch_bounds__(kRkThreads, 1) lora_project_tc(const __grid_constant__ RkProjParams P) {
+// Pass 1 (persistent).  An item is one group's 128-token tile x one slice of
+// L contraction steps; CTA b takes items b, b + gridDim.x, ...  Warp 0
+// streams the items' steps through the ring without pausing between items,
+// warp 1 issues each item's MMAs into one of two TMEM accumulators, and
+// warps 2..5 write the other accumulator (the previous item) to the item's
+// fp32 partial in global memory meanwhile.
+__global__ void __launch_bounds__(kPrjThreads, 1) lora_project_tc(const __grid_constant__ RkProjParams P) {
   extern __shared__ uint8_t rk_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(rk_smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t full[kRkStages], empty[kRkStages], done, drain;
+  __shared__ uint64_t full[kPrjStagesMax], empty[kPrjStagesMax], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
-  const uint32_t CS = cluster_nctarank();
-  const uint32_t crank = cluster_ctarank();
-  const int cluster = static_cast<int>(blockIdx.x / CS);
-  int gi = 0;
-  while (gi + 1 < P.n_groups && cluster >= P.g[gi + 1].cluster0) ++gi;
-  const RkProjGroup& G = P.g[gi];
-  const int tt = cluster - G.cluster0;
-  const int t0 = tt * 128;
   const int R = P.r_pad;
-  const int N = G.n_prob * R;
-  const int k_lo = static_cast<int>(static_cast<int64_t>(crank) * G.nk / CS);
-  const int k_hi = static_cast<int>(static_cast<int64_t>(crank + 1) * G.nk / CS);
-  const int nsteps = k_hi - k_lo;
-  const int stage_bytes = kRkZBytes + N * 128;
+  const int S = P.stages;
+  const int stage_bytes = kRkZBytes + P.max_n * 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tcols = tmem_cols_for(N);
+  const int tcols = P.tmem_cols;
+  // item -> (group, token tile, chunk, first step, steps)
+  auto item = [&](int it, int& gi, int& tt, int& ch, int& k_lo, int& nsteps) {
+    gi = 0;
+    while (gi + 1 < P.n_groups && it >= P.g[gi + 1].item0) ++gi;
+    const RkProjGroup& G = P.g[gi];
+    const int local = it - G.item0;
+    tt = local / G.chunks;
+    ch = local % G.chunks;
+    k_lo = ch * P.L;
+    nsteps = min(P.L, G.nk - k_lo);
+  };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kRkStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
     mbar_init(&drain, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_slot, static_cast<uint32_t>(tcols));
+    tmem_alloc(&tmem_slot, static_cast<uint32_t>(2 * tcols));
     tmem_relinquish();
   }
   tc_fence_before();
@@ -181,159 +177,210 @@ __global__ void __launch_bounds__(kRkThreads, 1) lora_project_tc(const __grid_co
   int last_load = -1;
   bool mma_issued = false;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ---------------------------------------------- TMA producer
-    for (int i = 0; i < nsteps; ++i) {
-      const int s = i % kRkStages;
-      if (i >= kRkStages &&
-          !mbar_wait(&empty[s], ((i / kRkStages) - 1) & 1, abort_p, &g_rank_flags,
-                     kRkFlagProducer))
-        break;
-      uint8_t* st = smem + s * stage_bytes;
-      const int kc = (k_lo + i) * 64;
-      mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(stage_bytes));
-      tma_load_2d(st, &G.map_z, &full[s], kc, t0);
-      uint8_t* ad = st + kRkZBytes;
-      if (!P.bwd) {
-        for (int q = 0; q < G.n_prob; ++q)
-          tma_load_2d(ad + q * R * 128, &P.p[G.prob[q]].map_adp, &full[s], kc, 0);
-      } else {
-        for (int a = 0; a < R / 16; ++a)
-          tma_load_2d(ad + a * 64 * 32, &P.p[G.prob[0]].map_adp, &full[s], a * 16, kc);
+    if (lane == 0) {
+      int g = 0, s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
+        int gi, tt, ch, k_lo, nsteps;
+        item(it, gi, tt, ch, k_lo, nsteps);
+        const RkProjGroup& G = P.g[gi];
+        const int N = G.n_prob * R;
+        for (int k = 0; k < nsteps; ++k, ++g) {
+          if (g >= S && !mbar_wait(&empty[s], ph ^ 1u, abort_p, &g_rank_flags, kRkFlagProducer)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * stage_bytes;
+          const int kc = (k_lo + k) * 64;
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRkZBytes + N * 128));
+          tma_load_2d(st, &G.map_z, &full[s], kc, tt * 128);
+          uint8_t* ad = st + kRkZBytes;
+          if (!P.bwd) {
+            for (int q = 0; q < G.n_prob; ++q)
+              tma_load_2d(ad + q * R * 128, &P.p[G.prob[q]].map_adp, &full[s], kc, 0);
+          } else {
+            for (int a = 0; a < R / 16; ++a)
+              tma_load_2d(ad + a * 64 * 32, &P.p[G.prob[0]].map_adp, &full[s], a * 16, kc);
+          }
+          last_load = g;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
       }
-      last_load = i;
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // ---------------------------------------------- MMA issuer
-    const uint32_t idesc = make_idesc_bf16(128, N, 0, P.bwd ? 1 : 0);
-    const uint64_t a0 = make_sdesc(smem_u32(smem), 16, 1024, kLayoutSw128);
-    const uint64_t b0 = P.bwd ? make_sdesc(smem_u32(smem + kRkZBytes), 64 * 32, 256, kLayoutSw32)
-                              : make_sdesc(smem_u32(smem + kRkZBytes), 16, 1024, kLayoutSw128);
-    // per 16-wide K step: 32 bytes along a 128B-swizzled row (K-major), or
-    // 16 rows of 32 bytes (MN-major, 32B swizzle)
-    const uint32_t b_k16 = P.bwd ? (512 >> 4) : (32 >> 4);
-    bool ok = true;
-    for (int i = 0; i < nsteps; ++i) {
-      const int s = i % kRkStages;
-      if (!mbar_wait(&full[s], (i / kRkStages) & 1, abort_p, &g_rank_flags, kRkFlagMma)) {
-        ok = false;
-        break;
+    if (lane == 0) {
+      const uint64_t a0 = make_sdesc(smem_u32(smem), 16, 1024, kLayoutSw128);
+      // adapters: K-major rows (forward A) or MN-major 16-rank atoms 2 KiB
+      // apart (backward B); a 16-wide K step is 32 B along a row, or 16 rows
+      // of 32 B
+      const uint64_t b0 = P.bwd ? make_sdesc(smem_u32(smem + kRkZBytes), 64 * 32, 256, kLayoutSw32)
+                                : make_sdesc(smem_u32(smem + kRkZBytes), 16, 1024, kLayoutSw128);
+      const uint32_t b_k16 = P.bwd ? (512 >> 4) : (32 >> 4);
+      int s = 0, li = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x, ++li) {
+        int gi, tt, ch, k_lo, nsteps;
+        item(it, gi, tt, ch, k_lo, nsteps);
+        const int N = P.g[gi].n_prob * R;
+        const uint32_t idesc = make_idesc_bf16(128, N, 0, P.bwd ? 1 : 0);
+        const int b = li & 1;
+        const uint32_t acc = tmem + static_cast<uint32_t>(b * tcols);
+        if (li >= 2) {  // the epilogue has drained this accumulator's previous item
+          if (!mbar_wait(&acc_empty[b], ((li >> 1) - 1) & 1, abort_p, &g_rank_flags,
+                         kRkFlagMma))
+            break;
+          tc_fence_after();
+        }
+        for (int k = 0; k < nsteps; ++k) {
+          if (!mbar_wait(&full[s], ph, abort_p, &g_rank_flags, kRkFlagMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t so = static_cast<uint64_t>((s * stage_bytes) >> 4);
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16)
+            umma_bf16(acc, a0 + so + k16 * 2, b0 + so + k16 * b_k16, idesc,
+                      (k > 0 || k16 > 0) ? 1u : 0u);
+          mma_issued = true;
+          umma_commit(&empty[s]);
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[b]);
       }
+    }
+  } else {
+    // ---------------------------------------------- epilogue (warps 2..5)
+    const int q4 = warp & 3;         // TMEM lane quarter of this warp
+    const int row = q4 * 32 + lane;  // accumulator row = token row of the tile
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    int li = 0;
+    for (int it = blockIdx.x; it < P.n_items; it += gridDim.x, ++li) {
+      int gi, tt, ch, k_lo, nsteps;
+      item(it, gi, tt, ch, k_lo, nsteps);
+      const RkProjGroup& G = P.g[gi];
+      const int N = G.n_prob * R;
+      const int b = li & 1;
+      if (!mbar_wait(&acc_full[b], (li >> 1) & 1, abort_p, &g_rank_flags, kRkFlagEpilogue))
+        break;
       tc_fence_after();
-      const uint64_t ad = a0 + static_cast<uint64_t>((s * stage_bytes) >> 4);
-      const uint64_t bd = b0 + static_cast<uint64_t>((s * stage_bytes) >> 4);
+      // partials of a token are contiguous over slices: [token][slice][N]
+      float* dst = G.part + (static_cast<int64_t>(tt * 128 + row) * G.chunks + ch) * N;
+      for (int c0 = 0; c0 < N; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + static_cast<uint32_t>(b * tcols) + lane_base + static_cast<uint32_t>(c0), v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int k16 = 0; k16 < 4; ++k16)
-        umma_bf16(tmem, ad + k16 * 2, bd + k16 * b_k16, idesc, (i > 0 || k16 > 0) ? 1u : 0u);
-      mma_issued = true;
-      umma_commit(&empty[s]);
+        for (int j = 0; j < 16; j += 4)
+          __stcg(reinterpret_cast<float4*>(dst + c0 + j),
+                 make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                             __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])));
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[b]);
     }
-    if (ok && nsteps > 0) umma_commit(&done);
   }
-  __syncwarp();
 
-  // ---------------------------------------------- accumulator -> own partial
-  // The ring is free once the last MMA completed: the partial tile (fp32
-  // [128][N + 4]: rows 16-byte aligned, the pad spreads rows over banks)
-  // reuses it.
-  float* part = reinterpret_cast<float*>(smem);
-  const int PS = N + 4;
-  const int row = threadIdx.x;  // TMEM lane = token row of the tile
-  bool have = nsteps > 0;
-  if (have)
-    have = mbar_wait(&done, 0, abort_p, &g_rank_flags, kRkFlagEpilogue);
-  if (have) {
-    tc_fence_after();
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    for (int c0 = 0; c0 < N; c0 += 16) {
-      uint32_t v[16];
-      tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c0), v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(part + row * PS + c0 + j) =
-            make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                        __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-    }
-  } else if (!*abort_p) {
-    for (int c = 0; c < N; c += 4)
-      *reinterpret_cast<float4*>(part + row * PS + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
   __syncthreads();  // every thread sees the final abort word
   if (*abort_p) {
-    // drain what this CTA started before its shared memory and TMEM go away
     volatile int never = 0;
     if (warp == 0 && lane == 0)
-      for (int i = (last_load - kRkStages + 1 > 0 ? last_load - kRkStages + 1 : 0);
-           i <= last_load; ++i)
-        if (!mbar_wait(&full[i % kRkStages], (i / kRkStages) & 1, &never, &g_rank_flags,
-                       kRkFlagDrain))
-          break;
+      for (int g = (last_load - S + 1 > 0 ? last_load - S + 1 : 0); g <= last_load; ++g)
+        if (!mbar_wait(&full[g % S], (g / S) & 1, &never, &g_rank_flags, kRkFlagDrain)) break;
     if (warp == 1 && lane == 0 && mma_issued) {
       umma_commit(&drain);
       mbar_wait(&drain, 0, &never, &g_rank_flags, kRkFlagDrain);
     }
   }
   tc_fence_before();
-  cluster_sync();  // every CTA's partial written (or this cluster gave up)
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, static_cast<uint32_t>(2 * tcols));
+  }
+}
 
-  // ---------------------------------------------- ordered cluster sum
-  // This CTA owns rows [crank * 128 / CS, (crank + 1) * 128 / CS) of the
-  // token tile; each thread takes 4 consecutive columns of one row and adds
-  // the CS partials in slice order.
-  const int r_lo = static_cast<int>(crank * 128 / CS), r_hi = static_cast<int>((crank + 1) * 128 / CS);
-  const int quads = N / 4;
-  const bool failed = *abort_p != 0;
-  for (int e = threadIdx.x; e < (r_hi - r_lo) * quads && !failed; e += kRkThreads) {
-    const int rr = r_lo + e / quads, c = (e % quads) * 4;
-    const int t = t0 + rr;
-    if (t >= P.T) continue;
-    const uint32_t addr = smem_u32(part + rr * PS + c);
-    float4 acc = ld_dsmem_f32x4(addr, 0);
-    for (uint32_t src = 1; src < CS; ++src) {
-      const float4 v = ld_dsmem_f32x4(addr, src);
+// Pass 2: one warp per (group, token); the token's partials are contiguous
+// ([slice][N]).  With Q = N / 4 column quads rounded up to a power of two,
+// lane l takes quad l % Q and adds the slices l / Q, l / Q + 32 / Q, ... in
+// order; a fixed butterfly then adds the 32 / Q lane sums of each quad (the
+// order depends only on the sizes, never on timing).  The lanes holding a
+// quad's total write t, s t and the optional bf16 parts.
+__global__ void __launch_bounds__(256) lora_project_reduce(const __grid_constant__ RkProjParams P) {
+  const int idx = static_cast<int>(blockIdx.x) * 8 + static_cast<int>(threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (idx >= P.n_out) return;
+  int gi = 0;
+  while (gi + 1 < P.n_groups && idx >= P.g[gi + 1].out0) ++gi;
+  const RkProjGroup& G = P.g[gi];
+  const int R = P.r_pad, N = G.n_prob * R, quads = N / 4;
+  const int t = idx - G.out0;
+  int Q = 1;
+  while (Q < quads) Q <<= 1;
+  const int S = 32 / Q;  // lanes per quad
+  const int q4 = lane % Q, sub = lane / Q;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (q4 < quads) {
+    const float4* src =
+        reinterpret_cast<const float4*>(G.part + static_cast<int64_t>(t) * G.chunks * N) + q4;
+    for (int ch = sub; ch < G.chunks; ch += S) {
+      const float4 v = __ldcg(src + static_cast<int64_t>(ch) * quads);
       acc.x += v.x;
       acc.y += v.y;
       acc.z += v.z;
       acc.w += v.w;
     }
-    const int q = c / R, j = c % R;  // 4 columns of problem q, ranks j .. j + 3
-    const RkProjProb& pr = P.p[G.prob[q]];
-    const float a[4] = {acc.x, acc.y, acc.z, acc.w};
-    uint16_t zsv[4], hv[4], lv[4];
+  }
+  for (int m = Q; m < 32; m <<= 1) {
+    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
+    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
+    acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
+    acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
+  }
+  if (sub != 0 || q4 >= quads) return;
+  const int c = q4 * 4;
+  const int q = c / R, j = c % R;  // 4 columns of problem q, ranks j .. j + 3
+  const RkProjProb& pr = P.p[G.prob[q]];
+  const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+  uint16_t zsv[4], hv[4], lv[4];
+#pragma unroll
+  for (int e4 = 0; e4 < 4; ++e4) {
+    const bool real = j + e4 < P.r;
+    if (real) pr.t_out[static_cast<int64_t>(t) * P.r + j + e4] = a[e4];
+    zsv[e4] = (real && !pr.zero_zs) ? bf16_bits_rn(__fmul_rn(P.s, a[e4])) : 0;
+    split_bf16(real ? a[e4] : 0.0f, hv[e4], lv[e4]);
+  }
+  const int64_t o = static_cast<int64_t>(t) * R + j;
+  *reinterpret_cast<uint2*>(pr.zs + o) =
+      make_uint2(zsv[0] | (uint32_t(zsv[1]) << 16), zsv[2] | (uint32_t(zsv[3]) << 16));
+  if (pr.hi) {
+    *reinterpret_cast<uint2*>(pr.hi + o) =
+        make_uint2(hv[0] | (uint32_t(hv[1]) << 16), hv[2] | (uint32_t(hv[3]) << 16));
+    *reinterpret_cast<uint2*>(pr.lo + o) =
+        make_uint2(lv[0] | (uint32_t(lv[1]) << 16), lv[2] | (uint32_t(lv[3]) << 16));
+  }
+  if (pr.split_src) {  // the forward's t of the same token, as two bf16 parts
 #pragma unroll
     for (int e4 = 0; e4 < 4; ++e4) {
-      const bool real = j + e4 < P.r;
-      if (real) pr.t_out[static_cast<int64_t>(t) * P.r + j + e4] = a[e4];
-      zsv[e4] = (real && !pr.zero_zs) ? bf16_bits_rn(__fmul_rn(P.s, a[e4])) : 0;
-      split_bf16(real ? a[e4] : 0.0f, hv[e4], lv[e4]);
+      const float x = (j + e4 < P.r) ? pr.split_src[static_cast<int64_t>(t) * P.r + j + e4] : 0.f;
+      split_bf16(x, hv[e4], lv[e4]);
     }
-    const int64_t o = static_cast<int64_t>(t) * R + j;
-    *reinterpret_cast<uint2*>(pr.zs + o) =
-        make_uint2(zsv[0] | (uint32_t(zsv[1]) << 16), zsv[2] | (uint32_t(zsv[3]) << 16));
-    if (pr.hi) {
-      *reinterpret_cast<uint2*>(pr.hi + o) =
-          make_uint2(hv[0] | (uint32_t(hv[1]) << 16), hv[2] | (uint32_t(hv[3]) << 16));
-      *reinterpret_cast<uint2*>(pr.lo + o) =
-          make_uint2(lv[0] | (uint32_t(lv[1]) << 16), lv[2] | (uint32_t(lv[3]) << 16));
-    }
-    if (pr.split_src) {  // the forward's t of the same rows, as two bf16 parts
-#pragma unroll
-      for (int e4 = 0; e4 < 4; ++e4) {
-        const float x = (j + e4 < P.r) ? pr.split_src[static_cast<int64_t>(t) * P.r + j + e4] : 0.f;
-        split_bf16(x, hv[e4], lv[e4]);
-      }
-      *reinterpret_cast<uint2*>(pr.split_hi + o) =
-          make_uint2(hv[0] | (uint32_t(hv[1]) << 16), hv[2] | (uint32_t(hv[3]) << 16));
-      *reinterpret_cast<uint2*>(pr.split_lo + o) =
-          make_uint2(lv[0] | (uint32_t(lv[1]) << 16), lv[2] | (uint32_t(lv[3]) << 16));
-    }
-  }
-  tc_fence_before();
-  cluster_sync();  // no CTA leaves while a peer may still read its partial
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, static_cast<uint32_t>(tcols));
+    *reinterpret_cast<uint2*>(pr.split_hi + o) =
+        make_uint2(hv[0] | (uint32_t(hv[1]) << 16), hv[2] | (uint32_t(hv[3]) << 16));
+    *reinterpret_cast<uint2*>(pr.split_lo + o) =
+        make_uint2(lv[0] | (uint32_t(lv[1]) << 16), lv[2] | (uint32_t(lv[3]) << 16));
   }
 }
 
@@ -357,42 +404,59 @@ struct RkGradGroup {
 struct RkGradParams {
   RkGradGroup g[2 * kRkMaxGroups];
   RkGradProb p[2 * kRkMaxProbs];
-  int n_groups, T, r, r_pad, nk;
+  int n_groups, n_items, T, r, r_pad, nk, max_n, stages, tmem_cols;
   float s;
 };
 
-__global__ void __launch_bounds__(kRkThreads, 1) lora_grad_tc(const __grid_constant__ RkGradParams P) {
+constexpr int kGrdStagesMax = 8;
+constexpr int kGrdMT = 2;                   // 128-row M tiles per item
+constexpr int kGrdCols = 128 * kGrdMT;      // columns of Z per item
+constexpr int kGrdZBytes = kGrdMT * 16384;  // Z per step: kGrdCols x 64 tokens
+
+// Persistent: CTA b takes items b, b + gridDim.x, ... (an item = one group's
+// 128-column tile over every token).  Warp 0 streams the items' steps
+// through the ring without pausing between items, warp 1 issues each item's
+// MMAs into one of two TMEM accumulators, and warps 2..5 drain the other
+// accumulator (the previous item) meanwhile, so loads stay in flight across
+// item boundaries.
+constexpr int kGrdThreads = 192;
+
+__global__ void __launch_bounds__(kGrdThreads, 1) lora_grad_tc(const __grid_constant__ RkGradParams P) {
   extern __shared__ uint8_t rk_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(rk_smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t full[kRkStages], empty[kRkStages], done, drain;
+  __shared__ uint64_t full[kGrdStagesMax], empty[kGrdStagesMax], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
-  int gi = 0;
-  while (gi + 1 < P.n_groups && static_cast<int>(blockIdx.x) >= P.g[gi + 1].cta0) ++gi;
-  const RkGradGroup& G = P.g[gi];
-  const int c0 = (static_cast<int>(blockIdx.x) - G.cta0) * 128;
   const int R = P.r_pad;
-  const int N = G.n_prob * R;
-  const int vbytes = N * 64 * 2;                 // one V part of a step: N ranks x 64 tokens
-  const int stage_bytes = kRkZBytes + 2 * vbytes;
+  const int S = P.stages;
+  const int stage_bytes = kGrdZBytes + 2 * P.max_n * 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tcols = tmem_cols_for(N);
+  const int tcols = P.tmem_cols;  // per accumulator; 2 x kGrdMT of them
   const int nsteps = P.nk;
+  // item -> (group, first column)
+  auto item_of = [&](int it, int& gi, int& c0) {
+    gi = 0;
+    while (gi + 1 < P.n_groups && it >= P.g[gi + 1].cta0) ++gi;
+    c0 = (it - P.g[gi].cta0) * kGrdCols;
+  };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kRkStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
     mbar_init(&drain, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_slot, static_cast<uint32_t>(tcols));
+    tmem_alloc(&tmem_slot, static_cast<uint32_t>(2 * kGrdMT * tcols));
     tmem_relinquish();
   }
   tc_fence_before();
@@ -403,95 +467,161 @@ __global__ void __launch_bounds__(kRkThreads, 1) lora_grad_tc(const __grid_const
   int last_load = -1;
   bool mma_issued = false;
 
-  if (warp == 0 && lane == 0) {
-    for (int i = 0; i < nsteps; ++i) {
-      const int s = i % kRkStages;
-      if (i >= kRkStages &&
-          !mbar_wait(&empty[s], ((i / kRkStages) - 1) & 1, abort_p, &g_rank_flags,
-                     kRkFlagProducer))
+  if (warp == 0) {
+    // ---------------------------------------------- TMA producer
+    if (lane == 0) {
+      int g = 0, s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
+        int gi, c0;
+        item_of(it, gi, c0);
+        const RkGradGroup& G = P.g[gi];
+        const int vbytes = G.n_prob * R * 128;
+        for (int i = 0; i < nsteps; ++i, ++g) {
+          if (g >= S && !mbar_wait(&empty[s], ph ^ 1u, abort_p, &g_rank_flags, kRkFlagProducer)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * stage_bytes;
+          const int tk = i * 64;
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kGrdZBytes + 2 * vbytes));
+          // Z: per 128-column M tile two 64-column atoms (rows = tokens), the
+          // MN-major operand layout; the tiles of an item are adjacent columns
+          for (int a = 0; a < 2 * kGrdMT; ++a)
+            tma_load_2d(st + a * 8192, &G.map_z, &full[s], c0 + 64 * a, tk);
+          uint8_t* vh = st + kGrdZBytes;
+          for (int q = 0; q < G.n_prob; ++q) {
+            const RkGradProb& pr = P.p[G.prob[q]];
+            for (int a = 0; a < R / 16; ++a) {
+              const int atom = q * (R / 16) + a;
+              tma_load_2d(vh + atom * 2048, &pr.map_hi, &full[s], a * 16, tk);
+              tma_load_2d(vh + vbytes + atom * 2048, &pr.map_lo, &full[s], a * 16, tk);
+            }
+          }
+          last_load = g;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------- MMA issuer
+    if (lane == 0) {
+      // A = Z MN-major: two 64-column atoms 8 KiB apart (LBO), 8-token groups
+      // 1 KiB apart (SBO), 16 tokens = 2 KiB per K step.  B = V MN-major, 32B
+      // swizzle: 16-rank atoms 2 KiB apart (LBO), 8-token groups 256 B apart
+      // (SBO), 16 tokens = 512 B per K step; the lo parts follow the hi parts.
+      const uint64_t a0 = make_sdesc(smem_u32(smem), 64 * 128, 1024, kLayoutSw128);
+      const uint64_t b0 = make_sdesc(smem_u32(smem + kGrdZBytes), 2048, 256, kLayoutSw32);
+      int s = 0, li = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x, ++li) {
+        int gi, c0;
+        item_of(it, gi, c0);
+        const int N = P.g[gi].n_prob * R;
+        const uint32_t idesc = make_idesc_bf16(128, N, 1, 1);
+        const uint32_t lo_off = static_cast<uint32_t>(N * 128) >> 4;  // V lo after V hi
+        const int b = li & 1;
+        const uint32_t acc = tmem + static_cast<uint32_t>(b * kGrdMT * tcols);
+        if (li >= 2) {  // the epilogue has drained these accumulators' previous item
+          if (!mbar_wait(&acc_empty[b], ((li >> 1) - 1) & 1, abort_p, &g_rank_flags,
+                         kRkFlagMma))
+            break;
+          tc_fence_after();
+        }
+        for (int i = 0; i < nsteps; ++i) {
+          if (!mbar_wait(&full[s], ph, abort_p, &g_rank_flags, kRkFlagMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t so = static_cast<uint64_t>((s * stage_bytes) >> 4);
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16) {
+            const uint64_t bd = b0 + so + k16 * (512 >> 4);
+#pragma unroll
+            for (int m = 0; m < kGrdMT; ++m) {
+              const uint64_t ad = a0 + so + (m * 16384 >> 4) + k16 * (2048 >> 4);
+              const uint32_t d = acc + static_cast<uint32_t>(m * tcols);
+              umma_bf16(d, ad, bd, idesc, (i > 0 || k16 > 0) ? 1u : 0u);
+              umma_bf16(d, ad, bd + lo_off, idesc, 1u);
+            }
+          }
+          mma_issued = true;
+          umma_commit(&empty[s]);
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[b]);
+      }
+    }
+  } else {
+    // ---------------------------------------------- epilogue (warps 2..5)
+    const int q4 = warp & 3;                      // TMEM lane quarter of this warp
+    const int row = q4 * 32 + lane;               // accumulator row = column c0 + row
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    int li = 0;
+    for (int it = blockIdx.x; it < P.n_items; it += gridDim.x, ++li) {
+      int gi, c0;
+      item_of(it, gi, c0);
+      const RkGradGroup& G = P.g[gi];
+      const int b = li & 1;
+      if (!mbar_wait(&acc_full[b], (li >> 1) & 1, abort_p, &g_rank_flags, kRkFlagEpilogue))
         break;
-      uint8_t* st = smem + s * stage_bytes;
-      const int tk = i * 64;
-      mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(stage_bytes));
-      // Z: two 64-column atoms (rows = tokens), the MN-major operand layout
-      tma_load_2d(st, &G.map_z, &full[s], c0, tk);
-      tma_load_2d(st + kRkZBytes / 2, &G.map_z, &full[s], c0 + 64, tk);
-      uint8_t* vh = st + kRkZBytes;
+      tc_fence_after();
+      for (int m = 0; m < kGrdMT; ++m) {
+      const int c = c0 + m * 128 + row;
+      const uint32_t accm = tmem + static_cast<uint32_t>((b * kGrdMT + m) * tcols) + lane_base;
       for (int q = 0; q < G.n_prob; ++q) {
         const RkGradProb& pr = P.p[G.prob[q]];
-        for (int a = 0; a < R / 16; ++a) {
-          const int atom = q * (R / 16) + a;
-          tma_load_2d(vh + atom * 2048, &pr.map_hi, &full[s], a * 16, tk);
-          tma_load_2d(vh + vbytes + atom * 2048, &pr.map_lo, &full[s], a * 16, tk);
+        for (int jc = 0; jc < R; jc += 16) {
+          uint32_t v[16];
+          tmem_ld16(accm + static_cast<uint32_t>(q * R + jc), v);
+          tmem_wait_ld();
+          if (c >= G.C) continue;
+          if (pr.c_major) {  // dB [C, r]: this thread's row, 16 consecutive ranks
+            float* o = pr.out + static_cast<int64_t>(c) * P.r + jc;
+            if (P.r - jc >= 16 && (P.r % 4) == 0) {
+#pragma unroll
+              for (int j = 0; j < 16; j += 4)
+                *reinterpret_cast<float4*>(o + j) =
+                    make_float4(__fmul_rn(P.s, __uint_as_float(v[j])),
+                                __fmul_rn(P.s, __uint_as_float(v[j + 1])),
+                                __fmul_rn(P.s, __uint_as_float(v[j + 2])),
+                                __fmul_rn(P.s, __uint_as_float(v[j + 3])));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (jc + j < P.r) o[j] = __fmul_rn(P.s, __uint_as_float(v[j]));
+            }
+          } else {  // dA [r, C]: one column, coalesced across the warp
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (jc + j < P.r)
+                pr.out[static_cast<int64_t>(jc + j) * G.C + c] =
+                    __fmul_rn(P.s, __uint_as_float(v[j]));
+          }
         }
       }
-      last_load = i;
-    }
-  } else if (warp == 1 && lane == 0) {
-    const uint32_t idesc = make_idesc_bf16(128, N, 1, 1);
-    // A = Z MN-major: two 64-column atoms 8 KiB apart (LBO), 8-token groups
-    // 1 KiB apart (SBO), 16 tokens = 2 KiB per K step.  B = V MN-major, 32B
-    // swizzle: 16-rank atoms 2 KiB apart (LBO), 8-token groups 256 B apart
-    // (SBO), 16 tokens = 512 B per K step.
-    const uint64_t a0 = make_sdesc(smem_u32(smem), 64 * 128, 1024, kLayoutSw128);
-    const uint64_t bh0 = make_sdesc(smem_u32(smem + kRkZBytes), 2048, 256, kLayoutSw32);
-    const uint64_t bl0 = make_sdesc(smem_u32(smem + kRkZBytes + vbytes), 2048, 256, kLayoutSw32);
-    bool ok = true;
-    for (int i = 0; i < nsteps; ++i) {
-      const int s = i % kRkStages;
-      if (!mbar_wait(&full[s], (i / kRkStages) & 1, abort_p, &g_rank_flags, kRkFlagMma)) {
-        ok = false;
-        break;
       }
-      tc_fence_after();
-      const uint64_t so = static_cast<uint64_t>((s * stage_bytes) >> 4);
-#pragma unroll
-      for (int k16 = 0; k16 < 4; ++k16) {
-        umma_bf16(tmem, a0 + so + k16 * (2048 >> 4), bh0 + so + k16 * (512 >> 4), idesc,
-                  (i > 0 || k16 > 0) ? 1u : 0u);
-        umma_bf16(tmem, a0 + so + k16 * (2048 >> 4), bl0 + so + k16 * (512 >> 4), idesc, 1u);
-      }
-      mma_issued = true;
-      umma_commit(&empty[s]);
+      tc_fence_before();
+      mbar_arrive(&acc_empty[b]);
     }
-    if (ok && nsteps > 0) umma_commit(&done);
   }
-  __syncwarp();
 
-  // ---------------------------------------------- epilogue: row c of D
-  const int c = c0 + static_cast<int>(threadIdx.x);
-  bool ok = nsteps > 0 && mbar_wait(&done, 0, abort_p, &g_rank_flags, kRkFlagEpilogue);
-  if (ok) {
-    tc_fence_after();
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    for (int q = 0; q < G.n_prob; ++q) {
-      const RkGradProb& pr = P.p[G.prob[q]];
-      for (int jc = 0; jc < R; jc += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + lane_base + static_cast<uint32_t>(q * R + jc), v);
-        tmem_wait_ld();
-        if (c >= G.C) continue;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          if (jc + j >= P.r) break;
-          const float val = __fmul_rn(P.s, __uint_as_float(v[j]));
-          if (pr.c_major)
-            pr.out[static_cast<int64_t>(c) * P.r + jc + j] = val;
-          else
-            pr.out[static_cast<int64_t>(jc + j) * G.C + c] = val;
-        }
-      }
-    }
-  }
   __syncthreads();  // every thread sees the final abort word
   if (*abort_p) {
     volatile int never = 0;
     if (warp == 0 && lane == 0)
-      for (int i = (last_load - kRkStages + 1 > 0 ? last_load - kRkStages + 1 : 0);
-           i <= last_load; ++i)
-        if (!mbar_wait(&full[i % kRkStages], (i / kRkStages) & 1, &never, &g_rank_flags,
-                       kRkFlagDrain))
-          break;
+      for (int g = (last_load - S + 1 > 0 ? last_load - S + 1 : 0); g <= last_load; ++g)
+        if (!mbar_wait(&full[g % S], (g / S) & 1, &never, &g_rank_flags, kRkFlagDrain)) break;
     if (warp == 1 && lane == 0 && mma_issued) {
       umma_commit(&drain);
       mbar_wait(&drain, 0, &never, &g_rank_flags, kRkFlagDrain);
@@ -501,16 +631,16 @@ __global__ void __launch_bounds__(kRkThreads, 1) lora_grad_tc(const __grid_const
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, static_cast<uint32_t>(tcols));
+    tmem_dealloc(tmem, static_cast<uint32_t>(2 * kGrdMT * tcols));
   }
 }
 
 // ---------------------------------------------------------------- host side
 
 static int project_stage_bytes(int N) { return kRkZBytes + N * 128; }
-static int grad_stage_bytes(int N) { return kRkZBytes + 2 * N * 128; }
+static int grad_stage_bytes(int N) { return kGrdZBytes + 2 * N * 128; }
 
-constexpr int kRkMaxSmem = kRkStages * (kRkZBytes + 2 * kRkMaxN * 128) + 1024;
+constexpr int kRkMaxSmem = 200 * 1024 + 1024;
 
 static cudaError_t rk_configure() {
   static cudaError_t rc = cudaSuccess;
@@ -518,9 +648,6 @@ static cudaError_t rk_configure() {
   std::call_once(once, [] {
     rc = cudaFuncSetAttribute(lora_project_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               kRkMaxSmem);
-    if (rc == cudaSuccess)
-      rc = cudaFuncSetAttribute(lora_project_tc, cudaFuncAttributeNonPortableClusterSizeAllowed,
-                                1);
     if (rc == cudaSuccess)
       rc = cudaFuncSetAttribute(lora_grad_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 kRkMaxSmem);
@@ -555,16 +682,74 @@ static int stack_groups(int n, int r_pad, GetZ getz, int (*members)[kRkMaxProbs]
   return ng;
 }
 
-size_t project_workspace_bytes(const ProjectDesc*, int, int64_t, int) { return 0; }
+// The launch plan of a projection group: the stacked groups, the slice
+// length L (steps) and each group's partial offset; fills P (maps aside) and
+// returns the partial bytes (0 for invalid sizes).
+struct PrjPlan {
+  int ng, L, t_tiles, max_n;
+  int members[kRkMaxGroups][kRkMaxProbs], counts[kRkMaxGroups];
+  int64_t part_off[kRkMaxGroups];  // bytes
+  int64_t part_bytes;
+};
+
+static bool prj_plan(const ProjectDesc* d, int n, int64_t T, int r, PrjPlan* pl) {
+  if (n < 1 || n > kRkMaxProbs || T < 1 || r < 1) return false;
+  const int R = (r + 15) / 16 * 16;
+  const bool bwd = !d[0].r_major;
+  if (bwd) {  // backward problems read distinct dY: one problem per group
+    pl->ng = n;
+    for (int q = 0; q < n; ++q) {
+      pl->members[q][0] = q;
+      pl->counts[q] = 1;
+    }
+  } else {
+    pl->ng = stack_groups(n, R, [&](int q) { return std::make_pair(d[q].Z, d[q].C); },
+                          pl->members, pl->counts);
+  }
+  pl->t_tiles = static_cast<int>((T + 127) / 128);
+  int64_t total_steps = 0;
+  pl->max_n = 0;
+  for (int g = 0; g < pl->ng; ++g) {
+    total_steps += static_cast<int64_t>(pl->t_tiles) * (d[pl->members[g][0]].C / 64);
+    pl->max_n = std::max(pl->max_n, pl->counts[g] * R);
+  }
+  // slices of about total / (4 x SMs) steps: every SM gets a few items and
+  // long contractions are cut into many
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  else
+    cudaGetLastError();
+  pl->L = static_cast<int>(std::max<int64_t>(4, (total_steps + 4 * sms - 1) / (4 * sms)));
+  int64_t off = 0;
+  for (int g = 0; g < pl->ng; ++g) {
+    const int64_t nk = d[pl->members[g][0]].C / 64;
+    const int64_t chunks = (nk + pl->L - 1) / pl->L;
+    pl->part_off[g] = off;
+    off += static_cast<int64_t>(round_up(
+        static_cast<size_t>(pl->t_tiles * chunks * 128 * pl->counts[g] * R) * 4, 256));
+  }
+  pl->part_bytes = off;
+  return true;
+}
+
+size_t project_workspace_bytes(const ProjectDesc* d, int n, int64_t T, int r) {
+  PrjPlan pl;
+  if (!prj_plan(d, n, T, r, &pl)) return 0;
+  return static_cast<size_t>(pl.part_bytes);
+}
 
 cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, int r, float s,
-                                      void*, cudaStream_t st) {
+                                      void* ws, cudaStream_t st) {
   if (n < 1 || n > kRkMaxProbs) return cudaErrorInvalidValue;
   cudaError_t e = rk_configure();
   if (e != cudaSuccess) return e;
   static RkProjParams P;  // large: built on the host, copied into the launch
+  static PrjPlan pl;
   static std::mutex mu;
   std::lock_guard<std::mutex> lk(mu);
+  if (!prj_plan(d, n, T, r, &pl)) return cudaErrorInvalidValue;
+  if (pl.part_bytes > 0 && !ws) return cudaErrorInvalidValue;
   memset(&P, 0, sizeof P);
   const bool bwd = !d[0].r_major;
   P.T = static_cast<int>(T);
@@ -572,7 +757,7 @@ cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, in
   P.r_pad = (r + 15) / 16 * 16;
   P.s = s;
   P.bwd = bwd ? 1 : 0;
-  P.t_tiles = static_cast<int>((T + 127) / 128);
+  P.L = pl.L;
   const int R = P.r_pad;
   for (int q = 0; q < n; ++q) {
     RkProjProb& p = P.p[q];
@@ -593,86 +778,46 @@ cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, in
     p.split_lo = static_cast<uint16_t*>(d[q].split_lo);
     p.zero_zs = d[q].zero_zs ? 1 : 0;
   }
-  // backward problems read distinct dY: one problem per group there
-  int members[kRkMaxGroups][kRkMaxProbs], counts[kRkMaxGroups];
-  int ng;
-  if (bwd) {
-    ng = n;
-    for (int q = 0; q < n; ++q) {
-      members[q][0] = q;
-      counts[q] = 1;
-    }
-  } else {
-    ng = stack_groups(n, R, [&](int q) { return std::make_pair(d[q].Z, d[q].C); }, members,
-                      counts);
-  }
-  // cluster size: the widest (16, else 8) whose grid still fits about two
-  // waves; every cluster splits one token tile's contraction
-  int max_n = 0, cl = 0;
-  for (int g = 0; g < ng; ++g) {
+  int items = 0, outs = 0;
+  double bytes = 0;
+  for (int g = 0; g < pl.ng; ++g) {
     RkProjGroup& G = P.g[g];
-    const int q0 = members[g][0];
+    const int q0 = pl.members[g][0];
     if (!encode_tma_2d(&G.map_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d[q0].Z, d[q0].C, T,
                        d[q0].C * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
+    G.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.part_off[g]);
     G.nk = static_cast<int>(d[q0].C / 64);
-    G.n_prob = counts[g];
-    for (int k = 0; k < counts[g]; ++k) G.prob[k] = members[g][k];
-    G.cluster0 = cl;
-    cl += P.t_tiles;
-    max_n = std::max(max_n, counts[g] * R);
+    G.chunks = (G.nk + pl.L - 1) / pl.L;
+    G.n_prob = pl.counts[g];
+    for (int k = 0; k < pl.counts[g]; ++k) G.prob[k] = pl.members[g][k];
+    G.item0 = items;
+    items += pl.t_tiles * G.chunks;
+    G.out0 = outs;
+    outs += static_cast<int>(T);  // one warp per token
+    bytes += 2.0 * T * d[q0].C;
   }
-  P.n_groups = ng;
-  int nk_max = 0;
-  for (int g = 0; g < ng; ++g) nk_max = std::max(nk_max, P.g[g].nk);
-  const int smem = kRkStages * project_stage_bytes(max_n) + 1024;
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kRkThreads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  // cluster size: the one with the smallest estimated time, counting the
-  // rounds of clusters the GPU can hold at once and the longest slice
-  // (decided once per launch shape)
-  static std::map<std::tuple<int, int, int, int>, int> cs_cache;
-  int dev = 0;
+  P.n_groups = pl.ng;
+  P.n_items = items;
+  P.n_out = outs;
+  P.max_n = pl.max_n;
+  P.tmem_cols = tmem_cols_for(pl.max_n);
+  const int stage = project_stage_bytes(pl.max_n);
+  P.stages = std::max(2, std::min(kPrjStagesMax, (190 * 1024) / stage));
+  const int smem = P.stages * stage + 1024;
+  int dev = 0, sms = 148;
   cudaGetDevice(&dev);
-  const auto key = std::make_tuple(dev, cl, nk_max, smem);
-  int CS = 0;
-  int64_t best = 0;
-  const auto hit = cs_cache.find(key);
-  if (hit != cs_cache.end()) CS = hit->second;
-  for (int cs : {16, 8, 4}) {
-    if (hit != cs_cache.end()) break;
-    attr[0].val.clusterDim.x = cs;
-    cfg.gridDim = dim3(static_cast<unsigned>(cl * cs));
-    int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, lora_project_tc, &cfg) != cudaSuccess ||
-        active < 1) {
-      cudaGetLastError();  // a size the device cannot co-schedule: not a launch error
-      continue;
-    }
-    const int64_t rounds = (cl + active - 1) / active;
-    const int64_t cost = rounds * ((nk_max + cs - 1) / cs + 6);
-    if (CS == 0 || cost < best) {
-      CS = cs;
-      best = cost;
-    }
-  }
-  if (CS == 0) return cudaErrorInvalidConfiguration;
-  cs_cache[key] = CS;
-  attr[0].val.clusterDim.x = CS;
-  cfg.gridDim = dim3(static_cast<unsigned>(cl * CS));
-  double bytes = 0;
-  for (int g = 0; g < ng; ++g) bytes += 2.0 * T * d[members[g][0]].C;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = std::min(items, sms);
   void* prof = prof_begin(st);
   count_launch();
-  e = cudaLaunchKernelEx(&cfg, lora_project_tc, P);
+  lora_project_tc<<<grid, kPrjThreads, smem, st>>>(P);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    count_launch();
+    lora_project_reduce<<<(outs + 7) / 8, 256, 0, st>>>(P);
+    e = cudaGetLastError();
+  }
   prof_end(prof, kProfProject, bytes, st);
   return e;
 }
@@ -721,16 +866,26 @@ cudaError_t launch_lora_grad_group(const GradDesc* d, int n, int64_t T, int r, f
     G.C = d[q0].C;
     G.n_prob = counts[g];
     for (int k = 0; k < counts[g]; ++k) G.prob[k] = members[g][k];
-    G.cta0 = ctas;
-    ctas += static_cast<int>((d[q0].C + 127) / 128);
+    G.cta0 = ctas;  // first item of this group
+    ctas += static_cast<int>((d[q0].C + kGrdCols - 1) / kGrdCols);
     max_n = std::max(max_n, counts[g] * R);
     bytes += 2.0 * T * d[q0].C;
   }
   P.n_groups = ng;
-  const int smem = kRkStages * grad_stage_bytes(max_n) + 1024;
+  P.n_items = ctas;
+  P.max_n = max_n;
+  P.tmem_cols = tmem_cols_for(max_n);
+  // ring: as many stages as fit about 190 KiB (one CTA per SM)
+  const int stage = grad_stage_bytes(max_n);
+  P.stages = std::max(2, std::min(kGrdStagesMax, (190 * 1024) / stage));
+  const int smem = P.stages * stage + 1024;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = std::min(ctas, sms);
   void* prof = prof_begin(st);
   count_launch();
-  lora_grad_tc<<<ctas, kRkThreads, smem, st>>>(P);
+  lora_grad_tc<<<grid, kGrdThreads, smem, st>>>(P);
   e = cudaGetLastError();
   prof_end(prof, kProfGrad, bytes, st);
   return e;

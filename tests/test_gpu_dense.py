@@ -120,7 +120,10 @@ def _ulp_diff(a_bits, b_bits):
 
 
 @pytest.mark.parametrize("N,K,r,alpha", [(64, 64, 8, 16.0), (192, 320, 16, 32.0),
-                                         (512, 1152, 64, 128.0), (128, 640, 24, 7.0)])
+                                         (512, 1152, 64, 128.0), (128, 640, 24, 7.0),
+                                         # more 128 x 128 tiles than the persistent
+                                         # grid has CTAs: each CTA takes several
+                                         (4096, 4160, 16, 32.0)])
 @pytest.mark.parametrize("base", ["nf4", "bf16"])
 def test_merge_vs_oracle(orc, N, K, r, alpha, base):
     case = synth.linear_case(4000 + N + K + r, 1, N, K, r=r, alpha=alpha, b_std=0.05)
