@@ -178,38 +178,42 @@ __global__ void __launch_bounds__(kPrjThreads, 1) lora_project_tc(const __grid_c
   bool mma_issued = false;
 
   if (warp == 0) {
-    // ---------------------------------------------- TMA producer
-    if (lane == 0) {
-      int g = 0, s = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
-        int gi, tt, ch, k_lo, nsteps;
-        item(it, gi, tt, ch, k_lo, nsteps);
-        const RkProjGroup& G = P.g[gi];
-        const int N = G.n_prob * R;
-        for (int k = 0; k < nsteps; ++k, ++g) {
-          if (g >= S && !mbar_wait(&empty[s], ph ^ 1u, abort_p, &g_rank_flags, kRkFlagProducer)) {
-            ok = false;
-            break;
-          }
-          uint8_t* st = smem + s * stage_bytes;
-          const int kc = (k_lo + k) * 64;
+    // ---------------------------------------------- TMA producer (the whole
+    // warp: lane 0 waits for the stage and arms its barrier, then the lanes
+    // issue the step's boxes side by side)
+    int g = 0, s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
+      int gi, tt, ch, k_lo, nsteps;
+      item(it, gi, tt, ch, k_lo, nsteps);
+      const RkProjGroup& G = P.g[gi];
+      const int N = G.n_prob * R;
+      const int n_adp = P.bwd ? R / 16 : G.n_prob;  // adapter boxes per step
+      for (int k = 0; k < nsteps; ++k, ++g) {
+        if (lane == 0 && g >= S)
+          ok = mbar_wait(&empty[s], ph ^ 1u, abort_p, &g_rank_flags, kRkFlagProducer);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        uint8_t* st = smem + s * stage_bytes;
+        const int kc = (k_lo + k) * 64;
+        if (lane == 0)
           mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRkZBytes + N * 128));
+        __syncwarp();
+        uint8_t* ad = st + kRkZBytes;
+        if (lane == 0) {
           tma_load_2d(st, &G.map_z, &full[s], kc, tt * 128);
-          uint8_t* ad = st + kRkZBytes;
-          if (!P.bwd) {
-            for (int q = 0; q < G.n_prob; ++q)
-              tma_load_2d(ad + q * R * 128, &P.p[G.prob[q]].map_adp, &full[s], kc, 0);
-          } else {
-            for (int a = 0; a < R / 16; ++a)
-              tma_load_2d(ad + a * 64 * 32, &P.p[G.prob[0]].map_adp, &full[s], a * 16, kc);
-          }
-          last_load = g;
-          if (++s == S) {
-            s = 0;
-            ph ^= 1u;
-          }
+        } else if (lane <= n_adp) {
+          const int a = lane - 1;
+          if (!P.bwd)
+            tma_load_2d(ad + a * R * 128, &P.p[G.prob[a]].map_adp, &full[s], kc, 0);
+          else
+            tma_load_2d(ad + a * 64 * 32, &P.p[G.prob[0]].map_adp, &full[s], a * 16, kc);
+        }
+        last_load = g;
+        if (++s == S) {
+          s = 0;
+          ph ^= 1u;
         }
       }
     }
@@ -335,7 +339,20 @@ __global__ void __launch_bounds__(256) lora_project_reduce(const __grid_constant
   if (q4 < quads) {
     const float4* src =
         reinterpret_cast<const float4*>(G.part + static_cast<int64_t>(t) * G.chunks * N) + q4;
-    for (int ch = sub; ch < G.chunks; ch += S) {
+    int ch = sub;
+    for (; ch + 7 * S < G.chunks; ch += 8 * S) {  // eight loads in flight, adds in order
+      float4 v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = __ldcg(src + static_cast<int64_t>(ch + k * S) * quads);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        acc.x += v[k].x;
+        acc.y += v[k].y;
+        acc.z += v[k].z;
+        acc.w += v[k].w;
+      }
+    }
+    for (; ch < G.chunks; ch += S) {
       const float4 v = __ldcg(src + static_cast<int64_t>(ch) * quads);
       acc.x += v.x;
       acc.y += v.y;
@@ -468,42 +485,47 @@ __global__ void __launch_bounds__(kGrdThreads, 1) lora_grad_tc(const __grid_cons
   bool mma_issued = false;
 
   if (warp == 0) {
-    // ---------------------------------------------- TMA producer
-    if (lane == 0) {
-      int g = 0, s = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
-        int gi, c0;
-        item_of(it, gi, c0);
-        const RkGradGroup& G = P.g[gi];
-        const int vbytes = G.n_prob * R * 128;
-        for (int i = 0; i < nsteps; ++i, ++g) {
-          if (g >= S && !mbar_wait(&empty[s], ph ^ 1u, abort_p, &g_rank_flags, kRkFlagProducer)) {
-            ok = false;
-            break;
-          }
-          uint8_t* st = smem + s * stage_bytes;
-          const int tk = i * 64;
+    // ---------------------------------------------- TMA producer (the whole
+    // warp: lane 0 waits for the stage and arms its barrier, then the lanes
+    // issue the step's boxes side by side)
+    int g = 0, s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < P.n_items && ok; it += gridDim.x) {
+      int gi, c0;
+      item_of(it, gi, c0);
+      const RkGradGroup& G = P.g[gi];
+      const int vbytes = G.n_prob * R * 128;
+      const int n_atoms = G.n_prob * (R / 16);  // 16-rank V atoms per part
+      for (int i = 0; i < nsteps; ++i, ++g) {
+        if (lane == 0 && g >= S)
+          ok = mbar_wait(&empty[s], ph ^ 1u, abort_p, &g_rank_flags, kRkFlagProducer);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        uint8_t* st = smem + s * stage_bytes;
+        const int tk = i * 64;
+        if (lane == 0)
           mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kGrdZBytes + 2 * vbytes));
-          // Z: per 128-column M tile two 64-column atoms (rows = tokens), the
-          // MN-major operand layout; the tiles of an item are adjacent columns
-          for (int a = 0; a < 2 * kGrdMT; ++a)
-            tma_load_2d(st + a * 8192, &G.map_z, &full[s], c0 + 64 * a, tk);
-          uint8_t* vh = st + kGrdZBytes;
-          for (int q = 0; q < G.n_prob; ++q) {
-            const RkGradProb& pr = P.p[G.prob[q]];
-            for (int a = 0; a < R / 16; ++a) {
-              const int atom = q * (R / 16) + a;
-              tma_load_2d(vh + atom * 2048, &pr.map_hi, &full[s], a * 16, tk);
-              tma_load_2d(vh + vbytes + atom * 2048, &pr.map_lo, &full[s], a * 16, tk);
-            }
+        __syncwarp();
+        // Z: per 128-column M tile two 64-column atoms (rows = tokens), the
+        // MN-major operand layout; the tiles of an item are adjacent columns.
+        // The first lanes load them, the next lanes the V atoms (hi parts,
+        // then lo parts), one box per lane.
+        for (int box = lane; box < 2 * kGrdMT + 2 * n_atoms; box += 32) {
+          if (box < 2 * kGrdMT) {
+            tma_load_2d(st + box * 8192, &G.map_z, &full[s], c0 + 64 * box, tk);
+          } else {
+            const int v = box - 2 * kGrdMT;
+            const int part = v / n_atoms, atom = v % n_atoms;  // part 0: hi, 1: lo
+            const RkGradProb& pr = P.p[G.prob[atom / (R / 16)]];
+            tma_load_2d(st + kGrdZBytes + part * vbytes + atom * 2048,
+                        part ? &pr.map_lo : &pr.map_hi, &full[s], (atom % (R / 16)) * 16, tk);
           }
-          last_load = g;
-          if (++s == S) {
-            s = 0;
-            ph ^= 1u;
-          }
+        }
+        last_load = g;
+        if (++s == S) {
+          s = 0;
+          ph ^= 1u;
         }
       }
     }
