@@ -87,7 +87,8 @@ constexpr int kWarpEpi = 8, kWarpProdX = 12, kWarpProdC = 13, kWarpMma = 14;
 
 struct GemmProblem {
   CUtensorMap map_act;    // X / dY: bf16 [T, contraction], box {64, min(BN/2,128)}, 128B swizzle
-  CUtensorMap map_codes;  // uint8 [n_out, k_in/2]; box {32, 128} fwd, {64, 64} dx; dense:
+  CUtensorMap map_codes;  // uint8 [n_out, k_in/2]; box {32, 128} fwd (32B swizzle), {64, 64}
+                          // dx (64B swizzle); dense:
                           // bf16 [n_out, k_in], box {64, 128} fwd, {64, 64} dx, 128B swizzle
   CUtensorMap map_lo_a;   // fwd: B [n_out, r] box {16, 128} 32B; dx: A [r, k_in] box {64, r_pad} 128B
   CUtensorMap map_lo_b;   // s*t or s*u: bf16 [T, r_pad], box {16, min(BN/2,128)}, 32B swizzle
@@ -492,7 +493,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int grp = warp >> 2;        // 0 or 1: takes the K steps with g % 2 == grp
     const int i = threadIdx.x & 127;  // this thread's line of the A tile
     const int line = (MODE == kGemmFwd) ? i : ((i >> 6) * 64 + (i & 63));
-    const int code_off = (MODE == kGemmFwd) ? i * 32 : (i & 63) * 64 + (i >> 6) * 32;
+    // this thread's two 16-byte chunks of the step's code tile.  The tile is
+    // TMA-swizzled so that a warp's loads hit distinct banks: fwd rows of 32 B
+    // (32B swizzle: chunk c of row w at c ^ ((w >> 2) & 1)), dx rows of 64 B
+    // (64B swizzle: chunk c of row w at c ^ ((w >> 1) & 3))
+    int code_chunk0, code_chunk1;  // in 16-byte units from the tile start
+    if (MODE == kGemmFwd) {
+      const int sw = (i >> 2) & 1;
+      code_chunk0 = i * 2 + (0 ^ sw);
+      code_chunk1 = i * 2 + (1 ^ sw);
+    } else {
+      const int row = i & 63, h = i >> 6, sw = (row >> 1) & 3;
+      code_chunk0 = row * 4 + ((2 * h) ^ sw);
+      code_chunk1 = row * 4 + ((2 * h + 1) ^ sw);
+    }
     // this thread's absmax for K step kb of unit U (0 past the weight's edge)
     auto absmax_at = [&](const Unit& U, int kb) -> float {
       const GemmProblem& pr = P.prob[U.p];
@@ -548,10 +562,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
-      const uint4* src = reinterpret_cast<const uint4*>(c_tile(sc) + code_off);
-      const uint4 c0 = src[0], c1 = src[1];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&c_empty[sc]);
+      const uint4* src = reinterpret_cast<const uint4*>(c_tile(sc));
+      const uint4 c0 = src[code_chunk0], c1 = src[code_chunk1];
+      // the warp's code loads have returned (the reduction consumes every
+      // lane's words) before lane 0 releases the code stage to the producer
+      const uint32_t dep = __reduce_or_sync(
+          0xffffffffu, c0.x ^ c0.y ^ c0.z ^ c0.w ^ c1.x ^ c1.y ^ c1.z ^ c1.w);
+      if (lane == 0) mbar_arrive_after(&c_empty[sc], dep);
       const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
       const Nf4Table tab = nf4_make_table(P.cb, a);
       if (gc >= SA && !mbar_wait(&a_empty[sa], pha ^ 1u, abort_flag, &g_gemm_flags,
@@ -1082,13 +1099,13 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     if (mode == kGemmFwd) {
       if (!d.dense)
         ok = ok && encode_tma_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
-                             d.n_out, d.k_in / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+                             d.n_out, d.k_in / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_32B);
       ok = ok && encode_tma_2d(&g.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_a, r, d.n_out,
                            r * 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
     } else {
       if (!d.dense)
         ok = ok && encode_tma_2d(&g.map_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.codes, d.k_in / 2,
-                             d.n_out, d.k_in / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+                             d.n_out, d.k_in / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B);
       ok = ok && encode_tma_2d(&g.map_lo_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.lo_a, d.k_in, r,
                            d.k_in * 2, 64, r_pad, CU_TENSOR_MAP_SWIZZLE_128B);
     }

@@ -37,6 +37,12 @@ enum : unsigned int {
 };
 
 constexpr int kMrgTile = 128;
+// Buffering, and CTAs per SM they allow: TMEM holds 512 columns per SM
+// (kMrgAccBufs x 128 per CTA), shared memory ~227 KB.
+constexpr int kMrgAccBufs = 2;  // TMEM accumulators per CTA
+constexpr int kMrgOutBufs = 2;  // output staging tiles per expanding warpgroup
+constexpr int kMrgCtasPerSm = 2;
+static_assert(kMrgAccBufs * kMrgTile * kMrgCtasPerSm <= 512, "TMEM columns per SM");
 
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -82,7 +88,7 @@ __host__ __device__ inline MergeSmem merge_smem(int dense, int r_pad) {
   m.a = m.b + (r_pad / 16) * 4096;   // B: r_pad / 16 slices of 128 rows x 32 B
   m.stage = m.a + 2 * r_pad * 128;   // A: two 64-column atoms of r_pad rows x 128 B
   m.out = 2 * m.stage;               // W': per buffer two 64-column boxes of 128 rows x 128 B
-  m.total = m.out + 2 * 32768;
+  m.total = m.out + kMrgOutBufs * 32768;
   return m;
 }
 
@@ -97,7 +103,7 @@ static_assert(kMrgExpand == 256, "two warpgroups expand the tile");
 // time, expand the matching base bytes, add, round and write the bf16 row
 // into one of two staging tiles, which one thread stores with TMA while the
 // next tile is expanded.
-__global__ void __launch_bounds__(kMrgThreads, 2) lora_merge_kernel(const __grid_constant__ MergeParams P) {
+__global__ void __launch_bounds__(kMrgThreads, kMrgCtasPerSm) lora_merge_kernel(const __grid_constant__ MergeParams P) {
   extern __shared__ uint8_t mrg_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(mrg_smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -121,7 +127,7 @@ __global__ void __launch_bounds__(kMrgThreads, 2) lora_merge_kernel(const __grid
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_slot, 2 * kMrgTile);
+    tmem_alloc(&tmem_slot, kMrgAccBufs * kMrgTile);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -168,9 +174,10 @@ __global__ void __launch_bounds__(kMrgThreads, 2) lora_merge_kernel(const __grid
       const uint32_t idesc = make_idesc_bf16(kMrgTile, kMrgTile, 0, 1);
       int li = 0;
       for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++li) {
-        const int s = li & 1, b = li & 1;
+        const int s = li & 1, b = li % kMrgAccBufs;
         if (!mbar_wait(&st_full[s], (li >> 1) & 1, abort_p, &g_merge_flags, kMrgFlagMma)) break;
-        if (li >= 2 && !mbar_wait(&acc_empty[b], ((li >> 1) - 1) & 1, abort_p, &g_merge_flags,
+        if (li >= kMrgAccBufs &&
+            !mbar_wait(&acc_empty[b], ((li / kMrgAccBufs) - 1) & 1, abort_p, &g_merge_flags,
                                   kMrgFlagMma))
           break;
         tc_fence_after();
@@ -206,70 +213,85 @@ __global__ void __launch_bounds__(kMrgThreads, 2) lora_merge_kernel(const __grid
     int li = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++li) {
-      const int s = li & 1, b = li & 1;
+      const int s = li & 1, b = li % kMrgAccBufs, ob = li % kMrgOutBufs;
       const float am = am_next;
       am_next = absmax_of(tile + gridDim.x);
       const int n0 = (tile / P.col_tiles) * kMrgTile, k0 = (tile % P.col_tiles) * kMrgTile;
       ok = mbar_wait(&st_full[s], (li >> 1) & 1, abort_p, &g_merge_flags, kMrgFlagMma) &&
-           mbar_wait(&acc_full[b], (li >> 1) & 1, abort_p, &g_merge_flags, kMrgFlagMma);
-      // the staging box written two tiles ago has been read by its store
-      if (et == 0) bulk_wait_group_read<1>();
+           mbar_wait(&acc_full[b], (li / kMrgAccBufs) & 1, abort_p, &g_merge_flags, kMrgFlagMma);
+      // the staging box this tile writes has been read by its earlier store
+      if (et == 0) bulk_wait_group_read<kMrgOutBufs - 1>();
       if (!named_sync_and_mrg(1 + h, 128, ok)) break;
       tc_fence_after();
       const uint8_t* st = smem + s * L.stage;
-      uint8_t* out_box = smem + L.out + b * 32768 + h * 16384;
+      uint8_t* out_box = smem + L.out + ob * 32768 + h * 16384;
       Nf4Table tab;
       if (!P.dense) tab = nf4_make_table(P.cb, am);
+      const uint64_t s2 = f32x2_pack(P.s, P.s);
+      // this row's 64 code bytes of the warpgroup's 128 columns (NF4): 64-byte
+      // code rows, 64B swizzle, 16-byte chunk q of row i at chunk q ^ ((i >> 1) & 3)
+      uint32_t cw[8];
+      if (!P.dense) {
 #pragma unroll
-      for (int cc = 0; cc < 64; cc += 32) {
-        const int c = 64 * h + cc;
-        uint32_t v[32];
-        tmem_ld32(tmem + static_cast<uint32_t>(b * kMrgTile) + lane_base + static_cast<uint32_t>(c), v);
-        tmem_wait_ld();
-        // the base's 32 bf16 values of this row, columns c .. c + 31
-        uint32_t w[16];
+        for (int q = 0; q < 2; ++q) {
+          const int chunk = (2 * h + q) ^ ((tid >> 1) & 3);
+          const uint4 x = *reinterpret_cast<const uint4*>(st + tid * 64 + chunk * 16);
+          cw[4 * q] = x.x, cw[4 * q + 1] = x.y, cw[4 * q + 2] = x.z, cw[4 * q + 3] = x.w;
+        }
+        // once this row's codes are in registers (the stage's B and A are
+        // read only by the MMAs, whose commit arrives too) the producer may
+        // refill the stage while this tile is expanded
+        mbar_arrive_after(&st_empty[s],
+                          cw[0] ^ cw[1] ^ cw[2] ^ cw[3] ^ cw[4] ^ cw[5] ^ cw[6] ^ cw[7]);
+      }
+      // 16 columns at a time; the product of the next 16 is read from tensor
+      // memory while this 16 is expanded
+      const uint32_t tcol = tmem + static_cast<uint32_t>(b * kMrgTile + 64 * h) + lane_base;
+      uint32_t v[2][16];
+      tmem_ld16(tcol, v[0]);
+      tmem_wait_ld_for(v[0]);
+      const uint8_t* drow = st + h * 16384 + tid * 128;  // dense: this row's 128 B of the base
+      uint8_t* orow = out_box + tid * 128;               // this row of the output box
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (j < 3) tmem_ld16(tcol + static_cast<uint32_t>(16 * (j + 1)), v[(j + 1) & 1]);
+        const uint32_t(&acc)[16] = v[j & 1];
+        // the base's 16 bf16 values of this row, columns 16 j .. 16 j + 15 of the block
+        uint32_t w[8];
         if (P.dense) {
-          const uint8_t* row = st + h * 16384 + tid * 128;
+          // 128B swizzle: 16-byte chunk q of row i at chunk q ^ (i & 7)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int chunk = (cc / 8 + q) ^ (tid & 7);
-            const uint4 x = *reinterpret_cast<const uint4*>(row + chunk * 16);
+          for (int q = 0; q < 2; ++q) {
+            const uint4 x =
+                *reinterpret_cast<const uint4*>(drow + (((2 * j + q) ^ (tid & 7)) * 16));
             w[4 * q] = x.x, w[4 * q + 1] = x.y, w[4 * q + 2] = x.z, w[4 * q + 3] = x.w;
           }
         } else {
-          // 64-byte code rows, 64B swizzle: 16-byte chunk q of row i sits at
-          // chunk q ^ ((i >> 1) & 3)
-          const int chunk = (c / 32) ^ ((tid >> 1) & 3);
-          const uint4 x = *reinterpret_cast<const uint4*>(st + tid * 64 + chunk * 16);
-          const uint32_t cw[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 d = nf4_dequant8(cw[q], tab);
+          for (int q = 0; q < 2; ++q) {
+            const uint4 d = nf4_dequant8(cw[2 * j + q], tab);
             w[4 * q] = d.x, w[4 * q + 1] = d.y, w[4 * q + 2] = d.z, w[4 * q + 3] = d.w;
           }
         }
-        uint32_t o[16];
+        // fp32(deq + fp32(s * acc)), two columns per instruction, then one
+        // rounding to bf16
+        uint32_t o[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
-          const __nv_bfloat162 m =
-              __floats2bfloat162_rn(__fadd_rn(lo, __fmul_rn(P.s, __uint_as_float(v[2 * e]))),
-                                    __fadd_rn(hi, __fmul_rn(P.s, __uint_as_float(v[2 * e + 1]))));
-          o[e] = *reinterpret_cast<const uint32_t*>(&m);
+        for (int e = 0; e < 8; ++e) {
+          const uint64_t base = f32x2_pack_bits(w[e] << 16, w[e] & 0xFFFF0000u);
+          const uint64_t pr = f32x2_pack_bits(acc[2 * e], acc[2 * e + 1]);
+          o[e] = f32x2_to_bf16x2(f32x2_add_rn(base, f32x2_mul_rn(pr, s2)));
         }
-        // row of the 128B-swizzled output box: 16-byte chunk q of row i at
-        // chunk q ^ (i & 7)
-        uint8_t* orow = out_box + tid * 128;
+        // the 128B-swizzled output box, same chunk rule as the dense base
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = (cc / 8 + q) ^ (tid & 7);
-          *reinterpret_cast<uint4*>(orow + chunk * 16) =
+        for (int q = 0; q < 2; ++q)
+          *reinterpret_cast<uint4*>(orow + (((2 * j + q) ^ (tid & 7)) * 16)) =
               make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-        }
+        if (j < 3) tmem_wait_ld_for(v[(j + 1) & 1]);
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[b]);  // the accumulator is read
-      mbar_arrive(&st_empty[s]);   // and this row of the base
+      mbar_arrive(&acc_empty[b]);            // the accumulator is read
+      if (P.dense) mbar_arrive(&st_empty[s]);  // and this row of the base
       fence_proxy_async_smem();
       named_sync(1 + h, 128);
       if (et == 0) {
@@ -297,7 +319,7 @@ __global__ void __launch_bounds__(kMrgThreads, 2) lora_merge_kernel(const __grid
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * kMrgTile);
+    tmem_dealloc(tmem, kMrgAccBufs * kMrgTile);
   }
 }
 
@@ -341,7 +363,7 @@ cudaError_t launch_lora_merge(const void* base, const float* absmax, bool dense,
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int per_sm = std::max(1, std::min(2, (227 * 1024) / smem));  // TMEM: 2 x 256 columns
+  const int per_sm = std::max(1, std::min(kMrgCtasPerSm, (227 * 1024) / smem));
   const int grid = static_cast<int>(std::min<int64_t>(tiles, static_cast<int64_t>(per_sm) * sms));
   void* prof = prof_begin(st);
   count_launch();

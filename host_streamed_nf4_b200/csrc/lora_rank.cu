@@ -339,25 +339,21 @@ __global__ void __launch_bounds__(256) lora_project_reduce(const __grid_constant
   if (q4 < quads) {
     const float4* src =
         reinterpret_cast<const float4*>(G.part + static_cast<int64_t>(t) * G.chunks * N) + q4;
-    int ch = sub;
-    for (; ch + 7 * S < G.chunks; ch += 8 * S) {  // eight loads in flight, adds in order
-      float4 v[8];
+    // sixteen loads in flight (the tail of a batch predicated off), then the
+    // adds in slice order
+    for (int ch0 = sub; ch0 < G.chunks; ch0 += 16 * S) {
+      float4 v[16];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = __ldcg(src + static_cast<int64_t>(ch + k * S) * quads);
+      for (int k = 0; k < 16; ++k)
+        if (ch0 + k * S < G.chunks) v[k] = __ldcg(src + static_cast<int64_t>(ch0 + k * S) * quads);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        acc.x += v[k].x;
-        acc.y += v[k].y;
-        acc.z += v[k].z;
-        acc.w += v[k].w;
-      }
-    }
-    for (; ch < G.chunks; ch += S) {
-      const float4 v = __ldcg(src + static_cast<int64_t>(ch) * quads);
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+      for (int k = 0; k < 16; ++k)
+        if (ch0 + k * S < G.chunks) {
+          acc.x += v[k].x;
+          acc.y += v[k].y;
+          acc.z += v[k].z;
+          acc.w += v[k].w;
+        }
     }
   }
   for (int m = Q; m < 32; m <<= 1) {

@@ -155,6 +155,46 @@ def test_merge_vs_oracle(orc, N, K, r, alpha, base):
     assert (d > 0).mean() <= 1e-3, f"{(d > 0).mean():.2e} of the elements differ from the oracle"
 
 
+def test_merge_repeatable_on_a_full_size_gate(orc):
+    """The Qwen2.5-72B gate projection (29568 x 8192, r 16): about 50 tiles
+    per CTA, so every stage and accumulator buffer is reused many times while
+    the producer runs ahead.  Every launch gives the same bits (a stage
+    released before its reads completed showed up here as a few hundred wrong
+    elements in most launches), and sampled rows, first and last tiles among
+    them, agree with the oracle within the merge bound."""
+    N, K, r, alpha = 29568, 8192, 16, 32.0
+    case = synth.linear_case(4343, 1, N, K, r=r, alpha=alpha, b_std=0.05)
+    W = hsnf4.nf4_quantize_pack(to_dev_bf16(case.W))
+    A, B = to_dev_bf16(case.A), to_dev_bf16(case.B)
+    first = hsnf4.lora_merge(W, A, B, alpha)
+    out = torch.empty_like(first)
+    for _ in range(5):
+        hsnf4.lora_merge(W, A, B, alpha, out=out)
+        torch.cuda.synchronize()
+        assert torch.equal(out, first)
+    assert hsnf4.device_status() == 0
+    rows = np.array([0, 1, 127, 128, 8191, 14783, 29439, 29567])
+    codes, absmax = orc.quantize(case.W[rows])
+    # the GPU quantizer's codes of these rows are the oracle's (codec parity)
+    kb = K // 64
+    gpu_codes = W.codes.view(N, K // 2)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    gpu_absmax = W.absmax.view(N, kb)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    assert np.array_equal(gpu_codes.reshape(-1), codes)
+    assert np.array_equal(gpu_absmax.reshape(-1), absmax)
+    ref = orc.lora_merge(case.A, case.B[rows], alpha, codes=codes, absmax=absmax, N=len(rows),
+                         K=K)
+    got = bf16_bits(first[torch.from_numpy(rows).cuda()])
+    deq = synth.bits_to_f32(orc.dequant(codes, absmax, len(rows), K))
+    mag = (alpha / r) * (np.abs(synth.bits_to_f32(case.B[rows])).astype(np.float64) @
+                         np.abs(synth.bits_to_f32(case.A)).astype(np.float64))
+    mag += np.abs(deq.astype(np.float64))
+    fp32_err = 2 * (r + 2) * 2.0 ** -24 * mag
+    g64, r64 = synth.bits_to_f32(got).astype(np.float64), synth.bits_to_f32(ref).astype(np.float64)
+    ulp = np.abs(synth.bits_to_f32(_next_up(ref)).astype(np.float64) - r64)
+    assert not (np.abs(g64 - r64) > ulp + fp32_err).any()
+    assert (_ulp_diff(got, ref) > 0).mean() <= 1e-3
+
+
 def test_merge_zero_adapter_is_dequant_bitwise():
     case = synth.linear_case(41, 1, 384, 512)
     W = hsnf4.nf4_quantize_pack(to_dev_bf16(case.W))
