@@ -8,15 +8,17 @@
 // the tensor cores (exact bf16 products, fp32 accumulate), is scaled by s in
 // fp32, added to deq(W) in fp32 and rounded once to bf16.
 //
-// CTA = a 128 x 128 tile of W' (sm_100a).  One thread loads the tile's base
-// (NF4 codes or bf16 weight), B's 128 rows and A's 128 columns with TMA,
-// then issues r/16 tcgen05 MMAs (M = 128 rows, N = 128 columns, K = 16
-// ranks each; B read K-major, A read MN-major) into a 128-column fp32
-// accumulator in tensor memory.  Each of the 128 threads then owns one row:
-// it reads its product row back from tensor memory 32 columns at a time,
-// expands the matching base bytes, adds, rounds and writes the bf16 row into
-// a staging tile that two TMA stores write out.  HBM traffic is the base read
-// once plus W' written once; several CTAs per SM keep loads in flight.
+// Persistent CTAs (sm_100a), each taking 128 x 128 tiles of W' in turn.
+// Warp 0 loads a tile's base (NF4 codes or bf16 weight), B's 128 rows and
+// A's 128 columns with TMA into one of two stages; warp 1 issues r/16
+// tcgen05 MMAs (M = 128 rows, N = 128 columns, K = 16 ranks each; B read
+// K-major, A read MN-major) into a 128-column fp32 accumulator in tensor
+// memory.  Two warpgroups then expand the tile, each thread one row of 64
+// columns: it reads its product row back from tensor memory 16 columns at a
+// time, expands the matching base bytes, adds, rounds and writes the bf16
+// row into a 128B-swizzled staging box that one thread per warpgroup stores
+// with TMA.  HBM traffic is the base read once plus W' written once; several
+// CTAs per SM keep loads and stores in flight.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -37,12 +39,21 @@ enum : unsigned int {
 };
 
 constexpr int kMrgTile = 128;
-// Buffering, and CTAs per SM they allow: TMEM holds 512 columns per SM
-// (kMrgAccBufs x 128 per CTA), shared memory ~227 KB.
-constexpr int kMrgAccBufs = 2;  // TMEM accumulators per CTA
-constexpr int kMrgOutBufs = 2;  // output staging tiles per expanding warpgroup
-constexpr int kMrgCtasPerSm = 2;
-static_assert(kMrgAccBufs * kMrgTile * kMrgCtasPerSm <= 512, "TMEM columns per SM");
+// Buffering per base format, and the CTAs per SM it allows (TMEM: 512
+// columns per SM, kAccBufs x 128 per CTA; shared memory ~227 KB; registers
+// 64 K).  NF4: one accumulator and one staging tile per warpgroup, three
+// CTAs per SM (measured ~10% faster than two double-buffered CTAs: more
+// expanding warps hide the waits).  Dense: the 32 KB base tiles allow two
+// CTAs, each double-buffered.
+template <bool DENSE>
+struct MrgCfg {
+  static constexpr int kAccBufs = DENSE ? 2 : 1;  // TMEM accumulators per CTA
+  static constexpr int kOutBufs = DENSE ? 2 : 1;  // output staging tiles per warpgroup
+  static constexpr int kCtasPerSm = DENSE ? 2 : 3;
+  static_assert(kAccBufs * kMrgTile * kCtasPerSm <= 512, "TMEM columns per SM");
+};
+constexpr int kMrgCols = 16;  // columns per TMEM read of the expanding loop (8 or 16)
+static_assert(kMrgCols == 8 || kMrgCols == 16, "TMEM read width");
 
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -88,7 +99,7 @@ __host__ __device__ inline MergeSmem merge_smem(int dense, int r_pad) {
   m.a = m.b + (r_pad / 16) * 4096;   // B: r_pad / 16 slices of 128 rows x 32 B
   m.stage = m.a + 2 * r_pad * 128;   // A: two 64-column atoms of r_pad rows x 128 B
   m.out = 2 * m.stage;               // W': per buffer two 64-column boxes of 128 rows x 128 B
-  m.total = m.out + kMrgOutBufs * 32768;
+  m.total = m.out + (dense ? MrgCfg<true>::kOutBufs : MrgCfg<false>::kOutBufs) * 32768;
   return m;
 }
 
@@ -98,19 +109,21 @@ static_assert(kMrgExpand == 256, "two warpgroups expand the tile");
 
 // Persistent: CTA b takes tiles b, b + gridDim.x, ...  Warp 0 loads the next
 // tile into the other stage while the current one is processed; warp 1
-// issues each tile's r/16 MMAs into one of two TMEM accumulators; warps 2..5
-// (one row of the tile per thread) read the product row back 32 columns at a
-// time, expand the matching base bytes, add, round and write the bf16 row
-// into one of two staging tiles, which one thread stores with TMA while the
-// next tile is expanded.
-__global__ void __launch_bounds__(kMrgThreads, kMrgCtasPerSm) lora_merge_kernel(const __grid_constant__ MergeParams P) {
+// issues each tile's MMAs into a TMEM accumulator (MrgCfg: one or two per
+// CTA); warps 2..9 (two warpgroups, one row of the tile per thread) expand
+// it into staging boxes (one or two per warpgroup) that TMA stores write
+// out while the next tile is expanded.
+template <bool DENSE>
+__global__ void __launch_bounds__(kMrgThreads, MrgCfg<DENSE>::kCtasPerSm)
+    lora_merge_kernel(const __grid_constant__ MergeParams P) {
   extern __shared__ uint8_t mrg_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(mrg_smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   __shared__ uint64_t st_full[2], st_empty[2], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
-  const MergeSmem L = merge_smem(P.dense, P.r_pad);
+  constexpr int kMrgAccBufs = MrgCfg<DENSE>::kAccBufs, kMrgOutBufs = MrgCfg<DENSE>::kOutBufs;
+  const MergeSmem L = merge_smem(DENSE, P.r_pad);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = P.row_tiles * P.col_tiles;
   const int slices = P.r_pad / 16;
@@ -151,7 +164,7 @@ __global__ void __launch_bounds__(kMrgThreads, kMrgCtasPerSm) lora_merge_kernel(
         const int n0 = (tile / P.col_tiles) * kMrgTile, k0 = (tile % P.col_tiles) * kMrgTile;
         uint8_t* st = smem + s * L.stage;
         mbar_arrive_expect_tx(&st_full[s], bytes);
-        if (P.dense) {
+        if (DENSE) {
           tma_load_2d(st, &P.map_base, &st_full[s], k0, n0);
           tma_load_2d(st + 16384, &P.map_base, &st_full[s], k0 + 64, n0);
         } else {
@@ -204,7 +217,7 @@ __global__ void __launch_bounds__(kMrgThreads, kMrgCtasPerSm) lora_merge_kernel(
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     // this row's absmax for the warpgroup's block of a tile, loaded one tile ahead
     auto absmax_of = [&](int tile) -> float {
-      if (P.dense || tile >= n_tiles) return 0.f;
+      if (DENSE || tile >= n_tiles) return 0.f;
       const int n = (tile / P.col_tiles) * kMrgTile + tid, k0 = (tile % P.col_tiles) * kMrgTile;
       if (n >= P.N || k0 + 64 * h >= P.K) return 0.f;
       return __ldg(P.absmax + static_cast<int64_t>(n) * (P.K / 64) + k0 / 64 + h);
@@ -226,12 +239,12 @@ __global__ void __launch_bounds__(kMrgThreads, kMrgCtasPerSm) lora_merge_kernel(
       const uint8_t* st = smem + s * L.stage;
       uint8_t* out_box = smem + L.out + ob * 32768 + h * 16384;
       Nf4Table tab;
-      if (!P.dense) tab = nf4_make_table(P.cb, am);
+      if (!DENSE) tab = nf4_make_table(P.cb, am);
       const uint64_t s2 = f32x2_pack(P.s, P.s);
       // this row's 64 code bytes of the warpgroup's 128 columns (NF4): 64-byte
       // code rows, 64B swizzle, 16-byte chunk q of row i at chunk q ^ ((i >> 1) & 3)
       uint32_t cw[8];
-      if (!P.dense) {
+      if (!DENSE) {
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int chunk = (2 * h + q) ^ ((tid >> 1) & 3);
@@ -244,54 +257,49 @@ __global__ void __launch_bounds__(kMrgThreads, kMrgCtasPerSm) lora_merge_kernel(
         mbar_arrive_after(&st_empty[s],
                           cw[0] ^ cw[1] ^ cw[2] ^ cw[3] ^ cw[4] ^ cw[5] ^ cw[6] ^ cw[7]);
       }
-      // 16 columns at a time; the product of the next 16 is read from tensor
-      // memory while this 16 is expanded
+      // kMrgCols columns at a time; the product of the next kMrgCols is read
+      // from tensor memory while these are expanded
+      constexpr int C = kMrgCols, NCH = 64 / C;
       const uint32_t tcol = tmem + static_cast<uint32_t>(b * kMrgTile + 64 * h) + lane_base;
-      uint32_t v[2][16];
-      tmem_ld16(tcol, v[0]);
+      uint32_t v[2][C];
+      tmem_ld(tcol, v[0]);
       tmem_wait_ld_for(v[0]);
       const uint8_t* drow = st + h * 16384 + tid * 128;  // dense: this row's 128 B of the base
       uint8_t* orow = out_box + tid * 128;               // this row of the output box
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (j < 3) tmem_ld16(tcol + static_cast<uint32_t>(16 * (j + 1)), v[(j + 1) & 1]);
-        const uint32_t(&acc)[16] = v[j & 1];
-        // the base's 16 bf16 values of this row, columns 16 j .. 16 j + 15 of the block
-        uint32_t w[8];
-        if (P.dense) {
-          // 128B swizzle: 16-byte chunk q of row i at chunk q ^ (i & 7)
+      for (int j = 0; j < NCH; ++j) {
+        if (j < NCH - 1) tmem_ld(tcol + static_cast<uint32_t>(C * (j + 1)), v[(j + 1) & 1]);
+        const uint32_t(&acc)[C] = v[j & 1];
+        // the base's C bf16 values of this row, columns C j .. C j + C - 1 of the block
+        uint32_t w[C / 2];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const uint4 x =
-                *reinterpret_cast<const uint4*>(drow + (((2 * j + q) ^ (tid & 7)) * 16));
-            w[4 * q] = x.x, w[4 * q + 1] = x.y, w[4 * q + 2] = x.z, w[4 * q + 3] = x.w;
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const uint4 d = nf4_dequant8(cw[2 * j + q], tab);
-            w[4 * q] = d.x, w[4 * q + 1] = d.y, w[4 * q + 2] = d.z, w[4 * q + 3] = d.w;
-          }
+        for (int q = 0; q < C / 8; ++q) {
+          uint4 x;
+          if constexpr (DENSE)  // 128B swizzle: 16-byte chunk q of row i at chunk q ^ (i & 7)
+            x = *reinterpret_cast<const uint4*>(drow + ((((C / 8) * j + q) ^ (tid & 7)) * 16));
+          else
+            x = nf4_dequant8(cw[(C / 8) * j + q], tab);
+          w[4 * q] = x.x, w[4 * q + 1] = x.y, w[4 * q + 2] = x.z, w[4 * q + 3] = x.w;
         }
         // fp32(deq + fp32(s * acc)), two columns per instruction, then one
         // rounding to bf16
-        uint32_t o[8];
+        uint32_t o[C / 2];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < C / 2; ++e) {
           const uint64_t base = f32x2_pack_bits(w[e] << 16, w[e] & 0xFFFF0000u);
           const uint64_t pr = f32x2_pack_bits(acc[2 * e], acc[2 * e + 1]);
           o[e] = f32x2_to_bf16x2(f32x2_add_rn(base, f32x2_mul_rn(pr, s2)));
         }
         // the 128B-swizzled output box, same chunk rule as the dense base
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
-          *reinterpret_cast<uint4*>(orow + (((2 * j + q) ^ (tid & 7)) * 16)) =
+        for (int q = 0; q < C / 8; ++q)
+          *reinterpret_cast<uint4*>(orow + ((((C / 8) * j + q) ^ (tid & 7)) * 16)) =
               make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-        if (j < 3) tmem_wait_ld_for(v[(j + 1) & 1]);
+        if (j < NCH - 1) tmem_wait_ld_for(v[(j + 1) & 1]);
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[b]);            // the accumulator is read
-      if (P.dense) mbar_arrive(&st_empty[s]);  // and this row of the base
+      if (DENSE) mbar_arrive(&st_empty[s]);  // and this row of the base
       fence_proxy_async_smem();
       named_sync(1 + h, 128);
       if (et == 0) {
@@ -353,8 +361,13 @@ cudaError_t launch_lora_merge(const void* base, const float* absmax, bool dense,
   static cudaError_t attr_rc = cudaSuccess;
   static std::once_flag once;
   std::call_once(once, [] {
-    attr_rc = cudaFuncSetAttribute(lora_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_rc = cudaFuncSetAttribute(lora_merge_kernel<true>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    merge_smem(1, 64).total + 1024);
+    if (attr_rc == cudaSuccess)
+      attr_rc = cudaFuncSetAttribute(lora_merge_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     merge_smem(0, 64).total + 1024);
   });
   if (attr_rc != cudaSuccess) return attr_rc;
   P.row_tiles = static_cast<int>((N + kMrgTile - 1) / kMrgTile);
@@ -363,11 +376,16 @@ cudaError_t launch_lora_merge(const void* base, const float* absmax, bool dense,
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int per_sm = std::max(1, std::min(kMrgCtasPerSm, (227 * 1024) / smem));
+  const int per_sm = std::max(
+      1, std::min(P.dense ? MrgCfg<true>::kCtasPerSm : MrgCfg<false>::kCtasPerSm,
+                  (227 * 1024) / smem));
   const int grid = static_cast<int>(std::min<int64_t>(tiles, static_cast<int64_t>(per_sm) * sms));
   void* prof = prof_begin(st);
   count_launch();
-  lora_merge_kernel<<<grid, kMrgThreads, smem, st>>>(P);
+  if (P.dense)
+    lora_merge_kernel<true><<<grid, kMrgThreads, smem, st>>>(P);
+  else
+    lora_merge_kernel<false><<<grid, kMrgThreads, smem, st>>>(P);
   const cudaError_t e = cudaGetLastError();
   // algorithmic bytes per element: the base read (0.5625 B NF4, 2 B dense) + 2 B written
   if (prof) prof_end(prof, kProfMerge, (dense ? 4.0 : 2.5625) * static_cast<double>(N) * K, st);
