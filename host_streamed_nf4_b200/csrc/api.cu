@@ -465,15 +465,18 @@ int lora_group_bwd(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r, fl
   rc = cuda_status(launch_lora_project_group(pd, n, T, r, s, ws + L.prj, st),
                    "lora_group_bwd: projection launch");
   if (rc) return rc;
+  // The adapter gradients need only u, t, X and dY: they run before the dX
+  // GEMM, while the dY the projection has just read (and X) are still in L2,
+  // instead of after the GEMM has streamed the base through it.
+  rc = cuda_status(launch_lora_grad_group(grd, 2 * n, T, r, s, st),
+                   "lora_group_bwd: gradient launch");
+  if (rc) return rc;
   rc = launch_lora_gemm_group(kGemmDx, gd, n, T, r, ws + L.gemm, L.total - L.gemm, st);
   if (rc) return rc;
-  if (nd) {
+  if (nd)
     rc = cuda_status(launch_dx_dropout_add(da, nd, T, r, s, st),
                      "lora_group_bwd: dropout dX launch");
-    if (rc) return rc;
-  }
-  return cuda_status(launch_lora_grad_group(grd, 2 * n, T, r, s, st),
-                     "lora_group_bwd: gradient launch");
+  return rc;
 }
 
 int lora_merge(const hsnf4_nf4_weight* W, const void* A, const void* B, int r, float alpha,
