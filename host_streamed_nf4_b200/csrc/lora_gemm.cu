@@ -597,7 +597,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const Unit U = unpack_unit(P, P.units[ui]);
       const GemmProblem& pr = P.prob[U.p];
       const int m0 = U.mt * kPairM + row0, t0 = U.tt * BN;
-      const int M = pr.m_total;
       const int NB = P.n_buf;
       const int buf = NB > 1 ? (lu & 1) : 0;
       const uint32_t acc0 = tmem + static_cast<uint32_t>(buf * 256) + lane_base;
