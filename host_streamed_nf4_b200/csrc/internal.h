@@ -115,6 +115,26 @@ cudaError_t launch_lora_merge(const void* base, const float* absmax, bool dense,
 // Process-wide count of kernels this library launched (hsnf4_kernel_launches).
 void count_launch();
 
+// Launch with programmatic stream serialization: the kernel's CTAs may start
+// before the previous kernel in the stream completes.  Only for kernels that
+// call pdl_wait_then_release() before any global-memory access.
+template <typename Params>
+inline cudaError_t launch_pdl(void (*kernel)(Params), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, const Params& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 // ---- LoRA dropout, grouped (lora_dropout.cu): apply writes out = X_d;
 // dx add updates out = dX += keep * scale * s * (u A).
 struct DropDesc {

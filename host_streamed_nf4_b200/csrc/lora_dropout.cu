@@ -21,6 +21,7 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 #include "philox.cuh"
 
 namespace hsnf4 {
@@ -68,6 +69,7 @@ __device__ __forceinline__ uint32_t keep8(const DropProblem& pr, int64_t g) {
 }
 
 __global__ void __launch_bounds__(256) lora_dropout_apply(const __grid_constant__ DropParams P) {
+  pdl_wait_then_release();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < P.total;
        g += stride) {
@@ -102,6 +104,7 @@ constexpr int kDxTok = 32, kDxCols = 256, kDxMaxR = 64;
 __global__ void __launch_bounds__(256) lora_dx_dropout_add(const __grid_constant__ DropParams P) {
   __shared__ __align__(16) uint16_t a_s[kDxMaxR * kDxCols];  // A[j][c], this tile's columns
   __shared__ __align__(16) float u_s[kDxTok * kDxMaxR];      // u[t][j], this tile's tokens
+  pdl_wait_then_release();
   const int q = drop_problem(P, blockIdx.x);
   const DropProblem& pr = P.p[q];
   const int64_t local = static_cast<int64_t>(blockIdx.x) - pr.g0;
@@ -222,12 +225,8 @@ static cudaError_t launch_drop(bool dx, const DropDesc* d, int n, int64_t T, int
   if (grid > static_cast<int64_t>(sms) * 16) grid = static_cast<int64_t>(sms) * 16;
   if (dx) grid = g;  // one CTA per tile
   if (grid < 1) grid = 1;
-  count_launch();
-  if (dx)
-    lora_dx_dropout_add<<<static_cast<unsigned>(grid), 256, 0, st>>>(P);
-  else
-    lora_dropout_apply<<<static_cast<unsigned>(grid), 256, 0, st>>>(P);
-  return cudaGetLastError();
+  return launch_pdl(dx ? lora_dx_dropout_add : lora_dropout_apply,
+                    dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, P);
 }
 
 cudaError_t launch_dropout_apply(const DropDesc* d, int n, int64_t T, cudaStream_t st) {

@@ -274,6 +274,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_before();
   cluster_sync();  // barriers of both CTAs initialised before any cross-CTA arrive
   tc_fence_after();
+  pdl_wait_then_release();
   const uint32_t tmem = *tmem_slot;
 
   int last_x = -1, last_c = -1, last_l = -1;  // producers: last issued sequence numbers
@@ -728,6 +729,7 @@ struct ReduceParams {
 };
 
 __global__ void __launch_bounds__(128) lora_splitk_reduce(const __grid_constant__ ReduceParams R) {
+  pdl_wait_then_release();
   // CTA: one tile, 8 tokens; warp w the tokens 2w, 2w + 1 of them; lane l
   // rows 4l .. 4l + 3 (one 16-byte piece of each partial, 512 contiguous
   // bytes per token across the warp).  All of a token's split loads are in
@@ -1120,12 +1122,8 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     return fail(HSNF4_ERR_CUDA, "lora gemm: smem attribute");
   const int smem = smem_plan(mode, BN, tl.sx, tl.sc, tl.sa, r_pad).total + 1024;
   void* prof = prof_begin(st);
-  count_launch();
-  if (mode == kGemmFwd)
-    lora_gemm_kernel<kGemmFwd><<<2 * G, kThreads, smem, st>>>(P);  // G clusters of 2
-  else
-    lora_gemm_kernel<kGemmDx><<<2 * G, kThreads, smem, st>>>(P);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(mode == kGemmFwd ? lora_gemm_kernel<kGemmFwd> : lora_gemm_kernel<kGemmDx>,
+                             dim3(2 * G), dim3(kThreads), smem, st, P);  // G clusters of 2
   if (e == cudaSuccess && L.need) {
     // add the K-split partials in split order and write the bf16 outputs
     static ReduceParams R;
@@ -1141,8 +1139,9 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
             const int m0 = mt * kPairM + c * kTileM;
             if (m0 >= g.m_total) continue;
             if (R.n_tiles == kMaxReduceTiles) {
-              count_launch();
-              lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 128, 0, st>>>(R);
+              e = launch_pdl(lora_splitk_reduce, dim3(R.n_tiles * (BN / kReduceTok)), dim3(128),
+                             0, st, R);
+              if (e != cudaSuccess) break;
               R.n_tiles = 0;
             }
             const int tile = (tt * g.m_tiles + mt) * 2 + c;
@@ -1150,11 +1149,8 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
                                    g.out, m0, tt * BN, g.m_total, g.splits};
           }
     }
-    if (R.n_tiles) {
-      count_launch();
-      lora_splitk_reduce<<<R.n_tiles * (BN / kReduceTok), 128, 0, st>>>(R);
-    }
-    e = cudaGetLastError();
+    if (e == cudaSuccess && R.n_tiles)
+      e = launch_pdl(lora_splitk_reduce, dim3(R.n_tiles * (BN / kReduceTok)), dim3(128), 0, st, R);
   }
   if (prof) {
     // algorithmic FLOPs: the base products plus the rank-r slices

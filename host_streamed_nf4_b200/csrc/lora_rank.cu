@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(kPrjThreads, 1) lora_project_tc(const __grid_c
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait_then_release();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_p = &abort_flag;
   int last_load = -1;
@@ -323,6 +324,7 @@ __global__ void __launch_bounds__(kPrjThreads, 1) lora_project_tc(const __grid_c
 // order depends only on the sizes, never on timing).  The lanes holding a
 // quad's total write t, s t and the optional bf16 parts.
 __global__ void __launch_bounds__(256) lora_project_reduce(const __grid_constant__ RkProjParams P) {
+  pdl_wait_then_release();
   const int idx = static_cast<int>(blockIdx.x) * 8 + static_cast<int>(threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (idx >= P.n_out) return;
@@ -475,6 +477,7 @@ __global__ void __launch_bounds__(kGrdThreads, 1) lora_grad_tc(const __grid_cons
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait_then_release();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_p = &abort_flag;
   int last_load = -1;
@@ -828,14 +831,9 @@ cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, in
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(items, sms);
   void* prof = prof_begin(st);
-  count_launch();
-  lora_project_tc<<<grid, kPrjThreads, smem, st>>>(P);
-  e = cudaGetLastError();
-  if (e == cudaSuccess) {
-    count_launch();
-    lora_project_reduce<<<(outs + 7) / 8, 256, 0, st>>>(P);
-    e = cudaGetLastError();
-  }
+  e = launch_pdl(lora_project_tc, dim3(grid), dim3(kPrjThreads), smem, st, P);
+  if (e == cudaSuccess)
+    e = launch_pdl(lora_project_reduce, dim3((outs + 7) / 8), dim3(256), 0, st, P);
   prof_end(prof, kProfProject, bytes, st);
   return e;
 }
@@ -902,9 +900,7 @@ cudaError_t launch_lora_grad_group(const GradDesc* d, int n, int64_t T, int r, f
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(ctas, sms);
   void* prof = prof_begin(st);
-  count_launch();
-  lora_grad_tc<<<grid, kGrdThreads, smem, st>>>(P);
-  e = cudaGetLastError();
+  e = launch_pdl(lora_grad_tc, dim3(grid), dim3(kGrdThreads), smem, st, P);
   prof_end(prof, kProfGrad, bytes, st);
   return e;
 }

@@ -134,6 +134,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// ---------------------------------------------------------------- launch order
+
+// Programmatic dependent launch.  The training step's kernels are launched
+// with programmatic stream serialization, so that a kernel's CTAs may be
+// scheduled (and set up shared memory, barriers and TMEM) while the previous
+// kernel in the stream is still finishing.  Every thread calls this before
+// its first global-memory access, read or write: the wait returns once the
+// previous grid has completed and its writes are visible, exactly as plain
+// stream order would give.  Then the next kernel may be scheduled.
+__device__ __forceinline__ void pdl_wait_then_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
