@@ -182,7 +182,7 @@ enum ProfKind {
   kProfKinds = 6
 };
 bool profiling();
-void* prof_begin(cudaStream_t st);
+void* prof_begin(cudaStream_t st, int kind);
 void prof_end(void* token, int kind, double work, cudaStream_t st);
 
 // Read and clear the device failure flags the GEMM kernels record.

@@ -1121,7 +1121,7 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
   if (configure_once<kGemmFwd>() != 0 || configure_once<kGemmDx>() != 0)
     return fail(HSNF4_ERR_CUDA, "lora gemm: smem attribute");
   const int smem = smem_plan(mode, BN, tl.sx, tl.sc, tl.sa, r_pad).total + 1024;
-  void* prof = prof_begin(st);
+  void* prof = prof_begin(st, mode == kGemmFwd ? kProfGemmFwd : kProfGemmDx);
   cudaError_t e = launch_pdl(mode == kGemmFwd ? lora_gemm_kernel<kGemmFwd> : lora_gemm_kernel<kGemmDx>,
                              dim3(2 * G), dim3(kThreads), smem, st, P);  // G clusters of 2
   if (e == cudaSuccess && L.need) {

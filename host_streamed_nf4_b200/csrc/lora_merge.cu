@@ -380,7 +380,7 @@ cudaError_t launch_lora_merge(const void* base, const float* absmax, bool dense,
       1, std::min(P.dense ? MrgCfg<true>::kCtasPerSm : MrgCfg<false>::kCtasPerSm,
                   (227 * 1024) / smem));
   const int grid = static_cast<int>(std::min<int64_t>(tiles, static_cast<int64_t>(per_sm) * sms));
-  void* prof = prof_begin(st);
+  void* prof = prof_begin(st, kProfMerge);
   count_launch();
   if (P.dense)
     lora_merge_kernel<true><<<grid, kMrgThreads, smem, st>>>(P);

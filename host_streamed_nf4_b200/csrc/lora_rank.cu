@@ -830,7 +830,7 @@ cudaError_t launch_lora_project_group(const ProjectDesc* d, int n, int64_t T, in
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(items, sms);
-  void* prof = prof_begin(st);
+  void* prof = prof_begin(st, kProfProject);
   e = launch_pdl(lora_project_tc, dim3(grid), dim3(kPrjThreads), smem, st, P);
   if (e == cudaSuccess)
     e = launch_pdl(lora_project_reduce, dim3((outs + 7) / 8), dim3(256), 0, st, P);
@@ -899,7 +899,7 @@ cudaError_t launch_lora_grad_group(const GradDesc* d, int n, int64_t T, int r, f
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(ctas, sms);
-  void* prof = prof_begin(st);
+  void* prof = prof_begin(st, kProfGrad);
   e = launch_pdl(lora_grad_tc, dim3(grid), dim3(kGrdThreads), smem, st, P);
   prof_end(prof, kProfGrad, bytes, st);
   return e;

@@ -160,7 +160,7 @@ cudaError_t launch_nf4_dequant(const void* codes, const float* absmax, int64_t n
   const int64_t cap = static_cast<int64_t>(sms) * 4;  // resident at 52 registers: one wave
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  void* prof = prof_begin(st);
+  void* prof = prof_begin(st, kProfDequant);
   count_launch();
   nf4_dequant_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(
       static_cast<const uint4*>(codes), absmax, static_cast<uint4*>(out), n_quads, codebook());

@@ -22,6 +22,7 @@ struct Rec {
 
 std::mutex g_mu;
 bool g_on = false;
+unsigned g_kinds = 0;  // bit k: time launches of kind k
 std::vector<Rec> g_recs;
 
 const char* kKindName[kProfKinds] = {"lora_gemm_fwd", "lora_gemm_dx", "nf4_dequant",
@@ -35,8 +36,8 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 bool profiling() { return g_on; }
 
-void* prof_begin(cudaStream_t st) {
-  if (!g_on) return nullptr;
+void* prof_begin(cudaStream_t st, int kind) {
+  if (!g_on || !((g_kinds >> kind) & 1u)) return nullptr;
   cudaEvent_t a;
   if (cudaEventCreate(&a) != cudaSuccess) return nullptr;
   cudaEventRecord(a, st);
@@ -75,6 +76,15 @@ int hsnf4_profile(int enable) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (enable) clear_locked();
   g_on = enable != 0;
+  g_kinds = (1u << kProfKinds) - 1;
+  return HSNF4_OK;
+}
+
+int hsnf4_profile_kinds(unsigned int kinds) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  clear_locked();
+  g_kinds = kinds & ((1u << kProfKinds) - 1);
+  g_on = g_kinds != 0;
   return HSNF4_OK;
 }
 

@@ -84,6 +84,7 @@ _SIGS = {
     "hsnf4_inject_fault": ([c_char_p], c_int),
     "hsnf4_selftest_stall": ([c_void_p], c_int),
     "hsnf4_profile": ([c_int], c_int),
+    "hsnf4_profile_kinds": ([c_uint32], c_int),
     "hsnf4_kernel_launches": ([], c_uint64),
     "hsnf4_profile_read": ([POINTER(KernelTime), c_int], c_int),
     "nf4_codebook": ([POINTER(c_float)], c_int),
@@ -211,8 +212,20 @@ def kernel_launches() -> int:
     return int(lib().hsnf4_kernel_launches())
 
 
-def profile(enable: bool):
-    _check(lib().hsnf4_profile(int(bool(enable))))
+PROFILE_KINDS = ("lora_gemm_fwd", "lora_gemm_dx", "nf4_dequant", "lora_merge", "lora_project",
+                 "lora_grad")
+
+
+def profile(enable: bool, kinds=None):
+    """Start (clearing) or stop kernel timing; `kinds`, a subset of
+    PROFILE_KINDS, times only those launches."""
+    if enable and kinds is not None:
+        mask = 0
+        for k in kinds:
+            mask |= 1 << PROFILE_KINDS.index(k)
+        _check(lib().hsnf4_profile_kinds(mask))
+    else:
+        _check(lib().hsnf4_profile(int(bool(enable))))
 
 
 def profile_read() -> dict:

@@ -117,21 +117,27 @@ int hsnf4_device_status(void *stream, uint32_t *flags);
 int hsnf4_selftest_stall(void *stream);
 
 /* Kernel timing for roofline reports.  While enabled, the library brackets
- * every launch of its fused GEMM (forward and dX modes) and of the NF4
- * dequant kernel with CUDA events on the launch stream, and accumulates
- * per kernel: launches, device time and algorithmic work (FLOPs for the
- * GEMMs, bytes read + written for dequant).  hsnf4_profile(1) starts (and
- * clears), hsnf4_profile(0) stops.  hsnf4_profile_read synchronizes on the
+ * every launch of the enabled kernel kinds with CUDA events on the launch
+ * stream, and accumulates per kind: launches, device time and algorithmic
+ * work (FLOPs for the fused GEMM; bytes read + written for the dequant and
+ * the merge; distinct activation bytes read for the rank-r projection and
+ * gradient kernels).  Kinds, by bit: 0 lora_gemm_fwd, 1 lora_gemm_dx,
+ * 2 nf4_dequant, 3 lora_merge, 4 lora_project, 5 lora_grad.
+ * hsnf4_profile(1) starts (and clears) timing of every kind,
+ * hsnf4_profile_kinds(mask) of the kinds whose bits are set (events between
+ * launches delay the next launch, so timing fewer kinds disturbs a run
+ * less), hsnf4_profile(0) stops.  hsnf4_profile_read synchronizes on the
  * recorded events and fills out[0..n) (host), returning the number of
  * entries (<= max_out) or a negative status. */
 typedef struct {
-  char name[32];        /* "lora_gemm_fwd", "lora_gemm_dx", "nf4_dequant" */
+  char name[32];        /* the kind's name, as listed above */
   uint64_t launches;
   double total_ms;      /* sum of per-launch event durations */
   double work;          /* total algorithmic FLOPs or bytes */
 } hsnf4_kernel_time;
 
 int hsnf4_profile(int enable);
+int hsnf4_profile_kinds(unsigned int kinds);
 int hsnf4_profile_read(hsnf4_kernel_time *out, int max_out);
 
 /* Number of kernels this library has launched in this process (every
