@@ -53,6 +53,7 @@
 #include <climits>
 #include <cstddef>
 #include <map>
+#include <tuple>
 #include <mutex>
 #include <queue>
 #include <vector>
@@ -96,12 +97,13 @@ struct GemmProblem {
   const float* absmax;
   uint16_t* out;          // bf16 [T, m_total]
   float* partial;         // split-K partial tiles (fp32 [BN tokens][128 rows] each), or null
-  int n_out, k_in, m_total, nk, kblocks, m_tiles, splits;  // m_tiles: 256-row tiles
+  int n_out, k_in, m_total, nk, kblocks, m_tiles;  // m_tiles: 256-row tiles
+  int splits;             // partial slots per tile: the most K segments any tile has
 };
 
 constexpr int kMaxProblems = 8;
 constexpr int kMaxPairs = 80;
-constexpr int kMaxUnits = 3072;
+constexpr int kMaxUnits = 2560;
 
 struct GemmParams {
   GemmProblem prob[kMaxProblems];
@@ -111,27 +113,39 @@ struct GemmParams {
               // overlaps the next unit's MMAs) or 1 (BN = 512 fills TMEM)
   int dense;  // 1: map_codes is the bf16 weight, TMA-loaded straight into the A ring
   uint16_t pair_off[kMaxPairs + 1];  // units of pair c: units[pair_off[c] .. pair_off[c+1])
-  uint32_t units[kMaxUnits];  // problem(3) | split(5) | token tile(6) | row tile(18)
+  uint32_t units[kMaxUnits];   // problem(3) | K segment(5) | token tile(6) | row tile(18)
+  uint32_t unit_k[kMaxUnits];  // first K step(15) | end K step(15) | writes a partial(1)
 };
+static_assert(sizeof(GemmParams) <= 32764, "kernel parameter block");
+
+__host__ __device__ inline uint32_t pack_unit_k(int kb0, int kb1, bool partial) {
+  return static_cast<uint32_t>(kb0) | (static_cast<uint32_t>(kb1) << 15) |
+         (partial ? (1u << 30) : 0u);
+}
 
 __host__ __device__ inline uint32_t pack_unit(int p, int s, int tt, int mt) {
   return (static_cast<uint32_t>(p) << 29) | (static_cast<uint32_t>(s) << 24) |
          (static_cast<uint32_t>(tt) << 18) | static_cast<uint32_t>(mt);
 }
 
+// A work unit: one K segment [kb0, kb1) of one (problem, token tile, 256-row
+// tile).  A tile cut into several segments has each write an fp32 partial
+// (slot `split` of the tile) that a second pass adds in segment order.
 struct Unit {
   int p, split, tt, mt, kb0, kb1;
+  bool partial;
 };
 
-__device__ __forceinline__ Unit unpack_unit(const GemmParams& P, uint32_t u) {
+__device__ __forceinline__ Unit unpack_unit(const GemmParams& P, int ui) {
+  const uint32_t u = P.units[ui], k = P.unit_k[ui];
   Unit r;
   r.p = u >> 29;
   r.split = (u >> 24) & 31;
   r.tt = (u >> 18) & 63;
   r.mt = u & 0x3FFFF;
-  const int nk = P.prob[r.p].nk, S = P.prob[r.p].splits;
-  r.kb0 = r.split * nk / S;
-  r.kb1 = (r.split + 1) * nk / S;
+  r.kb0 = k & 0x7FFF;
+  r.kb1 = (k >> 15) & 0x7FFF;
+  r.partial = ((k >> 30) & 1u) != 0;
   return r;
 }
 
@@ -288,7 +302,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t lora_tx = static_cast<uint32_t>(plan.st_off - plan.la_off);
       bool ok = true;
       for (int ui = u_begin; ui < u_end && ok; ++ui, ++lu) {
-        const Unit U = unpack_unit(P, P.units[ui]);
+        const Unit U = unpack_unit(P, ui);
         const GemmProblem& pr = P.prob[U.p];
         const int m0 = U.mt * kPairM + row0, t0 = U.tt * BN;
         for (int kb = U.kb0; kb < U.kb1; ++kb, ++g, xr.step(SX)) {
@@ -335,7 +349,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int CS = P.dense ? SA : SC;
       bool ok = true;
       for (int ui = u_begin; ui < u_end && ok; ++ui) {
-        const Unit U = unpack_unit(P, P.units[ui]);
+        const Unit U = unpack_unit(P, ui);
         const GemmProblem& pr = P.prob[U.p];
         const int m0 = U.mt * kPairM + row0;
         for (int kb = U.kb0; kb < U.kb1; ++kb, ++g, cr.step(CS)) {
@@ -383,7 +397,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       Ring xr, ar, pr_;
       bool ok = true;
       for (int ui = u_begin; ui < u_end && ok; ++ui, ++lu) {
-        const Unit U = unpack_unit(P, P.units[ui]);
+        const Unit U = unpack_unit(P, ui);
         const int buf = NB > 1 ? (lu & 1) : 0;
         if (lu >= NB) {
           if (!mbar_wait(&acc_empty[buf], ((lu / NB) - 1) & 1, abort_flag, &g_gemm_flags,
@@ -435,7 +449,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       Ring xr, ar, pr_;
       bool ok = true;
       for (int ui = u_begin; ui < u_end && ok; ++ui, ++lu) {
-        const Unit U = unpack_unit(P, P.units[ui]);
+        const Unit U = unpack_unit(P, ui);
         const int buf = NB > 1 ? (lu & 1) : 0;
         const uint32_t acc0 = tmem + static_cast<uint32_t>(buf * 256);
         if (lu >= NB) {  // both epilogues have drained this buffer's previous unit
@@ -528,7 +542,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       while (kb >= U.kb1) {
         const int over = kb - U.kb1;
         if (++ui >= u_end) return false;
-        U = unpack_unit(P, P.units[ui]);
+        U = unpack_unit(P, ui);
         kb = U.kb0 + over;
       }
       return true;
@@ -540,7 +554,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     Unit U{};
     bool have = ui < u_end;
     if (have) {
-      U = unpack_unit(P, P.units[ui]);
+      U = unpack_unit(P, ui);
       kb = U.kb0;
       have = advance(ui, kb, U, grp);
     }
@@ -595,7 +609,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int lu = 0;
     int epi_step = 0;  // 32-token output steps so far (picks the staging buffer pair)
     for (int ui = u_begin; ui < u_end; ++ui, ++lu) {
-      const Unit U = unpack_unit(P, P.units[ui]);
+      const Unit U = unpack_unit(P, ui);
       const GemmProblem& pr = P.prob[U.p];
       const int m0 = U.mt * kPairM + row0, t0 = U.tt * BN;
       const int NB = P.n_buf;
@@ -609,7 +623,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // this CTA's 128-row half of the unit's tile
       const int tile = (U.tt * pr.m_tiles + U.mt) * 2 + static_cast<int>(crank);
-      if (pr.splits > 1) {
+      if (U.partial) {
         // this split's fp32 tile -> workspace, token-major ([BN][128]) so that a
         // warp's 32 rows of one token are 128 contiguous bytes; the splits are
         // added in split order by lora_splitk_reduce after this kernel
@@ -870,73 +884,196 @@ static int64_t lpt_makespan(std::vector<int64_t>& costs, int sms) {
   return mk;
 }
 
-// K splits per problem.  Objective: the simulated makespan of the
-// longest-first schedule (in K steps) plus the split-K reduce pass, whose
-// partial reads are charged at ~16 KiB per K step per SM.  Search: starting
-// from no splits, repeatedly add one split to the problem holding the
-// longest unit (pieces of at least 16 K steps, at most 8 splits), keeping
-// the best objective seen.  Deterministic in the shapes and the SM count.
-static void plan_splits(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int BN,
-                        int sms, std::vector<int>* splits) {
-  std::vector<int64_t> tiles(n), nk(n);
-  for (int p = 0; p < n; ++p) {
-    const int64_t mdim = (mode == kGemmFwd) ? probs[p].n_out : probs[p].k_in;
-    const int64_t contraction = (mode == kGemmFwd) ? probs[p].k_in : probs[p].n_out;
-    tiles[p] = ((mdim + kPairM - 1) / kPairM) * ((T + BN - 1) / BN);
-    nk[p] = contraction / kStepK;
-  }
-  auto objective = [&](const std::vector<int>& sp) -> int64_t {
-    std::vector<int64_t> costs;
-    double reduce_bytes = 0;
-    for (int p = 0; p < n; ++p) {
-      for (int s = 0; s < sp[p]; ++s) {
-        const int64_t ks = (s + 1) * nk[p] / sp[p] - s * nk[p] / sp[p];
-        costs.insert(costs.end(), static_cast<size_t>(tiles[p]), unit_cost(ks, sp[p]));
-      }
-      if (sp[p] > 1) reduce_bytes += static_cast<double>(tiles[p]) * sp[p] * kPairM * BN * 4;
+// The LPT plan's objective for K splits `sp` (per problem): the simulated
+// makespan of the longest-first schedule (in K steps) plus the split-K
+// reduce pass, whose partial reads are charged at ~16 KiB per K step per SM.
+static int64_t lpt_objective(const std::vector<int64_t>& tiles, const std::vector<int64_t>& nk,
+                             const std::vector<int>& sp, int BN, int sms) {
+  std::vector<int64_t> costs;
+  double reduce_bytes = 0;
+  for (size_t p = 0; p < tiles.size(); ++p) {
+    for (int s = 0; s < sp[p]; ++s) {
+      const int64_t ks = (s + 1) * nk[p] / sp[p] - s * nk[p] / sp[p];
+      costs.insert(costs.end(), static_cast<size_t>(tiles[p]), unit_cost(ks, sp[p]));
     }
-    if (costs.size() > static_cast<size_t>(3072)) return INT64_MAX;  // over the unit limit
-    const int64_t reduce = reduce_bytes > 0
-                               ? 4 + static_cast<int64_t>(reduce_bytes / (16384.0 * sms))
-                               : 0;
-    return lpt_makespan(costs, sms / 2) + reduce;  // units run on CTA pairs
-  };
+    if (sp[p] > 1) reduce_bytes += static_cast<double>(tiles[p]) * sp[p] * kPairM * BN * 4;
+  }
+  if (costs.size() > static_cast<size_t>(kMaxUnits)) return INT64_MAX;  // over the unit limit
+  const int64_t reduce =
+      reduce_bytes > 0 ? 4 + static_cast<int64_t>(reduce_bytes / (16384.0 * sms)) : 0;
+  return lpt_makespan(costs, sms / 2) + reduce;  // units run on CTA pairs
+}
+
+// K splits per problem for the LPT plan.  Search: starting from no splits,
+// repeatedly add one split to the problem holding the longest unit (pieces
+// of at least 16 K steps, at most 8 splits), keeping the best objective seen.
+static int64_t plan_splits(const std::vector<int64_t>& tiles, const std::vector<int64_t>& nk,
+                           int BN, int sms, std::vector<int>* splits) {
+  const size_t n = tiles.size();
   std::vector<int> cur(n, 1);
   *splits = cur;
-  int64_t best = objective(cur);
+  int64_t best = lpt_objective(tiles, nk, cur, BN, sms);
   for (int it = 0; it < 24; ++it) {
     int worst = -1;
     int64_t worst_cost = -1;
-    for (int p = 0; p < n; ++p) {
+    for (size_t p = 0; p < n; ++p) {
       const int64_t c = unit_cost(nk[p] / cur[p] + (nk[p] % cur[p] ? 1 : 0), cur[p]);
       if (c > worst_cost && cur[p] < kMaxSplits && nk[p] / (cur[p] + 1) >= 16) {
-        worst = p;
+        worst = static_cast<int>(p);
         worst_cost = c;
       }
     }
     if (worst < 0) break;
     cur[worst] += 1;
-    const int64_t obj = objective(cur);
+    const int64_t obj = lpt_objective(tiles, nk, cur, BN, sms);
     if (obj < best) {
       best = obj;
       *splits = cur;
     }
   }
+  return best;
 }
 
-struct SplitLayout {
-  std::vector<int> splits;
+// The stream-K plan: every pair gets an equal share C = ceil(W / G) of all
+// K steps, walking the tiles in (problem, token tile, row tile) order and
+// cutting a tile's K range where a share ends (no piece shorter than
+// kMinSegment steps).  A tile cut into pieces has each write an fp32 partial.
+// Balances launches with fewer tiles than pairs, or tiles that do not
+// divide evenly among them, at the cost of the partials.
+struct Segment {
+  int p, tt, mt, kb0, kb1, seg, nseg, pair;
+};
+constexpr int kMinSegment = 8;
+
+static int64_t streamk_cut(const std::vector<int64_t>& mt_n, const std::vector<int64_t>& nk,
+                           int t_tiles, int BN, int G, int sms, int64_t C,
+                           std::vector<Segment>* out);
+
+static int64_t streamk_segments(const std::vector<int64_t>& mt_n, const std::vector<int64_t>& nk,
+                                int t_tiles, int BN, int G, int sms, std::vector<Segment>* out) {
+  int64_t W = 0;
+  for (size_t p = 0; p < nk.size(); ++p) W += mt_n[p] * t_tiles * nk[p];
+  // the smallest share that leaves the last pair no more than the others
+  // (pieces are never cut below kMinSegment, so an exact W / G can overflow)
+  int64_t best = INT64_MAX;
+  std::vector<Segment> trial;
+  for (int64_t C = (W + G - 1) / G, step = std::max<int64_t>(1, C / 32), it = 0; it < 24;
+       ++it, C += step) {
+    const int64_t obj = streamk_cut(mt_n, nk, t_tiles, BN, G, sms, C, &trial);
+    if (obj < best) {
+      best = obj;
+      *out = trial;
+    }
+  }
+  return best;
+}
+
+static int64_t streamk_cut(const std::vector<int64_t>& mt_n, const std::vector<int64_t>& nk,
+                           int t_tiles, int BN, int G, int sms, int64_t C,
+                           std::vector<Segment>* out) {
+  out->clear();
+  int pair = 0;
+  int64_t load = 0;
+  std::vector<int64_t> cost(G, 0);
+  double reduce_bytes = 0;
+  for (size_t p = 0; p < nk.size(); ++p)
+    for (int tt = 0; tt < t_tiles; ++tt)
+      for (int mt = 0; mt < mt_n[p]; ++mt) {
+        const size_t first = out->size();
+        int kb = 0, seg = 0;
+        while (kb < nk[p]) {
+          if (pair < G - 1 && load > 0 && C - load < kMinSegment) {
+            ++pair;
+            load = 0;
+          }
+          int64_t take = pair == G - 1 ? nk[p] - kb : std::min<int64_t>(nk[p] - kb, C - load);
+          if (nk[p] - kb - take < kMinSegment) take = nk[p] - kb;  // no sliver left behind
+          out->push_back({static_cast<int>(p), tt, mt, kb, static_cast<int>(kb + take), seg, 0,
+                          pair});
+          kb += static_cast<int>(take);
+          load += take;
+          ++seg;
+          if (pair < G - 1 && load >= C) {
+            ++pair;
+            load = 0;
+          }
+        }
+        for (size_t i = first; i < out->size(); ++i) {
+          Segment& s = (*out)[i];
+          s.nseg = seg;
+          cost[s.pair] += unit_cost(s.kb1 - s.kb0, seg);
+        }
+        if (seg > 1) reduce_bytes += static_cast<double>(seg) * kPairM * BN * 4;
+        if (seg > kMaxSplits) return INT64_MAX;  // the reduce pass adds at most kMaxSplits
+      }
+  if (out->size() > static_cast<size_t>(kMaxUnits)) return INT64_MAX;
+  const int64_t reduce =
+      reduce_bytes > 0 ? 4 + static_cast<int64_t>(reduce_bytes / (16384.0 * sms)) : 0;
+  return *std::max_element(cost.begin(), cost.end()) + reduce;
+}
+
+// The launch's work plan: LPT over uniform K splits, or stream-K where the
+// cost model puts it at least 4% lower.  Deterministic in the shapes and the
+// SM count.
+struct GemmPlan {
+  bool stream_k = false;
+  std::vector<int> splits;       // LPT: K splits per problem
+  std::vector<int> slots;        // partial slots per tile of each problem (1: no partials)
   std::vector<size_t> part_base;
-  size_t need = 0;
+  size_t need = 0;               // workspace bytes of the partials
 };
 
-// plan_splits results, cached by (mode, T, BN, SM count, shapes)
-static std::vector<int> cached_splits(GemmMode mode, const GemmProblemDesc* probs, int n,
-                                      int64_t T, int BN) {
-  static std::mutex mu;
-  static std::map<std::vector<int64_t>, std::vector<int>> cache;
+static void plan_dims(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int BN,
+                      std::vector<int64_t>* mt_n, std::vector<int64_t>* nk, int* t_tiles) {
+  *t_tiles = static_cast<int>((T + BN - 1) / BN);
+  mt_n->assign(n, 0);
+  nk->assign(n, 0);
+  for (int p = 0; p < n; ++p) {
+    const int64_t mdim = (mode == kGemmFwd) ? probs[p].n_out : probs[p].k_in;
+    const int64_t contraction = (mode == kGemmFwd) ? probs[p].k_in : probs[p].n_out;
+    (*mt_n)[p] = (mdim + kPairM - 1) / kPairM;
+    (*nk)[p] = contraction / kStepK;
+  }
+}
+
+static int plan_pairs(int sms) { return std::min(sms / 2, kMaxPairs); }
+
+static GemmPlan make_plan(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int BN) {
   const int sms = sm_count();
-  std::vector<int64_t> key = {static_cast<int64_t>(mode), T, BN, sms};
+  std::vector<int64_t> mt_n, nk;
+  int t_tiles = 0;
+  plan_dims(mode, probs, n, T, BN, &mt_n, &nk, &t_tiles);
+  std::vector<int64_t> tiles(n);
+  for (int p = 0; p < n; ++p) tiles[p] = mt_n[p] * t_tiles;
+  GemmPlan pl;
+  const int64_t lpt = plan_splits(tiles, nk, BN, sms, &pl.splits);
+  std::vector<Segment> segs;
+  const int64_t sk = streamk_segments(mt_n, nk, t_tiles, BN, plan_pairs(sms), sms, &segs);
+  // stream-K only for a clear predicted gain: measured on Qwen2.5-72B decoder
+  // launches, the model undercharges the partial tiles (their epilogue and
+  // the reduce pass), so predicted gains of ~3% turned into losses of ~5%
+  pl.stream_k = sk < lpt - lpt / 25;
+  pl.slots.assign(n, 1);
+  if (pl.stream_k) {
+    for (const Segment& s : segs) pl.slots[s.p] = std::max(pl.slots[s.p], s.nseg);
+  } else {
+    for (int p = 0; p < n; ++p) pl.slots[p] = pl.splits[p];
+  }
+  pl.part_base.assign(n, 0);
+  for (int p = 0; p < n; ++p) {
+    if (pl.slots[p] <= 1) continue;
+    pl.part_base[p] = pl.need;
+    pl.need += round_up(static_cast<size_t>(tiles[p]) * pl.slots[p] * kPairM * BN * 4, 256);
+  }
+  return pl;
+}
+
+// make_plan results, cached by (mode, T, BN, SM count, shapes)
+static GemmPlan cached_plan(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T,
+                            int BN) {
+  static std::mutex mu;
+  static std::map<std::vector<int64_t>, GemmPlan> cache;
+  std::vector<int64_t> key = {static_cast<int64_t>(mode), T, BN, sm_count()};
   for (int p = 0; p < n; ++p) {
     key.push_back(probs[p].n_out);
     key.push_back(probs[p].k_in);
@@ -944,35 +1081,16 @@ static std::vector<int> cached_splits(GemmMode mode, const GemmProblemDesc* prob
   std::lock_guard<std::mutex> lk(mu);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
-  std::vector<int> sp;
-  plan_splits(mode, probs, n, T, BN, sms, &sp);
+  GemmPlan pl = make_plan(mode, probs, n, T, BN);
   if (cache.size() > 4096) cache.clear();
-  cache.emplace(key, sp);
-  return sp;
-}
-
-static void split_layout(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int BN,
-                         SplitLayout* L) {
-  L->splits = cached_splits(mode, probs, n, T, BN);
-  L->part_base.assign(n, 0);
-  size_t part = 0;
-  const int64_t t_tiles = (T + BN - 1) / BN;
-  for (int p = 0; p < n; ++p) {
-    if (L->splits[p] <= 1) continue;
-    const int64_t mdim = (mode == kGemmFwd) ? probs[p].n_out : probs[p].k_in;
-    const int64_t tiles = ((mdim + kPairM - 1) / kPairM) * t_tiles;
-    L->part_base[p] = part;
-    part += round_up(static_cast<size_t>(tiles) * L->splits[p] * kPairM * BN * 4, 256);
-  }
-  L->need = part;
+  cache.emplace(key, pl);
+  return pl;
 }
 
 size_t gemm_workspace_bytes(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r) {
   Tiling tl;
   if (!choose_tiling(mode, T, (r + 15) / 16 * 16, &tl)) return 0;
-  SplitLayout L;
-  split_layout(mode, probs, n, T, tl.BN, &L);
-  return L.need;
+  return cached_plan(mode, probs, n, T, tl.BN).need;
 }
 
 int check_gemm_tokens(GemmMode mode, int64_t T, int r) {
@@ -1022,55 +1140,83 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
   while (tc < BN) tc <<= 1;
   P.tmem_cols = P.n_buf == 2 ? 512 : tc;  // two 256-column buffers, or one of BN
   const int sms = sm_count();
-  SplitLayout L;
-  split_layout(mode, probs, n, T, BN, &L);
+  const GemmPlan L = cached_plan(mode, probs, n, T, BN);
   if (L.need > ws_bytes || (L.need && !workspace))
     return fail(HSNF4_ERR_OOM, "lora gemm: workspace too small: need %zu bytes, given %zu",
                 L.need, ws_bytes);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  std::vector<int64_t> mt_n, nks;
+  int t_tiles_p = 0;
+  plan_dims(mode, probs, n, T, BN, &mt_n, &nks, &t_tiles_p);
+  for (int p = 0; p < n; ++p)
+    if (mt_n[p] > (1 << 18) || nks[p] >= (1 << 15))
+      return fail(HSNF4_ERR_INVALID, "lora gemm: problem %d exceeds the tile index range", p);
 
-  // units, longest first, each to the least loaded CTA so far
-  struct U {
-    int64_t cost;
-    uint32_t code;
-  };
-  std::vector<U> units;
-  for (int p = 0; p < n; ++p) {
-    const GemmProblemDesc& d = probs[p];
-    const int64_t mdim = (mode == kGemmFwd) ? d.n_out : d.k_in;
-    const int64_t nk = ((mode == kGemmFwd) ? d.k_in : d.n_out) / kStepK;
-    const int mt_n = static_cast<int>((mdim + kPairM - 1) / kPairM);
-    if (mt_n > (1 << 18))
-      return fail(HSNF4_ERR_INVALID, "lora gemm: %lld rows exceed the tile index range",
-                  (long long)mdim);
-    const int S = L.splits[p];
-    for (int s = 0; s < S; ++s) {
-      const int64_t cost = unit_cost((s + 1) * nk / S - s * nk / S, S);
-      for (int tt = 0; tt < t_tiles; ++tt)
-        for (int mt = 0; mt < mt_n; ++mt) units.push_back({cost, pack_unit(p, s, tt, mt)});
+  // per pair: the (unit code, K range) of its work units, in order
+  std::vector<std::vector<std::pair<uint32_t, uint32_t>>> per;
+  // K segments of each tile that writes partials: (problem, token tile, row tile) -> count
+  std::map<std::tuple<int, int, int>, int> nseg;
+  if (L.stream_k) {
+    std::vector<Segment> segs;
+    const int G = plan_pairs(sms);
+    if (streamk_segments(mt_n, nks, t_tiles, BN, G, sms, &segs) == INT64_MAX)
+      return fail(HSNF4_ERR_INVALID, "lora gemm: no stream-K plan within the unit limit");
+    per.assign(G, {});
+    for (const Segment& sg : segs) {
+      per[sg.pair].push_back({pack_unit(sg.p, sg.seg, sg.tt, sg.mt),
+                              pack_unit_k(sg.kb0, sg.kb1, sg.nseg > 1)});
+      if (sg.nseg > 1) nseg[{sg.p, sg.tt, sg.mt}] = sg.nseg;
+    }
+  } else {
+    // units, longest first, each to the least loaded pair so far
+    struct U {
+      int64_t cost;
+      uint32_t code, k;
+    };
+    std::vector<U> units;
+    for (int p = 0; p < n; ++p) {
+      const int S = L.splits[p];
+      for (int sp = 0; sp < S; ++sp) {
+        const int kb0 = static_cast<int>(sp * nks[p] / S);
+        const int kb1 = static_cast<int>((sp + 1) * nks[p] / S);
+        const int64_t cost = unit_cost(kb1 - kb0, S);
+        for (int tt = 0; tt < t_tiles; ++tt)
+          for (int mt = 0; mt < mt_n[p]; ++mt) {
+            units.push_back({cost, pack_unit(p, sp, tt, mt), pack_unit_k(kb0, kb1, S > 1)});
+            if (S > 1) nseg[{p, tt, mt}] = S;
+          }
+      }
+    }
+    if (units.size() > static_cast<size_t>(kMaxUnits))
+      return fail(HSNF4_ERR_INVALID, "lora gemm: %zu work units exceed the per-launch limit %d",
+                  units.size(), kMaxUnits);
+    std::stable_sort(units.begin(), units.end(),
+                     [](const U& a, const U& b) { return a.cost > b.cost; });
+    // persistent CTA pairs: one per two SMs
+    const int G = static_cast<int>(std::min<size_t>(units.size(), plan_pairs(sms)));
+    per.assign(G, {});
+    using Load = std::pair<int64_t, int>;
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+    for (int c = 0; c < G; ++c) heap.push({0, c});
+    for (const U& u : units) {
+      Load top = heap.top();
+      heap.pop();
+      per[top.second].push_back({u.code, u.k});
+      heap.push({top.first + u.cost, top.second});
     }
   }
-  if (units.size() > static_cast<size_t>(kMaxUnits))
-    return fail(HSNF4_ERR_INVALID, "lora gemm: %zu work units exceed the per-launch limit %d",
-                units.size(), kMaxUnits);
-  std::stable_sort(units.begin(), units.end(),
-                   [](const U& a, const U& b) { return a.cost > b.cost; });
-  // persistent CTA pairs: one per two SMs
-  const int G = static_cast<int>(std::min<size_t>(units.size(), std::min(sms / 2, kMaxPairs)));
-  std::vector<std::vector<uint32_t>> per(G);
-  using Load = std::pair<int64_t, int>;
-  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
-  for (int c = 0; c < G; ++c) heap.push({0, c});
-  for (const U& u : units) {
-    Load top = heap.top();
-    heap.pop();
-    per[top.second].push_back(u.code);
-    heap.push({top.first + u.cost, top.second});
-  }
+  const int G = static_cast<int>(per.size());
   int k = 0;
   for (int c = 0; c < G; ++c) {
     P.pair_off[c] = static_cast<uint16_t>(k);
-    for (uint32_t code : per[c]) P.units[k++] = code;
+    for (const auto& uk : per[c]) {
+      if (k == kMaxUnits)
+        return fail(HSNF4_ERR_INVALID, "lora gemm: work units exceed the per-launch limit %d",
+                    kMaxUnits);
+      P.units[k] = uk.first;
+      P.unit_k[k] = uk.second;
+      ++k;
+    }
   }
   P.pair_off[G] = static_cast<uint16_t>(k);
 
@@ -1089,7 +1235,7 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     g.nk = static_cast<int>(contraction / kStepK);
     g.kblocks = static_cast<int>(d.k_in / 64);
     g.m_tiles = (g.m_total + kPairM - 1) / kPairM;
-    g.splits = L.splits[p];
+    g.splits = L.slots[p];
     if (g.splits > 1) g.partial = reinterpret_cast<float*>(ws + L.part_base[p]);
     ok = ok && encode_tma_2d(&g.map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.act, contraction, T,
                          contraction * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -1134,7 +1280,9 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
       const GemmProblem& g = P.prob[p];
       if (g.splits <= 1) continue;
       for (int tt = 0; tt < t_tiles; ++tt)
-        for (int mt = 0; mt < g.m_tiles; ++mt)
+        for (int mt = 0; mt < g.m_tiles; ++mt) {
+          const auto it = nseg.find({p, tt, mt});
+          if (it == nseg.end()) continue;  // a tile in one piece wrote its output directly
           for (int c = 0; c < 2; ++c) {  // the two 128-row halves of the pair's tile
             const int m0 = mt * kPairM + c * kTileM;
             if (m0 >= g.m_total) continue;
@@ -1146,8 +1294,9 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
             }
             const int tile = (tt * g.m_tiles + mt) * 2 + c;
             R.tile[R.n_tiles++] = {g.partial + static_cast<int64_t>(tile) * g.splits * kTileM * BN,
-                                   g.out, m0, tt * BN, g.m_total, g.splits};
+                                   g.out, m0, tt * BN, g.m_total, it->second};
           }
+        }
     }
     if (e == cudaSuccess && R.n_tiles)
       e = launch_pdl(lora_splitk_reduce, dim3(R.n_tiles * (BN / kReduceTok)), dim3(128), 0, st, R);
