@@ -321,6 +321,27 @@ size_t lora_group_fwd_workspace(const hsnf4_lora_fwd_args* probs, int n, int64_t
   return L.total;
 }
 
+int hsnf4_gemm_plan(int mode, const int64_t* n_out, const int64_t* k_in, int n, int64_t T,
+                    int r, hsnf4_gemm_plan_info* out) {
+  if (!n_out || !k_in || !out)
+    return fail(HSNF4_ERR_INVALID, "hsnf4_gemm_plan: NULL argument");
+  if (mode != 0 && mode != 1)
+    return fail(HSNF4_ERR_INVALID, "hsnf4_gemm_plan: mode %d (0 forward, 1 dX)", mode);
+  if (n < 1 || n > 8 || T < 1 || r < 1 || r > 64)
+    return fail(HSNF4_ERR_INVALID, "hsnf4_gemm_plan: n=%d T=%lld r=%d", n, (long long)T, r);
+  GemmProblemDesc d[8] = {};
+  for (int i = 0; i < n; ++i) {
+    if (n_out[i] < 64 || k_in[i] < 64 || n_out[i] % 64 || k_in[i] % 64)
+      return fail(HSNF4_ERR_INVALID, "hsnf4_gemm_plan: problem %d: %lld x %lld", i,
+                  (long long)n_out[i], (long long)k_in[i]);
+    d[i].n_out = n_out[i];
+    d[i].k_in = k_in[i];
+  }
+  const int rc = check_gemm_tokens(mode == 0 ? kGemmFwd : kGemmDx, T, r);
+  if (rc) return rc;
+  return gemm_plan_info(mode == 0 ? kGemmFwd : kGemmDx, d, n, T, r, out);
+}
+
 size_t lora_group_bwd_workspace(const hsnf4_lora_bwd_args* probs, int n, int64_t T, int r) {
   if (!probs || n < 1 || n > 8 || T < 1 || r < 1) return 0;
   BwdLayout L;

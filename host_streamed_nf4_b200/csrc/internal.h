@@ -98,6 +98,8 @@ struct GemmProblemDesc {
   bool dense;  // codes is a bf16 [n_out, k_in] weight (no absmax, no dequant)
 };
 size_t gemm_workspace_bytes(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r);
+int gemm_plan_info(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r,
+                   hsnf4_gemm_plan_info* out);
 // HSNF4_OK if the fused GEMM takes T tokens at rank r in this mode (a tiling
 // fits shared memory and T spans at most 64 token tiles); else the error,
 // recorded.  Needs only the sizes, so callers check it before any launch.

@@ -50,6 +50,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <array>
 #include <climits>
 #include <cstddef>
 #include <map>
@@ -1093,6 +1094,137 @@ size_t gemm_workspace_bytes(GemmMode mode, const GemmProblemDesc* probs, int n, 
   return cached_plan(mode, probs, n, T, tl.BN).need;
 }
 
+// The launch's work units per CTA pair, in order: (unit code, K range) of
+// each.  nseg: the K pieces of each tile cut into several (problem, token
+// tile, row tile).  HSNF4_OK or the error, recorded.
+using PairUnits = std::vector<std::vector<std::pair<uint32_t, uint32_t>>>;
+using TilePieces = std::map<std::tuple<int, int, int>, int>;
+
+static int build_units(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int BN,
+                       const GemmPlan& L, PairUnits* per, TilePieces* nseg) {
+  std::vector<int64_t> mt_n, nks;
+  int t_tiles_p = 0;
+  plan_dims(mode, probs, n, T, BN, &mt_n, &nks, &t_tiles_p);
+  for (int p = 0; p < n; ++p)
+    if (mt_n[p] > (1 << 18) || nks[p] >= (1 << 15))
+      return fail(HSNF4_ERR_INVALID, "lora gemm: problem %d exceeds the tile index range", p);
+
+  const int sms = sm_count();
+  const int t_tiles = t_tiles_p;
+  per->clear();
+  nseg->clear();
+  if (L.stream_k) {
+    std::vector<Segment> segs;
+    const int G = plan_pairs(sms);
+    if (streamk_segments(mt_n, nks, t_tiles, BN, G, sms, &segs) == INT64_MAX)
+      return fail(HSNF4_ERR_INVALID, "lora gemm: no stream-K plan within the unit limit");
+    per->assign(G, {});
+    for (const Segment& sg : segs) {
+      (*per)[sg.pair].push_back({pack_unit(sg.p, sg.seg, sg.tt, sg.mt),
+                              pack_unit_k(sg.kb0, sg.kb1, sg.nseg > 1)});
+      if (sg.nseg > 1) (*nseg)[{sg.p, sg.tt, sg.mt}] = sg.nseg;
+    }
+  } else {
+    // units, longest first, each to the least loaded pair so far
+    struct U {
+      int64_t cost;
+      uint32_t code, k;
+    };
+    std::vector<U> units;
+    for (int p = 0; p < n; ++p) {
+      const int S = L.splits[p];
+      for (int sp = 0; sp < S; ++sp) {
+        const int kb0 = static_cast<int>(sp * nks[p] / S);
+        const int kb1 = static_cast<int>((sp + 1) * nks[p] / S);
+        const int64_t cost = unit_cost(kb1 - kb0, S);
+        for (int tt = 0; tt < t_tiles; ++tt)
+          for (int mt = 0; mt < mt_n[p]; ++mt) {
+            units.push_back({cost, pack_unit(p, sp, tt, mt), pack_unit_k(kb0, kb1, S > 1)});
+            if (S > 1) (*nseg)[{p, tt, mt}] = S;
+          }
+      }
+    }
+    if (units.size() > static_cast<size_t>(kMaxUnits))
+      return fail(HSNF4_ERR_INVALID, "lora gemm: %zu work units exceed the per-launch limit %d",
+                  units.size(), kMaxUnits);
+    std::stable_sort(units.begin(), units.end(),
+                     [](const U& a, const U& b) { return a.cost > b.cost; });
+    // persistent CTA pairs: one per two SMs
+    const int G = static_cast<int>(std::min<size_t>(units.size(), plan_pairs(sms)));
+    per->assign(G, {});
+    using Load = std::pair<int64_t, int>;
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+    for (int c = 0; c < G; ++c) heap.push({0, c});
+    for (const U& u : units) {
+      Load top = heap.top();
+      heap.pop();
+      (*per)[top.second].push_back({u.code, u.k});
+      heap.push({top.first + u.cost, top.second});
+    }
+  }
+  return HSNF4_OK;
+}
+
+// Work-plan introspection (hsnf4_gemm_plan): the launch's units decoded
+// back and checked, every tile's K range covered once by pieces in order.
+int gemm_plan_info(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r,
+                   hsnf4_gemm_plan_info* out) {
+  Tiling tl;
+  if (!choose_tiling(mode, T, (r + 15) / 16 * 16, &tl))
+    return fail(HSNF4_ERR_INVALID, "lora gemm: no tiling fits shared memory (T=%lld, r=%d)",
+                (long long)T, r);
+  const GemmPlan L = cached_plan(mode, probs, n, T, tl.BN);
+  PairUnits per;
+  TilePieces nseg;
+  const int rc = build_units(mode, probs, n, T, tl.BN, L, &per, &nseg);
+  if (rc != HSNF4_OK) return rc;
+  std::vector<int64_t> mt_n, nks;
+  int t_tiles = 0;
+  plan_dims(mode, probs, n, T, tl.BN, &mt_n, &nks, &t_tiles);
+  memset(out, 0, sizeof *out);
+  out->stream_k = L.stream_k ? 1 : 0;
+  out->pairs = static_cast<int32_t>(per.size());
+  out->split_tiles = static_cast<int32_t>(nseg.size());
+  out->min_pair_steps = INT64_MAX;
+  // tile -> its pieces (segment index, kb0, kb1, writes a partial)
+  std::map<std::tuple<int, int, int>, std::vector<std::array<int, 4>>> pieces;
+  for (const auto& pair : per) {
+    int64_t steps = 0;
+    for (const auto& uk : pair) {
+      const uint32_t u = uk.first, kk = uk.second;
+      const int p = static_cast<int>(u >> 29), seg = static_cast<int>((u >> 24) & 31);
+      const int tt = static_cast<int>((u >> 18) & 63), mt = static_cast<int>(u & 0x3FFFF);
+      const int kb0 = static_cast<int>(kk & 0x7FFF), kb1 = static_cast<int>((kk >> 15) & 0x7FFF);
+      pieces[{p, tt, mt}].push_back({seg, kb0, kb1, static_cast<int>((kk >> 30) & 1)});
+      steps += kb1 - kb0;
+      out->units += 1;
+    }
+    out->total_steps += steps;
+    out->max_pair_steps = std::max(out->max_pair_steps, steps);
+    out->min_pair_steps = std::min(out->min_pair_steps, steps);
+  }
+  bool ok = true;
+  int64_t tiles = 0;
+  for (int p = 0; p < n; ++p) tiles += mt_n[p] * t_tiles;
+  ok = ok && static_cast<int64_t>(pieces.size()) == tiles;
+  for (auto& kv : pieces) {
+    auto& v = kv.second;
+    std::sort(v.begin(), v.end());
+    const int np = static_cast<int>(v.size());
+    const auto it = nseg.find(kv.first);
+    ok = ok && (np > 1 ? (it != nseg.end() && it->second == np) : it == nseg.end());
+    int kb = 0;
+    for (int i = 0; i < np; ++i) {
+      ok = ok && v[i][0] == i && v[i][1] == kb && v[i][2] > v[i][1] && v[i][3] == (np > 1);
+      kb = v[i][2];
+    }
+    ok = ok && kb == nks[std::get<0>(kv.first)];
+  }
+  out->covered = ok ? 1 : 0;
+  if (out->min_pair_steps == INT64_MAX) out->min_pair_steps = 0;
+  return HSNF4_OK;
+}
+
 int check_gemm_tokens(GemmMode mode, int64_t T, int r) {
   Tiling tl;
   if (!choose_tiling(mode, T, (r + 15) / 16 * 16, &tl))
@@ -1145,65 +1277,11 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     return fail(HSNF4_ERR_OOM, "lora gemm: workspace too small: need %zu bytes, given %zu",
                 L.need, ws_bytes);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  std::vector<int64_t> mt_n, nks;
-  int t_tiles_p = 0;
-  plan_dims(mode, probs, n, T, BN, &mt_n, &nks, &t_tiles_p);
-  for (int p = 0; p < n; ++p)
-    if (mt_n[p] > (1 << 18) || nks[p] >= (1 << 15))
-      return fail(HSNF4_ERR_INVALID, "lora gemm: problem %d exceeds the tile index range", p);
-
-  // per pair: the (unit code, K range) of its work units, in order
-  std::vector<std::vector<std::pair<uint32_t, uint32_t>>> per;
-  // K segments of each tile that writes partials: (problem, token tile, row tile) -> count
-  std::map<std::tuple<int, int, int>, int> nseg;
-  if (L.stream_k) {
-    std::vector<Segment> segs;
-    const int G = plan_pairs(sms);
-    if (streamk_segments(mt_n, nks, t_tiles, BN, G, sms, &segs) == INT64_MAX)
-      return fail(HSNF4_ERR_INVALID, "lora gemm: no stream-K plan within the unit limit");
-    per.assign(G, {});
-    for (const Segment& sg : segs) {
-      per[sg.pair].push_back({pack_unit(sg.p, sg.seg, sg.tt, sg.mt),
-                              pack_unit_k(sg.kb0, sg.kb1, sg.nseg > 1)});
-      if (sg.nseg > 1) nseg[{sg.p, sg.tt, sg.mt}] = sg.nseg;
-    }
-  } else {
-    // units, longest first, each to the least loaded pair so far
-    struct U {
-      int64_t cost;
-      uint32_t code, k;
-    };
-    std::vector<U> units;
-    for (int p = 0; p < n; ++p) {
-      const int S = L.splits[p];
-      for (int sp = 0; sp < S; ++sp) {
-        const int kb0 = static_cast<int>(sp * nks[p] / S);
-        const int kb1 = static_cast<int>((sp + 1) * nks[p] / S);
-        const int64_t cost = unit_cost(kb1 - kb0, S);
-        for (int tt = 0; tt < t_tiles; ++tt)
-          for (int mt = 0; mt < mt_n[p]; ++mt) {
-            units.push_back({cost, pack_unit(p, sp, tt, mt), pack_unit_k(kb0, kb1, S > 1)});
-            if (S > 1) nseg[{p, tt, mt}] = S;
-          }
-      }
-    }
-    if (units.size() > static_cast<size_t>(kMaxUnits))
-      return fail(HSNF4_ERR_INVALID, "lora gemm: %zu work units exceed the per-launch limit %d",
-                  units.size(), kMaxUnits);
-    std::stable_sort(units.begin(), units.end(),
-                     [](const U& a, const U& b) { return a.cost > b.cost; });
-    // persistent CTA pairs: one per two SMs
-    const int G = static_cast<int>(std::min<size_t>(units.size(), plan_pairs(sms)));
-    per.assign(G, {});
-    using Load = std::pair<int64_t, int>;
-    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
-    for (int c = 0; c < G; ++c) heap.push({0, c});
-    for (const U& u : units) {
-      Load top = heap.top();
-      heap.pop();
-      per[top.second].push_back({u.code, u.k});
-      heap.push({top.first + u.cost, top.second});
-    }
+  PairUnits per;
+  TilePieces nseg;
+  {
+    const int rc = build_units(mode, probs, n, T, BN, L, &per, &nseg);
+    if (rc != HSNF4_OK) return rc;
   }
   const int G = static_cast<int>(per.size());
   int k = 0;

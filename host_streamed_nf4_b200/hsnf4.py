@@ -68,6 +68,14 @@ class KernelTime(Structure):
                 ("work", ctypes.c_double)]
 
 
+class GemmPlanInfo(Structure):
+    _fields_ = [("stream_k", ctypes.c_int32), ("pairs", ctypes.c_int32),
+                ("units", ctypes.c_int32), ("split_tiles", ctypes.c_int32),
+                ("total_steps", c_int64), ("max_pair_steps", c_int64),
+                ("min_pair_steps", c_int64), ("covered", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
 class HsNf4Error(RuntimeError):
     def __init__(self, status: int, detail: str):
         super().__init__(f"[{status}] {detail}")
@@ -117,6 +125,8 @@ _SIGS = {
                          c_void_p], c_int),
     "lora_linear_fwd_noalloc": ([POINTER(Nf4WeightC), c_void_p, c_int64, c_void_p, c_void_p, c_int,
                                  c_float, c_void_p, c_void_p, c_void_p], c_int),
+    "hsnf4_gemm_plan": ([c_int, POINTER(c_int64), POINTER(c_int64), c_int, c_int64, c_int,
+                         POINTER(GemmPlanInfo)], c_int),
     "lora_group_fwd_workspace": ([POINTER(FwdArgs), c_int, c_int64, c_int], c_size_t),
     "lora_group_bwd_workspace": ([POINTER(BwdArgs), c_int, c_int64, c_int], c_size_t),
     "lora_group_fwd": ([POINTER(FwdArgs), c_int, c_int64, c_int, c_float, c_void_p, c_size_t,
@@ -226,6 +236,18 @@ def profile(enable: bool, kinds=None):
         _check(lib().hsnf4_profile_kinds(mask))
     else:
         _check(lib().hsnf4_profile(int(bool(enable))))
+
+
+def gemm_plan(mode: str, shapes, T: int, r: int) -> dict:
+    """The fused GEMM's work plan for a group of (n_out, k_in) shapes (host
+    only): mode "fwd" or "dx"."""
+    n = len(shapes)
+    n_out = (c_int64 * n)(*[s[0] for s in shapes])
+    k_in = (c_int64 * n)(*[s[1] for s in shapes])
+    info = GemmPlanInfo()
+    _check(lib().hsnf4_gemm_plan({"fwd": 0, "dx": 1}[mode], n_out, k_in, n, T, r,
+                                 ctypes.byref(info)))
+    return {f[0]: getattr(info, f[0]) for f in GemmPlanInfo._fields_ if f[0] != "reserved"}
 
 
 def profile_read() -> dict:

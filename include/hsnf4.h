@@ -321,6 +321,29 @@ size_t lora_group_bwd_workspace(const hsnf4_lora_bwd_args *probs, int n, int64_t
 
 int lora_group_fwd(const hsnf4_lora_fwd_args *probs, int n, int64_t T, int r, float alpha,
                    void *workspace, size_t ws_bytes, void *stream);
+
+/* The fused GEMM's work plan for a group, built exactly as a launch builds
+ * it, from the shapes alone (host only; no device memory, no GPU needed):
+ * n problems of n_out[i] x k_in[i] weights at T tokens and rank r, mode 0
+ * (forward; contraction k_in) or 1 (dX; contraction n_out).  A plan cuts the
+ * 256-row x up-to-512-token tiles' K ranges (64-step units) into pieces
+ * spread over CTA pairs: longest-first over uniform splits, or stream-K
+ * (equal shares of all K steps per pair).  `covered` is 1 when every tile's
+ * K range is covered once by pieces in order.  Errors: INVALID. */
+typedef struct {
+  int32_t stream_k;        /* 1: stream-K plan; 0: longest-first over uniform K splits */
+  int32_t pairs;           /* CTA pairs given work */
+  int32_t units;           /* work units (K pieces) */
+  int32_t split_tiles;     /* tiles cut into several pieces (each piece writes a partial) */
+  int64_t total_steps;     /* 64-wide K steps over all units */
+  int64_t max_pair_steps;  /* the most K steps any pair runs */
+  int64_t min_pair_steps;
+  int32_t covered;
+  int32_t reserved;
+} hsnf4_gemm_plan_info;
+
+int hsnf4_gemm_plan(int mode, const int64_t *n_out, const int64_t *k_in, int n, int64_t T,
+                    int r, hsnf4_gemm_plan_info *out);
 int lora_group_bwd(const hsnf4_lora_bwd_args *probs, int n, int64_t T, int r, float alpha,
                    void *workspace, size_t ws_bytes, void *stream);
 
