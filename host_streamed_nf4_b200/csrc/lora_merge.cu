@@ -16,9 +16,10 @@
 // memory.  Two warpgroups then expand the tile, each thread one row of 64
 // columns: it reads its product row back from tensor memory 16 columns at a
 // time, expands the matching base bytes, adds, rounds and writes the bf16
-// row into a 128B-swizzled staging box that one thread per warpgroup stores
-// with TMA.  HBM traffic is the base read once plus W' written once; several
-// CTAs per SM keep loads and stores in flight.
+// row into a 128B-swizzled staging box; each warp stores its own 32 rows
+// with TMA as soon as it has written them, so no warp waits for another's
+// rows or stores.  HBM traffic is the base read once plus W' written once;
+// several CTAs per SM keep loads and stores in flight.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -55,31 +56,12 @@ struct MrgCfg {
 constexpr int kMrgCols = 16;  // columns per TMEM read of the expanding loop (8 or 16)
 static_assert(kMrgCols == 8 || kMrgCols == 16, "TMEM read width");
 
-__device__ __forceinline__ void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-// named barrier that also ANDs a predicate over its n threads, so that a
-// group leaving its loop on a failed wait leaves it together
-__device__ __forceinline__ bool named_sync_and_mrg(int id, int n, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, %2, %3, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-
 struct MergeParams {
   CUtensorMap map_base;  // NF4: codes uint8 [N, K/2], box {64, 128}, 64B swizzle
                          // dense: bf16 [N, K], box {64, 128}, 128B swizzle (two per tile)
   CUtensorMap map_a;     // A bf16 [r, K], box {64, r_pad}, 128B swizzle (MN-major operand)
   CUtensorMap map_b;     // B bf16 [N, r], box {16, 128}, 32B swizzle (K-major operand)
-  CUtensorMap map_out;   // W' bf16 [N, K], box {64, 128}, 128B swizzle
+  CUtensorMap map_out;   // W' bf16 [N, K], box {64, 32} (one warp's rows), 128B swizzle
   const float* absmax;   // NF4 only: fp32 [N, K/64]
   int64_t N, K;
   int r_pad, dense, col_tiles, row_tiles;
@@ -111,8 +93,8 @@ static_assert(kMrgExpand == 256, "two warpgroups expand the tile");
 // tile into the other stage while the current one is processed; warp 1
 // issues each tile's MMAs into a TMEM accumulator (MrgCfg: one or two per
 // CTA); warps 2..9 (two warpgroups, one row of the tile per thread) expand
-// it into staging boxes (one or two per warpgroup) that TMA stores write
-// out while the next tile is expanded.
+// it into staging boxes (one or two per warpgroup), each warp's 32 rows
+// written out by a TMA store of its own while the next tile is expanded.
 template <bool DENSE>
 __global__ void __launch_bounds__(kMrgThreads, MrgCfg<DENSE>::kCtasPerSm)
     lora_merge_kernel(const __grid_constant__ MergeParams P) {
@@ -209,11 +191,10 @@ __global__ void __launch_bounds__(kMrgThreads, MrgCfg<DENSE>::kCtasPerSm)
   } else {
     // ---------------------------------------------- expand, add, round, store
     // warpgroup h (warps 2..5 or 6..9) takes columns 64 h .. 64 h + 63, one
-    // row of the tile per thread, and stores its own 64-column box
+    // row of the tile per thread; each warp stores its 32 rows of them
     const int h = (warp - 2) >> 2;
     const int q4 = warp & 3;           // TMEM lane quarter of this warp
     const int tid = q4 * 32 + lane;    // this thread's row of the tile
-    const int et = (threadIdx.x - 64) & 127;  // 0 issues the warpgroup's stores
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     // this row's absmax for the warpgroup's block of a tile, loaded one tile ahead
     auto absmax_of = [&](int tile) -> float {
@@ -232,9 +213,11 @@ __global__ void __launch_bounds__(kMrgThreads, MrgCfg<DENSE>::kCtasPerSm)
       const int n0 = (tile / P.col_tiles) * kMrgTile, k0 = (tile % P.col_tiles) * kMrgTile;
       ok = mbar_wait(&st_full[s], (li >> 1) & 1, abort_p, &g_merge_flags, kMrgFlagMma) &&
            mbar_wait(&acc_full[b], (li / kMrgAccBufs) & 1, abort_p, &g_merge_flags, kMrgFlagMma);
-      // the staging box this tile writes has been read by its earlier store
-      if (et == 0) bulk_wait_group_read<kMrgOutBufs - 1>();
-      if (!named_sync_and_mrg(1 + h, 128, ok)) break;
+      // the staging rows this warp writes have been read by its earlier store
+      // (issued by the same lane); a warp leaving on a failed wait leaves whole
+      if (lane == 0) bulk_wait_group_read<kMrgOutBufs - 1>();
+      if (!__all_sync(0xffffffffu, ok)) break;
+      __syncwarp();
       tc_fence_after();
       const uint8_t* st = smem + s * L.stage;
       uint8_t* out_box = smem + L.out + ob * 32768 + h * 16384;
@@ -301,13 +284,14 @@ __global__ void __launch_bounds__(kMrgThreads, MrgCfg<DENSE>::kCtasPerSm)
       mbar_arrive(&acc_empty[b]);            // the accumulator is read
       if (DENSE) mbar_arrive(&st_empty[s]);  // and this row of the base
       fence_proxy_async_smem();
-      named_sync(1 + h, 128);
-      if (et == 0) {
-        if (k0 + 64 * h < P.K) tma_store_2d(&P.map_out, out_box, k0 + 64 * h, n0);
+      __syncwarp();
+      if (lane == 0) {
+        if (k0 + 64 * h < P.K && n0 + 32 * q4 < P.N)
+          tma_store_2d(&P.map_out, out_box + q4 * 4096, k0 + 64 * h, n0 + 32 * q4);
         bulk_commit_group();
       }
     }
-    if (et == 0) bulk_wait_group_read<0>();  // the stores have read their staging boxes
+    if (lane == 0) bulk_wait_group_read<0>();  // the stores have read their staging boxes
   }
 
   __syncthreads();  // every thread sees the final abort word
@@ -355,7 +339,7 @@ cudaError_t launch_lora_merge(const void* base, const float* absmax, bool dense,
   ok = ok && encode_tma_2d(&P.map_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, r, N,
                            static_cast<uint64_t>(r) * 2, 16, kMrgTile, CU_TENSOR_MAP_SWIZZLE_32B);
   ok = ok && encode_tma_2d(&P.map_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, K, N, K * 2, 64,
-                           kMrgTile, CU_TENSOR_MAP_SWIZZLE_128B);
+                           32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
   const int smem = merge_smem(P.dense, P.r_pad).total + 1024;
   static cudaError_t attr_rc = cudaSuccess;
