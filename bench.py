@@ -608,32 +608,49 @@ def cublas_probe(fam, T, kernel, dev, reps=10):
 def merge_roofline(stack, dev):
     """lora_merge (merge_and_unload) of the layer's largest projection, timed
     with CUDA events on the launch stream, against the measured HBM copy
-    rate: algorithmic bytes are the base read plus the bf16 W' written."""
+    rate: algorithmic bytes are the base read plus the bf16 W' written.
+    Launches rotate over base/output sets that together hold at least 4x the
+    L2 capacity, so no launch finds its base, or dirty lines of its output,
+    still in L2."""
+    import math
+
     import torch
 
     from host_streamed_nf4_b200 import hsnf4
     p = max(range(len(stack.projs)), key=lambda i: stack.projs[i][1] * stack.projs[i][2])
     _, n, k = stack.projs[p]
-    keep = W = stack.device_weight(0, p)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    base_bytes = n * k * 2 if stack.base == "bf16" else n * k // 2 + n * k // 16
+    set_bytes = base_bytes + n * k * 2
+    n_sets = max(2, math.ceil(4 * l2 / set_bytes))
+    W0 = stack.device_weight(0, p)
     A, B = stack.A[0][p], stack.B[0][p]
-    out = torch.empty(n, k, dtype=torch.bfloat16, device=dev)
-    for _ in range(3):
+    sets = []
+    for _ in range(n_sets):
+        W = (hsnf4.Bf16Weight(W0.w.clone()) if stack.base == "bf16" else
+             hsnf4.Nf4Weight(W0.codes.clone(), W0.absmax.clone(), n, k))
+        sets.append((W, torch.empty(n, k, dtype=torch.bfloat16, device=dev)))
+    del W0
+    for W, out in sets:
         hsnf4.lora_merge(W, A, B, stack.alpha, out=out)
     torch.cuda.synchronize(dev)
+    reps = max(10, 2 * n_sets)
     hsnf4.profile(True)
     busy_ahead()
-    for _ in range(10):
+    for i in range(reps):
+        W, out = sets[i % n_sets]
         hsnf4.lora_merge(W, A, B, stack.alpha, out=out)
     torch.cuda.synchronize(dev)
     d = hsnf4.profile_read()["lora_merge"]
     hsnf4.profile(False)
+    del sets
     hbm, _, _, src = measured_peaks()
     gbs = d["work"] / (d["total_ms"] / 1e3) / 1e9
-    del keep, out
     return {"bound": "hbm", "shape": [n, k], "base": stack.base, "achieved": round(gbs, 1),
             "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
             "bytes_per_launch": int(d["work"] / d["launches"]),
             "avg_launch_us": round(d["total_ms"] / d["launches"] * 1e3, 2),
+            "rotation": {"sets": n_sets, "bytes": n_sets * set_bytes, "l2_bytes": l2},
             "peak_source": f"{src} hbm_gbs (copy read+write)"}
 
 
