@@ -53,7 +53,10 @@ struct MrgCfg {
   static constexpr int kCtasPerSm = DENSE ? 2 : 3;
   static_assert(kAccBufs * kMrgTile * kCtasPerSm <= 512, "TMEM columns per SM");
 };
-constexpr int kMrgCols = 16;  // columns per TMEM read of the expanding loop (8 or 16)
+// columns per TMEM read of the expanding loop (8 or 16).  8: the NF4
+// instance fits the 64 registers a thread has at three CTAs per SM without
+// spilling (16 spilled one register and ran 3-4% slower).
+constexpr int kMrgCols = 8;
 static_assert(kMrgCols == 8 || kMrgCols == 16, "TMEM read width");
 
 struct MergeParams {
