@@ -227,9 +227,10 @@ static int check_group(const char* fn, int n, int64_t T, int r, float alpha) {
 //   [s*t bf16 [T, r_pad] per problem][t fp32 [T, r] per problem without t_save]
 //   [X_d bf16 [T, k_in] per problem with dropout]
 //   [projection partials][GEMM split-K partial tiles]
-// Every byte of it that a call reads was written earlier in the same call
-// (the split-K partials are summed by a separate reduce kernel, not through
-// counters), so nothing in it needs clearing between calls.
+// Nothing in it needs clearing between calls: every byte a call reads was
+// written earlier in the same call, except the GEMM's K-split arrival words,
+// which each launch tags with a fresh 56-bit value (a word holding any other
+// value counts as no arrivals).
 struct FwdLayout {
   size_t zs[8], tscratch[8], xd[8], prj, gemm, total;
 };
@@ -274,7 +275,7 @@ static void fwd_layout(const hsnf4_lora_fwd_args* p, int n, int64_t T, int r, Fw
 //   [X_d bf16 [T, k_in] and its keep-mask bytes [T, k_in / 8] per problem
 //    with dropout]
 //   [projection partials][GEMM split-K partial tiles]
-// As for the forward, every byte read was written earlier in the same call.
+// As for the forward, nothing in it needs clearing between calls.
 struct BwdLayout {
   size_t su[8], u[8], parts[8], xd[8], bits[8], prj, gemm, total;
 };

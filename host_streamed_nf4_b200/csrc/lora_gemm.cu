@@ -29,8 +29,13 @@
 // Work units are (problem, 256-row tile, token tile, K split).  The host
 // assigns them to persistent CTA pairs longest-first (static,
 // deterministic).  A problem whose units are long and few is split along K:
-// each split writes its fp32 tile to workspace and a second pass adds them
-// in split order, so the sum does not depend on timing.
+// each piece writes its fp32 tile to workspace, and the pieces are added in
+// split order, so the sum does not depend on timing.  In a longest-first
+// plan the pieces are among the first units to run: each counts itself on
+// the tile's arrival word, and the last to arrive adds the pieces and writes
+// the output while its pair goes on with later units.  In a stream-K plan a
+// tile's first piece often ends its pair's share, so the pieces are added
+// by lora_splitk_reduce, spread over the whole GPU, after the kernel.
 //
 // CTA roles (15 warps, the same in both CTAs of a pair):
 //   warps 0-3, 4-7   two dequant warpgroups taking alternate K steps: raw
@@ -38,7 +43,9 @@
 //                    layout, one 64-element block (one 128-byte line) per
 //                    thread;
 //   warps 8-11       epilogue: TMEM -> registers -> smem transpose ->
-//                    coalesced bf16 rows of the output (or fp32 partials);
+//                    coalesced bf16 rows of the output (or fp32 partials,
+//                    and in a longest-first plan the sum of a split tile's
+//                    partials by its last piece);
 //   warp 12          TMA producer of the activation tiles and rank-r operands;
 //   warp 13          TMA producer of the raw code tiles;
 //   warp 14          TMEM owner; UMMA issuer of the pair (even CTA) or the
@@ -49,8 +56,12 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <unistd.h>
+
 #include <algorithm>
 #include <array>
+#include <atomic>
+#include <chrono>
 #include <climits>
 #include <cstddef>
 #include <map>
@@ -74,6 +85,7 @@ enum : unsigned int {
   kFlagEpilogue = 16u,
   kFlagDrain = 32u,
   kFlagSelftest = 64u,
+  kFlagArrive = 128u,
 };
 
 constexpr int kTileM = 128;                    // rows of one CTA (W rows or k_in columns)
@@ -98,6 +110,7 @@ struct GemmProblem {
   const float* absmax;
   uint16_t* out;          // bf16 [T, m_total]
   float* partial;         // split-K partial tiles (fp32 [BN tokens][128 rows] each), or null
+  unsigned long long* arrive;  // split problems: one arrival word per 128-row half-tile
   int n_out, k_in, m_total, nk, kblocks, m_tiles;  // m_tiles: 256-row tiles
   int splits;             // partial slots per tile: the most K segments any tile has
 };
@@ -105,6 +118,7 @@ struct GemmProblem {
 constexpr int kMaxProblems = 8;
 constexpr int kMaxPairs = 80;
 constexpr int kMaxUnits = 2560;
+constexpr int kMaxSplits = 8;  // pieces of one tile at most (the planners' limit)
 
 struct GemmParams {
   GemmProblem prob[kMaxProblems];
@@ -114,8 +128,14 @@ struct GemmParams {
               // overlaps the next unit's MMAs) or 1 (BN = 512 fills TMEM)
   int dense;  // 1: map_codes is the bf16 weight, TMA-loaded straight into the A ring
   uint16_t pair_off[kMaxPairs + 1];  // units of pair c: units[pair_off[c] .. pair_off[c+1])
-  uint32_t units[kMaxUnits];   // problem(3) | K segment(5) | token tile(6) | row tile(18)
+  // problem(3) | K segment(3) | pieces of the tile - 1 (3) | the tile's last
+  // piece adds the pieces (1; else lora_splitk_reduce does, after the
+  // kernel) | token tile(6) | row tile(16)
+  uint32_t units[kMaxUnits];
   uint32_t unit_k[kMaxUnits];  // first K step(15) | end K step(15) | writes a partial(1)
+  // this launch's tag of the arrival words (56 bits, never reused in the
+  // process; a word holding another tag counts as no arrivals)
+  unsigned long long token;
 };
 static_assert(sizeof(GemmParams) <= 32764, "kernel parameter block");
 
@@ -125,25 +145,36 @@ __host__ __device__ inline uint32_t pack_unit_k(int kb0, int kb1, bool partial) 
 }
 
 __host__ __device__ inline uint32_t pack_unit(int p, int s, int tt, int mt) {
-  return (static_cast<uint32_t>(p) << 29) | (static_cast<uint32_t>(s) << 24) |
-         (static_cast<uint32_t>(tt) << 18) | static_cast<uint32_t>(mt);
+  return (static_cast<uint32_t>(p) << 29) | (static_cast<uint32_t>(s) << 26) |
+         (static_cast<uint32_t>(tt) << 16) | static_cast<uint32_t>(mt);
 }
+// the pieces of the unit's tile and whether its last piece adds them
+__host__ __device__ inline uint32_t with_pieces(uint32_t u, int nseg, bool fixup) {
+  return u | (static_cast<uint32_t>(nseg - 1) << 23) | (fixup ? (1u << 22) : 0u);
+}
+__host__ __device__ inline int unit_problem(uint32_t u) { return static_cast<int>(u >> 29); }
+__host__ __device__ inline int unit_segment(uint32_t u) { return static_cast<int>((u >> 26) & 7); }
+__host__ __device__ inline int unit_tt(uint32_t u) { return static_cast<int>((u >> 16) & 63); }
+__host__ __device__ inline int unit_mt(uint32_t u) { return static_cast<int>(u & 0xFFFF); }
 
 // A work unit: one K segment [kb0, kb1) of one (problem, token tile, 256-row
-// tile).  A tile cut into several segments has each write an fp32 partial
-// (slot `split` of the tile) that a second pass adds in segment order.
+// tile).  A tile cut into nseg segments has each write an fp32 partial
+// (slot `split` of the tile); the nseg partials are added in segment order
+// by the last of them to finish (longest-first plans) or by a second pass.
 struct Unit {
-  int p, split, tt, mt, kb0, kb1;
-  bool partial;
+  int p, split, tt, mt, kb0, kb1, nseg;
+  bool partial, fixup;
 };
 
 __device__ __forceinline__ Unit unpack_unit(const GemmParams& P, int ui) {
   const uint32_t u = P.units[ui], k = P.unit_k[ui];
   Unit r;
-  r.p = u >> 29;
-  r.split = (u >> 24) & 31;
-  r.tt = (u >> 18) & 63;
-  r.mt = u & 0x3FFFF;
+  r.p = unit_problem(u);
+  r.split = unit_segment(u);
+  r.tt = unit_tt(u);
+  r.mt = unit_mt(u);
+  r.nseg = static_cast<int>((u >> 23) & 7) + 1;
+  r.fixup = ((u >> 22) & 1u) != 0;
   r.kb0 = k & 0x7FFF;
   r.kb1 = (k >> 15) & 0x7FFF;
   r.partial = ((k >> 30) & 1u) != 0;
@@ -210,6 +241,32 @@ struct Ring {
     }
   }
 };
+
+// Counts one piece of a split tile on the tile's arrival word: the word
+// holds this launch's token in its high 56 bits and the pieces counted so
+// far in its low 8; a word holding another token (memory never written, or
+// a launch that stopped early) counts as none.  The piece that completes
+// the count gets true and clears the word, so a completed launch leaves
+// every word 0 (a replayed graph reuses its token).  Every failed
+// compare-and-swap means another piece was counted, so at most nseg - 1
+// attempts fail.
+__device__ __forceinline__ bool piece_arrive(unsigned long long* w, unsigned long long token,
+                                             int nseg) {
+  const unsigned long long tag = token << 8;
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(w);
+  for (int attempt = 0; attempt <= 2 * kMaxSplits; ++attempt) {
+    const unsigned long long nxt = (cur & ~0xFFull) == tag ? cur + 1 : (tag | 1ull);
+    const unsigned long long prev = atomicCAS(w, cur, nxt);
+    if (prev == cur) {
+      if ((nxt & 0xFFull) != static_cast<unsigned long long>(nseg)) return false;
+      atomicExch(w, 0ull);
+      return true;
+    }
+    cur = prev;
+  }
+  atomicOr(&g_gemm_flags, kFlagArrive);
+  return false;
+}
 
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -625,11 +682,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // this CTA's 128-row half of the unit's tile
       const int tile = (U.tt * pr.m_tiles + U.mt) * 2 + static_cast<int>(crank);
       if (U.partial) {
-        // this split's fp32 tile -> workspace, token-major ([BN][128]) so that a
-        // warp's 32 rows of one token are 128 contiguous bytes; the splits are
-        // added in split order by lora_splitk_reduce after this kernel
-        float* mine = pr.partial +
-                      (static_cast<int64_t>(tile) * pr.splits + U.split) * kTileM * BN + i;
+        // this piece's fp32 tile -> workspace, token-major ([BN][128]) so that
+        // a warp's 32 rows of one token are 128 contiguous bytes
+        float* const slots = pr.partial + static_cast<int64_t>(tile) * pr.splits * kTileM * BN + i;
+        float* const mine = slots + static_cast<int64_t>(U.split) * kTileM * BN;
         for (int c = 0; c < BN; c += 16) {
           uint32_t v[16];
           tmem_ld16(acc0 + static_cast<uint32_t>(c), v);
@@ -640,6 +696,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[buf]);
+        // Once every thread's rows are visible at device scope, thread 0
+        // counts the piece on this half-tile's arrival word; the piece that
+        // completes the count adds the tile's pieces in split order (their
+        // rows read from L2) and writes the bf16 output like a whole tile.
+        // Halves wholly past the output's edge have nothing to write.
+        if (!U.fixup || m0 >= pr.m_total) continue;
+        __threadfence();
+        named_sync(1, 128);
+        const int nseg = U.nseg;
+        bool last = true;
+        if (i == 0) {
+          last = piece_arrive(pr.arrive + tile, P.token, nseg);
+          __threadfence();
+        }
+        if (!named_sync_and(1, 128, last)) continue;
+        for (int c = 0; c < BN; c += 32) {
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __ldcg(slots + static_cast<int64_t>(c + j) * kTileM);
+          for (int sp = 1; sp < nseg; ++sp) {
+            const float* q = slots + static_cast<int64_t>(sp) * kTileM * BN;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += __ldcg(q + static_cast<int64_t>(c + j) * kTileM);
+          }
+          uint16_t* sb = stage + (epi_step & 1) * 2 * kStageElems;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const __nv_bfloat16 b = __float2bfloat16_rn(v[j]);
+            sb[j * kTileM + i] = *reinterpret_cast<const uint16_t*>(&b);
+          }
+          fence_proxy_async_smem();
+          if (i == 0) bulk_wait_group_read<0>();
+          named_sync(1, 128);
+          if (i == 0) {
+            for (int h = 0; h < 2; ++h)
+              if (t0 + c + 16 * h < P.T)
+                tma_store_2d(&pr.map_out, sb + h * kStageElems, m0, t0 + c + 16 * h);
+            bulk_commit_group();
+          }
+          ++epi_step;
+        }
         continue;
       }
       // 32 tokens per step: one TMEM load, a transpose into two 16-token x
@@ -725,7 +822,7 @@ cudaError_t launch_selftest_stall(cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// Adds the K-split partial tiles of every split problem in split order and
+// Adds the K-split partial tiles of a stream-K launch in split order and
 // writes the bf16 outputs.  One CTA per (problem tile, 8-token slice);
 // thread i owns row pair (2i, 2i+1) of the tile.
 struct ReduceTile {
@@ -735,7 +832,6 @@ struct ReduceTile {
 };
 
 constexpr int kReduceTok = 8;
-constexpr int kMaxSplits = 8;  // the split planner's limit
 constexpr int kMaxReduceTiles = 768;  // 32 B each: the parameter block stays < 32 KiB
 
 struct ReduceParams {
@@ -886,8 +982,8 @@ static int64_t lpt_makespan(std::vector<int64_t>& costs, int sms) {
 }
 
 // The LPT plan's objective for K splits `sp` (per problem): the simulated
-// makespan of the longest-first schedule (in K steps) plus the split-K
-// reduce pass, whose partial reads are charged at ~16 KiB per K step per SM.
+// makespan of the longest-first schedule (in K steps) plus the split tiles'
+// partial reads by their last pieces, charged at ~16 KiB per K step per SM.
 static int64_t lpt_objective(const std::vector<int64_t>& tiles, const std::vector<int64_t>& nk,
                              const std::vector<int>& sp, int BN, int sms) {
   std::vector<int64_t> costs;
@@ -1005,7 +1101,7 @@ static int64_t streamk_cut(const std::vector<int64_t>& mt_n, const std::vector<i
           cost[s.pair] += unit_cost(s.kb1 - s.kb0, seg);
         }
         if (seg > 1) reduce_bytes += static_cast<double>(seg) * kPairM * BN * 4;
-        if (seg > kMaxSplits) return INT64_MAX;  // the reduce pass adds at most kMaxSplits
+        if (seg > kMaxSplits) return INT64_MAX;  // a tile's last piece adds at most kMaxSplits
       }
   if (out->size() > static_cast<size_t>(kMaxUnits)) return INT64_MAX;
   const int64_t reduce =
@@ -1021,7 +1117,8 @@ struct GemmPlan {
   std::vector<int> splits;       // LPT: K splits per problem
   std::vector<int> slots;        // partial slots per tile of each problem (1: no partials)
   std::vector<size_t> part_base;
-  size_t need = 0;               // workspace bytes of the partials
+  std::vector<size_t> arrive_base;  // arrival words of the split problems' half-tiles
+  size_t need = 0;               // workspace bytes of the partials and arrival words
 };
 
 static void plan_dims(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int BN,
@@ -1061,10 +1158,13 @@ static GemmPlan make_plan(GemmMode mode, const GemmProblemDesc* probs, int n, in
     for (int p = 0; p < n; ++p) pl.slots[p] = pl.splits[p];
   }
   pl.part_base.assign(n, 0);
+  pl.arrive_base.assign(n, 0);
   for (int p = 0; p < n; ++p) {
     if (pl.slots[p] <= 1) continue;
     pl.part_base[p] = pl.need;
     pl.need += round_up(static_cast<size_t>(tiles[p]) * pl.slots[p] * kPairM * BN * 4, 256);
+    pl.arrive_base[p] = pl.need;
+    pl.need += round_up(static_cast<size_t>(tiles[p]) * 2 * sizeof(unsigned long long), 256);
   }
   return pl;
 }
@@ -1106,7 +1206,7 @@ static int build_units(GemmMode mode, const GemmProblemDesc* probs, int n, int64
   int t_tiles_p = 0;
   plan_dims(mode, probs, n, T, BN, &mt_n, &nks, &t_tiles_p);
   for (int p = 0; p < n; ++p)
-    if (mt_n[p] > (1 << 18) || nks[p] >= (1 << 15))
+    if (mt_n[p] > (1 << 16) || nks[p] >= (1 << 15))
       return fail(HSNF4_ERR_INVALID, "lora gemm: problem %d exceeds the tile index range", p);
 
   const int sms = sm_count();
@@ -1165,6 +1265,44 @@ static int build_units(GemmMode mode, const GemmProblemDesc* probs, int n, int64
   return HSNF4_OK;
 }
 
+// Split tiles whose last piece adds the pieces in the kernel: those whose
+// every piece has at least kFixupCover K steps of cover in its pair -- the
+// pair's later units plus the steps by which the pair finishes before the
+// busiest pair -- so the adding (reads of the other pieces from L2) overlaps
+// other work or idle time.  The others (a stream-K share's first piece, a
+// launch with no more units than pairs) are added by the reduce pass after
+// the kernel.
+using FixupTiles = std::map<std::tuple<int, int, int>, bool>;
+constexpr int64_t kFixupCover = 32;
+
+static int64_t unit_steps(uint32_t kk) {
+  return static_cast<int64_t>((kk >> 15) & 0x7FFF) - static_cast<int64_t>(kk & 0x7FFF);
+}
+
+static FixupTiles fixup_tiles(const PairUnits& per, const TilePieces& nseg) {
+  FixupTiles fixup;
+  for (const auto& kv : nseg) fixup[kv.first] = true;
+  int64_t busiest = 0;
+  for (const auto& pair : per) {
+    int64_t steps = 0;
+    for (const auto& uk : pair) steps += unit_steps(uk.second);
+    busiest = std::max(busiest, steps);
+  }
+  for (const auto& pair : per) {
+    int64_t cover = busiest;  // after the current unit: later units + the pair's slack
+    for (const auto& uk : pair) cover -= unit_steps(uk.second);
+    for (auto it = pair.rbegin(); it != pair.rend(); ++it) {
+      const uint32_t u = it->first, kk = it->second;
+      if ((kk >> 30) & 1u) {
+        const std::tuple<int, int, int> key{unit_problem(u), unit_tt(u), unit_mt(u)};
+        if (cover < kFixupCover) fixup[key] = false;
+      }
+      cover += unit_steps(kk);
+    }
+  }
+  return fixup;
+}
+
 // Work-plan introspection (hsnf4_gemm_plan): the launch's units decoded
 // back and checked, every tile's K range covered once by pieces in order.
 int gemm_plan_info(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r,
@@ -1185,6 +1323,7 @@ int gemm_plan_info(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T
   out->stream_k = L.stream_k ? 1 : 0;
   out->pairs = static_cast<int32_t>(per.size());
   out->split_tiles = static_cast<int32_t>(nseg.size());
+  for (const auto& kv : fixup_tiles(per, nseg)) out->fixup_tiles += kv.second ? 1 : 0;
   out->min_pair_steps = INT64_MAX;
   // tile -> its pieces (segment index, kb0, kb1, writes a partial)
   std::map<std::tuple<int, int, int>, std::vector<std::array<int, 4>>> pieces;
@@ -1192,8 +1331,8 @@ int gemm_plan_info(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T
     int64_t steps = 0;
     for (const auto& uk : pair) {
       const uint32_t u = uk.first, kk = uk.second;
-      const int p = static_cast<int>(u >> 29), seg = static_cast<int>((u >> 24) & 31);
-      const int tt = static_cast<int>((u >> 18) & 63), mt = static_cast<int>(u & 0x3FFFF);
+      const int p = unit_problem(u), seg = unit_segment(u);
+      const int tt = unit_tt(u), mt = unit_mt(u);
       const int kb0 = static_cast<int>(kk & 0x7FFF), kb1 = static_cast<int>((kk >> 15) & 0x7FFF);
       pieces[{p, tt, mt}].push_back({seg, kb0, kb1, static_cast<int>((kk >> 30) & 1)});
       steps += kb1 - kb0;
@@ -1234,6 +1373,24 @@ int check_gemm_tokens(GemmMode mode, int64_t T, int r) {
     return fail(HSNF4_ERR_INVALID, "lora gemm: T=%lld exceeds %d tokens per launch",
                 (long long)T, 64 * tl.BN);
   return HSNF4_OK;
+}
+
+// A tag for the arrival words of one launch: 56 bits, consecutive launches
+// consecutive values from a start drawn once per process, so no two
+// launches of the process share one and a word left by another process or
+// never written matches only by a 2^-56 chance.
+static unsigned long long next_launch_token() {
+  static std::atomic<unsigned long long> next{0};
+  static const unsigned long long start = [] {
+    unsigned long long z = static_cast<unsigned long long>(
+        std::chrono::steady_clock::now().time_since_epoch().count()) ^
+        (static_cast<unsigned long long>(getpid()) << 32) ^
+        reinterpret_cast<uintptr_t>(&next);
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;  // splitmix64 finaliser
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+  }();
+  return (start + next.fetch_add(1)) & ((1ull << 56) - 1);
 }
 
 int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, int64_t T, int r,
@@ -1284,6 +1441,9 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     if (rc != HSNF4_OK) return rc;
   }
   const int G = static_cast<int>(per.size());
+  const FixupTiles fixup = fixup_tiles(per, nseg);
+  bool any_reduce = false;
+  for (const auto& kv : fixup) any_reduce = any_reduce || !kv.second;
   int k = 0;
   for (int c = 0; c < G; ++c) {
     P.pair_off[c] = static_cast<uint16_t>(k);
@@ -1293,6 +1453,14 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
                     kMaxUnits);
       P.units[k] = uk.first;
       P.unit_k[k] = uk.second;
+      if ((uk.second >> 30) & 1u) {  // a piece of a split tile: its pieces, who adds them
+        const std::tuple<int, int, int> key{unit_problem(uk.first), unit_tt(uk.first),
+                                            unit_mt(uk.first)};
+        const auto it = nseg.find(key);
+        if (it == nseg.end() || it->second < 2 || it->second > kMaxSplits)
+          return fail(HSNF4_ERR_INVALID, "lora gemm: inconsistent split plan");
+        P.units[k] = with_pieces(uk.first, it->second, fixup.at(key));
+      }
       ++k;
     }
   }
@@ -1314,7 +1482,10 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
     g.kblocks = static_cast<int>(d.k_in / 64);
     g.m_tiles = (g.m_total + kPairM - 1) / kPairM;
     g.splits = L.slots[p];
-    if (g.splits > 1) g.partial = reinterpret_cast<float*>(ws + L.part_base[p]);
+    if (g.splits > 1) {
+      g.partial = reinterpret_cast<float*>(ws + L.part_base[p]);
+      g.arrive = reinterpret_cast<unsigned long long*>(ws + L.arrive_base[p]);
+    }
     ok = ok && encode_tma_2d(&g.map_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.act, contraction, T,
                          contraction * 2, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
     if (d.dense)  // bf16 [n_out, k_in]: 64 k x (128 rows fwd | 64 rows dx), 128B swizzle
@@ -1345,10 +1516,11 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
   if (configure_once<kGemmFwd>() != 0 || configure_once<kGemmDx>() != 0)
     return fail(HSNF4_ERR_CUDA, "lora gemm: smem attribute");
   const int smem = smem_plan(mode, BN, tl.sx, tl.sc, tl.sa, r_pad).total + 1024;
+  P.token = next_launch_token();
   void* prof = prof_begin(st, mode == kGemmFwd ? kProfGemmFwd : kProfGemmDx);
   cudaError_t e = launch_pdl(mode == kGemmFwd ? lora_gemm_kernel<kGemmFwd> : lora_gemm_kernel<kGemmDx>,
                              dim3(2 * G), dim3(kThreads), smem, st, P);  // G clusters of 2
-  if (e == cudaSuccess && L.need) {
+  if (e == cudaSuccess && any_reduce) {
     // add the K-split partials in split order and write the bf16 outputs
     static ReduceParams R;
     R.n_tiles = 0;
@@ -1361,6 +1533,7 @@ int launch_lora_gemm_group(GemmMode mode, const GemmProblemDesc* probs, int n, i
         for (int mt = 0; mt < g.m_tiles; ++mt) {
           const auto it = nseg.find({p, tt, mt});
           if (it == nseg.end()) continue;  // a tile in one piece wrote its output directly
+          if (fixup.at({p, tt, mt})) continue;  // its last piece added the pieces
           for (int c = 0; c < 2; ++c) {  // the two 128-row halves of the pair's tile
             const int m0 = mt * kPairM + c * kTileM;
             if (m0 >= g.m_total) continue;

@@ -24,10 +24,11 @@
 //
 // Every call shares the one array and the array keeps the last call's
 // contents.  Nothing needs clearing: every scratch byte a call reads was
-// written earlier in that same call (split-K partial tiles are summed by a
-// separate reduce kernel, with no counters).  Calls whose work overlaps on
-// the GPU -- on different streams, or from different host threads -- race
-// on the scratch; serialize them.
+// written earlier in that same call, except the GEMM's K-split arrival
+// words, which each launch tags with a fresh 56-bit value so that whatever
+// an earlier call left in them counts as no arrivals.  Calls whose work
+// overlaps on the GPU -- on different streams, or from different host
+// threads -- race on the scratch; serialize them.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

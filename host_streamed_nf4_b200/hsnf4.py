@@ -73,7 +73,7 @@ class GemmPlanInfo(Structure):
                 ("units", ctypes.c_int32), ("split_tiles", ctypes.c_int32),
                 ("total_steps", c_int64), ("max_pair_steps", c_int64),
                 ("min_pair_steps", c_int64), ("covered", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("fixup_tiles", ctypes.c_int32)]
 
 
 class HsNf4Error(RuntimeError):
@@ -247,7 +247,7 @@ def gemm_plan(mode: str, shapes, T: int, r: int) -> dict:
     info = GemmPlanInfo()
     _check(lib().hsnf4_gemm_plan({"fwd": 0, "dx": 1}[mode], n_out, k_in, n, T, r,
                                  ctypes.byref(info)))
-    return {f[0]: getattr(info, f[0]) for f in GemmPlanInfo._fields_ if f[0] != "reserved"}
+    return {f[0]: getattr(info, f[0]) for f in GemmPlanInfo._fields_}
 
 
 def profile_read() -> dict:

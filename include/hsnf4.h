@@ -209,8 +209,12 @@ size_t lora_linear_fwd_workspace(int64_t T, int64_t n_out, int64_t k_in, int r);
  * W: NF4 weight [n_out, k_in];  X bf16 [T, k_in];  A bf16 [r, k_in];
  * B bf16 [n_out, r];  Y bf16 [T, n_out];  t_save fp32 [T, r] or NULL.
  * workspace: device scratch of >= lora_linear_fwd_workspace() bytes,
- * 256-byte aligned, not read before being written, free after the stream
- * passes the call.  Errors: INVALID (sizes, rank, pointers), OOM
+ * 256-byte aligned, free after the stream passes the call; its contents on
+ * entry do not matter (the only words read before this call writes them
+ * are the K-split arrival counters, which each launch tags with a fresh
+ * 56-bit value, so a never-written word counts as empty, and which a
+ * completed launch leaves at 0, so a replayed graph finds them empty too;
+ * after a device-side wait timeout, capture such a graph again).  Errors: INVALID (sizes, rank, pointers), OOM
  * (workspace too small; detail gives needed vs given). */
 int lora_linear_fwd(const hsnf4_nf4_weight *W, const void *X, int64_t T,
                     const void *A, const void *B, int r, float alpha, void *Y,
@@ -234,9 +238,9 @@ int lora_linear_fwd(const hsnf4_nf4_weight *W, const void *X, int64_t T,
  *     cudaDeviceReset, for one) looks the address up again on its first
  *     call, which then likewise belongs before any capture.
  *   - All calls share the one array, which keeps the last call's contents.
- *     Nothing in it needs clearing: every byte a call reads was written
- *     earlier in the same call.  Calls whose GPU work overlaps -- other
- *     streams, other host threads -- race on it; serialize them.
+ *     Nothing in it needs clearing (as for lora_linear_fwd's workspace).
+ *     Calls whose GPU work overlaps -- other streams, other host threads --
+ *     race on it; serialize them.
  * Arguments, results and errors are otherwise those of lora_linear_fwd. */
 int lora_linear_fwd_noalloc(const hsnf4_nf4_weight *W, const void *X, int64_t T,
                             const void *A, const void *B, int r, float alpha, void *Y,
@@ -329,7 +333,10 @@ int lora_group_fwd(const hsnf4_lora_fwd_args *probs, int n, int64_t T, int r, fl
  * 256-row x up-to-512-token tiles' K ranges (64-step units) into pieces
  * spread over CTA pairs: longest-first over uniform splits, or stream-K
  * (equal shares of all K steps per pair).  `covered` is 1 when every tile's
- * K range is covered once by pieces in order.  Errors: INVALID. */
+ * K range is covered once by pieces in order.  A split tile's pieces are
+ * added in split order either by the last of them to finish, inside the
+ * kernel (when every piece has later work in its pair to overlap with:
+ * `fixup_tiles`), or by a reduce pass after it.  Errors: INVALID. */
 typedef struct {
   int32_t stream_k;        /* 1: stream-K plan; 0: longest-first over uniform K splits */
   int32_t pairs;           /* CTA pairs given work */
@@ -339,7 +346,7 @@ typedef struct {
   int64_t max_pair_steps;  /* the most K steps any pair runs */
   int64_t min_pair_steps;
   int32_t covered;
-  int32_t reserved;
+  int32_t fixup_tiles;     /* split tiles whose pieces are added inside the kernel */
 } hsnf4_gemm_plan_info;
 
 int hsnf4_gemm_plan(int mode, const int64_t *n_out, const int64_t *k_in, int n, int64_t T,

@@ -54,6 +54,25 @@ def test_plan_kinds_on_the_benchmarked_shapes():
     assert info["stream_k"] == 1 and info["split_tiles"] == 14 and info["pairs"] == 74
 
 
+@pytest.mark.parametrize("family", ["qwen2.5-7b", "qwen2.5-72b", "llama-3.1-8b"])
+@pytest.mark.parametrize("mode", ["fwd", "dx"])
+def test_split_tiles_are_added_in_kernel_only_with_cover(family, mode):
+    """A split tile's pieces are added by its last piece inside the kernel
+    only where every piece has later work (or idle time) in its pair: all
+    of them in the layer-grouped launches, whose pieces are the longest
+    units and run first; none in launches with no more units than pairs,
+    where every piece ends its pair's work."""
+    g = _groups(family)
+    for name, shapes in g.items():
+        for T in (512, 100):
+            info = hsnf4.gemm_plan(mode, shapes, T, 16)
+            assert 0 <= info["fixup_tiles"] <= info["split_tiles"], (name, T, info)
+            if info["units"] <= info["pairs"]:
+                assert info["fixup_tiles"] == 0, (name, T, info)
+    info = hsnf4.gemm_plan(mode, g["layer"], 512, 16)
+    assert info["fixup_tiles"] == info["split_tiles"], info
+
+
 def test_plan_rejects_bad_shapes():
     with pytest.raises(hsnf4.HsNf4Error):
         hsnf4.gemm_plan("fwd", [(100, 512)], 512, 16)
