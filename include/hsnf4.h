@@ -105,8 +105,10 @@ const char *hsnf4_status_string(int status);
 int hsnf4_last_error(char *buf, size_t n);
 
 /* Synchronize `stream`, then read and clear the device-side failure flags
- * that bounded waits in the kernels record (bit set = a wait gave up).
- * *flags (host) receives the flags; returns HSNF4_ERR_DEVICE if any was set. */
+ * that bounded waits in the kernels record (bit set = a wait gave up; in
+ * the fused GEMM, 0x80 = a K-split arrival count that did not settle, which
+ * leaves that tile's output unwritten).  *flags (host) receives the flags;
+ * returns HSNF4_ERR_DEVICE if any was set. */
 int hsnf4_device_status(void *stream, uint32_t *flags);
 
 /* Self-test of the kernels' bounded waits: launches one CTA whose thread
