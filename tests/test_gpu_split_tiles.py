@@ -6,9 +6,10 @@ that completes the count adds the pieces in split order and writes the
 output.  The result must not depend on which piece finishes last, on what
 the workspace held before the call (each launch tags its arrival words
 with a fresh token; a word holding anything else counts as empty), or on
-earlier calls (a completed launch leaves its words 0).  The Qwen2.5-7B
-layer's grouped forward and dX launches are such plans: every split tile
-of both is added in the kernel.
+earlier calls (a completed launch leaves its words 0).  The grouped
+forward and dX launches of a Qwen2.5-7B layer (T = 512, and a ragged 100)
+and of a Llama-3.1-8B layer (T = 256) are such plans: every split tile of
+both is added in the kernel.
 """
 import pytest
 import torch
@@ -26,13 +27,15 @@ def _outputs(stack):
             list(stack.dA[0]) + list(stack.dB[0])]
 
 
-def test_in_kernel_split_adds_are_repeatable_whatever_the_workspace_held():
-    fam = synth.FAMILIES["qwen2.5-7b"]
+@pytest.mark.parametrize("family,T", [("qwen2.5-7b", 512), ("qwen2.5-7b", 100),
+                                      ("llama-3.1-8b", 256)])
+def test_in_kernel_split_adds_are_repeatable_whatever_the_workspace_held(family, T):
+    fam = synth.FAMILIES[family]
     shapes = [(n, k) for _, n, k in fam.projections()]
     for mode in ("fwd", "dx"):
-        info = hsnf4.gemm_plan(mode, shapes, 512, 16)
+        info = hsnf4.gemm_plan(mode, shapes, T, 16)
         assert info["split_tiles"] > 0 and info["fixup_tiles"] == info["split_tiles"], info
-    s = LayerStack(fam, 1, 512, block_size=1, streamed=False)
+    s = LayerStack(fam, 1, T, block_size=1, streamed=False)
     try:
         ref = _outputs(s)
         for fill in ("as left", "random", "ones", "zeros", "as left"):
