@@ -78,3 +78,41 @@ def test_plan_rejects_bad_shapes():
         hsnf4.gemm_plan("fwd", [(100, 512)], 512, 16)
     with pytest.raises(hsnf4.HsNf4Error):
         hsnf4.gemm_plan("fwd", [(512, 512)], 512, 0)
+
+
+def _check_plan(mode, shapes, T, r):
+    """Every plan the launch would run covers each tile's K range once, in
+    order; its step count is the problem's; split tiles added in the kernel
+    are a subset of the split tiles.  (A launch with fewer tiles than CTA
+    pairs leaves some pairs without work; they exit at once.)"""
+    info = hsnf4.gemm_plan(mode, shapes, T, r)
+    assert info["covered"] == 1, (mode, shapes, T, r, info)
+    contraction = [(k if mode == "fwd" else n) // 64 for n, k in shapes]
+    rows = [(n if mode == "fwd" else k) for n, k in shapes]
+    t_tiles = -(-T // (512 if T > 256 else -(-T // 16) * 16))
+    steps = sum(-(-m // 256) * t_tiles * c for m, c in zip(rows, contraction))
+    assert info["total_steps"] == steps, (mode, shapes, T, info)
+    assert info["units"] >= 1 and info["max_pair_steps"] >= -(-steps // info["pairs"]), info
+    assert 0 <= info["fixup_tiles"] <= info["split_tiles"], info
+    return info
+
+
+def test_plans_hold_on_random_groups():
+    """Random groups of 1-8 problems (dimensions multiples of 64 up to
+    32768), random T and ranks: every plan is valid, or the launch refuses
+    it with an error (never a wrong plan)."""
+    hypothesis = pytest.importorskip("hypothesis")
+    st = hypothesis.strategies
+    dim = st.integers(1, 512).map(lambda x: 64 * x)
+
+    @hypothesis.settings(max_examples=400, deadline=None, derandomize=True)
+    @hypothesis.given(mode=st.sampled_from(["fwd", "dx"]),
+                      shapes=st.lists(st.tuples(dim, dim), min_size=1, max_size=8),
+                      T=st.integers(1, 4096), r=st.sampled_from([8, 16, 32, 64]))
+    def run(mode, shapes, T, r):
+        try:
+            _check_plan(mode, shapes, T, r)
+        except hsnf4.HsNf4Error as e:  # refused: too many units or tiles for one launch
+            assert e.status == 1, e
+
+    run()
